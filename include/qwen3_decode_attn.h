@@ -1,0 +1,210 @@
+/*
+ * qwen3_decode_attn.h -- C ABI of the Qwen3-0.6B decode-attention step for
+ * NVIDIA B200 (sm_100a).
+ *
+ * One call performs, for every sequence b of a decode batch, the attention
+ * nodes of the Qwen3-0.6B Model Spec (docs.theformalera.com/models/qwen3-0-6b,
+ * table "Compute-graph nodes"):
+ *
+ *   attn.qk_norm  per-head RMSNorm of the 16 query and 8 key heads over their
+ *                 128 dims, eps = 1e-6, one gain vector shared by every head
+ *                 (also: nnterp encyclopedia, qwen3, "Queries and keys are
+ *                 normed per head, before the rotary");
+ *   attn.rope     rotation of each pair (x_i, x_{i+64}), i < 64, by the angle
+ *                 pos * theta^(-2i/128), theta = 1e6, counter-clockwise:
+ *                 (a, b) -> (a cos - b sin, b cos + a sin);
+ *   cache append  the new key (rounded once to bf16, nearest-even) and the new
+ *                 value (its bits) are written to cache slot seq_lens[b]-1 of a
+ *                 paged cache with 16-token pages (Model Spec, "At a glance",
+ *                 shape domain);
+ *   attn.core     decodeGQA: o[b,h] = sum_{s < seq_lens[b]} softmax_s(
+ *                 <q[b,h], k[b,s,h/2]> / sqrt(128)) v[b,s,h/2], 16 query heads
+ *                 over 8 kv heads (Supported models page, "What every spec
+ *                 covers": one new query per sequence over seq_lens[b] cached
+ *                 positions; nnterp qwen3, "Grouped-query attention").
+ *
+ * Tensor layouts (all little-endian, row-major, no padding):
+ *
+ *   qkv          bf16 [B][4096]: 16 q heads x 128 | 8 k heads x 128 |
+ *                8 v heads x 128, the attn.qkv_proj output row (N = 4096).
+ *   q_norm_w     bf16 [128]; k_norm_w bf16 [128].
+ *   seq_lens     int32 [B]. Counts the new token: 1 <= seq_lens[b] <= the
+ *                handle's max_seq_len (<= 40960) and <= 16 * block_table_stride.
+ *   positions    int32 [B] RoPE positions, or NULL for seq_lens[b]-1. The cache
+ *                slot is seq_lens[b]-1 either way.
+ *   block_table  int32 [B][block_table_stride]; logical slot t of sequence b
+ *                lives in page block_table[b][t/16], row t%16. Entries past
+ *                ceil(seq_lens[b]/16) are never read.
+ *   k_cache,     bf16 [num_pages][16][8][128] each: page, token row, kv head,
+ *   v_cache      dim. One page of one cache is 32 KiB, contiguous.
+ *   o            bf16 [B][16][128].
+ *
+ * Numbers: q and k are normed and rotated in double precision; q is kept in
+ * float (never rounded to bf16); k is rounded once to bf16 when stored; the
+ * scores, the softmax and the value accumulation are float; o is rounded once
+ * to bf16 (nearest-even).
+ *
+ * Ownership: every tensor is caller-owned memory. The handle owns only its
+ * workspace (device scratch for split partials, merge counters and the status
+ * word, and the staging buffers of the host-buffer entry point), allocated by
+ * qwen3_decode_attn_create and freed by qwen3_decode_attn_destroy.
+ *
+ * Streams: the attention entry points are asynchronous on the given stream
+ * (a cudaStream_t passed as void*, NULL for the legacy default stream) and do
+ * not synchronize. A handle's workspace serves one call at a time: calls that
+ * share a handle must be ordered (same stream, or explicit events).
+ *
+ * Errors: functions return QDA_OK (0) or a negative QDA_ERR_* code; nothing
+ * aborts, traps or prints. Argument errors are found on the host before any
+ * launch. Errors found on the device (an index out of range, a bounded wait
+ * that ran out) are recorded in the handle's sticky status word and returned
+ * by qwen3_decode_attn_check.
+ *
+ * Preconditions the library relies on and does not check: the page that
+ * receives a sequence's new token is not read or written by another sequence
+ * of the same call; tensors do not overlap one another.
+ */
+#ifndef QWEN3_DECODE_ATTN_H
+#define QWEN3_DECODE_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Geometry compiled into the kernels (Model Spec, "Published configuration":
+ * num_attention_heads 16, num_key_value_heads 8, head_dim 128; "At a glance":
+ * page size 16, B <= 256, S <= 40960; attn.qkv_proj N = 4096). */
+#define QDA_NUM_Q_HEADS   16
+#define QDA_NUM_KV_HEADS  8
+#define QDA_HEAD_DIM      128
+#define QDA_PAGE_SIZE     16
+#define QDA_QKV_WIDTH     4096
+#define QDA_MAX_BATCH     256
+#define QDA_MAX_SEQ_LEN   40960
+
+/* Return codes. */
+#define QDA_OK               0
+#define QDA_ERR_INVALID_ARG  (-1) /* null/misaligned pointer, size outside the domain */
+#define QDA_ERR_CUDA         (-2) /* a CUDA runtime call or a launch failed */
+#define QDA_ERR_UNSUPPORTED  (-3) /* config geometry differs from the compiled one */
+#define QDA_ERR_BOUNDS       (-4) /* device: a seq_len or a block-table entry out of range */
+#define QDA_ERR_TIMEOUT      (-5) /* device: a bounded wait ran out */
+
+/* Create-time flags. */
+#define QDA_FLAG_INJECT_WAIT_TIMEOUT 0x1u /* test only: every launch makes one warp
+                                             wait on a barrier that nothing completes,
+                                             until wait_timeout_ns runs out; the call
+                                             still computes its result and records
+                                             QDA_ERR_TIMEOUT */
+
+typedef struct qda_handle qda_handle; /* opaque */
+
+typedef struct {
+    int num_q_heads;        /* must be 16 */
+    int num_kv_heads;       /* must be 8 */
+    int head_dim;           /* must be 128 */
+    int page_size;          /* must be 16 */
+    int max_batch;          /* 1..256: largest B a call may pass */
+    int max_seq_len;        /* 1..40960: largest seq_lens[b] accepted */
+    int max_pages_per_seq;  /* block-table row capacity of the host-buffer entry
+                               point's staging; >= ceil(max_seq_len/16) */
+    double rope_theta;      /* RoPE base, > 0 (1e6 for Qwen3-0.6B) */
+    double rms_eps;         /* RMSNorm epsilon, >= 0 (1e-6 for Qwen3-0.6B) */
+    int grid_ctas;          /* 0: one CTA per SM. > 0: exactly that many CTAs
+                               (<= 4096), which changes how the key range of a
+                               sequence is split; the result must not change */
+    unsigned flags;         /* QDA_FLAG_* */
+    int64_t wait_timeout_ns;/* limit of every device-side wait; 0: 1 second */
+} qda_config;
+
+/* Fill *cfg with the Qwen3-0.6B values: 16/8/128/16, max_batch 256,
+ * max_seq_len 40960, max_pages_per_seq 2560, theta 1e6, eps 1e-6, grid 0,
+ * flags 0, timeout 0. */
+void qwen3_decode_attn_default_config(qda_config *cfg);
+
+/* Create a handle bound to CUDA device `device` (made current during the
+ * call). Allocates the workspace on that device. On success *out receives the
+ * handle; on failure *out is set to NULL.
+ * Errors: INVALID_ARG (null pointer, a size outside its range),
+ *         UNSUPPORTED (head counts, head_dim or page_size not 16/8/128/16),
+ *         CUDA (no such device, allocation failure). */
+int qwen3_decode_attn_create(const qda_config *cfg, int device, qda_handle **out);
+
+/* The decode-attention step on device buffers (layouts above). Every pointer
+ * is a device pointer. qkv, k_cache, v_cache and o must be 16-byte aligned;
+ * q_norm_w, k_norm_w, seq_lens, positions and block_table 4-byte aligned.
+ * `batch` is B (1..max_batch); `num_pages` (>= 1) bounds every block-table
+ * entry the call reads; `block_table_stride` (>= 1) is the row pitch in
+ * entries.
+ * On return the work is queued on `cuda_stream`. When it has run: k_cache and
+ * v_cache hold the appended tokens (no other cache byte changes) and o holds
+ * the attention output.
+ * Errors: INVALID_ARG (found on the host; nothing is launched), CUDA (the
+ * launch failed). Device-side errors go to the status word: a seq_len outside
+ * [1, min(max_seq_len, 16*block_table_stride)] makes the call skip that
+ * sequence (its o rows and cache are left untouched); a block-table entry
+ * outside [0, num_pages) is not dereferenced (that page is skipped, the
+ * sequence's o rows are then unspecified, and no append goes to it). */
+int qwen3_decode_attn_append_and_attend(qda_handle *h,
+                                        const void *qkv,
+                                        const void *q_norm_w,
+                                        const void *k_norm_w,
+                                        const int32_t *seq_lens,
+                                        const int32_t *positions,
+                                        const int32_t *block_table,
+                                        int block_table_stride,
+                                        void *k_cache,
+                                        void *v_cache,
+                                        int num_pages,
+                                        void *o,
+                                        int batch,
+                                        void *cuda_stream);
+
+/* The same step for a caller whose per-step tensors are in HOST memory:
+ * qkv_host, seq_lens_host, positions_host (or NULL) and block_table_host are
+ * host pointers (pinned memory makes the copies asynchronous), and o_host is
+ * the host destination of o. q_norm_w, k_norm_w, k_cache and v_cache stay
+ * device pointers (weights and cache are device-resident state). The call
+ * queues host-to-device copies into the handle's staging buffers, the step,
+ * and the device-to-host copy of o, all on `cuda_stream`, and returns; o_host
+ * is valid after the stream is synchronized. Requires block_table_stride <=
+ * max_pages_per_seq. Errors as for qwen3_decode_attn_append_and_attend. */
+int qwen3_decode_attn_append_and_attend_host(qda_handle *h,
+                                             const void *qkv_host,
+                                             const void *q_norm_w,
+                                             const void *k_norm_w,
+                                             const int32_t *seq_lens_host,
+                                             const int32_t *positions_host,
+                                             const int32_t *block_table_host,
+                                             int block_table_stride,
+                                             void *k_cache,
+                                             void *v_cache,
+                                             int num_pages,
+                                             void *o_host,
+                                             int batch,
+                                             void *cuda_stream);
+
+/* Synchronize `cuda_stream`, read and clear the status word, and return the
+ * first device error recorded since the last check (QDA_OK if none;
+ * QDA_ERR_BOUNDS or QDA_ERR_TIMEOUT otherwise). After an error the handle's
+ * merge counters are reset, so the handle stays usable. CUDA if a runtime call
+ * fails. */
+int qwen3_decode_attn_check(qda_handle *h, void *cuda_stream);
+
+/* Number of CTAs one call launches (the grid size). */
+int qwen3_decode_attn_grid_ctas(const qda_handle *h);
+
+/* Free the workspace and the handle. NULL is ignored. The caller must ensure
+ * no work that uses the handle is still queued. */
+void qwen3_decode_attn_destroy(qda_handle *h);
+
+/* Static, human-readable text for a return code. */
+const char *qwen3_decode_attn_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QWEN3_DECODE_ATTN_H */

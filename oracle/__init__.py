@@ -1,0 +1,162 @@
+"""Float64 CPU oracle of the Qwen3-0.6B decode-attention step (ctypes wrapper).
+
+TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the benchmark's
+CPU-baseline leg use this package; the CUDA library and its Python binding never
+import it. The arithmetic lives in ``qwen3_decode_oracle.c`` (plain C, double
+precision, written from the Qwen3-0.6B Model Spec's "Compute-graph nodes"
+table); this module only marshals numpy arrays into it. bf16 tensors travel as
+``numpy.uint16`` arrays of their bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "qwen3_decode_oracle.c")
+LIBRARY = os.path.join(_HERE, "liboracle.so")
+
+NUM_Q_HEADS = 16
+NUM_KV_HEADS = 8
+HEAD_DIM = 128
+PAGE = 16
+QKV_WIDTH = 4096
+
+_ERRORS = {-1: "invalid argument", -4: "seq_len or block-table entry out of range"}
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (IEEE double, no contraction into FMA)."""
+    if force or not os.path.exists(LIBRARY) or os.path.getmtime(LIBRARY) < os.path.getmtime(SOURCE):
+        cmd = ["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math",
+               "-shared", "-fPIC", "-o", LIBRARY, SOURCE, "-lm"]
+        subprocess.run(cmd, check=True)
+    return LIBRARY
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(LIBRARY)
+        dp = ctypes.POINTER(ctypes.c_double)
+        u16p = ctypes.POINTER(ctypes.c_uint16)
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        lib.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        lib.oracle_bf16_to_f64.restype = ctypes.c_double
+        lib.oracle_f64_to_bf16_rne.argtypes = [ctypes.c_double]
+        lib.oracle_f64_to_bf16_rne.restype = ctypes.c_uint16
+        lib.oracle_bf16_to_f64_array.argtypes = [u16p, dp, ctypes.c_size_t]
+        lib.oracle_f64_to_bf16_rne_array.argtypes = [dp, u16p, ctypes.c_size_t]
+        lib.oracle_rmsnorm.argtypes = [dp, dp, ctypes.c_int, ctypes.c_double, dp]
+        lib.oracle_rope.argtypes = [dp, ctypes.c_int, ctypes.c_double, ctypes.c_double]
+        lib.oracle_decode_head.argtypes = [dp, ctypes.c_int, i32p, u16p, u16p, ctypes.c_int, dp, dp]
+        lib.oracle_append_and_attend.argtypes = [
+            u16p, u16p, u16p, i32p, i32p, i32p, ctypes.c_int, u16p, u16p, ctypes.c_int,
+            dp, ctypes.c_int, ctypes.c_double, ctypes.c_double, dp, dp]
+        lib.oracle_append_and_attend.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray | None, ctype):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def bf16_to_f64(bits) -> np.ndarray:
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    out = np.empty(bits.shape, dtype=np.float64)
+    _load().oracle_bf16_to_f64_array(_ptr(bits, ctypes.c_uint16), _ptr(out, ctypes.c_double), bits.size)
+    return out
+
+
+def f64_to_bf16_rne(x) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(x.shape, dtype=np.uint16)
+    _load().oracle_f64_to_bf16_rne_array(_ptr(x, ctypes.c_double), _ptr(out, ctypes.c_uint16), x.size)
+    return out
+
+
+def rmsnorm(x, w, eps: float = 1e-6) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    assert x.ndim == 1 and w.shape == x.shape
+    y = np.empty_like(x)
+    _load().oracle_rmsnorm(_ptr(x, ctypes.c_double), _ptr(w, ctypes.c_double), x.size, eps,
+                           _ptr(y, ctypes.c_double))
+    return y
+
+
+def rope(x, pos: float, theta: float = 1e6) -> np.ndarray:
+    y = np.array(x, dtype=np.float64, copy=True)
+    assert y.ndim == 1 and y.size % 2 == 0
+    _load().oracle_rope(_ptr(y, ctypes.c_double), y.size, float(pos), float(theta))
+    return y
+
+
+def decode_head(q, seq_len: int, bt_row, k_cache, v_cache, kv_head: int) -> np.ndarray:
+    """One query head of decodeGQA over the paged cache (bf16 bit arrays)."""
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    bt_row = np.ascontiguousarray(bt_row, dtype=np.int32)
+    k_cache = np.ascontiguousarray(k_cache, dtype=np.uint16)
+    v_cache = np.ascontiguousarray(v_cache, dtype=np.uint16)
+    scores = np.empty(seq_len, dtype=np.float64)
+    o = np.empty(HEAD_DIM, dtype=np.float64)
+    _load().oracle_decode_head(_ptr(q, ctypes.c_double), seq_len, _ptr(bt_row, ctypes.c_int32),
+                               _ptr(k_cache, ctypes.c_uint16), _ptr(v_cache, ctypes.c_uint16),
+                               kv_head, _ptr(scores, ctypes.c_double), _ptr(o, ctypes.c_double))
+    return o
+
+
+def append_and_attend(qkv, q_norm_w, k_norm_w, seq_lens, block_table, k_cache, v_cache,
+                      positions=None, rope_theta: float = 1e6, rms_eps: float = 1e-6,
+                      inplace: bool = False, want_qk: bool = False) -> dict:
+    """Run the whole step. bf16 inputs are uint16 bit arrays.
+
+    Returns a dict with ``o`` (float64 [B,16,128]), ``k_cache`` and ``v_cache``
+    (uint16, after the append; the inputs themselves when ``inplace``), and,
+    when ``want_qk``, ``q`` (float64 [B,16,128]) and ``k`` (float64 [B,8,128],
+    the new k before its rounding to bf16).
+    """
+    qkv = np.ascontiguousarray(qkv, dtype=np.uint16)
+    B = qkv.shape[0]
+    assert qkv.shape == (B, QKV_WIDTH)
+    q_norm_w = np.ascontiguousarray(q_norm_w, dtype=np.uint16)
+    k_norm_w = np.ascontiguousarray(k_norm_w, dtype=np.uint16)
+    seq_lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    block_table = np.ascontiguousarray(block_table, dtype=np.int32)
+    assert block_table.ndim == 2 and block_table.shape[0] == B
+    if positions is not None:
+        positions = np.ascontiguousarray(positions, dtype=np.int32)
+    if not inplace:
+        k_cache = np.array(k_cache, dtype=np.uint16, copy=True)
+        v_cache = np.array(v_cache, dtype=np.uint16, copy=True)
+    assert k_cache.dtype == np.uint16 and k_cache.flags["C_CONTIGUOUS"]
+    assert v_cache.dtype == np.uint16 and v_cache.flags["C_CONTIGUOUS"]
+    num_pages = k_cache.shape[0]
+    assert k_cache.shape == (num_pages, PAGE, NUM_KV_HEADS, HEAD_DIM) == v_cache.shape
+    o = np.empty((B, NUM_Q_HEADS, HEAD_DIM), dtype=np.float64)
+    q = np.empty((B, NUM_Q_HEADS, HEAD_DIM), dtype=np.float64) if want_qk else None
+    k = np.empty((B, NUM_KV_HEADS, HEAD_DIM), dtype=np.float64) if want_qk else None
+    rc = _load().oracle_append_and_attend(
+        _ptr(qkv, ctypes.c_uint16), _ptr(q_norm_w, ctypes.c_uint16), _ptr(k_norm_w, ctypes.c_uint16),
+        _ptr(seq_lens, ctypes.c_int32), _ptr(positions, ctypes.c_int32),
+        _ptr(block_table, ctypes.c_int32), block_table.shape[1],
+        _ptr(k_cache, ctypes.c_uint16), _ptr(v_cache, ctypes.c_uint16), num_pages,
+        _ptr(o, ctypes.c_double), B, rope_theta, rms_eps,
+        _ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double))
+    if rc != 0:
+        raise ValueError(f"oracle_append_and_attend: {_ERRORS.get(rc, rc)}")
+    out = {"o": o, "k_cache": k_cache, "v_cache": v_cache}
+    if want_qk:
+        out["q"], out["k"] = q, k
+    return out

@@ -1,0 +1,295 @@
+/*
+ * Float64 CPU oracle of the Qwen3-0.6B decode-attention step.
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is built into oracle/liboracle.so and is
+ * loaded by the test suite, by the smoke check and by the benchmark's CPU
+ * baseline leg. The CUDA library never links, loads or calls it, and it shares
+ * no source, header, table or helper with the CUDA library.
+ *
+ * What it computes is the plain definition of the step, written out in double
+ * precision in the order the specification states it, with no blocking, no
+ * online softmax and no fusion:
+ *
+ *   qkv row -> split into 16 q heads | 8 k heads | 8 v heads of 128
+ *        (Qwen3-0.6B Model Spec, "Compute-graph nodes", attn.qkv_proj N=4096;
+ *         nnterp qwen3 page, "Queries and keys are normed per head, before the
+ *         rotary": q_proj(x).view(..., num_heads, 128))
+ *   q, k -> per-head RMSNorm over 128 dims with one shared gain vector
+ *        (Model Spec, "Compute-graph nodes", attn.qk_norm, eps=1e-06)
+ *   q, k -> RoPE: pairs (i, i+64), i < 64, rotated by pos * theta^(-2i/128)
+ *        (Model Spec, "Compute-graph nodes", attn.rope, theta=1000000)
+ *   k, v -> appended to the paged cache at slot seq_len-1
+ *        (Model Spec, "At a glance", shape domain: page size 16;
+ *         Supported models page, "What every spec covers": one new query per
+ *         sequence over seq_lens[b] cached positions)
+ *   o[b,h] = sum_{s < seq_lens[b]} softmax_s(<q[b,h], k[b,s,h/2]> / sqrt(128)) v[b,s,h/2]
+ *        (Model Spec, "Compute-graph nodes", attn.core decodeGQA)
+ *
+ * Readings taken where the pages leave a step open (each one is listed with
+ * its reason in the design notes of the repository):
+ *   - the rotation is the counter-clockwise one: (a, b) -> (a cos - b sin,
+ *     b cos + a sin) for the pair (x_i, x_{i+64});
+ *   - seq_lens[b] counts the new token; the new token sits in cache slot
+ *     seq_lens[b]-1 and, unless positions are given, has that position too;
+ *   - the paged cache is [num_pages][16 slots][8 kv heads][128] bf16 and
+ *     logical slot t of sequence b lives in page block_table[b][t/16], row t%16;
+ *   - nothing is rounded until an output: k is rounded once, from double, to
+ *     bf16 with round-to-nearest-even when it is written to the cache; the
+ *     attention then reads the cache as stored (the rounded k); o stays double.
+ *
+ * Every function names the passage it follows. The pins that tie this file to
+ * the pages and to mathematics (closed forms, invariants, library routines,
+ * brute force) live in tests/test_oracle_pins.py.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* Constants of the Qwen3-0.6B Model Spec ("Published configuration" and the
+ * attn.* rows of "Compute-graph nodes"). */
+enum {
+    ORC_NUM_Q_HEADS = 16,
+    ORC_NUM_KV_HEADS = 8,
+    ORC_HEAD_DIM = 128,
+    ORC_ROPE_PAIRS = 64,          /* attn.rope: active = 64, rot = 128 */
+    ORC_PAGE = 16,                /* "At a glance": page size 16 */
+    ORC_Q_WIDTH = ORC_NUM_Q_HEADS * ORC_HEAD_DIM,   /* 2048 */
+    ORC_KV_WIDTH = ORC_NUM_KV_HEADS * ORC_HEAD_DIM, /* 1024 */
+    ORC_QKV_WIDTH = ORC_Q_WIDTH + 2 * ORC_KV_WIDTH, /* 4096 = attn.qkv_proj N */
+    ORC_PAGE_ELEMS = ORC_PAGE * ORC_KV_WIDTH,       /* elements in one page */
+    ORC_MAX_BATCH = 256,          /* "At a glance": B in [1, 256] */
+    ORC_MAX_SEQ = 40960           /* "At a glance": S in [1, 40960] */
+};
+
+enum {
+    ORC_OK = 0,
+    ORC_ERR_ARG = -1,      /* a null pointer or a size outside the domain */
+    ORC_ERR_BOUNDS = -4    /* a seq_len or a block-table entry out of range */
+};
+
+/* ---- bf16 <-> double --------------------------------------------------- */
+
+/* bf16 is the upper half of an IEEE binary32 word, so widening is exact. */
+double oracle_bf16_to_f64(uint16_t bits)
+{
+    uint32_t w = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &w, sizeof f);
+    return (double)f;
+}
+
+/* Round a double to the nearest bf16 value, ties to even, straight from the
+ * double (no intermediate float rounding). bf16 keeps 8 significant bits and
+ * the binary32 exponent range: normal numbers are spaced 2^(E-7) within the
+ * binade [2^E, 2^(E+1)), subnormals are spaced 2^-133, and the largest finite
+ * value is (2 - 2^-7) * 2^127. Scaling by the spacing is exact, nearbyint()
+ * rounds half to even under the default rounding mode, and scaling back is
+ * exact; what is left is an exact bf16 value that is re-encoded. */
+uint16_t oracle_f64_to_bf16_rne(double x)
+{
+    uint16_t sign = signbit(x) ? 0x8000u : 0u;
+    if (isnan(x)) return (uint16_t)(sign | 0x7FC0u);
+    double a = fabs(x);
+    if (a == 0.0) return sign;
+    if (isinf(a)) return (uint16_t)(sign | 0x7F80u);
+
+    int e2;
+    (void)frexp(a, &e2);               /* a = f * 2^e2, f in [0.5, 1) */
+    int E = e2 - 1;                    /* a in [2^E, 2^(E+1)) */
+    int spacing_exp = (E < -126) ? -133 : E - 7;
+    double q = ldexp(a, -spacing_exp); /* exact */
+    double r = nearbyint(q);           /* round half to even */
+    double v = ldexp(r, spacing_exp);  /* exact */
+
+    const double bf16_max = ldexp(255.0, 120); /* (2 - 2^-7) * 2^127 */
+    if (v > bf16_max) return (uint16_t)(sign | 0x7F80u);
+
+    float f = (float)v; /* exact: v has at most 8 significant bits */
+    uint32_t w;
+    memcpy(&w, &f, sizeof w);
+    return (uint16_t)(sign | (uint16_t)(w >> 16));
+}
+
+/* ---- attn.qk_norm ------------------------------------------------------- */
+
+/* Model Spec, "Compute-graph nodes", rmsnorm row:
+ *   y[i] = x[i] / sqrt(sum_j x[j]^2 / H + eps) * w[i]
+ * with the sum running j = 0 .. n-1 in index order. */
+void oracle_rmsnorm(const double *x, const double *w, int n, double eps, double *y)
+{
+    double ss = 0.0;
+    for (int j = 0; j < n; ++j) ss += x[j] * x[j];
+    double r = sqrt(ss / (double)n + eps);
+    for (int i = 0; i < n; ++i) y[i] = x[i] / r * w[i];
+}
+
+/* ---- attn.rope ---------------------------------------------------------- */
+
+/* Model Spec, "Compute-graph nodes", attn.rope row: rotate the pair
+ * (x[i], x[i + d/2]) for i < d/2 by the angle pos * theta^(-2i/d); with
+ * d = rot = 128 every coordinate is in a pair, so none is left unchanged.
+ * The rotation is the counter-clockwise one (the reading named above). */
+void oracle_rope(double *x, int d, double pos, double theta)
+{
+    int half = d / 2;
+    for (int i = 0; i < half; ++i) {
+        double angle = pos * pow(theta, -2.0 * (double)i / (double)d);
+        double c = cos(angle), s = sin(angle);
+        double a = x[i], b = x[i + half];
+        x[i] = a * c - b * s;
+        x[i + half] = b * c + a * s;
+    }
+}
+
+/* ---- attn.core (decodeGQA) for one query head --------------------------- */
+
+/* Model Spec, "Compute-graph nodes", attn.core row:
+ *   o = sum_{s < L} softmax_s(<q, k_s> / sqrt(128)) v_s
+ * k_s and v_s are kv head `kvh` of logical slot s, read through the block
+ * table from the paged cache. The softmax is evaluated as exp(z - max z) / sum,
+ * which equals the definition by the softmax_shift theorem (Supported models
+ * page, "Facts proved about the specs"). `scores` must hold L doubles. */
+void oracle_decode_head(const double *q, int L, const int32_t *bt_row,
+                        const uint16_t *k_cache, const uint16_t *v_cache,
+                        int kvh, double *scores, double *o)
+{
+    const double scale = 1.0 / sqrt((double)ORC_HEAD_DIM);
+    double m = -INFINITY;
+    for (int s = 0; s < L; ++s) {
+        size_t base = (size_t)bt_row[s / ORC_PAGE] * ORC_PAGE_ELEMS
+                    + (size_t)(s % ORC_PAGE) * ORC_KV_WIDTH + (size_t)kvh * ORC_HEAD_DIM;
+        double dot = 0.0;
+        for (int d = 0; d < ORC_HEAD_DIM; ++d)
+            dot += q[d] * oracle_bf16_to_f64(k_cache[base + d]);
+        scores[s] = dot * scale;
+        if (scores[s] > m) m = scores[s];
+    }
+    double z = 0.0;
+    for (int s = 0; s < L; ++s) {
+        scores[s] = exp(scores[s] - m);
+        z += scores[s];
+    }
+    for (int d = 0; d < ORC_HEAD_DIM; ++d) o[d] = 0.0;
+    for (int s = 0; s < L; ++s) {
+        size_t base = (size_t)bt_row[s / ORC_PAGE] * ORC_PAGE_ELEMS
+                    + (size_t)(s % ORC_PAGE) * ORC_KV_WIDTH + (size_t)kvh * ORC_HEAD_DIM;
+        double p = scores[s] / z;
+        for (int d = 0; d < ORC_HEAD_DIM; ++d)
+            o[d] += p * oracle_bf16_to_f64(v_cache[base + d]);
+    }
+}
+
+/* ---- the whole step ------------------------------------------------------ */
+
+/* The decode-attention step for a batch, in the order the specification
+ * gives it: for every sequence, norm and rotate q and k, append the new k and
+ * v to the cache; then, over the cache as it stands after the append, attend.
+ *
+ *   qkv          bf16 [B][4096], q | k | v, head-major (attn.qkv_proj output)
+ *   q_norm_w     bf16 [128], k_norm_w bf16 [128] (one gain for every head)
+ *   seq_lens     [B], counts the new token, 1 <= L <= 40960 and <= 16*bt_stride
+ *   positions    [B] RoPE positions, or NULL for seq_lens[b]-1
+ *   block_table  [B][bt_stride] page ids; entries past ceil(L/16) are not read
+ *   k_cache, v_cache  bf16 [num_pages][16][8][128], updated in place
+ *   o            double [B][16][128] (output)
+ *   q_out        double [B][16][128] or NULL: q after norm and RoPE
+ *   k_out        double [B][8][128] or NULL: new k after norm and RoPE, before
+ *                its rounding to bf16
+ *
+ * Returns 0, ORC_ERR_ARG, or ORC_ERR_BOUNDS (nothing is written then). */
+int oracle_append_and_attend(const uint16_t *qkv, const uint16_t *q_norm_w,
+                             const uint16_t *k_norm_w, const int32_t *seq_lens,
+                             const int32_t *positions, const int32_t *block_table,
+                             int bt_stride, uint16_t *k_cache, uint16_t *v_cache,
+                             int num_pages, double *o, int B, double rope_theta,
+                             double rms_eps, double *q_out, double *k_out)
+{
+    if (!qkv || !q_norm_w || !k_norm_w || !seq_lens || !block_table || !k_cache ||
+        !v_cache || !o || B < 1 || B > ORC_MAX_BATCH || bt_stride < 1 || num_pages < 1)
+        return ORC_ERR_ARG;
+
+    /* Validate every index the step will use before touching anything. */
+    for (int b = 0; b < B; ++b) {
+        int L = seq_lens[b];
+        if (L < 1 || L > ORC_MAX_SEQ || L > ORC_PAGE * bt_stride) return ORC_ERR_BOUNDS;
+        for (int p = 0; p < (L + ORC_PAGE - 1) / ORC_PAGE; ++p) {
+            int32_t id = block_table[(size_t)b * bt_stride + p];
+            if (id < 0 || id >= num_pages) return ORC_ERR_BOUNDS;
+        }
+    }
+
+    double wq[ORC_HEAD_DIM], wk[ORC_HEAD_DIM];
+    for (int i = 0; i < ORC_HEAD_DIM; ++i) {
+        wq[i] = oracle_bf16_to_f64(q_norm_w[i]);
+        wk[i] = oracle_bf16_to_f64(k_norm_w[i]);
+    }
+
+    double *q_all = (double *)malloc(sizeof(double) * (size_t)B * ORC_Q_WIDTH);
+    if (!q_all) return ORC_ERR_ARG;
+
+    /* Norm, rotation and append, sequence by sequence. */
+    for (int b = 0; b < B; ++b) {
+        const uint16_t *row = qkv + (size_t)b * ORC_QKV_WIDTH;
+        int L = seq_lens[b];
+        int slot = L - 1;
+        double pos = positions ? (double)positions[b] : (double)slot;
+        double x[ORC_HEAD_DIM], y[ORC_HEAD_DIM];
+
+        for (int h = 0; h < ORC_NUM_Q_HEADS; ++h) {
+            for (int i = 0; i < ORC_HEAD_DIM; ++i)
+                x[i] = oracle_bf16_to_f64(row[h * ORC_HEAD_DIM + i]);
+            oracle_rmsnorm(x, wq, ORC_HEAD_DIM, rms_eps, y);
+            oracle_rope(y, ORC_HEAD_DIM, pos, rope_theta);
+            memcpy(q_all + ((size_t)b * ORC_NUM_Q_HEADS + h) * ORC_HEAD_DIM, y, sizeof y);
+        }
+
+        int32_t page = block_table[(size_t)b * bt_stride + slot / ORC_PAGE];
+        size_t slot_base = (size_t)page * ORC_PAGE_ELEMS + (size_t)(slot % ORC_PAGE) * ORC_KV_WIDTH;
+        for (int j = 0; j < ORC_NUM_KV_HEADS; ++j) {
+            for (int i = 0; i < ORC_HEAD_DIM; ++i)
+                x[i] = oracle_bf16_to_f64(row[ORC_Q_WIDTH + j * ORC_HEAD_DIM + i]);
+            oracle_rmsnorm(x, wk, ORC_HEAD_DIM, rms_eps, y);
+            oracle_rope(y, ORC_HEAD_DIM, pos, rope_theta);
+            if (k_out) memcpy(k_out + ((size_t)b * ORC_NUM_KV_HEADS + j) * ORC_HEAD_DIM, y, sizeof y);
+            for (int i = 0; i < ORC_HEAD_DIM; ++i) {
+                k_cache[slot_base + (size_t)j * ORC_HEAD_DIM + i] = oracle_f64_to_bf16_rne(y[i]);
+                /* v has no norm and no rotation: its bits are copied. */
+                v_cache[slot_base + (size_t)j * ORC_HEAD_DIM + i] =
+                    row[ORC_Q_WIDTH + ORC_KV_WIDTH + j * ORC_HEAD_DIM + i];
+            }
+        }
+    }
+
+    /* Attention over the cache as it stands after every append. Query head h
+     * reads kv head h/2 (Model Spec attn.core; nnterp qwen3 page, "Grouped-query
+     * attention": kv head j reaches query heads 2j and 2j+1). */
+    int max_L = 0;
+    for (int b = 0; b < B; ++b) if (seq_lens[b] > max_L) max_L = seq_lens[b];
+    double *scores = (double *)malloc(sizeof(double) * (size_t)max_L);
+    if (!scores) { free(q_all); return ORC_ERR_ARG; }
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < ORC_NUM_Q_HEADS; ++h) {
+            oracle_decode_head(q_all + ((size_t)b * ORC_NUM_Q_HEADS + h) * ORC_HEAD_DIM,
+                               seq_lens[b], block_table + (size_t)b * bt_stride,
+                               k_cache, v_cache, h / (ORC_NUM_Q_HEADS / ORC_NUM_KV_HEADS),
+                               scores, o + ((size_t)b * ORC_NUM_Q_HEADS + h) * ORC_HEAD_DIM);
+        }
+    }
+    if (q_out) memcpy(q_out, q_all, sizeof(double) * (size_t)B * ORC_Q_WIDTH);
+    free(scores);
+    free(q_all);
+    return ORC_OK;
+}
+
+/* ---- array forms of the conversions, for the tests ---------------------- */
+
+void oracle_bf16_to_f64_array(const uint16_t *in, double *out, size_t n)
+{
+    for (size_t i = 0; i < n; ++i) out[i] = oracle_bf16_to_f64(in[i]);
+}
+
+void oracle_f64_to_bf16_rne_array(const double *in, uint16_t *out, size_t n)
+{
+    for (size_t i = 0; i < n; ++i) out[i] = oracle_f64_to_bf16_rne(in[i]);
+}
