@@ -1,0 +1,559 @@
+"""Benchmark of the Qwen3-0.6B decode-attention step on B200.
+
+One step is one pass of the whole path (q/k norm, RoPE, cache append,
+decodeGQA) over one batch: one library call for a single-layer workload, 28
+calls for the 28-layer one. Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload cfg2]
+  python bench.py --impl reference ...   (the float64 CPU oracle, host cores)
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own replica of
+the workload (sequences are independent; no collective on the data path);
+timing is the max over ranks, the value the sum of all ranks' bytes over it.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from decode_attention_qk_b200 import inputs  # noqa: E402
+
+METRIC = "decode-attn KV GB/s and µs/call (1 B200) as fraction of HBM roofline"
+KV_BYTES_PER_TOKEN = 2 * inputs.NUM_KV_HEADS * inputs.HEAD_DIM * 2      # K and V rows: 4096 B
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+L2_BYTES = 126 * 2 ** 20
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = [os.path.join(ROOT, "decode_attention_qk_b200", "csrc", f)
+                  for f in ("qda_decode_kernel.cu", "qda_internal.h")]
+
+WORKLOADS = {
+    "cfg1": "B=2, seq_lens={7,12} incl. new token, 4 pages, random block table",
+    "cfg2": "B=32, seq_lens~U[1,4096], page 16, shuffled pool of 8192 pages",
+    "cfg3": "B=256, seq_len=2048, 28 independent layer caches (2.15 GB KV each), one step = 28 calls",
+    "cfg4": "B=4, seq_len=40960 (max context), 10240 shuffled pages",
+    "cfg5": "B=256, seq_lens lognormal(7,1.5) clipped to [1,40960], 10% gap pages",
+}
+
+
+# ----------------------------------------------------------------------------
+# workloads and byte counts
+
+def make_layers(name: str, device, rank: int = 0):
+    """The layers of one step (one Workload per library call)."""
+    off = 100 * rank
+    if name == "cfg1":
+        return [inputs.config1(device)] if rank == 0 else [inputs.custom([7, 12], seed=off, device=device)]
+    if name == "cfg2":
+        return [inputs.config2(device, seed=2000 + off)]
+    if name == "cfg3":
+        return [inputs.config3_layer(i, device, seed=3000 + off) for i in range(inputs.CONFIG3_LAYERS)]
+    if name == "cfg4":
+        return [inputs.config4(device, seed=4000 + off)]
+    if name == "cfg5":
+        return [inputs.config5(device, seed=5000 + off)]
+    raise ValueError(name)
+
+
+def kv_bytes(seq_lens) -> int:
+    """K and V bytes the attention reads: every position incl. the new one, 4096 B each."""
+    return int(torch.as_tensor(seq_lens, dtype=torch.int64).sum()) * KV_BYTES_PER_TOKEN
+
+
+def algorithmic_bytes(seq_lens) -> int:
+    """Least HBM traffic of one call: the cached K/V rows read (L-1 per sequence),
+    the new k/v rows written, the qkv row read, o written, the block-table
+    entries and seq_lens read, and the two gain vectors."""
+    L = torch.as_tensor(seq_lens, dtype=torch.int64)
+    B = int(L.numel())
+    pages = int(((L + 15) // 16).sum())
+    return (int((L - 1).sum()) * KV_BYTES_PER_TOKEN + B * KV_BYTES_PER_TOKEN
+            + B * inputs.QKV_WIDTH * 2 + B * inputs.NUM_Q_HEADS * inputs.HEAD_DIM * 2
+            + pages * 4 + B * 4 + 2 * inputs.HEAD_DIM * 2)
+
+
+def hbm_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def traffic_per_launch(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    this kernel source and workload (else None)."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    entry = t.get(workload)
+    if not entry or entry.get("kernel_source_sha256") != kernel_source_hash():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------
+# clocks
+
+_REASONS = [(0x1, "gpu_idle"), (0x2, "applications_clocks_setting"), (0x4, "sw_power_cap"),
+            (0x8, "hw_slowdown"), (0x10, "sync_boost"), (0x20, "sw_thermal_slowdown"),
+            (0x40, "hw_thermal_slowdown"), (0x80, "hw_power_brake_slowdown"), (0x100, "display_clock_setting")]
+BAD_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons every ~5 ms (NVML) in a thread."""
+
+    def __init__(self, device_index: int):
+        self.samples = []   # (t, sm_mhz, reasons_mask)
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                mhz = n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM)
+                reasons = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append((time.perf_counter(), mhz, reasons))
+            except Exception:
+                pass
+            self._stop.wait(0.005)
+
+    def start(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self, t0: float, t1: float, t_warm: float):
+        if self._nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "note": "NVML unavailable"}
+        window = [s for s in self.samples if t0 <= s[0] <= t1]
+        note = "timed region"
+        if len(window) < 3:
+            window = [s for s in self.samples if t_warm <= s[0] <= t1]
+            note = "warm-up + timed region (timed region shorter than the sampling period)"
+        if not window:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0, "note": note}
+        mask = 0
+        for s in window:
+            mask |= s[2]
+        reasons = [name for bit, name in _REASONS if mask & bit]
+        return {"sm_mhz": statistics.median(s[1] for s in window), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(window), "window": note}
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing (timing only; the data path has no collective)
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist, int(os.environ["RANK"]), world, local
+    if n_gpus != 1:
+        raise SystemExit("--gpus N > 1 must be launched with torchrun, one process per GPU")
+    return None, 0, 1, 0
+
+
+def reduce_max(dist, value: float, device) -> float:
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(dist, value: float, device) -> float:
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(dist, device):
+    if dist is not None:
+        dist.barrier(device_ids=[device.index])
+    torch.cuda.synchronize(device)
+
+
+# ----------------------------------------------------------------------------
+# the oracle on the host (CPU baseline and the reference arm)
+
+def compact_host(w: inputs.Workload, seqs):
+    """Host bytes of the sequences `seqs` over a pool holding only their pages."""
+    pages, rows = [], []
+    for b in seqs:
+        n = (int(w.seq_lens[b]) + 15) // 16
+        rows.append(list(range(len(pages), len(pages) + n)))
+        pages.extend(w.block_table[b, :n].tolist())
+    stride = max(len(r) for r in rows)
+    bt = torch.full((len(seqs), stride), -1, dtype=torch.int32)
+    for i, r in enumerate(rows):
+        bt[i, :len(r)] = torch.tensor(r, dtype=torch.int32)
+    idx = torch.tensor(pages, dtype=torch.int64, device=w.k_cache.device)
+    sel = torch.tensor(list(seqs), dtype=torch.int64)
+    return dict(qkv=inputs.bf16_bits(w.qkv[sel.to(w.qkv.device)]), q_norm_w=inputs.bf16_bits(w.q_norm_w),
+                k_norm_w=inputs.bf16_bits(w.k_norm_w), seq_lens=w.seq_lens[sel].numpy(), block_table=bt.numpy(),
+                k_cache=inputs.bf16_bits(w.k_cache.index_select(0, idx)),
+                v_cache=inputs.bf16_bits(w.v_cache.index_select(0, idx)))
+
+
+def time_oracle(batch: dict) -> float:
+    import oracle
+    t0 = time.perf_counter()
+    oracle.append_and_attend(**batch, inplace=True)
+    return time.perf_counter() - t0
+
+
+def pick_sample(layers, budget_bytes: float):
+    """(layer, sequences) pairs in order until the KV bytes reach `budget_bytes`
+    (at least one sequence)."""
+    picked, total = [], 0
+    for li, w in enumerate(layers):
+        seqs = []
+        for b in range(w.batch):
+            if total >= budget_bytes and (picked or seqs):
+                break
+            seqs.append(b)
+            total += int(w.seq_lens[b]) * KV_BYTES_PER_TOKEN
+        if seqs:
+            picked.append((li, seqs))
+        if total >= budget_bytes:
+            break
+    return picked, total
+
+
+def cpu_baseline(layers, seconds: float = 12.0):
+    """The oracle as it stands, single-threaded, on a bounded sample of the step."""
+    import oracle
+    oracle.build()
+    probe = min(range(layers[0].batch), key=lambda b: int(layers[0].seq_lens[b]))
+    warm = compact_host(layers[0], [probe])
+    dt = time_oracle(warm)
+    rate = max(int(layers[0].seq_lens[probe]) * KV_BYTES_PER_TOKEN / max(dt, 1e-6), 1e6)
+    picked, total_bytes = pick_sample(layers, rate * seconds)
+    elapsed = 0.0
+    for li, seqs in picked:
+        elapsed += time_oracle(compact_host(layers[li], seqs))
+    n_seq = sum(len(s) for _, s in picked)
+    all_seq = sum(w.batch for w in layers)
+    return {"value": total_bytes / elapsed / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n_seq} of {all_seq} sequences of the step ({total_bytes / 1e9:.3f} GB of KV), "
+                      f"{elapsed:.1f} s, single thread",
+            "seconds": elapsed}
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+
+def run_gpu(args):
+    from decode_attention_qk_b200 import binding
+
+    dist, rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    lib = binding.load_library()
+    attn = binding.DecodeAttention(device=local)
+
+    # R resident copies of the step's inputs, so that a call never finds its
+    # K/V in L2 from the previous call (each copy's KV is > L2 or R copies are).
+    first = make_layers(args.workload, dev, rank)
+    step_kv = sum(kv_bytes(w.seq_lens) for w in first)
+    rotate = args.rotate or max(1, min(8, math.ceil(4 * L2_BYTES / max(step_kv, 1))))
+    sets = [first] + [make_layers(args.workload, dev, rank + 1000 * r) for r in range(1, rotate)]
+    calls_per_step = len(first)
+    stream = torch.cuda.current_stream(dev)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+
+    def prepared(layers):
+        out = []
+        for w in layers:
+            t = dict(qkv=w.qkv, q=w.q_norm_w, k=w.k_norm_w, sl=w.seq_lens.to(dev), bt=w.block_table.to(dev),
+                     kc=w.k_cache, vc=w.v_cache,
+                     o=torch.empty((w.batch, 16, 128), dtype=torch.bfloat16, device=dev))
+            c = (attn.handle, ctypes.c_void_p(t["qkv"].data_ptr()), ctypes.c_void_p(t["q"].data_ptr()),
+                 ctypes.c_void_p(t["k"].data_ptr()),
+                 ctypes.cast(ctypes.c_void_p(t["sl"].data_ptr()), ctypes.POINTER(ctypes.c_int32)), None,
+                 ctypes.cast(ctypes.c_void_p(t["bt"].data_ptr()), ctypes.POINTER(ctypes.c_int32)),
+                 int(w.block_table.shape[1]), ctypes.c_void_p(t["kc"].data_ptr()),
+                 ctypes.c_void_p(t["vc"].data_ptr()), int(w.num_pages), ctypes.c_void_p(t["o"].data_ptr()),
+                 int(w.batch), sp)
+            out.append((c, t))
+        return out
+
+    calls = [prepared(layers) for layers in sets]
+    fn = lib.qwen3_decode_attn_append_and_attend
+
+    def step(i):
+        for c, _ in calls[i % rotate]:
+            rc = fn(*c)
+            if rc != 0:
+                raise binding.QdaError(rc, "append_and_attend")
+
+    clocks = ClockSampler(dev.index).start()
+    t_warm = time.perf_counter()
+    for i in range(args.warmup):
+        step(i)
+    rc = attn.check()
+    if rc != 0:
+        raise binding.QdaError(rc, "device status after warm-up")
+
+    # timed region: K steps, an event pair around every launch
+    n_launch = args.steps * calls_per_step
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n_launch)]
+    barrier(dist, dev)
+    t0 = time.perf_counter()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    k = 0
+    for i in range(args.steps):
+        for c, _ in calls[i % rotate]:
+            ev[2 * k].record(stream)
+            rc = fn(*c)
+            ev[2 * k + 1].record(stream)
+            if rc != 0:
+                raise binding.QdaError(rc, "append_and_attend")
+            k += 1
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    t1 = time.perf_counter()
+    barrier(dist, dev)
+    clocks.stop()
+    rc = attn.check()
+    if rc != 0:
+        raise binding.QdaError(rc, "device status after the timed region")
+
+    ms_local = start.elapsed_time(end)
+    kernel_ms = [ev[2 * j].elapsed_time(ev[2 * j + 1]) for j in range(n_launch)]
+    ms = reduce_max(dist, ms_local, dev)
+    ms_per_step = ms / args.steps
+    # every rotation set has its own lengths (cfg2/cfg5 draw them); average the bytes per step
+    kv_per_step_local = sum(sum(kv_bytes(w.seq_lens) for w in s) for s in (sets[i % rotate] for i in range(args.steps))) / args.steps
+    alg_per_step_local = sum(sum(algorithmic_bytes(w.seq_lens) for w in s) for s in (sets[i % rotate] for i in range(args.steps))) / args.steps
+    kv_total = reduce_sum(dist, kv_per_step_local, dev)
+    value = kv_total / (ms_per_step * 1e-3) / 1e9
+
+    # dominant kernel roofline: algorithmic bytes per launch / mean launch duration
+    mean_kernel_ms = statistics.fmean(kernel_ms)
+    alg_per_launch = alg_per_step_local / calls_per_step
+    peak, peak_kind = hbm_peak()
+    achieved = alg_per_launch / (mean_kernel_ms * 1e-3) / 1e9
+    traffic = traffic_per_launch(args.workload)
+
+    # end to end through the host-buffer entry point: per step the H2D copy of the
+    # step's inputs from pinned memory, the call, and the D2H copy of o
+    e2e = run_e2e(args, attn, sets, dev, stream, dist, rotate)
+
+    result = None
+    if rank == 0:
+        clk = clocks.summary(t0, t1, t_warm)
+        result = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
+            "us_per_call": round(ms_per_step * 1e3 / calls_per_step, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "io_dtype": "bf16", "data": "synthetic (seeded; N(0,1) bf16 qkv and cache, gains 1+U(-0.5,0.5))",
+            "config": {"workload": f"{args.workload}: {WORKLOADS[args.workload]}",
+                       "batch": first[0].batch, "layers_per_step": calls_per_step,
+                       "sum_seq_lens_per_step": int(sum(int(w.seq_lens.sum()) for w in first)),
+                       "page_size": 16, "heads": "16 q / 8 kv, D=128",
+                       "l2": f"{rotate} resident input sets rotated; {rotate * step_kv / 1e9:.2f} GB of KV cycled "
+                             f"(> {L2_BYTES / 2**20:.0f} MiB L2)",
+                       "grid_ctas": attn.grid_ctas, "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                         "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+                         "traffic": traffic, "algorithmic_bytes_per_launch": int(alg_per_launch),
+                         "kernel_us_mean": round(mean_kernel_ms * 1e3, 3),
+                         "kernel_us_median": round(statistics.median(kernel_ms) * 1e3, 3)},
+            "e2e": e2e,
+            "gpu_launches": n_launch,
+            "clocks": clk,
+        }
+    if dist is not None:
+        dist.barrier(device_ids=[dev.index])
+    attn.close()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(first)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_e2e(args, attn, sets, dev, stream, dist, rotate):
+    from decode_attention_qk_b200 import binding
+    lib = binding.load_library()
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    host = []
+    for layers in sets:
+        hl = []
+        for w in layers:
+            h = dict(qkv=w.qkv.cpu().pin_memory(), sl=w.seq_lens.clone().pin_memory(),
+                     bt=w.block_table.clone().pin_memory(),
+                     o=torch.empty((w.batch, 16, 128), dtype=torch.bfloat16).pin_memory())
+            c = (attn.handle, ctypes.c_void_p(h["qkv"].data_ptr()), ctypes.c_void_p(w.q_norm_w.data_ptr()),
+                 ctypes.c_void_p(w.k_norm_w.data_ptr()),
+                 ctypes.cast(ctypes.c_void_p(h["sl"].data_ptr()), ctypes.POINTER(ctypes.c_int32)), None,
+                 ctypes.cast(ctypes.c_void_p(h["bt"].data_ptr()), ctypes.POINTER(ctypes.c_int32)),
+                 int(w.block_table.shape[1]), ctypes.c_void_p(w.k_cache.data_ptr()),
+                 ctypes.c_void_p(w.v_cache.data_ptr()), int(w.num_pages), ctypes.c_void_p(h["o"].data_ptr()),
+                 int(w.batch), sp)
+            hl.append((c, h, w))
+        host.append(hl)
+    fn = lib.qwen3_decode_attn_append_and_attend_host
+    for i in range(args.warmup):
+        for c, _, _ in host[i % rotate]:
+            fn(*c)
+    barrier(dist, dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    h2d = d2h = 0
+    for i in range(args.steps):
+        for c, h, w in host[i % rotate]:
+            rc = fn(*c)
+            if rc != 0:
+                raise binding.QdaError(rc, "append_and_attend_host")
+            h2d += h["qkv"].nbytes + h["sl"].nbytes + h["bt"].nbytes
+            d2h += h["o"].nbytes
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    if attn.check() != 0:
+        raise RuntimeError("device status after the e2e region")
+    ms = reduce_max(dist, start.elapsed_time(end), dev) / args.steps
+    kv = sum(sum(kv_bytes(w.seq_lens) for w in sets[i % rotate]) for i in range(args.steps)) / args.steps
+    kv_total = reduce_sum(dist, kv, dev)
+    return {"value": round(kv_total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d // args.steps), "d2h_bytes_per_step": int(d2h // args.steps),
+            "ms_per_step": round(ms, 6), "api": "qwen3_decode_attn_append_and_attend_host"}
+
+
+# ----------------------------------------------------------------------------
+# reference arm: the float64 oracle on the host cores
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    layers = make_layers(args.workload, "cpu", 0)
+    # size each step's sample so that warm-up + timed steps take ~2 minutes
+    probe = min(range(layers[0].batch), key=lambda b: int(layers[0].seq_lens[b]))
+    dt = time_oracle(compact_host(layers[0], [probe]))
+    rate = max(int(layers[0].seq_lens[probe]) * KV_BYTES_PER_TOKEN / max(dt, 1e-6), 1e6)
+    per_step_budget = rate * min(20.0, 120.0 / max(1, args.steps + args.warmup))
+    # a rotating window over the step's sequences
+    flat = [(li, b) for li, w in enumerate(layers) for b in range(w.batch)]
+    pos = 0
+
+    def sample():
+        nonlocal pos
+        got, total = {}, 0
+        while True:
+            li, b = flat[pos % len(flat)]
+            pos += 1
+            got.setdefault(li, []).append(b)
+            total += int(layers[li].seq_lens[b]) * KV_BYTES_PER_TOKEN
+            if total >= per_step_budget or len(got.get(li, [])) >= layers[li].batch:
+                return [(li, s) for li, s in got.items()], total
+
+    for _ in range(args.warmup):
+        picked, _ = sample()
+        for li, s in picked:
+            time_oracle(compact_host(layers[li], s))
+    elapsed, nbytes, nseq = 0.0, 0, 0
+    for _ in range(args.steps):
+        picked, total = sample()
+        for li, s in picked:
+            elapsed += time_oracle(compact_host(layers[li], s))
+            nseq += len(s)
+        nbytes += total
+    value = nbytes / elapsed / 1e9
+    ms_per_step = elapsed * 1e3 / args.steps
+    all_seq = sum(w.batch for w in layers)
+    sample_desc = (f"per step a window of the step's sequences (~{per_step_budget / 1e6:.1f} MB of KV, "
+                   f"{nseq / args.steps:.1f} of {all_seq} sequences on average), single thread")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; same recipe as the GPU arm, drawn on the host)",
+        "config": {"workload": f"{args.workload}: {WORKLOADS[args.workload]}", "batch": layers[0].batch,
+                   "layers_per_step": len(layers), "page_size": 16, "heads": "16 q / 8 kv, D=128"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample_desc},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="cfg2")
+    ap.add_argument("--rotate", type=int, default=0, help="resident input sets cycled (0: enough to defeat L2)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,226 @@
+"""Python binding of the decode-attention C ABI (include/qwen3_decode_attn.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library. The functions carry the C names; tensors are torch tensors whose
+device pointers are passed through, and the stream is torch's current stream
+unless one is given. Loading fails loudly when the library has not been built;
+there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+LIBRARY_PATH = _build.LIBRARY
+
+QDA_OK = 0
+QDA_ERR_INVALID_ARG = -1
+QDA_ERR_CUDA = -2
+QDA_ERR_UNSUPPORTED = -3
+QDA_ERR_BOUNDS = -4
+QDA_ERR_TIMEOUT = -5
+QDA_FLAG_INJECT_WAIT_TIMEOUT = 0x1
+
+NUM_Q_HEADS, NUM_KV_HEADS, HEAD_DIM, PAGE_SIZE, QKV_WIDTH = 16, 8, 128, 16, 4096
+
+
+class qda_config(ctypes.Structure):
+    _fields_ = [
+        ("num_q_heads", ctypes.c_int),
+        ("num_kv_heads", ctypes.c_int),
+        ("head_dim", ctypes.c_int),
+        ("page_size", ctypes.c_int),
+        ("max_batch", ctypes.c_int),
+        ("max_seq_len", ctypes.c_int),
+        ("max_pages_per_seq", ctypes.c_int),
+        ("rope_theta", ctypes.c_double),
+        ("rms_eps", ctypes.c_double),
+        ("grid_ctas", ctypes.c_int),
+        ("flags", ctypes.c_uint),
+        ("wait_timeout_ns", ctypes.c_int64),
+    ]
+
+
+class QdaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {qwen3_decode_attn_strerror(code)} (code {code})")
+
+
+_lib = None
+
+
+def load_library():
+    """Load libqwen3_decode_attn.so (built by decode_attention_qk_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIBRARY_PATH):
+            raise RuntimeError(
+                f"CUDA library {LIBRARY_PATH} is missing; build it with "
+                "`python -m decode_attention_qk_b200.build` (there is no CPU fallback)")
+        lib = ctypes.CDLL(LIBRARY_PATH)
+        vp, i32p = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32)
+        lib.qwen3_decode_attn_default_config.argtypes = [ctypes.POINTER(qda_config)]
+        lib.qwen3_decode_attn_default_config.restype = None
+        lib.qwen3_decode_attn_create.argtypes = [ctypes.POINTER(qda_config), ctypes.c_int, ctypes.POINTER(vp)]
+        lib.qwen3_decode_attn_create.restype = ctypes.c_int
+        call = [vp, vp, vp, vp, i32p, i32p, i32p, ctypes.c_int, vp, vp, ctypes.c_int, vp, ctypes.c_int, vp]
+        lib.qwen3_decode_attn_append_and_attend.argtypes = call
+        lib.qwen3_decode_attn_append_and_attend.restype = ctypes.c_int
+        lib.qwen3_decode_attn_append_and_attend_host.argtypes = call
+        lib.qwen3_decode_attn_append_and_attend_host.restype = ctypes.c_int
+        lib.qwen3_decode_attn_check.argtypes = [vp, vp]
+        lib.qwen3_decode_attn_check.restype = ctypes.c_int
+        lib.qwen3_decode_attn_grid_ctas.argtypes = [vp]
+        lib.qwen3_decode_attn_grid_ctas.restype = ctypes.c_int
+        lib.qwen3_decode_attn_destroy.argtypes = [vp]
+        lib.qwen3_decode_attn_destroy.restype = None
+        lib.qwen3_decode_attn_strerror.argtypes = [ctypes.c_int]
+        lib.qwen3_decode_attn_strerror.restype = ctypes.c_char_p
+        _lib = lib
+    return _lib
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _i32p(t: torch.Tensor | None):
+    return None if t is None else ctypes.cast(ctypes.c_void_p(t.data_ptr()), ctypes.POINTER(ctypes.c_int32))
+
+
+def _stream(stream, device) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _expect(t: torch.Tensor, name: str, dtype, shape, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+
+
+def qwen3_decode_attn_strerror(code: int) -> str:
+    return load_library().qwen3_decode_attn_strerror(int(code)).decode()
+
+
+def qwen3_decode_attn_default_config(**overrides) -> qda_config:
+    cfg = qda_config()
+    load_library().qwen3_decode_attn_default_config(ctypes.byref(cfg))
+    for k, v in overrides.items():
+        setattr(cfg, k, v)
+    return cfg
+
+
+def qwen3_decode_attn_create(cfg: qda_config | None = None, device: int = 0) -> ctypes.c_void_p:
+    cfg = cfg if cfg is not None else qwen3_decode_attn_default_config()
+    h = ctypes.c_void_p()
+    rc = load_library().qwen3_decode_attn_create(ctypes.byref(cfg), int(device), ctypes.byref(h))
+    if rc != QDA_OK:
+        raise QdaError(rc, "qwen3_decode_attn_create")
+    return h
+
+
+def _step_args(qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, k_cache, v_cache, o,
+               dev_of_step, dev_of_state):
+    B = qkv.shape[0] if qkv.dim() == 2 else -1
+    _expect(qkv, "qkv", torch.bfloat16, (B, QKV_WIDTH), dev_of_step)
+    _expect(q_norm_w, "q_norm_w", torch.bfloat16, (HEAD_DIM,), dev_of_state)
+    _expect(k_norm_w, "k_norm_w", torch.bfloat16, (HEAD_DIM,), dev_of_state)
+    _expect(seq_lens, "seq_lens", torch.int32, (B,), dev_of_step)
+    if positions is not None:
+        _expect(positions, "positions", torch.int32, (B,), dev_of_step)
+    if block_table.dim() != 2:
+        raise ValueError("block_table must be [B, stride]")
+    _expect(block_table, "block_table", torch.int32, (B, block_table.shape[1]), dev_of_step)
+    P = k_cache.shape[0]
+    _expect(k_cache, "k_cache", torch.bfloat16, (P, PAGE_SIZE, NUM_KV_HEADS, HEAD_DIM), dev_of_state)
+    _expect(v_cache, "v_cache", torch.bfloat16, (P, PAGE_SIZE, NUM_KV_HEADS, HEAD_DIM), dev_of_state)
+    _expect(o, "o", torch.bfloat16, (B, NUM_Q_HEADS, HEAD_DIM), dev_of_step)
+    return (_ptr(qkv), _ptr(q_norm_w), _ptr(k_norm_w), _i32p(seq_lens), _i32p(positions),
+            _i32p(block_table), int(block_table.shape[1]), _ptr(k_cache), _ptr(v_cache), int(P),
+            _ptr(o), int(B))
+
+
+def qwen3_decode_attn_append_and_attend(handle, qkv, q_norm_w, k_norm_w, seq_lens, positions,
+                                        block_table, k_cache, v_cache, o, stream=None) -> None:
+    """The step on device tensors; asynchronous on `stream`. Raises QdaError on a host-side error."""
+    dev = qkv.device
+    if dev.type != "cuda":
+        raise ValueError("qkv must be a CUDA tensor")
+    args = _step_args(qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, k_cache, v_cache, o, dev, dev)
+    rc = load_library().qwen3_decode_attn_append_and_attend(handle, *args, _stream(stream, dev))
+    if rc != QDA_OK:
+        raise QdaError(rc, "qwen3_decode_attn_append_and_attend")
+
+
+def qwen3_decode_attn_append_and_attend_host(handle, qkv, q_norm_w, k_norm_w, seq_lens, positions,
+                                             block_table, k_cache, v_cache, o, stream=None) -> None:
+    """The step with per-step tensors (qkv, seq_lens, positions, block_table, o) in host
+    memory and weights/cache on the device; o is valid after the stream synchronizes."""
+    dev = k_cache.device
+    cpu = torch.device("cpu")
+    args = _step_args(qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, k_cache, v_cache, o, cpu, dev)
+    rc = load_library().qwen3_decode_attn_append_and_attend_host(handle, *args, _stream(stream, dev))
+    if rc != QDA_OK:
+        raise QdaError(rc, "qwen3_decode_attn_append_and_attend_host")
+
+
+def qwen3_decode_attn_check(handle, stream=None, device=None) -> int:
+    """Synchronize the stream and return (and clear) the device status code."""
+    return int(load_library().qwen3_decode_attn_check(handle, _stream(stream, device)))
+
+
+def qwen3_decode_attn_grid_ctas(handle) -> int:
+    return int(load_library().qwen3_decode_attn_grid_ctas(handle))
+
+
+def qwen3_decode_attn_destroy(handle) -> None:
+    load_library().qwen3_decode_attn_destroy(handle)
+
+
+class DecodeAttention:
+    """A handle with its lifetime: DecodeAttention(device=0, **config fields)."""
+
+    def __init__(self, device: int = 0, **config):
+        self.device = torch.device("cuda", device)
+        self.config = qwen3_decode_attn_default_config(**config)
+        self.handle = qwen3_decode_attn_create(self.config, device)
+
+    @property
+    def grid_ctas(self) -> int:
+        return qwen3_decode_attn_grid_ctas(self.handle)
+
+    def __call__(self, qkv, q_norm_w, k_norm_w, seq_lens, block_table, k_cache, v_cache, o=None,
+                 positions=None, stream=None) -> torch.Tensor:
+        if o is None:
+            o = torch.empty((qkv.shape[0], NUM_Q_HEADS, HEAD_DIM), dtype=torch.bfloat16, device=qkv.device)
+        qwen3_decode_attn_append_and_attend(self.handle, qkv, q_norm_w, k_norm_w, seq_lens, positions,
+                                            block_table, k_cache, v_cache, o, stream)
+        return o
+
+    def check(self, stream=None) -> int:
+        return qwen3_decode_attn_check(self.handle, stream, self.device)
+
+    def close(self) -> None:
+        if getattr(self, "handle", None) is not None:
+            qwen3_decode_attn_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,273 @@
+// C-ABI entry points of the decode-attention library (declared in
+// include/qwen3_decode_attn.h): argument checks, workspace ownership and the
+// launch. All arithmetic of the step runs in the kernel (qda_decode_kernel.cu).
+#include <cstdint>
+#include <cstring>
+#include <new>
+
+#include <cuda_runtime.h>
+
+#include "qda_internal.h"
+#include "qwen3_decode_attn.h"
+
+struct qda_handle {
+    int device = 0;
+    qda_config cfg{};
+    int grid = 0;
+    float* part_acc = nullptr;
+    float2* part_ml = nullptr;
+    int* counters = nullptr;
+    int* status = nullptr;
+    // staging of the host-buffer entry point
+    uint16_t* st_qkv = nullptr;
+    int32_t* st_seq_lens = nullptr;
+    int32_t* st_positions = nullptr;
+    int32_t* st_block_table = nullptr;
+    uint16_t* st_o = nullptr;
+};
+
+namespace {
+
+constexpr int64_t kDefaultTimeoutNs = 1000000000;  // 1 s
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Makes `device` current for the lifetime of the guard, then restores the
+// caller's device.
+class DeviceGuard {
+  public:
+    explicit DeviceGuard(int device) {
+        ok_ = cudaGetDevice(&prev_) == cudaSuccess && cudaSetDevice(device) == cudaSuccess;
+    }
+    ~DeviceGuard() {
+        if (ok_) cudaSetDevice(prev_);
+    }
+    bool ok() const { return ok_; }
+
+  private:
+    int prev_ = 0;
+    bool ok_ = false;
+};
+
+void free_workspace(qda_handle* h) {
+    cudaFree(h->part_acc);
+    cudaFree(h->part_ml);
+    cudaFree(h->counters);
+    cudaFree(h->status);
+    cudaFree(h->st_qkv);
+    cudaFree(h->st_seq_lens);
+    cudaFree(h->st_positions);
+    cudaFree(h->st_block_table);
+    cudaFree(h->st_o);
+}
+
+template <typename T>
+bool alloc(T** p, size_t bytes) {
+    return cudaMalloc(reinterpret_cast<void**>(p), bytes) == cudaSuccess;
+}
+
+int check_call(const qda_handle* h, const void* qkv, const void* q_norm_w, const void* k_norm_w,
+               const int32_t* seq_lens, const int32_t* positions, const int32_t* block_table,
+               int block_table_stride, const void* k_cache, const void* v_cache, int num_pages, const void* o,
+               int batch) {
+    if (h == nullptr || qkv == nullptr || q_norm_w == nullptr || k_norm_w == nullptr || seq_lens == nullptr ||
+        block_table == nullptr || k_cache == nullptr || v_cache == nullptr || o == nullptr)
+        return QDA_ERR_INVALID_ARG;
+    if (batch < 1 || batch > h->cfg.max_batch || block_table_stride < 1 || num_pages < 1)
+        return QDA_ERR_INVALID_ARG;
+    if (!aligned(qkv, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) ||
+        !aligned(q_norm_w, 4) || !aligned(k_norm_w, 4) || !aligned(seq_lens, 4) || !aligned(block_table, 4) ||
+        (positions != nullptr && !aligned(positions, 4)))
+        return QDA_ERR_INVALID_ARG;
+    return QDA_OK;
+}
+
+qda::Params make_params(const qda_handle* h, const void* qkv, const void* q_norm_w, const void* k_norm_w,
+                        const int32_t* seq_lens, const int32_t* positions, const int32_t* block_table,
+                        int block_table_stride, void* k_cache, void* v_cache, int num_pages, void* o, int batch) {
+    qda::Params p{};
+    p.qkv = static_cast<const uint16_t*>(qkv);
+    p.q_norm_w = static_cast<const uint16_t*>(q_norm_w);
+    p.k_norm_w = static_cast<const uint16_t*>(k_norm_w);
+    p.seq_lens = seq_lens;
+    p.positions = positions;
+    p.block_table = block_table;
+    p.k_cache = static_cast<uint16_t*>(k_cache);
+    p.v_cache = static_cast<uint16_t*>(v_cache);
+    p.o = static_cast<uint16_t*>(o);
+    p.bt_stride = block_table_stride;
+    p.num_pages = num_pages;
+    p.batch = batch;
+    p.max_seq_len = h->cfg.max_seq_len;
+    p.rope_theta = h->cfg.rope_theta;
+    p.rms_eps = h->cfg.rms_eps;
+    p.part_acc = h->part_acc;
+    p.part_ml = h->part_ml;
+    p.counters = h->counters;
+    p.status = h->status;
+    p.timeout_ns = h->cfg.wait_timeout_ns > 0 ? h->cfg.wait_timeout_ns : kDefaultTimeoutNs;
+    p.flags = h->cfg.flags;
+    return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+void qwen3_decode_attn_default_config(qda_config* cfg) {
+    if (cfg == nullptr) return;
+    std::memset(cfg, 0, sizeof(*cfg));
+    cfg->num_q_heads = QDA_NUM_Q_HEADS;
+    cfg->num_kv_heads = QDA_NUM_KV_HEADS;
+    cfg->head_dim = QDA_HEAD_DIM;
+    cfg->page_size = QDA_PAGE_SIZE;
+    cfg->max_batch = QDA_MAX_BATCH;
+    cfg->max_seq_len = QDA_MAX_SEQ_LEN;
+    cfg->max_pages_per_seq = QDA_MAX_SEQ_LEN / QDA_PAGE_SIZE;
+    cfg->rope_theta = 1.0e6;
+    cfg->rms_eps = 1.0e-6;
+    cfg->grid_ctas = 0;
+    cfg->flags = 0u;
+    cfg->wait_timeout_ns = 0;
+}
+
+int qwen3_decode_attn_create(const qda_config* cfg, int device, qda_handle** out) {
+    if (out == nullptr) return QDA_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (cfg == nullptr) return QDA_ERR_INVALID_ARG;
+    if (cfg->num_q_heads != QDA_NUM_Q_HEADS || cfg->num_kv_heads != QDA_NUM_KV_HEADS ||
+        cfg->head_dim != QDA_HEAD_DIM || cfg->page_size != QDA_PAGE_SIZE)
+        return QDA_ERR_UNSUPPORTED;
+    if (cfg->max_batch < 1 || cfg->max_batch > QDA_MAX_BATCH || cfg->max_seq_len < 1 ||
+        cfg->max_seq_len > QDA_MAX_SEQ_LEN ||
+        cfg->max_pages_per_seq < (cfg->max_seq_len + QDA_PAGE_SIZE - 1) / QDA_PAGE_SIZE ||
+        !(cfg->rope_theta > 0.0) || !(cfg->rms_eps >= 0.0) || cfg->grid_ctas < 0 ||
+        cfg->grid_ctas > qda::kMaxGridCtas || cfg->wait_timeout_ns < 0 ||
+        (cfg->flags & ~QDA_FLAG_INJECT_WAIT_TIMEOUT) != 0u)
+        return QDA_ERR_INVALID_ARG;
+    if (device < 0) return QDA_ERR_INVALID_ARG;
+
+    DeviceGuard guard(device);
+    if (!guard.ok()) return QDA_ERR_CUDA;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms < 1)
+        return QDA_ERR_CUDA;
+    if (qda::prepare_device() != cudaSuccess) return QDA_ERR_CUDA;
+
+    qda_handle* h = new (std::nothrow) qda_handle();
+    if (h == nullptr) return QDA_ERR_CUDA;
+    h->device = device;
+    h->cfg = *cfg;
+    h->grid = cfg->grid_ctas > 0 ? cfg->grid_ctas : sms;
+
+    const size_t slots = (size_t)qda::num_slots(h->grid, cfg->max_batch);
+    const size_t B = (size_t)cfg->max_batch;
+    bool ok = alloc(&h->part_acc, slots * qda::kNumQHeads * qda::kHeadDim * sizeof(float)) &&
+              alloc(&h->part_ml, slots * qda::kNumQHeads * sizeof(float2)) &&
+              alloc(&h->counters, (size_t)qda::kMaxBatch * qda::kNumKvHeads * sizeof(int)) &&
+              alloc(&h->status, sizeof(int)) &&
+              alloc(&h->st_qkv, B * qda::kQkvWidth * sizeof(uint16_t)) &&
+              alloc(&h->st_seq_lens, B * sizeof(int32_t)) && alloc(&h->st_positions, B * sizeof(int32_t)) &&
+              alloc(&h->st_block_table, B * (size_t)cfg->max_pages_per_seq * sizeof(int32_t)) &&
+              alloc(&h->st_o, B * qda::kNumQHeads * qda::kHeadDim * sizeof(uint16_t));
+    ok = ok && cudaMemset(h->counters, 0, (size_t)qda::kMaxBatch * qda::kNumKvHeads * sizeof(int)) == cudaSuccess &&
+         cudaMemset(h->status, 0, sizeof(int)) == cudaSuccess && cudaDeviceSynchronize() == cudaSuccess;
+    if (!ok) {
+        free_workspace(h);
+        delete h;
+        cudaGetLastError();  // clear the sticky-free allocation error
+        return QDA_ERR_CUDA;
+    }
+    *out = h;
+    return QDA_OK;
+}
+
+int qwen3_decode_attn_append_and_attend(qda_handle* h, const void* qkv, const void* q_norm_w, const void* k_norm_w,
+                                        const int32_t* seq_lens, const int32_t* positions,
+                                        const int32_t* block_table, int block_table_stride, void* k_cache,
+                                        void* v_cache, int num_pages, void* o, int batch, void* cuda_stream) {
+    int rc = check_call(h, qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, block_table_stride, k_cache,
+                        v_cache, num_pages, o, batch);
+    if (rc != QDA_OK) return rc;
+    DeviceGuard guard(h->device);
+    if (!guard.ok()) return QDA_ERR_CUDA;
+    const qda::Params p = make_params(h, qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table,
+                                      block_table_stride, k_cache, v_cache, num_pages, o, batch);
+    return qda::launch(p, h->grid, static_cast<cudaStream_t>(cuda_stream)) == cudaSuccess ? QDA_OK : QDA_ERR_CUDA;
+}
+
+int qwen3_decode_attn_append_and_attend_host(qda_handle* h, const void* qkv_host, const void* q_norm_w,
+                                             const void* k_norm_w, const int32_t* seq_lens_host,
+                                             const int32_t* positions_host, const int32_t* block_table_host,
+                                             int block_table_stride, void* k_cache, void* v_cache, int num_pages,
+                                             void* o_host, int batch, void* cuda_stream) {
+    if (h == nullptr) return QDA_ERR_INVALID_ARG;
+    int rc = check_call(h, qkv_host, q_norm_w, k_norm_w, seq_lens_host, positions_host, block_table_host,
+                        block_table_stride, k_cache, v_cache, num_pages, h->st_o, batch);
+    if (rc != QDA_OK) return rc;
+    if (o_host == nullptr || block_table_stride > h->cfg.max_pages_per_seq) return QDA_ERR_INVALID_ARG;
+    DeviceGuard guard(h->device);
+    if (!guard.ok()) return QDA_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    const size_t B = (size_t)batch;
+    bool ok = cudaMemcpyAsync(h->st_qkv, qkv_host, B * qda::kQkvWidth * sizeof(uint16_t), cudaMemcpyHostToDevice,
+                              st) == cudaSuccess &&
+              cudaMemcpyAsync(h->st_seq_lens, seq_lens_host, B * sizeof(int32_t), cudaMemcpyHostToDevice, st) ==
+                  cudaSuccess &&
+              cudaMemcpyAsync(h->st_block_table, block_table_host, B * (size_t)block_table_stride * sizeof(int32_t),
+                              cudaMemcpyHostToDevice, st) == cudaSuccess &&
+              (positions_host == nullptr ||
+               cudaMemcpyAsync(h->st_positions, positions_host, B * sizeof(int32_t), cudaMemcpyHostToDevice, st) ==
+                   cudaSuccess);
+    if (!ok) return QDA_ERR_CUDA;
+    const qda::Params p = make_params(h, h->st_qkv, q_norm_w, k_norm_w, h->st_seq_lens,
+                                      positions_host != nullptr ? h->st_positions : nullptr, h->st_block_table,
+                                      block_table_stride, k_cache, v_cache, num_pages, h->st_o, batch);
+    if (qda::launch(p, h->grid, st) != cudaSuccess) return QDA_ERR_CUDA;
+    if (cudaMemcpyAsync(o_host, h->st_o, B * qda::kNumQHeads * qda::kHeadDim * sizeof(uint16_t),
+                        cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return QDA_ERR_CUDA;
+    return QDA_OK;
+}
+
+int qwen3_decode_attn_check(qda_handle* h, void* cuda_stream) {
+    if (h == nullptr) return QDA_ERR_INVALID_ARG;
+    DeviceGuard guard(h->device);
+    if (!guard.ok()) return QDA_ERR_CUDA;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess) return QDA_ERR_CUDA;
+    int status = 0;
+    if (cudaMemcpy(&status, h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return QDA_ERR_CUDA;
+    if (status != 0) {
+        // an aborted launch may leave merge counters mid-count: start them over
+        if (cudaMemset(h->status, 0, sizeof(int)) != cudaSuccess ||
+            cudaMemset(h->counters, 0, (size_t)qda::kMaxBatch * qda::kNumKvHeads * sizeof(int)) != cudaSuccess ||
+            cudaDeviceSynchronize() != cudaSuccess)
+            return QDA_ERR_CUDA;
+    }
+    return status;
+}
+
+int qwen3_decode_attn_grid_ctas(const qda_handle* h) { return h == nullptr ? 0 : h->grid; }
+
+void qwen3_decode_attn_destroy(qda_handle* h) {
+    if (h == nullptr) return;
+    {
+        DeviceGuard guard(h->device);
+        free_workspace(h);
+    }
+    delete h;
+}
+
+const char* qwen3_decode_attn_strerror(int code) {
+    switch (code) {
+        case QDA_OK: return "success";
+        case QDA_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, or a size outside its range)";
+        case QDA_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+        case QDA_ERR_UNSUPPORTED: return "configuration differs from the compiled head geometry (16/8/128, page 16)";
+        case QDA_ERR_BOUNDS: return "a seq_len or block-table entry was out of range on the device";
+        case QDA_ERR_TIMEOUT: return "a device-side wait ran out of time";
+        default: return "unknown error code";
+    }
+}
+
+}  // extern "C"

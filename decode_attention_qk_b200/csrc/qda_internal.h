@@ -1,0 +1,65 @@
+// Internal interface between the C-ABI host code and the decode-attention
+// kernel. Not installed; the public boundary is include/qwen3_decode_attn.h.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace qda {
+
+// Geometry of Qwen3-0.6B attention (Model Spec, "Published configuration").
+constexpr int kNumQHeads = 16;
+constexpr int kNumKvHeads = 8;
+constexpr int kGroup = kNumQHeads / kNumKvHeads;   // query heads per kv head
+constexpr int kHeadDim = 128;
+constexpr int kPage = 16;                          // tokens per cache page
+constexpr int kQkvWidth = 4096;                    // 2048 q | 1024 k | 1024 v
+constexpr int kMaxBatch = 256;
+constexpr int kMaxSeqLen = 40960;
+constexpr int kMaxGridCtas = 4096;
+
+// One token row of a page holds every kv head: 8 x 128 bf16 = 2 KiB; a page of
+// one cache is 16 rows = 32 KiB, contiguous.
+constexpr int kRowBytes = kNumKvHeads * kHeadDim * 2;
+constexpr int kPageBytes = kPage * kRowBytes;
+
+// Everything one launch needs. Pointers are device pointers.
+struct Params {
+    const uint16_t* qkv;          // bf16 [B][4096]
+    const uint16_t* q_norm_w;     // bf16 [128]
+    const uint16_t* k_norm_w;     // bf16 [128]
+    const int32_t* seq_lens;      // [B]
+    const int32_t* positions;     // [B] or nullptr
+    const int32_t* block_table;   // [B][bt_stride]
+    uint16_t* k_cache;            // bf16 [num_pages][16][8][128]
+    uint16_t* v_cache;
+    uint16_t* o;                  // bf16 [B][16][128]
+    int bt_stride;
+    int num_pages;
+    int batch;
+    int max_seq_len;
+    double rope_theta;
+    double rms_eps;
+    // workspace
+    float* part_acc;              // [num_slots][16][128] un-normalised partial sums
+    float2* part_ml;              // [num_slots][16] (running max in log2 units, sum)
+    int* counters;                // [kMaxBatch][8] merge arrival counters, zero between calls
+    int* status;                  // sticky device error (0 = none)
+    int64_t timeout_ns;           // limit of every device-side wait
+    unsigned flags;
+};
+
+// Scratch a launch with `grid` CTAs and batches up to `max_batch` needs.
+inline int64_t num_slots(int grid, int max_batch) { return (int64_t)grid + max_batch; }
+
+// Dynamic shared memory of one CTA.
+size_t smem_bytes();
+
+// Prepare the kernel for launch on the current device (raises its dynamic
+// shared-memory limit). Returns the first CUDA error.
+cudaError_t prepare_device();
+
+// Launch one decode-attention step with `grid` CTAs on `stream`.
+cudaError_t launch(const Params& p, int grid, cudaStream_t stream);
+
+}  // namespace qda

@@ -1,0 +1,154 @@
+"""Helpers that compare the CUDA library with the float64 oracle.
+
+Tolerances for o (bf16 output of a float computation):
+  gate    max |o - o_ref| <= 2e-2 and ||o - o_ref|| / ||o_ref|| <= 1e-2 over
+          the whole output (the required tolerance);
+  strict  |o - o_ref| <= 2^-8 |o_ref| + 1e-4 element by element: one bf16
+          rounding of o (at most 2^-9 relative) plus float error in the
+          scores, exp2 and sums (~1e-5 absolute at O(1) values). It catches
+          a dropped or doubled token, which the gate alone would not.
+The cache is compared bit for bit.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from decode_attention_qk_b200 import inputs
+
+GATE_ABS, GATE_REL = 2e-2, 1e-2
+STRICT_REL, STRICT_ABS = 2.0 ** -8, 1e-4
+
+
+def device_args(w: inputs.Workload, dev, positions=None):
+    """The per-step tensors of a workload on `dev` (caches are used in place)."""
+    pos = positions if positions is not None else w.positions
+    return dict(qkv=w.qkv.to(dev), q_norm_w=w.q_norm_w.to(dev), k_norm_w=w.k_norm_w.to(dev),
+                seq_lens=w.seq_lens.to(dev), block_table=w.block_table.to(dev),
+                positions=None if pos is None else pos.to(dev))
+
+
+def run(attn, w: inputs.Workload, dev, k_cache, v_cache, positions=None, o=None):
+    a = device_args(w, dev, positions)
+    o = attn(a["qkv"], a["q_norm_w"], a["k_norm_w"], a["seq_lens"], a["block_table"], k_cache, v_cache,
+             o=o, positions=a["positions"])
+    return o
+
+
+def oracle_full(w: inputs.Workload, k_cache_pre, v_cache_pre, positions=None):
+    """The oracle on the whole batch; caches given as tensors (any device), pre-call."""
+    pos = positions if positions is not None else w.positions
+    return oracle.append_and_attend(
+        inputs.bf16_bits(w.qkv), inputs.bf16_bits(w.q_norm_w), inputs.bf16_bits(w.k_norm_w),
+        w.seq_lens.numpy(), w.block_table.numpy(), inputs.bf16_bits(k_cache_pre), inputs.bf16_bits(v_cache_pre),
+        positions=None if pos is None else pos.cpu().numpy(), inplace=True, want_qk=True)
+
+
+def _compact(w, seqs, k_pre, v_pre, last_page_only=False):
+    """A sub-batch of the sequences `seqs` over a pool holding only their pages."""
+    lens = w.seq_lens[seqs]
+    rows, pages = [], []
+    for b in seqs.tolist():
+        n = (int(w.seq_lens[b]) + 15) // 16
+        ids = w.block_table[b, n - 1:n] if last_page_only else w.block_table[b, :n]
+        rows.append(torch.arange(len(pages), len(pages) + len(ids), dtype=torch.int32))
+        pages.extend(ids.tolist())
+    stride = max(len(r) for r in rows)
+    bt = torch.full((len(seqs), stride), -1, dtype=torch.int32)
+    for i, r in enumerate(rows):
+        bt[i, :len(r)] = r
+    idx = torch.tensor(pages, dtype=torch.int64, device=k_pre.device)
+    kc = inputs.bf16_bits(k_pre.index_select(0, idx))
+    vc = inputs.bf16_bits(v_pre.index_select(0, idx))
+    return lens, bt, kc, vc
+
+
+def oracle_sampled(w: inputs.Workload, seqs, k_pre, v_pre):
+    """Oracle o for the sequences `seqs` only ([len(seqs), 16, 128] float64)."""
+    seqs = torch.as_tensor(seqs, dtype=torch.int64)
+    lens, bt, kc, vc = _compact(w, seqs, k_pre, v_pre)
+    pos = None if w.positions is None else w.positions[seqs].numpy()
+    out = oracle.append_and_attend(
+        inputs.bf16_bits(w.qkv[seqs.to(w.qkv.device)]), inputs.bf16_bits(w.q_norm_w),
+        inputs.bf16_bits(w.k_norm_w), lens.numpy(), bt.numpy(), kc, vc, positions=pos, inplace=True)
+    return out["o"]
+
+
+def oracle_appended_rows(w: inputs.Workload, k_pre, v_pre):
+    """The oracle's appended k/v rows for every sequence, cheaply: each sequence is
+    replaced by its last page alone, with its true RoPE position.
+
+    Returns (k_rows, v_rows) uint16 [B, 8, 128] and k64, the new k in float64.
+    """
+    B = w.batch
+    seqs = torch.arange(B)
+    lens, bt, kc, vc = _compact(w, seqs, k_pre, v_pre, last_page_only=True)
+    short = ((lens - 1) % 16 + 1).to(torch.int32)
+    pos = (w.seq_lens - 1) if w.positions is None else w.positions
+    out = oracle.append_and_attend(
+        inputs.bf16_bits(w.qkv), inputs.bf16_bits(w.q_norm_w), inputs.bf16_bits(w.k_norm_w), short.numpy(),
+        bt.numpy(), kc, vc, positions=pos.numpy().astype(np.int32), inplace=True, want_qk=True)
+    rows = ((short - 1) % 16).numpy()
+    k_rows = np.stack([out["k_cache"][b, rows[b]] for b in range(B)])
+    v_rows = np.stack([out["v_cache"][b, rows[b]] for b in range(B)])
+    return k_rows, v_rows, out["k"]
+
+
+def expected_cache(w: inputs.Workload, k_pre, v_pre, k_rows, v_rows):
+    """The pre-call caches (device) with each sequence's appended row written in."""
+    k_exp, v_exp = k_pre.clone(), v_pre.clone()
+    dev = k_pre.device
+    for b in range(w.batch):
+        L = int(w.seq_lens[b])
+        page, row = int(w.block_table[b, (L - 1) // 16]), (L - 1) % 16
+        k_exp[page, row] = torch.from_numpy(k_rows[b].view(np.int16)).view(torch.bfloat16).to(dev)
+        v_exp[page, row] = torch.from_numpy(v_rows[b].view(np.int16)).view(torch.bfloat16).to(dev)
+    return k_exp, v_exp
+
+
+def describe_k_mismatch(got_bits, want_bits, k64):
+    """For a differing appended k, how far the float64 value sat from a bf16 midpoint."""
+    bad = np.argwhere(got_bits != want_bits)
+    lines = []
+    for idx in bad[:8]:
+        x = float(k64[tuple(idx)])
+        lo = oracle.bf16_to_f64(np.array([want_bits[tuple(idx)]], np.uint16))[0]
+        hi = oracle.bf16_to_f64(np.array([got_bits[tuple(idx)]], np.uint16))[0]
+        mid = (lo + hi) / 2
+        lines.append(f"{tuple(idx)}: k64={x!r} gpu={hi!r} oracle={lo!r} |k64-mid|/|k64|={abs(x - mid) / abs(x):.3g}")
+    return f"{len(bad)} appended k values differ:\n" + "\n".join(lines)
+
+
+def assert_cache_equal(k_got, v_got, k_exp, v_exp, k64=None, w=None):
+    if torch.equal(k_got.view(torch.int16), k_exp.view(torch.int16)) and \
+            torch.equal(v_got.view(torch.int16), v_exp.view(torch.int16)):
+        return
+    msg = "cache differs from the oracle"
+    if k64 is not None and w is not None:
+        gb, wb = [], []
+        for b in range(w.batch):
+            L = int(w.seq_lens[b])
+            page, row = int(w.block_table[b, (L - 1) // 16]), (L - 1) % 16
+            gb.append(inputs.bf16_bits(k_got[page, row]))
+            wb.append(inputs.bf16_bits(k_exp[page, row]))
+        msg += "\n" + describe_k_mismatch(np.stack(gb), np.stack(wb), k64)
+    kd = (k_got.view(torch.int16) != k_exp.view(torch.int16)).nonzero()[:5].tolist()
+    vd = (v_got.view(torch.int16) != v_exp.view(torch.int16)).nonzero()[:5].tolist()
+    raise AssertionError(f"{msg}; first k diffs {kd}, v diffs {vd}")
+
+
+def o_errors(o_got, o_ref):
+    got = o_got.detach().float().cpu().numpy().astype(np.float64)
+    ref = np.asarray(o_ref, dtype=np.float64)
+    err = np.abs(got - ref)
+    rel = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+    strict_excess = float(np.max(err - (STRICT_REL * np.abs(ref) + STRICT_ABS)))
+    return float(err.max()), rel, strict_excess
+
+
+def assert_o_close(o_got, o_ref, label=""):
+    max_abs, rel, strict_excess = o_errors(o_got, o_ref)
+    assert max_abs <= GATE_ABS and rel <= GATE_REL, f"{label}: max abs {max_abs:.3g}, rel rms {rel:.3g}"
+    assert strict_excess <= 0.0, f"{label}: strict bound exceeded by {strict_excess:.3g} (max abs {max_abs:.3g})"
+    return max_abs, rel

@@ -1,0 +1,68 @@
+"""Host logic of bench.py, on the CPU: byte counts, the JSON contract's
+reductions over ranks (gloo, world size 2) and rank-distinct replicas."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+from decode_attention_qk_b200 import inputs
+
+
+def test_byte_counts():
+    L = torch.tensor([1, 16, 17, 4096], dtype=torch.int32)
+    assert bench.kv_bytes(L) == int(L.sum()) * 4096
+    pages = 1 + 1 + 2 + 256
+    want = (0 + 15 + 16 + 4095) * 4096 + 4 * 4096 + 4 * 8192 + 4 * 4096 + pages * 4 + 4 * 4 + 512
+    assert bench.algorithmic_bytes(L) == want
+
+
+def test_cpu_baseline_sample_is_bounded():
+    layers = [inputs.custom([100, 200, 300, 400], seed=1)]
+    picked, total = bench.pick_sample(layers, 250 * 4096)
+    assert picked == [(0, [0, 1])] and total == 300 * 4096
+    picked, total = bench.pick_sample(layers, 1)
+    assert picked == [(0, [0])]
+
+
+def test_replicas_differ_by_rank():
+    a = bench.make_layers("cfg1", "cpu", 0)[0]
+    b = bench.make_layers("cfg1", "cpu", 1)[0]
+    assert not torch.equal(a.qkv, b.qkv)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    ms = [3.0, 5.0][rank]                 # per-rank elapsed time
+    nbytes = [100.0, 300.0][rank]         # per-rank KV bytes per step
+    mx = bench.reduce_max(dist, ms, torch.device("cpu"))
+    tot = bench.reduce_sum(dist, nbytes, torch.device("cpu"))
+    q.put((rank, mx, tot))
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(120)
+def test_reductions_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(90)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=5) for _ in range(2))
+    assert got == [(0, 5.0, 400.0), (1, 5.0, 400.0)]
