@@ -10,6 +10,7 @@ _BINDING_NAMES = {
     "DecodeAttention", "QdaError", "qda_config", "load_library", "LIBRARY_PATH",
     "qwen3_decode_attn_default_config", "qwen3_decode_attn_create",
     "qwen3_decode_attn_append_and_attend", "qwen3_decode_attn_append_and_attend_host",
+    "qwen3_decode_attn_append_and_attend_noalloc",
     "qwen3_decode_attn_check", "qwen3_decode_attn_destroy", "qwen3_decode_attn_strerror",
 }
 

@@ -178,6 +178,25 @@ def qwen3_decode_attn_append_and_attend_host(handle, qkv, q_norm_w, k_norm_w, se
         raise QdaError(rc, "qwen3_decode_attn_append_and_attend_host")
 
 
+def qwen3_decode_attn_append_and_attend_noalloc(qkv, q_norm_w, k_norm_w, seq_lens, positions,
+                                                block_table, k_cache, v_cache, o, stream=None) -> None:
+    """The step without a handle, for callers that cannot allocate device memory:
+    its scratch is a fixed array inside the library (see the C header). Runs on
+    the current device, asynchronously on `stream`; raises QdaError on a
+    host-side error."""
+    dev = qkv.device
+    if dev.type != "cuda":
+        raise ValueError("qkv must be a CUDA tensor")
+    args = _step_args(qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, k_cache, v_cache, o, dev, dev)
+    f = load_library().qwen3_decode_attn_append_and_attend_noalloc
+    vp, i32p = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32)
+    f.argtypes = [vp, vp, vp, i32p, i32p, i32p, ctypes.c_int, vp, vp, ctypes.c_int, vp, ctypes.c_int, vp]
+    f.restype = ctypes.c_int
+    rc = f(*args, _stream(stream, dev))
+    if rc != QDA_OK:
+        raise QdaError(rc, "qwen3_decode_attn_append_and_attend_noalloc")
+
+
 def qwen3_decode_attn_check(handle, stream=None, device=None) -> int:
     """Synchronize the stream and return (and clear) the device status code."""
     return int(load_library().qwen3_decode_attn_check(handle, _stream(stream, device)))

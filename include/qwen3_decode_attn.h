@@ -186,6 +186,51 @@ int qwen3_decode_attn_append_and_attend_host(qda_handle *h,
                                              int batch,
                                              void *cuda_stream);
 
+/* The same step for callers that must not allocate device memory. The pages
+ * have no counterpart of this entry point; it exists for users of this
+ * library who cannot call cudaMalloc: code embedded in a framework or server
+ * that owns all device memory through its own pool and forbids allocations on
+ * the side, plugins that are handed only pre-allocated buffers, and
+ * latency-critical loops where an allocation (which can synchronize the
+ * device, or fail for lack of memory at call time) is not acceptable. It needs
+ * no handle, and it allocates and frees nothing.
+ *
+ * It computes what qwen3_decode_attn_append_and_attend computes, with the
+ * Qwen3-0.6B constants (theta 1e6, eps 1e-6, max_seq_len 40960), on the
+ * calling thread's current device; every pointer is a device pointer of that
+ * device, with the layouts and alignment stated above. The caller still
+ * passes every input and output. The kernel's scratch (partials of sequences
+ * split across CTAs, merge counters, a status word) is one fixed device array
+ * of 3,469,568 bytes that every GPU which loads the library holds until the
+ * process exits. It is sized for at most 256 sequences per call (a larger
+ * batch returns QDA_ERR_INVALID_ARG) and at most 160 CTAs per launch (the call
+ * launches min(SM count, 160)).
+ *
+ * The first call on each device performs a one-time set-up there (it looks up
+ * the array's device address and raises the kernel's shared-memory limit);
+ * make that first call before any stream capture. Each call then zeroes the
+ * merge counters and the status word on `cuda_stream` before it launches. All
+ * calls share the one array, which keeps the last call's contents: calls that
+ * overlap on the GPU (different streams or threads without ordering between
+ * them) race on it and produce wrong results. Device-side errors (an
+ * out-of-range seq_len or page id) are not reported by this entry point,
+ * though the kernel still never reads or writes out of range.
+ * Errors: INVALID_ARG (as for qwen3_decode_attn_append_and_attend, or batch
+ * > 256), CUDA (the set-up, the memset or the launch failed). */
+int qwen3_decode_attn_append_and_attend_noalloc(const void *qkv,
+                                                const void *q_norm_w,
+                                                const void *k_norm_w,
+                                                const int32_t *seq_lens,
+                                                const int32_t *positions,
+                                                const int32_t *block_table,
+                                                int block_table_stride,
+                                                void *k_cache,
+                                                void *v_cache,
+                                                int num_pages,
+                                                void *o,
+                                                int batch,
+                                                void *cuda_stream);
+
 /* Synchronize `cuda_stream`, read and clear the status word, and return the
  * first device error recorded since the last check (QDA_OK if none;
  * QDA_ERR_BOUNDS or QDA_ERR_TIMEOUT otherwise). After an error the handle's
