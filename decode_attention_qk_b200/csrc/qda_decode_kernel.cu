@@ -22,20 +22,23 @@
 //
 // Inside a CTA. Warp 8 is the producer: lane 0 issues one bulk copy of the
 // K rows and one of the V rows of a page (up to 32 KiB each, all 8 kv heads)
-// into a 3-stage shared-memory ring, completed on an mbarrier. Warps 0..7 are
+// into a 3-stage shared-memory ring, completed on an mbarrier; with the first
+// page of each sequence piece it also copies that sequence's 8 KiB qkv row,
+// so consumers never wait on a global load of their own. Warps 0..7 are
 // consumers; warp j serves kv head j and both query heads 2j, 2j+1 that read
 // it (nnterp qwen3, "Grouped-query attention"), so every K/V byte is read from
 // HBM once. Lane (grp = lane/8, c = lane%8) owns head dims [8c, 8c+8) and
-// [64+8c, 64+8c+8) and the tokens 4i + grp of each page; each of the 4 token
-// groups keeps its own running max per head, so the only cross-lane work per
-// page is a 3-step reduce-scatter of 8 partial dot products, a 3-step max and
-// an 8-way gather of probabilities.
+// [64+8c, 64+8c+8) -- the two halves of the rotation pairs 8c..8c+7 -- and
+// the tokens 4i + grp of each page; each of the 4 token groups keeps its own
+// running max per head, so the only cross-lane work per page is a 3-step
+// reduce-scatter of 8 partial dot products, a 3-step max and an 8-way gather
+// of probabilities. Products use the packed two-float FMA of sm_100.
 //
-// q and the new k are normed and rotated in double precision; q is kept in
-// float, pre-multiplied by log2(e)/sqrt(128) so scores are in log2 units; the
-// new k is rounded once to bf16 (nearest-even) and both written to the cache
-// and patched into the staged page, so it never makes a round trip through
-// HBM. Every wait is bounded in time; on expiry the kernel records
+// Numbers. q and the new k are normed and rotated in double precision; q is
+// kept in float, pre-multiplied by log2(e)/sqrt(128) so scores are in log2
+// units; the new k is rounded once to bf16 (nearest-even) and both written to
+// the cache and patched into the staged page, so it never makes a round trip
+// through HBM. Every wait is bounded in time; on expiry the kernel records
 // QDA_ERR_TIMEOUT, stops issuing work, drains its own copies and returns.
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -52,18 +55,32 @@ constexpr int kThreads = (kConsumerWarps + 1) * 32;   // + the producer warp
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr float kRescaleThreshold = 8.0f;             // log2 units: rescale only when the max grows by > 2^8
 constexpr double kQScale = 1.4426950408889634 * 0.088388347648318441;  // log2(e) / sqrt(128)
+constexpr int kQkvBytes = kQkvWidth * 2;              // one bf16 qkv row: 8 KiB
 
-// Shared-memory layout (bytes).
-constexpr int kStageBytes = 2 * kPageBytes;           // K rows, then V rows
-constexpr int kSmemQ = kStages * kStageBytes;         // per consumer warp: float [2][128]
-constexpr int kSmemSeg = kSmemQ + kConsumerWarps * kGroup * kHeadDim * 4;  // int [kMaxBatch + 4]
+// Shared-memory layout (bytes). A stage holds the K rows and V rows of one
+// page and, for the first page of a sequence piece, the sequence's qkv row.
+constexpr int kStageK = 0;
+constexpr int kStageV = kPageBytes;
+constexpr int kStageQkv = 2 * kPageBytes;
+constexpr int kStageBytes = 2 * kPageBytes + kQkvBytes;
+constexpr int kSmemSeg = kStages * kStageBytes;                            // int [kMaxBatch + 4]
 constexpr int kSmemLens = kSmemSeg + (kMaxBatch + 4) * 4;                  // int [kMaxBatch]
 constexpr int kSmemInvFreq = kSmemLens + kMaxBatch * 4;                    // double [64]
-constexpr int kSmemBars = kSmemInvFreq + 64 * 8;                           // uint64 [2*kStages + 1]
-constexpr int kSmemFlags = kSmemBars + (2 * kStages + 1) * 8;              // int [kStages] + abort
-constexpr int kSmemTotal = kSmemFlags + 8 * 4;
-static_assert(kSmemInvFreq % 8 == 0 && kSmemBars % 8 == 0, "8-byte alignment");
+constexpr int kSmemGains = kSmemInvFreq + 64 * 8;                          // bf16 [2][128]
+constexpr int kSmemMeta = kSmemGains + 2 * kHeadDim * 2;                   // StageMeta [kStages]
+constexpr int kSmemBars = kSmemMeta + kStages * 16;                        // uint64 [2*kStages + 1]
+constexpr int kSmemFlags = kSmemBars + (2 * kStages + 1) * 8;              // abort flag
+constexpr int kSmemTotal = kSmemFlags + 16;
+static_assert(kStageBytes % 128 == 0 && kSmemInvFreq % 8 == 0 && kSmemBars % 8 == 0, "alignment");
 static_assert(kSmemTotal <= 227 * 1024, "fits one CTA per SM");
+
+// What the producer tells the consumers about a stage.
+struct StageMeta {
+    int page;   // cache page id of the staged page
+    int bad;    // the block-table entry was out of range: nothing was copied
+    int pos;    // RoPE position of the sequence (valid when a qkv row was staged)
+    int pad;
+};
 
 // ---------------------------------------------------------------------------
 // PTX wrappers: mbarrier, bulk copy, timer, exp2
@@ -166,44 +183,80 @@ __device__ __forceinline__ double warp_sum(double v) {
     return v;
 }
 
-// Partial dot product of 16 q values with 16 bf16 k values (two 16-byte rows).
-__device__ __forceinline__ float dot16(const float* q, const uint4& lo, const uint4& hi) {
-    float a = q[0] * bf_lo(lo.x);
-    float b = q[8] * bf_lo(hi.x);
-    a = fmaf(q[1], bf_hi(lo.x), a);
-    b = fmaf(q[9], bf_hi(hi.x), b);
-    a = fmaf(q[2], bf_lo(lo.y), a);
-    b = fmaf(q[10], bf_lo(hi.y), b);
-    a = fmaf(q[3], bf_hi(lo.y), a);
-    b = fmaf(q[11], bf_hi(hi.y), b);
-    a = fmaf(q[4], bf_lo(lo.z), a);
-    b = fmaf(q[12], bf_lo(hi.z), b);
-    a = fmaf(q[5], bf_hi(lo.z), a);
-    b = fmaf(q[13], bf_hi(hi.z), b);
-    a = fmaf(q[6], bf_lo(lo.w), a);
-    b = fmaf(q[14], bf_lo(hi.w), b);
-    a = fmaf(q[7], bf_hi(lo.w), a);
-    b = fmaf(q[15], bf_hi(hi.w), b);
-    return a + b;
+// Two floats in one 64-bit register pair (low word first), for the packed
+// f32x2 arithmetic of sm_100: one instruction does two float FMAs.
+typedef unsigned long long f32x2;
+
+__device__ __forceinline__ f32x2 pack2(float lo, float hi) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
 }
 
-__device__ __forceinline__ void axpy16(float* acc, float p, const uint4& lo, const uint4& hi) {
-    acc[0] = fmaf(p, bf_lo(lo.x), acc[0]);
-    acc[1] = fmaf(p, bf_hi(lo.x), acc[1]);
-    acc[2] = fmaf(p, bf_lo(lo.y), acc[2]);
-    acc[3] = fmaf(p, bf_hi(lo.y), acc[3]);
-    acc[4] = fmaf(p, bf_lo(lo.z), acc[4]);
-    acc[5] = fmaf(p, bf_hi(lo.z), acc[5]);
-    acc[6] = fmaf(p, bf_lo(lo.w), acc[6]);
-    acc[7] = fmaf(p, bf_hi(lo.w), acc[7]);
-    acc[8] = fmaf(p, bf_lo(hi.x), acc[8]);
-    acc[9] = fmaf(p, bf_hi(hi.x), acc[9]);
-    acc[10] = fmaf(p, bf_lo(hi.y), acc[10]);
-    acc[11] = fmaf(p, bf_hi(hi.y), acc[11]);
-    acc[12] = fmaf(p, bf_lo(hi.z), acc[12]);
-    acc[13] = fmaf(p, bf_hi(hi.z), acc[13]);
-    acc[14] = fmaf(p, bf_lo(hi.w), acc[14]);
-    acc[15] = fmaf(p, bf_hi(hi.w), acc[15]);
+__device__ __forceinline__ float2 unpack2(f32x2 v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// A word holding two bf16 (first element in the low half) as two floats.
+__device__ __forceinline__ f32x2 bf2(uint32_t w) { return pack2(bf_lo(w), bf_hi(w)); }
+
+// Partial dot products of one staged k row (this lane's 16 dims: words 0..3
+// are dims 8c..8c+7, words 4..7 dims 64+8c..64+8c+7) with both query heads.
+__device__ __forceinline__ void dot_row(const f32x2* q0, const f32x2* q1, const uint4& lo, const uint4& hi,
+                                        float& d0, float& d1) {
+    const f32x2 k0 = bf2(lo.x), k1 = bf2(lo.y), k2 = bf2(lo.z), k3 = bf2(lo.w);
+    const f32x2 k4 = bf2(hi.x), k5 = bf2(hi.y), k6 = bf2(hi.z), k7 = bf2(hi.w);
+    f32x2 a0 = mul2(q0[0], k0), b0 = mul2(q0[4], k4);
+    f32x2 a1 = mul2(q1[0], k0), b1 = mul2(q1[4], k4);
+    a0 = fma2(q0[1], k1, a0);
+    b0 = fma2(q0[5], k5, b0);
+    a1 = fma2(q1[1], k1, a1);
+    b1 = fma2(q1[5], k5, b1);
+    a0 = fma2(q0[2], k2, a0);
+    b0 = fma2(q0[6], k6, b0);
+    a1 = fma2(q1[2], k2, a1);
+    b1 = fma2(q1[6], k6, b1);
+    a0 = fma2(q0[3], k3, a0);
+    b0 = fma2(q0[7], k7, b0);
+    a1 = fma2(q1[3], k3, a1);
+    b1 = fma2(q1[7], k7, b1);
+    const float2 r0 = unpack2(add2(a0, b0));
+    const float2 r1 = unpack2(add2(a1, b1));
+    d0 = r0.x + r0.y;
+    d1 = r1.x + r1.y;
+}
+
+// acc_h += p_h * v for one staged v row (same dim layout as dot_row).
+__device__ __forceinline__ void axpy_row(f32x2* acc0, f32x2* acc1, float p0, float p1, const uint4& lo,
+                                         const uint4& hi) {
+    const f32x2 pp0 = pack2(p0, p0), pp1 = pack2(p1, p1);
+    const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const f32x2 v = bf2(w[k]);
+        acc0[k] = fma2(pp0, v, acc0[k]);
+        acc1[k] = fma2(pp1, v, acc1[k]);
+    }
 }
 
 // Largest b in [0, B) with seg[b] <= page: the sequence holding global page
@@ -220,19 +273,19 @@ __device__ __forceinline__ int find_seq(const int* seg, int B, int page) {
 
 struct Shared {
     uint8_t* stages;
-    float* q;
     int* seg;        // seg[b] = first global page of sequence b; seg[B] = P
     int* lens;       // seq_lens as read
     double* inv_freq;
+    const uint16_t* gains;  // q_norm_w then k_norm_w
+    volatile StageMeta* meta;
     uint64_t* full_bar;
     uint64_t* empty_bar;
     uint64_t* never_bar;
-    volatile int* slot_bad;
     volatile int* abort_flag;
 };
 
 // ---------------------------------------------------------------------------
-// Producer warp: stream the CTA's pages into the ring.
+// Producer warp: stream the CTA's pages (and each piece's qkv row) into the ring.
 
 __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, int B, int start, int end, int lane) {
     const int count = end - start;
@@ -241,9 +294,9 @@ __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, i
     uint32_t armed = 0, armed_parity = 0;   // lane 0: slots with a phase armed, and its parity
     bool aborted = false;
     for (int base = 0; base < count && !aborted; base += 32) {
-        // 32 pages' ids fetched at once, one per lane.
+        // 32 pages' descriptions fetched at once, one per lane.
         const int gp = start + base + lane;
-        int id = 0, rows = 0;
+        int id = 0, rows = 0, qkv_b = -1, pos = 0;
         if (gp < end) {
             const int b = find_seq(s.seg, B, gp);
             const int i = gp - s.seg[b];
@@ -252,26 +305,41 @@ __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, i
             // the sequence's last page holds the new token at row (L-1)%16; only
             // the rows before it are read from the cache
             rows = (i == nb - 1) ? (s.lens[b] - 1) - kPage * i : kPage;
+            if (gp == start || i == 0) {
+                qkv_b = b;
+                pos = p.positions != nullptr ? __ldg(p.positions + b) : s.lens[b] - 1;
+            }
         }
         const int n = min(32, count - base);
         for (int kk = 0; kk < n; ++kk) {
             const int page_id = __shfl_sync(kFull, id, kk);
             const int page_rows = __shfl_sync(kFull, rows, kk);
+            const int seq_qkv = __shfl_sync(kFull, qkv_b, kk);
+            const int seq_pos = __shfl_sync(kFull, pos, kk);
             int ok = 1;
             if (lane == 0) {
-                ok = mbar_wait(&s.empty_bar[slot], phase ^ 1u, p.timeout_ns, s.abort_flag);
+                ok = mbar_try_wait(&s.empty_bar[slot], phase ^ 1u) ||
+                     mbar_wait(&s.empty_bar[slot], phase ^ 1u, p.timeout_ns, s.abort_flag);
                 if (ok) {
                     const bool bad = page_id < 0 || page_id >= p.num_pages;
-                    s.slot_bad[slot] = bad ? 1 : 0;
+                    s.meta[slot].page = page_id;
+                    s.meta[slot].bad = bad ? 1 : 0;
+                    s.meta[slot].pos = seq_pos;
                     if (bad) record_error(p.status, QDA_ERR_BOUNDS);
-                    const uint32_t bytes = bad ? 0u : (uint32_t)page_rows * kRowBytes;
-                    if (bytes != 0) {
+                    const uint32_t kv_bytes = bad ? 0u : (uint32_t)page_rows * kRowBytes;
+                    const uint32_t qkv_bytes = seq_qkv >= 0 ? (uint32_t)kQkvBytes : 0u;
+                    if (kv_bytes + qkv_bytes != 0) {
                         uint8_t* dst = s.stages + slot * kStageBytes;
                         const size_t off = (size_t)page_id * kPageBytes;
-                        mbar_arrive_expect_tx(&s.full_bar[slot], 2u * bytes);
-                        bulk_g2s(dst, reinterpret_cast<const uint8_t*>(p.k_cache) + off, bytes, &s.full_bar[slot]);
-                        bulk_g2s(dst + kPageBytes, reinterpret_cast<const uint8_t*>(p.v_cache) + off, bytes,
-                                 &s.full_bar[slot]);
+                        mbar_arrive_expect_tx(&s.full_bar[slot], 2u * kv_bytes + qkv_bytes);
+                        if (qkv_bytes != 0)
+                            bulk_g2s(dst + kStageQkv, p.qkv + (size_t)seq_qkv * kQkvWidth, qkv_bytes, &s.full_bar[slot]);
+                        if (kv_bytes != 0) {
+                            bulk_g2s(dst + kStageK, reinterpret_cast<const uint8_t*>(p.k_cache) + off, kv_bytes,
+                                     &s.full_bar[slot]);
+                            bulk_g2s(dst + kStageV, reinterpret_cast<const uint8_t*>(p.v_cache) + off, kv_bytes,
+                                     &s.full_bar[slot]);
+                        }
                         armed |= 1u << slot;
                         armed_parity = (armed_parity & ~(1u << slot)) | (phase << slot);
                     } else {
@@ -305,69 +373,90 @@ __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, i
 // Consumer warps.
 
 struct HeadState {
-    float q0[16], q1[16];       // query heads 2j, 2j+1 at this lane's 16 dims (log2-scaled)
-    float acc0[16], acc1[16];   // un-normalised outputs of this lane's token group
+    f32x2 q0[8], q1[8];         // query heads 2j, 2j+1 at this lane's 16 dims (log2-scaled), in pairs
+    f32x2 acc0[8], acc1[8];     // un-normalised outputs of this lane's token group, in pairs
     float m0, m1;               // running max of the token group (log2 units)
     float lsum;                 // partial softmax sum of this lane's (token, head) slot
     uint32_t k_lo, k_hi, v_lo, v_hi;  // this lane's words of the appended k/v row
 };
 
-// Norm and rotate q (and, when this CTA appends for sequence b, k), in double.
-// Lane l handles the rotation pairs 2l and 2l+1: dims 2l, 2l+1, 64+2l, 65+2l.
-__device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s, int b, int j, int lane, int c,
-                               bool appends, HeadState& st) {
-    const int L = s.lens[b];
-    const double pos = (double)(p.positions != nullptr ? p.positions[b] : L - 1);
-    double sn0, cs0, sn1, cs1;
-    sincos(pos * s.inv_freq[2 * lane], &sn0, &cs0);
-    sincos(pos * s.inv_freq[2 * lane + 1], &sn1, &cs1);
+__device__ __forceinline__ double warp_sum8(double v) {   // over the 8 lanes of a token group
+    v += __shfl_xor_sync(kFull, v, 1);
+    v += __shfl_xor_sync(kFull, v, 2);
+    v += __shfl_xor_sync(kFull, v, 4);
+    return v;
+}
 
-    const uint16_t* row = p.qkv + (size_t)b * kQkvWidth;
-    float* qs = s.q + j * (kGroup * kHeadDim);
-    const uint32_t wq_lo = *reinterpret_cast<const uint32_t*>(p.q_norm_w + 2 * lane);
-    const uint32_t wq_hi = *reinterpret_cast<const uint32_t*>(p.q_norm_w + 64 + 2 * lane);
-    __syncwarp();  // the previous sequence's q may still be being read
-#pragma unroll
-    for (int h = 0; h < kGroup; ++h) {
-        const uint16_t* x = row + (kGroup * j + h) * kHeadDim;
-        const uint32_t xlo = *reinterpret_cast<const uint32_t*>(x + 2 * lane);
-        const uint32_t xhi = *reinterpret_cast<const uint32_t*>(x + 64 + 2 * lane);
-        double a0 = bf_to_d(xlo & 0xFFFFu), a1 = bf_to_d(xlo >> 16);
-        double b0 = bf_to_d(xhi & 0xFFFFu), b1 = bf_to_d(xhi >> 16);
-        const double r = sqrt(warp_sum(a0 * a0 + a1 * a1 + b0 * b0 + b1 * b1) / 128.0 + p.rms_eps);
-        a0 = a0 / r * bf_to_d(wq_lo & 0xFFFFu);
-        a1 = a1 / r * bf_to_d(wq_lo >> 16);
-        b0 = b0 / r * bf_to_d(wq_hi & 0xFFFFu);
-        b1 = b1 / r * bf_to_d(wq_hi >> 16);
-        const double ra0 = a0 * cs0 - b0 * sn0, rb0 = b0 * cs0 + a0 * sn0;
-        const double ra1 = a1 * cs1 - b1 * sn1, rb1 = b1 * cs1 + a1 * sn1;
-        float2* qh = reinterpret_cast<float2*>(qs + h * kHeadDim);
-        qh[lane] = make_float2((float)(ra0 * kQScale), (float)(ra1 * kQScale));
-        qh[32 + lane] = make_float2((float)(rb0 * kQScale), (float)(rb1 * kQScale));
-    }
-    __syncwarp();
+// Start sequence b: norm and rotate q from the staged qkv row, in double, and,
+// when this CTA holds the sequence's last page, the new k. Lane l computes the
+// rotation angles of pairs 2l and 2l+1; lane (grp, c) then gathers those of
+// pairs 8c..8c+7, whose two halves are exactly its q dims.
+__device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s, const uint8_t* qkv_row, int pos,
+                                               int j, int lane, int c, bool appends, HeadState& st) {
+    double cs0, sn0, cs1, sn1;
     {
-        const float4* q0 = reinterpret_cast<const float4*>(qs + 8 * c);
-        const float4* q0h = reinterpret_cast<const float4*>(qs + 64 + 8 * c);
-        const float4* q1 = reinterpret_cast<const float4*>(qs + kHeadDim + 8 * c);
-        const float4* q1h = reinterpret_cast<const float4*>(qs + kHeadDim + 64 + 8 * c);
-        float4 v;
-        v = q0[0];  st.q0[0] = v.x;  st.q0[1] = v.y;  st.q0[2] = v.z;  st.q0[3] = v.w;
-        v = q0[1];  st.q0[4] = v.x;  st.q0[5] = v.y;  st.q0[6] = v.z;  st.q0[7] = v.w;
-        v = q0h[0]; st.q0[8] = v.x;  st.q0[9] = v.y;  st.q0[10] = v.z; st.q0[11] = v.w;
-        v = q0h[1]; st.q0[12] = v.x; st.q0[13] = v.y; st.q0[14] = v.z; st.q0[15] = v.w;
-        v = q1[0];  st.q1[0] = v.x;  st.q1[1] = v.y;  st.q1[2] = v.z;  st.q1[3] = v.w;
-        v = q1[1];  st.q1[4] = v.x;  st.q1[5] = v.y;  st.q1[6] = v.z;  st.q1[7] = v.w;
-        v = q1h[0]; st.q1[8] = v.x;  st.q1[9] = v.y;  st.q1[10] = v.z; st.q1[11] = v.w;
-        v = q1h[1]; st.q1[12] = v.x; st.q1[13] = v.y; st.q1[14] = v.z; st.q1[15] = v.w;
+        const double fpos = (double)pos;
+        sincos(fpos * s.inv_freq[2 * lane], &sn0, &cs0);
+        sincos(fpos * s.inv_freq[2 * lane + 1], &sn1, &cs1);
+    }
+    // this lane's 16 dims of heads 2j, 2j+1: words 0..3 dims 8c..8c+7, 4..7 dims 64+8c..
+    uint32_t x0[8], x1[8];
+    {
+        const uint8_t* xh = qkv_row + (kGroup * j) * (kHeadDim * 2);
+        const uint4 a0 = *reinterpret_cast<const uint4*>(xh + 16 * c);
+        const uint4 b0 = *reinterpret_cast<const uint4*>(xh + 128 + 16 * c);
+        const uint4 a1 = *reinterpret_cast<const uint4*>(xh + kHeadDim * 2 + 16 * c);
+        const uint4 b1 = *reinterpret_cast<const uint4*>(xh + kHeadDim * 2 + 128 + 16 * c);
+        x0[0] = a0.x; x0[1] = a0.y; x0[2] = a0.z; x0[3] = a0.w; x0[4] = b0.x; x0[5] = b0.y; x0[6] = b0.z; x0[7] = b0.w;
+        x1[0] = a1.x; x1[1] = a1.y; x1[2] = a1.z; x1[3] = a1.w; x1[4] = b1.x; x1[5] = b1.y; x1[6] = b1.z; x1[7] = b1.w;
+    }
+    double ss0 = 0.0, ss1 = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+        const double e0 = bf_to_d(x0[w] & 0xFFFFu), o0 = bf_to_d(x0[w] >> 16);
+        const double e1 = bf_to_d(x1[w] & 0xFFFFu), o1 = bf_to_d(x1[w] >> 16);
+        ss0 = fma(e0, e0, fma(o0, o0, ss0));
+        ss1 = fma(e1, e1, fma(o1, o1, ss1));
+    }
+    const double inv_r0 = 1.0 / sqrt(warp_sum8(ss0) / 128.0 + p.rms_eps);
+    const double inv_r1 = 1.0 / sqrt(warp_sum8(ss1) / 128.0 + p.rms_eps);
+    const uint4 wa = *reinterpret_cast<const uint4*>(s.gains + 8 * c);        // q gains, dims 8c..
+    const uint4 wb = *reinterpret_cast<const uint4*>(s.gains + 64 + 8 * c);   // dims 64+8c..
+    const uint32_t wq[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+    // pair 8c + k: dims 8c+k (word k/2 of the low half) and 64+8c+k (word 4 + k/2)
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        float q0a[2], q0b[2], q1a[2], q1b[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int k = 2 * m + e;
+            const int src = 4 * c + (k >> 1);
+            const double cs = __shfl_sync(kFull, e ? cs1 : cs0, src);
+            const double sn = __shfl_sync(kFull, e ? sn1 : sn0, src);
+            const int sh = e ? 16 : 0;
+            const double wlo = bf_to_d((wq[m] >> sh) & 0xFFFFu), whi = bf_to_d((wq[4 + m] >> sh) & 0xFFFFu);
+            const double ya0 = bf_to_d((x0[m] >> sh) & 0xFFFFu) * inv_r0 * wlo;
+            const double yb0 = bf_to_d((x0[4 + m] >> sh) & 0xFFFFu) * inv_r0 * whi;
+            const double ya1 = bf_to_d((x1[m] >> sh) & 0xFFFFu) * inv_r1 * wlo;
+            const double yb1 = bf_to_d((x1[4 + m] >> sh) & 0xFFFFu) * inv_r1 * whi;
+            q0a[e] = (float)((ya0 * cs - yb0 * sn) * kQScale);
+            q0b[e] = (float)((yb0 * cs + ya0 * sn) * kQScale);
+            q1a[e] = (float)((ya1 * cs - yb1 * sn) * kQScale);
+            q1b[e] = (float)((yb1 * cs + ya1 * sn) * kQScale);
+        }
+        st.q0[m] = pack2(q0a[0], q0a[1]);
+        st.q0[4 + m] = pack2(q0b[0], q0b[1]);
+        st.q1[m] = pack2(q1a[0], q1a[1]);
+        st.q1[4 + m] = pack2(q1b[0], q1b[1]);
     }
 
     if (appends) {
-        const uint16_t* x = row + kNumQHeads * kHeadDim + j * kHeadDim;
-        const uint32_t xlo = *reinterpret_cast<const uint32_t*>(x + 2 * lane);
-        const uint32_t xhi = *reinterpret_cast<const uint32_t*>(x + 64 + 2 * lane);
-        const uint32_t wk_lo = *reinterpret_cast<const uint32_t*>(p.k_norm_w + 2 * lane);
-        const uint32_t wk_hi = *reinterpret_cast<const uint32_t*>(p.k_norm_w + 64 + 2 * lane);
+        // lane l: dims 2l, 2l+1 (word l of the head) and 64+2l, 65+2l (word 32+l)
+        const uint32_t* xk = reinterpret_cast<const uint32_t*>(qkv_row + (kNumQHeads + j) * (kHeadDim * 2));
+        const uint32_t* xv = reinterpret_cast<const uint32_t*>(qkv_row + (kNumQHeads + kNumKvHeads + j) * (kHeadDim * 2));
+        const uint32_t* gk = reinterpret_cast<const uint32_t*>(s.gains + kHeadDim);
+        const uint32_t xlo = xk[lane], xhi = xk[32 + lane];
+        const uint32_t wk_lo = gk[lane], wk_hi = gk[32 + lane];
         double a0 = bf_to_d(xlo & 0xFFFFu), a1 = bf_to_d(xlo >> 16);
         double b0 = bf_to_d(xhi & 0xFFFFu), b1 = bf_to_d(xhi >> 16);
         const double r = sqrt(warp_sum(a0 * a0 + a1 * a1 + b0 * b0 + b1 * b1) / 128.0 + p.rms_eps);
@@ -379,35 +468,23 @@ __device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s,
         const double ra1 = a1 * cs1 - b1 * sn1, rb1 = b1 * cs1 + a1 * sn1;
         st.k_lo = d_to_bf(ra0) | (d_to_bf(ra1) << 16);
         st.k_hi = d_to_bf(rb0) | (d_to_bf(rb1) << 16);
-        const uint16_t* v = row + (kNumQHeads + kNumKvHeads) * kHeadDim + j * kHeadDim;
-        st.v_lo = *reinterpret_cast<const uint32_t*>(v + 2 * lane);
-        st.v_hi = *reinterpret_cast<const uint32_t*>(v + 64 + 2 * lane);
-
-        const int nb = s.seg[b + 1] - s.seg[b];
-        const int page = p.block_table[(size_t)b * p.bt_stride + nb - 1];
-        if (page >= 0 && page < p.num_pages) {
-            const size_t off = (size_t)page * (kPageBytes / 2) + (size_t)((L - 1) % kPage) * (kRowBytes / 2) +
-                               (size_t)j * kHeadDim;
-            uint32_t* kd = reinterpret_cast<uint32_t*>(p.k_cache + off);
-            uint32_t* vd = reinterpret_cast<uint32_t*>(p.v_cache + off);
-            kd[lane] = st.k_lo;
-            kd[32 + lane] = st.k_hi;
-            vd[lane] = st.v_lo;
-            vd[32 + lane] = st.v_hi;
-        }
+        st.v_lo = xv[lane];
+        st.v_hi = xv[32 + lane];
     }
 
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        st.acc0[k] = 0.f;
-        st.acc1[k] = 0.f;
+    for (int k = 0; k < 8; ++k) {
+        st.acc0[k] = 0ull;  // +0.0f, +0.0f
+        st.acc1[k] = 0ull;
     }
     st.m0 = -INFINITY;
     st.m1 = -INFINITY;
     st.lsum = 0.f;
 }
-
-// Scores, online softmax and value accumulation over one staged page.
+// Scores, online softmax and value accumulation over one staged page. With
+// kFull every one of the 16 rows is a token of the sequence; otherwise the
+// rows >= ntok are skipped.
+template <bool kFull>
 __device__ __forceinline__ void attend_page(const uint8_t* kst, const uint8_t* vst, int ntok, int j, int grp,
                                             int c, int lane, HeadState& st) {
     const uint8_t* kb = kst + j * (kHeadDim * 2) + c * 16;
@@ -419,11 +496,10 @@ __device__ __forceinline__ void attend_page(const uint8_t* kst, const uint8_t* v
     for (int ii = 0; ii < 4; ++ii) {
         const int t = 4 * ii + grp;
         float d0 = 0.f, d1 = 0.f;
-        if (t < ntok) {
+        if (kFull || t < ntok) {
             const uint4 lo = *reinterpret_cast<const uint4*>(kb + t * kRowBytes);
             const uint4 hi = *reinterpret_cast<const uint4*>(kb + t * kRowBytes + 128);
-            d0 = dot16(st.q0, lo, hi);
-            d1 = dot16(st.q1, lo, hi);
+            dot_row(st.q0, st.q1, lo, hi, d0, d1);
         }
         sc[2 * ii] = d0;
         sc[2 * ii + 1] = d1;
@@ -456,8 +532,8 @@ __device__ __forceinline__ void attend_page(const uint8_t* kst, const uint8_t* v
         const float keep = up ? r2[1] : r2[0];
         score = keep + __shfl_xor_sync(kFull, send, 1);
     }
-    const bool valid = (4 * (c >> 1) + grp) < ntok;
-    score = valid ? score : -INFINITY;
+    const bool valid = kFull || (4 * (c >> 1) + grp) < ntok;
+    if (!kFull) score = valid ? score : -INFINITY;
 
     // Page max per head within the group, then the lazy rescale.
     float mx = fmaxf(score, __shfl_xor_sync(kFull, score, 2));
@@ -472,10 +548,11 @@ __device__ __forceinline__ void attend_page(const uint8_t* kst, const uint8_t* v
         const float n1 = grow1 ? mp1 : st.m1;
         const float a0 = grow0 ? exp2_approx(st.m0 - n0) : 1.f;   // exp2(-inf) = 0 on the first page
         const float a1 = grow1 ? exp2_approx(st.m1 - n1) : 1.f;
+        const f32x2 aa0 = pack2(a0, a0), aa1 = pack2(a1, a1);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            st.acc0[k] *= a0;
-            st.acc1[k] *= a1;
+        for (int k = 0; k < 8; ++k) {
+            st.acc0[k] = mul2(st.acc0[k], aa0);
+            st.acc1[k] = mul2(st.acc1[k], aa1);
         }
         st.lsum *= (c & 1) ? a1 : a0;
         st.m0 = n0;
@@ -491,11 +568,10 @@ __device__ __forceinline__ void attend_page(const uint8_t* kst, const uint8_t* v
 #pragma unroll
     for (int ii = 0; ii < 4; ++ii) {
         const int t = 4 * ii + grp;
-        if (t < ntok) {
+        if (kFull || t < ntok) {
             const uint4 lo = *reinterpret_cast<const uint4*>(vb + t * kRowBytes);
             const uint4 hi = *reinterpret_cast<const uint4*>(vb + t * kRowBytes + 128);
-            axpy16(st.acc0, pv[2 * ii], lo, hi);
-            axpy16(st.acc1, pv[2 * ii + 1], lo, hi);
+            axpy_row(st.acc0, st.acc1, pv[2 * ii], pv[2 * ii + 1], lo, hi);
         }
     }
 }
@@ -512,7 +588,7 @@ __device__ __forceinline__ void store_bf16x8(uint16_t* dst, const float* v, floa
 // Merge the 4 token groups; write o directly when this CTA holds the whole
 // sequence, else write a partial and let the last CTA of the sequence combine.
 __device__ __forceinline__ void end_sequence(const Params& p, const Shared& s, int b, int j, int lane, int grp, int c,
-                             int per_cta, HeadState& st) {
+                                             int per_cta, HeadState& st) {
     const int hb = grp & 1;    // this lane writes head 2j + hb ...
     const int hf = grp >> 1;   // ... dims [64*hf + 8c, 64*hf + 8c + 8)
     float M0 = st.m0, M1 = st.m1;
@@ -533,11 +609,20 @@ __device__ __forceinline__ void end_sequence(const Params& p, const Shared& s, i
     const float l0 = (c & 1) ? l_other : l;
     const float l1 = (c & 1) ? l : l_other;
 
+    float acc0[16], acc1[16];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const float2 x0 = unpack2(st.acc0[k]), x1 = unpack2(st.acc1[k]);
+        acc0[2 * k] = x0.x;
+        acc0[2 * k + 1] = x0.y;
+        acc1[2 * k] = x1.x;
+        acc1[2 * k + 1] = x1.y;
+    }
     float r[16], out[8];
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
-        const float send = hb ? st.acc0[k] * f0 : st.acc1[k] * f1;
-        const float keep = hb ? st.acc1[k] * f1 : st.acc0[k] * f0;
+        const float send = hb ? acc0[k] * f0 : acc1[k] * f1;
+        const float keep = hb ? acc1[k] * f1 : acc0[k] * f0;
         r[k] = keep + __shfl_xor_sync(kFull, send, 8);
     }
 #pragma unroll
@@ -573,37 +658,78 @@ __device__ __forceinline__ void end_sequence(const Params& p, const Shared& s, i
     if (prev != nparts - 1) return;
 
     // Last arrival: combine every piece of this sequence for heads 2j, 2j+1.
+    // Pass 1: lanes read the pieces' (max, sum) in parallel; M = overall max.
     __threadfence();
-    float M = -INFINITY, Ls = 0.f, A[8];
+    const float4* ml_base = reinterpret_cast<const float4*>(p.part_ml + (size_t)kGroup * j);  // heads 2j, 2j+1
+    float Mx0 = -INFINITY, Mx1 = -INFINITY;
+    for (int t = lane; t < nparts; t += 32) {
+        const float4 ml = __ldcg(ml_base + (size_t)(part_first + t + b) * (kNumQHeads / 2));
+        Mx0 = fmaxf(Mx0, ml.x);
+        Mx1 = fmaxf(Mx1, ml.z);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        Mx0 = fmaxf(Mx0, __shfl_xor_sync(kFull, Mx0, off));
+        Mx1 = fmaxf(Mx1, __shfl_xor_sync(kFull, Mx1, off));
+    }
+    // Pass 2: weights 2^(m_t - M) per piece (lane t), then every lane sums its
+    // 8 output dims over the pieces with many loads in flight.
+    float Ls0 = 0.f, Ls1 = 0.f, A[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) A[k] = 0.f;
-    for (int t = 0; t < nparts; ++t) {
-        const int sid = part_first + t + b;
-        const float2 ml = __ldcg(p.part_ml + (size_t)sid * kNumQHeads + head);
-        const float4* src =
-            reinterpret_cast<const float4*>(p.part_acc + ((size_t)sid * kNumQHeads + head) * kHeadDim + dim0);
-        const float4 x0 = __ldcg(src), x1 = __ldcg(src + 1);
-        if (ml.x == -INFINITY) continue;  // a piece whose pages were all skipped
-        const float Mn = fmaxf(M, ml.x);
-        const float sa = exp2_approx(M - Mn);
-        const float sb = exp2_approx(ml.x - Mn);
-        Ls = Ls * sa + ml.y * sb;
-        A[0] = A[0] * sa + x0.x * sb;
-        A[1] = A[1] * sa + x0.y * sb;
-        A[2] = A[2] * sa + x0.z * sb;
-        A[3] = A[3] * sa + x0.w * sb;
-        A[4] = A[4] * sa + x1.x * sb;
-        A[5] = A[5] * sa + x1.y * sb;
-        A[6] = A[6] * sa + x1.z * sb;
-        A[7] = A[7] * sa + x1.w * sb;
-        M = Mn;
+    constexpr int kMergeBatch = 4;  // pieces whose loads are in flight together
+    const float* acc_base = p.part_acc + (size_t)head * kHeadDim + dim0;
+    for (int t0 = 0; t0 < nparts; t0 += 32) {
+        float w0 = 0.f, w1 = 0.f;
+        if (t0 + lane < nparts) {
+            const float4 ml = __ldcg(ml_base + (size_t)(part_first + t0 + lane + b) * (kNumQHeads / 2));
+            w0 = (ml.x == -INFINITY) ? 0.f : exp2_approx(ml.x - Mx0);   // a piece whose pages were all skipped
+            w1 = (ml.z == -INFINITY) ? 0.f : exp2_approx(ml.z - Mx1);
+            Ls0 += w0 * ml.y;
+            Ls1 += w1 * ml.w;
+        }
+        const int n = min(32, nparts - t0);
+        for (int u0 = 0; u0 < n; u0 += kMergeBatch) {
+            float4 x0[kMergeBatch], x1[kMergeBatch];
+#pragma unroll
+            for (int u = 0; u < kMergeBatch; ++u) {
+                if (u0 + u < n) {
+                    const float4* src = reinterpret_cast<const float4*>(
+                        acc_base + (size_t)(part_first + t0 + u0 + u + b) * (kNumQHeads * kHeadDim));
+                    x0[u] = __ldcg(src);
+                    x1[u] = __ldcg(src + 1);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kMergeBatch; ++u) {
+                const float wa = __shfl_sync(kFull, w0, (u0 + u) & 31);
+                const float wb = __shfl_sync(kFull, w1, (u0 + u) & 31);
+                if (u0 + u < n) {
+                    const float w = hb ? wb : wa;
+                    A[0] = fmaf(w, x0[u].x, A[0]);
+                    A[1] = fmaf(w, x0[u].y, A[1]);
+                    A[2] = fmaf(w, x0[u].z, A[2]);
+                    A[3] = fmaf(w, x0[u].w, A[3]);
+                    A[4] = fmaf(w, x1[u].x, A[4]);
+                    A[5] = fmaf(w, x1[u].y, A[5]);
+                    A[6] = fmaf(w, x1[u].z, A[6]);
+                    A[7] = fmaf(w, x1[u].w, A[7]);
+                }
+            }
+        }
     }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        Ls0 += __shfl_xor_sync(kFull, Ls0, off);
+        Ls1 += __shfl_xor_sync(kFull, Ls1, off);
+    }
+    const float Ls = hb ? Ls1 : Ls0;
     store_bf16x8(o, A, Ls > 0.f ? 1.f / Ls : 0.f);
     if (lane == 0) p.counters[b * kNumKvHeads + j] = 0;  // ready for the next call
 }
 
-__device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, int B, int start, int end, int per_cta, int warp,
-                             int lane) {
+__device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, int B, int start, int end, int per_cta,
+                                             int warp, int lane) {
     const int j = warp;
     const int grp = lane >> 3;
     const int c = lane & 7;
@@ -619,26 +745,38 @@ __device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, i
         const int nb = s.seg[b + 1] - s.seg[b];
         const int L = s.lens[b];
         const bool last = (i == nb - 1);
-        if (k == 0 || i == 0) begin_sequence(p, s, b, j, lane, c, /*appends=*/s.seg[b + 1] <= end, st);
         const int new_row = (L - 1) - kPage * i;   // row of the new token on the last page
         const int ntok = last ? new_row + 1 : kPage;
 
-        bool ok = mbar_wait(&s.full_bar[slot], phase, p.timeout_ns, s.abort_flag);
-        ok = __all_sync(kFull, ok || mbar_try_wait(&s.full_bar[slot], phase));
-        if (!ok) {
-            if (lane == 0) {
-                *s.abort_flag = 1;
-                record_error(p.status, QDA_ERR_TIMEOUT);
+        bool ok = mbar_try_wait(&s.full_bar[slot], phase);
+        if (!__all_sync(kFull, ok)) {
+            ok = ok || mbar_wait(&s.full_bar[slot], phase, p.timeout_ns, s.abort_flag);
+            ok = __all_sync(kFull, ok || mbar_try_wait(&s.full_bar[slot], phase));
+            if (!ok) {
+                if (lane == 0) {
+                    *s.abort_flag = 1;
+                    record_error(p.status, QDA_ERR_TIMEOUT);
+                }
+                return;
             }
-            return;
         }
-        uint8_t* kst = s.stages + slot * kStageBytes;
-        uint8_t* vst = kst + kPageBytes;
-        if (s.slot_bad[slot] == 0) {
+        uint8_t* stage = s.stages + slot * kStageBytes;
+        if (k == 0 || i == 0)
+            begin_sequence(p, s, stage + kStageQkv, s.meta[slot].pos, j, lane, c, /*appends=*/s.seg[b + 1] <= end, st);
+        if (s.meta[slot].bad == 0) {
             if (last) {
-                // the new token: this warp's head slice of the row the copy left out
-                uint32_t* kr = reinterpret_cast<uint32_t*>(kst + new_row * kRowBytes + j * kHeadDim * 2);
-                uint32_t* vr = reinterpret_cast<uint32_t*>(vst + new_row * kRowBytes + j * kHeadDim * 2);
+                // the new token: written to the cache, and patched into the
+                // staged page (this warp's head slice of the row the copy left out)
+                const int page = s.meta[slot].page;
+                const size_t off = (size_t)page * (kPageBytes / 2) + (size_t)new_row * (kRowBytes / 2) + (size_t)j * kHeadDim;
+                uint32_t* kd = reinterpret_cast<uint32_t*>(p.k_cache + off);
+                uint32_t* vd = reinterpret_cast<uint32_t*>(p.v_cache + off);
+                kd[lane] = st.k_lo;
+                kd[32 + lane] = st.k_hi;
+                vd[lane] = st.v_lo;
+                vd[32 + lane] = st.v_hi;
+                uint32_t* kr = reinterpret_cast<uint32_t*>(stage + kStageK + new_row * kRowBytes + j * kHeadDim * 2);
+                uint32_t* vr = reinterpret_cast<uint32_t*>(stage + kStageV + new_row * kRowBytes + j * kHeadDim * 2);
                 kr[lane] = st.k_lo;
                 kr[32 + lane] = st.k_hi;
                 vr[lane] = st.v_lo;
@@ -647,7 +785,8 @@ __device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, i
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
             }
-            attend_page(kst, vst, ntok, j, grp, c, lane, st);
+            if (ntok == kPage) attend_page<true>(stage + kStageK, stage + kStageV, ntok, j, grp, c, lane, st);
+            else attend_page<false>(stage + kStageK, stage + kStageV, ntok, j, grp, c, lane, st);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.empty_bar[slot]);
@@ -669,15 +808,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_kernel(const Par
     const int lane = threadIdx.x & 31;
     Shared s;
     s.stages = smem;
-    s.q = reinterpret_cast<float*>(smem + kSmemQ);
     s.seg = reinterpret_cast<int*>(smem + kSmemSeg);
     s.lens = reinterpret_cast<int*>(smem + kSmemLens);
     s.inv_freq = reinterpret_cast<double*>(smem + kSmemInvFreq);
+    s.gains = reinterpret_cast<const uint16_t*>(smem + kSmemGains);
+    s.meta = reinterpret_cast<volatile StageMeta*>(smem + kSmemMeta);
     s.full_bar = reinterpret_cast<uint64_t*>(smem + kSmemBars);
     s.empty_bar = s.full_bar + kStages;
     s.never_bar = s.empty_bar + kStages;
-    s.slot_bad = reinterpret_cast<volatile int*>(smem + kSmemFlags);
-    s.abort_flag = s.slot_bad + kStages;
+    s.abort_flag = reinterpret_cast<volatile int*>(smem + kSmemFlags);
 
     // Pages per sequence (0 for a sequence whose length is out of range).
     const int B = p.batch;
@@ -688,12 +827,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_kernel(const Par
         s.lens[b] = L;
         s.seg[b + 1] = ok ? (L + kPage - 1) / kPage : 0;
     }
-    if (threadIdx.x < 64) s.inv_freq[threadIdx.x] = pow(p.rope_theta, -2.0 * threadIdx.x / 128.0);
+    if (threadIdx.x < 64) {
+        // both gain vectors, one 8-byte word per thread
+        const uint16_t* src = threadIdx.x < 32 ? p.q_norm_w : p.k_norm_w;
+        reinterpret_cast<uint2*>(smem + kSmemGains)[threadIdx.x] =
+            *reinterpret_cast<const uint2*>(src + 4 * (threadIdx.x & 31));
+    } else if (threadIdx.x < 128) {
+        const int i = threadIdx.x - 64;
+        s.inv_freq[i] = pow(p.rope_theta, -2.0 * i / 128.0);
+    }
     if (threadIdx.x == 0) {
         for (int k = 0; k < kStages; ++k) {
             mbar_init(&s.full_bar[k], 1);
             mbar_init(&s.empty_bar[k], kConsumerWarps);
-            s.slot_bad[k] = 0;
         }
         mbar_init(s.never_bar, 1);
         *s.abort_flag = 0;
