@@ -380,24 +380,27 @@ struct HeadState {
     uint32_t k_lo, k_hi, v_lo, v_hi;  // this lane's words of the appended k/v row
 };
 
-__device__ __forceinline__ double warp_sum8(double v) {   // over the 8 lanes of a token group
-    v += __shfl_xor_sync(kFull, v, 1);
-    v += __shfl_xor_sync(kFull, v, 2);
-    v += __shfl_xor_sync(kFull, v, 4);
-    return v;
-}
-
-// Start sequence b: norm and rotate q from the staged qkv row, in double, and,
-// when this CTA holds the sequence's last page, the new k. Lane l computes the
-// rotation angles of pairs 2l and 2l+1; lane (grp, c) then gathers those of
-// pairs 8c..8c+7, whose two halves are exactly its q dims.
+// Start sequence b from its staged qkv row. q is normed and rotated in float:
+// each rotation angle pos * theta^(-2i/128) is formed and reduced modulo 2*pi
+// in double (Cody-Waite, two-part 2*pi) before its float sine and cosine, so
+// q keeps float accuracy at any position. When this CTA holds the sequence's
+// last page, the new k is normed and rotated entirely in double and rounded
+// once to bf16. Lane l computes the angles of pairs 2l and 2l+1; lane (grp, c)
+// gathers those of pairs 8c..8c+7, whose two halves are exactly its q dims.
 __device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s, const uint8_t* qkv_row, int pos,
                                                int j, int lane, int c, bool appends, HeadState& st) {
-    double cs0, sn0, cs1, sn1;
+    constexpr double kTwoPiHi = 6.2831853069365025;      // 2*pi rounded to 32 significant bits
+    constexpr double kTwoPiLo = 2.430840202602477e-10;   // 2*pi - kTwoPiHi
+    constexpr double kInvTwoPi = 0.15915494309189535;
+    const double ang0 = (double)pos * s.inv_freq[2 * lane];
+    const double ang1 = (double)pos * s.inv_freq[2 * lane + 1];
+    float cf0, sf0, cf1, sf1;
     {
-        const double fpos = (double)pos;
-        sincos(fpos * s.inv_freq[2 * lane], &sn0, &cs0);
-        sincos(fpos * s.inv_freq[2 * lane + 1], &sn1, &cs1);
+        const double n0 = rint(ang0 * kInvTwoPi), n1 = rint(ang1 * kInvTwoPi);
+        const double r0 = fma(-n0, kTwoPiLo, fma(-n0, kTwoPiHi, ang0));
+        const double r1 = fma(-n1, kTwoPiLo, fma(-n1, kTwoPiHi, ang1));
+        sincosf((float)r0, &sf0, &cf0);
+        sincosf((float)r1, &sf1, &cf1);
     }
     // this lane's 16 dims of heads 2j, 2j+1: words 0..3 dims 8c..8c+7, 4..7 dims 64+8c..
     uint32_t x0[8], x1[8];
@@ -410,39 +413,43 @@ __device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s,
         x0[0] = a0.x; x0[1] = a0.y; x0[2] = a0.z; x0[3] = a0.w; x0[4] = b0.x; x0[5] = b0.y; x0[6] = b0.z; x0[7] = b0.w;
         x1[0] = a1.x; x1[1] = a1.y; x1[2] = a1.z; x1[3] = a1.w; x1[4] = b1.x; x1[5] = b1.y; x1[6] = b1.z; x1[7] = b1.w;
     }
-    double ss0 = 0.0, ss1 = 0.0;
+    float ss0 = 0.f, ss1 = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
-        const double e0 = bf_to_d(x0[w] & 0xFFFFu), o0 = bf_to_d(x0[w] >> 16);
-        const double e1 = bf_to_d(x1[w] & 0xFFFFu), o1 = bf_to_d(x1[w] >> 16);
-        ss0 = fma(e0, e0, fma(o0, o0, ss0));
-        ss1 = fma(e1, e1, fma(o1, o1, ss1));
+        ss0 = fmaf(bf_lo(x0[w]), bf_lo(x0[w]), fmaf(bf_hi(x0[w]), bf_hi(x0[w]), ss0));
+        ss1 = fmaf(bf_lo(x1[w]), bf_lo(x1[w]), fmaf(bf_hi(x1[w]), bf_hi(x1[w]), ss1));
     }
-    const double inv_r0 = 1.0 / sqrt(warp_sum8(ss0) / 128.0 + p.rms_eps);
-    const double inv_r1 = 1.0 / sqrt(warp_sum8(ss1) / 128.0 + p.rms_eps);
+#pragma unroll
+    for (int off = 1; off < 8; off <<= 1) {   // over the 8 lanes of the token group
+        ss0 += __shfl_xor_sync(kFull, ss0, off);
+        ss1 += __shfl_xor_sync(kFull, ss1, off);
+    }
+    const float eps = (float)p.rms_eps;
+    const float inv_r0 = rsqrtf(ss0 * (1.f / 128.f) + eps);
+    const float inv_r1 = rsqrtf(ss1 * (1.f / 128.f) + eps);
     const uint4 wa = *reinterpret_cast<const uint4*>(s.gains + 8 * c);        // q gains, dims 8c..
     const uint4 wb = *reinterpret_cast<const uint4*>(s.gains + 64 + 8 * c);   // dims 64+8c..
     const uint32_t wq[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+    const float scale = (float)kQScale;
     // pair 8c + k: dims 8c+k (word k/2 of the low half) and 64+8c+k (word 4 + k/2)
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
         float q0a[2], q0b[2], q1a[2], q1b[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            const int k = 2 * m + e;
-            const int src = 4 * c + (k >> 1);
-            const double cs = __shfl_sync(kFull, e ? cs1 : cs0, src);
-            const double sn = __shfl_sync(kFull, e ? sn1 : sn0, src);
-            const int sh = e ? 16 : 0;
-            const double wlo = bf_to_d((wq[m] >> sh) & 0xFFFFu), whi = bf_to_d((wq[4 + m] >> sh) & 0xFFFFu);
-            const double ya0 = bf_to_d((x0[m] >> sh) & 0xFFFFu) * inv_r0 * wlo;
-            const double yb0 = bf_to_d((x0[4 + m] >> sh) & 0xFFFFu) * inv_r0 * whi;
-            const double ya1 = bf_to_d((x1[m] >> sh) & 0xFFFFu) * inv_r1 * wlo;
-            const double yb1 = bf_to_d((x1[4 + m] >> sh) & 0xFFFFu) * inv_r1 * whi;
-            q0a[e] = (float)((ya0 * cs - yb0 * sn) * kQScale);
-            q0b[e] = (float)((yb0 * cs + ya0 * sn) * kQScale);
-            q1a[e] = (float)((ya1 * cs - yb1 * sn) * kQScale);
-            q1b[e] = (float)((yb1 * cs + ya1 * sn) * kQScale);
+            const int src = 4 * c + m;   // lane holding pairs 8c + 2m and 8c + 2m + 1
+            const float cs = __shfl_sync(kFull, e ? cf1 : cf0, src);
+            const float sn = __shfl_sync(kFull, e ? sf1 : sf0, src);
+            const float wlo = e ? bf_hi(wq[m]) : bf_lo(wq[m]);
+            const float whi = e ? bf_hi(wq[4 + m]) : bf_lo(wq[4 + m]);
+            const float ya0 = (e ? bf_hi(x0[m]) : bf_lo(x0[m])) * inv_r0 * wlo;
+            const float yb0 = (e ? bf_hi(x0[4 + m]) : bf_lo(x0[4 + m])) * inv_r0 * whi;
+            const float ya1 = (e ? bf_hi(x1[m]) : bf_lo(x1[m])) * inv_r1 * wlo;
+            const float yb1 = (e ? bf_hi(x1[4 + m]) : bf_lo(x1[4 + m])) * inv_r1 * whi;
+            q0a[e] = fmaf(ya0, cs, -yb0 * sn) * scale;
+            q0b[e] = fmaf(yb0, cs, ya0 * sn) * scale;
+            q1a[e] = fmaf(ya1, cs, -yb1 * sn) * scale;
+            q1b[e] = fmaf(yb1, cs, ya1 * sn) * scale;
         }
         st.q0[m] = pack2(q0a[0], q0a[1]);
         st.q0[4 + m] = pack2(q0b[0], q0b[1]);
@@ -451,7 +458,10 @@ __device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s,
     }
 
     if (appends) {
-        // lane l: dims 2l, 2l+1 (word l of the head) and 64+2l, 65+2l (word 32+l)
+        // lane l: dims 2l, 2l+1 (word l of the head) and 64+2l, 65+2l (word 32+l), all in double
+        double cs0, sn0, cs1, sn1;
+        sincos(ang0, &sn0, &cs0);
+        sincos(ang1, &sn1, &cs1);
         const uint32_t* xk = reinterpret_cast<const uint32_t*>(qkv_row + (kNumQHeads + j) * (kHeadDim * 2));
         const uint32_t* xv = reinterpret_cast<const uint32_t*>(qkv_row + (kNumQHeads + kNumKvHeads + j) * (kHeadDim * 2));
         const uint32_t* gk = reinterpret_cast<const uint32_t*>(s.gains + kHeadDim);
@@ -481,6 +491,7 @@ __device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s,
     st.m1 = -INFINITY;
     st.lsum = 0.f;
 }
+
 // Scores, online softmax and value accumulation over one staged page. With
 // kFull every one of the 16 rows is a token of the sequence; otherwise the
 // rows >= ntok are skipped.
@@ -585,9 +596,11 @@ __device__ __forceinline__ void store_bf16x8(uint16_t* dst, const float* v, floa
     *reinterpret_cast<uint4*>(dst) = w;
 }
 
-// Merge the 4 token groups; write o directly when this CTA holds the whole
-// sequence, else write a partial and let the last CTA of the sequence combine.
-__device__ __forceinline__ void end_sequence(const Params& p, const Shared& s, int b, int j, int lane, int grp, int c,
+// End of a sequence piece: merge the 4 token groups, then write o directly
+// when this CTA holds the whole sequence, else write this piece's partial
+// (un-normalised output and its running max and sum) to scratch slot
+// blockIdx.x + b. Returns whether a partial was written.
+__device__ __forceinline__ bool finish_piece(const Params& p, const Shared& s, int b, int j, int grp, int c,
                                              int per_cta, HeadState& st) {
     const int hb = grp & 1;    // this lane writes head 2j + hb ...
     const int hf = grp >> 1;   // ... dims [64*hf + 8c, 64*hf + 8c + 8)
@@ -635,30 +648,39 @@ __device__ __forceinline__ void end_sequence(const Params& p, const Shared& s, i
     const float Lh = hb ? l1 : l0;
     const int head = kGroup * j + hb;
     const int dim0 = 64 * hf + 8 * c;
-    uint16_t* o = p.o + ((size_t)b * kNumQHeads + head) * kHeadDim + dim0;
 
     const int part_first = s.seg[b] / per_cta;
     const int part_last = (s.seg[b + 1] - 1) / per_cta;
-    const int nparts = part_last - part_first + 1;
-    if (nparts == 1) {
-        store_bf16x8(o, out, Lh > 0.f ? 1.f / Lh : 0.f);
-        return;
+    if (part_first == part_last) {
+        store_bf16x8(p.o + ((size_t)b * kNumQHeads + head) * kHeadDim + dim0, out, Lh > 0.f ? 1.f / Lh : 0.f);
+        return false;
     }
-
     const int slot = blockIdx.x + b;
     float4* pa = reinterpret_cast<float4*>(p.part_acc + ((size_t)slot * kNumQHeads + head) * kHeadDim + dim0);
     __stcg(pa, make_float4(out[0], out[1], out[2], out[3]));
     __stcg(pa + 1, make_float4(out[4], out[5], out[6], out[7]));
     if (c == 0 && hf == 0) __stcg(p.part_ml + (size_t)slot * kNumQHeads + head, make_float2(Mh, Lh));
-    __threadfence();
-    __syncwarp();
+    return true;
+}
+
+// Count this CTA's piece of sequence b as done; the last piece to arrive
+// combines every piece's partial for heads 2j, 2j+1 and writes o. The caller
+// has made its partial stores visible (__threadfence) before calling.
+__device__ __forceinline__ void arrive_and_merge(const Params& p, const Shared& s, int b, int j, int lane, int grp,
+                                                 int c, int per_cta) {
+    const int hb = grp & 1;
+    const int hf = grp >> 1;
+    const int head = kGroup * j + hb;
+    const int dim0 = 64 * hf + 8 * c;
+    const int part_first = s.seg[b] / per_cta;
+    const int part_last = (s.seg[b + 1] - 1) / per_cta;
+    const int nparts = part_last - part_first + 1;
     int prev = 0;
     if (lane == 0) prev = atomicAdd(p.counters + b * kNumKvHeads + j, 1);
     prev = __shfl_sync(kFull, prev, 0);
     if (prev != nparts - 1) return;
 
-    // Last arrival: combine every piece of this sequence for heads 2j, 2j+1.
-    // Pass 1: lanes read the pieces' (max, sum) in parallel; M = overall max.
+    // Last arrival. Pass 1: lanes read the pieces' (max, sum) in parallel; M = overall max.
     __threadfence();
     const float4* ml_base = reinterpret_cast<const float4*>(p.part_ml + (size_t)kGroup * j);  // heads 2j, 2j+1
     float Mx0 = -INFINITY, Mx1 = -INFINITY;
@@ -674,10 +696,10 @@ __device__ __forceinline__ void end_sequence(const Params& p, const Shared& s, i
     }
     // Pass 2: weights 2^(m_t - M) per piece (lane t), then every lane sums its
     // 8 output dims over the pieces with many loads in flight.
+    constexpr int kMergeBatch = 8;
     float Ls0 = 0.f, Ls1 = 0.f, A[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) A[k] = 0.f;
-    constexpr int kMergeBatch = 4;  // pieces whose loads are in flight together
     const float* acc_base = p.part_acc + (size_t)head * kHeadDim + dim0;
     for (int t0 = 0; t0 < nparts; t0 += 32) {
         float w0 = 0.f, w1 = 0.f;
@@ -724,10 +746,66 @@ __device__ __forceinline__ void end_sequence(const Params& p, const Shared& s, i
         Ls1 += __shfl_xor_sync(kFull, Ls1, off);
     }
     const float Ls = hb ? Ls1 : Ls0;
-    store_bf16x8(o, A, Ls > 0.f ? 1.f / Ls : 0.f);
+    store_bf16x8(p.o + ((size_t)b * kNumQHeads + head) * kHeadDim + dim0, A, Ls > 0.f ? 1.f / Ls : 0.f);
     if (lane == 0) p.counters[b * kNumKvHeads + j] = 0;  // ready for the next call
 }
 
+// Wait for the page in `slot`; returns false when the wait ran out (the
+// kernel is then aborting).
+__device__ __forceinline__ bool wait_full(const Params& p, const Shared& s, int slot, uint32_t phase, int lane) {
+    bool ok = mbar_try_wait(&s.full_bar[slot], phase);
+    if (__all_sync(kFull, ok)) return true;
+    ok = ok || mbar_wait(&s.full_bar[slot], phase, p.timeout_ns, s.abort_flag);
+    ok = __all_sync(kFull, ok || mbar_try_wait(&s.full_bar[slot], phase));
+    if (!ok && lane == 0) {
+        *s.abort_flag = 1;
+        record_error(p.status, QDA_ERR_TIMEOUT);
+    }
+    return ok;
+}
+
+// Attend over the staged page in `slot` (page i of a sequence of nb pages and
+// length L), appending the new token first when it is the last page, then
+// release the slot.
+__device__ __forceinline__ void consume_page(const Params& p, const Shared& s, int slot, int i, int nb, int L, int j,
+                                             int grp, int c, int lane, HeadState& st) {
+    uint8_t* stage = s.stages + slot * kStageBytes;
+    const bool last = (i == nb - 1);
+    const int new_row = (L - 1) - kPage * i;   // row of the new token on the last page
+    const int ntok = last ? new_row + 1 : kPage;
+    if (s.meta[slot].bad == 0) {
+        if (last) {
+            // the new token: written to the cache, and patched into the staged
+            // page (this warp's head slice of the row the copy left out)
+            const int page = s.meta[slot].page;
+            const size_t off =
+                (size_t)page * (kPageBytes / 2) + (size_t)new_row * (kRowBytes / 2) + (size_t)j * kHeadDim;
+            uint32_t* kd = reinterpret_cast<uint32_t*>(p.k_cache + off);
+            uint32_t* vd = reinterpret_cast<uint32_t*>(p.v_cache + off);
+            kd[lane] = st.k_lo;
+            kd[32 + lane] = st.k_hi;
+            vd[lane] = st.v_lo;
+            vd[32 + lane] = st.v_hi;
+            uint32_t* kr = reinterpret_cast<uint32_t*>(stage + kStageK + new_row * kRowBytes + j * kHeadDim * 2);
+            uint32_t* vr = reinterpret_cast<uint32_t*>(stage + kStageV + new_row * kRowBytes + j * kHeadDim * 2);
+            kr[lane] = st.k_lo;
+            kr[32 + lane] = st.k_hi;
+            vr[lane] = st.v_lo;
+            vr[32 + lane] = st.v_hi;
+            // order these generic writes before the next bulk copy into the slot
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+        }
+        if (ntok == kPage) attend_page<true>(stage + kStageK, stage + kStageV, ntok, j, grp, c, lane, st);
+        else attend_page<false>(stage + kStageK, stage + kStageV, ntok, j, grp, c, lane, st);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.empty_bar[slot]);
+}
+
+// Consumer warp j: walk the CTA's pages piece by piece (a piece = the pages of
+// one sequence inside the CTA's range). Only the first and the last piece can
+// be split with other CTAs; their arrivals (and any merge) wait for the end.
 __device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, int B, int start, int end, int per_cta,
                                              int warp, int lane) {
     const int j = warp;
@@ -737,68 +815,41 @@ __device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, i
     st.k_lo = st.k_hi = st.v_lo = st.v_hi = 0u;
 
     int b = find_seq(s.seg, B, start);
-    int i = start - s.seg[b];
+    int i0 = start - s.seg[b];       // first page of the piece within its sequence
     int slot = 0;
     uint32_t phase = 0;
+    int pending0 = -1, pending1 = -1;  // split pieces whose arrival waits for the end
     const int count = end - start;
-    for (int k = 0; k < count; ++k) {
+    int k = 0;
+    while (k < count) {
         const int nb = s.seg[b + 1] - s.seg[b];
         const int L = s.lens[b];
-        const bool last = (i == nb - 1);
-        const int new_row = (L - 1) - kPage * i;   // row of the new token on the last page
-        const int ntok = last ? new_row + 1 : kPage;
-
-        bool ok = mbar_try_wait(&s.full_bar[slot], phase);
-        if (!__all_sync(kFull, ok)) {
-            ok = ok || mbar_wait(&s.full_bar[slot], phase, p.timeout_ns, s.abort_flag);
-            ok = __all_sync(kFull, ok || mbar_try_wait(&s.full_bar[slot], phase));
-            if (!ok) {
-                if (lane == 0) {
-                    *s.abort_flag = 1;
-                    record_error(p.status, QDA_ERR_TIMEOUT);
-                }
-                return;
-            }
+        const int n_here = min(nb - i0, count - k);
+        // first page of the piece: it carries the sequence's qkv row
+        if (!wait_full(p, s, slot, phase, lane)) return;
+        begin_sequence(p, s, s.stages + slot * kStageBytes + kStageQkv, s.meta[slot].pos, j, lane, c,
+                       /*appends=*/s.seg[b + 1] <= end, st);
+        consume_page(p, s, slot, i0, nb, L, j, grp, c, lane, st);
+        if (++slot == kStages) { slot = 0; phase ^= 1u; }
+        for (int u = 1; u < n_here; ++u) {
+            if (!wait_full(p, s, slot, phase, lane)) return;
+            consume_page(p, s, slot, i0 + u, nb, L, j, grp, c, lane, st);
+            if (++slot == kStages) { slot = 0; phase ^= 1u; }
         }
-        uint8_t* stage = s.stages + slot * kStageBytes;
-        if (k == 0 || i == 0)
-            begin_sequence(p, s, stage + kStageQkv, s.meta[slot].pos, j, lane, c, /*appends=*/s.seg[b + 1] <= end, st);
-        if (s.meta[slot].bad == 0) {
-            if (last) {
-                // the new token: written to the cache, and patched into the
-                // staged page (this warp's head slice of the row the copy left out)
-                const int page = s.meta[slot].page;
-                const size_t off = (size_t)page * (kPageBytes / 2) + (size_t)new_row * (kRowBytes / 2) + (size_t)j * kHeadDim;
-                uint32_t* kd = reinterpret_cast<uint32_t*>(p.k_cache + off);
-                uint32_t* vd = reinterpret_cast<uint32_t*>(p.v_cache + off);
-                kd[lane] = st.k_lo;
-                kd[32 + lane] = st.k_hi;
-                vd[lane] = st.v_lo;
-                vd[32 + lane] = st.v_hi;
-                uint32_t* kr = reinterpret_cast<uint32_t*>(stage + kStageK + new_row * kRowBytes + j * kHeadDim * 2);
-                uint32_t* vr = reinterpret_cast<uint32_t*>(stage + kStageV + new_row * kRowBytes + j * kHeadDim * 2);
-                kr[lane] = st.k_lo;
-                kr[32 + lane] = st.k_hi;
-                vr[lane] = st.v_lo;
-                vr[32 + lane] = st.v_hi;
-                // order these generic writes before the next bulk copy into the slot
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
-            }
-            if (ntok == kPage) attend_page<true>(stage + kStageK, stage + kStageV, ntok, j, grp, c, lane, st);
-            else attend_page<false>(stage + kStageK, stage + kStageV, ntok, j, grp, c, lane, st);
+        k += n_here;
+        if (finish_piece(p, s, b, j, grp, c, per_cta, st)) {
+            if (pending0 < 0) pending0 = b;
+            else pending1 = b;
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.empty_bar[slot]);
-        if (++slot == kStages) {
-            slot = 0;
-            phase ^= 1u;
-        }
-        if (last || k == count - 1) end_sequence(p, s, b, j, lane, grp, c, per_cta, st);
-        if (++i == nb) {
-            i = 0;
+        if (k < count) {
             do { ++b; } while (b < B && s.seg[b + 1] == s.seg[b]);
+            i0 = 0;
         }
+    }
+    if (pending0 >= 0) {
+        __threadfence();   // this warp's partial stores before its arrivals
+        arrive_and_merge(p, s, pending0, j, lane, grp, c, per_cta);
+        if (pending1 >= 0) arrive_and_merge(p, s, pending1, j, lane, grp, c, per_cta);
     }
 }
 

@@ -39,10 +39,11 @@
  *   v_cache      dim. One page of one cache is 32 KiB, contiguous.
  *   o            bf16 [B][16][128].
  *
- * Numbers: q and k are normed and rotated in double precision; q is kept in
- * float (never rounded to bf16); k is rounded once to bf16 when stored; the
- * scores, the softmax and the value accumulation are float; o is rounded once
- * to bf16 (nearest-even).
+ * Numbers: the new k is normed and rotated in double precision and rounded
+ * once to bf16 (nearest-even) when stored; q is normed and rotated in float,
+ * its rotation angle formed and reduced modulo 2*pi in double, and is never
+ * rounded to bf16; the scores, the softmax and the value accumulation are
+ * float; o is rounded once to bf16 (nearest-even).
  *
  * Ownership: every tensor is caller-owned memory. The handle owns only its
  * workspace (device scratch for split partials, merge counters and the status
