@@ -11,7 +11,8 @@ page size 16) and the conformance method of the "Model conformance" page
 ("How the comparison works", step 1: norm weights perturbed away from their
 identity value):
 
-  qkv                 bf16 [B, 4096] ~ N(0, 1)
+  qkv                 bf16 [B, (Hq + 16) * 128] ~ N(0, 1) (Hq = 16 for Qwen3-0.6B;
+                      32, 40 or 64 for the 4B/8B, 14B and 32B sizes)
   q_norm_w, k_norm_w  bf16 [128] = 1 + U(-0.5, 0.5)
   k_cache, v_cache    bf16 [num_pages, 16, 8, 128] ~ N(0, 1)
   block_table         int32 [B, stride], distinct pages drawn from a random
@@ -44,7 +45,7 @@ class Workload:
     seq_lens: torch.Tensor          # int32 [B], CPU; counts the new token
     block_table: torch.Tensor       # int32 [B, stride], CPU; -1 where unused
     num_pages: int
-    qkv: torch.Tensor               # bf16 [B, 4096] on `device`
+    qkv: torch.Tensor               # bf16 [B, (Hq + 16) * 128] on `device`
     q_norm_w: torch.Tensor          # bf16 [128] on `device`
     k_norm_w: torch.Tensor          # bf16 [128] on `device`
     k_cache: torch.Tensor           # bf16 [num_pages, 16, 8, 128] on `device`
@@ -58,6 +59,10 @@ class Workload:
     @property
     def device(self) -> torch.device:
         return self.qkv.device
+
+    @property
+    def num_q_heads(self) -> int:
+        return int(self.qkv.shape[1]) // HEAD_DIM - 2 * NUM_KV_HEADS
 
 
 def pages_for(seq_lens: torch.Tensor) -> torch.Tensor:
@@ -99,9 +104,14 @@ def assign_pages(seq_lens: torch.Tensor, pool_pages: int, seed: int,
     return bt
 
 
-def _values(B: int, num_pages: int, seed: int, device) -> dict:
+def qkv_width(num_q_heads: int) -> int:
+    """Width of the fused qkv row: Hq query heads, then 8 k and 8 v heads, of 128."""
+    return (num_q_heads + 2 * NUM_KV_HEADS) * HEAD_DIM
+
+
+def _values(B: int, num_pages: int, seed: int, device, num_q_heads: int = NUM_Q_HEADS) -> dict:
     dev = torch.device(device)
-    qkv = torch.randn((B, QKV_WIDTH), generator=_gen(seed * 16 + 1, dev), device=dev,
+    qkv = torch.randn((B, qkv_width(num_q_heads)), generator=_gen(seed * 16 + 1, dev), device=dev,
                       dtype=torch.float32).to(torch.bfloat16)
     gq = torch.rand(HEAD_DIM, generator=_gen(seed * 16 + 2, dev), device=dev, dtype=torch.float32)
     gk = torch.rand(HEAD_DIM, generator=_gen(seed * 16 + 3, dev), device=dev, dtype=torch.float32)
@@ -114,14 +124,14 @@ def _values(B: int, num_pages: int, seed: int, device) -> dict:
 
 def custom(seq_lens, seed: int = 0, device="cpu", pool_pages: int | None = None,
            stride: int | None = None, gap_fraction: float = 0.0, positions=None,
-           name: str = "custom") -> Workload:
+           name: str = "custom", num_q_heads: int = NUM_Q_HEADS) -> Workload:
     """A workload with the given sequence lengths and the standard value recipe."""
     seq_lens = torch.as_tensor(seq_lens, dtype=torch.int32).reshape(-1)
     need = int(pages_for(seq_lens).sum())
     if pool_pages is None:
         pool_pages = need + (int(math.ceil(gap_fraction * need)) if gap_fraction > 0 else 0)
     bt = assign_pages(seq_lens, pool_pages, seed, stride=stride, gap_fraction=gap_fraction)
-    vals = _values(seq_lens.numel(), pool_pages, seed, device)
+    vals = _values(seq_lens.numel(), pool_pages, seed, device, num_q_heads)
     pos = None if positions is None else torch.as_tensor(positions, dtype=torch.int32).reshape(-1)
     return Workload(name=name, seq_lens=seq_lens, block_table=bt, num_pages=pool_pages,
                     positions=pos, **vals)
@@ -142,12 +152,12 @@ def config1(device="cpu") -> Workload:
                     block_table=bt, num_pages=4, **vals)
 
 
-def config2(device="cpu", seed: int = 2000) -> Workload:
+def config2(device="cpu", seed: int = 2000, num_q_heads: int = NUM_Q_HEADS) -> Workload:
     """B=32, seq_lens ~ U{1..4096}, pool of 32*256 shuffled pages."""
     seq_lens = torch.randint(1, 4097, (32,), generator=_gen(seed, "cpu"), dtype=torch.int64).to(torch.int32)
     pool = 32 * 256
     bt = assign_pages(seq_lens, pool, seed + 1, stride=256)
-    vals = _values(32, pool, seed, device)
+    vals = _values(32, pool, seed, device, num_q_heads)
     return Workload(name="cfg2: B=32, seq_lens~U[1,4096], page 16, shuffled pool of 8192 pages",
                     seq_lens=seq_lens, block_table=bt, num_pages=pool, **vals)
 
@@ -166,12 +176,12 @@ def config3_layer(layer: int, device="cpu", seed: int = 3000) -> Workload:
 CONFIG3_LAYERS = 28
 
 
-def config4(device="cpu", seed: int = 4000) -> Workload:
+def config4(device="cpu", seed: int = 4000, num_q_heads: int = NUM_Q_HEADS) -> Workload:
     """B=4, seq_len 40960 (the maximum context), 10240 shuffled pages."""
     seq_lens = torch.full((4,), MAX_SEQ, dtype=torch.int32)
     pool = 4 * MAX_PAGES_PER_SEQ
     bt = assign_pages(seq_lens, pool, seed + 1, stride=MAX_PAGES_PER_SEQ)
-    vals = _values(4, pool, seed, device)
+    vals = _values(4, pool, seed, device, num_q_heads)
     return Workload(name="cfg4: B=4, seq_len=40960, 10240 shuffled pages",
                     seq_lens=seq_lens, block_table=bt, num_pages=pool, **vals)
 
@@ -182,13 +192,13 @@ def config5_lengths(seed: int = 5000) -> torch.Tensor:
     return torch.exp(7.0 + 1.5 * z).round().clamp(1, MAX_SEQ).to(torch.int32)
 
 
-def config5(device="cpu", seed: int = 5000) -> Workload:
+def config5(device="cpu", seed: int = 5000, num_q_heads: int = NUM_Q_HEADS) -> Workload:
     """B=256 ragged lognormal lengths; pool 1.1x the pages in use, gaps interleaved."""
     seq_lens = config5_lengths(seed)
     need = int(pages_for(seq_lens).sum())
     pool = int(math.ceil(1.1 * need))
     bt = assign_pages(seq_lens, pool, seed + 1, stride=MAX_PAGES_PER_SEQ, gap_fraction=0.1)
-    vals = _values(256, pool, seed, device)
+    vals = _values(256, pool, seed, device, num_q_heads)
     return Workload(name="cfg5: B=256, seq_lens lognormal(7,1.5) clipped, 10% gap pages",
                     seq_lens=seq_lens, block_table=bt, num_pages=pool, **vals)
 

@@ -61,6 +61,10 @@ def _load():
             u16p, u16p, u16p, i32p, i32p, i32p, ctypes.c_int, u16p, u16p, ctypes.c_int,
             dp, ctypes.c_int, ctypes.c_double, ctypes.c_double, dp, dp]
         lib.oracle_append_and_attend.restype = ctypes.c_int
+        lib.oracle_append_and_attend_gqa.argtypes = [
+            u16p, u16p, u16p, i32p, i32p, i32p, ctypes.c_int, u16p, u16p, ctypes.c_int,
+            dp, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_double, dp, dp]
+        lib.oracle_append_and_attend_gqa.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -122,14 +126,17 @@ def append_and_attend(qkv, q_norm_w, k_norm_w, seq_lens, block_table, k_cache, v
                       inplace: bool = False, want_qk: bool = False) -> dict:
     """Run the whole step. bf16 inputs are uint16 bit arrays.
 
-    Returns a dict with ``o`` (float64 [B,16,128]), ``k_cache`` and ``v_cache``
+    The number of query heads follows from the qkv row width,
+    (num_q_heads + 16) * 128: 16 for Qwen3-0.6B, 32, 40 or 64 for larger sizes.
+    Returns a dict with ``o`` (float64 [B,Hq,128]), ``k_cache`` and ``v_cache``
     (uint16, after the append; the inputs themselves when ``inplace``), and,
-    when ``want_qk``, ``q`` (float64 [B,16,128]) and ``k`` (float64 [B,8,128],
+    when ``want_qk``, ``q`` (float64 [B,Hq,128]) and ``k`` (float64 [B,8,128],
     the new k before its rounding to bf16).
     """
     qkv = np.ascontiguousarray(qkv, dtype=np.uint16)
     B = qkv.shape[0]
-    assert qkv.shape == (B, QKV_WIDTH)
+    assert qkv.ndim == 2 and qkv.shape[1] % HEAD_DIM == 0
+    Hq = qkv.shape[1] // HEAD_DIM - 2 * NUM_KV_HEADS
     q_norm_w = np.ascontiguousarray(q_norm_w, dtype=np.uint16)
     k_norm_w = np.ascontiguousarray(k_norm_w, dtype=np.uint16)
     seq_lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
@@ -144,15 +151,15 @@ def append_and_attend(qkv, q_norm_w, k_norm_w, seq_lens, block_table, k_cache, v
     assert v_cache.dtype == np.uint16 and v_cache.flags["C_CONTIGUOUS"]
     num_pages = k_cache.shape[0]
     assert k_cache.shape == (num_pages, PAGE, NUM_KV_HEADS, HEAD_DIM) == v_cache.shape
-    o = np.empty((B, NUM_Q_HEADS, HEAD_DIM), dtype=np.float64)
-    q = np.empty((B, NUM_Q_HEADS, HEAD_DIM), dtype=np.float64) if want_qk else None
+    o = np.empty((B, Hq, HEAD_DIM), dtype=np.float64)
+    q = np.empty((B, Hq, HEAD_DIM), dtype=np.float64) if want_qk else None
     k = np.empty((B, NUM_KV_HEADS, HEAD_DIM), dtype=np.float64) if want_qk else None
-    rc = _load().oracle_append_and_attend(
+    rc = _load().oracle_append_and_attend_gqa(
         _ptr(qkv, ctypes.c_uint16), _ptr(q_norm_w, ctypes.c_uint16), _ptr(k_norm_w, ctypes.c_uint16),
         _ptr(seq_lens, ctypes.c_int32), _ptr(positions, ctypes.c_int32),
         _ptr(block_table, ctypes.c_int32), block_table.shape[1],
         _ptr(k_cache, ctypes.c_uint16), _ptr(v_cache, ctypes.c_uint16), num_pages,
-        _ptr(o, ctypes.c_double), B, rope_theta, rms_eps,
+        _ptr(o, ctypes.c_double), B, Hq, rope_theta, rms_eps,
         _ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double))
     if rc != 0:
         raise ValueError(f"oracle_append_and_attend: {_ERRORS.get(rc, rc)}")

@@ -56,7 +56,6 @@ enum {
     ORC_PAGE = 16,                /* "At a glance": page size 16 */
     ORC_Q_WIDTH = ORC_NUM_Q_HEADS * ORC_HEAD_DIM,   /* 2048 */
     ORC_KV_WIDTH = ORC_NUM_KV_HEADS * ORC_HEAD_DIM, /* 1024 */
-    ORC_QKV_WIDTH = ORC_Q_WIDTH + 2 * ORC_KV_WIDTH, /* 4096 = attn.qkv_proj N */
     ORC_PAGE_ELEMS = ORC_PAGE * ORC_KV_WIDTH,       /* elements in one page */
     ORC_MAX_BATCH = 256,          /* "At a glance": B in [1, 256] */
     ORC_MAX_SEQ = 40960           /* "At a glance": S in [1, 40960] */
@@ -185,29 +184,38 @@ void oracle_decode_head(const double *q, int L, const int32_t *bt_row,
 /* The decode-attention step for a batch, in the order the specification
  * gives it: for every sequence, norm and rotate q and k, append the new k and
  * v to the cache; then, over the cache as it stands after the append, attend.
+ * num_q_heads query heads share the 8 kv heads: 16 for Qwen3-0.6B and 1.7B,
+ * 32 for 4B/8B, 40 for 14B, 64 for 32B (nnterp qwen3, "Grouped-query
+ * attention, with 128-wide heads on every size"); query head h reads kv head
+ * h / (num_q_heads / 8), which is h / 2 for 0.6B (Model Spec attn.core).
  *
- *   qkv          bf16 [B][4096], q | k | v, head-major (attn.qkv_proj output)
+ *   qkv          bf16 [B][(num_q_heads + 16) * 128], q | k | v, head-major
  *   q_norm_w     bf16 [128], k_norm_w bf16 [128] (one gain for every head)
  *   seq_lens     [B], counts the new token, 1 <= L <= 40960 and <= 16*bt_stride
  *   positions    [B] RoPE positions, or NULL for seq_lens[b]-1
  *   block_table  [B][bt_stride] page ids; entries past ceil(L/16) are not read
  *   k_cache, v_cache  bf16 [num_pages][16][8][128], updated in place
- *   o            double [B][16][128] (output)
- *   q_out        double [B][16][128] or NULL: q after norm and RoPE
+ *   o            double [B][num_q_heads][128] (output)
+ *   q_out        double [B][num_q_heads][128] or NULL: q after norm and RoPE
  *   k_out        double [B][8][128] or NULL: new k after norm and RoPE, before
  *                its rounding to bf16
  *
  * Returns 0, ORC_ERR_ARG, or ORC_ERR_BOUNDS (nothing is written then). */
-int oracle_append_and_attend(const uint16_t *qkv, const uint16_t *q_norm_w,
-                             const uint16_t *k_norm_w, const int32_t *seq_lens,
-                             const int32_t *positions, const int32_t *block_table,
-                             int bt_stride, uint16_t *k_cache, uint16_t *v_cache,
-                             int num_pages, double *o, int B, double rope_theta,
-                             double rms_eps, double *q_out, double *k_out)
+int oracle_append_and_attend_gqa(const uint16_t *qkv, const uint16_t *q_norm_w,
+                                 const uint16_t *k_norm_w, const int32_t *seq_lens,
+                                 const int32_t *positions, const int32_t *block_table,
+                                 int bt_stride, uint16_t *k_cache, uint16_t *v_cache,
+                                 int num_pages, double *o, int B, int num_q_heads,
+                                 double rope_theta, double rms_eps, double *q_out,
+                                 double *k_out)
 {
     if (!qkv || !q_norm_w || !k_norm_w || !seq_lens || !block_table || !k_cache ||
-        !v_cache || !o || B < 1 || B > ORC_MAX_BATCH || bt_stride < 1 || num_pages < 1)
+        !v_cache || !o || B < 1 || B > ORC_MAX_BATCH || bt_stride < 1 || num_pages < 1 ||
+        num_q_heads < ORC_NUM_KV_HEADS || num_q_heads % ORC_NUM_KV_HEADS != 0 || num_q_heads > 64)
         return ORC_ERR_ARG;
+    const int group = num_q_heads / ORC_NUM_KV_HEADS;
+    const int q_width = num_q_heads * ORC_HEAD_DIM;
+    const size_t row_width = (size_t)q_width + 2 * ORC_KV_WIDTH;
 
     /* Validate every index the step will use before touching anything. */
     for (int b = 0; b < B; ++b) {
@@ -225,30 +233,30 @@ int oracle_append_and_attend(const uint16_t *qkv, const uint16_t *q_norm_w,
         wk[i] = oracle_bf16_to_f64(k_norm_w[i]);
     }
 
-    double *q_all = (double *)malloc(sizeof(double) * (size_t)B * ORC_Q_WIDTH);
+    double *q_all = (double *)malloc(sizeof(double) * (size_t)B * q_width);
     if (!q_all) return ORC_ERR_ARG;
 
     /* Norm, rotation and append, sequence by sequence. */
     for (int b = 0; b < B; ++b) {
-        const uint16_t *row = qkv + (size_t)b * ORC_QKV_WIDTH;
+        const uint16_t *row = qkv + (size_t)b * row_width;
         int L = seq_lens[b];
         int slot = L - 1;
         double pos = positions ? (double)positions[b] : (double)slot;
         double x[ORC_HEAD_DIM], y[ORC_HEAD_DIM];
 
-        for (int h = 0; h < ORC_NUM_Q_HEADS; ++h) {
+        for (int h = 0; h < num_q_heads; ++h) {
             for (int i = 0; i < ORC_HEAD_DIM; ++i)
                 x[i] = oracle_bf16_to_f64(row[h * ORC_HEAD_DIM + i]);
             oracle_rmsnorm(x, wq, ORC_HEAD_DIM, rms_eps, y);
             oracle_rope(y, ORC_HEAD_DIM, pos, rope_theta);
-            memcpy(q_all + ((size_t)b * ORC_NUM_Q_HEADS + h) * ORC_HEAD_DIM, y, sizeof y);
+            memcpy(q_all + ((size_t)b * num_q_heads + h) * ORC_HEAD_DIM, y, sizeof y);
         }
 
         int32_t page = block_table[(size_t)b * bt_stride + slot / ORC_PAGE];
         size_t slot_base = (size_t)page * ORC_PAGE_ELEMS + (size_t)(slot % ORC_PAGE) * ORC_KV_WIDTH;
         for (int j = 0; j < ORC_NUM_KV_HEADS; ++j) {
             for (int i = 0; i < ORC_HEAD_DIM; ++i)
-                x[i] = oracle_bf16_to_f64(row[ORC_Q_WIDTH + j * ORC_HEAD_DIM + i]);
+                x[i] = oracle_bf16_to_f64(row[q_width + j * ORC_HEAD_DIM + i]);
             oracle_rmsnorm(x, wk, ORC_HEAD_DIM, rms_eps, y);
             oracle_rope(y, ORC_HEAD_DIM, pos, rope_theta);
             if (k_out) memcpy(k_out + ((size_t)b * ORC_NUM_KV_HEADS + j) * ORC_HEAD_DIM, y, sizeof y);
@@ -256,30 +264,41 @@ int oracle_append_and_attend(const uint16_t *qkv, const uint16_t *q_norm_w,
                 k_cache[slot_base + (size_t)j * ORC_HEAD_DIM + i] = oracle_f64_to_bf16_rne(y[i]);
                 /* v has no norm and no rotation: its bits are copied. */
                 v_cache[slot_base + (size_t)j * ORC_HEAD_DIM + i] =
-                    row[ORC_Q_WIDTH + ORC_KV_WIDTH + j * ORC_HEAD_DIM + i];
+                    row[q_width + ORC_KV_WIDTH + j * ORC_HEAD_DIM + i];
             }
         }
     }
 
-    /* Attention over the cache as it stands after every append. Query head h
-     * reads kv head h/2 (Model Spec attn.core; nnterp qwen3 page, "Grouped-query
-     * attention": kv head j reaches query heads 2j and 2j+1). */
+    /* Attention over the cache as it stands after every append. */
     int max_L = 0;
     for (int b = 0; b < B; ++b) if (seq_lens[b] > max_L) max_L = seq_lens[b];
     double *scores = (double *)malloc(sizeof(double) * (size_t)max_L);
     if (!scores) { free(q_all); return ORC_ERR_ARG; }
     for (int b = 0; b < B; ++b) {
-        for (int h = 0; h < ORC_NUM_Q_HEADS; ++h) {
-            oracle_decode_head(q_all + ((size_t)b * ORC_NUM_Q_HEADS + h) * ORC_HEAD_DIM,
+        for (int h = 0; h < num_q_heads; ++h) {
+            oracle_decode_head(q_all + ((size_t)b * num_q_heads + h) * ORC_HEAD_DIM,
                                seq_lens[b], block_table + (size_t)b * bt_stride,
-                               k_cache, v_cache, h / (ORC_NUM_Q_HEADS / ORC_NUM_KV_HEADS),
-                               scores, o + ((size_t)b * ORC_NUM_Q_HEADS + h) * ORC_HEAD_DIM);
+                               k_cache, v_cache, h / group,
+                               scores, o + ((size_t)b * num_q_heads + h) * ORC_HEAD_DIM);
         }
     }
-    if (q_out) memcpy(q_out, q_all, sizeof(double) * (size_t)B * ORC_Q_WIDTH);
+    if (q_out) memcpy(q_out, q_all, sizeof(double) * (size_t)B * q_width);
     free(scores);
     free(q_all);
     return ORC_OK;
+}
+
+/* The Qwen3-0.6B step: 16 query heads over 8 kv heads (Model Spec attn.core). */
+int oracle_append_and_attend(const uint16_t *qkv, const uint16_t *q_norm_w,
+                             const uint16_t *k_norm_w, const int32_t *seq_lens,
+                             const int32_t *positions, const int32_t *block_table,
+                             int bt_stride, uint16_t *k_cache, uint16_t *v_cache,
+                             int num_pages, double *o, int B, double rope_theta,
+                             double rms_eps, double *q_out, double *k_out)
+{
+    return oracle_append_and_attend_gqa(qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table,
+                                        bt_stride, k_cache, v_cache, num_pages, o, B,
+                                        ORC_NUM_Q_HEADS, rope_theta, rms_eps, q_out, k_out);
 }
 
 /* ---- array forms of the conversions, for the tests ---------------------- */

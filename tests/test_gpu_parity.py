@@ -274,3 +274,19 @@ def test_config3_all_layers(attn):
         # the oracle reads the pre-call cache; rows other than the appended ones are unchanged
         ref = ph.oracle_sampled(w, sample, w.k_cache, w.v_cache)
         ph.assert_o_close(outs[i][torch.as_tensor(sample)], ref, f"cfg3 layer {i}")
+
+
+def test_rope_theta_is_a_runtime_parameter():
+    """nnterp qwen3, "What loads as this family": rope_theta is 1e6 everywhere but the
+    4B-2507 pair (5e6). The base is a create-time parameter; the oracle takes the same."""
+    a = binding.DecodeAttention(device=0, rope_theta=5.0e6)
+    w = inputs.custom([40960, 3, 1000, 17], seed=24, device="cuda", stride=2560)
+    k, v = w.k_cache.clone(), w.v_cache.clone()
+    ref = ph.oracle.append_and_attend(
+        inputs.bf16_bits(w.qkv), inputs.bf16_bits(w.q_norm_w), inputs.bf16_bits(w.k_norm_w),
+        w.seq_lens.numpy(), w.block_table.numpy(), inputs.bf16_bits(k), inputs.bf16_bits(v), rope_theta=5.0e6)
+    o = ph.run(a, w, DEV, k, v)
+    assert a.check() == 0
+    assert np.array_equal(inputs.bf16_bits(k), ref["k_cache"]) and np.array_equal(inputs.bf16_bits(v), ref["v_cache"])
+    ph.assert_o_close(o, ref["o"], "theta 5e6")
+    a.close()

@@ -441,3 +441,45 @@ def test_parameter_count_fixes_shared_head_gains():
     assert V * H + N * per_layer + H == SPEC["parameters"]
     per_head_gains = per_layer - 2 * D + (SPEC["num_attention_heads"] + SPEC["num_key_value_heads"]) * D
     assert V * H + N * per_head_gains + H != SPEC["parameters"]
+
+
+# ----------------------------------------------------------------------------
+# larger Qwen3 sizes: 32, 40 or 64 query heads over the same 8 kv heads
+# (nnterp qwen3, "Grouped-query attention, with 128-wide heads on every size")
+
+@pytest.mark.parametrize("num_q_heads", [32, 40, 64])
+def test_step_with_larger_groups_matches_torch_sdpa(oracle_mod, num_q_heads):
+    from decode_attention_qk_b200 import inputs
+    w = inputs.custom([1, 17, 40], seed=30, num_q_heads=num_q_heads, pool_pages=6)
+    out = oracle_mod.append_and_attend(inputs.bf16_bits(w.qkv), inputs.bf16_bits(w.q_norm_w),
+                                       inputs.bf16_bits(w.k_norm_w), w.seq_lens.numpy(), w.block_table.numpy(),
+                                       inputs.bf16_bits(w.k_cache), inputs.bf16_bits(w.v_cache), want_qk=True)
+    assert out["o"].shape == (3, num_q_heads, 128)
+    kc, vc = out["k_cache"], out["v_cache"]
+    for b, L in enumerate(w.seq_lens.tolist()):
+        bt = w.block_table[b].numpy()
+        K = np.stack([oracle_mod.bf16_to_f64(kc[bt[t // 16], t % 16]) for t in range(L)], axis=1)
+        V = np.stack([oracle_mod.bf16_to_f64(vc[bt[t // 16], t % 16]) for t in range(L)], axis=1)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(out["q"][b])[None, :, None, :], torch.from_numpy(K)[None], torch.from_numpy(V)[None],
+            enable_gqa=True)[0, :, 0].numpy()
+        assert np.max(np.abs(out["o"][b] - ref)) <= 1e-9 * np.max(np.abs(ref))
+
+
+@pytest.mark.parametrize("num_q_heads", [32, 40, 64])
+def test_larger_group_head_mapping(oracle_mod, num_q_heads):
+    """kv head j serves query heads G*j .. G*j+G-1, G = num_q_heads / 8."""
+    from decode_attention_qk_b200 import inputs
+    G = num_q_heads // 8
+    w = inputs.custom([20], seed=31, num_q_heads=num_q_heads)
+    args = [inputs.bf16_bits(w.qkv), inputs.bf16_bits(w.q_norm_w), inputs.bf16_bits(w.k_norm_w),
+            w.seq_lens.numpy(), w.block_table.numpy()]
+    kc, vc = inputs.bf16_bits(w.k_cache), inputs.bf16_bits(w.v_cache)
+    base = oracle_mod.append_and_attend(*args, kc, vc)["o"]
+    for j in (0, 5, 7):
+        vc2 = vc.copy()
+        for t in range(19):
+            vc2[w.block_table[0, t // 16], t % 16, j] ^= 0x0100
+        o = oracle_mod.append_and_attend(*args, kc, vc2)["o"]
+        changed = [h for h in range(num_q_heads) if not np.array_equal(o[0, h], base[0, h])]
+        assert changed == list(range(G * j, G * j + G))
