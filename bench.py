@@ -55,19 +55,22 @@ WORKLOADS = {
 # ----------------------------------------------------------------------------
 # workloads and byte counts
 
-def make_layers(name: str, device, rank: int = 0):
-    """The layers of one step (one Workload per library call)."""
+def make_layers(name: str, device, rank: int = 0, num_q_heads: int = 16):
+    """The layers of one step (one Workload per library call). num_q_heads picks the
+    Qwen3 size: 16 (0.6B), 32 (4B/8B), 40 (14B) or 64 (32B); cfg1 and cfg3 are 0.6B only."""
     off = 100 * rank
+    if name in ("cfg1", "cfg3") and num_q_heads != 16:
+        raise ValueError(f"{name} is defined for Qwen3-0.6B (16 query heads)")
     if name == "cfg1":
         return [inputs.config1(device)] if rank == 0 else [inputs.custom([7, 12], seed=off, device=device)]
     if name == "cfg2":
-        return [inputs.config2(device, seed=2000 + off)]
+        return [inputs.config2(device, seed=2000 + off, num_q_heads=num_q_heads)]
     if name == "cfg3":
         return [inputs.config3_layer(i, device, seed=3000 + off) for i in range(inputs.CONFIG3_LAYERS)]
     if name == "cfg4":
-        return [inputs.config4(device, seed=4000 + off)]
+        return [inputs.config4(device, seed=4000 + off, num_q_heads=num_q_heads)]
     if name == "cfg5":
-        return [inputs.config5(device, seed=5000 + off)]
+        return [inputs.config5(device, seed=5000 + off, num_q_heads=num_q_heads)]
     raise ValueError(name)
 
 
@@ -76,7 +79,7 @@ def kv_bytes(seq_lens) -> int:
     return int(torch.as_tensor(seq_lens, dtype=torch.int64).sum()) * KV_BYTES_PER_TOKEN
 
 
-def algorithmic_bytes(seq_lens) -> int:
+def algorithmic_bytes(seq_lens, num_q_heads: int = 16) -> int:
     """Least HBM traffic of one call: the cached K/V rows read (L-1 per sequence),
     the new k/v rows written, the qkv row read, o written, the block-table
     entries and seq_lens read, and the two gain vectors."""
@@ -84,7 +87,7 @@ def algorithmic_bytes(seq_lens) -> int:
     B = int(L.numel())
     pages = int(((L + 15) // 16).sum())
     return (int((L - 1).sum()) * KV_BYTES_PER_TOKEN + B * KV_BYTES_PER_TOKEN
-            + B * inputs.QKV_WIDTH * 2 + B * inputs.NUM_Q_HEADS * inputs.HEAD_DIM * 2
+            + B * inputs.qkv_width(num_q_heads) * 2 + B * num_q_heads * inputs.HEAD_DIM * 2
             + pages * 4 + B * 4 + 2 * inputs.HEAD_DIM * 2)
 
 
@@ -301,15 +304,15 @@ def run_gpu(args):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     lib = binding.load_library()
-    attn = binding.DecodeAttention(device=local)
+    attn = binding.DecodeAttention(device=local, num_q_heads=args.num_q_heads)
 
     # R resident copies of the step's inputs, so that a call never finds its
     # K/V in L2 from the previous call (each copy's KV is > L2 or R copies are).
-    first = make_layers(args.workload, dev, rank)
+    first = make_layers(args.workload, dev, rank, args.num_q_heads)
     step_kv = sum(kv_bytes(w.seq_lens) for w in first)
     rotate = args.rotate or max(1, min(8, math.ceil(4 * L2_BYTES / max(step_kv, 1))))
     # the copies hold the same bytes in different memory, so every timed launch does the same work
-    sets = [first] + [make_layers(args.workload, dev, rank) for r in range(1, rotate)]
+    sets = [first] + [make_layers(args.workload, dev, rank, args.num_q_heads) for r in range(1, rotate)]
     calls_per_step = len(first)
     stream = torch.cuda.current_stream(dev)
     sp = ctypes.c_void_p(stream.cuda_stream)
@@ -319,7 +322,7 @@ def run_gpu(args):
         for w in layers:
             t = dict(qkv=w.qkv, q=w.q_norm_w, k=w.k_norm_w, sl=w.seq_lens.to(dev), bt=w.block_table.to(dev),
                      kc=w.k_cache, vc=w.v_cache,
-                     o=torch.empty((w.batch, 16, 128), dtype=torch.bfloat16, device=dev))
+                     o=torch.empty((w.batch, w.num_q_heads, 128), dtype=torch.bfloat16, device=dev))
             c = (attn.handle, ctypes.c_void_p(t["qkv"].data_ptr()), ctypes.c_void_p(t["q"].data_ptr()),
                  ctypes.c_void_p(t["k"].data_ptr()),
                  ctypes.cast(ctypes.c_void_p(t["sl"].data_ptr()), ctypes.POINTER(ctypes.c_int32)), None,
@@ -378,7 +381,8 @@ def run_gpu(args):
     ms_per_step = ms / args.steps
     # every rotation set has its own lengths (cfg2/cfg5 draw them); average the bytes per step
     kv_per_step_local = sum(sum(kv_bytes(w.seq_lens) for w in s) for s in (sets[i % rotate] for i in range(args.steps))) / args.steps
-    alg_per_step_local = sum(sum(algorithmic_bytes(w.seq_lens) for w in s) for s in (sets[i % rotate] for i in range(args.steps))) / args.steps
+    alg_per_step_local = sum(sum(algorithmic_bytes(w.seq_lens, w.num_q_heads) for w in s)
+                             for s in (sets[i % rotate] for i in range(args.steps))) / args.steps
     kv_total = reduce_sum(dist, kv_per_step_local, dev)
     value = kv_total / (ms_per_step * 1e-3) / 1e9
 
@@ -387,7 +391,8 @@ def run_gpu(args):
     alg_per_launch = alg_per_step_local / calls_per_step
     peak, peak_kind = hbm_peak()
     achieved = alg_per_launch / (mean_kernel_ms * 1e-3) / 1e9
-    traffic = traffic_per_launch(args.workload)
+    workload_key = args.workload if args.num_q_heads == 16 else f"{args.workload}-h{args.num_q_heads}"
+    traffic = traffic_per_launch(workload_key)
 
     # end to end through the host-buffer entry point: per step the H2D copy of the
     # step's inputs from pinned memory, the call, and the D2H copy of o
@@ -402,10 +407,11 @@ def run_gpu(args):
             "us_per_call": round(ms_per_step * 1e3 / calls_per_step, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "io_dtype": "bf16", "data": "synthetic (seeded; N(0,1) bf16 qkv and cache, gains 1+U(-0.5,0.5))",
-            "config": {"workload": f"{args.workload}: {WORKLOADS[args.workload]}",
+            "config": {"workload": f"{args.workload}: {WORKLOADS[args.workload]}"
+                                   + ("" if args.num_q_heads == 16 else f", {args.num_q_heads} query heads"),
                        "batch": first[0].batch, "layers_per_step": calls_per_step,
                        "sum_seq_lens_per_step": int(sum(int(w.seq_lens.sum()) for w in first)),
-                       "page_size": 16, "heads": "16 q / 8 kv, D=128",
+                       "page_size": 16, "heads": f"{args.num_q_heads} q / 8 kv, D=128",
                        "l2": f"{rotate} resident input sets rotated; {rotate * step_kv / 1e9:.2f} GB of KV cycled "
                              f"(> {L2_BYTES / 2**20:.0f} MiB L2)",
                        "grid_ctas": attn.grid_ctas, "parallelism": f"replicas x{world}"},
@@ -416,7 +422,8 @@ def run_gpu(args):
                          "kernel_us_mean": round(mean_kernel_ms * 1e3, 3),
                          "kernel_us_median": round(statistics.median(kernel_ms) * 1e3, 3)},
             "e2e": e2e,
-            "gpu_launches": n_launch,
+            # one kernel per call at 16 query heads; attention + combine launches otherwise
+            "gpu_launches": n_launch * (1 if args.num_q_heads == 16 else 2),
             "clocks": clk,
         }
     if dist is not None:
@@ -440,7 +447,7 @@ def run_e2e(args, attn, sets, dev, stream, dist, rotate):
         for w in layers:
             h = dict(qkv=w.qkv.cpu().pin_memory(), sl=w.seq_lens.clone().pin_memory(),
                      bt=w.block_table.clone().pin_memory(),
-                     o=torch.empty((w.batch, 16, 128), dtype=torch.bfloat16).pin_memory())
+                     o=torch.empty((w.batch, w.num_q_heads, 128), dtype=torch.bfloat16).pin_memory())
             c = (attn.handle, ctypes.c_void_p(h["qkv"].data_ptr()), ctypes.c_void_p(w.q_norm_w.data_ptr()),
                  ctypes.c_void_p(w.k_norm_w.data_ptr()),
                  ctypes.cast(ctypes.c_void_p(h["sl"].data_ptr()), ctypes.POINTER(ctypes.c_int32)), None,
@@ -488,7 +495,7 @@ def run_reference(args):
         return
     import oracle
     oracle.build()
-    layers = make_layers(args.workload, "cpu", 0)
+    layers = make_layers(args.workload, "cpu", 0, args.num_q_heads)
     # size each step's sample so that warm-up + timed steps take ~2 minutes
     probe = min(range(layers[0].batch), key=lambda b: int(layers[0].seq_lens[b]))
     dt = time_oracle(compact_host(layers[0], [probe]))
@@ -530,8 +537,10 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded; same recipe as the GPU arm, drawn on the host)",
-        "config": {"workload": f"{args.workload}: {WORKLOADS[args.workload]}", "batch": layers[0].batch,
-                   "layers_per_step": len(layers), "page_size": 16, "heads": "16 q / 8 kv, D=128"},
+        "config": {"workload": f"{args.workload}: {WORKLOADS[args.workload]}"
+                               + ("" if args.num_q_heads == 16 else f", {args.num_q_heads} query heads"),
+                   "batch": layers[0].batch, "layers_per_step": len(layers), "page_size": 16,
+                   "heads": f"{args.num_q_heads} q / 8 kv, D=128"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": sample_desc},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -545,6 +554,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="cfg2")
+    ap.add_argument("--num-q-heads", type=int, choices=[16, 32, 40, 64], default=16,
+                    help="query heads: 16 = Qwen3-0.6B (the default workload); 32/40/64 = 4B-8B/14B/32B")
     ap.add_argument("--rotate", type=int, default=0, help="resident input sets cycled (0: enough to defeat L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -26,6 +26,7 @@ QDA_ERR_TIMEOUT = -5
 QDA_FLAG_INJECT_WAIT_TIMEOUT = 0x1
 
 NUM_Q_HEADS, NUM_KV_HEADS, HEAD_DIM, PAGE_SIZE, QKV_WIDTH = 16, 8, 128, 16, 4096
+SUPPORTED_Q_HEADS = (16, 32, 40, 64)   # Qwen3 0.6B/1.7B, 4B/8B, 14B, 32B
 
 
 class qda_config(ctypes.Structure):
@@ -133,10 +134,18 @@ def qwen3_decode_attn_create(cfg: qda_config | None = None, device: int = 0) -> 
     return h
 
 
+def num_q_heads_of(qkv: torch.Tensor) -> int:
+    """Query heads of a fused qkv row of (Hq + 16) * 128 values."""
+    if qkv.dim() != 2 or qkv.shape[1] % HEAD_DIM != 0:
+        raise ValueError("qkv must be [B, (num_q_heads + 16) * 128]")
+    return int(qkv.shape[1]) // HEAD_DIM - 2 * NUM_KV_HEADS
+
+
 def _step_args(qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, k_cache, v_cache, o,
                dev_of_step, dev_of_state):
-    B = qkv.shape[0] if qkv.dim() == 2 else -1
-    _expect(qkv, "qkv", torch.bfloat16, (B, QKV_WIDTH), dev_of_step)
+    Hq = num_q_heads_of(qkv)
+    B = qkv.shape[0]
+    _expect(qkv, "qkv", torch.bfloat16, (B, (Hq + 2 * NUM_KV_HEADS) * HEAD_DIM), dev_of_step)
     _expect(q_norm_w, "q_norm_w", torch.bfloat16, (HEAD_DIM,), dev_of_state)
     _expect(k_norm_w, "k_norm_w", torch.bfloat16, (HEAD_DIM,), dev_of_state)
     _expect(seq_lens, "seq_lens", torch.int32, (B,), dev_of_step)
@@ -148,7 +157,7 @@ def _step_args(qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, k_cach
     P = k_cache.shape[0]
     _expect(k_cache, "k_cache", torch.bfloat16, (P, PAGE_SIZE, NUM_KV_HEADS, HEAD_DIM), dev_of_state)
     _expect(v_cache, "v_cache", torch.bfloat16, (P, PAGE_SIZE, NUM_KV_HEADS, HEAD_DIM), dev_of_state)
-    _expect(o, "o", torch.bfloat16, (B, NUM_Q_HEADS, HEAD_DIM), dev_of_step)
+    _expect(o, "o", torch.bfloat16, (B, Hq, HEAD_DIM), dev_of_step)
     return (_ptr(qkv), _ptr(q_norm_w), _ptr(k_norm_w), _i32p(seq_lens), _i32p(positions),
             _i32p(block_table), int(block_table.shape[1]), _ptr(k_cache), _ptr(v_cache), int(P),
             _ptr(o), int(B))
@@ -211,7 +220,10 @@ def qwen3_decode_attn_destroy(handle) -> None:
 
 
 class DecodeAttention:
-    """A handle with its lifetime: DecodeAttention(device=0, **config fields)."""
+    """A handle with its lifetime: DecodeAttention(device=0, **config fields).
+
+    `num_q_heads` (16, 32, 40 or 64) selects the Qwen3 size; calls must pass qkv
+    rows of (num_q_heads + 16) * 128 values."""
 
     def __init__(self, device: int = 0, **config):
         self.device = torch.device("cuda", device)
@@ -224,8 +236,12 @@ class DecodeAttention:
 
     def __call__(self, qkv, q_norm_w, k_norm_w, seq_lens, block_table, k_cache, v_cache, o=None,
                  positions=None, stream=None) -> torch.Tensor:
+        if num_q_heads_of(qkv) != self.config.num_q_heads:
+            raise ValueError(f"qkv rows hold {num_q_heads_of(qkv)} query heads; the handle was made for "
+                             f"{self.config.num_q_heads}")
         if o is None:
-            o = torch.empty((qkv.shape[0], NUM_Q_HEADS, HEAD_DIM), dtype=torch.bfloat16, device=qkv.device)
+            o = torch.empty((qkv.shape[0], self.config.num_q_heads, HEAD_DIM), dtype=torch.bfloat16,
+                            device=qkv.device)
         qwen3_decode_attn_append_and_attend(self.handle, qkv, q_norm_w, k_norm_w, seq_lens, positions,
                                             block_table, k_cache, v_cache, o, stream)
         return o

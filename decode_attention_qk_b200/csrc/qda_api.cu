@@ -18,6 +18,7 @@ struct qda_handle {
     float2* part_ml = nullptr;
     int* counters = nullptr;
     int* status = nullptr;
+    int* seg = nullptr;
     // staging of the host-buffer entry point
     uint16_t* st_qkv = nullptr;
     int32_t* st_seq_lens = nullptr;
@@ -31,6 +32,12 @@ namespace {
 constexpr int64_t kDefaultTimeoutNs = 1000000000;  // 1 s
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// The query-head counts of the Qwen3 sizes: 16 (0.6B, 1.7B), 32 (4B, 8B),
+// 40 (14B), 64 (32B), all over 8 kv heads of 128.
+bool supported_q_heads(int n) { return n == 16 || n == 32 || n == 40 || n == 64; }
+
+size_t qkv_elems(int num_q_heads) { return (size_t)(num_q_heads + 2 * qda::kNumKvHeads) * qda::kHeadDim; }
 
 // Makes `device` current for the lifetime of the guard, then restores the
 // caller's device.
@@ -54,6 +61,7 @@ void free_workspace(qda_handle* h) {
     cudaFree(h->part_ml);
     cudaFree(h->counters);
     cudaFree(h->status);
+    cudaFree(h->seg);
     cudaFree(h->st_qkv);
     cudaFree(h->st_seq_lens);
     cudaFree(h->st_positions);
@@ -95,6 +103,7 @@ qda::Params make_params(const qda_handle* h, const void* qkv, const void* q_norm
     p.k_cache = static_cast<uint16_t*>(k_cache);
     p.v_cache = static_cast<uint16_t*>(v_cache);
     p.o = static_cast<uint16_t*>(o);
+    p.num_q_heads = h->cfg.num_q_heads;
     p.bt_stride = block_table_stride;
     p.num_pages = num_pages;
     p.batch = batch;
@@ -104,10 +113,16 @@ qda::Params make_params(const qda_handle* h, const void* qkv, const void* q_norm
     p.part_acc = h->part_acc;
     p.part_ml = h->part_ml;
     p.counters = h->counters;
+    p.seg = h->seg;
     p.status = h->status;
     p.timeout_ns = h->cfg.wait_timeout_ns > 0 ? h->cfg.wait_timeout_ns : kDefaultTimeoutNs;
     p.flags = h->cfg.flags;
     return p;
+}
+
+cudaError_t launch_step(const qda_handle* h, const qda::Params& p, cudaStream_t stream) {
+    return h->cfg.num_q_heads == qda::kNumQHeads ? qda::launch(p, h->grid, stream)
+                                                 : qda::launch_grouped(p, h->grid, stream);
 }
 
 }  // namespace
@@ -135,7 +150,7 @@ int qwen3_decode_attn_create(const qda_config* cfg, int device, qda_handle** out
     if (out == nullptr) return QDA_ERR_INVALID_ARG;
     *out = nullptr;
     if (cfg == nullptr) return QDA_ERR_INVALID_ARG;
-    if (cfg->num_q_heads != QDA_NUM_Q_HEADS || cfg->num_kv_heads != QDA_NUM_KV_HEADS ||
+    if (!supported_q_heads(cfg->num_q_heads) || cfg->num_kv_heads != QDA_NUM_KV_HEADS ||
         cfg->head_dim != QDA_HEAD_DIM || cfg->page_size != QDA_PAGE_SIZE)
         return QDA_ERR_UNSUPPORTED;
     if (cfg->max_batch < 1 || cfg->max_batch > QDA_MAX_BATCH || cfg->max_seq_len < 1 ||
@@ -152,7 +167,7 @@ int qwen3_decode_attn_create(const qda_config* cfg, int device, qda_handle** out
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms < 1)
         return QDA_ERR_CUDA;
-    if (qda::prepare_device() != cudaSuccess) return QDA_ERR_CUDA;
+    if (qda::prepare_device() != cudaSuccess || qda::prepare_grouped() != cudaSuccess) return QDA_ERR_CUDA;
 
     qda_handle* h = new (std::nothrow) qda_handle();
     if (h == nullptr) return QDA_ERR_CUDA;
@@ -162,14 +177,15 @@ int qwen3_decode_attn_create(const qda_config* cfg, int device, qda_handle** out
 
     const size_t slots = (size_t)qda::num_slots(h->grid, cfg->max_batch);
     const size_t B = (size_t)cfg->max_batch;
-    bool ok = alloc(&h->part_acc, slots * qda::kNumQHeads * qda::kHeadDim * sizeof(float)) &&
-              alloc(&h->part_ml, slots * qda::kNumQHeads * sizeof(float2)) &&
+    const size_t Hq = (size_t)cfg->num_q_heads;
+    bool ok = alloc(&h->part_acc, slots * Hq * qda::kHeadDim * sizeof(float)) &&
+              alloc(&h->part_ml, slots * Hq * sizeof(float2)) &&
               alloc(&h->counters, (size_t)qda::kMaxBatch * qda::kNumKvHeads * sizeof(int)) &&
-              alloc(&h->status, sizeof(int)) &&
-              alloc(&h->st_qkv, B * qda::kQkvWidth * sizeof(uint16_t)) &&
+              alloc(&h->status, sizeof(int)) && alloc(&h->seg, (size_t)(qda::kMaxBatch + 1) * sizeof(int)) &&
+              alloc(&h->st_qkv, B * qkv_elems(cfg->num_q_heads) * sizeof(uint16_t)) &&
               alloc(&h->st_seq_lens, B * sizeof(int32_t)) && alloc(&h->st_positions, B * sizeof(int32_t)) &&
               alloc(&h->st_block_table, B * (size_t)cfg->max_pages_per_seq * sizeof(int32_t)) &&
-              alloc(&h->st_o, B * qda::kNumQHeads * qda::kHeadDim * sizeof(uint16_t));
+              alloc(&h->st_o, B * Hq * qda::kHeadDim * sizeof(uint16_t));
     ok = ok && cudaMemset(h->counters, 0, (size_t)qda::kMaxBatch * qda::kNumKvHeads * sizeof(int)) == cudaSuccess &&
          cudaMemset(h->status, 0, sizeof(int)) == cudaSuccess && cudaDeviceSynchronize() == cudaSuccess;
     if (!ok) {
@@ -193,7 +209,7 @@ int qwen3_decode_attn_append_and_attend(qda_handle* h, const void* qkv, const vo
     if (!guard.ok()) return QDA_ERR_CUDA;
     const qda::Params p = make_params(h, qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table,
                                       block_table_stride, k_cache, v_cache, num_pages, o, batch);
-    return qda::launch(p, h->grid, static_cast<cudaStream_t>(cuda_stream)) == cudaSuccess ? QDA_OK : QDA_ERR_CUDA;
+    return launch_step(h, p, static_cast<cudaStream_t>(cuda_stream)) == cudaSuccess ? QDA_OK : QDA_ERR_CUDA;
 }
 
 int qwen3_decode_attn_append_and_attend_host(qda_handle* h, const void* qkv_host, const void* q_norm_w,
@@ -210,8 +226,8 @@ int qwen3_decode_attn_append_and_attend_host(qda_handle* h, const void* qkv_host
     if (!guard.ok()) return QDA_ERR_CUDA;
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     const size_t B = (size_t)batch;
-    bool ok = cudaMemcpyAsync(h->st_qkv, qkv_host, B * qda::kQkvWidth * sizeof(uint16_t), cudaMemcpyHostToDevice,
-                              st) == cudaSuccess &&
+    bool ok = cudaMemcpyAsync(h->st_qkv, qkv_host, B * qkv_elems(h->cfg.num_q_heads) * sizeof(uint16_t),
+                              cudaMemcpyHostToDevice, st) == cudaSuccess &&
               cudaMemcpyAsync(h->st_seq_lens, seq_lens_host, B * sizeof(int32_t), cudaMemcpyHostToDevice, st) ==
                   cudaSuccess &&
               cudaMemcpyAsync(h->st_block_table, block_table_host, B * (size_t)block_table_stride * sizeof(int32_t),
@@ -223,8 +239,8 @@ int qwen3_decode_attn_append_and_attend_host(qda_handle* h, const void* qkv_host
     const qda::Params p = make_params(h, h->st_qkv, q_norm_w, k_norm_w, h->st_seq_lens,
                                       positions_host != nullptr ? h->st_positions : nullptr, h->st_block_table,
                                       block_table_stride, k_cache, v_cache, num_pages, h->st_o, batch);
-    if (qda::launch(p, h->grid, st) != cudaSuccess) return QDA_ERR_CUDA;
-    if (cudaMemcpyAsync(o_host, h->st_o, B * qda::kNumQHeads * qda::kHeadDim * sizeof(uint16_t),
+    if (launch_step(h, p, st) != cudaSuccess) return QDA_ERR_CUDA;
+    if (cudaMemcpyAsync(o_host, h->st_o, B * (size_t)h->cfg.num_q_heads * qda::kHeadDim * sizeof(uint16_t),
                         cudaMemcpyDeviceToHost, st) != cudaSuccess)
         return QDA_ERR_CUDA;
     return QDA_OK;
@@ -263,7 +279,9 @@ const char* qwen3_decode_attn_strerror(int code) {
         case QDA_OK: return "success";
         case QDA_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, or a size outside its range)";
         case QDA_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
-        case QDA_ERR_UNSUPPORTED: return "configuration differs from the compiled head geometry (16/8/128, page 16)";
+        case QDA_ERR_UNSUPPORTED:
+            return "configuration differs from the compiled head geometry (16/32/40/64 query heads, 8 kv heads, "
+                   "head dim 128, page 16)";
         case QDA_ERR_BOUNDS: return "a seq_len or block-table entry was out of range on the device";
         case QDA_ERR_TIMEOUT: return "a device-side wait ran out of time";
         default: return "unknown error code";

@@ -1,0 +1,672 @@
+// Decode-attention step for the larger Qwen3 sizes: 32, 40 or 64 query heads
+// over 8 kv heads of 128 (nnterp qwen3, "Grouped-query attention, with
+// 128-wide heads on every size"), i.e. G = 4, 5 or 8 query heads per kv head.
+// Same computation as the 16-head kernel (Qwen3-0.6B Model Spec,
+// "Compute-graph nodes": attn.qk_norm, attn.rope, attn.core, and the append
+// to the 16-token paged cache); query head h reads kv head h / G.
+//
+// Why tensor cores here. Per kv head and page the scores and the value sums
+// are a [G x 128] x [128 x 16] and a [G x 16] x [16 x 128] product: 2G flops
+// per byte of K/V, 16 at G = 8, above what the CUDA cores sustain at HBM
+// speed. Warp j (kv head j) runs them as mma.sync m16n8k16 bf16 products with
+// float accumulators. The 16 rows of the A operand hold, for head g < G, row g
+// = the bf16 value of q (or of the probabilities) and row g + 8 = the bf16 of
+// the remainder, so the products carry ~16 significant bits of q and p; the
+// two rows are added back in float. The score accumulator fragment of lane
+// (g = lane/4, t = lane%4) holds head g at tokens 2t, 2t+1, 8+2t, 9+2t, which is
+// exactly its A fragment for the value product, so probabilities never leave
+// registers.
+//
+// Staging. A producer warp bulk-copies each token row (2 KiB, all 8 kv heads)
+// into a stage whose rows are 2064 bytes apart, so that the 8 rows an
+// ldmatrix phase reads start in 8 different 16-byte bank groups (at the
+// cache's own 2048-byte pitch they would all hit the same banks). Each
+// sequence piece's qkv row goes to one slot of its own, released by the
+// consumers once they have formed q.
+//
+// Split sequences. The work split is the 16-head kernel's (equal page ranges
+// per CTA, scratch slot g + b per piece). A piece that covers its whole
+// sequence writes o; a piece of a split sequence writes its partial, and a
+// second launch (one CTA per sequence and query head, one thread per dim)
+// combines them with the log-sum-exp rule (Supported models, "Facts proved
+// about the specs": flashAttn_eq, softmax_shift), spreading long merges over
+// many SMs. That launch uses programmatic dependent launch so its start
+// overlaps the first kernel's tail.
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "qda_device.cuh"
+#include "qda_internal.h"
+#include "qwen3_decode_attn.h"
+
+namespace qda {
+namespace {
+
+constexpr int kStages = 3;
+constexpr int kConsumerWarps = kNumKvHeads;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kRowPitch = kRowBytes + 16;           // staged token-row pitch: 2064 bytes
+constexpr int kStageK = 0;
+constexpr int kStageV = kPage * kRowPitch;
+constexpr int kStageBytes = 2 * kPage * kRowPitch;  // 66048
+constexpr int kCombineThreads = kHeadDim;           // combine launch: one thread per dim
+
+template <int G>
+struct Layout {
+    static constexpr int kHq = G * kNumKvHeads;
+    static constexpr int kQkvW = (kHq + 2 * kNumKvHeads) * kHeadDim;   // elements in a qkv row
+    static constexpr int kQkvBytes = kQkvW * 2;
+    static constexpr int kSmemQkv = kStages * kStageBytes;
+    static constexpr int kSmemSeg = kSmemQkv + kQkvBytes;                   // int [kMaxBatch + 4]
+    static constexpr int kSmemLens = kSmemSeg + (kMaxBatch + 4) * 4;        // int [kMaxBatch]
+    static constexpr int kSmemInvFreq = kSmemLens + kMaxBatch * 4;          // double [64]
+    static constexpr int kSmemGains = kSmemInvFreq + 64 * 8;                // bf16 [2][128]
+    static constexpr int kSmemMeta = kSmemGains + 2 * kHeadDim * 2;         // StageMeta [kStages] + qkv position
+    static constexpr int kSmemBars = kSmemMeta + (kStages + 1) * 16;        // full, empty, qkv_full, qkv_empty, never
+    static constexpr int kSmemFlags = kSmemBars + (2 * kStages + 3) * 8;
+    static constexpr int kSmemTotal = kSmemFlags + 16;
+    static_assert(kSmemQkv % 16 == 0 && kSmemInvFreq % 8 == 0 && kSmemBars % 8 == 0, "alignment");
+    static_assert(kSmemTotal <= 227 * 1024, "fits one CTA per SM");
+};
+
+struct Shared {
+    uint8_t* stages;
+    uint8_t* qkv;         // the current sequence piece's qkv row
+    int* seg;
+    int* lens;
+    double* inv_freq;
+    const uint16_t* gains;
+    volatile StageMeta* meta;
+    volatile int* qkv_pos;
+    uint64_t* full_bar;
+    uint64_t* empty_bar;
+    uint64_t* qkv_full;
+    uint64_t* qkv_empty;
+    uint64_t* never_bar;
+    volatile int* abort_flag;
+};
+
+// ---------------------------------------------------------------------------
+// Producer warp.
+
+template <int G>
+__device__ __forceinline__ void run_producer(const Params& p, const Shared& s, int B, int start, int end, int lane) {
+    using Lay = Layout<G>;
+    const int count = end - start;
+    int slot = 0;
+    uint32_t phase = 0, qphase = 0;
+    uint32_t armed = 0, armed_parity = 0;
+    bool qarmed = false;
+    uint32_t qarmed_parity = 0;
+    bool aborted = false;
+    for (int base = 0; base < count && !aborted; base += 32) {
+        const int gp = start + base + lane;
+        int id = 0, rows = 0, qkv_b = -1, pos = 0;
+        if (gp < end) {
+            const int b = find_seq(s.seg, B, gp);
+            const int i = gp - s.seg[b];
+            const int nb = s.seg[b + 1] - s.seg[b];
+            id = __ldg(p.block_table + (size_t)b * p.bt_stride + i);
+            rows = (i == nb - 1) ? (s.lens[b] - 1) - kPage * i : kPage;
+            if (gp == start || i == 0) {
+                qkv_b = b;
+                pos = p.positions != nullptr ? __ldg(p.positions + b) : s.lens[b] - 1;
+            }
+        }
+        const int n = min(32, count - base);
+        for (int kk = 0; kk < n; ++kk) {
+            const int page_id = __shfl_sync(kFull, id, kk);
+            const int page_rows = __shfl_sync(kFull, rows, kk);
+            const int seq_qkv = __shfl_sync(kFull, qkv_b, kk);
+            const int seq_pos = __shfl_sync(kFull, pos, kk);
+            int ok = 1;
+            uint32_t kv_bytes = 0;
+            if (lane == 0) {
+                if (seq_qkv >= 0) {
+                    // the qkv slot frees once every consumer has formed q from it
+                    ok = mbar_try_wait(s.qkv_empty, qphase ^ 1u) ||
+                         mbar_wait(s.qkv_empty, qphase ^ 1u, p.timeout_ns, s.abort_flag);
+                    if (ok) {
+                        *s.qkv_pos = seq_pos;
+                        mbar_arrive_expect_tx(s.qkv_full, (uint32_t)Lay::kQkvBytes);
+                        bulk_g2s(s.qkv, p.qkv + (size_t)seq_qkv * Lay::kQkvW, (uint32_t)Lay::kQkvBytes, s.qkv_full);
+                        qarmed = true;
+                        qarmed_parity = qphase;
+                        qphase ^= 1u;
+                    }
+                }
+                if (ok)
+                    ok = mbar_try_wait(&s.empty_bar[slot], phase ^ 1u) ||
+                         mbar_wait(&s.empty_bar[slot], phase ^ 1u, p.timeout_ns, s.abort_flag);
+                if (ok) {
+                    const bool bad = page_id < 0 || page_id >= p.num_pages;
+                    s.meta[slot].page = page_id;
+                    s.meta[slot].bad = bad ? 1 : 0;
+                    if (bad) record_error(p.status, QDA_ERR_BOUNDS);
+                    kv_bytes = bad ? 0u : (uint32_t)page_rows * kRowBytes;
+                    if (kv_bytes != 0) {
+                        mbar_arrive_expect_tx(&s.full_bar[slot], 2u * kv_bytes);
+                        armed |= 1u << slot;
+                        armed_parity = (armed_parity & ~(1u << slot)) | (phase << slot);
+                    } else {
+                        mbar_arrive(&s.full_bar[slot]);
+                    }
+                } else {
+                    *s.abort_flag = 1;
+                    record_error(p.status, QDA_ERR_TIMEOUT);
+                }
+            }
+            ok = __shfl_sync(kFull, ok, 0);
+            if (!ok) {
+                aborted = true;
+                break;
+            }
+            // one row copy per lane: lanes 0..15 the K rows, 16..31 the V rows
+            kv_bytes = __shfl_sync(kFull, kv_bytes, 0);
+            if (kv_bytes != 0 && (lane & 15) < page_rows) {
+                const int r = lane & 15;
+                const bool is_v = lane >= 16;
+                uint8_t* dst = s.stages + slot * kStageBytes + (is_v ? kStageV : kStageK) + r * kRowPitch;
+                const uint8_t* src = reinterpret_cast<const uint8_t*>(is_v ? p.v_cache : p.k_cache) +
+                                     (size_t)page_id * kPageBytes + (size_t)r * kRowBytes;
+                bulk_g2s(dst, src, (uint32_t)kRowBytes, &s.full_bar[slot]);
+            }
+            if (++slot == kStages) {
+                slot = 0;
+                phase ^= 1u;
+            }
+        }
+    }
+    if (lane == 0 && *s.abort_flag != 0) {
+        for (int k = 0; k < kStages; ++k)
+            if (armed & (1u << k)) (void)mbar_wait(&s.full_bar[k], (armed_parity >> k) & 1u, p.timeout_ns, nullptr);
+        if (qarmed) (void)mbar_wait(s.qkv_full, qarmed_parity, p.timeout_ns, nullptr);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Consumer warps.
+
+struct State {
+    uint32_t qa[8][4];    // A fragments of q per 16-dim step: rows g (bf16 of q) and g+8 (remainder)
+    float o[16][4];       // value accumulators: 16 tiles of 8 dims, rows g and g+8
+    float m;              // running max of head g (log2 units)
+    float lsum;           // partial softmax sum of this lane's tokens
+    uint32_t k_lo, k_hi, v_lo, v_hi;   // this lane's words of the appended k/v row
+};
+
+// Start a sequence piece from the staged qkv row: q of head G*j + g for lane
+// (g, t) at dims 8m + 2t, 8m + 2t + 1 (m = 0..15), i.e. both halves of the
+// rotation pairs 8m' + 2t + e, m' < 8; the angles of pairs 2l, 2l+1 are formed
+// by lane l (reduced modulo 2*pi in double, then float sin/cos) and shared by
+// shuffles. The new k, when this CTA appends, is formed in double.
+template <int G>
+__device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s, int pos, int j, int lane,
+                                               bool appends, State& st) {
+    using Lay = Layout<G>;
+    constexpr double kTwoPiHi = 6.2831853069365025;      // 2*pi rounded to 32 significant bits
+    constexpr double kTwoPiLo = 2.430840202602477e-10;   // 2*pi - kTwoPiHi
+    constexpr double kInvTwoPi = 0.15915494309189535;
+    const int g = lane >> 2, t = lane & 3;
+    const double ang0 = (double)pos * s.inv_freq[2 * lane];
+    const double ang1 = (double)pos * s.inv_freq[2 * lane + 1];
+    float cf0, sf0, cf1, sf1;
+    {
+        const double n0 = rint(ang0 * kInvTwoPi), n1 = rint(ang1 * kInvTwoPi);
+        sincosf((float)fma(-n0, kTwoPiLo, fma(-n0, kTwoPiHi, ang0)), &sf0, &cf0);
+        sincosf((float)fma(-n1, kTwoPiLo, fma(-n1, kTwoPiHi, ang1)), &sf1, &cf1);
+    }
+    const bool active = g < G;
+    const uint32_t* xq = reinterpret_cast<const uint32_t*>(s.qkv + (G * j + (active ? g : 0)) * (kHeadDim * 2));
+    const uint32_t* gq = reinterpret_cast<const uint32_t*>(s.gains);
+    uint32_t xw[16];
+    float ss = 0.f;
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+        xw[m] = xq[4 * m + t];
+        ss = fmaf(bf_lo(xw[m]), bf_lo(xw[m]), fmaf(bf_hi(xw[m]), bf_hi(xw[m]), ss));
+    }
+    ss += __shfl_xor_sync(kFull, ss, 1);
+    ss += __shfl_xor_sync(kFull, ss, 2);
+    const float inv_r = rsqrtf(ss * (1.f / 128.f) + (float)p.rms_eps);
+    const float scale = (float)kQScale;
+#pragma unroll
+    for (int mp = 0; mp < 8; ++mp) {
+        float qa[2], qb[2];
+        const uint32_t wlo = gq[4 * mp + t], whi = gq[32 + 4 * mp + t];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const float cs = __shfl_sync(kFull, e ? cf1 : cf0, 4 * mp + t);
+            const float sn = __shfl_sync(kFull, e ? sf1 : sf0, 4 * mp + t);
+            const float ya = (e ? bf_hi(xw[mp]) : bf_lo(xw[mp])) * inv_r * (e ? bf_hi(wlo) : bf_lo(wlo));
+            const float yb = (e ? bf_hi(xw[mp + 8]) : bf_lo(xw[mp + 8])) * inv_r * (e ? bf_hi(whi) : bf_lo(whi));
+            qa[e] = fmaf(ya, cs, -yb * sn) * scale;   // dim 8*mp + 2t + e
+            qb[e] = fmaf(yb, cs, ya * sn) * scale;    // dim 64 + 8*mp + 2t + e
+        }
+        uint16_t ha0, la0, ha1, la1, hb0, lb0, hb1, lb1;
+        split_bf16(qa[0], ha0, la0);
+        split_bf16(qa[1], ha1, la1);
+        split_bf16(qb[0], hb0, lb0);
+        split_bf16(qb[1], hb1, lb1);
+        const int part = (mp & 1) ? 2 : 0;   // dims 16s + 2t (+1) or 16s + 8 + 2t (+1)
+        st.qa[mp >> 1][part] = active ? ((uint32_t)ha1 << 16 | ha0) : 0u;
+        st.qa[mp >> 1][part + 1] = active ? ((uint32_t)la1 << 16 | la0) : 0u;
+        st.qa[4 + (mp >> 1)][part] = active ? ((uint32_t)hb1 << 16 | hb0) : 0u;
+        st.qa[4 + (mp >> 1)][part + 1] = active ? ((uint32_t)lb1 << 16 | lb0) : 0u;
+    }
+
+    if (appends) {
+        // lane l: dims 2l, 2l+1 (word l of the head) and 64+2l, 65+2l (word 32+l), all in double
+        double cs0, sn0, cs1, sn1;
+        sincos(ang0, &sn0, &cs0);
+        sincos(ang1, &sn1, &cs1);
+        const uint32_t* xk = reinterpret_cast<const uint32_t*>(s.qkv + (Lay::kHq + j) * (kHeadDim * 2));
+        const uint32_t* xv = reinterpret_cast<const uint32_t*>(s.qkv + (Lay::kHq + kNumKvHeads + j) * (kHeadDim * 2));
+        const uint32_t* gk = reinterpret_cast<const uint32_t*>(s.gains + kHeadDim);
+        const uint32_t xlo = xk[lane], xhi = xk[32 + lane];
+        const uint32_t wk_lo = gk[lane], wk_hi = gk[32 + lane];
+        double a0 = bf_to_d(xlo & 0xFFFFu), a1 = bf_to_d(xlo >> 16);
+        double b0 = bf_to_d(xhi & 0xFFFFu), b1 = bf_to_d(xhi >> 16);
+        const double r = sqrt(warp_sum(a0 * a0 + a1 * a1 + b0 * b0 + b1 * b1) / 128.0 + p.rms_eps);
+        a0 = a0 / r * bf_to_d(wk_lo & 0xFFFFu);
+        a1 = a1 / r * bf_to_d(wk_lo >> 16);
+        b0 = b0 / r * bf_to_d(wk_hi & 0xFFFFu);
+        b1 = b1 / r * bf_to_d(wk_hi >> 16);
+        const double ra0 = a0 * cs0 - b0 * sn0, rb0 = b0 * cs0 + a0 * sn0;
+        const double ra1 = a1 * cs1 - b1 * sn1, rb1 = b1 * cs1 + a1 * sn1;
+        st.k_lo = d_to_bf(ra0) | (d_to_bf(ra1) << 16);
+        st.k_hi = d_to_bf(rb0) | (d_to_bf(rb1) << 16);
+        st.v_lo = xv[lane];
+        st.v_hi = xv[32 + lane];
+    }
+
+#pragma unroll
+    for (int n = 0; n < 16; ++n)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) st.o[n][k] = 0.f;
+    st.m = -INFINITY;
+    st.lsum = 0.f;
+}
+
+// Scores, online softmax and value accumulation over one staged page.
+template <int G, bool kFullPage>
+__device__ __forceinline__ void attend_page(const uint8_t* stage, int ntok, int j, int lane, State& st) {
+    const int g = lane >> 2, t = lane & 3;
+    // K rows as the column-major B operand: matrix l/8 = (tokens 0-7 | 8-15) x (dims +0 | +8)
+    const uint32_t kaddr = smem_addr(stage + kStageK) + j * (kHeadDim * 2) +
+                           ((lane & 7) + ((lane >> 4) << 3)) * kRowPitch + ((lane >> 3) & 1) * 16;
+    float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kaddr + s * 32, b0, b1, b2, b3);
+        mma_bf16_16816(c0, st.qa[s], b0, b1);
+        mma_bf16_16816(c1, st.qa[s], b2, b3);
+    }
+    // head g's scores at tokens 2t, 2t+1, 8+2t, 9+2t (row g plus row g+8)
+    float sc[4] = {c0[0] + c0[2], c0[1] + c0[3], c1[0] + c1[2], c1[1] + c1[3]};
+    if (!kFullPage) {
+        sc[0] = (2 * t < ntok) ? sc[0] : -INFINITY;
+        sc[1] = (2 * t + 1 < ntok) ? sc[1] : -INFINITY;
+        sc[2] = (8 + 2 * t < ntok) ? sc[2] : -INFINITY;
+        sc[3] = (9 + 2 * t < ntok) ? sc[3] : -INFINITY;
+    }
+    float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+    const bool grow = mx > st.m + kRescaleThreshold;
+    if (__any_sync(kFull, grow)) {
+        const float nm = grow ? mx : st.m;
+        const float a = grow ? exp2_approx(st.m - nm) : 1.f;   // exp2(-inf) = 0 on the first page
+#pragma unroll
+        for (int n = 0; n < 16; ++n)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) st.o[n][k] *= a;
+        st.lsum *= a;
+        st.m = nm;
+    }
+    float pr[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pr[i] = (sc[i] == -INFINITY || g >= G) ? 0.f : exp2_approx(sc[i] - st.m);
+    st.lsum += (pr[0] + pr[1]) + (pr[2] + pr[3]);
+    uint32_t pa[4];
+    {
+        uint16_t h0, l0, h1, l1, h2, l2, h3, l3;
+        split_bf16(pr[0], h0, l0);
+        split_bf16(pr[1], h1, l1);
+        split_bf16(pr[2], h2, l2);
+        split_bf16(pr[3], h3, l3);
+        pa[0] = (uint32_t)h1 << 16 | h0;   // row g, tokens 2t, 2t+1
+        pa[1] = (uint32_t)l1 << 16 | l0;   // row g+8
+        pa[2] = (uint32_t)h3 << 16 | h2;   // row g, tokens 8+2t, 9+2t
+        pa[3] = (uint32_t)l3 << 16 | l2;   // row g+8
+    }
+    // V rows as the column-major B operand (transposed load): matrix l/8 =
+    // (tokens 0-7 | 8-15) x (dims +0 | +8)
+    const uint32_t vaddr = smem_addr(stage + kStageV) + j * (kHeadDim * 2) +
+                           ((lane & 7) + (((lane >> 3) & 1) << 3)) * kRowPitch + ((lane >> 4) & 1) * 16;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_trans(vaddr + u * 32, b0, b1, b2, b3);
+        mma_bf16_16816(st.o[2 * u], pa, b0, b1);
+        mma_bf16_16816(st.o[2 * u + 1], pa, b2, b3);
+    }
+}
+
+template <int G>
+__device__ __forceinline__ bool wait_full(const Params& p, const Shared& s, uint64_t* bar, uint32_t phase, int lane) {
+    bool ok = mbar_try_wait(bar, phase);
+    if (__all_sync(kFull, ok)) return true;
+    ok = ok || mbar_wait(bar, phase, p.timeout_ns, s.abort_flag);
+    ok = __all_sync(kFull, ok || mbar_try_wait(bar, phase));
+    if (!ok && lane == 0) {
+        *s.abort_flag = 1;
+        record_error(p.status, QDA_ERR_TIMEOUT);
+    }
+    return ok;
+}
+
+template <int G>
+__device__ __forceinline__ void consume_page(const Params& p, const Shared& s, int slot, int i, int nb, int L, int j,
+                                             int lane, State& st) {
+    uint8_t* stage = s.stages + slot * kStageBytes;
+    const bool last = (i == nb - 1);
+    const int new_row = (L - 1) - kPage * i;
+    const int ntok = last ? new_row + 1 : kPage;
+    if (s.meta[slot].bad == 0) {
+        if (last) {
+            // the new token: written to the cache and patched into the staged page
+            const int page = s.meta[slot].page;
+            const size_t off =
+                (size_t)page * (kPageBytes / 2) + (size_t)new_row * (kRowBytes / 2) + (size_t)j * kHeadDim;
+            uint32_t* kd = reinterpret_cast<uint32_t*>(p.k_cache + off);
+            uint32_t* vd = reinterpret_cast<uint32_t*>(p.v_cache + off);
+            kd[lane] = st.k_lo;
+            kd[32 + lane] = st.k_hi;
+            vd[lane] = st.v_lo;
+            vd[32 + lane] = st.v_hi;
+            uint32_t* kr = reinterpret_cast<uint32_t*>(stage + kStageK + new_row * kRowPitch + j * kHeadDim * 2);
+            uint32_t* vr = reinterpret_cast<uint32_t*>(stage + kStageV + new_row * kRowPitch + j * kHeadDim * 2);
+            kr[lane] = st.k_lo;
+            kr[32 + lane] = st.k_hi;
+            vr[lane] = st.v_lo;
+            vr[32 + lane] = st.v_hi;
+            // the rows after the new token hold stale bytes; the value product
+            // would turn a stale NaN into NaN even at probability 0, so clear them
+            for (int r = ntok; r < kPage; ++r) {
+                uint32_t* z = reinterpret_cast<uint32_t*>(stage + kStageV + r * kRowPitch + j * kHeadDim * 2);
+                z[lane] = 0u;
+                z[32 + lane] = 0u;
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+        }
+        if (ntok == kPage) attend_page<G, true>(stage, ntok, j, lane, st);
+        else attend_page<G, false>(stage, ntok, j, lane, st);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.empty_bar[slot]);
+}
+
+// End of a sequence piece: o directly when the piece is the whole sequence,
+// else this piece's partial at scratch slot blockIdx.x + b.
+template <int G>
+__device__ __forceinline__ void finish_piece(const Params& p, const Shared& s, int b, int j, int lane, int per_cta,
+                                             State& st) {
+    using Lay = Layout<G>;
+    const int g = lane >> 2, t = lane & 3;
+    float l = st.lsum;
+    l += __shfl_xor_sync(kFull, l, 1);
+    l += __shfl_xor_sync(kFull, l, 2);
+    if (g >= G) return;
+    const int head = G * j + g;
+    const int part_first = s.seg[b] / per_cta;
+    const int part_last = (s.seg[b + 1] - 1) / per_cta;
+    if (part_first == part_last) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        uint32_t* dst = reinterpret_cast<uint32_t*>(p.o + ((size_t)b * Lay::kHq + head) * kHeadDim);
+#pragma unroll
+        for (int n = 0; n < 16; ++n)
+            dst[4 * n + t] = pack_bf2((st.o[n][0] + st.o[n][2]) * inv, (st.o[n][1] + st.o[n][3]) * inv);
+        return;
+    }
+    const int slot = blockIdx.x + b;
+    float2* pa = reinterpret_cast<float2*>(p.part_acc + ((size_t)slot * Lay::kHq + head) * kHeadDim);
+#pragma unroll
+    for (int n = 0; n < 16; ++n) __stcg(pa + 4 * n + t, make_float2(st.o[n][0] + st.o[n][2], st.o[n][1] + st.o[n][3]));
+    if (t == 0) __stcg(p.part_ml + (size_t)slot * Lay::kHq + head, make_float2(st.m, l));
+}
+
+template <int G>
+__device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, int B, int start, int end, int per_cta,
+                                             int warp, int lane) {
+    const int j = warp;
+    State st;
+    st.k_lo = st.k_hi = st.v_lo = st.v_hi = 0u;
+    int b = find_seq(s.seg, B, start);
+    int i0 = start - s.seg[b];
+    int slot = 0;
+    uint32_t phase = 0, qphase = 0;
+    const int count = end - start;
+    int k = 0;
+    while (k < count) {
+        const int nb = s.seg[b + 1] - s.seg[b];
+        const int L = s.lens[b];
+        const int n_here = min(nb - i0, count - k);
+        if (!wait_full<G>(p, s, s.qkv_full, qphase, lane)) return;
+        begin_sequence<G>(p, s, *s.qkv_pos, j, lane, /*appends=*/s.seg[b + 1] <= end, st);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s.qkv_empty);
+        qphase ^= 1u;
+        for (int u = 0; u < n_here; ++u) {
+            if (!wait_full<G>(p, s, &s.full_bar[slot], phase, lane)) return;
+            consume_page<G>(p, s, slot, i0 + u, nb, L, j, lane, st);
+            if (++slot == kStages) {
+                slot = 0;
+                phase ^= 1u;
+            }
+        }
+        k += n_here;
+        finish_piece<G>(p, s, b, j, lane, per_cta, st);
+        if (k < count) {
+            do { ++b; } while (b < B && s.seg[b + 1] == s.seg[b]);
+            i0 = 0;
+        }
+    }
+}
+
+template <int G>
+__global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Params p) {
+    using Lay = Layout<G>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    Shared s;
+    s.stages = smem;
+    s.qkv = smem + Lay::kSmemQkv;
+    s.seg = reinterpret_cast<int*>(smem + Lay::kSmemSeg);
+    s.lens = reinterpret_cast<int*>(smem + Lay::kSmemLens);
+    s.inv_freq = reinterpret_cast<double*>(smem + Lay::kSmemInvFreq);
+    s.gains = reinterpret_cast<const uint16_t*>(smem + Lay::kSmemGains);
+    s.meta = reinterpret_cast<volatile StageMeta*>(smem + Lay::kSmemMeta);
+    s.qkv_pos = reinterpret_cast<volatile int*>(smem + Lay::kSmemMeta + kStages * 16);
+    s.full_bar = reinterpret_cast<uint64_t*>(smem + Lay::kSmemBars);
+    s.empty_bar = s.full_bar + kStages;
+    s.qkv_full = s.empty_bar + kStages;
+    s.qkv_empty = s.qkv_full + 1;
+    s.never_bar = s.qkv_empty + 1;
+    s.abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kSmemFlags);
+
+    const int B = p.batch;
+    for (int b = threadIdx.x; b < B; b += kThreads) {
+        const int L = p.seq_lens[b];
+        const bool ok = L >= 1 && L <= p.max_seq_len && L <= kPage * p.bt_stride;
+        if (!ok && blockIdx.x == 0) record_error(p.status, QDA_ERR_BOUNDS);
+        s.lens[b] = L;
+        s.seg[b + 1] = ok ? (L + kPage - 1) / kPage : 0;
+    }
+    if (threadIdx.x < 64) {
+        const uint16_t* src = threadIdx.x < 32 ? p.q_norm_w : p.k_norm_w;
+        reinterpret_cast<uint2*>(smem + Lay::kSmemGains)[threadIdx.x] =
+            *reinterpret_cast<const uint2*>(src + 4 * (threadIdx.x & 31));
+    } else if (threadIdx.x < 128) {
+        const int i = threadIdx.x - 64;
+        s.inv_freq[i] = pow(p.rope_theta, -2.0 * i / 128.0);
+    }
+    if (threadIdx.x == 0) {
+        for (int k = 0; k < kStages; ++k) {
+            mbar_init(&s.full_bar[k], 1);
+            mbar_init(&s.empty_bar[k], kConsumerWarps);
+        }
+        mbar_init(s.qkv_full, 1);
+        mbar_init(s.qkv_empty, kConsumerWarps);
+        mbar_init(s.never_bar, 1);
+        *s.abort_flag = 0;
+        s.seg[0] = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (warp == 0) {  // inclusive scan of the page counts
+        int v[8];
+        int run = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int idx = 1 + 8 * lane + k;
+            run += (idx <= B) ? s.seg[idx] : 0;
+            v[k] = run;
+        }
+        int incl = run;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int t = __shfl_up_sync(kFull, incl, off);
+            if (lane >= off) incl += t;
+        }
+        const int excl = incl - run;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int idx = 1 + 8 * lane + k;
+            if (idx <= B) s.seg[idx] = excl + v[k];
+        }
+    }
+    __syncthreads();
+    if (blockIdx.x == 0)   // page offsets for the combine launch
+        for (int b = threadIdx.x; b <= B; b += kThreads) p.seg[b] = s.seg[b];
+
+    const int total = s.seg[B];
+    const int per_cta = (total + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int start = (int)blockIdx.x * per_cta;
+    const int end = min(start + per_cta, total);
+    if (start < end) {
+        if (warp == kConsumerWarps) run_producer<G>(p, s, B, start, end, lane);
+        else run_consumer<G>(p, s, B, start, end, per_cta, warp, lane);
+    }
+    if ((p.flags & QDA_FLAG_INJECT_WAIT_TIMEOUT) != 0u && blockIdx.x == 0 && warp == 0) {
+        if (!mbar_wait(s.never_bar, 0u, p.timeout_ns, nullptr) && lane == 0) record_error(p.status, QDA_ERR_TIMEOUT);
+    }
+    pdl_launch_dependents();
+}
+
+// Combine the partials of one split sequence (blockIdx.x) for one query head
+// (blockIdx.y): o = sum_t 2^(m_t - M) acc_t / sum_t 2^(m_t - M) l_t, M = max_t m_t.
+// Thread d handles dim d. Sequences held whole by one CTA were written by the
+// first launch and are skipped.
+template <int G>
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const Params p, int main_grid) {
+    using Lay = Layout<G>;
+    __shared__ float w[kMaxGridCtas + 1];
+    __shared__ float red[kCombineThreads / 32];
+    pdl_wait();   // the first launch has finished and its writes are visible
+    const int b = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
+    const int lo = p.seg[b], hi = p.seg[b + 1], total = p.seg[p.batch];
+    if (hi == lo) return;   // a sequence the first launch skipped
+    const int per_cta = (total + main_grid - 1) / main_grid;
+    const int first = lo / per_cta, n = (hi - 1) / per_cta - first + 1;
+    if (n == 1) return;
+    // the pieces' maxima and sums
+    float mx = -INFINITY;
+    for (int t = d; t < n; t += kCombineThreads) {
+        const float2 ml = __ldcg(p.part_ml + (size_t)(first + t + b) * Lay::kHq + h);
+        w[t] = ml.x;
+        mx = fmaxf(mx, ml.x);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
+    if ((d & 31) == 0) red[d >> 5] = mx;
+    __syncthreads();
+    float M = red[0];
+#pragma unroll
+    for (int k = 1; k < kCombineThreads / 32; ++k) M = fmaxf(M, red[k]);
+    __syncthreads();
+    float ls = 0.f;
+    for (int t = d; t < n; t += kCombineThreads) {
+        const float m = w[t];
+        const float wt = (m == -INFINITY) ? 0.f : exp2_approx(m - M);   // a piece whose pages were all skipped
+        w[t] = wt;
+        ls += wt * __ldcg(p.part_ml + (size_t)(first + t + b) * Lay::kHq + h).y;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ls += __shfl_xor_sync(kFull, ls, off);
+    if ((d & 31) == 0) red[d >> 5] = ls;
+    __syncthreads();
+    float L = 0.f;
+#pragma unroll
+    for (int k = 0; k < kCombineThreads / 32; ++k) L += red[k];
+    float acc = 0.f;
+    const float* src = p.part_acc + ((size_t)(first + b) * Lay::kHq + h) * kHeadDim + d;
+    constexpr size_t kSlotStride = (size_t)Lay::kHq * kHeadDim;
+    int t = 0;
+    for (; t + 8 <= n; t += 8) {
+        float x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] = __ldcg(src + (size_t)(t + u) * kSlotStride);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc = fmaf(w[t + u], x[u], acc);
+    }
+    for (; t < n; ++t) acc = fmaf(w[t], __ldcg(src + (size_t)t * kSlotStride), acc);
+    p.o[((size_t)b * Lay::kHq + h) * kHeadDim + d] = __bfloat16_as_ushort(__float2bfloat16_rn(L > 0.f ? acc / L : 0.f));
+}
+
+template <int G>
+cudaError_t prepare_one() {
+    return cudaFuncSetAttribute(grouped_attention_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Layout<G>::kSmemTotal);
+}
+
+template <int G>
+cudaError_t launch_one(const Params& p, int grid, cudaStream_t stream) {
+    grouped_attention_kernel<G><<<grid, kThreads, Layout<G>::kSmemTotal, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.batch, (unsigned)Layout<G>::kHq, 1);
+    cfg.blockDim = dim3(kCombineThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, combine_kernel<G>, p, grid);
+}
+
+}  // namespace
+
+cudaError_t prepare_grouped() {
+    cudaError_t e = prepare_one<4>();
+    if (e == cudaSuccess) e = prepare_one<5>();
+    if (e == cudaSuccess) e = prepare_one<8>();
+    return e;
+}
+
+cudaError_t launch_grouped(const Params& p, int grid, cudaStream_t stream) {
+    switch (p.num_q_heads) {
+        case 32: return launch_one<4>(p, grid, stream);
+        case 40: return launch_one<5>(p, grid, stream);
+        case 64: return launch_one<8>(p, grid, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace qda

@@ -8,6 +8,9 @@
 namespace qda {
 
 // Geometry of Qwen3-0.6B attention (Model Spec, "Published configuration").
+// The larger Qwen3 sizes keep 8 kv heads of 128 and have 32, 40 or 64 query
+// heads (nnterp qwen3, "Grouped-query attention, with 128-wide heads on every
+// size"); kNumQHeads and kGroup are the 0.6B values.
 constexpr int kNumQHeads = 16;
 constexpr int kNumKvHeads = 8;
 constexpr int kGroup = kNumQHeads / kNumKvHeads;   // query heads per kv head
@@ -25,7 +28,7 @@ constexpr int kPageBytes = kPage * kRowBytes;
 
 // Everything one launch needs. Pointers are device pointers.
 struct Params {
-    const uint16_t* qkv;          // bf16 [B][4096]
+    const uint16_t* qkv;          // bf16 [B][(num_q_heads + 16) * 128]
     const uint16_t* q_norm_w;     // bf16 [128]
     const uint16_t* k_norm_w;     // bf16 [128]
     const int32_t* seq_lens;      // [B]
@@ -33,7 +36,8 @@ struct Params {
     const int32_t* block_table;   // [B][bt_stride]
     uint16_t* k_cache;            // bf16 [num_pages][16][8][128]
     uint16_t* v_cache;
-    uint16_t* o;                  // bf16 [B][16][128]
+    uint16_t* o;                  // bf16 [B][num_q_heads][128]
+    int num_q_heads;              // 16, 32, 40 or 64
     int bt_stride;
     int num_pages;
     int batch;
@@ -41,8 +45,10 @@ struct Params {
     double rope_theta;
     double rms_eps;
     // workspace
-    float* part_acc;              // [num_slots][16][128] un-normalised partial sums
-    float2* part_ml;              // [num_slots][16] (running max in log2 units, sum)
+    float* part_acc;              // [num_slots][num_q_heads][128] un-normalised partial sums
+    float2* part_ml;              // [num_slots][num_q_heads] (running max in log2 units, sum)
+    int* seg;                     // [kMaxBatch + 1] page offsets of the sequences (written for the combine
+                                  // launch of the 32/40/64-head kernels; unused at 16 heads)
     int* counters;                // [kMaxBatch][8] merge arrival counters, zero between calls
     int* status;                  // sticky device error (0 = none)
     int64_t timeout_ns;           // limit of every device-side wait
@@ -59,7 +65,14 @@ size_t smem_bytes();
 // shared-memory limit). Returns the first CUDA error.
 cudaError_t prepare_device();
 
-// Launch one decode-attention step with `grid` CTAs on `stream`.
+// Launch one decode-attention step with `grid` CTAs on `stream` (16 query heads).
 cudaError_t launch(const Params& p, int grid, cudaStream_t stream);
+
+// The step at 32, 40 or 64 query heads: the attention launch, then a launch
+// that combines the partials of sequences split across CTAs.
+cudaError_t launch_grouped(const Params& p, int grid, cudaStream_t stream);
+
+// Prepare the 32/40/64-head kernels on the current device.
+cudaError_t prepare_grouped();
 
 }  // namespace qda

@@ -105,6 +105,7 @@ extern "C" int qwen3_decode_attn_append_and_attend_noalloc(const void* qkv, cons
     p.k_cache = static_cast<uint16_t*>(k_cache);
     p.v_cache = static_cast<uint16_t*>(v_cache);
     p.o = static_cast<uint16_t*>(o);
+    p.num_q_heads = qda::kNumQHeads;
     p.bt_stride = block_table_stride;
     p.num_pages = num_pages;
     p.batch = batch;
@@ -114,6 +115,7 @@ extern "C" int qwen3_decode_attn_append_and_attend_noalloc(const void* qkv, cons
     p.part_acc = reinterpret_cast<float*>(s.scratch);
     p.part_ml = reinterpret_cast<float2*>(s.scratch + kOffPartMl);
     p.counters = reinterpret_cast<int*>(s.scratch + kOffCounters);
+    p.seg = nullptr;
     p.status = reinterpret_cast<int*>(s.scratch + kOffStatus);
     p.timeout_ns = kTimeoutNs;
     p.flags = 0u;

@@ -23,10 +23,16 @@
  *                 covers": one new query per sequence over seq_lens[b] cached
  *                 positions; nnterp qwen3, "Grouped-query attention").
  *
+ * The larger Qwen3 sizes have the same attention with 32 (4B, 8B), 40 (14B)
+ * or 64 (32B) query heads over the same 8 kv heads of 128 (nnterp qwen3,
+ * "Grouped-query attention, with 128-wide heads on every size"); a handle
+ * created with num_q_heads = Hq serves that size, and query head h then reads
+ * kv head h / (Hq / 8). Below, Hq = 16 for Qwen3-0.6B.
+ *
  * Tensor layouts (all little-endian, row-major, no padding):
  *
- *   qkv          bf16 [B][4096]: 16 q heads x 128 | 8 k heads x 128 |
- *                8 v heads x 128, the attn.qkv_proj output row (N = 4096).
+ *   qkv          bf16 [B][(Hq + 16) * 128]: Hq q heads x 128 | 8 k heads x 128 |
+ *                8 v heads x 128, the attn.qkv_proj output row (N = 4096 at Hq = 16).
  *   q_norm_w     bf16 [128]; k_norm_w bf16 [128].
  *   seq_lens     int32 [B]. Counts the new token: 1 <= seq_lens[b] <= the
  *                handle's max_seq_len (<= 40960) and <= 16 * block_table_stride.
@@ -37,7 +43,7 @@
  *                ceil(seq_lens[b]/16) are never read.
  *   k_cache,     bf16 [num_pages][16][8][128] each: page, token row, kv head,
  *   v_cache      dim. One page of one cache is 32 KiB, contiguous.
- *   o            bf16 [B][16][128].
+ *   o            bf16 [B][Hq][128].
  *
  * Numbers: the new k is normed and rotated in double precision and rounded
  * once to bf16 (nearest-even) when stored; q is normed and rotated in float,
@@ -74,9 +80,10 @@
 extern "C" {
 #endif
 
-/* Geometry compiled into the kernels (Model Spec, "Published configuration":
+/* Geometry of Qwen3-0.6B (Model Spec, "Published configuration":
  * num_attention_heads 16, num_key_value_heads 8, head_dim 128; "At a glance":
- * page size 16, B <= 256, S <= 40960; attn.qkv_proj N = 4096). */
+ * page size 16, B <= 256, S <= 40960; attn.qkv_proj N = 4096). The kernels are
+ * also compiled for 32, 40 and 64 query heads over the same 8 kv heads. */
 #define QDA_NUM_Q_HEADS   16
 #define QDA_NUM_KV_HEADS  8
 #define QDA_HEAD_DIM      128
@@ -103,7 +110,7 @@ extern "C" {
 typedef struct qda_handle qda_handle; /* opaque */
 
 typedef struct {
-    int num_q_heads;        /* must be 16 */
+    int num_q_heads;        /* 16 (Qwen3-0.6B, 1.7B), 32 (4B, 8B), 40 (14B) or 64 (32B) */
     int num_kv_heads;       /* must be 8 */
     int head_dim;           /* must be 128 */
     int page_size;          /* must be 16 */
@@ -129,12 +136,15 @@ void qwen3_decode_attn_default_config(qda_config *cfg);
  * call). Allocates the workspace on that device. On success *out receives the
  * handle; on failure *out is set to NULL.
  * Errors: INVALID_ARG (null pointer, a size outside its range),
- *         UNSUPPORTED (head counts, head_dim or page_size not 16/8/128/16),
+ *         UNSUPPORTED (query heads not 16/32/40/64, or kv heads, head_dim or
+ *         page_size not 8/128/16),
  *         CUDA (no such device, allocation failure). */
 int qwen3_decode_attn_create(const qda_config *cfg, int device, qda_handle **out);
 
-/* The decode-attention step on device buffers (layouts above). Every pointer
- * is a device pointer. qkv, k_cache, v_cache and o must be 16-byte aligned;
+/* The decode-attention step on device buffers (layouts above, with the
+ * handle's Hq). At 16 query heads it is one kernel launch; at 32, 40 or 64 a
+ * second launch combines sequences split across CTAs. Every pointer is a
+ * device pointer. qkv, k_cache, v_cache and o must be 16-byte aligned;
  * q_norm_w, k_norm_w, seq_lens, positions and block_table 4-byte aligned.
  * `batch` is B (1..max_batch); `num_pages` (>= 1) bounds every block-table
  * entry the call reads; `block_table_stride` (>= 1) is the row pitch in

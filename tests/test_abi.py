@@ -83,7 +83,9 @@ def test_strerror_covers_every_code(lib):
 def test_create_rejects_bad_configs_on_the_host(lib):
     from decode_attention_qk_b200 import binding
     h = ctypes.c_void_p(1234)
-    cases = [({"num_q_heads": 32}, binding.QDA_ERR_UNSUPPORTED),
+    cases = [({"num_q_heads": 24}, binding.QDA_ERR_UNSUPPORTED),
+             ({"num_q_heads": 128}, binding.QDA_ERR_UNSUPPORTED),
+             ({"num_kv_heads": 4}, binding.QDA_ERR_UNSUPPORTED),
              ({"head_dim": 64}, binding.QDA_ERR_UNSUPPORTED),
              ({"page_size": 32}, binding.QDA_ERR_UNSUPPORTED),
              ({"max_batch": 0}, binding.QDA_ERR_INVALID_ARG),
