@@ -40,8 +40,11 @@ FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
 L2_BYTES = 126 * 2 ** 20
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = [os.path.join(ROOT, "decode_attention_qk_b200", "csrc", f)
-                  for f in ("qda_decode_kernel.cu", "qda_internal.h")]
+_CSRC = os.path.join(ROOT, "decode_attention_qk_b200", "csrc")
+KERNEL_SOURCES = {   # the files each attention kernel is built from
+    16: [os.path.join(_CSRC, f) for f in ("qda_decode_kernel.cu", "qda_device.cuh", "qda_internal.h")],
+    "grouped": [os.path.join(_CSRC, f) for f in ("qda_decode_mma.cu", "qda_device.cuh", "qda_internal.h")],
+}
 
 WORKLOADS = {
     "cfg1": "B=2, seq_lens={7,12} incl. new token, 4 pages, random block table",
@@ -99,16 +102,16 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(num_q_heads: int = 16) -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in KERNEL_SOURCES[16 if num_q_heads == 16 else "grouped"]:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
 
-def traffic_per_launch(workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+def traffic_per_launch(workload: str, num_q_heads: int = 16):
+    """DRAM bytes per call from the committed ncu summary, if it was taken on
     this kernel source and workload (else None)."""
     try:
         with open(TRAFFIC_FILE) as f:
@@ -116,7 +119,7 @@ def traffic_per_launch(workload: str):
     except (OSError, ValueError):
         return None
     entry = t.get(workload)
-    if not entry or entry.get("kernel_source_sha256") != kernel_source_hash():
+    if not entry or entry.get("kernel_source_sha256") != kernel_source_hash(num_q_heads):
         return None
     return entry.get("dram_bytes_per_launch")
 
@@ -392,7 +395,7 @@ def run_gpu(args):
     peak, peak_kind = hbm_peak()
     achieved = alg_per_launch / (mean_kernel_ms * 1e-3) / 1e9
     workload_key = args.workload if args.num_q_heads == 16 else f"{args.workload}-h{args.num_q_heads}"
-    traffic = traffic_per_launch(workload_key)
+    traffic = traffic_per_launch(workload_key, args.num_q_heads)
 
     # end to end through the host-buffer entry point: per step the H2D copy of the
     # step's inputs from pinned memory, the call, and the D2H copy of o

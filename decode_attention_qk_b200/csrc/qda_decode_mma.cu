@@ -27,7 +27,7 @@
 // Split sequences. The work split is the 16-head kernel's (equal page ranges
 // per CTA, scratch slot g + b per piece). A piece that covers its whole
 // sequence writes o; a piece of a split sequence writes its partial, and a
-// second launch (one CTA per sequence and query head, one thread per dim)
+// second launch (one CTA per sequence and kv head, one warp per query head)
 // combines them with the log-sum-exp rule (Supported models, "Facts proved
 // about the specs": flashAttn_eq, softmax_shift), spreading long merges over
 // many SMs. That launch uses programmatic dependent launch so its start
@@ -49,7 +49,6 @@ constexpr int kRowPitch = kRowBytes + 16;           // staged token-row pitch: 2
 constexpr int kStageK = 0;
 constexpr int kStageV = kPage * kRowPitch;
 constexpr int kStageBytes = 2 * kPage * kRowPitch;  // 66048
-constexpr int kCombineThreads = kHeadDim;           // combine launch: one thread per dim
 
 template <int G>
 struct Layout {
@@ -567,64 +566,63 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
     pdl_launch_dependents();
 }
 
-// Combine the partials of one split sequence (blockIdx.x) for one query head
-// (blockIdx.y): o = sum_t 2^(m_t - M) acc_t / sum_t 2^(m_t - M) l_t, M = max_t m_t.
-// Thread d handles dim d. Sequences held whole by one CTA were written by the
-// first launch and are skipped.
+// Combine the partials of one split sequence (blockIdx.x) for the G query
+// heads of one kv head (blockIdx.y): warp g handles head G*y + g and lane l
+// its dims 4l..4l+3; o = sum_t 2^(m_t - M) acc_t / sum_t 2^(m_t - M) l_t with
+// M = max_t m_t. Sequences held whole by one CTA were written by the first
+// launch and are skipped.
 template <int G>
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const Params p, int main_grid) {
+__global__ void __launch_bounds__(32 * G) combine_kernel(const Params p, int main_grid) {
     using Lay = Layout<G>;
-    __shared__ float w[kMaxGridCtas + 1];
-    __shared__ float red[kCombineThreads / 32];
     pdl_wait();   // the first launch has finished and its writes are visible
-    const int b = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
+    const int b = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = G * blockIdx.y + warp;
     const int lo = p.seg[b], hi = p.seg[b + 1], total = p.seg[p.batch];
     if (hi == lo) return;   // a sequence the first launch skipped
     const int per_cta = (total + main_grid - 1) / main_grid;
     const int first = lo / per_cta, n = (hi - 1) / per_cta - first + 1;
     if (n == 1) return;
-    // the pieces' maxima and sums
-    float mx = -INFINITY;
-    for (int t = d; t < n; t += kCombineThreads) {
-        const float2 ml = __ldcg(p.part_ml + (size_t)(first + t + b) * Lay::kHq + h);
-        w[t] = ml.x;
-        mx = fmaxf(mx, ml.x);
+    const float2* ml = p.part_ml + (size_t)(first + b) * Lay::kHq + h;   // piece t at ml[t * kHq]
+    float M = -INFINITY;
+    for (int t = lane; t < n; t += 32) M = fmaxf(M, __ldcg(ml + (size_t)t * Lay::kHq).x);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+    const float4* src = reinterpret_cast<const float4*>(p.part_acc + ((size_t)(first + b) * Lay::kHq + h) * kHeadDim) + lane;
+    constexpr size_t kSlotStride = (size_t)Lay::kHq * kHeadDim / 4;   // float4 per scratch slot
+    float Ls = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int t0 = 0; t0 < n; t0 += 32) {
+        float wt = 0.f;
+        if (t0 + lane < n) {
+            const float2 v = __ldcg(ml + (size_t)(t0 + lane) * Lay::kHq);
+            wt = (v.x == -INFINITY) ? 0.f : exp2_approx(v.x - M);   // a piece whose pages were all skipped
+            Ls = fmaf(wt, v.y, Ls);
+        }
+        const int m = min(32, n - t0);
+        for (int u0 = 0; u0 < m; u0 += 8) {
+            float4 x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (u0 + u < m) x[u] = __ldcg(src + (size_t)(t0 + u0 + u) * kSlotStride);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float w = __shfl_sync(kFull, wt, (u0 + u) & 31);
+                if (u0 + u < m) {
+                    acc.x = fmaf(w, x[u].x, acc.x);
+                    acc.y = fmaf(w, x[u].y, acc.y);
+                    acc.z = fmaf(w, x[u].z, acc.z);
+                    acc.w = fmaf(w, x[u].w, acc.w);
+                }
+            }
+        }
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
-    if ((d & 31) == 0) red[d >> 5] = mx;
-    __syncthreads();
-    float M = red[0];
-#pragma unroll
-    for (int k = 1; k < kCombineThreads / 32; ++k) M = fmaxf(M, red[k]);
-    __syncthreads();
-    float ls = 0.f;
-    for (int t = d; t < n; t += kCombineThreads) {
-        const float m = w[t];
-        const float wt = (m == -INFINITY) ? 0.f : exp2_approx(m - M);   // a piece whose pages were all skipped
-        w[t] = wt;
-        ls += wt * __ldcg(p.part_ml + (size_t)(first + t + b) * Lay::kHq + h).y;
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) ls += __shfl_xor_sync(kFull, ls, off);
-    if ((d & 31) == 0) red[d >> 5] = ls;
-    __syncthreads();
-    float L = 0.f;
-#pragma unroll
-    for (int k = 0; k < kCombineThreads / 32; ++k) L += red[k];
-    float acc = 0.f;
-    const float* src = p.part_acc + ((size_t)(first + b) * Lay::kHq + h) * kHeadDim + d;
-    constexpr size_t kSlotStride = (size_t)Lay::kHq * kHeadDim;
-    int t = 0;
-    for (; t + 8 <= n; t += 8) {
-        float x[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) x[u] = __ldcg(src + (size_t)(t + u) * kSlotStride);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) acc = fmaf(w[t + u], x[u], acc);
-    }
-    for (; t < n; ++t) acc = fmaf(w[t], __ldcg(src + (size_t)t * kSlotStride), acc);
-    p.o[((size_t)b * Lay::kHq + h) * kHeadDim + d] = __bfloat16_as_ushort(__float2bfloat16_rn(L > 0.f ? acc / L : 0.f));
+    for (int off = 16; off > 0; off >>= 1) Ls += __shfl_xor_sync(kFull, Ls, off);
+    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+    uint2 out;
+    out.x = pack_bf2(acc.x * inv, acc.y * inv);
+    out.y = pack_bf2(acc.z * inv, acc.w * inv);
+    reinterpret_cast<uint2*>(p.o + ((size_t)b * Lay::kHq + h) * kHeadDim)[lane] = out;
 }
 
 template <int G>
@@ -639,8 +637,8 @@ cudaError_t launch_one(const Params& p, int grid, cudaStream_t stream) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)p.batch, (unsigned)Layout<G>::kHq, 1);
-    cfg.blockDim = dim3(kCombineThreads, 1, 1);
+    cfg.gridDim = dim3((unsigned)p.batch, (unsigned)kNumKvHeads, 1);
+    cfg.blockDim = dim3(32 * G, 1, 1);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
