@@ -45,7 +45,7 @@ class Workload:
     seq_lens: torch.Tensor          # int32 [B], CPU; counts the new token
     block_table: torch.Tensor       # int32 [B, stride], CPU; -1 where unused
     num_pages: int
-    qkv: torch.Tensor               # bf16 [B, (Hq + 16) * 128] on `device`
+    qkv: torch.Tensor               # bf16 [B, (Hq + 16) * 128], or [B, T, ...] for T new tokens, on `device`
     q_norm_w: torch.Tensor          # bf16 [128] on `device`
     k_norm_w: torch.Tensor          # bf16 [128] on `device`
     k_cache: torch.Tensor           # bf16 [num_pages, 16, 8, 128] on `device`
@@ -62,7 +62,11 @@ class Workload:
 
     @property
     def num_q_heads(self) -> int:
-        return int(self.qkv.shape[1]) // HEAD_DIM - 2 * NUM_KV_HEADS
+        return int(self.qkv.shape[-1]) // HEAD_DIM - 2 * NUM_KV_HEADS
+
+    @property
+    def new_tokens(self) -> int:
+        return 1 if self.qkv.dim() == 2 else int(self.qkv.shape[1])
 
 
 def pages_for(seq_lens: torch.Tensor) -> torch.Tensor:
@@ -109,9 +113,11 @@ def qkv_width(num_q_heads: int) -> int:
     return (num_q_heads + 2 * NUM_KV_HEADS) * HEAD_DIM
 
 
-def _values(B: int, num_pages: int, seed: int, device, num_q_heads: int = NUM_Q_HEADS) -> dict:
+def _values(B: int, num_pages: int, seed: int, device, num_q_heads: int = NUM_Q_HEADS,
+            new_tokens: int = 1) -> dict:
     dev = torch.device(device)
-    qkv = torch.randn((B, qkv_width(num_q_heads)), generator=_gen(seed * 16 + 1, dev), device=dev,
+    shape = (B, qkv_width(num_q_heads)) if new_tokens == 1 else (B, new_tokens, qkv_width(num_q_heads))
+    qkv = torch.randn(shape, generator=_gen(seed * 16 + 1, dev), device=dev,
                       dtype=torch.float32).to(torch.bfloat16)
     gq = torch.rand(HEAD_DIM, generator=_gen(seed * 16 + 2, dev), device=dev, dtype=torch.float32)
     gk = torch.rand(HEAD_DIM, generator=_gen(seed * 16 + 3, dev), device=dev, dtype=torch.float32)
@@ -124,14 +130,15 @@ def _values(B: int, num_pages: int, seed: int, device, num_q_heads: int = NUM_Q_
 
 def custom(seq_lens, seed: int = 0, device="cpu", pool_pages: int | None = None,
            stride: int | None = None, gap_fraction: float = 0.0, positions=None,
-           name: str = "custom", num_q_heads: int = NUM_Q_HEADS) -> Workload:
-    """A workload with the given sequence lengths and the standard value recipe."""
+           name: str = "custom", num_q_heads: int = NUM_Q_HEADS, new_tokens: int = 1) -> Workload:
+    """A workload with the given sequence lengths (counting the new tokens) and the
+    standard value recipe; with new_tokens = T > 1, qkv is [B, T, width]."""
     seq_lens = torch.as_tensor(seq_lens, dtype=torch.int32).reshape(-1)
     need = int(pages_for(seq_lens).sum())
     if pool_pages is None:
         pool_pages = need + (int(math.ceil(gap_fraction * need)) if gap_fraction > 0 else 0)
     bt = assign_pages(seq_lens, pool_pages, seed, stride=stride, gap_fraction=gap_fraction)
-    vals = _values(seq_lens.numel(), pool_pages, seed, device, num_q_heads)
+    vals = _values(seq_lens.numel(), pool_pages, seed, device, num_q_heads, new_tokens)
     pos = None if positions is None else torch.as_tensor(positions, dtype=torch.int32).reshape(-1)
     return Workload(name=name, seq_lens=seq_lens, block_table=bt, num_pages=pool_pages,
                     positions=pos, **vals)
@@ -152,12 +159,13 @@ def config1(device="cpu") -> Workload:
                     block_table=bt, num_pages=4, **vals)
 
 
-def config2(device="cpu", seed: int = 2000, num_q_heads: int = NUM_Q_HEADS) -> Workload:
-    """B=32, seq_lens ~ U{1..4096}, pool of 32*256 shuffled pages."""
+def config2(device="cpu", seed: int = 2000, num_q_heads: int = NUM_Q_HEADS, new_tokens: int = 1) -> Workload:
+    """B=32, seq_lens ~ U{1..4096} (at least new_tokens), pool of 32*256 shuffled pages."""
     seq_lens = torch.randint(1, 4097, (32,), generator=_gen(seed, "cpu"), dtype=torch.int64).to(torch.int32)
+    seq_lens = seq_lens.clamp(min=new_tokens)
     pool = 32 * 256
     bt = assign_pages(seq_lens, pool, seed + 1, stride=256)
-    vals = _values(32, pool, seed, device, num_q_heads)
+    vals = _values(32, pool, seed, device, num_q_heads, new_tokens)
     return Workload(name="cfg2: B=32, seq_lens~U[1,4096], page 16, shuffled pool of 8192 pages",
                     seq_lens=seq_lens, block_table=bt, num_pages=pool, **vals)
 
@@ -176,12 +184,12 @@ def config3_layer(layer: int, device="cpu", seed: int = 3000) -> Workload:
 CONFIG3_LAYERS = 28
 
 
-def config4(device="cpu", seed: int = 4000, num_q_heads: int = NUM_Q_HEADS) -> Workload:
+def config4(device="cpu", seed: int = 4000, num_q_heads: int = NUM_Q_HEADS, new_tokens: int = 1) -> Workload:
     """B=4, seq_len 40960 (the maximum context), 10240 shuffled pages."""
     seq_lens = torch.full((4,), MAX_SEQ, dtype=torch.int32)
     pool = 4 * MAX_PAGES_PER_SEQ
     bt = assign_pages(seq_lens, pool, seed + 1, stride=MAX_PAGES_PER_SEQ)
-    vals = _values(4, pool, seed, device, num_q_heads)
+    vals = _values(4, pool, seed, device, num_q_heads, new_tokens)
     return Workload(name="cfg4: B=4, seq_len=40960, 10240 shuffled pages",
                     seq_lens=seq_lens, block_table=bt, num_pages=pool, **vals)
 

@@ -65,6 +65,10 @@ def _load():
             u16p, u16p, u16p, i32p, i32p, i32p, ctypes.c_int, u16p, u16p, ctypes.c_int,
             dp, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_double, dp, dp]
         lib.oracle_append_and_attend_gqa.restype = ctypes.c_int
+        lib.oracle_append_and_attend_tokens.argtypes = [
+            u16p, u16p, u16p, i32p, i32p, i32p, ctypes.c_int, u16p, u16p, ctypes.c_int,
+            dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_double, dp, dp]
+        lib.oracle_append_and_attend_tokens.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -124,7 +128,8 @@ def decode_head(q, seq_len: int, bt_row, k_cache, v_cache, kv_head: int) -> np.n
 def append_and_attend(qkv, q_norm_w, k_norm_w, seq_lens, block_table, k_cache, v_cache,
                       positions=None, rope_theta: float = 1e6, rms_eps: float = 1e-6,
                       inplace: bool = False, want_qk: bool = False) -> dict:
-    """Run the whole step. bf16 inputs are uint16 bit arrays.
+    """Run the whole step with one new token per sequence. bf16 inputs are
+    uint16 bit arrays.
 
     The number of query heads follows from the qkv row width,
     (num_q_heads + 16) * 128: 16 for Qwen3-0.6B, 32, 40 or 64 for larger sizes.
@@ -134,9 +139,27 @@ def append_and_attend(qkv, q_norm_w, k_norm_w, seq_lens, block_table, k_cache, v
     the new k before its rounding to bf16).
     """
     qkv = np.ascontiguousarray(qkv, dtype=np.uint16)
-    B = qkv.shape[0]
-    assert qkv.ndim == 2 and qkv.shape[1] % HEAD_DIM == 0
-    Hq = qkv.shape[1] // HEAD_DIM - 2 * NUM_KV_HEADS
+    out = append_and_attend_tokens(qkv[:, None, :], q_norm_w, k_norm_w, seq_lens, block_table, k_cache,
+                                   v_cache, positions=positions, rope_theta=rope_theta, rms_eps=rms_eps,
+                                   inplace=inplace, want_qk=want_qk)
+    out["o"] = out["o"][:, 0]
+    if want_qk:
+        out["q"], out["k"] = out["q"][:, 0], out["k"][:, 0]
+    return out
+
+
+def append_and_attend_tokens(qkv, q_norm_w, k_norm_w, seq_lens, block_table, k_cache, v_cache,
+                             positions=None, rope_theta: float = 1e6, rms_eps: float = 1e-6,
+                             inplace: bool = False, want_qk: bool = False) -> dict:
+    """The step with T new tokens per sequence: qkv is [B, T, (Hq + 16) * 128];
+    token t goes to slot L - T + t and attends causally over slots <= L - T + t.
+    ``positions`` (if given) are the first new token's RoPE positions.
+    Returns ``o`` float64 [B, T, Hq, 128], the caches, and with ``want_qk``
+    ``q`` [B, T, Hq, 128] and ``k`` [B, T, 8, 128]."""
+    qkv = np.ascontiguousarray(qkv, dtype=np.uint16)
+    assert qkv.ndim == 3 and qkv.shape[2] % HEAD_DIM == 0
+    B, T = qkv.shape[0], qkv.shape[1]
+    Hq = qkv.shape[2] // HEAD_DIM - 2 * NUM_KV_HEADS
     q_norm_w = np.ascontiguousarray(q_norm_w, dtype=np.uint16)
     k_norm_w = np.ascontiguousarray(k_norm_w, dtype=np.uint16)
     seq_lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
@@ -151,15 +174,15 @@ def append_and_attend(qkv, q_norm_w, k_norm_w, seq_lens, block_table, k_cache, v
     assert v_cache.dtype == np.uint16 and v_cache.flags["C_CONTIGUOUS"]
     num_pages = k_cache.shape[0]
     assert k_cache.shape == (num_pages, PAGE, NUM_KV_HEADS, HEAD_DIM) == v_cache.shape
-    o = np.empty((B, Hq, HEAD_DIM), dtype=np.float64)
-    q = np.empty((B, Hq, HEAD_DIM), dtype=np.float64) if want_qk else None
-    k = np.empty((B, NUM_KV_HEADS, HEAD_DIM), dtype=np.float64) if want_qk else None
-    rc = _load().oracle_append_and_attend_gqa(
+    o = np.empty((B, T, Hq, HEAD_DIM), dtype=np.float64)
+    q = np.empty((B, T, Hq, HEAD_DIM), dtype=np.float64) if want_qk else None
+    k = np.empty((B, T, NUM_KV_HEADS, HEAD_DIM), dtype=np.float64) if want_qk else None
+    rc = _load().oracle_append_and_attend_tokens(
         _ptr(qkv, ctypes.c_uint16), _ptr(q_norm_w, ctypes.c_uint16), _ptr(k_norm_w, ctypes.c_uint16),
         _ptr(seq_lens, ctypes.c_int32), _ptr(positions, ctypes.c_int32),
         _ptr(block_table, ctypes.c_int32), block_table.shape[1],
         _ptr(k_cache, ctypes.c_uint16), _ptr(v_cache, ctypes.c_uint16), num_pages,
-        _ptr(o, ctypes.c_double), B, Hq, rope_theta, rms_eps,
+        _ptr(o, ctypes.c_double), B, T, Hq, rope_theta, rms_eps,
         _ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double))
     if rc != 0:
         raise ValueError(f"oracle_append_and_attend: {_ERRORS.get(rc, rc)}")

@@ -181,36 +181,43 @@ void oracle_decode_head(const double *q, int L, const int32_t *bt_row,
 
 /* ---- the whole step ------------------------------------------------------ */
 
-/* The decode-attention step for a batch, in the order the specification
- * gives it: for every sequence, norm and rotate q and k, append the new k and
- * v to the cache; then, over the cache as it stands after the append, attend.
+/* The attention step for a batch with T new tokens per sequence, in the
+ * order the specification gives it: for every sequence and new token, norm
+ * and rotate q and k, append the new k and v to the cache; then, over the
+ * cache as it stands after the appends, attend causally: new token t of
+ * sequence b sits in cache slot L - T + t (L = seq_lens[b] counts the new
+ * tokens) and its query reads slots 0 .. L - T + t (Model Spec, "What to
+ * watch for": every layer is full causal attention; "At a glance": T tokens;
+ * Supported models, forward_causal). T = 1 is decodeGQA (attn.core).
  * num_q_heads query heads share the 8 kv heads: 16 for Qwen3-0.6B and 1.7B,
  * 32 for 4B/8B, 40 for 14B, 64 for 32B (nnterp qwen3, "Grouped-query
  * attention, with 128-wide heads on every size"); query head h reads kv head
  * h / (num_q_heads / 8), which is h / 2 for 0.6B (Model Spec attn.core).
  *
- *   qkv          bf16 [B][(num_q_heads + 16) * 128], q | k | v, head-major
+ *   qkv          bf16 [B][T][(num_q_heads + 16) * 128], q | k | v, head-major
  *   q_norm_w     bf16 [128], k_norm_w bf16 [128] (one gain for every head)
- *   seq_lens     [B], counts the new token, 1 <= L <= 40960 and <= 16*bt_stride
- *   positions    [B] RoPE positions, or NULL for seq_lens[b]-1
+ *   seq_lens     [B], counts the new tokens, T <= L <= 40960 and <= 16*bt_stride
+ *   positions    [B] RoPE position of each sequence's first new token (token
+ *                t has positions[b] + t), or NULL for L - T
  *   block_table  [B][bt_stride] page ids; entries past ceil(L/16) are not read
  *   k_cache, v_cache  bf16 [num_pages][16][8][128], updated in place
- *   o            double [B][num_q_heads][128] (output)
- *   q_out        double [B][num_q_heads][128] or NULL: q after norm and RoPE
- *   k_out        double [B][8][128] or NULL: new k after norm and RoPE, before
- *                its rounding to bf16
+ *   o            double [B][T][num_q_heads][128] (output)
+ *   q_out        double [B][T][num_q_heads][128] or NULL: q after norm and RoPE
+ *   k_out        double [B][T][8][128] or NULL: new k after norm and RoPE,
+ *                before its rounding to bf16
  *
  * Returns 0, ORC_ERR_ARG, or ORC_ERR_BOUNDS (nothing is written then). */
-int oracle_append_and_attend_gqa(const uint16_t *qkv, const uint16_t *q_norm_w,
-                                 const uint16_t *k_norm_w, const int32_t *seq_lens,
-                                 const int32_t *positions, const int32_t *block_table,
-                                 int bt_stride, uint16_t *k_cache, uint16_t *v_cache,
-                                 int num_pages, double *o, int B, int num_q_heads,
-                                 double rope_theta, double rms_eps, double *q_out,
-                                 double *k_out)
+int oracle_append_and_attend_tokens(const uint16_t *qkv, const uint16_t *q_norm_w,
+                                    const uint16_t *k_norm_w, const int32_t *seq_lens,
+                                    const int32_t *positions, const int32_t *block_table,
+                                    int bt_stride, uint16_t *k_cache, uint16_t *v_cache,
+                                    int num_pages, double *o, int B, int T, int num_q_heads,
+                                    double rope_theta, double rms_eps, double *q_out,
+                                    double *k_out)
 {
     if (!qkv || !q_norm_w || !k_norm_w || !seq_lens || !block_table || !k_cache ||
         !v_cache || !o || B < 1 || B > ORC_MAX_BATCH || bt_stride < 1 || num_pages < 1 ||
+        T < 1 || T > 16 ||
         num_q_heads < ORC_NUM_KV_HEADS || num_q_heads % ORC_NUM_KV_HEADS != 0 || num_q_heads > 64)
         return ORC_ERR_ARG;
     const int group = num_q_heads / ORC_NUM_KV_HEADS;
@@ -220,7 +227,7 @@ int oracle_append_and_attend_gqa(const uint16_t *qkv, const uint16_t *q_norm_w,
     /* Validate every index the step will use before touching anything. */
     for (int b = 0; b < B; ++b) {
         int L = seq_lens[b];
-        if (L < 1 || L > ORC_MAX_SEQ || L > ORC_PAGE * bt_stride) return ORC_ERR_BOUNDS;
+        if (L < T || L > ORC_MAX_SEQ || L > ORC_PAGE * bt_stride) return ORC_ERR_BOUNDS;
         for (int p = 0; p < (L + ORC_PAGE - 1) / ORC_PAGE; ++p) {
             int32_t id = block_table[(size_t)b * bt_stride + p];
             if (id < 0 || id >= num_pages) return ORC_ERR_BOUNDS;
@@ -233,59 +240,79 @@ int oracle_append_and_attend_gqa(const uint16_t *qkv, const uint16_t *q_norm_w,
         wk[i] = oracle_bf16_to_f64(k_norm_w[i]);
     }
 
-    double *q_all = (double *)malloc(sizeof(double) * (size_t)B * q_width);
+    double *q_all = (double *)malloc(sizeof(double) * (size_t)B * T * q_width);
     if (!q_all) return ORC_ERR_ARG;
 
-    /* Norm, rotation and append, sequence by sequence. */
+    /* Norm, rotation and append, sequence by sequence, token by token. */
     for (int b = 0; b < B; ++b) {
-        const uint16_t *row = qkv + (size_t)b * row_width;
         int L = seq_lens[b];
-        int slot = L - 1;
-        double pos = positions ? (double)positions[b] : (double)slot;
-        double x[ORC_HEAD_DIM], y[ORC_HEAD_DIM];
+        for (int t = 0; t < T; ++t) {
+            const uint16_t *row = qkv + ((size_t)b * T + t) * row_width;
+            int slot = L - T + t;
+            double pos = positions ? (double)positions[b] + t : (double)slot;
+            double x[ORC_HEAD_DIM], y[ORC_HEAD_DIM];
 
-        for (int h = 0; h < num_q_heads; ++h) {
-            for (int i = 0; i < ORC_HEAD_DIM; ++i)
-                x[i] = oracle_bf16_to_f64(row[h * ORC_HEAD_DIM + i]);
-            oracle_rmsnorm(x, wq, ORC_HEAD_DIM, rms_eps, y);
-            oracle_rope(y, ORC_HEAD_DIM, pos, rope_theta);
-            memcpy(q_all + ((size_t)b * num_q_heads + h) * ORC_HEAD_DIM, y, sizeof y);
-        }
+            for (int h = 0; h < num_q_heads; ++h) {
+                for (int i = 0; i < ORC_HEAD_DIM; ++i)
+                    x[i] = oracle_bf16_to_f64(row[h * ORC_HEAD_DIM + i]);
+                oracle_rmsnorm(x, wq, ORC_HEAD_DIM, rms_eps, y);
+                oracle_rope(y, ORC_HEAD_DIM, pos, rope_theta);
+                memcpy(q_all + (((size_t)b * T + t) * num_q_heads + h) * ORC_HEAD_DIM, y, sizeof y);
+            }
 
-        int32_t page = block_table[(size_t)b * bt_stride + slot / ORC_PAGE];
-        size_t slot_base = (size_t)page * ORC_PAGE_ELEMS + (size_t)(slot % ORC_PAGE) * ORC_KV_WIDTH;
-        for (int j = 0; j < ORC_NUM_KV_HEADS; ++j) {
-            for (int i = 0; i < ORC_HEAD_DIM; ++i)
-                x[i] = oracle_bf16_to_f64(row[q_width + j * ORC_HEAD_DIM + i]);
-            oracle_rmsnorm(x, wk, ORC_HEAD_DIM, rms_eps, y);
-            oracle_rope(y, ORC_HEAD_DIM, pos, rope_theta);
-            if (k_out) memcpy(k_out + ((size_t)b * ORC_NUM_KV_HEADS + j) * ORC_HEAD_DIM, y, sizeof y);
-            for (int i = 0; i < ORC_HEAD_DIM; ++i) {
-                k_cache[slot_base + (size_t)j * ORC_HEAD_DIM + i] = oracle_f64_to_bf16_rne(y[i]);
-                /* v has no norm and no rotation: its bits are copied. */
-                v_cache[slot_base + (size_t)j * ORC_HEAD_DIM + i] =
-                    row[q_width + ORC_KV_WIDTH + j * ORC_HEAD_DIM + i];
+            int32_t page = block_table[(size_t)b * bt_stride + slot / ORC_PAGE];
+            size_t slot_base = (size_t)page * ORC_PAGE_ELEMS + (size_t)(slot % ORC_PAGE) * ORC_KV_WIDTH;
+            for (int j = 0; j < ORC_NUM_KV_HEADS; ++j) {
+                for (int i = 0; i < ORC_HEAD_DIM; ++i)
+                    x[i] = oracle_bf16_to_f64(row[q_width + j * ORC_HEAD_DIM + i]);
+                oracle_rmsnorm(x, wk, ORC_HEAD_DIM, rms_eps, y);
+                oracle_rope(y, ORC_HEAD_DIM, pos, rope_theta);
+                if (k_out)
+                    memcpy(k_out + (((size_t)b * T + t) * ORC_NUM_KV_HEADS + j) * ORC_HEAD_DIM, y, sizeof y);
+                for (int i = 0; i < ORC_HEAD_DIM; ++i) {
+                    k_cache[slot_base + (size_t)j * ORC_HEAD_DIM + i] = oracle_f64_to_bf16_rne(y[i]);
+                    /* v has no norm and no rotation: its bits are copied. */
+                    v_cache[slot_base + (size_t)j * ORC_HEAD_DIM + i] =
+                        row[q_width + ORC_KV_WIDTH + j * ORC_HEAD_DIM + i];
+                }
             }
         }
     }
 
-    /* Attention over the cache as it stands after every append. */
+    /* Causal attention over the cache as it stands after every append: new
+     * token t reads the L - T + t + 1 slots up to and including its own. */
     int max_L = 0;
     for (int b = 0; b < B; ++b) if (seq_lens[b] > max_L) max_L = seq_lens[b];
     double *scores = (double *)malloc(sizeof(double) * (size_t)max_L);
     if (!scores) { free(q_all); return ORC_ERR_ARG; }
     for (int b = 0; b < B; ++b) {
-        for (int h = 0; h < num_q_heads; ++h) {
-            oracle_decode_head(q_all + ((size_t)b * num_q_heads + h) * ORC_HEAD_DIM,
-                               seq_lens[b], block_table + (size_t)b * bt_stride,
-                               k_cache, v_cache, h / group,
-                               scores, o + ((size_t)b * num_q_heads + h) * ORC_HEAD_DIM);
+        for (int t = 0; t < T; ++t) {
+            int visible = seq_lens[b] - T + t + 1;
+            for (int h = 0; h < num_q_heads; ++h) {
+                size_t r = ((size_t)b * T + t) * num_q_heads + h;
+                oracle_decode_head(q_all + r * ORC_HEAD_DIM, visible, block_table + (size_t)b * bt_stride,
+                                   k_cache, v_cache, h / group, scores, o + r * ORC_HEAD_DIM);
+            }
         }
     }
-    if (q_out) memcpy(q_out, q_all, sizeof(double) * (size_t)B * q_width);
+    if (q_out) memcpy(q_out, q_all, sizeof(double) * (size_t)B * T * q_width);
     free(scores);
     free(q_all);
     return ORC_OK;
+}
+
+/* One new token per sequence (decodeGQA, Model Spec attn.core). */
+int oracle_append_and_attend_gqa(const uint16_t *qkv, const uint16_t *q_norm_w,
+                                 const uint16_t *k_norm_w, const int32_t *seq_lens,
+                                 const int32_t *positions, const int32_t *block_table,
+                                 int bt_stride, uint16_t *k_cache, uint16_t *v_cache,
+                                 int num_pages, double *o, int B, int num_q_heads,
+                                 double rope_theta, double rms_eps, double *q_out,
+                                 double *k_out)
+{
+    return oracle_append_and_attend_tokens(qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table,
+                                           bt_stride, k_cache, v_cache, num_pages, o, B, 1, num_q_heads,
+                                           rope_theta, rms_eps, q_out, k_out);
 }
 
 /* The Qwen3-0.6B step: 16 query heads over 8 kv heads (Model Spec attn.core). */

@@ -483,3 +483,78 @@ def test_larger_group_head_mapping(oracle_mod, num_q_heads):
         o = oracle_mod.append_and_attend(*args, kc, vc2)["o"]
         changed = [h for h in range(num_q_heads) if not np.array_equal(o[0, h], base[0, h])]
         assert changed == list(range(G * j, G * j + G))
+
+
+# ----------------------------------------------------------------------------
+# several new tokens per sequence, causal inside the new block
+# (Model Spec, "What to watch for": every layer is full causal attention;
+#  "At a glance": T tokens; Supported models: forward_causal)
+
+def _tok_args(w, oracle_mod):
+    from decode_attention_qk_b200 import inputs
+    return dict(qkv=inputs.bf16_bits(w.qkv), q_norm_w=inputs.bf16_bits(w.q_norm_w),
+                k_norm_w=inputs.bf16_bits(w.k_norm_w), seq_lens=w.seq_lens.numpy(),
+                block_table=w.block_table.numpy(), k_cache=inputs.bf16_bits(w.k_cache),
+                v_cache=inputs.bf16_bits(w.v_cache))
+
+
+@pytest.mark.parametrize("T,hq", [(2, 16), (3, 16), (4, 16), (2, 32)])
+def test_tokens_match_sdpa_with_bottom_right_causal_mask(oracle_mod, T, hq):
+    from decode_attention_qk_b200 import inputs
+    w = inputs.custom([T, 17, 40], seed=50 + T, num_q_heads=hq, new_tokens=T, pool_pages=6)
+    out = oracle_mod.append_and_attend_tokens(**_tok_args(w, oracle_mod), want_qk=True)
+    kc, vc = out["k_cache"], out["v_cache"]
+    for b, L in enumerate(w.seq_lens.tolist()):
+        bt = w.block_table[b].numpy()
+        K = np.stack([oracle_mod.bf16_to_f64(kc[bt[t // 16], t % 16]) for t in range(L)], axis=1)
+        V = np.stack([oracle_mod.bf16_to_f64(vc[bt[t // 16], t % 16]) for t in range(L)], axis=1)
+        mask = torch.tensor([[s <= L - T + t for s in range(L)] for t in range(T)])   # query t, key s
+        q = torch.from_numpy(out["q"][b]).permute(1, 0, 2)[None]                   # [1, Hq, T, 128]
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q, torch.from_numpy(K)[None], torch.from_numpy(V)[None], attn_mask=mask, enable_gqa=True)
+        ref = ref[0].permute(1, 0, 2).numpy()                                      # [T, Hq, 128]
+        assert np.max(np.abs(out["o"][b] - ref)) <= 1e-9 * np.max(np.abs(ref))
+
+
+def test_tokens_equal_successive_single_token_steps(oracle_mod):
+    """T new tokens in one step give exactly what T one-token steps give, one after
+    the other: same cache, same outputs (the decode step is the T = 1 case)."""
+    from decode_attention_qk_b200 import inputs
+    T = 3
+    w = inputs.custom([20, 3, 50], seed=53, new_tokens=T, pool_pages=7)
+    a = _tok_args(w, oracle_mod)
+    multi = oracle_mod.append_and_attend_tokens(**a)
+    kc, vc = a["k_cache"].copy(), a["v_cache"].copy()
+    for t in range(T):
+        lens = w.seq_lens.numpy() - (T - 1 - t)
+        one = oracle_mod.append_and_attend(a["qkv"][:, t], a["q_norm_w"], a["k_norm_w"], lens, a["block_table"],
+                                           kc, vc, inplace=True)
+        assert np.array_equal(one["o"], multi["o"][:, t])
+    assert np.array_equal(kc, multi["k_cache"]) and np.array_equal(vc, multi["v_cache"])
+
+
+def test_tokens_causality(oracle_mod):
+    """Model conformance, "Causality": changing a later new token's q, k and v never
+    changes an earlier new token's output (the earlier outputs stay bit-identical)."""
+    from decode_attention_qk_b200 import inputs
+    T = 4
+    w = inputs.custom([30, 4], seed=54, new_tokens=T)
+    a = _tok_args(w, oracle_mod)
+    base = oracle_mod.append_and_attend_tokens(**a)["o"]
+    for t in range(T):
+        a2 = dict(a)
+        qkv = a["qkv"].copy()
+        qkv[:, t, :] ^= 0x0040          # perturb token t's whole row
+        a2["qkv"] = qkv
+        o = oracle_mod.append_and_attend_tokens(**a2)["o"]
+        assert np.array_equal(o[:, :t], base[:, :t])
+        assert not np.array_equal(o[:, t], base[:, t])
+
+
+def test_tokens_default_positions(oracle_mod):
+    from decode_attention_qk_b200 import inputs
+    w = inputs.custom([9, 33], seed=55, new_tokens=2)
+    a = _tok_args(w, oracle_mod)
+    o1 = oracle_mod.append_and_attend_tokens(**a)["o"]
+    o2 = oracle_mod.append_and_attend_tokens(**a, positions=w.seq_lens.numpy() - 2)["o"]
+    assert np.array_equal(o1, o2)
