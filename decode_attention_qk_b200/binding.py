@@ -27,6 +27,9 @@ QDA_FLAG_INJECT_WAIT_TIMEOUT = 0x1
 
 NUM_Q_HEADS, NUM_KV_HEADS, HEAD_DIM, PAGE_SIZE, QKV_WIDTH = 16, 8, 128, 16, 4096
 SUPPORTED_Q_HEADS = (16, 32, 40, 64)   # Qwen3 0.6B/1.7B, 4B/8B, 14B, 32B
+MAX_NEW_TOKENS = 4
+# (query heads, new tokens) pairs with a kernel for more than one new token
+SUPPORTED_MULTI_TOKEN = ((16, 2), (16, 3), (16, 4), (32, 2))
 
 
 class qda_config(ctypes.Structure):
@@ -74,6 +77,8 @@ def load_library():
         lib.qwen3_decode_attn_append_and_attend.restype = ctypes.c_int
         lib.qwen3_decode_attn_append_and_attend_host.argtypes = call
         lib.qwen3_decode_attn_append_and_attend_host.restype = ctypes.c_int
+        lib.qwen3_decode_attn_append_and_attend_tokens.argtypes = call[:-1] + [ctypes.c_int, vp]
+        lib.qwen3_decode_attn_append_and_attend_tokens.restype = ctypes.c_int
         lib.qwen3_decode_attn_check.argtypes = [vp, vp]
         lib.qwen3_decode_attn_check.restype = ctypes.c_int
         lib.qwen3_decode_attn_grid_ctas.argtypes = [vp]
@@ -135,17 +140,18 @@ def qwen3_decode_attn_create(cfg: qda_config | None = None, device: int = 0) -> 
 
 
 def num_q_heads_of(qkv: torch.Tensor) -> int:
-    """Query heads of a fused qkv row of (Hq + 16) * 128 values."""
-    if qkv.dim() != 2 or qkv.shape[1] % HEAD_DIM != 0:
-        raise ValueError("qkv must be [B, (num_q_heads + 16) * 128]")
-    return int(qkv.shape[1]) // HEAD_DIM - 2 * NUM_KV_HEADS
+    """Query heads of a fused qkv row of (Hq + 16) * 128 values (qkv [B, W] or [B, T, W])."""
+    if qkv.dim() not in (2, 3) or qkv.shape[-1] % HEAD_DIM != 0:
+        raise ValueError("qkv must be [B, (num_q_heads + 16) * 128] or [B, T, (num_q_heads + 16) * 128]")
+    return int(qkv.shape[-1]) // HEAD_DIM - 2 * NUM_KV_HEADS
 
 
 def _step_args(qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, k_cache, v_cache, o,
                dev_of_step, dev_of_state):
     Hq = num_q_heads_of(qkv)
     B = qkv.shape[0]
-    _expect(qkv, "qkv", torch.bfloat16, (B, (Hq + 2 * NUM_KV_HEADS) * HEAD_DIM), dev_of_step)
+    tokens = tuple(qkv.shape[1:-1])   # () for one new token, (T,) for several
+    _expect(qkv, "qkv", torch.bfloat16, (B, *tokens, (Hq + 2 * NUM_KV_HEADS) * HEAD_DIM), dev_of_step)
     _expect(q_norm_w, "q_norm_w", torch.bfloat16, (HEAD_DIM,), dev_of_state)
     _expect(k_norm_w, "k_norm_w", torch.bfloat16, (HEAD_DIM,), dev_of_state)
     _expect(seq_lens, "seq_lens", torch.int32, (B,), dev_of_step)
@@ -157,7 +163,7 @@ def _step_args(qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, k_cach
     P = k_cache.shape[0]
     _expect(k_cache, "k_cache", torch.bfloat16, (P, PAGE_SIZE, NUM_KV_HEADS, HEAD_DIM), dev_of_state)
     _expect(v_cache, "v_cache", torch.bfloat16, (P, PAGE_SIZE, NUM_KV_HEADS, HEAD_DIM), dev_of_state)
-    _expect(o, "o", torch.bfloat16, (B, Hq, HEAD_DIM), dev_of_step)
+    _expect(o, "o", torch.bfloat16, (B, *tokens, Hq, HEAD_DIM), dev_of_step)
     return (_ptr(qkv), _ptr(q_norm_w), _ptr(k_norm_w), _i32p(seq_lens), _i32p(positions),
             _i32p(block_table), int(block_table.shape[1]), _ptr(k_cache), _ptr(v_cache), int(P),
             _ptr(o), int(B))
@@ -169,10 +175,30 @@ def qwen3_decode_attn_append_and_attend(handle, qkv, q_norm_w, k_norm_w, seq_len
     dev = qkv.device
     if dev.type != "cuda":
         raise ValueError("qkv must be a CUDA tensor")
+    if qkv.dim() != 2:
+        raise ValueError("qkv must be [B, (num_q_heads + 16) * 128]; several new tokens go through "
+                         "qwen3_decode_attn_append_and_attend_tokens")
     args = _step_args(qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, k_cache, v_cache, o, dev, dev)
     rc = load_library().qwen3_decode_attn_append_and_attend(handle, *args, _stream(stream, dev))
     if rc != QDA_OK:
         raise QdaError(rc, "qwen3_decode_attn_append_and_attend")
+
+
+def qwen3_decode_attn_append_and_attend_tokens(handle, qkv, q_norm_w, k_norm_w, seq_lens, positions,
+                                               block_table, k_cache, v_cache, o, stream=None) -> None:
+    """The step with T new tokens per sequence: qkv [B, T, W], o [B, T, Hq, 128];
+    token t goes to cache slot seq_lens[b] - T + t and attends causally up to it.
+    Asynchronous on `stream`; raises QdaError on a host-side error."""
+    dev = qkv.device
+    if dev.type != "cuda":
+        raise ValueError("qkv must be a CUDA tensor")
+    if qkv.dim() != 3:
+        raise ValueError("qkv must be [B, T, (num_q_heads + 16) * 128]")
+    args = _step_args(qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, k_cache, v_cache, o, dev, dev)
+    rc = load_library().qwen3_decode_attn_append_and_attend_tokens(handle, *args, int(qkv.shape[1]),
+                                                                   _stream(stream, dev))
+    if rc != QDA_OK:
+        raise QdaError(rc, "qwen3_decode_attn_append_and_attend_tokens")
 
 
 def qwen3_decode_attn_append_and_attend_host(handle, qkv, q_norm_w, k_norm_w, seq_lens, positions,
@@ -182,6 +208,8 @@ def qwen3_decode_attn_append_and_attend_host(handle, qkv, q_norm_w, k_norm_w, se
     dev = k_cache.device
     cpu = torch.device("cpu")
     args = _step_args(qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, k_cache, v_cache, o, cpu, dev)
+    if qkv.dim() != 2:
+        raise ValueError("the host-buffer entry point takes one new token per sequence: qkv [B, W]")
     rc = load_library().qwen3_decode_attn_append_and_attend_host(handle, *args, _stream(stream, dev))
     if rc != QDA_OK:
         raise QdaError(rc, "qwen3_decode_attn_append_and_attend_host")
@@ -196,6 +224,8 @@ def qwen3_decode_attn_append_and_attend_noalloc(qkv, q_norm_w, k_norm_w, seq_len
     dev = qkv.device
     if dev.type != "cuda":
         raise ValueError("qkv must be a CUDA tensor")
+    if qkv.dim() != 2:
+        raise ValueError("the no-allocation entry point takes one new token per sequence: qkv [B, W]")
     args = _step_args(qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, k_cache, v_cache, o, dev, dev)
     f = load_library().qwen3_decode_attn_append_and_attend_noalloc
     vp, i32p = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32)
@@ -223,7 +253,8 @@ class DecodeAttention:
     """A handle with its lifetime: DecodeAttention(device=0, **config fields).
 
     `num_q_heads` (16, 32, 40 or 64) selects the Qwen3 size; calls must pass qkv
-    rows of (num_q_heads + 16) * 128 values."""
+    rows of (num_q_heads + 16) * 128 values: qkv [B, W] for one new token per
+    sequence (o [B, Hq, 128]), or [B, T, W] for T new tokens (o [B, T, Hq, 128])."""
 
     def __init__(self, device: int = 0, **config):
         self.device = torch.device("cuda", device)
@@ -240,10 +271,10 @@ class DecodeAttention:
             raise ValueError(f"qkv rows hold {num_q_heads_of(qkv)} query heads; the handle was made for "
                              f"{self.config.num_q_heads}")
         if o is None:
-            o = torch.empty((qkv.shape[0], self.config.num_q_heads, HEAD_DIM), dtype=torch.bfloat16,
+            o = torch.empty((*qkv.shape[:-1], self.config.num_q_heads, HEAD_DIM), dtype=torch.bfloat16,
                             device=qkv.device)
-        qwen3_decode_attn_append_and_attend(self.handle, qkv, q_norm_w, k_norm_w, seq_lens, positions,
-                                            block_table, k_cache, v_cache, o, stream)
+        step = qwen3_decode_attn_append_and_attend_tokens if qkv.dim() == 3 else qwen3_decode_attn_append_and_attend
+        step(self.handle, qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, k_cache, v_cache, o, stream)
         return o
 
     def check(self, stream=None) -> int:

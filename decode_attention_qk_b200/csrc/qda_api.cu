@@ -104,6 +104,7 @@ qda::Params make_params(const qda_handle* h, const void* qkv, const void* q_norm
     p.v_cache = static_cast<uint16_t*>(v_cache);
     p.o = static_cast<uint16_t*>(o);
     p.num_q_heads = h->cfg.num_q_heads;
+    p.new_tokens = 1;
     p.bt_stride = block_table_stride;
     p.num_pages = num_pages;
     p.batch = batch;
@@ -121,8 +122,8 @@ qda::Params make_params(const qda_handle* h, const void* qkv, const void* q_norm
 }
 
 cudaError_t launch_step(const qda_handle* h, const qda::Params& p, cudaStream_t stream) {
-    return h->cfg.num_q_heads == qda::kNumQHeads ? qda::launch(p, h->grid, stream)
-                                                 : qda::launch_grouped(p, h->grid, stream);
+    return p.num_q_heads == qda::kNumQHeads && p.new_tokens == 1 ? qda::launch(p, h->grid, stream)
+                                                                 : qda::launch_grouped(p, h->grid, stream);
 }
 
 }  // namespace
@@ -178,8 +179,11 @@ int qwen3_decode_attn_create(const qda_config* cfg, int device, qda_handle** out
     const size_t slots = (size_t)qda::num_slots(h->grid, cfg->max_batch);
     const size_t B = (size_t)cfg->max_batch;
     const size_t Hq = (size_t)cfg->num_q_heads;
-    bool ok = alloc(&h->part_acc, slots * Hq * qda::kHeadDim * sizeof(float)) &&
-              alloc(&h->part_ml, slots * Hq * sizeof(float2)) &&
+    // partial rows per slot: 16 for the 16-head decode kernel, kPartRows (new
+    // tokens x query heads) for the tensor-core kernel; size for the larger
+    const size_t rows = (size_t)qda::kPartRows;
+    bool ok = alloc(&h->part_acc, slots * rows * qda::kHeadDim * sizeof(float)) &&
+              alloc(&h->part_ml, slots * rows * sizeof(float2)) &&
               alloc(&h->counters, (size_t)qda::kMaxBatch * qda::kNumKvHeads * sizeof(int)) &&
               alloc(&h->status, sizeof(int)) && alloc(&h->seg, (size_t)(qda::kMaxBatch + 1) * sizeof(int)) &&
               alloc(&h->st_qkv, B * qkv_elems(cfg->num_q_heads) * sizeof(uint16_t)) &&
@@ -209,6 +213,24 @@ int qwen3_decode_attn_append_and_attend(qda_handle* h, const void* qkv, const vo
     if (!guard.ok()) return QDA_ERR_CUDA;
     const qda::Params p = make_params(h, qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table,
                                       block_table_stride, k_cache, v_cache, num_pages, o, batch);
+    return launch_step(h, p, static_cast<cudaStream_t>(cuda_stream)) == cudaSuccess ? QDA_OK : QDA_ERR_CUDA;
+}
+
+int qwen3_decode_attn_append_and_attend_tokens(qda_handle* h, const void* qkv, const void* q_norm_w,
+                                               const void* k_norm_w, const int32_t* seq_lens,
+                                               const int32_t* positions, const int32_t* block_table,
+                                               int block_table_stride, void* k_cache, void* v_cache, int num_pages,
+                                               void* o, int batch, int new_tokens, void* cuda_stream) {
+    int rc = check_call(h, qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, block_table_stride, k_cache,
+                        v_cache, num_pages, o, batch);
+    if (rc != QDA_OK) return rc;
+    if (new_tokens < 1 || new_tokens > QDA_MAX_NEW_TOKENS) return QDA_ERR_INVALID_ARG;
+    if (new_tokens > 1 && !qda::grouped_supported(h->cfg.num_q_heads, new_tokens)) return QDA_ERR_UNSUPPORTED;
+    DeviceGuard guard(h->device);
+    if (!guard.ok()) return QDA_ERR_CUDA;
+    qda::Params p = make_params(h, qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, block_table_stride,
+                                k_cache, v_cache, num_pages, o, batch);
+    p.new_tokens = new_tokens;
     return launch_step(h, p, static_cast<cudaStream_t>(cuda_stream)) == cudaSuccess ? QDA_OK : QDA_ERR_CUDA;
 }
 
@@ -281,7 +303,7 @@ const char* qwen3_decode_attn_strerror(int code) {
         case QDA_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
         case QDA_ERR_UNSUPPORTED:
             return "configuration differs from the compiled head geometry (16/32/40/64 query heads, 8 kv heads, "
-                   "head dim 128, page 16)";
+                   "head dim 128, page 16) or has no kernel for this count of new tokens";
         case QDA_ERR_BOUNDS: return "a seq_len or block-table entry was out of range on the device";
         case QDA_ERR_TIMEOUT: return "a device-side wait ran out of time";
         default: return "unknown error code";

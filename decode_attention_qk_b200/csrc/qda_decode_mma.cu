@@ -1,33 +1,41 @@
-// Decode-attention step for the larger Qwen3 sizes: 32, 40 or 64 query heads
-// over 8 kv heads of 128 (nnterp qwen3, "Grouped-query attention, with
-// 128-wide heads on every size"), i.e. G = 4, 5 or 8 query heads per kv head.
-// Same computation as the 16-head kernel (Qwen3-0.6B Model Spec,
+// Tensor-core attention step for the larger Qwen3 sizes -- 32, 40 or 64 query
+// heads over 8 kv heads of 128 (nnterp qwen3, "Grouped-query attention, with
+// 128-wide heads on every size"), i.e. G = 4, 5 or 8 query heads per kv head --
+// and for T > 1 new tokens per sequence at any size with T*G <= 8. Same
+// computation as the 16-head decode kernel (Qwen3-0.6B Model Spec,
 // "Compute-graph nodes": attn.qk_norm, attn.rope, attn.core, and the append
-// to the 16-token paged cache); query head h reads kv head h / G.
+// to the 16-token paged cache); query head h reads kv head h / G. With T new
+// tokens, token t sits in cache slot L - T + t and attends over slots up to
+// its own (Model Spec, "What to watch for": every layer is full causal
+// attention).
 //
 // Why tensor cores here. Per kv head and page the scores and the value sums
 // are a [G x 128] x [128 x 16] and a [G x 16] x [16 x 128] product: 2G flops
 // per byte of K/V, 16 at G = 8, above what the CUDA cores sustain at HBM
 // speed. Warp j (kv head j) runs them as mma.sync m16n8k16 bf16 products with
-// float accumulators. The 16 rows of the A operand hold, for head g < G, row g
-// = the bf16 value of q (or of the probabilities) and row g + 8 = the bf16 of
-// the remainder, so the products carry ~16 significant bits of q and p; the
-// two rows are added back in float. The score accumulator fragment of lane
-// (g = lane/4, t = lane%4) holds head g at tokens 2t, 2t+1, 8+2t, 9+2t, which is
-// exactly its A fragment for the value product, so probabilities never leave
-// registers.
+// float accumulators. Query row r < T*G stands for new token r / G and head
+// G*j + r % G; the 16 rows of the A operand hold, for row r, row r = the bf16
+// value of q (or of the probabilities) and row r + 8 = the bf16 of the
+// remainder, so the products carry ~16 significant bits of q and p; the two
+// rows are added back in float. The score accumulator fragment of lane
+// (r = lane/4, t = lane%4) holds row r at page tokens 2t, 2t+1, 8+2t, 9+2t,
+// which is exactly its A fragment for the value product, so probabilities
+// never leave registers. Each row masks the tokens after its own slot.
 //
 // Staging. A producer warp bulk-copies each token row (2 KiB, all 8 kv heads)
 // into a stage whose rows are 2064 bytes apart, so that the 8 rows an
 // ldmatrix phase reads start in 8 different 16-byte bank groups (at the
 // cache's own 2048-byte pitch they would all hit the same banks). Each
-// sequence piece's qkv row goes to one slot of its own, released by the
-// consumers once they have formed q.
+// sequence piece's T qkv rows go to one slot of their own, released by the
+// consumers once they have formed q. Only cache rows older than the new
+// tokens are copied; the new tokens' k (formed in double, rounded once to
+// bf16) and v are appended to the cache by the CTA holding their page and
+// patched into its staged page.
 //
 // Split sequences. The work split is the 16-head kernel's (equal page ranges
 // per CTA, scratch slot g + b per piece). A piece that covers its whole
 // sequence writes o; a piece of a split sequence writes its partial, and a
-// second launch (one CTA per sequence and kv head, one warp per query head)
+// second launch (one CTA per sequence and kv head, one warp per query row)
 // combines them with the log-sum-exp rule (Supported models, "Facts proved
 // about the specs": flashAttn_eq, softmax_shift), spreading long merges over
 // many SMs. That launch uses programmatic dependent launch so its start
@@ -42,7 +50,6 @@
 namespace qda {
 namespace {
 
-constexpr int kStages = 3;
 constexpr int kConsumerWarps = kNumKvHeads;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kRowPitch = kRowBytes + 16;           // staged token-row pitch: 2064 bytes
@@ -50,13 +57,16 @@ constexpr int kStageK = 0;
 constexpr int kStageV = kPage * kRowPitch;
 constexpr int kStageBytes = 2 * kPage * kRowPitch;  // 66048
 
-template <int G>
+template <int G, int T>
 struct Layout {
     static constexpr int kHq = G * kNumKvHeads;
-    static constexpr int kQkvW = (kHq + 2 * kNumKvHeads) * kHeadDim;   // elements in a qkv row
+    static constexpr int kRows = G * T;                                  // query rows per kv head
+    static constexpr int kQkvW = (kHq + 2 * kNumKvHeads) * kHeadDim;     // elements in one token's qkv row
     static constexpr int kQkvBytes = kQkvW * 2;
+    static constexpr int kSlotBytes = T * kQkvBytes;                     // a sequence's T rows
+    static constexpr int kStages = kSlotBytes <= 24576 ? 3 : 2;          // what fits next to the qkv slot
     static constexpr int kSmemQkv = kStages * kStageBytes;
-    static constexpr int kSmemSeg = kSmemQkv + kQkvBytes;                   // int [kMaxBatch + 4]
+    static constexpr int kSmemSeg = kSmemQkv + kSlotBytes;                  // int [kMaxBatch + 4]
     static constexpr int kSmemLens = kSmemSeg + (kMaxBatch + 4) * 4;        // int [kMaxBatch]
     static constexpr int kSmemInvFreq = kSmemLens + kMaxBatch * 4;          // double [64]
     static constexpr int kSmemGains = kSmemInvFreq + 64 * 8;                // bf16 [2][128]
@@ -64,13 +74,14 @@ struct Layout {
     static constexpr int kSmemBars = kSmemMeta + (kStages + 1) * 16;        // full, empty, qkv_full, qkv_empty, never
     static constexpr int kSmemFlags = kSmemBars + (2 * kStages + 3) * 8;
     static constexpr int kSmemTotal = kSmemFlags + 16;
+    static_assert(kRows <= 8, "at most 8 query rows per kv head");
     static_assert(kSmemQkv % 16 == 0 && kSmemInvFreq % 8 == 0 && kSmemBars % 8 == 0, "alignment");
     static_assert(kSmemTotal <= 227 * 1024, "fits one CTA per SM");
 };
 
 struct Shared {
     uint8_t* stages;
-    uint8_t* qkv;         // the current sequence piece's qkv row
+    uint8_t* qkv;         // the current sequence piece's T qkv rows
     int* seg;
     int* lens;
     double* inv_freq;
@@ -88,9 +99,10 @@ struct Shared {
 // ---------------------------------------------------------------------------
 // Producer warp.
 
-template <int G>
+template <int G, int T>
 __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, int B, int start, int end, int lane) {
-    using Lay = Layout<G>;
+    using Lay = Layout<G, T>;
+    constexpr int kStages = Lay::kStages;
     const int count = end - start;
     int slot = 0;
     uint32_t phase = 0, qphase = 0;
@@ -104,12 +116,12 @@ __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, i
         if (gp < end) {
             const int b = find_seq(s.seg, B, gp);
             const int i = gp - s.seg[b];
-            const int nb = s.seg[b + 1] - s.seg[b];
             id = __ldg(p.block_table + (size_t)b * p.bt_stride + i);
-            rows = (i == nb - 1) ? (s.lens[b] - 1) - kPage * i : kPage;
+            // only the rows older than the T new tokens are read from the cache
+            rows = min(kPage, max(0, (s.lens[b] - T) - kPage * i));
             if (gp == start || i == 0) {
                 qkv_b = b;
-                pos = p.positions != nullptr ? __ldg(p.positions + b) : s.lens[b] - 1;
+                pos = p.positions != nullptr ? __ldg(p.positions + b) : s.lens[b] - T;
             }
         }
         const int n = min(32, count - base);
@@ -127,8 +139,9 @@ __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, i
                          mbar_wait(s.qkv_empty, qphase ^ 1u, p.timeout_ns, s.abort_flag);
                     if (ok) {
                         *s.qkv_pos = seq_pos;
-                        mbar_arrive_expect_tx(s.qkv_full, (uint32_t)Lay::kQkvBytes);
-                        bulk_g2s(s.qkv, p.qkv + (size_t)seq_qkv * Lay::kQkvW, (uint32_t)Lay::kQkvBytes, s.qkv_full);
+                        mbar_arrive_expect_tx(s.qkv_full, (uint32_t)Lay::kSlotBytes);
+                        bulk_g2s(s.qkv, p.qkv + (size_t)seq_qkv * T * Lay::kQkvW, (uint32_t)Lay::kSlotBytes,
+                                 s.qkv_full);
                         qarmed = true;
                         qarmed_parity = qphase;
                         qphase ^= 1u;
@@ -186,37 +199,43 @@ __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, i
 // ---------------------------------------------------------------------------
 // Consumer warps.
 
+template <int T>
 struct State {
-    uint32_t qa[8][4];    // A fragments of q per 16-dim step: rows g (bf16 of q) and g+8 (remainder)
-    float o[16][4];       // value accumulators: 16 tiles of 8 dims, rows g and g+8
-    float m;              // running max of head g (log2 units)
+    uint32_t qa[8][4];    // A fragments of q per 16-dim step: rows r (bf16 of q) and r+8 (remainder)
+    float o[16][4];       // value accumulators: 16 tiles of 8 dims, rows r and r+8
+    float m;              // running max of row r (log2 units)
     float lsum;           // partial softmax sum of this lane's tokens
-    uint32_t k_lo, k_hi, v_lo, v_hi;   // this lane's words of the appended k/v row
+    uint32_t k_lo[T], k_hi[T], v_lo[T], v_hi[T];   // this lane's words of the appended k/v rows
 };
 
-// Start a sequence piece from the staged qkv row: q of head G*j + g for lane
-// (g, t) at dims 8m + 2t, 8m + 2t + 1 (m = 0..15), i.e. both halves of the
-// rotation pairs 8m' + 2t + e, m' < 8; the angles of pairs 2l, 2l+1 are formed
-// by lane l (reduced modulo 2*pi in double, then float sin/cos) and shared by
-// shuffles. The new k, when this CTA appends, is formed in double.
-template <int G>
-__device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s, int pos, int j, int lane,
-                                               bool appends, State& st) {
-    using Lay = Layout<G>;
+// Start a sequence piece from the staged qkv rows: q of row r = lane/4 (new
+// token r / G, head G*j + r % G) at dims 8m + 2t, 8m + 2t + 1 (t = lane%4,
+// m = 0..15), i.e. both halves of the rotation pairs 8m' + 2t + e, m' < 8.
+// Lane l forms the angles of pairs 2l, 2l+1 for every new token (reduced
+// modulo 2*pi in double, then float sin/cos); lanes fetch theirs by shuffles.
+// When this CTA holds a page with new tokens, their k is formed in double.
+template <int G, int T>
+__device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s, int pos0, int j, int lane,
+                                               bool appends, State<T>& st) {
+    using Lay = Layout<G, T>;
     constexpr double kTwoPiHi = 6.2831853069365025;      // 2*pi rounded to 32 significant bits
     constexpr double kTwoPiLo = 2.430840202602477e-10;   // 2*pi - kTwoPiHi
     constexpr double kInvTwoPi = 0.15915494309189535;
-    const int g = lane >> 2, t = lane & 3;
-    const double ang0 = (double)pos * s.inv_freq[2 * lane];
-    const double ang1 = (double)pos * s.inv_freq[2 * lane + 1];
-    float cf0, sf0, cf1, sf1;
-    {
-        const double n0 = rint(ang0 * kInvTwoPi), n1 = rint(ang1 * kInvTwoPi);
-        sincosf((float)fma(-n0, kTwoPiLo, fma(-n0, kTwoPiHi, ang0)), &sf0, &cf0);
-        sincosf((float)fma(-n1, kTwoPiLo, fma(-n1, kTwoPiHi, ang1)), &sf1, &cf1);
-    }
-    const bool active = g < G;
-    const uint32_t* xq = reinterpret_cast<const uint32_t*>(s.qkv + (G * j + (active ? g : 0)) * (kHeadDim * 2));
+    const int r = lane >> 2, t = lane & 3;
+    const bool active = r < Lay::kRows;
+    const int tt = active ? r / G : 0;          // this row's new token
+    const int head = G * j + (active ? r % G : 0);
+    float cf[T][2], sf[T][2];
+#pragma unroll
+    for (int u = 0; u < T; ++u)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const double ang = (double)(pos0 + u) * s.inv_freq[2 * lane + e];
+            const double n = rint(ang * kInvTwoPi);
+            sincosf((float)fma(-n, kTwoPiLo, fma(-n, kTwoPiHi, ang)), &sf[u][e], &cf[u][e]);
+        }
+    const uint32_t* xq =
+        reinterpret_cast<const uint32_t*>(s.qkv + tt * Lay::kQkvBytes + head * (kHeadDim * 2));
     const uint32_t* gq = reinterpret_cast<const uint32_t*>(s.gains);
     uint32_t xw[16];
     float ss = 0.f;
@@ -235,8 +254,14 @@ __device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s,
         const uint32_t wlo = gq[4 * mp + t], whi = gq[32 + 4 * mp + t];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            const float cs = __shfl_sync(kFull, e ? cf1 : cf0, 4 * mp + t);
-            const float sn = __shfl_sync(kFull, e ? sf1 : sf0, 4 * mp + t);
+            float cs = 0.f, sn = 0.f;
+#pragma unroll
+            for (int u = 0; u < T; ++u) {   // the angle of pair 8*mp + 2t + e at this row's token
+                const float cu = __shfl_sync(kFull, cf[u][e], 4 * mp + t);
+                const float su = __shfl_sync(kFull, sf[u][e], 4 * mp + t);
+                cs = (u == tt) ? cu : cs;
+                sn = (u == tt) ? su : sn;
+            }
             const float ya = (e ? bf_hi(xw[mp]) : bf_lo(xw[mp])) * inv_r * (e ? bf_hi(wlo) : bf_lo(wlo));
             const float yb = (e ? bf_hi(xw[mp + 8]) : bf_lo(xw[mp + 8])) * inv_r * (e ? bf_hi(whi) : bf_lo(whi));
             qa[e] = fmaf(ya, cs, -yb * sn) * scale;   // dim 8*mp + 2t + e
@@ -256,27 +281,31 @@ __device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s,
 
     if (appends) {
         // lane l: dims 2l, 2l+1 (word l of the head) and 64+2l, 65+2l (word 32+l), all in double
-        double cs0, sn0, cs1, sn1;
-        sincos(ang0, &sn0, &cs0);
-        sincos(ang1, &sn1, &cs1);
-        const uint32_t* xk = reinterpret_cast<const uint32_t*>(s.qkv + (Lay::kHq + j) * (kHeadDim * 2));
-        const uint32_t* xv = reinterpret_cast<const uint32_t*>(s.qkv + (Lay::kHq + kNumKvHeads + j) * (kHeadDim * 2));
         const uint32_t* gk = reinterpret_cast<const uint32_t*>(s.gains + kHeadDim);
-        const uint32_t xlo = xk[lane], xhi = xk[32 + lane];
         const uint32_t wk_lo = gk[lane], wk_hi = gk[32 + lane];
-        double a0 = bf_to_d(xlo & 0xFFFFu), a1 = bf_to_d(xlo >> 16);
-        double b0 = bf_to_d(xhi & 0xFFFFu), b1 = bf_to_d(xhi >> 16);
-        const double r = sqrt(warp_sum(a0 * a0 + a1 * a1 + b0 * b0 + b1 * b1) / 128.0 + p.rms_eps);
-        a0 = a0 / r * bf_to_d(wk_lo & 0xFFFFu);
-        a1 = a1 / r * bf_to_d(wk_lo >> 16);
-        b0 = b0 / r * bf_to_d(wk_hi & 0xFFFFu);
-        b1 = b1 / r * bf_to_d(wk_hi >> 16);
-        const double ra0 = a0 * cs0 - b0 * sn0, rb0 = b0 * cs0 + a0 * sn0;
-        const double ra1 = a1 * cs1 - b1 * sn1, rb1 = b1 * cs1 + a1 * sn1;
-        st.k_lo = d_to_bf(ra0) | (d_to_bf(ra1) << 16);
-        st.k_hi = d_to_bf(rb0) | (d_to_bf(rb1) << 16);
-        st.v_lo = xv[lane];
-        st.v_hi = xv[32 + lane];
+#pragma unroll
+        for (int u = 0; u < T; ++u) {
+            double cs0, sn0, cs1, sn1;
+            sincos((double)(pos0 + u) * s.inv_freq[2 * lane], &sn0, &cs0);
+            sincos((double)(pos0 + u) * s.inv_freq[2 * lane + 1], &sn1, &cs1);
+            const uint8_t* row = s.qkv + u * Lay::kQkvBytes;
+            const uint32_t* xk = reinterpret_cast<const uint32_t*>(row + (Lay::kHq + j) * (kHeadDim * 2));
+            const uint32_t* xv = reinterpret_cast<const uint32_t*>(row + (Lay::kHq + kNumKvHeads + j) * (kHeadDim * 2));
+            const uint32_t xlo = xk[lane], xhi = xk[32 + lane];
+            double a0 = bf_to_d(xlo & 0xFFFFu), a1 = bf_to_d(xlo >> 16);
+            double b0 = bf_to_d(xhi & 0xFFFFu), b1 = bf_to_d(xhi >> 16);
+            const double rr = sqrt(warp_sum(a0 * a0 + a1 * a1 + b0 * b0 + b1 * b1) / 128.0 + p.rms_eps);
+            a0 = a0 / rr * bf_to_d(wk_lo & 0xFFFFu);
+            a1 = a1 / rr * bf_to_d(wk_lo >> 16);
+            b0 = b0 / rr * bf_to_d(wk_hi & 0xFFFFu);
+            b1 = b1 / rr * bf_to_d(wk_hi >> 16);
+            const double ra0 = a0 * cs0 - b0 * sn0, rb0 = b0 * cs0 + a0 * sn0;
+            const double ra1 = a1 * cs1 - b1 * sn1, rb1 = b1 * cs1 + a1 * sn1;
+            st.k_lo[u] = d_to_bf(ra0) | (d_to_bf(ra1) << 16);
+            st.k_hi[u] = d_to_bf(rb0) | (d_to_bf(rb1) << 16);
+            st.v_lo[u] = xv[lane];
+            st.v_hi[u] = xv[32 + lane];
+        }
     }
 
 #pragma unroll
@@ -287,10 +316,12 @@ __device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s,
     st.lsum = 0.f;
 }
 
-// Scores, online softmax and value accumulation over one staged page.
-template <int G, bool kFullPage>
-__device__ __forceinline__ void attend_page(const uint8_t* stage, int ntok, int j, int lane, State& st) {
-    const int g = lane >> 2, t = lane & 3;
+// Scores, online softmax and value accumulation over one staged page. Unless
+// kFullPage, this lane's row sees page tokens 0..limit only (its causal
+// limit, which also excludes rows past the sequence).
+template <int G, int T, bool kFullPage>
+__device__ __forceinline__ void attend_page(const uint8_t* stage, int limit, int j, int lane, State<T>& st) {
+    const int r = lane >> 2, t = lane & 3;
     // K rows as the column-major B operand: matrix l/8 = (tokens 0-7 | 8-15) x (dims +0 | +8)
     const uint32_t kaddr = smem_addr(stage + kStageK) + j * (kHeadDim * 2) +
                            ((lane & 7) + ((lane >> 4) << 3)) * kRowPitch + ((lane >> 3) & 1) * 16;
@@ -302,13 +333,13 @@ __device__ __forceinline__ void attend_page(const uint8_t* stage, int ntok, int 
         mma_bf16_16816(c0, st.qa[s], b0, b1);
         mma_bf16_16816(c1, st.qa[s], b2, b3);
     }
-    // head g's scores at tokens 2t, 2t+1, 8+2t, 9+2t (row g plus row g+8)
+    // row r's scores at tokens 2t, 2t+1, 8+2t, 9+2t (accumulator row r plus row r+8)
     float sc[4] = {c0[0] + c0[2], c0[1] + c0[3], c1[0] + c1[2], c1[1] + c1[3]};
     if (!kFullPage) {
-        sc[0] = (2 * t < ntok) ? sc[0] : -INFINITY;
-        sc[1] = (2 * t + 1 < ntok) ? sc[1] : -INFINITY;
-        sc[2] = (8 + 2 * t < ntok) ? sc[2] : -INFINITY;
-        sc[3] = (9 + 2 * t < ntok) ? sc[3] : -INFINITY;
+        sc[0] = (2 * t <= limit) ? sc[0] : -INFINITY;
+        sc[1] = (2 * t + 1 <= limit) ? sc[1] : -INFINITY;
+        sc[2] = (8 + 2 * t <= limit) ? sc[2] : -INFINITY;
+        sc[3] = (9 + 2 * t <= limit) ? sc[3] : -INFINITY;
     }
     float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
     mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
@@ -326,7 +357,8 @@ __device__ __forceinline__ void attend_page(const uint8_t* stage, int ntok, int 
     }
     float pr[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) pr[i] = (sc[i] == -INFINITY || g >= G) ? 0.f : exp2_approx(sc[i] - st.m);
+    for (int i = 0; i < 4; ++i)
+        pr[i] = (sc[i] == -INFINITY || r >= Layout<G, T>::kRows) ? 0.f : exp2_approx(sc[i] - st.m);
     st.lsum += (pr[0] + pr[1]) + (pr[2] + pr[3]);
     uint32_t pa[4];
     {
@@ -335,10 +367,10 @@ __device__ __forceinline__ void attend_page(const uint8_t* stage, int ntok, int 
         split_bf16(pr[1], h1, l1);
         split_bf16(pr[2], h2, l2);
         split_bf16(pr[3], h3, l3);
-        pa[0] = (uint32_t)h1 << 16 | h0;   // row g, tokens 2t, 2t+1
-        pa[1] = (uint32_t)l1 << 16 | l0;   // row g+8
-        pa[2] = (uint32_t)h3 << 16 | h2;   // row g, tokens 8+2t, 9+2t
-        pa[3] = (uint32_t)l3 << 16 | l2;   // row g+8
+        pa[0] = (uint32_t)h1 << 16 | h0;   // row r, tokens 2t, 2t+1
+        pa[1] = (uint32_t)l1 << 16 | l0;   // row r+8
+        pa[2] = (uint32_t)h3 << 16 | h2;   // row r, tokens 8+2t, 9+2t
+        pa[3] = (uint32_t)l3 << 16 | l2;   // row r+8
     }
     // V rows as the column-major B operand (transposed load): matrix l/8 =
     // (tokens 0-7 | 8-15) x (dims +0 | +8)
@@ -353,7 +385,6 @@ __device__ __forceinline__ void attend_page(const uint8_t* stage, int ntok, int 
     }
 }
 
-template <int G>
 __device__ __forceinline__ bool wait_full(const Params& p, const Shared& s, uint64_t* bar, uint32_t phase, int lane) {
     bool ok = mbar_try_wait(bar, phase);
     if (__all_sync(kFull, ok)) return true;
@@ -366,83 +397,98 @@ __device__ __forceinline__ bool wait_full(const Params& p, const Shared& s, uint
     return ok;
 }
 
-template <int G>
-__device__ __forceinline__ void consume_page(const Params& p, const Shared& s, int slot, int i, int nb, int L, int j,
-                                             int lane, State& st) {
+// Attend over the staged page in `slot`: page i of a sequence of length L
+// whose last T slots are the new tokens. New tokens on this page are written
+// to the cache and patched into the staged page first.
+template <int G, int T>
+__device__ __forceinline__ void consume_page(const Params& p, const Shared& s, int slot, int i, int L, int j,
+                                             int lane, State<T>& st) {
     uint8_t* stage = s.stages + slot * kStageBytes;
-    const bool last = (i == nb - 1);
-    const int new_row = (L - 1) - kPage * i;
-    const int ntok = last ? new_row + 1 : kPage;
+    const int first_new = L - T;                    // slot of the first new token
+    const int ntok = min(kPage, L - kPage * i);     // rows of this page inside the sequence
     if (s.meta[slot].bad == 0) {
-        if (last) {
-            // the new token: written to the cache and patched into the staged page
+        if (kPage * i + kPage > first_new) {
+            // new tokens on this page: to the cache and into the staged page
             const int page = s.meta[slot].page;
-            const size_t off =
-                (size_t)page * (kPageBytes / 2) + (size_t)new_row * (kRowBytes / 2) + (size_t)j * kHeadDim;
-            uint32_t* kd = reinterpret_cast<uint32_t*>(p.k_cache + off);
-            uint32_t* vd = reinterpret_cast<uint32_t*>(p.v_cache + off);
-            kd[lane] = st.k_lo;
-            kd[32 + lane] = st.k_hi;
-            vd[lane] = st.v_lo;
-            vd[32 + lane] = st.v_hi;
-            uint32_t* kr = reinterpret_cast<uint32_t*>(stage + kStageK + new_row * kRowPitch + j * kHeadDim * 2);
-            uint32_t* vr = reinterpret_cast<uint32_t*>(stage + kStageV + new_row * kRowPitch + j * kHeadDim * 2);
-            kr[lane] = st.k_lo;
-            kr[32 + lane] = st.k_hi;
-            vr[lane] = st.v_lo;
-            vr[32 + lane] = st.v_hi;
-            // the rows after the new token hold stale bytes; the value product
-            // would turn a stale NaN into NaN even at probability 0, so clear them
-            for (int r = ntok; r < kPage; ++r) {
-                uint32_t* z = reinterpret_cast<uint32_t*>(stage + kStageV + r * kRowPitch + j * kHeadDim * 2);
+#pragma unroll
+            for (int u = 0; u < T; ++u) {
+                const int row = first_new + u - kPage * i;
+                if (row < 0 || row >= kPage) continue;
+                const size_t off =
+                    (size_t)page * (kPageBytes / 2) + (size_t)row * (kRowBytes / 2) + (size_t)j * kHeadDim;
+                uint32_t* kd = reinterpret_cast<uint32_t*>(p.k_cache + off);
+                uint32_t* vd = reinterpret_cast<uint32_t*>(p.v_cache + off);
+                kd[lane] = st.k_lo[u];
+                kd[32 + lane] = st.k_hi[u];
+                vd[lane] = st.v_lo[u];
+                vd[32 + lane] = st.v_hi[u];
+                uint32_t* kr = reinterpret_cast<uint32_t*>(stage + kStageK + row * kRowPitch + j * kHeadDim * 2);
+                uint32_t* vr = reinterpret_cast<uint32_t*>(stage + kStageV + row * kRowPitch + j * kHeadDim * 2);
+                kr[lane] = st.k_lo[u];
+                kr[32 + lane] = st.k_hi[u];
+                vr[lane] = st.v_lo[u];
+                vr[32 + lane] = st.v_hi[u];
+            }
+            // rows after the sequence hold stale bytes; the value product would
+            // turn a stale NaN into NaN even at probability 0, so clear them
+            for (int rr = ntok; rr < kPage; ++rr) {
+                uint32_t* z = reinterpret_cast<uint32_t*>(stage + kStageV + rr * kRowPitch + j * kHeadDim * 2);
                 z[lane] = 0u;
                 z[32 + lane] = 0u;
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
         }
-        if (ntok == kPage) attend_page<G, true>(stage, ntok, j, lane, st);
-        else attend_page<G, false>(stage, ntok, j, lane, st);
+        // this lane's row (new token tt) sees slots <= first_new + tt
+        const int r = lane >> 2;
+        const int tt = r < Layout<G, T>::kRows ? r / G : 0;
+        const int limit = first_new + tt - kPage * i;
+        if (first_new - kPage * i >= kPage) attend_page<G, T, true>(stage, limit, j, lane, st);
+        else attend_page<G, T, false>(stage, limit, j, lane, st);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.empty_bar[slot]);
 }
 
 // End of a sequence piece: o directly when the piece is the whole sequence,
-// else this piece's partial at scratch slot blockIdx.x + b.
-template <int G>
+// else this piece's partial at scratch slot blockIdx.x + b, row t*Hq + head of
+// the slot's kPartRows.
+template <int G, int T>
 __device__ __forceinline__ void finish_piece(const Params& p, const Shared& s, int b, int j, int lane, int per_cta,
-                                             State& st) {
-    using Lay = Layout<G>;
-    const int g = lane >> 2, t = lane & 3;
+                                             State<T>& st) {
+    using Lay = Layout<G, T>;
+    const int r = lane >> 2, t = lane & 3;
     float l = st.lsum;
     l += __shfl_xor_sync(kFull, l, 1);
     l += __shfl_xor_sync(kFull, l, 2);
-    if (g >= G) return;
-    const int head = G * j + g;
+    if (r >= Lay::kRows) return;
+    const int tt = r / G;
+    const int head = G * j + r % G;
     const int part_first = s.seg[b] / per_cta;
     const int part_last = (s.seg[b + 1] - 1) / per_cta;
     if (part_first == part_last) {
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        uint32_t* dst = reinterpret_cast<uint32_t*>(p.o + ((size_t)b * Lay::kHq + head) * kHeadDim);
+        uint32_t* dst = reinterpret_cast<uint32_t*>(p.o + (((size_t)b * T + tt) * Lay::kHq + head) * kHeadDim);
 #pragma unroll
         for (int n = 0; n < 16; ++n)
             dst[4 * n + t] = pack_bf2((st.o[n][0] + st.o[n][2]) * inv, (st.o[n][1] + st.o[n][3]) * inv);
         return;
     }
-    const int slot = blockIdx.x + b;
-    float2* pa = reinterpret_cast<float2*>(p.part_acc + ((size_t)slot * Lay::kHq + head) * kHeadDim);
+    const size_t prow = (size_t)(blockIdx.x + b) * kPartRows + tt * Lay::kHq + head;
+    float2* pa = reinterpret_cast<float2*>(p.part_acc + prow * kHeadDim);
 #pragma unroll
     for (int n = 0; n < 16; ++n) __stcg(pa + 4 * n + t, make_float2(st.o[n][0] + st.o[n][2], st.o[n][1] + st.o[n][3]));
-    if (t == 0) __stcg(p.part_ml + (size_t)slot * Lay::kHq + head, make_float2(st.m, l));
+    if (t == 0) __stcg(p.part_ml + prow, make_float2(st.m, l));
 }
 
-template <int G>
+template <int G, int T>
 __device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, int B, int start, int end, int per_cta,
                                              int warp, int lane) {
+    constexpr int kStages = Layout<G, T>::kStages;
     const int j = warp;
-    State st;
-    st.k_lo = st.k_hi = st.v_lo = st.v_hi = 0u;
+    State<T> st;
+#pragma unroll
+    for (int u = 0; u < T; ++u) st.k_lo[u] = st.k_hi[u] = st.v_lo[u] = st.v_hi[u] = 0u;
     int b = find_seq(s.seg, B, start);
     int i0 = start - s.seg[b];
     int slot = 0;
@@ -453,21 +499,23 @@ __device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, i
         const int nb = s.seg[b + 1] - s.seg[b];
         const int L = s.lens[b];
         const int n_here = min(nb - i0, count - k);
-        if (!wait_full<G>(p, s, s.qkv_full, qphase, lane)) return;
-        begin_sequence<G>(p, s, *s.qkv_pos, j, lane, /*appends=*/s.seg[b + 1] <= end, st);
+        if (!wait_full(p, s, s.qkv_full, qphase, lane)) return;
+        // this CTA appends when it holds a page with one of the new tokens
+        const bool appends = s.seg[b] + (L - T) / kPage < end;
+        begin_sequence<G, T>(p, s, *s.qkv_pos, j, lane, appends, st);
         __syncwarp();
         if (lane == 0) mbar_arrive(s.qkv_empty);
         qphase ^= 1u;
         for (int u = 0; u < n_here; ++u) {
-            if (!wait_full<G>(p, s, &s.full_bar[slot], phase, lane)) return;
-            consume_page<G>(p, s, slot, i0 + u, nb, L, j, lane, st);
+            if (!wait_full(p, s, &s.full_bar[slot], phase, lane)) return;
+            consume_page<G, T>(p, s, slot, i0 + u, L, j, lane, st);
             if (++slot == kStages) {
                 slot = 0;
                 phase ^= 1u;
             }
         }
         k += n_here;
-        finish_piece<G>(p, s, b, j, lane, per_cta, st);
+        finish_piece<G, T>(p, s, b, j, lane, per_cta, st);
         if (k < count) {
             do { ++b; } while (b < B && s.seg[b + 1] == s.seg[b]);
             i0 = 0;
@@ -475,9 +523,10 @@ __device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, i
     }
 }
 
-template <int G>
+template <int G, int T>
 __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Params p) {
-    using Lay = Layout<G>;
+    using Lay = Layout<G, T>;
+    constexpr int kStages = Lay::kStages;
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -500,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
     const int B = p.batch;
     for (int b = threadIdx.x; b < B; b += kThreads) {
         const int L = p.seq_lens[b];
-        const bool ok = L >= 1 && L <= p.max_seq_len && L <= kPage * p.bt_stride;
+        const bool ok = L >= T && L <= p.max_seq_len && L <= kPage * p.bt_stride;
         if (!ok && blockIdx.x == 0) record_error(p.status, QDA_ERR_BOUNDS);
         s.lens[b] = L;
         s.seg[b + 1] = ok ? (L + kPage - 1) / kPage : 0;
@@ -557,8 +606,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
     const int start = (int)blockIdx.x * per_cta;
     const int end = min(start + per_cta, total);
     if (start < end) {
-        if (warp == kConsumerWarps) run_producer<G>(p, s, B, start, end, lane);
-        else run_consumer<G>(p, s, B, start, end, per_cta, warp, lane);
+        if (warp == kConsumerWarps) run_producer<G, T>(p, s, B, start, end, lane);
+        else run_consumer<G, T>(p, s, B, start, end, per_cta, warp, lane);
     }
     if ((p.flags & QDA_FLAG_INJECT_WAIT_TIMEOUT) != 0u && blockIdx.x == 0 && warp == 0) {
         if (!mbar_wait(s.never_bar, 0u, p.timeout_ns, nullptr) && lane == 0) record_error(p.status, QDA_ERR_TIMEOUT);
@@ -566,35 +615,37 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
     pdl_launch_dependents();
 }
 
-// Combine the partials of one split sequence (blockIdx.x) for the G query
-// heads of one kv head (blockIdx.y): warp g handles head G*y + g and lane l
-// its dims 4l..4l+3; o = sum_t 2^(m_t - M) acc_t / sum_t 2^(m_t - M) l_t with
-// M = max_t m_t. Sequences held whole by one CTA were written by the first
-// launch and are skipped.
-template <int G>
-__global__ void __launch_bounds__(32 * G) combine_kernel(const Params p, int main_grid) {
-    using Lay = Layout<G>;
+// Combine the partials of one split sequence (blockIdx.x) for the query rows
+// of one kv head (blockIdx.y): warp w handles new token w / G, head
+// G*y + w % G, and lane l its dims 4l..4l+3; o = sum_t 2^(m_t - M) acc_t /
+// sum_t 2^(m_t - M) l_t with M = max_t m_t. Sequences held whole by one CTA
+// were written by the first launch and are skipped.
+template <int G, int T>
+__global__ void __launch_bounds__(32 * G * T, 1) combine_kernel(const Params p, int main_grid) {
+    using Lay = Layout<G, T>;
     pdl_wait();   // the first launch has finished and its writes are visible
     const int b = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = G * blockIdx.y + warp;
+    const int tt = warp / G;
+    const int h = G * blockIdx.y + warp % G;
     const int lo = p.seg[b], hi = p.seg[b + 1], total = p.seg[p.batch];
     if (hi == lo) return;   // a sequence the first launch skipped
     const int per_cta = (total + main_grid - 1) / main_grid;
     const int first = lo / per_cta, n = (hi - 1) / per_cta - first + 1;
     if (n == 1) return;
-    const float2* ml = p.part_ml + (size_t)(first + b) * Lay::kHq + h;   // piece t at ml[t * kHq]
+    const size_t row0 = (size_t)(first + b) * kPartRows + tt * Lay::kHq + h;   // piece t at row0 + t*kPartRows
+    const float2* ml = p.part_ml + row0;
     float M = -INFINITY;
-    for (int t = lane; t < n; t += 32) M = fmaxf(M, __ldcg(ml + (size_t)t * Lay::kHq).x);
+    for (int t = lane; t < n; t += 32) M = fmaxf(M, __ldcg(ml + (size_t)t * kPartRows).x);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
-    const float4* src = reinterpret_cast<const float4*>(p.part_acc + ((size_t)(first + b) * Lay::kHq + h) * kHeadDim) + lane;
-    constexpr size_t kSlotStride = (size_t)Lay::kHq * kHeadDim / 4;   // float4 per scratch slot
+    const float4* src = reinterpret_cast<const float4*>(p.part_acc + row0 * kHeadDim) + lane;
+    constexpr size_t kSlotStride = (size_t)kPartRows * kHeadDim / 4;   // float4 per scratch slot
     float Ls = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int t0 = 0; t0 < n; t0 += 32) {
         float wt = 0.f;
         if (t0 + lane < n) {
-            const float2 v = __ldcg(ml + (size_t)(t0 + lane) * Lay::kHq);
+            const float2 v = __ldcg(ml + (size_t)(t0 + lane) * kPartRows);
             wt = (v.x == -INFINITY) ? 0.f : exp2_approx(v.x - M);   // a piece whose pages were all skipped
             Ls = fmaf(wt, v.y, Ls);
         }
@@ -622,23 +673,23 @@ __global__ void __launch_bounds__(32 * G) combine_kernel(const Params p, int mai
     uint2 out;
     out.x = pack_bf2(acc.x * inv, acc.y * inv);
     out.y = pack_bf2(acc.z * inv, acc.w * inv);
-    reinterpret_cast<uint2*>(p.o + ((size_t)b * Lay::kHq + h) * kHeadDim)[lane] = out;
+    reinterpret_cast<uint2*>(p.o + (((size_t)b * T + tt) * Lay::kHq + h) * kHeadDim)[lane] = out;
 }
 
-template <int G>
+template <int G, int T>
 cudaError_t prepare_one() {
-    return cudaFuncSetAttribute(grouped_attention_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                Layout<G>::kSmemTotal);
+    return cudaFuncSetAttribute(grouped_attention_kernel<G, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Layout<G, T>::kSmemTotal);
 }
 
-template <int G>
+template <int G, int T>
 cudaError_t launch_one(const Params& p, int grid, cudaStream_t stream) {
-    grouped_attention_kernel<G><<<grid, kThreads, Layout<G>::kSmemTotal, stream>>>(p);
+    grouped_attention_kernel<G, T><<<grid, kThreads, Layout<G, T>::kSmemTotal, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p.batch, (unsigned)kNumKvHeads, 1);
-    cfg.blockDim = dim3(32 * G, 1, 1);
+    cfg.blockDim = dim3(32 * G * T, 1, 1);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -646,23 +697,37 @@ cudaError_t launch_one(const Params& p, int grid, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, combine_kernel<G>, p, grid);
+    return cudaLaunchKernelEx(&cfg, combine_kernel<G, T>, p, grid);
 }
 
 }  // namespace
 
 cudaError_t prepare_grouped() {
-    cudaError_t e = prepare_one<4>();
-    if (e == cudaSuccess) e = prepare_one<5>();
-    if (e == cudaSuccess) e = prepare_one<8>();
+    cudaError_t e = prepare_one<4, 1>();
+    if (e == cudaSuccess) e = prepare_one<5, 1>();
+    if (e == cudaSuccess) e = prepare_one<8, 1>();
+    if (e == cudaSuccess) e = prepare_one<2, 2>();
+    if (e == cudaSuccess) e = prepare_one<2, 3>();
+    if (e == cudaSuccess) e = prepare_one<2, 4>();
+    if (e == cudaSuccess) e = prepare_one<4, 2>();
     return e;
 }
 
+bool grouped_supported(int num_q_heads, int new_tokens) {
+    const int G = num_q_heads / kNumKvHeads;
+    if (new_tokens == 1) return G == 4 || G == 5 || G == 8;
+    return (G == 2 && new_tokens >= 2 && new_tokens <= 4) || (G == 4 && new_tokens == 2);
+}
+
 cudaError_t launch_grouped(const Params& p, int grid, cudaStream_t stream) {
-    switch (p.num_q_heads) {
-        case 32: return launch_one<4>(p, grid, stream);
-        case 40: return launch_one<5>(p, grid, stream);
-        case 64: return launch_one<8>(p, grid, stream);
+    switch (p.num_q_heads * 16 + p.new_tokens) {
+        case 32 * 16 + 1: return launch_one<4, 1>(p, grid, stream);
+        case 40 * 16 + 1: return launch_one<5, 1>(p, grid, stream);
+        case 64 * 16 + 1: return launch_one<8, 1>(p, grid, stream);
+        case 16 * 16 + 2: return launch_one<2, 2>(p, grid, stream);
+        case 16 * 16 + 3: return launch_one<2, 3>(p, grid, stream);
+        case 16 * 16 + 4: return launch_one<2, 4>(p, grid, stream);
+        case 32 * 16 + 2: return launch_one<4, 2>(p, grid, stream);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -36,8 +36,9 @@ struct Params {
     const int32_t* block_table;   // [B][bt_stride]
     uint16_t* k_cache;            // bf16 [num_pages][16][8][128]
     uint16_t* v_cache;
-    uint16_t* o;                  // bf16 [B][num_q_heads][128]
+    uint16_t* o;                  // bf16 [B][new_tokens][num_q_heads][128]
     int num_q_heads;              // 16, 32, 40 or 64
+    int new_tokens;               // new tokens per sequence (qkv is [B][new_tokens][...])
     int bt_stride;
     int num_pages;
     int batch;
@@ -45,8 +46,9 @@ struct Params {
     double rope_theta;
     double rms_eps;
     // workspace
-    float* part_acc;              // [num_slots][num_q_heads][128] un-normalised partial sums
-    float2* part_ml;              // [num_slots][num_q_heads] (running max in log2 units, sum)
+    float* part_acc;              // [num_slots][rows][128] un-normalised partial sums; rows = 16 for the
+                                  // 16-head kernel, kPartRows for the tensor-core kernel
+    float2* part_ml;              // [num_slots][rows] (running max in log2 units, sum)
     int* seg;                     // [kMaxBatch + 1] page offsets of the sequences (written for the combine
                                   // launch of the 32/40/64-head kernels; unused at 16 heads)
     int* counters;                // [kMaxBatch][8] merge arrival counters, zero between calls
@@ -55,7 +57,11 @@ struct Params {
     unsigned flags;
 };
 
-// Scratch a launch with `grid` CTAs and batches up to `max_batch` needs.
+// Partial rows per scratch slot of the tensor-core kernel: new tokens x query
+// heads, at most 8 rows per kv head.
+constexpr int kPartRows = 8 * kNumKvHeads;
+
+// Scratch slots a launch with `grid` CTAs and batches up to `max_batch` needs.
 inline int64_t num_slots(int grid, int max_batch) { return (int64_t)grid + max_batch; }
 
 // Dynamic shared memory of one CTA.
@@ -68,11 +74,15 @@ cudaError_t prepare_device();
 // Launch one decode-attention step with `grid` CTAs on `stream` (16 query heads).
 cudaError_t launch(const Params& p, int grid, cudaStream_t stream);
 
-// The step at 32, 40 or 64 query heads: the attention launch, then a launch
-// that combines the partials of sequences split across CTAs.
+// The tensor-core step (32, 40 or 64 query heads with one new token; 16
+// heads with 2..4 new tokens, 32 heads with 2): the attention launch, then a
+// launch that combines the partials of sequences split across CTAs.
 cudaError_t launch_grouped(const Params& p, int grid, cudaStream_t stream);
 
-// Prepare the 32/40/64-head kernels on the current device.
+// Whether the tensor-core kernel has an instance for this head and token count.
+bool grouped_supported(int num_q_heads, int new_tokens);
+
+// Prepare the tensor-core kernels on the current device.
 cudaError_t prepare_grouped();
 
 }  // namespace qda

@@ -106,6 +106,7 @@ extern "C" int qwen3_decode_attn_append_and_attend_noalloc(const void* qkv, cons
     p.v_cache = static_cast<uint16_t*>(v_cache);
     p.o = static_cast<uint16_t*>(o);
     p.num_q_heads = qda::kNumQHeads;
+    p.new_tokens = 1;
     p.bt_stride = block_table_stride;
     p.num_pages = num_pages;
     p.batch = batch;

@@ -91,6 +91,7 @@ extern "C" {
 #define QDA_QKV_WIDTH     4096
 #define QDA_MAX_BATCH     256
 #define QDA_MAX_SEQ_LEN   40960
+#define QDA_MAX_NEW_TOKENS 4   /* new tokens per sequence of one call */
 
 /* Return codes. */
 #define QDA_OK               0
@@ -172,6 +173,40 @@ int qwen3_decode_attn_append_and_attend(qda_handle *h,
                                         void *o,
                                         int batch,
                                         void *cuda_stream);
+
+/* The step with T = new_tokens new tokens per sequence (several tokens
+ * decoded at once, e.g. draft tokens to verify). Model Spec, "Compute-graph
+ * nodes" (attn.qk_norm, attn.rope, attn.core, the paged append) applied to T
+ * tokens, under "What to watch for": every layer is full causal attention.
+ * Layouts: qkv is bf16 [B][T][(Hq + 16) * 128] (token t of sequence b at row
+ * b*T + t); o is bf16 [B][T][Hq][128]. seq_lens[b] = L counts the T new
+ * tokens, and L >= T. Token t is appended at cache slot L - T + t, with RoPE
+ * position positions[b] + t (or L - T + t when positions is NULL), and its
+ * query attends over slots 0 .. L - T + t: the cache before the call plus the
+ * new tokens up to and including itself.
+ * new_tokens = 1 is exactly qwen3_decode_attn_append_and_attend. For T > 1 the
+ * compiled instances are 16 query heads with T = 2, 3 or 4 and 32 query heads
+ * with T = 2 (at most 8 query rows per kv head); every call is two launches
+ * (attention, then the combine of split sequences).
+ * Errors as for qwen3_decode_attn_append_and_attend, plus INVALID_ARG for
+ * new_tokens outside [1, QDA_MAX_NEW_TOKENS] and UNSUPPORTED for a (query
+ * heads, new_tokens) pair with no instance; on the device, a seq_len below T
+ * is out of range like one above the limits. */
+int qwen3_decode_attn_append_and_attend_tokens(qda_handle *h,
+                                               const void *qkv,
+                                               const void *q_norm_w,
+                                               const void *k_norm_w,
+                                               const int32_t *seq_lens,
+                                               const int32_t *positions,
+                                               const int32_t *block_table,
+                                               int block_table_stride,
+                                               void *k_cache,
+                                               void *v_cache,
+                                               int num_pages,
+                                               void *o,
+                                               int batch,
+                                               int new_tokens,
+                                               void *cuda_stream);
 
 /* The same step for a caller whose per-step tensors are in HOST memory:
  * qkv_host, seq_lens_host, positions_host (or NULL) and block_table_host are

@@ -36,22 +36,38 @@ def run(attn, w: inputs.Workload, dev, k_cache, v_cache, positions=None, o=None)
     return o
 
 
+def _qkv3(w: inputs.Workload) -> np.ndarray:
+    """qkv bits as [B, T, W] (T = 1 for a single new token)."""
+    bits = inputs.bf16_bits(w.qkv)
+    return bits.reshape(w.batch, w.new_tokens, -1)
+
+
+def _o_shape(w: inputs.Workload, o: np.ndarray) -> np.ndarray:
+    """The oracle's [B, T, Hq, 128] o in the layout of the call: [B, Hq, 128] when T = 1."""
+    return o[:, 0] if w.qkv.dim() == 2 else o
+
+
 def oracle_full(w: inputs.Workload, k_cache_pre, v_cache_pre, positions=None):
     """The oracle on the whole batch; caches given as tensors (any device), pre-call."""
     pos = positions if positions is not None else w.positions
-    return oracle.append_and_attend(
-        inputs.bf16_bits(w.qkv), inputs.bf16_bits(w.q_norm_w), inputs.bf16_bits(w.k_norm_w),
+    out = oracle.append_and_attend_tokens(
+        _qkv3(w), inputs.bf16_bits(w.q_norm_w), inputs.bf16_bits(w.k_norm_w),
         w.seq_lens.numpy(), w.block_table.numpy(), inputs.bf16_bits(k_cache_pre), inputs.bf16_bits(v_cache_pre),
         positions=None if pos is None else pos.cpu().numpy(), inplace=True, want_qk=True)
+    out["o"] = _o_shape(w, out["o"])
+    return out
 
 
-def _compact(w, seqs, k_pre, v_pre, last_page_only=False):
-    """A sub-batch of the sequences `seqs` over a pool holding only their pages."""
+def _compact(w, seqs, k_pre, v_pre, tail_only=False):
+    """A sub-batch of the sequences `seqs` over a pool holding only their pages
+    (with `tail_only`, only the pages from the one holding the first new token)."""
     lens = w.seq_lens[seqs]
+    T = w.new_tokens
     rows, pages = [], []
     for b in seqs.tolist():
-        n = (int(w.seq_lens[b]) + 15) // 16
-        ids = w.block_table[b, n - 1:n] if last_page_only else w.block_table[b, :n]
+        L = int(w.seq_lens[b])
+        n = (L + 15) // 16
+        ids = w.block_table[b, (L - T) // 16:n] if tail_only else w.block_table[b, :n]
         rows.append(torch.arange(len(pages), len(pages) + len(ids), dtype=torch.int32))
         pages.extend(ids.tolist())
     stride = max(len(r) for r in rows)
@@ -65,45 +81,58 @@ def _compact(w, seqs, k_pre, v_pre, last_page_only=False):
 
 
 def oracle_sampled(w: inputs.Workload, seqs, k_pre, v_pre):
-    """Oracle o for the sequences `seqs` only ([len(seqs), 16, 128] float64)."""
+    """Oracle o for the sequences `seqs` only ([len(seqs), (T,) Hq, 128] float64)."""
     seqs = torch.as_tensor(seqs, dtype=torch.int64)
     lens, bt, kc, vc = _compact(w, seqs, k_pre, v_pre)
     pos = None if w.positions is None else w.positions[seqs].numpy()
-    out = oracle.append_and_attend(
-        inputs.bf16_bits(w.qkv[seqs.to(w.qkv.device)]), inputs.bf16_bits(w.q_norm_w),
+    out = oracle.append_and_attend_tokens(
+        _qkv3(w)[seqs.numpy()], inputs.bf16_bits(w.q_norm_w),
         inputs.bf16_bits(w.k_norm_w), lens.numpy(), bt.numpy(), kc, vc, positions=pos, inplace=True)
-    return out["o"]
+    return _o_shape(w, out["o"])
+
+
+def _new_slots(w: inputs.Workload):
+    """(b, t, page, row) of every appended token: token t of sequence b goes to slot L - T + t."""
+    T = w.new_tokens
+    for b in range(w.batch):
+        L = int(w.seq_lens[b])
+        for t in range(T):
+            slot = L - T + t
+            yield b, t, int(w.block_table[b, slot // 16]), slot % 16
 
 
 def oracle_appended_rows(w: inputs.Workload, k_pre, v_pre):
     """The oracle's appended k/v rows for every sequence, cheaply: each sequence is
-    replaced by its last page alone, with its true RoPE position.
+    replaced by its pages from the first new token's on, with its true RoPE
+    positions.
 
-    Returns (k_rows, v_rows) uint16 [B, 8, 128] and k64, the new k in float64.
+    Returns (k_rows, v_rows) uint16 [B, T, 8, 128] and k64, the new k in float64.
     """
-    B = w.batch
+    B, T = w.batch, w.new_tokens
     seqs = torch.arange(B)
-    lens, bt, kc, vc = _compact(w, seqs, k_pre, v_pre, last_page_only=True)
-    short = ((lens - 1) % 16 + 1).to(torch.int32)
-    pos = (w.seq_lens - 1) if w.positions is None else w.positions
-    out = oracle.append_and_attend(
-        inputs.bf16_bits(w.qkv), inputs.bf16_bits(w.q_norm_w), inputs.bf16_bits(w.k_norm_w), short.numpy(),
+    lens, bt, kc, vc = _compact(w, seqs, k_pre, v_pre, tail_only=True)
+    short = (lens - (lens - T) // 16 * 16).to(torch.int32)
+    pos = (w.seq_lens - T) if w.positions is None else w.positions
+    out = oracle.append_and_attend_tokens(
+        _qkv3(w), inputs.bf16_bits(w.q_norm_w), inputs.bf16_bits(w.k_norm_w), short.numpy(),
         bt.numpy(), kc, vc, positions=pos.numpy().astype(np.int32), inplace=True, want_qk=True)
-    rows = ((short - 1) % 16).numpy()
-    k_rows = np.stack([out["k_cache"][b, rows[b]] for b in range(B)])
-    v_rows = np.stack([out["v_cache"][b, rows[b]] for b in range(B)])
+    k_rows = np.empty((B, T, 8, 128), np.uint16)
+    v_rows = np.empty((B, T, 8, 128), np.uint16)
+    for b in range(B):
+        for t in range(T):
+            slot = int(short[b]) - T + t
+            k_rows[b, t] = out["k_cache"][bt[b, slot // 16], slot % 16]
+            v_rows[b, t] = out["v_cache"][bt[b, slot // 16], slot % 16]
     return k_rows, v_rows, out["k"]
 
 
 def expected_cache(w: inputs.Workload, k_pre, v_pre, k_rows, v_rows):
-    """The pre-call caches (device) with each sequence's appended row written in."""
+    """The pre-call caches (device) with each sequence's appended rows written in."""
     k_exp, v_exp = k_pre.clone(), v_pre.clone()
     dev = k_pre.device
-    for b in range(w.batch):
-        L = int(w.seq_lens[b])
-        page, row = int(w.block_table[b, (L - 1) // 16]), (L - 1) % 16
-        k_exp[page, row] = torch.from_numpy(k_rows[b].view(np.int16)).view(torch.bfloat16).to(dev)
-        v_exp[page, row] = torch.from_numpy(v_rows[b].view(np.int16)).view(torch.bfloat16).to(dev)
+    for b, t, page, row in _new_slots(w):
+        k_exp[page, row] = torch.from_numpy(k_rows[b, t].view(np.int16)).view(torch.bfloat16).to(dev)
+        v_exp[page, row] = torch.from_numpy(v_rows[b, t].view(np.int16)).view(torch.bfloat16).to(dev)
     return k_exp, v_exp
 
 
@@ -126,13 +155,13 @@ def assert_cache_equal(k_got, v_got, k_exp, v_exp, k64=None, w=None):
         return
     msg = "cache differs from the oracle"
     if k64 is not None and w is not None:
-        gb, wb = [], []
-        for b in range(w.batch):
-            L = int(w.seq_lens[b])
-            page, row = int(w.block_table[b, (L - 1) // 16]), (L - 1) % 16
-            gb.append(inputs.bf16_bits(k_got[page, row]))
-            wb.append(inputs.bf16_bits(k_exp[page, row]))
-        msg += "\n" + describe_k_mismatch(np.stack(gb), np.stack(wb), k64)
+        T = w.new_tokens
+        gb = np.empty((w.batch, T, 8, 128), np.uint16)
+        wb = np.empty((w.batch, T, 8, 128), np.uint16)
+        for b, t, page, row in _new_slots(w):
+            gb[b, t] = inputs.bf16_bits(k_got[page, row])
+            wb[b, t] = inputs.bf16_bits(k_exp[page, row])
+        msg += "\n" + describe_k_mismatch(gb, wb, k64.reshape(gb.shape))
     kd = (k_got.view(torch.int16) != k_exp.view(torch.int16)).nonzero()[:5].tolist()
     vd = (v_got.view(torch.int16) != v_exp.view(torch.int16)).nonzero()[:5].tolist()
     raise AssertionError(f"{msg}; first k diffs {kd}, v diffs {vd}")

@@ -121,6 +121,8 @@ def test_calls_on_a_null_handle_are_rejected(lib):
     i32 = ctypes.cast(p, ctypes.POINTER(ctypes.c_int32))
     for fn in (lib.qwen3_decode_attn_append_and_attend, lib.qwen3_decode_attn_append_and_attend_host):
         assert fn(None, p, p, p, i32, None, i32, 1, p, p, 1, p, 1, None) == binding.QDA_ERR_INVALID_ARG
+    assert lib.qwen3_decode_attn_append_and_attend_tokens(None, p, p, p, i32, None, i32, 1, p, p, 1, p, 1, 2,
+                                                          None) == binding.QDA_ERR_INVALID_ARG
     assert lib.qwen3_decode_attn_check(None, None) == binding.QDA_ERR_INVALID_ARG
     assert lib.qwen3_decode_attn_grid_ctas(None) == 0
     lib.qwen3_decode_attn_destroy(None)

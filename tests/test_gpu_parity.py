@@ -268,8 +268,8 @@ def test_config3_all_layers(attn):
             del k_exp, v_exp
         for b in range(w.batch):
             page, row = int(w.block_table[b, 127]), 15
-            assert np.array_equal(inputs.bf16_bits(w.k_cache[page, row]), k_rows[b])
-            assert np.array_equal(inputs.bf16_bits(w.v_cache[page, row]), v_rows[b])
+            assert np.array_equal(inputs.bf16_bits(w.k_cache[page, row]), k_rows[b, 0])
+            assert np.array_equal(inputs.bf16_bits(w.v_cache[page, row]), v_rows[b, 0])
         sample = torch.randint(0, 256, (8,), generator=g).tolist()
         # the oracle reads the pre-call cache; rows other than the appended ones are unchanged
         ref = ph.oracle_sampled(w, sample, w.k_cache, w.v_cache)

@@ -1,0 +1,218 @@
+"""Parity of the step with several new tokens per sequence (T = 2..4, causal
+inside the new block) with the float64 oracle, through the C ABI.
+
+Token t of sequence b goes to cache slot L - T + t (L = seq_lens[b] counts the
+new tokens) and its query attends over slots 0 .. L - T + t (Qwen3-0.6B Model
+Spec, "What to watch for": every layer is full causal attention). The checks
+are those of the one-token step: the whole cache bit for bit, o within the
+gate and the strict bound.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from decode_attention_qk_b200 import binding, inputs
+import parity_helpers as ph
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda", 0)
+CASES = list(binding.SUPPORTED_MULTI_TOKEN)   # (query heads, new tokens)
+
+
+@pytest.fixture(scope="module")
+def handles():
+    from decode_attention_qk_b200 import build
+    build.build_library()
+    hs = {hq: binding.DecodeAttention(device=0, num_q_heads=hq) for hq in (16, 32)}
+    yield hs
+    for h in hs.values():
+        h.close()
+
+
+def full_check(attn, w, label, positions=None):
+    k, v = w.k_cache.to(DEV), w.v_cache.to(DEV)
+    ref = ph.oracle_full(w, k, v, positions=positions)
+    o = ph.run(attn, w, DEV, k, v, positions=positions)
+    assert attn.check() == 0
+    assert o.shape == (w.batch, w.new_tokens, w.num_q_heads, 128)
+    got_k, got_v = inputs.bf16_bits(k), inputs.bf16_bits(v)
+    if not np.array_equal(got_k, ref["k_cache"]):
+        bad = np.argwhere(got_k != ref["k_cache"])[:8].tolist()
+        raise AssertionError(f"{label}: k cache differs at {bad}")
+    assert np.array_equal(got_v, ref["v_cache"]), f"{label}: v cache differs"
+    ph.assert_o_close(o, ref["o"], label)
+    return o, ref
+
+
+@pytest.mark.parametrize("hq,T", CASES)
+def test_page_edges(handles, hq, T):
+    """New blocks that start, end or straddle a page boundary."""
+    lens = [T, T + 1, 15, 16, 17, 18, 19, 20, 31, 32, 33, 34, 64, 65, 300, 1000]
+    w = inputs.custom(lens, seed=60 + 4 * hq + T, device="cuda", gap_fraction=0.2, num_q_heads=hq, new_tokens=T)
+    full_check(handles[hq], w, f"Hq={hq} T={T} page edges")
+
+
+@pytest.mark.parametrize("hq,T", CASES)
+def test_an_empty_cache_gives_the_first_token_its_own_v(handles, hq, T):
+    """L = T: the first new token sees only itself, so its o is its v, bit for bit."""
+    w = inputs.custom([T] * 5, seed=61, device="cuda", num_q_heads=hq, new_tokens=T)
+    o, _ = full_check(handles[hq], w, f"Hq={hq} T={T} L=T")
+    G = hq // 8
+    v0 = w.qkv[:, 0, (hq + 8) * 128:].reshape(5, 8, 1, 128).expand(5, 8, G, 128).reshape(5, hq, 128)
+    assert torch.equal(o[:, 0].contiguous().view(torch.int16), v0.contiguous().view(torch.int16))
+
+
+@pytest.mark.parametrize("hq", [16, 32])
+def test_one_token_through_the_tokens_entry_is_the_decode_step(handles, hq):
+    """new_tokens = 1 is the one-token step: same o and cache bits."""
+    w = inputs.custom([1, 17, 300, 45], seed=62, device="cuda", num_q_heads=hq)
+    k1, v1 = w.k_cache.clone(), w.v_cache.clone()
+    k2, v2 = w.k_cache.clone(), w.v_cache.clone()
+    o1 = ph.run(handles[hq], w, DEV, k1, v1)
+    o2 = ph.run(handles[hq], dataclasses.replace(w, qkv=w.qkv[:, None].contiguous()), DEV, k2, v2)
+    assert handles[hq].check() == 0
+    assert o2.shape == (4, 1, hq, 128)
+    assert torch.equal(o1.view(torch.int16), o2[:, 0].view(torch.int16))
+    assert torch.equal(k1.view(torch.int16), k2.view(torch.int16))
+    assert torch.equal(v1.view(torch.int16), v2.view(torch.int16))
+
+
+@pytest.mark.parametrize("hq,T", [(16, 4), (32, 2)])
+def test_successive_one_token_steps_append_the_same_rows(handles, hq, T):
+    """T one-token calls (L growing by one) leave the same cache bits as one
+    T-token call, and the last one's o equals the T-token call's last row
+    within the tolerance (two different kernels)."""
+    lens = torch.tensor([T, 16, 17, 40, 333], dtype=torch.int32)
+    w = inputs.custom(lens, seed=63, device="cuda", num_q_heads=hq, new_tokens=T)
+    ks, vs = w.k_cache.clone(), w.v_cache.clone()
+    for t in range(T):
+        wt = dataclasses.replace(w, qkv=w.qkv[:, t].contiguous(), seq_lens=lens - (T - 1 - t))
+        o_last = ph.run(handles[hq], wt, DEV, ks, vs)
+    km, vm = w.k_cache.clone(), w.v_cache.clone()
+    o = ph.run(handles[hq], w, DEV, km, vm)
+    assert handles[hq].check() == 0
+    assert torch.equal(ks.view(torch.int16), km.view(torch.int16))
+    assert torch.equal(vs.view(torch.int16), vm.view(torch.int16))
+    ref = ph.oracle_full(w, w.k_cache, w.v_cache)["o"]
+    ph.assert_o_close(o, ref, f"Hq={hq} T={T}")
+    ph.assert_o_close(o_last, ref[:, T - 1], f"Hq={hq} last of {T} single steps")
+
+
+@pytest.mark.parametrize("grid", [1, 3, 148, 1024])
+def test_split_count_does_not_change_the_result(grid):
+    """Any cut of the key range, including cuts inside the new block (then two
+    CTAs each append the new rows on their own pages)."""
+    a = binding.DecodeAttention(device=0, grid_ctas=grid)
+    w = inputs.custom([4, 16, 17, 18, 19, 300, 2000, 33], seed=64, device="cuda", gap_fraction=0.2, new_tokens=4)
+    full_check(a, w, f"T=4 grid {grid}")
+    a.close()
+
+
+def test_positions_argument(handles):
+    full_check(handles[16], inputs.custom([5, 100, 1234], seed=65, device="cuda", new_tokens=3),
+               "T=3 positions", positions=torch.tensor([0, 7000, 40000], dtype=torch.int32))
+
+
+def test_maximum_context(handles):
+    w = inputs.custom([40960, 40959, 7], seed=66, device="cuda", stride=2560, new_tokens=4)
+    full_check(handles[16], w, "T=4 L=40960")
+
+
+def test_locality_with_nan_in_unread_bytes(handles):
+    """The new tokens' rows (written, never read before), rows past a sequence,
+    pages it does not own and table entries past its last page may hold
+    anything (here NaN): o and the appended rows do not change."""
+    attn, T = handles[16], 4
+    w = inputs.custom([7, 12, 40, 16, 18], seed=67, device="cuda", pool_pages=16, stride=6, new_tokens=T)
+    ka, va = w.k_cache.clone(), w.v_cache.clone()
+    kb, vb = w.k_cache.clone(), w.v_cache.clone()
+    bt2 = w.block_table.clone()
+    used, slots = set(), []
+    for b, L in enumerate(w.seq_lens.tolist()):
+        n = (L + 15) // 16
+        used.update(w.block_table[b, :n].tolist())
+        for s in range(L - T, 16 * n):
+            page, row = int(w.block_table[b, s // 16]), s % 16
+            kb[page, row] = float("nan")
+            vb[page, row] = float("nan")
+            if s < L:
+                slots.append((page, row))
+        bt2[b, n:] = 10 ** 6
+    for p in range(w.num_pages):
+        if p not in used:
+            kb[p] = float("nan")
+            vb[p] = float("nan")
+    o1 = ph.run(attn, w, DEV, ka, va)
+    o2 = ph.run(attn, dataclasses.replace(w, block_table=bt2), DEV, kb, vb)
+    assert attn.check() == 0
+    assert not torch.isnan(o2.float()).any()
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    for page, row in slots:
+        assert torch.equal(ka[page, row].view(torch.int16), kb[page, row].view(torch.int16))
+        assert torch.equal(va[page, row].view(torch.int16), vb[page, row].view(torch.int16))
+
+
+def test_a_sequence_shorter_than_the_new_block_is_skipped(handles):
+    """seq_lens[b] < T is out of range on the device: that sequence is skipped
+    (its cache untouched), the others are computed, and the status says BOUNDS."""
+    attn = handles[16]
+    w = inputs.custom([40, 3, 30], seed=68, device="cuda", new_tokens=4)
+    lens = w.seq_lens.clone()
+    k, v = w.k_cache.clone(), w.v_cache.clone()
+    k0, v0 = w.k_cache.clone(), w.v_cache.clone()
+    o = ph.run(attn, w, DEV, k, v)
+    assert attn.check() == binding.QDA_ERR_BOUNDS
+    ref = ph.oracle_sampled(w, [0, 2], w.k_cache, w.v_cache)
+    ph.assert_o_close(o[[0, 2]], ref, "T=4 with a short sequence")
+    page1 = int(w.block_table[1, 0])
+    assert torch.equal(k[page1].view(torch.int16), k0[page1].view(torch.int16))
+    assert torch.equal(v[page1].view(torch.int16), v0[page1].view(torch.int16))
+    assert int(lens[1]) == 3
+    assert attn.check() == 0
+
+
+def test_host_side_errors(handles):
+    w = inputs.custom([20, 30], seed=69, device="cuda", new_tokens=2)
+    a = ph.device_args(w, DEV)
+    call = lambda h, qkv, o: binding.qwen3_decode_attn_append_and_attend_tokens(
+        h, qkv, a["q_norm_w"], a["k_norm_w"], a["seq_lens"], None, a["block_table"], w.k_cache, w.v_cache, o)
+    h40 = binding.DecodeAttention(device=0, num_q_heads=40)
+    w40 = inputs.custom([20, 30], seed=69, device="cuda", num_q_heads=40, new_tokens=2)
+    with pytest.raises(binding.QdaError) as e:
+        call(h40.handle, w40.qkv, torch.empty((2, 2, 40, 128), dtype=torch.bfloat16, device=DEV))
+    assert e.value.code == binding.QDA_ERR_UNSUPPORTED
+    h40.close()
+    qkv5 = torch.zeros((2, 5, 4096), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(binding.QdaError) as e:
+        call(handles[16].handle, qkv5, torch.empty((2, 5, 16, 128), dtype=torch.bfloat16, device=DEV))
+    assert e.value.code == binding.QDA_ERR_INVALID_ARG
+    with pytest.raises(ValueError):   # several tokens are not taken by the one-token entry point
+        binding.qwen3_decode_attn_append_and_attend(
+            handles[16].handle, a["qkv"], a["q_norm_w"], a["k_norm_w"], a["seq_lens"], None, a["block_table"],
+            w.k_cache, w.v_cache, torch.empty((2, 2, 16, 128), dtype=torch.bfloat16, device=DEV))
+    assert handles[16].check() == 0
+
+
+def full_size_check(attn, w, sample, label):
+    k_pre, v_pre = w.k_cache.clone(), w.v_cache.clone()
+    o = ph.run(attn, w, DEV, w.k_cache, w.v_cache)
+    assert attn.check() == 0
+    k_rows, v_rows, k64 = ph.oracle_appended_rows(w, k_pre, v_pre)
+    k_exp, v_exp = ph.expected_cache(w, k_pre, v_pre, k_rows, v_rows)
+    ph.assert_cache_equal(w.k_cache, w.v_cache, k_exp, v_exp, k64, w)
+    del k_exp, v_exp
+    ref = ph.oracle_sampled(w, sample, k_pre, v_pre)
+    return ph.assert_o_close(o[torch.as_tensor(sample)], ref, label)
+
+
+@pytest.mark.parametrize("hq,T", CASES)
+def test_config2_shape_full_size(handles, hq, T):
+    w = inputs.config2("cuda", num_q_heads=hq, new_tokens=T)
+    full_size_check(handles[hq], w, list(range(1, 32, 4)), f"cfg2 Hq={hq} T={T}")
+
+
+def test_config4_shape_full_size(handles):
+    w = inputs.config4("cuda", new_tokens=4)
+    full_size_check(handles[16], w, [1, 2], "cfg4 T=4")
