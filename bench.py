@@ -58,22 +58,24 @@ WORKLOADS = {
 # ----------------------------------------------------------------------------
 # workloads and byte counts
 
-def make_layers(name: str, device, rank: int = 0, num_q_heads: int = 16):
+def make_layers(name: str, device, rank: int = 0, num_q_heads: int = 16, new_tokens: int = 1):
     """The layers of one step (one Workload per library call). num_q_heads picks the
-    Qwen3 size: 16 (0.6B), 32 (4B/8B), 40 (14B) or 64 (32B); cfg1 and cfg3 are 0.6B only."""
+    Qwen3 size: 16 (0.6B), 32 (4B/8B), 40 (14B) or 64 (32B); new_tokens > 1 gives
+    every sequence that many new tokens (causal among themselves). cfg1 and cfg3
+    are 0.6B with one new token only."""
     off = 100 * rank
-    if name in ("cfg1", "cfg3") and num_q_heads != 16:
-        raise ValueError(f"{name} is defined for Qwen3-0.6B (16 query heads)")
+    if name in ("cfg1", "cfg3") and (num_q_heads != 16 or new_tokens != 1):
+        raise ValueError(f"{name} is defined for Qwen3-0.6B (16 query heads) and one new token")
     if name == "cfg1":
         return [inputs.config1(device)] if rank == 0 else [inputs.custom([7, 12], seed=off, device=device)]
     if name == "cfg2":
-        return [inputs.config2(device, seed=2000 + off, num_q_heads=num_q_heads)]
+        return [inputs.config2(device, seed=2000 + off, num_q_heads=num_q_heads, new_tokens=new_tokens)]
     if name == "cfg3":
         return [inputs.config3_layer(i, device, seed=3000 + off) for i in range(inputs.CONFIG3_LAYERS)]
     if name == "cfg4":
-        return [inputs.config4(device, seed=4000 + off, num_q_heads=num_q_heads)]
+        return [inputs.config4(device, seed=4000 + off, num_q_heads=num_q_heads, new_tokens=new_tokens)]
     if name == "cfg5":
-        return [inputs.config5(device, seed=5000 + off, num_q_heads=num_q_heads)]
+        return [inputs.config5(device, seed=5000 + off, num_q_heads=num_q_heads, new_tokens=new_tokens)]
     raise ValueError(name)
 
 
@@ -82,15 +84,16 @@ def kv_bytes(seq_lens) -> int:
     return int(torch.as_tensor(seq_lens, dtype=torch.int64).sum()) * KV_BYTES_PER_TOKEN
 
 
-def algorithmic_bytes(seq_lens, num_q_heads: int = 16) -> int:
-    """Least HBM traffic of one call: the cached K/V rows read (L-1 per sequence),
-    the new k/v rows written, the qkv row read, o written, the block-table
-    entries and seq_lens read, and the two gain vectors."""
+def algorithmic_bytes(seq_lens, num_q_heads: int = 16, new_tokens: int = 1) -> int:
+    """Least HBM traffic of one call with T = new_tokens: the cached K/V rows
+    read (L-T per sequence), the T new k/v rows written, the T qkv rows read,
+    o written, the block-table entries and seq_lens read, and the two gain
+    vectors."""
     L = torch.as_tensor(seq_lens, dtype=torch.int64)
-    B = int(L.numel())
+    B, T = int(L.numel()), new_tokens
     pages = int(((L + 15) // 16).sum())
-    return (int((L - 1).sum()) * KV_BYTES_PER_TOKEN + B * KV_BYTES_PER_TOKEN
-            + B * inputs.qkv_width(num_q_heads) * 2 + B * num_q_heads * inputs.HEAD_DIM * 2
+    return (int((L - T).sum()) * KV_BYTES_PER_TOKEN + B * T * KV_BYTES_PER_TOKEN
+            + B * T * inputs.qkv_width(num_q_heads) * 2 + B * T * num_q_heads * inputs.HEAD_DIM * 2
             + pages * 4 + B * 4 + 2 * inputs.HEAD_DIM * 2)
 
 
@@ -102,15 +105,24 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash(num_q_heads: int = 16) -> str:
+def kernel_key(num_q_heads: int = 16, new_tokens: int = 1):
+    """Which attention kernel a call runs: the 16-head decode kernel or the tensor-core one."""
+    return 16 if num_q_heads == 16 and new_tokens == 1 else "grouped"
+
+
+def workload_key(workload: str, num_q_heads: int = 16, new_tokens: int = 1) -> str:
+    return workload + ("" if num_q_heads == 16 else f"-h{num_q_heads}") + ("" if new_tokens == 1 else f"-t{new_tokens}")
+
+
+def kernel_source_hash(num_q_heads: int = 16, new_tokens: int = 1) -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES[16 if num_q_heads == 16 else "grouped"]:
+    for p in KERNEL_SOURCES[kernel_key(num_q_heads, new_tokens)]:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
 
-def traffic_per_launch(workload: str, num_q_heads: int = 16):
+def traffic_per_launch(workload: str, num_q_heads: int = 16, new_tokens: int = 1):
     """DRAM bytes per call from the committed ncu summary, if it was taken on
     this kernel source and workload (else None)."""
     try:
@@ -119,7 +131,7 @@ def traffic_per_launch(workload: str, num_q_heads: int = 16):
     except (OSError, ValueError):
         return None
     entry = t.get(workload)
-    if not entry or entry.get("kernel_source_sha256") != kernel_source_hash(num_q_heads):
+    if not entry or entry.get("kernel_source_sha256") != kernel_source_hash(num_q_heads, new_tokens):
         return None
     return entry.get("dram_bytes_per_launch")
 
@@ -254,8 +266,9 @@ def compact_host(w: inputs.Workload, seqs):
 
 def time_oracle(batch: dict) -> float:
     import oracle
+    step = oracle.append_and_attend_tokens if batch["qkv"].ndim == 3 else oracle.append_and_attend
     t0 = time.perf_counter()
-    oracle.append_and_attend(**batch, inplace=True)
+    step(**batch, inplace=True)
     return time.perf_counter() - t0
 
 
@@ -308,14 +321,15 @@ def run_gpu(args):
     torch.cuda.set_device(dev)
     lib = binding.load_library()
     attn = binding.DecodeAttention(device=local, num_q_heads=args.num_q_heads)
+    T = args.new_tokens
 
     # R resident copies of the step's inputs, so that a call never finds its
     # K/V in L2 from the previous call (each copy's KV is > L2 or R copies are).
-    first = make_layers(args.workload, dev, rank, args.num_q_heads)
+    first = make_layers(args.workload, dev, rank, args.num_q_heads, T)
     step_kv = sum(kv_bytes(w.seq_lens) for w in first)
     rotate = args.rotate or max(1, min(8, math.ceil(4 * L2_BYTES / max(step_kv, 1))))
     # the copies hold the same bytes in different memory, so every timed launch does the same work
-    sets = [first] + [make_layers(args.workload, dev, rank, args.num_q_heads) for r in range(1, rotate)]
+    sets = [first] + [make_layers(args.workload, dev, rank, args.num_q_heads, T) for r in range(1, rotate)]
     calls_per_step = len(first)
     stream = torch.cuda.current_stream(dev)
     sp = ctypes.c_void_p(stream.cuda_stream)
@@ -325,19 +339,19 @@ def run_gpu(args):
         for w in layers:
             t = dict(qkv=w.qkv, q=w.q_norm_w, k=w.k_norm_w, sl=w.seq_lens.to(dev), bt=w.block_table.to(dev),
                      kc=w.k_cache, vc=w.v_cache,
-                     o=torch.empty((w.batch, w.num_q_heads, 128), dtype=torch.bfloat16, device=dev))
+                     o=torch.empty((*w.qkv.shape[:-1], w.num_q_heads, 128), dtype=torch.bfloat16, device=dev))
             c = (attn.handle, ctypes.c_void_p(t["qkv"].data_ptr()), ctypes.c_void_p(t["q"].data_ptr()),
                  ctypes.c_void_p(t["k"].data_ptr()),
                  ctypes.cast(ctypes.c_void_p(t["sl"].data_ptr()), ctypes.POINTER(ctypes.c_int32)), None,
                  ctypes.cast(ctypes.c_void_p(t["bt"].data_ptr()), ctypes.POINTER(ctypes.c_int32)),
                  int(w.block_table.shape[1]), ctypes.c_void_p(t["kc"].data_ptr()),
                  ctypes.c_void_p(t["vc"].data_ptr()), int(w.num_pages), ctypes.c_void_p(t["o"].data_ptr()),
-                 int(w.batch), sp)
+                 int(w.batch)) + ((T,) if T > 1 else ()) + (sp,)
             out.append((c, t))
         return out
 
     calls = [prepared(layers) for layers in sets]
-    fn = lib.qwen3_decode_attn_append_and_attend
+    fn = lib.qwen3_decode_attn_append_and_attend_tokens if T > 1 else lib.qwen3_decode_attn_append_and_attend
 
     def step(i):
         for c, _ in calls[i % rotate]:
@@ -384,7 +398,7 @@ def run_gpu(args):
     ms_per_step = ms / args.steps
     # every rotation set has its own lengths (cfg2/cfg5 draw them); average the bytes per step
     kv_per_step_local = sum(sum(kv_bytes(w.seq_lens) for w in s) for s in (sets[i % rotate] for i in range(args.steps))) / args.steps
-    alg_per_step_local = sum(sum(algorithmic_bytes(w.seq_lens, w.num_q_heads) for w in s)
+    alg_per_step_local = sum(sum(algorithmic_bytes(w.seq_lens, w.num_q_heads, T) for w in s)
                              for s in (sets[i % rotate] for i in range(args.steps))) / args.steps
     kv_total = reduce_sum(dist, kv_per_step_local, dev)
     value = kv_total / (ms_per_step * 1e-3) / 1e9
@@ -394,12 +408,12 @@ def run_gpu(args):
     alg_per_launch = alg_per_step_local / calls_per_step
     peak, peak_kind = hbm_peak()
     achieved = alg_per_launch / (mean_kernel_ms * 1e-3) / 1e9
-    workload_key = args.workload if args.num_q_heads == 16 else f"{args.workload}-h{args.num_q_heads}"
-    traffic = traffic_per_launch(workload_key, args.num_q_heads)
+    traffic = traffic_per_launch(workload_key(args.workload, args.num_q_heads, T), args.num_q_heads, T)
 
-    # end to end through the host-buffer entry point: per step the H2D copy of the
-    # step's inputs from pinned memory, the call, and the D2H copy of o
-    e2e = run_e2e(args, attn, sets, dev, stream, dist, rotate)
+    # end to end: per step the H2D copy of the step's inputs from pinned memory,
+    # the call, and the D2H copy of o
+    e2e = (run_e2e(args, attn, sets, dev, stream, dist, rotate) if T == 1
+           else run_e2e_tokens(args, attn, sets, dev, stream, dist, rotate))
 
     result = None
     if rank == 0:
@@ -411,8 +425,9 @@ def run_gpu(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "io_dtype": "bf16", "data": "synthetic (seeded; N(0,1) bf16 qkv and cache, gains 1+U(-0.5,0.5))",
             "config": {"workload": f"{args.workload}: {WORKLOADS[args.workload]}"
-                                   + ("" if args.num_q_heads == 16 else f", {args.num_q_heads} query heads"),
-                       "batch": first[0].batch, "layers_per_step": calls_per_step,
+                                   + ("" if args.num_q_heads == 16 else f", {args.num_q_heads} query heads")
+                                   + ("" if T == 1 else f", {T} new tokens per sequence (causal among them)"),
+                       "batch": first[0].batch, "layers_per_step": calls_per_step, "new_tokens": T,
                        "sum_seq_lens_per_step": int(sum(int(w.seq_lens.sum()) for w in first)),
                        "page_size": 16, "heads": f"{args.num_q_heads} q / 8 kv, D=128",
                        "l2": f"{rotate} resident input sets rotated; {rotate * step_kv / 1e9:.2f} GB of KV cycled "
@@ -425,8 +440,8 @@ def run_gpu(args):
                          "kernel_us_mean": round(mean_kernel_ms * 1e3, 3),
                          "kernel_us_median": round(statistics.median(kernel_ms) * 1e3, 3)},
             "e2e": e2e,
-            # one kernel per call at 16 query heads; attention + combine launches otherwise
-            "gpu_launches": n_launch * (1 if args.num_q_heads == 16 else 2),
+            # one kernel per call on the 16-head decode kernel; attention + combine launches otherwise
+            "gpu_launches": n_launch * (1 if kernel_key(args.num_q_heads, T) == 16 else 2),
             "clocks": clk,
         }
     if dist is not None:
@@ -488,6 +503,67 @@ def run_e2e(args, attn, sets, dev, stream, dist, rotate):
             "ms_per_step": round(ms, 6), "api": "qwen3_decode_attn_append_and_attend_host"}
 
 
+def run_e2e_tokens(args, attn, sets, dev, stream, dist, rotate):
+    """End to end for T new tokens: the per-step tensors (qkv, seq_lens, block
+    table) copied from pinned host memory into device buffers, the call
+    through qwen3_decode_attn_append_and_attend_tokens, and o copied back."""
+    from decode_attention_qk_b200 import binding
+    lib = binding.load_library()
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    T = args.new_tokens
+    host = []
+    for layers in sets:
+        hl = []
+        for w in layers:
+            h = dict(qkv=w.qkv.cpu().pin_memory(), sl=w.seq_lens.clone().pin_memory(),
+                     bt=w.block_table.clone().pin_memory(),
+                     o=torch.empty((w.batch, T, w.num_q_heads, 128), dtype=torch.bfloat16).pin_memory())
+            d = {k: torch.empty_like(v, device=dev) for k, v in h.items()}
+            c = (attn.handle, ctypes.c_void_p(d["qkv"].data_ptr()), ctypes.c_void_p(w.q_norm_w.data_ptr()),
+                 ctypes.c_void_p(w.k_norm_w.data_ptr()),
+                 ctypes.cast(ctypes.c_void_p(d["sl"].data_ptr()), ctypes.POINTER(ctypes.c_int32)), None,
+                 ctypes.cast(ctypes.c_void_p(d["bt"].data_ptr()), ctypes.POINTER(ctypes.c_int32)),
+                 int(w.block_table.shape[1]), ctypes.c_void_p(w.k_cache.data_ptr()),
+                 ctypes.c_void_p(w.v_cache.data_ptr()), int(w.num_pages), ctypes.c_void_p(d["o"].data_ptr()),
+                 int(w.batch), T, sp)
+            hl.append((c, h, d))
+        host.append(hl)
+    fn = lib.qwen3_decode_attn_append_and_attend_tokens
+
+    def call(c, h, d):
+        for k in ("qkv", "sl", "bt"):
+            d[k].copy_(h[k], non_blocking=True)
+        rc = fn(*c)
+        if rc != 0:
+            raise binding.QdaError(rc, "append_and_attend_tokens")
+        h["o"].copy_(d["o"], non_blocking=True)
+
+    for i in range(args.warmup):
+        for c, h, d in host[i % rotate]:
+            call(c, h, d)
+    barrier(dist, dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    h2d = d2h = 0
+    for i in range(args.steps):
+        for c, h, d in host[i % rotate]:
+            call(c, h, d)
+            h2d += h["qkv"].nbytes + h["sl"].nbytes + h["bt"].nbytes
+            d2h += h["o"].nbytes
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    if attn.check() != 0:
+        raise RuntimeError("device status after the e2e region")
+    ms = reduce_max(dist, start.elapsed_time(end), dev) / args.steps
+    kv = sum(sum(kv_bytes(w.seq_lens) for w in sets[i % rotate]) for i in range(args.steps)) / args.steps
+    kv_total = reduce_sum(dist, kv, dev)
+    return {"value": round(kv_total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d // args.steps), "d2h_bytes_per_step": int(d2h // args.steps),
+            "ms_per_step": round(ms, 6),
+            "api": "pinned host->device copies + qwen3_decode_attn_append_and_attend_tokens + o device->host"}
+
+
 # ----------------------------------------------------------------------------
 # reference arm: the float64 oracle on the host cores
 
@@ -498,7 +574,7 @@ def run_reference(args):
         return
     import oracle
     oracle.build()
-    layers = make_layers(args.workload, "cpu", 0, args.num_q_heads)
+    layers = make_layers(args.workload, "cpu", 0, args.num_q_heads, args.new_tokens)
     # size each step's sample so that warm-up + timed steps take ~2 minutes
     probe = min(range(layers[0].batch), key=lambda b: int(layers[0].seq_lens[b]))
     dt = time_oracle(compact_host(layers[0], [probe]))
@@ -541,8 +617,11 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded; same recipe as the GPU arm, drawn on the host)",
         "config": {"workload": f"{args.workload}: {WORKLOADS[args.workload]}"
-                               + ("" if args.num_q_heads == 16 else f", {args.num_q_heads} query heads"),
-                   "batch": layers[0].batch, "layers_per_step": len(layers), "page_size": 16,
+                               + ("" if args.num_q_heads == 16 else f", {args.num_q_heads} query heads")
+                               + ("" if args.new_tokens == 1 else
+                                  f", {args.new_tokens} new tokens per sequence (causal among them)"),
+                   "batch": layers[0].batch, "layers_per_step": len(layers), "new_tokens": args.new_tokens,
+                   "page_size": 16,
                    "heads": f"{args.num_q_heads} q / 8 kv, D=128"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": sample_desc},
@@ -559,6 +638,8 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="cfg2")
     ap.add_argument("--num-q-heads", type=int, choices=[16, 32, 40, 64], default=16,
                     help="query heads: 16 = Qwen3-0.6B (the default workload); 32/40/64 = 4B-8B/14B/32B")
+    ap.add_argument("--new-tokens", type=int, default=1,
+                    help="new tokens per sequence (1 = decode; 2-4 at 16 heads, 2 at 32: several tokens at once)")
     ap.add_argument("--rotate", type=int, default=0, help="resident input sets cycled (0: enough to defeat L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

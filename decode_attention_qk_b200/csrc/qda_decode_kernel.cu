@@ -16,7 +16,9 @@
 // un-normalised output) per sequence piece it holds, and the last CTA to
 // finish a piece of a cut sequence merges the partials (log-sum-exp combine;
 // exact by the online-softmax theorem flashAttn_eq and softmax_shift on the
-// Supported models page, "Facts proved about the specs"). The piece of
+// Supported models page, "Facts proved about the specs"), bulk-copying them
+// into its then idle staging ring so that the merge costs one round trip to
+// L2 per 24 pieces rather than one per few pieces. The piece of
 // sequence b held by CTA g gets scratch slot g + b; these slots are distinct
 // because ranges and sequences are both ordered.
 //
@@ -67,10 +69,22 @@ constexpr int kSmemInvFreq = kSmemLens + kMaxBatch * 4;                    // do
 constexpr int kSmemGains = kSmemInvFreq + 64 * 8;                          // bf16 [2][128]
 constexpr int kSmemMeta = kSmemGains + 2 * kHeadDim * 2;                   // StageMeta [kStages]
 constexpr int kSmemBars = kSmemMeta + kStages * 16;                        // uint64 [2*kStages + 1]
-constexpr int kSmemFlags = kSmemBars + (2 * kStages + 1) * 8;              // abort flag
+constexpr int kSmemMergeBars = kSmemBars + (2 * kStages + 1) * 8;          // uint64 [kConsumerWarps + 1]
+constexpr int kSmemFlags = kSmemMergeBars + (kConsumerWarps + 1) * 8;      // abort flag
 constexpr int kSmemTotal = kSmemFlags + 16;
 static_assert(kStageBytes % 128 == 0 && kSmemInvFreq % 8 == 0 && kSmemBars % 8 == 0, "alignment");
 static_assert(kSmemTotal <= 227 * 1024, "fits one CTA per SM");
+
+// Merging split sequences. Once every consumer warp is past its last page the
+// ring is free: warp j merges in its own 1/8 of it, copying up to kMergeBatch
+// pieces' partials (1 KiB of un-normalised output for heads 2j, 2j+1, and 16 B
+// of running max and sum) with one bulk copy per piece and lane.
+constexpr int kMergeRegion = kStages * kStageBytes / kConsumerWarps;
+constexpr int kMergeRowBytes = kGroup * kHeadDim * 4;                      // 1 KiB
+constexpr int kMergeBatch = 24;
+constexpr int kMergeMlOff = kMergeBatch * kMergeRowBytes;
+static_assert(kMergeBatch <= 32 && kMergeMlOff + kMergeBatch * 16 <= kMergeRegion && kMergeRegion % 16 == 0,
+              "merge region");
 
 // Partial dot products of one staged k row (this lane's 16 dims: words 0..3
 // are dims 8c..8c+7, words 4..7 dims 64+8c..64+8c+7) with both query heads.
@@ -121,6 +135,8 @@ struct Shared {
     uint64_t* full_bar;
     uint64_t* empty_bar;
     uint64_t* never_bar;
+    uint64_t* merge_bar;    // [kConsumerWarps]: the merge copies of warp j
+    uint64_t* done_bar;     // every consumer warp is past its last page
     volatile int* abort_flag;
 };
 
@@ -503,105 +519,118 @@ __device__ __forceinline__ bool finish_piece(const Params& p, const Shared& s, i
     return true;
 }
 
-// Count this CTA's piece of sequence b as done; the last piece to arrive
-// combines every piece's partial for heads 2j, 2j+1 and writes o. The caller
-// has made its partial stores visible (__threadfence) before calling.
-__device__ __forceinline__ void arrive_and_merge(const Params& p, const Shared& s, int b, int j, int lane, int grp,
-                                                 int c, int per_cta) {
-    const int hb = grp & 1;
-    const int hf = grp >> 1;
-    const int head = kGroup * j + hb;
-    const int dim0 = 64 * hf + 8 * c;
-    const int part_first = s.seg[b] / per_cta;
-    const int part_last = (s.seg[b + 1] - 1) / per_cta;
-    const int nparts = part_last - part_first + 1;
-    int prev = 0;
-    if (lane == 0) prev = atomicAdd(p.counters + b * kNumKvHeads + j, 1);
-    prev = __shfl_sync(kFull, prev, 0);
-    if (prev != nparts - 1) return;
-
-    // Last arrival. Pass 1: lanes read the pieces' (max, sum) in parallel; M = overall max.
-    __threadfence();
-    const float4* ml_base = reinterpret_cast<const float4*>(p.part_ml + (size_t)kGroup * j);  // heads 2j, 2j+1
-    float Mx0 = -INFINITY, Mx1 = -INFINITY;
-    for (int t = lane; t < nparts; t += 32) {
-        const float4 ml = __ldcg(ml_base + (size_t)(part_first + t + b) * (kNumQHeads / 2));
-        Mx0 = fmaxf(Mx0, ml.x);
-        Mx1 = fmaxf(Mx1, ml.z);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        Mx0 = fmaxf(Mx0, __shfl_xor_sync(kFull, Mx0, off));
-        Mx1 = fmaxf(Mx1, __shfl_xor_sync(kFull, Mx1, off));
-    }
-    // Pass 2: weights 2^(m_t - M) per piece (lane t), then every lane sums its
-    // 8 output dims over the pieces with many loads in flight.
-    constexpr int kMergeBatch = 8;
-    float Ls0 = 0.f, Ls1 = 0.f, A[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) A[k] = 0.f;
-    const float* acc_base = p.part_acc + (size_t)head * kHeadDim + dim0;
-    for (int t0 = 0; t0 < nparts; t0 += 32) {
-        float w0 = 0.f, w1 = 0.f;
-        if (t0 + lane < nparts) {
-            const float4 ml = __ldcg(ml_base + (size_t)(part_first + t0 + lane + b) * (kNumQHeads / 2));
-            w0 = (ml.x == -INFINITY) ? 0.f : exp2_approx(ml.x - Mx0);   // a piece whose pages were all skipped
-            w1 = (ml.z == -INFINITY) ? 0.f : exp2_approx(ml.z - Mx1);
-            Ls0 += w0 * ml.y;
-            Ls1 += w1 * ml.w;
-        }
-        const int n = min(32, nparts - t0);
-        for (int u0 = 0; u0 < n; u0 += kMergeBatch) {
-            float4 x0[kMergeBatch], x1[kMergeBatch];
-#pragma unroll
-            for (int u = 0; u < kMergeBatch; ++u) {
-                if (u0 + u < n) {
-                    const float4* src = reinterpret_cast<const float4*>(
-                        acc_base + (size_t)(part_first + t0 + u0 + u + b) * (kNumQHeads * kHeadDim));
-                    x0[u] = __ldcg(src);
-                    x1[u] = __ldcg(src + 1);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kMergeBatch; ++u) {
-                const float wa = __shfl_sync(kFull, w0, (u0 + u) & 31);
-                const float wb = __shfl_sync(kFull, w1, (u0 + u) & 31);
-                if (u0 + u < n) {
-                    const float w = hb ? wb : wa;
-                    A[0] = fmaf(w, x0[u].x, A[0]);
-                    A[1] = fmaf(w, x0[u].y, A[1]);
-                    A[2] = fmaf(w, x0[u].z, A[2]);
-                    A[3] = fmaf(w, x0[u].w, A[3]);
-                    A[4] = fmaf(w, x1[u].x, A[4]);
-                    A[5] = fmaf(w, x1[u].y, A[5]);
-                    A[6] = fmaf(w, x1[u].z, A[6]);
-                    A[7] = fmaf(w, x1[u].w, A[7]);
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        Ls0 += __shfl_xor_sync(kFull, Ls0, off);
-        Ls1 += __shfl_xor_sync(kFull, Ls1, off);
-    }
-    const float Ls = hb ? Ls1 : Ls0;
-    store_bf16x8(p.o + ((size_t)b * kNumQHeads + head) * kHeadDim + dim0, A, Ls > 0.f ? 1.f / Ls : 0.f);
-    if (lane == 0) p.counters[b * kNumKvHeads + j] = 0;  // ready for the next call
-}
-
-// Wait for the page in `slot`; returns false when the wait ran out (the
-// kernel is then aborting).
-__device__ __forceinline__ bool wait_full(const Params& p, const Shared& s, int slot, uint32_t phase, int lane) {
-    bool ok = mbar_try_wait(&s.full_bar[slot], phase);
+// Bounded wait of a whole warp on `bar`; on expiry records QDA_ERR_TIMEOUT and
+// sets the CTA's abort flag.
+__device__ __forceinline__ bool warp_wait(const Params& p, const Shared& s, uint64_t* bar, uint32_t phase, int lane) {
+    bool ok = mbar_try_wait(bar, phase);
     if (__all_sync(kFull, ok)) return true;
-    ok = ok || mbar_wait(&s.full_bar[slot], phase, p.timeout_ns, s.abort_flag);
-    ok = __all_sync(kFull, ok || mbar_try_wait(&s.full_bar[slot], phase));
+    ok = ok || mbar_wait(bar, phase, p.timeout_ns, s.abort_flag);
+    ok = __all_sync(kFull, ok || mbar_try_wait(bar, phase));
     if (!ok && lane == 0) {
         *s.abort_flag = 1;
         record_error(p.status, QDA_ERR_TIMEOUT);
     }
     return ok;
+}
+
+// Pieces of sequence b: scratch slots first + b .. first + b + n - 1.
+__device__ __forceinline__ int pieces_of(const Shared& s, int b, int per_cta, int& first) {
+    first = s.seg[b] / per_cta;
+    return (s.seg[b + 1] - 1) / per_cta - first + 1;
+}
+
+// Merge every piece's partial of sequence b for heads 2j, 2j+1 and write o
+// (this warp was the last to arrive). Pieces come in batches of kMergeBatch
+// through this warp's merge region; o = sum_t 2^(m_t - M) acc_t / sum_t
+// 2^(m_t - M) l_t with M the running maximum, rescaled between batches.
+// Returns false when a wait ran out.
+__device__ __forceinline__ bool merge_sequence(const Params& p, const Shared& s, int b, int j, int lane, int grp, int c,
+                                               int per_cta, uint32_t& mphase) {
+    const int hb = grp & 1;
+    const int hf = grp >> 1;
+    const int head = kGroup * j + hb;
+    const int dim0 = 64 * hf + 8 * c;
+    int first = 0;
+    const int n = pieces_of(s, b, per_cta, first);
+    uint8_t* region = s.stages + j * kMergeRegion;
+    uint64_t* bar = &s.merge_bar[j];
+    float M0 = -INFINITY, M1 = -INFINITY, L0 = 0.f, L1 = 0.f, A[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) A[k] = 0.f;
+    for (int t0 = 0; t0 < n; t0 += kMergeBatch) {
+        const int nb = min(kMergeBatch, n - t0);
+        // earlier reads of the region come before the copies that overwrite it
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)nb * (kMergeRowBytes + 16));
+        __syncwarp();
+        if (lane < nb) {
+            const size_t row = (size_t)(first + b + t0 + lane) * kNumQHeads + kGroup * j;
+            bulk_g2s(region + lane * kMergeRowBytes, p.part_acc + row * kHeadDim, (uint32_t)kMergeRowBytes, bar);
+            bulk_g2s(region + kMergeMlOff + lane * 16, p.part_ml + row, 16u, bar);
+        }
+        if (!warp_wait(p, s, bar, mphase, lane)) {
+            // the copies may still be landing: wait once more (bounded) before leaving
+            if (lane == 0) (void)mbar_wait(bar, mphase, p.timeout_ns, nullptr);
+            __syncwarp();
+            return false;
+        }
+        mphase ^= 1u;
+        // lane t < nb holds piece t's (max, sum) of both heads
+        const float4 ml = lane < nb ? *reinterpret_cast<const float4*>(region + kMergeMlOff + lane * 16)
+                                    : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+        float bm0 = ml.x, bm1 = ml.z;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            bm0 = fmaxf(bm0, __shfl_xor_sync(kFull, bm0, off));
+            bm1 = fmaxf(bm1, __shfl_xor_sync(kFull, bm1, off));
+        }
+        const float nM0 = fmaxf(M0, bm0), nM1 = fmaxf(M1, bm1);
+        // what the earlier batches summed, rescaled to the new maximum (nothing on the first)
+        const float r0 = (M0 == -INFINITY) ? 0.f : exp2_approx(M0 - nM0);
+        const float r1 = (M1 == -INFINITY) ? 0.f : exp2_approx(M1 - nM1);
+        const float rh = hb ? r1 : r0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) A[k] *= rh;
+        // a piece whose pages were all skipped has max -inf and weight 0
+        const float w0 = (ml.x == -INFINITY) ? 0.f : exp2_approx(ml.x - nM0);
+        const float w1 = (ml.z == -INFINITY) ? 0.f : exp2_approx(ml.z - nM1);
+        L0 = fmaf(w0, ml.y, L0 * r0);
+        L1 = fmaf(w1, ml.w, L1 * r1);
+        const uint8_t* src = region + (hb * kHeadDim + dim0) * 4;
+        for (int t = 0; t < nb; ++t) {
+            const float wa = __shfl_sync(kFull, w0, t);
+            const float wb = __shfl_sync(kFull, w1, t);
+            const float w = hb ? wb : wa;
+            const float4 x0 = *reinterpret_cast<const float4*>(src + t * kMergeRowBytes);
+            const float4 x1 = *reinterpret_cast<const float4*>(src + t * kMergeRowBytes + 16);
+            A[0] = fmaf(w, x0.x, A[0]);
+            A[1] = fmaf(w, x0.y, A[1]);
+            A[2] = fmaf(w, x0.z, A[2]);
+            A[3] = fmaf(w, x0.w, A[3]);
+            A[4] = fmaf(w, x1.x, A[4]);
+            A[5] = fmaf(w, x1.y, A[5]);
+            A[6] = fmaf(w, x1.z, A[6]);
+            A[7] = fmaf(w, x1.w, A[7]);
+        }
+        M0 = nM0;
+        M1 = nM1;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        L0 += __shfl_xor_sync(kFull, L0, off);
+        L1 += __shfl_xor_sync(kFull, L1, off);
+    }
+    const float Ls = hb ? L1 : L0;
+    store_bf16x8(p.o + ((size_t)b * kNumQHeads + head) * kHeadDim + dim0, A, Ls > 0.f ? 1.f / Ls : 0.f);
+    if (lane == 0) p.counters[b * kNumKvHeads + j] = 0;  // ready for the next call
+    return true;
+}
+
+// Wait for the page in `slot`; returns false when the wait ran out (the
+// kernel is then aborting).
+__device__ __forceinline__ bool wait_full(const Params& p, const Shared& s, int slot, uint32_t phase, int lane) {
+    return warp_wait(p, s, &s.full_bar[slot], phase, lane);
 }
 
 // Attend over the staged page in `slot` (page i of a sequence of nb pages and
@@ -660,22 +689,30 @@ __device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, i
     uint32_t phase = 0;
     int pending0 = -1, pending1 = -1;  // split pieces whose arrival waits for the end
     const int count = end - start;
+    bool aborted = false;
     int k = 0;
-    while (k < count) {
+    while (k < count && !aborted) {
         const int nb = s.seg[b + 1] - s.seg[b];
         const int L = s.lens[b];
         const int n_here = min(nb - i0, count - k);
         // first page of the piece: it carries the sequence's qkv row
-        if (!wait_full(p, s, slot, phase, lane)) return;
+        if (!wait_full(p, s, slot, phase, lane)) {
+            aborted = true;
+            break;
+        }
         begin_sequence(p, s, s.stages + slot * kStageBytes + kStageQkv, s.meta[slot].pos, j, lane, c,
                        /*appends=*/s.seg[b + 1] <= end, st);
         consume_page(p, s, slot, i0, nb, L, j, grp, c, lane, st);
         if (++slot == kStages) { slot = 0; phase ^= 1u; }
         for (int u = 1; u < n_here; ++u) {
-            if (!wait_full(p, s, slot, phase, lane)) return;
+            if (!wait_full(p, s, slot, phase, lane)) {
+                aborted = true;
+                break;
+            }
             consume_page(p, s, slot, i0 + u, nb, L, j, grp, c, lane, st);
             if (++slot == kStages) { slot = 0; phase ^= 1u; }
         }
+        if (aborted) break;
         k += n_here;
         if (finish_piece(p, s, b, j, grp, c, per_cta, st)) {
             if (pending0 < 0) pending0 = b;
@@ -686,11 +723,32 @@ __device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, i
             i0 = 0;
         }
     }
-    if (pending0 >= 0) {
-        __threadfence();   // this warp's partial stores before its arrivals
-        arrive_and_merge(p, s, pending0, j, lane, grp, c, per_cta);
-        if (pending1 >= 0) arrive_and_merge(p, s, pending1, j, lane, grp, c, per_cta);
+    // this warp no longer reads the ring
+    __syncwarp();
+    if (lane == 0) mbar_arrive(s.done_bar);
+    if (aborted || pending0 < 0) return;
+
+    // Count this CTA's split pieces as done (lane 0: pending0, lane 1:
+    // pending1); the last piece of a sequence to arrive merges it.
+    __threadfence();   // this warp's partial stores before its arrivals
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    const int npend = pending1 >= 0 ? 2 : 1;
+    const int mine = lane == 0 ? pending0 : pending1;
+    int first = 0, prev = -1, need = 0;
+    if (lane < npend) {
+        need = pieces_of(s, mine, per_cta, first) - 1;
+        prev = atomicAdd(p.counters + mine * kNumKvHeads + j, 1);
     }
+    const bool last0 = __shfl_sync(kFull, prev == need, 0);
+    const bool last1 = __shfl_sync(kFull, prev == need, 1) && npend == 2;
+    if (!last0 && !last1) return;
+    // the other pieces' partials, read through the async proxy by the merge copies
+    __threadfence();
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    if (!warp_wait(p, s, s.done_bar, 0u, lane)) return;
+    uint32_t mphase = 0;
+    if (last0 && !merge_sequence(p, s, pending0, j, lane, grp, c, per_cta, mphase)) return;
+    if (last1) (void)merge_sequence(p, s, pending1, j, lane, grp, c, per_cta, mphase);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) decode_attention_kernel(const Params p) {
@@ -707,6 +765,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_kernel(const Par
     s.full_bar = reinterpret_cast<uint64_t*>(smem + kSmemBars);
     s.empty_bar = s.full_bar + kStages;
     s.never_bar = s.empty_bar + kStages;
+    s.merge_bar = reinterpret_cast<uint64_t*>(smem + kSmemMergeBars);
+    s.done_bar = s.merge_bar + kConsumerWarps;
     s.abort_flag = reinterpret_cast<volatile int*>(smem + kSmemFlags);
 
     // Pages per sequence (0 for a sequence whose length is out of range).
@@ -733,6 +793,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_kernel(const Par
             mbar_init(&s.empty_bar[k], kConsumerWarps);
         }
         mbar_init(s.never_bar, 1);
+        for (int k = 0; k < kConsumerWarps; ++k) mbar_init(&s.merge_bar[k], 1);
+        mbar_init(s.done_bar, kConsumerWarps);
         *s.abort_flag = 0;
         s.seg[0] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");

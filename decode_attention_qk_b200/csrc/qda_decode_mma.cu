@@ -64,9 +64,13 @@ struct Layout {
     static constexpr int kQkvW = (kHq + 2 * kNumKvHeads) * kHeadDim;     // elements in one token's qkv row
     static constexpr int kQkvBytes = kQkvW * 2;
     static constexpr int kSlotBytes = T * kQkvBytes;                     // a sequence's T rows
-    static constexpr int kStages = kSlotBytes <= 24576 ? 3 : 2;          // what fits next to the qkv slot
+    // Rows up to 24 KiB are staged in a shared-memory slot next to three K/V
+    // stages; larger ones (16 heads x 4 tokens: 32 KiB) would leave room for two
+    // stages only, so they are prefetched to L2 and read from global memory.
+    static constexpr bool kDirectQkv = kSlotBytes > 24576;
+    static constexpr int kStages = 3;
     static constexpr int kSmemQkv = kStages * kStageBytes;
-    static constexpr int kSmemSeg = kSmemQkv + kSlotBytes;                  // int [kMaxBatch + 4]
+    static constexpr int kSmemSeg = kSmemQkv + (kDirectQkv ? 0 : kSlotBytes);   // int [kMaxBatch + 4]
     static constexpr int kSmemLens = kSmemSeg + (kMaxBatch + 4) * 4;        // int [kMaxBatch]
     static constexpr int kSmemInvFreq = kSmemLens + kMaxBatch * 4;          // double [64]
     static constexpr int kSmemGains = kSmemInvFreq + 64 * 8;                // bf16 [2][128]
@@ -78,6 +82,11 @@ struct Layout {
     static_assert(kSmemQkv % 16 == 0 && kSmemInvFreq % 8 == 0 && kSmemBars % 8 == 0, "alignment");
     static_assert(kSmemTotal <= 227 * 1024, "fits one CTA per SM");
 };
+
+// Prefetch `bytes` (a multiple of 16, 16-byte aligned) from global memory to L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 
 struct Shared {
     uint8_t* stages;
@@ -133,7 +142,10 @@ __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, i
             int ok = 1;
             uint32_t kv_bytes = 0;
             if (lane == 0) {
-                if (seq_qkv >= 0) {
+                if (Lay::kDirectQkv && seq_qkv >= 0) {
+                    // the consumers read these rows from global memory: have them in L2 first
+                    bulk_prefetch_l2(p.qkv + (size_t)seq_qkv * T * Lay::kQkvW, (uint32_t)Lay::kSlotBytes);
+                } else if (seq_qkv >= 0) {
                     // the qkv slot frees once every consumer has formed q from it
                     ok = mbar_try_wait(s.qkv_empty, qphase ^ 1u) ||
                          mbar_wait(s.qkv_empty, qphase ^ 1u, p.timeout_ns, s.abort_flag);
@@ -208,15 +220,16 @@ struct State {
     uint32_t k_lo[T], k_hi[T], v_lo[T], v_hi[T];   // this lane's words of the appended k/v rows
 };
 
-// Start a sequence piece from the staged qkv rows: q of row r = lane/4 (new
+// Start a sequence piece from its T qkv rows `rows` (staged in shared memory,
+// or in global memory for the largest rows): q of row r = lane/4 (new
 // token r / G, head G*j + r % G) at dims 8m + 2t, 8m + 2t + 1 (t = lane%4,
 // m = 0..15), i.e. both halves of the rotation pairs 8m' + 2t + e, m' < 8.
 // Lane l forms the angles of pairs 2l, 2l+1 for every new token (reduced
 // modulo 2*pi in double, then float sin/cos); lanes fetch theirs by shuffles.
 // When this CTA holds a page with new tokens, their k is formed in double.
 template <int G, int T>
-__device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s, int pos0, int j, int lane,
-                                               bool appends, State<T>& st) {
+__device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s, const uint8_t* rows, int pos0,
+                                               int j, int lane, bool appends, State<T>& st) {
     using Lay = Layout<G, T>;
     constexpr double kTwoPiHi = 6.2831853069365025;      // 2*pi rounded to 32 significant bits
     constexpr double kTwoPiLo = 2.430840202602477e-10;   // 2*pi - kTwoPiHi
@@ -235,7 +248,7 @@ __device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s,
             sincosf((float)fma(-n, kTwoPiLo, fma(-n, kTwoPiHi, ang)), &sf[u][e], &cf[u][e]);
         }
     const uint32_t* xq =
-        reinterpret_cast<const uint32_t*>(s.qkv + tt * Lay::kQkvBytes + head * (kHeadDim * 2));
+        reinterpret_cast<const uint32_t*>(rows + tt * Lay::kQkvBytes + head * (kHeadDim * 2));
     const uint32_t* gq = reinterpret_cast<const uint32_t*>(s.gains);
     uint32_t xw[16];
     float ss = 0.f;
@@ -288,7 +301,7 @@ __device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s,
             double cs0, sn0, cs1, sn1;
             sincos((double)(pos0 + u) * s.inv_freq[2 * lane], &sn0, &cs0);
             sincos((double)(pos0 + u) * s.inv_freq[2 * lane + 1], &sn1, &cs1);
-            const uint8_t* row = s.qkv + u * Lay::kQkvBytes;
+            const uint8_t* row = rows + u * Lay::kQkvBytes;
             const uint32_t* xk = reinterpret_cast<const uint32_t*>(row + (Lay::kHq + j) * (kHeadDim * 2));
             const uint32_t* xv = reinterpret_cast<const uint32_t*>(row + (Lay::kHq + kNumKvHeads + j) * (kHeadDim * 2));
             const uint32_t xlo = xk[lane], xhi = xk[32 + lane];
@@ -499,13 +512,19 @@ __device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, i
         const int nb = s.seg[b + 1] - s.seg[b];
         const int L = s.lens[b];
         const int n_here = min(nb - i0, count - k);
-        if (!wait_full(p, s, s.qkv_full, qphase, lane)) return;
         // this CTA appends when it holds a page with one of the new tokens
         const bool appends = s.seg[b] + (L - T) / kPage < end;
-        begin_sequence<G, T>(p, s, *s.qkv_pos, j, lane, appends, st);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s.qkv_empty);
-        qphase ^= 1u;
+        if (Layout<G, T>::kDirectQkv) {
+            const int pos0 = p.positions != nullptr ? __ldg(p.positions + b) : L - T;
+            begin_sequence<G, T>(p, s, reinterpret_cast<const uint8_t*>(p.qkv + (size_t)b * T * Layout<G, T>::kQkvW),
+                                 pos0, j, lane, appends, st);
+        } else {
+            if (!wait_full(p, s, s.qkv_full, qphase, lane)) return;
+            begin_sequence<G, T>(p, s, s.qkv, *s.qkv_pos, j, lane, appends, st);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s.qkv_empty);
+            qphase ^= 1u;
+        }
         for (int u = 0; u < n_here; ++u) {
             if (!wait_full(p, s, &s.full_bar[slot], phase, lane)) return;
             consume_page<G, T>(p, s, slot, i0 + u, L, j, lane, st);

@@ -200,13 +200,13 @@ def config5_lengths(seed: int = 5000) -> torch.Tensor:
     return torch.exp(7.0 + 1.5 * z).round().clamp(1, MAX_SEQ).to(torch.int32)
 
 
-def config5(device="cpu", seed: int = 5000, num_q_heads: int = NUM_Q_HEADS) -> Workload:
-    """B=256 ragged lognormal lengths; pool 1.1x the pages in use, gaps interleaved."""
-    seq_lens = config5_lengths(seed)
+def config5(device="cpu", seed: int = 5000, num_q_heads: int = NUM_Q_HEADS, new_tokens: int = 1) -> Workload:
+    """B=256 ragged lognormal lengths (at least new_tokens); pool 1.1x the pages in use, gaps interleaved."""
+    seq_lens = config5_lengths(seed).clamp(min=new_tokens)
     need = int(pages_for(seq_lens).sum())
     pool = int(math.ceil(1.1 * need))
     bt = assign_pages(seq_lens, pool, seed + 1, stride=MAX_PAGES_PER_SEQ, gap_fraction=0.1)
-    vals = _values(256, pool, seed, device, num_q_heads)
+    vals = _values(256, pool, seed, device, num_q_heads, new_tokens)
     return Workload(name="cfg5: B=256, seq_lens lognormal(7,1.5) clipped, 10% gap pages",
                     seq_lens=seq_lens, block_table=bt, num_pages=pool, **vals)
 

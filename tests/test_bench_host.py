@@ -18,6 +18,24 @@ def test_byte_counts():
     pages = 1 + 1 + 2 + 256
     want = (0 + 15 + 16 + 4095) * 4096 + 4 * 4096 + 4 * 8192 + 4 * 4096 + pages * 4 + 4 * 4 + 512
     assert bench.algorithmic_bytes(L) == want
+    # T = 3 new tokens at 32 query heads: L - 3 cached rows read, 3 rows of qkv (12288 B each),
+    # 3 k/v rows written and 3 o rows (8192 B each) per sequence
+    L = torch.tensor([3, 16, 17, 4096], dtype=torch.int32)
+    pages = 1 + 1 + 2 + 256
+    want = (0 + 13 + 14 + 4093) * 4096 + 12 * 4096 + 12 * 12288 + 12 * 8192 + pages * 4 + 4 * 4 + 512
+    assert bench.algorithmic_bytes(L, 32, 3) == want
+
+
+def test_kernel_and_workload_keys():
+    assert bench.kernel_key(16, 1) == 16
+    assert bench.kernel_key(16, 2) == bench.kernel_key(64, 1) == "grouped"
+    assert bench.workload_key("cfg2") == "cfg2"
+    assert bench.workload_key("cfg2", 64) == "cfg2-h64"
+    assert bench.workload_key("cfg2", 16, 4) == "cfg2-t4"
+    with pytest.raises(ValueError):
+        bench.make_layers("cfg3", "cpu", 0, 16, 2)
+    w = bench.make_layers("cfg2", "cpu", 0, 16, 4)[0]
+    assert w.new_tokens == 4 and int(w.seq_lens.min()) >= 4
 
 
 def test_cpu_baseline_sample_is_bounded():
