@@ -290,24 +290,48 @@ def pick_sample(layers, budget_bytes: float):
     return picked, total
 
 
-def cpu_baseline(layers, seconds: float = 12.0):
-    """The oracle as it stands, single-threaded, on a bounded sample of the step."""
+def host_cpu():
+    """(usable cores, CPU model) of this host."""
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return cores, model
+
+
+def cpu_baseline(layers, seconds: float = 12.0, threads: int = 1):
+    """The oracle as it stands on a bounded sample of the step, its attention
+    loop on `threads` threads (the result does not depend on the count)."""
     import oracle
     oracle.build()
-    probe = min(range(layers[0].batch), key=lambda b: int(layers[0].seq_lens[b]))
-    warm = compact_host(layers[0], [probe])
-    dt = time_oracle(warm)
-    rate = max(int(layers[0].seq_lens[probe]) * KV_BYTES_PER_TOKEN / max(dt, 1e-6), 1e6)
-    picked, total_bytes = pick_sample(layers, rate * seconds)
-    elapsed = 0.0
-    for li, seqs in picked:
-        elapsed += time_oracle(compact_host(layers[li], seqs))
+    oracle.set_threads(threads)
+    try:
+        probe = min(range(layers[0].batch), key=lambda b: int(layers[0].seq_lens[b]))
+        warm = compact_host(layers[0], [probe])
+        dt = time_oracle(warm)
+        rate = max(int(layers[0].seq_lens[probe]) * KV_BYTES_PER_TOKEN / max(dt, 1e-6), 1e6)
+        picked, total_bytes = pick_sample(layers, rate * seconds)
+        elapsed = 0.0
+        for li, seqs in picked:
+            elapsed += time_oracle(compact_host(layers[li], seqs))
+    finally:
+        oracle.set_threads(1)
     n_seq = sum(len(s) for _, s in picked)
     all_seq = sum(w.batch for w in layers)
-    return {"value": total_bytes / elapsed / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+    _, model = host_cpu()
+    return {"value": total_bytes / elapsed / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": f"{n_seq} of {all_seq} sequences of the step ({total_bytes / 1e9:.3f} GB of KV), "
-                      f"{elapsed:.1f} s, single thread",
-            "seconds": elapsed}
+                      f"{elapsed:.1f} s, {threads} thread{'s' if threads > 1 else ''}",
+            "cpu_model": model, "seconds": elapsed}
 
 
 # ----------------------------------------------------------------------------
@@ -367,33 +391,35 @@ def run_gpu(args):
     if rc != 0:
         raise binding.QdaError(rc, "device status after warm-up")
 
-    # timed region: K steps, an event pair around every launch
     n_launch = args.steps * calls_per_step
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n_launch)]
-    barrier(dist, dev)
-    t0 = time.perf_counter()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    k = 0
-    for i in range(args.steps):
-        for c, _ in calls[i % rotate]:
-            ev[2 * k].record(stream)
-            rc = fn(*c)
-            ev[2 * k + 1].record(stream)
-            if rc != 0:
-                raise binding.QdaError(rc, "append_and_attend")
-            k += 1
-    end.record(stream)
-    torch.cuda.synchronize(dev)
-    t1 = time.perf_counter()
-    barrier(dist, dev)
+    if args.timing == "graph":
+        # The timed region replays one CUDA graph per step (graph i % rotate holds
+        # the calls of rotation set i % rotate): every call's kernel runs, back to
+        # back, with no host launch between them. Events bracket the K replays.
+        graphs = capture_graphs(calls, fn, dev, rotate)
+        for i in range(rotate):
+            graphs[i].replay()
+        torch.cuda.synchronize(dev)
+        barrier(dist, dev)
+        t0 = time.perf_counter()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(args.steps):
+            graphs[i % rotate].replay()
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        t1 = time.perf_counter()
+        barrier(dist, dev)
+        ms_local = start.elapsed_time(end)
+        kernel_ms = [ms_local / n_launch] * n_launch
+        del graphs
+    else:
+        t0, t1, ms_local, kernel_ms = timed_eager(args, calls, fn, dev, dist, stream, rotate, calls_per_step)
     clocks.stop()
     rc = attn.check()
     if rc != 0:
         raise binding.QdaError(rc, "device status after the timed region")
 
-    ms_local = start.elapsed_time(end)
-    kernel_ms = [ev[2 * j].elapsed_time(ev[2 * j + 1]) for j in range(n_launch)]
     ms = reduce_max(dist, ms_local, dev)
     ms_per_step = ms / args.steps
     # every rotation set has its own lengths (cfg2/cfg5 draw them); average the bytes per step
@@ -404,11 +430,24 @@ def run_gpu(args):
     value = kv_total / (ms_per_step * 1e-3) / 1e9
 
     # dominant kernel roofline: algorithmic bytes per launch / mean launch duration
-    mean_kernel_ms = statistics.fmean(kernel_ms)
+    mean_kernel_ms = reduce_max(dist, statistics.fmean(kernel_ms), dev)
     alg_per_launch = alg_per_step_local / calls_per_step
     peak, peak_kind = hbm_peak()
     achieved = alg_per_launch / (mean_kernel_ms * 1e-3) / 1e9
     traffic = traffic_per_launch(workload_key(args.workload, args.num_q_heads, T), args.num_q_heads, T)
+
+    # the other way of timing, for comparison: eager launches with an event pair around each
+    if args.timing == "graph":
+        _, _, e_ms, e_kernel = timed_eager(args, calls, fn, dev, dist, stream, rotate, calls_per_step)
+        other = {"timing": "eager launches, an event pair around each",
+                 "us_per_call": round(reduce_max(dist, e_ms, dev) * 1e3 / n_launch, 3),
+                 "kernel_us_mean": round(statistics.fmean(e_kernel) * 1e3, 3),
+                 "kernel_us_median": round(statistics.median(e_kernel) * 1e3, 3)}
+    else:
+        graph = run_graph(args, attn, calls, fn, dev, dist, rotate, calls_per_step, kv_per_step_local)
+        other = {"timing": "CUDA graph replay", **graph}
+    if attn.check() != 0:
+        raise RuntimeError("device status after the comparison timing")
 
     # end to end: per step the H2D copy of the step's inputs from pinned memory,
     # the call, and the D2H copy of o
@@ -440,6 +479,11 @@ def run_gpu(args):
                          "kernel_us_mean": round(mean_kernel_ms * 1e3, 3),
                          "kernel_us_median": round(statistics.median(kernel_ms) * 1e3, 3)},
             "e2e": e2e,
+            "timing": ("CUDA graph replay: one graph per step, K replays between two events; "
+                       "per-launch duration = region time / launches") if args.timing == "graph"
+                      else "eager launches, an event pair around each; per-launch duration = mean of the pairs",
+            ("eager" if args.timing == "graph" else "graph"): other,
+            "seq_per_s": round(first[0].batch / (ms_per_step * 1e-3) * world, 1),
             # one kernel per call on the 16-head decode kernel; attention + combine launches otherwise
             "gpu_launches": n_launch * (1 if kernel_key(args.num_q_heads, T) == 16 else 2),
             "clocks": clk,
@@ -449,10 +493,96 @@ def run_gpu(args):
     attn.close()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(first)
+        cores, _ = host_cpu()
+        if cores > 1:
+            result["cpu_baseline_all_cores"] = cpu_baseline(first, seconds=8.0, threads=cores)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if dist is not None:
         dist.destroy_process_group()
+
+
+def capture_graphs(calls, fn, dev, rotate):
+    """One CUDA graph per rotation set, each holding that set's calls (one step)."""
+    from decode_attention_qk_b200 import binding
+    graphs = []
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(torch.cuda.current_stream(dev))
+    for r in range(rotate):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            sp = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+            for c, _ in calls[r]:
+                rc = fn(*c[:-1], sp)
+                if rc != 0:
+                    raise binding.QdaError(rc, "capture")
+        graphs.append(g)
+    torch.cuda.current_stream(dev).wait_stream(cap)
+    return graphs
+
+
+def timed_eager(args, calls, fn, dev, dist, stream, rotate, calls_per_step):
+    """K steps of eager launches with an event pair around every launch.
+    Returns (t0, t1, region ms, per-launch ms list)."""
+    from decode_attention_qk_b200 import binding
+    n_launch = args.steps * calls_per_step
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n_launch)]
+    barrier(dist, dev)
+    t0 = time.perf_counter()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    k = 0
+    for i in range(args.steps):
+        for c, _ in calls[i % rotate]:
+            ev[2 * k].record(stream)
+            rc = fn(*c)
+            ev[2 * k + 1].record(stream)
+            if rc != 0:
+                raise binding.QdaError(rc, "append_and_attend")
+            k += 1
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    t1 = time.perf_counter()
+    barrier(dist, dev)
+    return t0, t1, start.elapsed_time(end), [ev[2 * j].elapsed_time(ev[2 * j + 1]) for j in range(n_launch)]
+
+
+def run_graph(args, attn, calls, fn, dev, dist, rotate, calls_per_step, kv_per_step):
+    """µs per call when the steps are replayed from a CUDA graph: one graph
+    holds a whole rotation cycle (rotate steps), replayed until at least
+    `steps` steps have run, timed by events around the replays."""
+    from decode_attention_qk_b200 import binding
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.graph(g, stream=cap):
+        sp = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+        for r in range(rotate):
+            for c, _ in calls[r]:
+                rc = fn(*c[:-1], sp)
+                if rc != 0:
+                    raise binding.QdaError(rc, "capture")
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(2):
+        g.replay()
+    replays = max(1, math.ceil(args.steps / rotate))
+    barrier(dist, dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(replays):
+        g.replay()
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    if attn.check() != 0:
+        raise RuntimeError("device status after the graph replays")
+    ms = reduce_max(dist, start.elapsed_time(end), dev)
+    steps = replays * rotate
+    ms_per_step = ms / steps
+    kv_total = reduce_sum(dist, kv_per_step, dev)
+    del g
+    return {"us_per_call": round(ms_per_step * 1e3 / calls_per_step, 3), "ms_per_step": round(ms_per_step, 6),
+            "value": round(kv_total / (ms_per_step * 1e-3) / 1e9, 2), "unit": "GB/s", "steps": steps}
 
 
 def run_e2e(args, attn, sets, dev, stream, dist, rotate):
@@ -574,6 +704,8 @@ def run_reference(args):
         return
     import oracle
     oracle.build()
+    cores, cpu_model = host_cpu()
+    oracle.set_threads(cores)
     layers = make_layers(args.workload, "cpu", 0, args.num_q_heads, args.new_tokens)
     # size each step's sample so that warm-up + timed steps take ~2 minutes
     probe = min(range(layers[0].batch), key=lambda b: int(layers[0].seq_lens[b]))
@@ -610,7 +742,7 @@ def run_reference(args):
     ms_per_step = elapsed * 1e3 / args.steps
     all_seq = sum(w.batch for w in layers)
     sample_desc = (f"per step a window of the step's sequences ({nbytes / args.steps / 1e6:.1f} MB of KV, "
-                   f"{nseq / args.steps:.1f} of {all_seq} sequences on average), single thread")
+                   f"{nseq / args.steps:.1f} of {all_seq} sequences on average), {cores} threads")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3),
@@ -623,8 +755,8 @@ def run_reference(args):
                    "batch": layers[0].batch, "layers_per_step": len(layers), "new_tokens": args.new_tokens,
                    "page_size": 16,
                    "heads": f"{args.num_q_heads} q / 8 kv, D=128"},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": sample_desc},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample_desc, "cpu_model": cpu_model},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
@@ -640,6 +772,9 @@ def main(argv=None):
                     help="query heads: 16 = Qwen3-0.6B (the default workload); 32/40/64 = 4B-8B/14B/32B")
     ap.add_argument("--new-tokens", type=int, default=1,
                     help="new tokens per sequence (1 = decode; 2-4 at 16 heads, 2 at 32: several tokens at once)")
+    ap.add_argument("--timing", choices=["graph", "eager"], default="graph",
+                    help="timed region: CUDA graph replay of the steps (default) or eager launches with "
+                         "an event pair around each; the line also carries the other figure")
     ap.add_argument("--rotate", type=int, default=0, help="resident input sets cycled (0: enough to defeat L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -31,7 +31,7 @@ _ERRORS = {-1: "invalid argument", -4: "seq_len or block-table entry out of rang
 def build(force: bool = False) -> str:
     """Compile the oracle with gcc (IEEE double, no contraction into FMA)."""
     if force or not os.path.exists(LIBRARY) or os.path.getmtime(LIBRARY) < os.path.getmtime(SOURCE):
-        cmd = ["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math",
+        cmd = ["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
                "-shared", "-fPIC", "-o", LIBRARY, SOURCE, "-lm"]
         subprocess.run(cmd, check=True)
     return LIBRARY
@@ -65,12 +65,25 @@ def _load():
             u16p, u16p, u16p, i32p, i32p, i32p, ctypes.c_int, u16p, u16p, ctypes.c_int,
             dp, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_double, dp, dp]
         lib.oracle_append_and_attend_gqa.restype = ctypes.c_int
+        lib.oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_threads.restype = None
+        lib.oracle_get_threads.argtypes = []
+        lib.oracle_get_threads.restype = ctypes.c_int
         lib.oracle_append_and_attend_tokens.argtypes = [
             u16p, u16p, u16p, i32p, i32p, i32p, ctypes.c_int, u16p, u16p, ctypes.c_int,
             dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_double, dp, dp]
         lib.oracle_append_and_attend_tokens.restype = ctypes.c_int
         _lib = lib
     return _lib
+
+
+def set_threads(n: int) -> None:
+    """Threads the step's attention loop uses (default 1); results do not depend on it."""
+    _load().oracle_set_threads(int(n))
+
+
+def get_threads() -> int:
+    return int(_load().oracle_get_threads())
 
 
 def _ptr(a: np.ndarray | None, ctype):

@@ -45,6 +45,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 /* Constants of the Qwen3-0.6B Model Spec ("Published configuration" and the
  * attn.* rows of "Compute-graph nodes"). */
@@ -179,6 +182,17 @@ void oracle_decode_head(const double *q, int L, const int32_t *bt_row,
     }
 }
 
+/* ---- threads -------------------------------------------------------------- */
+
+/* Threads the attention loop of the step may use (default 1). Test and
+ * baseline infrastructure only: the timed CPU baseline reports both one
+ * thread and every host core. */
+static int g_threads = 1;
+
+void oracle_set_threads(int n) { g_threads = n < 1 ? 1 : (n > 256 ? 256 : n); }
+
+int oracle_get_threads(void) { return g_threads; }
+
 /* ---- the whole step ------------------------------------------------------ */
 
 /* The attention step for a batch with T new tokens per sequence, in the
@@ -280,20 +294,31 @@ int oracle_append_and_attend_tokens(const uint16_t *qkv, const uint16_t *q_norm_
     }
 
     /* Causal attention over the cache as it stands after every append: new
-     * token t reads the L - T + t + 1 slots up to and including its own. */
+     * token t reads the L - T + t + 1 slots up to and including its own.
+     * Every (sequence, token, head) row is computed on its own, by the same
+     * sequential code whatever the thread count (oracle_set_threads), so the
+     * result does not depend on it. */
     int max_L = 0;
     for (int b = 0; b < B; ++b) if (seq_lens[b] > max_L) max_L = seq_lens[b];
-    double *scores = (double *)malloc(sizeof(double) * (size_t)max_L);
+    const int nthreads = g_threads;
+    double *scores = (double *)malloc(sizeof(double) * (size_t)max_L * (size_t)nthreads);
     if (!scores) { free(q_all); return ORC_ERR_ARG; }
-    for (int b = 0; b < B; ++b) {
-        for (int t = 0; t < T; ++t) {
-            int visible = seq_lens[b] - T + t + 1;
-            for (int h = 0; h < num_q_heads; ++h) {
-                size_t r = ((size_t)b * T + t) * num_q_heads + h;
-                oracle_decode_head(q_all + r * ORC_HEAD_DIM, visible, block_table + (size_t)b * bt_stride,
-                                   k_cache, v_cache, h / group, scores, o + r * ORC_HEAD_DIM);
-            }
-        }
+    const long rows = (long)B * T * num_q_heads;
+#ifdef _OPENMP
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1) if (nthreads > 1)
+#endif
+    for (long r = 0; r < rows; ++r) {
+        const int h = (int)(r % num_q_heads);
+        const int t = (int)((r / num_q_heads) % T);
+        const int b = (int)(r / ((long)num_q_heads * T));
+        const int visible = seq_lens[b] - T + t + 1;
+#ifdef _OPENMP
+        double *sc = scores + (size_t)omp_get_thread_num() * (size_t)max_L;
+#else
+        double *sc = scores;
+#endif
+        oracle_decode_head(q_all + (size_t)r * ORC_HEAD_DIM, visible, block_table + (size_t)b * bt_stride,
+                           k_cache, v_cache, h / group, sc, o + (size_t)r * ORC_HEAD_DIM);
     }
     if (q_out) memcpy(q_out, q_all, sizeof(double) * (size_t)B * T * q_width);
     free(scores);

@@ -558,3 +558,21 @@ def test_tokens_default_positions(oracle_mod):
     o1 = oracle_mod.append_and_attend_tokens(**a)["o"]
     o2 = oracle_mod.append_and_attend_tokens(**a, positions=w.seq_lens.numpy() - 2)["o"]
     assert np.array_equal(o1, o2)
+
+
+def test_thread_count_does_not_change_the_result(oracle_mod):
+    """The step's attention loop may run on several threads (for the timed CPU
+    baseline); every row is the same sequential computation either way."""
+    from decode_attention_qk_b200 import inputs
+    w = inputs.custom([300, 1000, 17, 2, 64], seed=77, gap_fraction=0.3, num_q_heads=32, new_tokens=2)
+    args = (inputs.bf16_bits(w.qkv), inputs.bf16_bits(w.q_norm_w), inputs.bf16_bits(w.k_norm_w),
+            w.seq_lens.numpy(), w.block_table.numpy(), inputs.bf16_bits(w.k_cache), inputs.bf16_bits(w.v_cache))
+    one = oracle_mod.append_and_attend_tokens(*args)
+    oracle_mod.set_threads(4)
+    try:
+        four = oracle_mod.append_and_attend_tokens(*args)
+    finally:
+        oracle_mod.set_threads(1)
+    assert oracle_mod.get_threads() == 1
+    assert np.array_equal(one["o"], four["o"])
+    assert np.array_equal(one["k_cache"], four["k_cache"]) and np.array_equal(one["v_cache"], four["v_cache"])
