@@ -211,6 +211,23 @@ def config5(device="cpu", seed: int = 5000, num_q_heads: int = NUM_Q_HEADS, new_
                     seq_lens=seq_lens, block_table=bt, num_pages=pool, **vals)
 
 
+HIDDEN = 1024   # Qwen3-0.6B hidden size (Model Spec, "Compute-graph nodes": input_norm H=1024)
+
+
+def hidden_inputs(B: int, seed: int = 0, device="cpu", hidden: int = HIDDEN,
+                  num_q_heads: int = NUM_Q_HEADS) -> dict:
+    """Inputs of input_norm + attn.qkv_proj: x bf16 [B, hidden] ~ N(0, 1); the
+    input_norm gain bf16 [hidden] = 1 + U(-0.5, 0.5) (perturbed away from 1, as
+    the conformance method does); the qkv_proj weight bf16 [(Hq + 16) * 128,
+    hidden] ~ N(0, 1/hidden), so that the outputs stay O(1)."""
+    dev = torch.device(device)
+    N = qkv_width(num_q_heads)
+    x = torch.randn((B, hidden), generator=_gen(seed * 16 + 6, dev), device=dev).to(torch.bfloat16)
+    g = (torch.rand(hidden, generator=_gen(seed * 16 + 7, dev), device=dev) + 0.5).to(torch.bfloat16)
+    w = (torch.randn((N, hidden), generator=_gen(seed * 16 + 8, dev), device=dev) / math.sqrt(hidden)).to(torch.bfloat16)
+    return dict(x=x, input_norm_w=g, w_qkv=w)
+
+
 def bf16_bits(t: torch.Tensor):
     """numpy uint16 view of a bf16 tensor's bits (copied to the host)."""
     return t.detach().to("cpu").contiguous().view(torch.int16).numpy().view("uint16")

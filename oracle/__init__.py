@@ -65,6 +65,9 @@ def _load():
             u16p, u16p, u16p, i32p, i32p, i32p, ctypes.c_int, u16p, u16p, ctypes.c_int,
             dp, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_double, dp, dp]
         lib.oracle_append_and_attend_gqa.restype = ctypes.c_int
+        lib.oracle_input_norm_qkv_proj.argtypes = [u16p, u16p, u16p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                    ctypes.c_double, dp, u16p]
+        lib.oracle_input_norm_qkv_proj.restype = ctypes.c_int
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_set_threads.restype = None
         lib.oracle_get_threads.argtypes = []
@@ -75,6 +78,26 @@ def _load():
         lib.oracle_append_and_attend_tokens.restype = ctypes.c_int
         _lib = lib
     return _lib
+
+
+def input_norm_qkv_proj(x, norm_w, w, rms_eps: float = 1e-6) -> dict:
+    """input_norm then attn.qkv_proj (Model Spec, "Compute-graph nodes"): x bf16 bits
+    [B, K], norm_w [K], w [N, K] (row n = output n). Returns ``y`` float64 [B, N]
+    (exact) and ``bits`` uint16 [B, N] (y rounded once to bf16, nearest-even)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    norm_w = np.ascontiguousarray(norm_w, dtype=np.uint16)
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    assert x.ndim == 2 and w.ndim == 2 and w.shape[1] == x.shape[1] and norm_w.shape == (x.shape[1],)
+    B, K = x.shape
+    N = w.shape[0]
+    y = np.empty((B, N), dtype=np.float64)
+    bits = np.empty((B, N), dtype=np.uint16)
+    rc = _load().oracle_input_norm_qkv_proj(_ptr(x, ctypes.c_uint16), _ptr(norm_w, ctypes.c_uint16),
+                                            _ptr(w, ctypes.c_uint16), B, K, N, rms_eps,
+                                            _ptr(y, ctypes.c_double), _ptr(bits, ctypes.c_uint16))
+    if rc != 0:
+        raise ValueError(f"oracle_input_norm_qkv_proj: {_ERRORS.get(rc, rc)}")
+    return {"y": y, "bits": bits}
 
 
 def set_threads(n: int) -> None:

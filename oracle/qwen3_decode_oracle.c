@@ -37,6 +37,10 @@
  *     bf16 with round-to-nearest-even when it is written to the cache; the
  *     attention then reads the cache as stored (the rounded k); o stays double.
  *
+ * It also holds the two nodes that produce the step's input, input_norm and
+ * attn.qkv_proj (oracle_input_norm_qkv_proj), with nothing rounded before the
+ * bf16 qkv row.
+ *
  * Every function names the passage it follows. The pins that tie this file to
  * the pages and to mathematics (closed forms, invariants, library routines,
  * brute force) live in tests/test_oracle_pins.py.
@@ -351,6 +355,49 @@ int oracle_append_and_attend(const uint16_t *qkv, const uint16_t *q_norm_w,
     return oracle_append_and_attend_gqa(qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table,
                                         bt_stride, k_cache, v_cache, num_pages, o, B,
                                         ORC_NUM_Q_HEADS, rope_theta, rms_eps, q_out, k_out);
+}
+
+/* ---- input_norm + attn.qkv_proj (the step's input) ------------------------ */
+
+/* The two nodes before the attention step, in the order of the Model Spec's
+ * "Compute-graph nodes" table: input_norm (rmsnorm over H = hidden, eps) and
+ * attn.qkv_proj (linear, y[t,n] = sum_k x[t,k] * w[n,k], K = hidden,
+ * N = (num_q_heads + 16) * 128, no bias: the parameter count leaves none).
+ * Rows t are the B sequences' new tokens.
+ *
+ *   x        bf16 [B][K]   the hidden state entering the layer
+ *   norm_w   bf16 [K]      input_norm gain
+ *   w        bf16 [N][K]   qkv_proj weight, row n = output feature n
+ *   y_out    double [B][N] the exact (double) projection, or NULL
+ *   y_bits   bf16 [B][N]   y rounded once to bf16 (nearest-even), or NULL
+ *
+ * Nothing is rounded before y (the normalised x stays double). The sum over
+ * k runs in index order. Returns 0 or ORC_ERR_ARG. */
+int oracle_input_norm_qkv_proj(const uint16_t *x, const uint16_t *norm_w, const uint16_t *w,
+                               int B, int K, int N, double eps, double *y_out, uint16_t *y_bits)
+{
+    if (!x || !norm_w || !w || B < 1 || K < 1 || N < 1 || !(eps >= 0.0) || (!y_out && !y_bits))
+        return ORC_ERR_ARG;
+    double *g = (double *)malloc(sizeof(double) * (size_t)K);
+    double *row = (double *)malloc(sizeof(double) * (size_t)K);
+    double *xn = (double *)malloc(sizeof(double) * (size_t)K);
+    if (!g || !row || !xn) { free(g); free(row); free(xn); return ORC_ERR_ARG; }
+    for (int k = 0; k < K; ++k) g[k] = oracle_bf16_to_f64(norm_w[k]);
+    for (int b = 0; b < B; ++b) {
+        for (int k = 0; k < K; ++k) row[k] = oracle_bf16_to_f64(x[(size_t)b * K + k]);
+        oracle_rmsnorm(row, g, K, eps, xn);                        /* input_norm */
+        for (int n = 0; n < N; ++n) {                              /* attn.qkv_proj */
+            const uint16_t *wn = w + (size_t)n * K;
+            double acc = 0.0;
+            for (int k = 0; k < K; ++k) acc += xn[k] * oracle_bf16_to_f64(wn[k]);
+            if (y_out) y_out[(size_t)b * N + n] = acc;
+            if (y_bits) y_bits[(size_t)b * N + n] = oracle_f64_to_bf16_rne(acc);
+        }
+    }
+    free(g);
+    free(row);
+    free(xn);
+    return 0;
 }
 
 /* ---- array forms of the conversions, for the tests ---------------------- */
