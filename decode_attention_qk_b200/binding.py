@@ -79,6 +79,11 @@ def load_library():
         lib.qwen3_decode_attn_append_and_attend_host.restype = ctypes.c_int
         lib.qwen3_decode_attn_append_and_attend_tokens.argtypes = call[:-1] + [ctypes.c_int, vp]
         lib.qwen3_decode_attn_append_and_attend_tokens.restype = ctypes.c_int
+        lib.qwen3_decode_attn_qkv_proj.argtypes = [vp, vp, vp, vp, ctypes.c_int, vp, ctypes.c_int, vp]
+        lib.qwen3_decode_attn_qkv_proj.restype = ctypes.c_int
+        lib.qwen3_decode_attn_from_hidden.argtypes = [vp, vp, vp, vp, ctypes.c_int, vp, vp, vp, i32p, i32p, i32p,
+                                                      ctypes.c_int, vp, vp, ctypes.c_int, vp, ctypes.c_int, vp]
+        lib.qwen3_decode_attn_from_hidden.restype = ctypes.c_int
         lib.qwen3_decode_attn_check.argtypes = [vp, vp]
         lib.qwen3_decode_attn_check.restype = ctypes.c_int
         lib.qwen3_decode_attn_grid_ctas.argtypes = [vp]
@@ -201,6 +206,40 @@ def qwen3_decode_attn_append_and_attend_tokens(handle, qkv, q_norm_w, k_norm_w, 
         raise QdaError(rc, "qwen3_decode_attn_append_and_attend_tokens")
 
 
+def _proj_args(qkv_width, x, input_norm_w, w_qkv, qkv, dev):
+    if x.dim() != 2:
+        raise ValueError("x must be [B, hidden]")
+    B, hidden = int(x.shape[0]), int(x.shape[1])
+    _expect(x, "x", torch.bfloat16, (B, hidden), dev)
+    _expect(input_norm_w, "input_norm_w", torch.bfloat16, (hidden,), dev)
+    _expect(w_qkv, "w_qkv", torch.bfloat16, (qkv_width, hidden), dev)
+    _expect(qkv, "qkv", torch.bfloat16, (B, qkv_width), dev)
+    return B, hidden
+
+
+def qwen3_decode_attn_qkv_proj(handle, num_q_heads, x, input_norm_w, w_qkv, qkv, stream=None) -> None:
+    """input_norm + attn.qkv_proj on device tensors: x [B, hidden], input_norm_w [hidden],
+    w_qkv [(Hq + 16) * 128, hidden] (rows q | k | v), qkv [B, (Hq + 16) * 128] (output)."""
+    dev = x.device
+    B, hidden = _proj_args((num_q_heads + 2 * NUM_KV_HEADS) * HEAD_DIM, x, input_norm_w, w_qkv, qkv, dev)
+    rc = load_library().qwen3_decode_attn_qkv_proj(handle, _ptr(x), _ptr(input_norm_w), _ptr(w_qkv), hidden,
+                                                   _ptr(qkv), B, _stream(stream, dev))
+    if rc != QDA_OK:
+        raise QdaError(rc, "qwen3_decode_attn_qkv_proj")
+
+
+def qwen3_decode_attn_from_hidden(handle, num_q_heads, x, input_norm_w, w_qkv, qkv, q_norm_w, k_norm_w, seq_lens,
+                                  positions, block_table, k_cache, v_cache, o, stream=None) -> None:
+    """qkv_proj into `qkv`, then the attention step on it (one new token per sequence)."""
+    dev = x.device
+    B, hidden = _proj_args((num_q_heads + 2 * NUM_KV_HEADS) * HEAD_DIM, x, input_norm_w, w_qkv, qkv, dev)
+    args = _step_args(qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, k_cache, v_cache, o, dev, dev)
+    rc = load_library().qwen3_decode_attn_from_hidden(handle, _ptr(x), _ptr(input_norm_w), _ptr(w_qkv), hidden,
+                                                      *args, _stream(stream, dev))
+    if rc != QDA_OK:
+        raise QdaError(rc, "qwen3_decode_attn_from_hidden")
+
+
 def qwen3_decode_attn_append_and_attend_host(handle, qkv, q_norm_w, k_norm_w, seq_lens, positions,
                                              block_table, k_cache, v_cache, o, stream=None) -> None:
     """The step with per-step tensors (qkv, seq_lens, positions, block_table, o) in host
@@ -276,6 +315,26 @@ class DecodeAttention:
         step = qwen3_decode_attn_append_and_attend_tokens if qkv.dim() == 3 else qwen3_decode_attn_append_and_attend
         step(self.handle, qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, k_cache, v_cache, o, stream)
         return o
+
+    def qkv_proj(self, x, input_norm_w, w_qkv, qkv=None, stream=None) -> torch.Tensor:
+        """input_norm + attn.qkv_proj: the step's qkv [B, (Hq + 16) * 128] from x [B, hidden]."""
+        if qkv is None:
+            qkv = torch.empty((x.shape[0], (self.config.num_q_heads + 16) * HEAD_DIM), dtype=torch.bfloat16,
+                              device=x.device)
+        qwen3_decode_attn_qkv_proj(self.handle, self.config.num_q_heads, x, input_norm_w, w_qkv, qkv, stream)
+        return qkv
+
+    def from_hidden(self, x, input_norm_w, w_qkv, q_norm_w, k_norm_w, seq_lens, block_table, k_cache, v_cache,
+                    qkv=None, o=None, positions=None, stream=None):
+        """The attention from the hidden state: returns (o, qkv)."""
+        B = x.shape[0]
+        if qkv is None:
+            qkv = torch.empty((B, (self.config.num_q_heads + 16) * HEAD_DIM), dtype=torch.bfloat16, device=x.device)
+        if o is None:
+            o = torch.empty((B, self.config.num_q_heads, HEAD_DIM), dtype=torch.bfloat16, device=x.device)
+        qwen3_decode_attn_from_hidden(self.handle, self.config.num_q_heads, x, input_norm_w, w_qkv, qkv, q_norm_w,
+                                      k_norm_w, seq_lens, positions, block_table, k_cache, v_cache, o, stream)
+        return o, qkv
 
     def check(self, stream=None) -> int:
         return qwen3_decode_attn_check(self.handle, stream, self.device)

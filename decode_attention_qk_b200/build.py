@@ -15,7 +15,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libqwen3_decode_attn.so")
-SOURCES = [os.path.join(CSRC, f) for f in ("qda_decode_kernel.cu", "qda_decode_mma.cu", "qda_api.cu", "qda_noalloc.cu")]
+SOURCES = [os.path.join(CSRC, f) for f in ("qda_decode_kernel.cu", "qda_decode_mma.cu", "qda_qkv_proj.cu", "qda_api.cu",
+                                           "qda_noalloc.cu")]
 HEADERS = [os.path.join(CSRC, "qda_internal.h"), os.path.join(CSRC, "qda_device.cuh"),
            os.path.join(INCLUDE, "qwen3_decode_attn.h")]
 

@@ -126,6 +126,34 @@ cudaError_t launch_step(const qda_handle* h, const qda::Params& p, cudaStream_t 
                                                                  : qda::launch_grouped(p, h->grid, stream);
 }
 
+// Host checks of the input_norm + qkv_proj arguments.
+int check_proj(const qda_handle* h, const void* x, const void* input_norm_w, const void* w_qkv, int hidden,
+               const void* qkv, int batch) {
+    if (h == nullptr || x == nullptr || input_norm_w == nullptr || w_qkv == nullptr || qkv == nullptr)
+        return QDA_ERR_INVALID_ARG;
+    if (batch < 1 || batch > h->cfg.max_batch || hidden < 256 || hidden > qda::kMaxHidden || hidden % 256 != 0)
+        return QDA_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(input_norm_w, 16) || !aligned(w_qkv, 16) || !aligned(qkv, 16))
+        return QDA_ERR_INVALID_ARG;
+    return QDA_OK;
+}
+
+qda::QkvProjParams make_proj_params(const qda_handle* h, const void* x, const void* input_norm_w, const void* w_qkv,
+                                    int hidden, void* qkv, int batch) {
+    qda::QkvProjParams p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.norm_w = static_cast<const uint16_t*>(input_norm_w);
+    p.w = static_cast<const uint16_t*>(w_qkv);
+    p.y = static_cast<uint16_t*>(qkv);
+    p.batch = batch;
+    p.hidden = hidden;
+    p.qkv_width = (int)qkv_elems(h->cfg.num_q_heads);
+    p.eps = h->cfg.rms_eps;
+    p.status = h->status;
+    p.timeout_ns = h->cfg.wait_timeout_ns > 0 ? h->cfg.wait_timeout_ns : kDefaultTimeoutNs;
+    return p;
+}
+
 }  // namespace
 
 extern "C" {
@@ -168,7 +196,9 @@ int qwen3_decode_attn_create(const qda_config* cfg, int device, qda_handle** out
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms < 1)
         return QDA_ERR_CUDA;
-    if (qda::prepare_device() != cudaSuccess || qda::prepare_grouped() != cudaSuccess) return QDA_ERR_CUDA;
+    if (qda::prepare_device() != cudaSuccess || qda::prepare_grouped() != cudaSuccess ||
+        qda::prepare_qkv_proj() != cudaSuccess)
+        return QDA_ERR_CUDA;
 
     qda_handle* h = new (std::nothrow) qda_handle();
     if (h == nullptr) return QDA_ERR_CUDA;
@@ -232,6 +262,36 @@ int qwen3_decode_attn_append_and_attend_tokens(qda_handle* h, const void* qkv, c
                                 k_cache, v_cache, num_pages, o, batch);
     p.new_tokens = new_tokens;
     return launch_step(h, p, static_cast<cudaStream_t>(cuda_stream)) == cudaSuccess ? QDA_OK : QDA_ERR_CUDA;
+}
+
+int qwen3_decode_attn_qkv_proj(qda_handle* h, const void* x, const void* input_norm_w, const void* w_qkv, int hidden,
+                               void* qkv, int batch, void* cuda_stream) {
+    int rc = check_proj(h, x, input_norm_w, w_qkv, hidden, qkv, batch);
+    if (rc != QDA_OK) return rc;
+    DeviceGuard guard(h->device);
+    if (!guard.ok()) return QDA_ERR_CUDA;
+    const qda::QkvProjParams p = make_proj_params(h, x, input_norm_w, w_qkv, hidden, qkv, batch);
+    return qda::launch_qkv_proj(p, static_cast<cudaStream_t>(cuda_stream)) == cudaSuccess ? QDA_OK : QDA_ERR_CUDA;
+}
+
+int qwen3_decode_attn_from_hidden(qda_handle* h, const void* x, const void* input_norm_w, const void* w_qkv,
+                                  int hidden, void* qkv, const void* q_norm_w, const void* k_norm_w,
+                                  const int32_t* seq_lens, const int32_t* positions, const int32_t* block_table,
+                                  int block_table_stride, void* k_cache, void* v_cache, int num_pages, void* o,
+                                  int batch, void* cuda_stream) {
+    int rc = check_proj(h, x, input_norm_w, w_qkv, hidden, qkv, batch);
+    if (rc != QDA_OK) return rc;
+    rc = check_call(h, qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, block_table_stride, k_cache,
+                    v_cache, num_pages, o, batch);
+    if (rc != QDA_OK) return rc;
+    DeviceGuard guard(h->device);
+    if (!guard.ok()) return QDA_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    const qda::QkvProjParams pp = make_proj_params(h, x, input_norm_w, w_qkv, hidden, qkv, batch);
+    if (qda::launch_qkv_proj(pp, st) != cudaSuccess) return QDA_ERR_CUDA;
+    const qda::Params p = make_params(h, qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table,
+                                      block_table_stride, k_cache, v_cache, num_pages, o, batch);
+    return launch_step(h, p, st) == cudaSuccess ? QDA_OK : QDA_ERR_CUDA;
 }
 
 int qwen3_decode_attn_append_and_attend_host(qda_handle* h, const void* qkv_host, const void* q_norm_w,

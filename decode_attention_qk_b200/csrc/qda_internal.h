@@ -79,6 +79,26 @@ cudaError_t launch(const Params& p, int grid, cudaStream_t stream);
 // launch that combines the partials of sequences split across CTAs.
 cudaError_t launch_grouped(const Params& p, int grid, cudaStream_t stream);
 
+// input_norm + attn.qkv_proj (qda_qkv_proj.cu): hidden size a multiple of 256,
+// at most kMaxHidden (the Qwen3 sizes: 1024, 2048, 2560, 4096, 5120).
+constexpr int kMaxHidden = 8192;
+
+struct QkvProjParams {
+    const uint16_t* x;        // bf16 [batch][hidden]
+    const uint16_t* norm_w;   // bf16 [hidden], input_norm gain
+    const uint16_t* w;        // bf16 [qkv_width][hidden], row n = output feature n
+    uint16_t* y;              // bf16 [batch][qkv_width]
+    int batch;
+    int hidden;
+    int qkv_width;            // (num_q_heads + 16) * 128, a multiple of 32
+    double eps;
+    int* status;
+    int64_t timeout_ns;
+};
+
+cudaError_t prepare_qkv_proj();
+cudaError_t launch_qkv_proj(const QkvProjParams& p, cudaStream_t stream);
+
 // Whether the tensor-core kernel has an instance for this head and token count.
 bool grouped_supported(int num_q_heads, int new_tokens);
 

@@ -208,6 +208,57 @@ int qwen3_decode_attn_append_and_attend_tokens(qda_handle *h,
                                                int new_tokens,
                                                void *cuda_stream);
 
+/* The step's input, from the hidden state: input_norm then attn.qkv_proj
+ * (Model Spec, "Compute-graph nodes": rmsnorm over H = hidden with a gain
+ * per feature and eps = the handle's rms_eps; then y[t,n] = sum_k x[t,k]
+ * w[n,k], no bias), one launch:
+ *   qkv[b,n] = sum_k (x[b,k] / sqrt(sum_j x[b,j]^2 / hidden + eps) * g[k]) * w_qkv[n,k]
+ * Layouts (device pointers, 16-byte aligned): x bf16 [B][hidden] (row
+ * stride hidden); input_norm_w bf16 [hidden]; w_qkv bf16 [N][hidden] with
+ * N = (num_q_heads + 16) * 128 of the handle (row n = output feature n, the
+ * layout of a torch Linear weight; q rows, then k rows, then v rows); qkv
+ * bf16 [B][N] (output). hidden is a multiple of 256 in [256, 8192]
+ * (Qwen3: 1024 for 0.6B, 2048, 2560, 4096, 5120 for the larger sizes).
+ * Nothing is rounded before qkv, which is rounded once to bf16: the products
+ * x*g are split exactly into two bf16 terms for the tensor cores and summed
+ * in float, so qkv is the correctly rounded value except where the float sum
+ * lies within about 2^-19 (relative) of a rounding midpoint, where it may be
+ * the neighbouring bf16 value.
+ * Errors: INVALID_ARG (null or misaligned pointer, batch outside
+ * [1, max_batch], hidden not a multiple of 256 in range), CUDA (the launch
+ * failed); a wait that ran out on the device goes to the status word. */
+int qwen3_decode_attn_qkv_proj(qda_handle *h,
+                               const void *x,
+                               const void *input_norm_w,
+                               const void *w_qkv,
+                               int hidden,
+                               void *qkv,
+                               int batch,
+                               void *cuda_stream);
+
+/* qwen3_decode_attn_qkv_proj into `qkv` (caller-owned, bf16 [B][N], it
+ * holds the step's qkv afterwards), then qwen3_decode_attn_append_and_attend
+ * on it: the layer's attention from the hidden state, two or three launches
+ * on `cuda_stream`. Arguments and errors as for those two calls. */
+int qwen3_decode_attn_from_hidden(qda_handle *h,
+                                  const void *x,
+                                  const void *input_norm_w,
+                                  const void *w_qkv,
+                                  int hidden,
+                                  void *qkv,
+                                  const void *q_norm_w,
+                                  const void *k_norm_w,
+                                  const int32_t *seq_lens,
+                                  const int32_t *positions,
+                                  const int32_t *block_table,
+                                  int block_table_stride,
+                                  void *k_cache,
+                                  void *v_cache,
+                                  int num_pages,
+                                  void *o,
+                                  int batch,
+                                  void *cuda_stream);
+
 /* The same step for a caller whose per-step tensors are in HOST memory:
  * qkv_host, seq_lens_host, positions_host (or NULL) and block_table_host are
  * host pointers (pinned memory makes the copies asynchronous), and o_host is
