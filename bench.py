@@ -34,6 +34,7 @@ if ROOT not in sys.path:
 from decode_attention_qk_b200 import inputs  # noqa: E402
 
 METRIC = "decode-attn KV GB/s and µs/call (1 B200) as fraction of HBM roofline"
+PROJ_METRIC = "input_norm + qkv_proj GB/s (weight + x + gain + qkv bytes) and µs/call (1 B200)"
 KV_BYTES_PER_TOKEN = 2 * inputs.NUM_KV_HEADS * inputs.HEAD_DIM * 2      # K and V rows: 4096 B
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
@@ -44,6 +45,7 @@ _CSRC = os.path.join(ROOT, "decode_attention_qk_b200", "csrc")
 KERNEL_SOURCES = {   # the files each attention kernel is built from
     16: [os.path.join(_CSRC, f) for f in ("qda_decode_kernel.cu", "qda_device.cuh", "qda_internal.h")],
     "grouped": [os.path.join(_CSRC, f) for f in ("qda_decode_mma.cu", "qda_device.cuh", "qda_internal.h")],
+    "qkv_proj": [os.path.join(_CSRC, f) for f in ("qda_qkv_proj.cu", "qda_device.cuh", "qda_internal.h")],
 }
 
 WORKLOADS = {
@@ -97,6 +99,25 @@ def algorithmic_bytes(seq_lens, num_q_heads: int = 16, new_tokens: int = 1) -> i
             + pages * 4 + B * 4 + 2 * inputs.HEAD_DIM * 2)
 
 
+def proj_bytes(batch: int, hidden: int = inputs.HIDDEN, num_q_heads: int = 16) -> int:
+    """Least HBM traffic of input_norm + qkv_proj: the weight, x, the gain and qkv."""
+    N = inputs.qkv_width(num_q_heads)
+    return N * hidden * 2 + batch * hidden * 2 + hidden * 2 + batch * N * 2
+
+
+def proj_flops(batch: int, hidden: int = inputs.HIDDEN, num_q_heads: int = 16) -> int:
+    """Multiply-adds of the projection, 2 flops each (the hi/lo split doubles the tensor work)."""
+    return 2 * batch * inputs.qkv_width(num_q_heads) * hidden
+
+
+def tensor_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback"
+
+
 def hbm_peak():
     try:
         with open(PEAKS_FILE) as f:
@@ -114,9 +135,9 @@ def workload_key(workload: str, num_q_heads: int = 16, new_tokens: int = 1) -> s
     return workload + ("" if num_q_heads == 16 else f"-h{num_q_heads}") + ("" if new_tokens == 1 else f"-t{new_tokens}")
 
 
-def kernel_source_hash(num_q_heads: int = 16, new_tokens: int = 1) -> str:
+def kernel_source_hash(num_q_heads: int = 16, new_tokens: int = 1, key=None) -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES[kernel_key(num_q_heads, new_tokens)]:
+    for p in KERNEL_SOURCES[key if key is not None else kernel_key(num_q_heads, new_tokens)]:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -334,6 +355,51 @@ def cpu_baseline(layers, seconds: float = 12.0, threads: int = 1):
             "cpu_model": model, "seconds": elapsed}
 
 
+def time_proj_oracle(w, rows) -> float:
+    """Seconds the oracle's input_norm + qkv_proj takes for the given rows of layer w."""
+    import oracle
+    d = w.hidden_in
+    sel = torch.tensor(list(rows), dtype=torch.int64, device=d["x"].device)
+    x = inputs.bf16_bits(d["x"].index_select(0, sel))
+    g, wq = inputs.bf16_bits(d["input_norm_w"]), inputs.bf16_bits(d["w_qkv"])
+    t0 = time.perf_counter()
+    oracle.input_norm_qkv_proj(x, g, wq)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline_proj(layers, mode, seconds: float = 12.0, threads: int = 1):
+    """The oracle on a bounded sample of the projection modes: qkv_proj alone
+    (value = projection bytes / s), or from the hidden state (the projection
+    of the sampled sequences plus their attention; value = K/V bytes / s)."""
+    import oracle
+    oracle.build()
+    oracle.set_threads(threads)
+    w0 = layers[0]
+    hidden = w0.hidden_in["x"].shape[1]
+    try:
+        per_row = time_proj_oracle(w0, [0])
+        if mode == "qkv_proj":
+            rows = list(range(min(w0.batch, max(1, int(seconds / max(per_row, 1e-6))))))
+            elapsed = time_proj_oracle(w0, rows)
+            units = proj_bytes(len(rows), hidden, w0.num_q_heads)
+            desc = f"{len(rows)} of {w0.batch} rows of one call"
+        else:
+            probe = min(range(w0.batch), key=lambda b: int(w0.seq_lens[b]))
+            dt = time_oracle(compact_host(w0, [probe])) + per_row
+            rate = max(int(w0.seq_lens[probe]) * KV_BYTES_PER_TOKEN / max(dt, 1e-6), 1e6)
+            picked, units = pick_sample(layers, rate * seconds)
+            elapsed = 0.0
+            for li, seqs in picked:
+                elapsed += time_proj_oracle(layers[li], seqs) + time_oracle(compact_host(layers[li], seqs))
+            desc = f"{sum(len(q) for _, q in picked)} of {sum(w.batch for w in layers)} sequences of the step"
+    finally:
+        oracle.set_threads(1)
+    _, model = host_cpu()
+    return {"value": units / elapsed / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{desc}, {elapsed:.1f} s, {threads} thread{'s' if threads > 1 else ''} "
+                      "(the projection runs on one)", "cpu_model": model, "seconds": elapsed}
+
+
 # ----------------------------------------------------------------------------
 # GPU arm
 
@@ -346,14 +412,31 @@ def run_gpu(args):
     lib = binding.load_library()
     attn = binding.DecodeAttention(device=local, num_q_heads=args.num_q_heads)
     T = args.new_tokens
+    mode = "qkv_proj" if args.op == "qkv_proj" else ("from_hidden" if args.from_hidden else "attention")
+    if mode != "attention" and T != 1:
+        raise SystemExit("--op qkv_proj and --from-hidden take one new token per sequence")
 
     # R resident copies of the step's inputs, so that a call never finds its
     # K/V in L2 from the previous call (each copy's KV is > L2 or R copies are).
     first = make_layers(args.workload, dev, rank, args.num_q_heads, T)
-    step_kv = sum(kv_bytes(w.seq_lens) for w in first)
-    rotate = args.rotate or max(1, min(8, math.ceil(4 * L2_BYTES / max(step_kv, 1))))
+    hidden = inputs.HIDDEN
+    if mode == "attention":
+        step_bytes = sum(kv_bytes(w.seq_lens) for w in first)
+    elif mode == "from_hidden":
+        step_bytes = sum(kv_bytes(w.seq_lens) + proj_bytes(w.batch, hidden, args.num_q_heads) for w in first)
+    else:
+        step_bytes = sum(proj_bytes(w.batch, hidden, args.num_q_heads) for w in first)
+    cap = 8 if mode == "attention" else 64
+    rotate = args.rotate or max(1, min(cap, math.ceil(4 * L2_BYTES / max(step_bytes, 1))))
+    step_kv = step_bytes
     # the copies hold the same bytes in different memory, so every timed launch does the same work
     sets = [first] + [make_layers(args.workload, dev, rank, args.num_q_heads, T) for r in range(1, rotate)]
+    if mode != "attention":
+        for si, layers in enumerate(sets):
+            for li, w in enumerate(layers):
+                # per layer and copy: its hidden state, input_norm gain and qkv_proj weight
+                w.hidden_in = inputs.hidden_inputs(w.batch, seed=7000 + 100 * rank + li, device=dev, hidden=hidden,
+                                                   num_q_heads=args.num_q_heads)
     calls_per_step = len(first)
     stream = torch.cuda.current_stream(dev)
     sp = ctypes.c_void_p(stream.cuda_stream)
@@ -364,18 +447,24 @@ def run_gpu(args):
             t = dict(qkv=w.qkv, q=w.q_norm_w, k=w.k_norm_w, sl=w.seq_lens.to(dev), bt=w.block_table.to(dev),
                      kc=w.k_cache, vc=w.v_cache,
                      o=torch.empty((*w.qkv.shape[:-1], w.num_q_heads, 128), dtype=torch.bfloat16, device=dev))
-            c = (attn.handle, ctypes.c_void_p(t["qkv"].data_ptr()), ctypes.c_void_p(t["q"].data_ptr()),
-                 ctypes.c_void_p(t["k"].data_ptr()),
-                 ctypes.cast(ctypes.c_void_p(t["sl"].data_ptr()), ctypes.POINTER(ctypes.c_int32)), None,
-                 ctypes.cast(ctypes.c_void_p(t["bt"].data_ptr()), ctypes.POINTER(ctypes.c_int32)),
-                 int(w.block_table.shape[1]), ctypes.c_void_p(t["kc"].data_ptr()),
-                 ctypes.c_void_p(t["vc"].data_ptr()), int(w.num_pages), ctypes.c_void_p(t["o"].data_ptr()),
-                 int(w.batch)) + ((T,) if T > 1 else ()) + (sp,)
+            vp = lambda k: ctypes.c_void_p(t[k].data_ptr())
+            i32 = lambda k: ctypes.cast(ctypes.c_void_p(t[k].data_ptr()), ctypes.POINTER(ctypes.c_int32))
+            if mode != "attention":
+                t.update(w.hidden_in)
+                t["qkv"] = torch.empty_like(w.qkv)   # written by the projection
+            proj = (vp("x"), vp("input_norm_w"), vp("w_qkv"), hidden) if mode != "attention" else ()
+            if mode == "qkv_proj":
+                c = (attn.handle, *proj, vp("qkv"), int(w.batch), sp)
+            else:
+                c = ((attn.handle, *proj, vp("qkv"), vp("q"), vp("k"), i32("sl"), None, i32("bt"),
+                      int(w.block_table.shape[1]), vp("kc"), vp("vc"), int(w.num_pages), vp("o"), int(w.batch))
+                     + ((T,) if T > 1 else ()) + (sp,))
             out.append((c, t))
         return out
 
     calls = [prepared(layers) for layers in sets]
-    fn = lib.qwen3_decode_attn_append_and_attend_tokens if T > 1 else lib.qwen3_decode_attn_append_and_attend
+    fn = {"qkv_proj": lib.qwen3_decode_attn_qkv_proj, "from_hidden": lib.qwen3_decode_attn_from_hidden}.get(
+        mode, lib.qwen3_decode_attn_append_and_attend_tokens if T > 1 else lib.qwen3_decode_attn_append_and_attend)
 
     def step(i):
         for c, _ in calls[i % rotate]:
@@ -423,8 +512,15 @@ def run_gpu(args):
     ms = reduce_max(dist, ms_local, dev)
     ms_per_step = ms / args.steps
     # every rotation set has its own lengths (cfg2/cfg5 draw them); average the bytes per step
-    kv_per_step_local = sum(sum(kv_bytes(w.seq_lens) for w in s) for s in (sets[i % rotate] for i in range(args.steps))) / args.steps
-    alg_per_step_local = sum(sum(algorithmic_bytes(w.seq_lens, w.num_q_heads, T) for w in s)
+    def unit_bytes(w):   # what `value` counts: the K/V bytes attended, or the projection's bytes
+        return proj_bytes(w.batch, hidden, w.num_q_heads) if mode == "qkv_proj" else kv_bytes(w.seq_lens)
+
+    def alg_bytes(w):
+        b = 0 if mode == "qkv_proj" else algorithmic_bytes(w.seq_lens, w.num_q_heads, T)
+        return b + (proj_bytes(w.batch, hidden, w.num_q_heads) if mode != "attention" else 0)
+
+    kv_per_step_local = sum(sum(unit_bytes(w) for w in s) for s in (sets[i % rotate] for i in range(args.steps))) / args.steps
+    alg_per_step_local = sum(sum(alg_bytes(w) for w in s)
                              for s in (sets[i % rotate] for i in range(args.steps))) / args.steps
     kv_total = reduce_sum(dist, kv_per_step_local, dev)
     value = kv_total / (ms_per_step * 1e-3) / 1e9
@@ -434,7 +530,8 @@ def run_gpu(args):
     alg_per_launch = alg_per_step_local / calls_per_step
     peak, peak_kind = hbm_peak()
     achieved = alg_per_launch / (mean_kernel_ms * 1e-3) / 1e9
-    traffic = traffic_per_launch(workload_key(args.workload, args.num_q_heads, T), args.num_q_heads, T)
+    traffic = (traffic_per_launch(workload_key(args.workload, args.num_q_heads, T), args.num_q_heads, T)
+               if mode == "attention" else None)
 
     # the other way of timing, for comparison: eager launches with an event pair around each
     if args.timing == "graph":
@@ -451,22 +548,39 @@ def run_gpu(args):
 
     # end to end: per step the H2D copy of the step's inputs from pinned memory,
     # the call, and the D2H copy of o
-    e2e = (run_e2e(args, attn, sets, dev, stream, dist, rotate) if T == 1
-           else run_e2e_tokens(args, attn, sets, dev, stream, dist, rotate))
+    if mode != "attention":
+        e2e = run_e2e_proj(args, attn, sets, dev, stream, dist, rotate, mode, fn, unit_bytes)
+    elif T == 1:
+        e2e = run_e2e(args, attn, sets, dev, stream, dist, rotate)
+    else:
+        e2e = run_e2e_tokens(args, attn, sets, dev, stream, dist, rotate)
 
     result = None
+    proj_tensor = None
+    if mode != "attention":
+        tp, tp_kind = tensor_peak()
+        fl = sum(proj_flops(w.batch, hidden, w.num_q_heads) for w in first) / calls_per_step
+        t_ach = fl / (mean_kernel_ms * 1e-3) / 1e12
+        proj_tensor = {"bound": "tensor", "achieved": round(t_ach, 1), "peak": tp, "unit": "TFLOP/s",
+                       "frac": round(t_ach / tp, 4), "peak_kind": tp_kind,
+                       "flops_per_launch": int(fl), "note": "algorithmic flops (2 per multiply-add); the exact "
+                       "hi/lo split issues twice as many on the tensor pipe"}
     if rank == 0:
         clk = clocks.summary(t0, t1, t_warm)
         result = {
-            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "metric": METRIC if mode != "qkv_proj" else PROJ_METRIC, "value": round(value, 2), "unit": "GB/s",
+            "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
             "us_per_call": round(ms_per_step * 1e3 / calls_per_step, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "io_dtype": "bf16", "data": "synthetic (seeded; N(0,1) bf16 qkv and cache, gains 1+U(-0.5,0.5))",
             "config": {"workload": f"{args.workload}: {WORKLOADS[args.workload]}"
                                    + ("" if args.num_q_heads == 16 else f", {args.num_q_heads} query heads")
-                                   + ("" if T == 1 else f", {T} new tokens per sequence (causal among them)"),
-                       "batch": first[0].batch, "layers_per_step": calls_per_step, "new_tokens": T,
+                                   + ("" if T == 1 else f", {T} new tokens per sequence (causal among them)")
+                                   + {"attention": "", "from_hidden": ", from the hidden state (input_norm + "
+                                      "qkv_proj, then the attention step)", "qkv_proj": ": input_norm + qkv_proj "
+                                      f"only (x [B, {hidden}] -> qkv)"}[mode],
+                       "op": mode, "batch": first[0].batch, "layers_per_step": calls_per_step, "new_tokens": T,
                        "sum_seq_lens_per_step": int(sum(int(w.seq_lens.sum()) for w in first)),
                        "page_size": 16, "heads": f"{args.num_q_heads} q / 8 kv, D=128",
                        "l2": f"{rotate} resident input sets rotated; {rotate * step_kv / 1e9:.2f} GB of KV cycled "
@@ -479,23 +593,29 @@ def run_gpu(args):
                          "kernel_us_mean": round(mean_kernel_ms * 1e3, 3),
                          "kernel_us_median": round(statistics.median(kernel_ms) * 1e3, 3)},
             "e2e": e2e,
+            **({"roofline_tensor": proj_tensor} if proj_tensor is not None else {}),
             "timing": ("CUDA graph replay: one graph per step, K replays between two events; "
                        "per-launch duration = region time / launches") if args.timing == "graph"
                       else "eager launches, an event pair around each; per-launch duration = mean of the pairs",
             ("eager" if args.timing == "graph" else "graph"): other,
             "seq_per_s": round(first[0].batch / (ms_per_step * 1e-3) * world, 1),
-            # one kernel per call on the 16-head decode kernel; attention + combine launches otherwise
-            "gpu_launches": n_launch * (1 if kernel_key(args.num_q_heads, T) == 16 else 2),
+            # one kernel per call on the 16-head decode kernel; attention + combine launches otherwise;
+            # one more per call for the projection
+            "gpu_launches": n_launch * ((0 if mode == "qkv_proj" else (1 if kernel_key(args.num_q_heads, T) == 16 else 2))
+                                        + (0 if mode == "attention" else 1)),
             "clocks": clk,
         }
     if dist is not None:
         dist.barrier(device_ids=[dev.index])
     attn.close()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(first)
         cores, _ = host_cpu()
-        if cores > 1:
-            result["cpu_baseline_all_cores"] = cpu_baseline(first, seconds=8.0, threads=cores)
+        if mode == "attention":
+            result["cpu_baseline"] = cpu_baseline(first)
+            if cores > 1:
+                result["cpu_baseline_all_cores"] = cpu_baseline(first, seconds=8.0, threads=cores)
+        else:
+            result["cpu_baseline"] = cpu_baseline_proj(first, mode)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if dist is not None:
@@ -583,6 +703,70 @@ def run_graph(args, attn, calls, fn, dev, dist, rotate, calls_per_step, kv_per_s
     del g
     return {"us_per_call": round(ms_per_step * 1e3 / calls_per_step, 3), "ms_per_step": round(ms_per_step, 6),
             "value": round(kv_total / (ms_per_step * 1e-3) / 1e9, 2), "unit": "GB/s", "steps": steps}
+
+
+def run_e2e_proj(args, attn, sets, dev, stream, dist, rotate, mode, fn, unit_bytes):
+    """End to end for the projection modes: x copied from pinned host memory into
+    the device buffer, the call, and the result (qkv, or o) copied back."""
+    from decode_attention_qk_b200 import binding
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    host = []
+    for layers in sets:
+        hl = []
+        for w in layers:
+            x_dev = w.hidden_in["x"]
+            out_dev = torch.empty_like(w.qkv) if mode == "qkv_proj" else \
+                torch.empty((w.batch, w.num_q_heads, 128), dtype=torch.bfloat16, device=dev)
+            qkv_dev = out_dev if mode == "qkv_proj" else torch.empty_like(w.qkv)
+            h = dict(x=x_dev.cpu().pin_memory(), out=torch.empty(out_dev.shape, dtype=torch.bfloat16).pin_memory(),
+                     sl=w.seq_lens.clone().pin_memory(), bt=w.block_table.clone().pin_memory())
+            d = dict(x=x_dev, out=out_dev, sl=w.seq_lens.to(dev), bt=w.block_table.to(dev))
+            vp = lambda t: ctypes.c_void_p(t.data_ptr())
+            i32 = lambda t: ctypes.cast(ctypes.c_void_p(t.data_ptr()), ctypes.POINTER(ctypes.c_int32))
+            proj = (vp(d["x"]), vp(w.hidden_in["input_norm_w"]), vp(w.hidden_in["w_qkv"]), inputs.HIDDEN)
+            if mode == "qkv_proj":
+                c = (attn.handle, *proj, vp(qkv_dev), int(w.batch), sp)
+            else:
+                c = (attn.handle, *proj, vp(qkv_dev), vp(w.q_norm_w), vp(w.k_norm_w), i32(d["sl"]), None,
+                     i32(d["bt"]), int(w.block_table.shape[1]), vp(w.k_cache), vp(w.v_cache), int(w.num_pages),
+                     vp(out_dev), int(w.batch), sp)
+            hl.append((c, h, d, qkv_dev))
+        host.append(hl)
+
+    def call(c, h, d):
+        d["x"].copy_(h["x"], non_blocking=True)
+        if mode != "qkv_proj":
+            d["sl"].copy_(h["sl"], non_blocking=True)
+            d["bt"].copy_(h["bt"], non_blocking=True)
+        rc = fn(*c)
+        if rc != 0:
+            raise binding.QdaError(rc, mode)
+        h["out"].copy_(d["out"], non_blocking=True)
+
+    for i in range(args.warmup):
+        for c, h, d, _ in host[i % rotate]:
+            call(c, h, d)
+    barrier(dist, dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    h2d = d2h = 0
+    for i in range(args.steps):
+        for c, h, d, _ in host[i % rotate]:
+            call(c, h, d)
+            h2d += h["x"].nbytes + (0 if mode == "qkv_proj" else h["sl"].nbytes + h["bt"].nbytes)
+            d2h += h["out"].nbytes
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    if attn.check() != 0:
+        raise RuntimeError("device status after the e2e region")
+    ms = reduce_max(dist, start.elapsed_time(end), dev) / args.steps
+    units = sum(sum(unit_bytes(w) for w in sets[i % rotate]) for i in range(args.steps)) / args.steps
+    total = reduce_sum(dist, units, dev)
+    return {"value": round(total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d // args.steps), "d2h_bytes_per_step": int(d2h // args.steps),
+            "ms_per_step": round(ms, 6),
+            "api": f"pinned host->device copy of x + qwen3_decode_attn_{mode} + result device->host"}
 
 
 def run_e2e(args, attn, sets, dev, stream, dist, rotate):
@@ -705,6 +889,9 @@ def run_reference(args):
     import oracle
     oracle.build()
     cores, cpu_model = host_cpu()
+    if args.op == "qkv_proj" or args.from_hidden:
+        run_reference_proj(args, cores, cpu_model)
+        return
     oracle.set_threads(cores)
     layers = make_layers(args.workload, "cpu", 0, args.num_q_heads, args.new_tokens)
     # size each step's sample so that warm-up + timed steps take ~2 minutes
@@ -761,6 +948,32 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_reference_proj(args, cores, cpu_model):
+    """The reference arm of the projection modes: the oracle's input_norm +
+    qkv_proj (and, from the hidden state, the attention too), per step a
+    bounded sample."""
+    mode = "qkv_proj" if args.op == "qkv_proj" else "from_hidden"
+    layers = make_layers(args.workload, "cpu", 0, args.num_q_heads, 1)
+    for li, w in enumerate(layers):
+        w.hidden_in = inputs.hidden_inputs(w.batch, seed=7000 + li, device="cpu", num_q_heads=args.num_q_heads)
+    budget = min(20.0, 120.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline_proj(layers, mode, seconds=budget, threads=cores)
+    runs = [cpu_baseline_proj(layers, mode, seconds=budget, threads=cores) for _ in range(args.steps)]
+    elapsed = sum(r["seconds"] for r in runs)
+    value = sum(r["value"] * r["seconds"] for r in runs) / elapsed
+    print(json.dumps({
+        "impl": "reference", "metric": PROJ_METRIC if mode == "qkv_proj" else METRIC, "value": round(value, 4),
+        "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(elapsed * 1e3 / args.steps, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; same recipe as the GPU arm, drawn on the host)",
+        "config": {"workload": f"{args.workload}: {WORKLOADS[args.workload]}, {mode}", "op": mode},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": runs[0]["sample"], "cpu_model": cpu_model},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -775,6 +988,10 @@ def main(argv=None):
     ap.add_argument("--timing", choices=["graph", "eager"], default="graph",
                     help="timed region: CUDA graph replay of the steps (default) or eager launches with "
                          "an event pair around each; the line also carries the other figure")
+    ap.add_argument("--op", choices=["step", "qkv_proj"], default="step",
+                    help="step: the attention step (default); qkv_proj: input_norm + qkv_proj alone")
+    ap.add_argument("--from-hidden", action="store_true",
+                    help="each call starts from the hidden state: input_norm + qkv_proj, then the attention step")
     ap.add_argument("--rotate", type=int, default=0, help="resident input sets cycled (0: enough to defeat L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -19,6 +19,10 @@ struct qda_handle {
     int* counters = nullptr;
     int* status = nullptr;
     int* seg = nullptr;
+    // input_norm + qkv_proj: the exact split of x*g, and 1/r per row
+    uint16_t* xg_hi = nullptr;
+    uint16_t* xg_lo = nullptr;
+    float* inv_r = nullptr;
     // staging of the host-buffer entry point
     uint16_t* st_qkv = nullptr;
     int32_t* st_seq_lens = nullptr;
@@ -62,6 +66,9 @@ void free_workspace(qda_handle* h) {
     cudaFree(h->counters);
     cudaFree(h->status);
     cudaFree(h->seg);
+    cudaFree(h->xg_hi);
+    cudaFree(h->xg_lo);
+    cudaFree(h->inv_r);
     cudaFree(h->st_qkv);
     cudaFree(h->st_seq_lens);
     cudaFree(h->st_positions);
@@ -131,7 +138,7 @@ int check_proj(const qda_handle* h, const void* x, const void* input_norm_w, con
                const void* qkv, int batch) {
     if (h == nullptr || x == nullptr || input_norm_w == nullptr || w_qkv == nullptr || qkv == nullptr)
         return QDA_ERR_INVALID_ARG;
-    if (batch < 1 || batch > h->cfg.max_batch || hidden < 256 || hidden > qda::kMaxHidden || hidden % 256 != 0)
+    if (batch < 1 || batch > h->cfg.max_batch || hidden < 512 || hidden > qda::kMaxHidden || hidden % 512 != 0)
         return QDA_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(input_norm_w, 16) || !aligned(w_qkv, 16) || !aligned(qkv, 16))
         return QDA_ERR_INVALID_ARG;
@@ -149,6 +156,9 @@ qda::QkvProjParams make_proj_params(const qda_handle* h, const void* x, const vo
     p.hidden = hidden;
     p.qkv_width = (int)qkv_elems(h->cfg.num_q_heads);
     p.eps = h->cfg.rms_eps;
+    p.xg_hi = h->xg_hi;
+    p.xg_lo = h->xg_lo;
+    p.inv_r = h->inv_r;
     p.status = h->status;
     p.timeout_ns = h->cfg.wait_timeout_ns > 0 ? h->cfg.wait_timeout_ns : kDefaultTimeoutNs;
     return p;
@@ -219,7 +229,10 @@ int qwen3_decode_attn_create(const qda_config* cfg, int device, qda_handle** out
               alloc(&h->st_qkv, B * qkv_elems(cfg->num_q_heads) * sizeof(uint16_t)) &&
               alloc(&h->st_seq_lens, B * sizeof(int32_t)) && alloc(&h->st_positions, B * sizeof(int32_t)) &&
               alloc(&h->st_block_table, B * (size_t)cfg->max_pages_per_seq * sizeof(int32_t)) &&
-              alloc(&h->st_o, B * Hq * qda::kHeadDim * sizeof(uint16_t));
+              alloc(&h->st_o, B * Hq * qda::kHeadDim * sizeof(uint16_t)) &&
+              alloc(&h->xg_hi, B * (size_t)qda::kMaxHidden * sizeof(uint16_t)) &&
+              alloc(&h->xg_lo, B * (size_t)qda::kMaxHidden * sizeof(uint16_t)) &&
+              alloc(&h->inv_r, B * sizeof(float));
     ok = ok && cudaMemset(h->counters, 0, (size_t)qda::kMaxBatch * qda::kNumKvHeads * sizeof(int)) == cudaSuccess &&
          cudaMemset(h->status, 0, sizeof(int)) == cudaSuccess && cudaDeviceSynchronize() == cudaSuccess;
     if (!ok) {

@@ -79,9 +79,12 @@ cudaError_t launch(const Params& p, int grid, cudaStream_t stream);
 // launch that combines the partials of sequences split across CTAs.
 cudaError_t launch_grouped(const Params& p, int grid, cudaStream_t stream);
 
-// input_norm + attn.qkv_proj (qda_qkv_proj.cu): hidden size a multiple of 256,
-// at most kMaxHidden (the Qwen3 sizes: 1024, 2048, 2560, 4096, 5120).
+// input_norm + attn.qkv_proj (qda_qkv_proj.cu): hidden size a multiple of 512,
+// at most kMaxHidden (the Qwen3 sizes: 1024, 2048, 2560, 4096, 5120). The
+// product is split over kProjKSplits CTAs along K (a thread-block cluster).
 constexpr int kMaxHidden = 8192;
+constexpr int kProjKSplits = 4;
+constexpr int kProjNTile = 128;     // output columns per CTA
 
 struct QkvProjParams {
     const uint16_t* x;        // bf16 [batch][hidden]
@@ -92,6 +95,11 @@ struct QkvProjParams {
     int hidden;
     int qkv_width;            // (num_q_heads + 16) * 128, a multiple of 32
     double eps;
+    // workspace: the exact split x*g = hi + lo, and 1 / r per row (batches
+    // above 32 rows, formed by a first launch)
+    uint16_t* xg_hi;          // bf16 [batch][hidden]
+    uint16_t* xg_lo;          // bf16 [batch][hidden]
+    float* inv_r;             // [batch]
     int* status;
     int64_t timeout_ns;
 };

@@ -6,23 +6,33 @@
 //
 // Numbers. Nothing is rounded before the bf16 qkv row. Since x and g are bf16,
 // their product has at most 16 significant bits and splits exactly into two
-// bf16 values, x*g = hi + lo; the tensor cores then form hi*W and lo*W exactly
-// and sum them in float. The factor 1/r_b (from float sums of the exact
-// squares x^2, finished in double) is applied to the float sums before the one
-// rounding to bf16. So qkv equals the correctly rounded value except where the
-// float sums land within ~2^-19 of a rounding midpoint.
+// bf16 values, x*g = hi + lo; the tensor cores form hi*W and lo*W exactly and
+// sum them in float. 1/r_b (from float sums of the exact squares x^2, finished
+// in double) scales the float sums just before the one rounding to bf16.
 //
-// Work split. CTA (nb, mb) owns output columns [32 nb, 32 nb + 32) for the
-// batch rows [MT mb, MT mb + MT) and the whole K. A producer warp streams K in
-// chunks of 256 through a 4-stage ring: each chunk brings the 32 weight rows'
-// 512-byte slices and the MT rows' slices of x, one bulk copy per row, into
-// rows 528 bytes apart (so that the 8 rows an ldmatrix phase reads fall in 8
-// different bank groups). Four consumer warps split each chunk's 16 k-steps
-// between them (k-step s goes to warp s % 4); warp w accumulates every row
-// and column of the tile over its k-steps with mma.sync m16n8k16 (bf16 in,
-// float accumulate), and the four partial tiles and squared sums are added
-// through shared memory at the end. For B <= 64 the grid is N / 32 = 128 CTAs
-// whose 4 stages together hold the whole weight in flight.
+// Work split. The product is cut along N into 128-column tiles and along K
+// into 4 quarters: CTA (n-tile, quarter, row block) reads the 128 weight rows'
+// quarter (64 KiB at H = 1024) and its rows' quarter of the split, and writes
+// a float partial tile into its own shared memory. The four quarters of a tile
+// form a thread-block cluster: after a cluster barrier, quarter q adds the
+// four partials of columns [32q, 32q + 32) in quarter order, reading its peers'
+// shared memory directly (so the result does not depend on timing and no
+// partial goes through L2), scales by 1/r_b and writes bf16 qkv. With 4 warps
+// of 32 columns each, a CTA needs no reduction of its own.
+//
+// Operands reach shared memory by 16-byte asynchronous copies (cp.async)
+// through a 3-stage ring of 128-wide K chunks, in rows 272 bytes apart so that
+// the 8 rows an ldmatrix phase reads fall in 8 different bank groups. (One
+// bulk copy per short row slice was tried first: at about one copy every
+// 45 ns per SM the copy count, not the bytes, set the time.)
+//
+// The split of x*g. For up to 32 rows each CTA forms it for its own quarter of
+// K from raw x staged next to the weight (4x less repeated work than forming
+// it for all of K, and no second launch). For more rows a first launch forms
+// it once per row (with 1/r_b) into workspace and the product launch starts
+// with programmatic dependent launch: it issues the weight copies of its first
+// stages before it waits for the first launch.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cstdint>
 
@@ -33,194 +43,206 @@
 namespace qda {
 namespace {
 
-constexpr int kNT = 32;                        // output columns per CTA
-constexpr int kKC = 256;                       // K per chunk
-constexpr int kStagesP = 4;
-constexpr int kPitch = kKC * 2 + 16;           // 528-byte staged row pitch
-constexpr int kConsumers = 4;
-constexpr int kThreadsP = (kConsumers + 1) * 32;
+constexpr int kNT = kProjNTile;                // output columns per CTA
+constexpr int kKS = kProjKSplits;              // K quarters
+constexpr int kKC = 128;                       // K per chunk
+constexpr int kPitch = kKC * 2 + 16;           // 272-byte staged row pitch
+constexpr int kPieces = kKC / 8;               // 16-byte pieces per row slice
+constexpr int kStages = 3;
+constexpr int kWarps = 4;
+constexpr int kThreadsP = kWarps * 32;
+constexpr int kPrepThreads = 128;
 
-template <int MT>
+// kConvert: the CTA forms the split itself from raw x (up to 32 rows); else it
+// copies the split formed by the first launch.
+template <int MT, bool kConvert>
 struct PLayout {
-    static constexpr int kRowsPerStage = kNT + MT;                 // weight rows, then x rows
-    static constexpr int kStageBytes = kRowsPerStage * kPitch;
-    static constexpr int kSmemGain = kStagesP * kStageBytes;       // bf16 [kMaxHidden]
-    static constexpr int kSmemBars = kSmemGain + kMaxHidden * 2;   // full[4], empty[4], gain
-    static constexpr int kSmemFlags = kSmemBars + (2 * kStagesP + 1) * 8;
-    static constexpr int kSmemTotal = kSmemFlags + 16;
-    // the end-of-loop reduction reuses the ring: 4 partial tiles and row sums
-    static constexpr int kRedBytes = kConsumers * MT * kNT * 4 + kConsumers * MT * 4 + MT * 4;
-    static_assert(kRedBytes <= kStagesP * kStageBytes, "reduction fits in the ring");
-    static_assert(kStageBytes % 16 == 0 && kSmemBars % 8 == 0, "alignment");
+    static constexpr int kARows = kConvert ? MT : 2 * MT;            // raw x, or hi and lo
+    static constexpr int kStageBytes = (kNT + kARows) * kPitch;
+    static constexpr int kSmemHiLo = kStages * kStageBytes;          // convert: hi, lo of the current chunk
+    static constexpr int kSmemGain = kSmemHiLo + (kConvert ? 2 * MT * kPitch : 0);   // bf16 [hidden / 4]
+    static constexpr int kSmemInvR = kSmemGain + (kConvert ? kMaxHidden / kKS * 2 : 0);  // float [MT]
+    static constexpr int kSmemTotal = kSmemInvR + MT * 4;
+    // after the K loop the ring holds this quarter's partial tile and sums of x^2
+    static_assert((MT * kNT + MT) * 4 <= kStages * kStageBytes, "partial tile fits in the ring");
     static_assert(kSmemTotal <= 227 * 1024, "fits one CTA per SM");
+    static_assert(kStageBytes % 16 == 0 && kPitch % 128 == 16, "alignment, conflict-free rows");
 };
 
-struct PShared {
-    uint8_t* stages;
-    const uint16_t* gain;
-    uint64_t* full_bar;
-    uint64_t* empty_bar;
-    uint64_t* gain_bar;
-    volatile int* abort_flag;
-};
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// Producer warp: the gain once, then K / 256 chunks of the tile's weight and x rows.
-template <int MT>
-__device__ __forceinline__ void proj_producer(const QkvProjParams& p, const PShared& s, int n0, int m0, int rows,
-                                              int lane) {
-    using Lay = PLayout<MT>;
-    const int chunks = p.hidden / kKC;
-    if (lane == 0) {
-        mbar_arrive_expect_tx(s.gain_bar, (uint32_t)p.hidden * 2u);
-        bulk_g2s(const_cast<uint16_t*>(s.gain), p.norm_w, (uint32_t)p.hidden * 2u, s.gain_bar);
-    }
-    uint32_t armed = 0, armed_parity = 0;
-    bool aborted = false;
-    for (int c = 0; c < chunks; ++c) {
-        const int slot = c % kStagesP;
-        const uint32_t phase = (uint32_t)(c / kStagesP) & 1u;
-        int ok = 1;
-        if (lane == 0) {
-            ok = mbar_try_wait(&s.empty_bar[slot], phase ^ 1u) ||
-                 mbar_wait(&s.empty_bar[slot], phase ^ 1u, p.timeout_ns, s.abort_flag);
-            if (ok) {
-                mbar_arrive_expect_tx(&s.full_bar[slot], (uint32_t)(kNT + rows) * (kKC * 2));
-                armed |= 1u << slot;
-                armed_parity = (armed_parity & ~(1u << slot)) | (phase << slot);
-            } else {
-                *s.abort_flag = 1;
-                record_error(p.status, QDA_ERR_TIMEOUT);
-            }
-        }
-        ok = __shfl_sync(kFull, ok, 0);
-        if (!ok) {
-            aborted = true;
-            break;
-        }
-        uint8_t* stage = s.stages + slot * Lay::kStageBytes;
-        const size_t koff = (size_t)c * kKC;
-        // lane l: weight row n0 + l, and x rows l and l + 32 of the tile
-        bulk_g2s(stage + lane * kPitch, p.w + (size_t)(n0 + lane) * p.hidden + koff, kKC * 2, &s.full_bar[slot]);
+__device__ __forceinline__ float warp_sum_f(float v) {
 #pragma unroll
-        for (int r = lane; r < MT; r += 32)
-            if (r < rows)
-                bulk_g2s(stage + (kNT + r) * kPitch, p.x + (size_t)(m0 + r) * p.hidden + koff, kKC * 2,
-                         &s.full_bar[slot]);
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+    return v;
+}
+
+// The exact split of the products x*g of one 16-byte piece (8 values): hi, lo
+// words, and the squares of x added to ss.
+__device__ __forceinline__ void split_piece(const uint4& xv, const uint32_t* gw, uint4& hv, uint4& lv, float& ss) {
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float x0 = bf_lo(xw[e]), x1 = bf_hi(xw[e]);
+        ss = fmaf(x0, x0, fmaf(x1, x1, ss));     // squares of bf16 values: exact in float
+        uint16_t h0, l0, h1, l1;
+        split_bf16(x0 * bf_lo(gw[e]), h0, l0);   // the product has <= 16 significant bits: exact
+        split_bf16(x1 * bf_hi(gw[e]), h1, l1);
+        hw[e] = (uint32_t)h1 << 16 | h0;
+        lw[e] = (uint32_t)l1 << 16 | l0;
     }
-    if (lane == 0 && (aborted || *s.abort_flag != 0)) {
-        for (int k = 0; k < kStagesP; ++k)
-            if (armed & (1u << k)) (void)mbar_wait(&s.full_bar[k], (armed_parity >> k) & 1u, p.timeout_ns, nullptr);
-        (void)mbar_wait(s.gain_bar, 0u, p.timeout_ns, nullptr);
+    hv = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    lv = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+}
+
+// ---------------------------------------------------------------------------
+// First launch (more than 32 rows): per row b, the split of x[b, k] * g[k] and 1 / r_b.
+
+__global__ void __launch_bounds__(kPrepThreads) input_norm_split_kernel(const QkvProjParams p) {
+    pdl_launch_dependents();   // the product may start streaming the weight now
+    const int b = blockIdx.x;
+    const uint4* xr = reinterpret_cast<const uint4*>(p.x + (size_t)b * p.hidden);
+    const uint4* gr = reinterpret_cast<const uint4*>(p.norm_w);
+    uint4* hr = reinterpret_cast<uint4*>(p.xg_hi + (size_t)b * p.hidden);
+    uint4* lr = reinterpret_cast<uint4*>(p.xg_lo + (size_t)b * p.hidden);
+    float ss = 0.f;
+    for (int v = threadIdx.x; v < p.hidden / 8; v += kPrepThreads) {
+        const uint4 gv = __ldg(gr + v);
+        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+        uint4 hv, lv;
+        split_piece(__ldg(xr + v), gw, hv, lv, ss);
+        hr[v] = hv;
+        lr[v] = lv;
+    }
+    __shared__ float part[kPrepThreads / 32];
+    ss = warp_sum_f(ss);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double sum = 0.0;
+        for (int w = 0; w < kPrepThreads / 32; ++w) sum += (double)part[w];
+        p.inv_r[b] = (float)(1.0 / sqrt(sum / (double)p.hidden + p.eps));
     }
 }
 
-// Split the exact product a*b of two bf16 values (at most 16 significant bits)
-// into hi + lo, both bf16, with nothing lost.
-__device__ __forceinline__ void split_product(float a, float b, uint16_t& hi, uint16_t& lo) {
-    const float prod = a * b;   // exact in float: 8-bit by 8-bit significands
-    const __nv_bfloat16 h = __float2bfloat16_rn(prod);
-    hi = __bfloat16_as_ushort(h);
-    lo = __bfloat16_as_ushort(__float2bfloat16_rn(prod - __bfloat162float(h)));   // exact remainder
-}
+// ---------------------------------------------------------------------------
+// The product, split along K.
 
-__device__ __forceinline__ bool proj_wait(const QkvProjParams& p, const PShared& s, uint64_t* bar, uint32_t phase,
-                                          int lane) {
-    bool ok = mbar_try_wait(bar, phase);
-    if (__all_sync(kFull, ok)) return true;
-    ok = ok || mbar_wait(bar, phase, p.timeout_ns, s.abort_flag);
-    ok = __all_sync(kFull, ok || mbar_try_wait(bar, phase));
-    if (!ok && lane == 0) {
-        *s.abort_flag = 1;
-        record_error(p.status, QDA_ERR_TIMEOUT);
-    }
-    return ok;
-}
-
-template <int MT>
+template <int MT, bool kConvert>
 __global__ void __launch_bounds__(kThreadsP, 1) qkv_proj_kernel(const QkvProjParams p) {
-    using Lay = PLayout<MT>;
+    using Lay = PLayout<MT, kConvert>;
     constexpr int kMTiles = MT / 16;
     extern __shared__ __align__(128) uint8_t smem[];
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    PShared s;
-    s.stages = smem;
-    s.gain = reinterpret_cast<const uint16_t*>(smem + Lay::kSmemGain);
-    s.full_bar = reinterpret_cast<uint64_t*>(smem + Lay::kSmemBars);
-    s.empty_bar = s.full_bar + kStagesP;
-    s.gain_bar = s.empty_bar + kStagesP;
-    s.abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kSmemFlags);
-
-    const int n0 = (int)blockIdx.x * kNT;
-    const int m0 = (int)blockIdx.y * MT;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int nt = (int)blockIdx.x, ks = (int)blockIdx.y, mb = (int)blockIdx.z;
+    const int n0 = nt * kNT;
+    const int m0 = mb * MT;
     const int rows = min(MT, p.batch - m0);
-    if (threadIdx.x == 0) {
-        for (int k = 0; k < kStagesP; ++k) {
-            mbar_init(&s.full_bar[k], 1);
-            mbar_init(&s.empty_bar[k], kConsumers);
+    const int kq = p.hidden / kKS;           // this CTA's K range: [ks*kq, ks*kq + kq)
+    const int kbase = ks * kq;
+    const int chunks = kq / kKC;
+    const uint32_t ring = smem_addr(smem);
+
+    auto weight_rows = [&](int c) {   // 128 rows x 128: needs nothing from a first launch
+        const uint32_t stage = ring + (c % kStages) * Lay::kStageBytes;
+        for (int i = tid; i < kNT * kPieces; i += kThreadsP) {
+            const int r = i / kPieces, q = i % kPieces;
+            cp_async16(stage + r * kPitch + q * 16,
+                       p.w + (size_t)(n0 + r) * p.hidden + (size_t)(kbase + c * kKC) + q * 8);
         }
-        mbar_init(s.gain_bar, 1);
-        *s.abort_flag = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncthreads();
-    if (warp == kConsumers) {
-        proj_producer<MT>(p, s, n0, m0, rows, lane);
-        return;
+    };
+    auto a_rows = [&](int c) {        // raw x rows, or hi and lo rows
+        const uint32_t stage = ring + (c % kStages) * Lay::kStageBytes + kNT * kPitch;
+        for (int i = tid; i < rows * kPieces; i += kThreadsP) {
+            const int r = i / kPieces, q = i % kPieces;
+            const size_t src = (size_t)(m0 + r) * p.hidden + (size_t)(kbase + c * kKC) + q * 8;
+            if (kConvert) {
+                cp_async16(stage + r * kPitch + q * 16, p.x + src);
+            } else {
+                cp_async16(stage + r * kPitch + q * 16, p.xg_hi + src);
+                cp_async16(stage + (MT + r) * kPitch + q * 16, p.xg_lo + src);
+            }
+        }
+    };
+    // Groups, oldest first: {gain quarter and weight of chunks 0..S-2}, {A of
+    // chunk 0}, ..., {A of chunk S-2}, then one group per later chunk.
+    const int pre = min(kStages - 1, chunks);
+    if (kConvert)
+        for (int i = tid; i < kq / 8; i += kThreadsP) cp_async16(ring + Lay::kSmemGain + i * 16, p.norm_w + kbase + i * 8);
+    for (int c = 0; c < pre; ++c) weight_rows(c);
+    cp_async_commit();
+    if (!kConvert) pdl_wait();   // hi, lo and 1/r are complete and visible from here on
+    for (int c = 0; c < kStages - 1; ++c) {
+        if (c < pre) a_rows(c);
+        cp_async_commit();
     }
 
-    // Consumer warp `warp`: k-steps warp, warp + 4, ... of every chunk.
     const int g = lane >> 2, t = lane & 3;
-    float acc[kMTiles][4][4];
-    float ss[kMTiles][2];   // this lane's squares of rows g and g + 8 of each m-tile
+    // kConvert: thread tid splits pieces tid + 128 m (row (tid + 128 m) / 16,
+    // piece tid % 16); the 16 threads of a half-warp share a row
+    constexpr int kConvPerThread = kConvert ? MT * kPieces / kThreadsP : 1;
+    float ss[kConvPerThread];
 #pragma unroll
-    for (int i = 0; i < kMTiles; ++i) {
-        ss[i][0] = ss[i][1] = 0.f;
+    for (int m = 0; m < kConvPerThread; ++m) ss[m] = 0.f;
+    float acc[kMTiles][4][4];
+#pragma unroll
+    for (int i = 0; i < kMTiles; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
-    }
-    bool ok = proj_wait(p, s, s.gain_bar, 0u, lane);
-    const uint32_t* gain_w = reinterpret_cast<const uint32_t*>(s.gain);
-    const int chunks = p.hidden / kKC;
-    for (int c = 0; c < chunks && ok; ++c) {
-        const int slot = c % kStagesP;
-        if (!proj_wait(p, s, &s.full_bar[slot], (uint32_t)(c / kStagesP) & 1u, lane)) {
-            ok = false;
-            break;
+    for (int c = 0; c < chunks; ++c) {
+        if (c + kStages - 1 < chunks) {
+            weight_rows(c + kStages - 1);
+            a_rows(c + kStages - 1);
         }
-        const uint8_t* stage = s.stages + slot * Lay::kStageBytes;
-        // ldmatrix row addresses: weight rows as the column-major B operand,
-        // x rows as the row-major A operand
-        const uint32_t wbase = smem_addr(stage) + ((lane & 7) + ((lane >> 4) << 3)) * kPitch + ((lane >> 3) & 1) * 16;
-        const uint32_t xbase =
-            smem_addr(stage) + (kNT + (lane & 7) + ((lane >> 3) & 1) * 8) * kPitch + ((lane >> 4) & 1) * 16;
+        cp_async_commit();
+        cp_async_wait<kStages - 1>();   // this thread's copies of chunk c have landed ...
+        __syncthreads();                // ... and everyone's
+        const uint32_t stage = ring + (c % kStages) * Lay::kStageBytes;
+        uint32_t abase_hi, abase_lo;
+        if (kConvert) {
+            const uint8_t* raw = smem + (c % kStages) * Lay::kStageBytes + kNT * kPitch;
+            const uint32_t* gw = reinterpret_cast<const uint32_t*>(smem + Lay::kSmemGain) + (c * kKC) / 2;
 #pragma unroll
-        for (int q = 0; q < kKC / 16 / kConsumers; ++q) {
-            const int k0 = (q * kConsumers + warp) * 16;   // within the chunk
+            for (int m = 0; m < kConvPerThread; ++m) {
+                const int i = tid + kThreadsP * m;
+                const int r = i / kPieces, q = i % kPieces;
+                uint4 hv, lv;
+                split_piece(*reinterpret_cast<const uint4*>(raw + r * kPitch + q * 16), gw + 4 * q, hv, lv, ss[m]);
+                *reinterpret_cast<uint4*>(smem + Lay::kSmemHiLo + r * kPitch + q * 16) = hv;
+                *reinterpret_cast<uint4*>(smem + Lay::kSmemHiLo + (MT + r) * kPitch + q * 16) = lv;
+            }
+            __syncthreads();
+            abase_hi = ring + Lay::kSmemHiLo;
+        } else {
+            abase_hi = stage + kNT * kPitch;
+        }
+        abase_lo = abase_hi + MT * kPitch;
+        // ldmatrix row addresses: this warp's 32 weight rows as the column-major
+        // B operand, hi and lo rows as the row-major A operand
+        const uint32_t wbase =
+            stage + (32 * warp + (lane & 7) + ((lane >> 4) << 3)) * kPitch + ((lane >> 3) & 1) * 16;
+        const uint32_t aoff = ((lane & 7) + ((lane >> 3) & 1) * 8) * kPitch + ((lane >> 4) & 1) * 16;
+#pragma unroll
+        for (int kstep = 0; kstep < kKC / 16; ++kstep) {
+            const int k0 = kstep * 16;
             uint32_t b[4][2];
             ldsm_x4(wbase + k0 * 2, b[0][0], b[0][1], b[1][0], b[1][1]);
             ldsm_x4(wbase + 16 * kPitch + k0 * 2, b[2][0], b[2][1], b[3][0], b[3][1]);
-            // gains of this lane's k columns: 2t, 2t+1 and 2t+8, 2t+9
-            const int kg = c * kKC + k0;
-            const uint32_t g01 = gain_w[(kg >> 1) + t], g89 = gain_w[(kg >> 1) + 4 + t];
 #pragma unroll
             for (int i = 0; i < kMTiles; ++i) {
-                uint32_t a[4];
-                ldsm_x4(xbase + i * 16 * kPitch + k0 * 2, a[0], a[1], a[2], a[3]);
                 uint32_t ahi[4], alo[4];
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const uint32_t gw = (r & 2) ? g89 : g01;
-                    const float x0 = bf_lo(a[r]), x1 = bf_hi(a[r]);
-                    ss[i][r & 1] = fmaf(x0, x0, fmaf(x1, x1, ss[i][r & 1]));
-                    uint16_t h0, l0, h1, l1;
-                    split_product(x0, bf_lo(gw), h0, l0);
-                    split_product(x1, bf_hi(gw), h1, l1);
-                    ahi[r] = (uint32_t)h1 << 16 | h0;
-                    alo[r] = (uint32_t)l1 << 16 | l0;
-                }
+                ldsm_x4(abase_hi + aoff + i * 16 * kPitch + k0 * 2, ahi[0], ahi[1], ahi[2], ahi[3]);
+                ldsm_x4(abase_lo + aoff + i * 16 * kPitch + k0 * 2, alo[0], alo[1], alo[2], alo[3]);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     mma_bf16_16816(acc[i][j], ahi, b[j][0], b[j][1]);
@@ -228,87 +250,115 @@ __global__ void __launch_bounds__(kThreadsP, 1) qkv_proj_kernel(const QkvProjPar
                 }
             }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.empty_bar[slot]);
+        __syncthreads();                // the stage (and the hi/lo buffer) may be refilled
     }
+    cp_async_wait<0>();
 
-    // All four consumer warps meet here whatever happened (no early return),
-    // so the named barrier always completes.
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");
-    if (*s.abort_flag != 0) return;
-    // Partial tiles and squared sums to shared memory (the ring is drained).
-    float* red = reinterpret_cast<float*>(s.stages);                    // [4][MT][32]
-    float* red_ss = red + kConsumers * MT * kNT;                        // [4][MT]
-    float* inv_r = red_ss + kConsumers * MT;                            // [MT]
+    // This quarter's partial tile (float) and, when converting, its sums of x^2,
+    // in shared memory for the cluster.
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    float* tile = reinterpret_cast<float*>(smem);   // [MT][kNT], the ring is drained
+    float* tss = tile + MT * kNT;                   // [MT]
 #pragma unroll
     for (int i = 0; i < kMTiles; ++i) {
-        float s0 = ss[i][0], s1 = ss[i][1];
-        s0 += __shfl_xor_sync(kFull, s0, 1);
-        s0 += __shfl_xor_sync(kFull, s0, 2);
-        s1 += __shfl_xor_sync(kFull, s1, 1);
-        s1 += __shfl_xor_sync(kFull, s1, 2);
-        if (t == 0) {
-            red_ss[warp * MT + 16 * i + g] = s0;
-            red_ss[warp * MT + 16 * i + g + 8] = s1;
-        }
+        const int r0 = 16 * i + g;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            float* r0 = red + ((size_t)warp * MT + 16 * i + g) * kNT + 8 * j + 2 * t;
-            float* r1 = r0 + 8 * kNT;
-            *reinterpret_cast<float2*>(r0) = make_float2(acc[i][j][0], acc[i][j][1]);
-            *reinterpret_cast<float2*>(r1) = make_float2(acc[i][j][2], acc[i][j][3]);
+            const int col = 32 * warp + 8 * j + 2 * t;
+            *reinterpret_cast<float2*>(tile + r0 * kNT + col) = make_float2(acc[i][j][0], acc[i][j][1]);
+            *reinterpret_cast<float2*>(tile + (r0 + 8) * kNT + col) = make_float2(acc[i][j][2], acc[i][j][3]);
         }
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");
-    const int tid = threadIdx.x;
-    for (int r = tid; r < MT; r += kConsumers * 32) {
-        const double sum = (double)red_ss[r] + (double)red_ss[MT + r] + (double)red_ss[2 * MT + r] +
-                           (double)red_ss[3 * MT + r];
-        inv_r[r] = (float)(1.0 / sqrt(sum / (double)p.hidden + p.eps));
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");
-    // two adjacent columns per thread: one 4-byte store each
-    for (int e = tid; e < MT * kNT / 2; e += kConsumers * 32) {
-        const int r = e / (kNT / 2), col = 2 * (e % (kNT / 2));
-        if (r >= rows) continue;
-        float v0 = 0.f, v1 = 0.f;
+    if (kConvert) {
 #pragma unroll
-        for (int w = 0; w < kConsumers; ++w) {
-            const float2 v = *reinterpret_cast<const float2*>(red + ((size_t)w * MT + r) * kNT + col);
-            v0 += v.x;
-            v1 += v.y;
+        for (int m = 0; m < kConvPerThread; ++m) {
+            float v = ss[m];
+            v += __shfl_xor_sync(kFull, v, 1);
+            v += __shfl_xor_sync(kFull, v, 2);
+            v += __shfl_xor_sync(kFull, v, 4);
+            v += __shfl_xor_sync(kFull, v, 8);
+            if ((lane & 15) == 0) tss[(tid + kThreadsP * m) / kPieces] = v;
+        }
+    }
+    cluster.sync();   // all four quarters' partials are in place
+    const int q = (int)cluster.block_rank();   // = ks
+    const float* peer[kKS];
+    const float* peer_ss[kKS];
+#pragma unroll
+    for (int r = 0; r < kKS; ++r) {
+        peer[r] = cluster.map_shared_rank(tile, r);
+        peer_ss[r] = cluster.map_shared_rank(tss, r);
+    }
+    float* inv_r = reinterpret_cast<float*>(smem + Lay::kSmemInvR);
+    for (int r = tid; r < rows; r += kThreadsP) {
+        if (kConvert) {
+            double sum = 0.0;
+#pragma unroll
+            for (int k = 0; k < kKS; ++k) sum += (double)peer_ss[k][r];
+            inv_r[r] = (float)(1.0 / sqrt(sum / (double)p.hidden + p.eps));
+        } else {
+            inv_r[r] = __ldg(p.inv_r + m0 + r);
+        }
+    }
+    __syncthreads();
+    // columns [32q, 32q + 32) of the tile: 16 column pairs per row
+    for (int e = tid; e < rows * 16; e += kThreadsP) {
+        const int r = e / 16, col = 32 * q + 2 * (e % 16);
+        float2 sum = *reinterpret_cast<const float2*>(peer[0] + r * kNT + col);
+#pragma unroll
+        for (int k = 1; k < kKS; ++k) {
+            const float2 v = *reinterpret_cast<const float2*>(peer[k] + r * kNT + col);
+            sum.x += v.x;
+            sum.y += v.y;
         }
         const float f = inv_r[r];
-        *reinterpret_cast<uint32_t*>(p.y + (size_t)(m0 + r) * p.qkv_width + n0 + col) = pack_bf2(v0 * f, v1 * f);
+        *reinterpret_cast<uint32_t*>(p.y + (size_t)(m0 + r) * p.qkv_width + n0 + col) = pack_bf2(sum.x * f, sum.y * f);
     }
+    cluster.sync();   // peers may still be reading this CTA's partial
 }
 
-template <int MT>
+template <int MT, bool kConvert>
 cudaError_t prepare_proj_one() {
-    return cudaFuncSetAttribute(qkv_proj_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                PLayout<MT>::kSmemTotal);
+    return cudaFuncSetAttribute(qkv_proj_kernel<MT, kConvert>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                PLayout<MT, kConvert>::kSmemTotal);
 }
 
-template <int MT>
+template <int MT, bool kConvert>
 cudaError_t launch_proj_one(const QkvProjParams& p, cudaStream_t stream) {
-    const dim3 grid((unsigned)(p.qkv_width / kNT), (unsigned)((p.batch + MT - 1) / MT), 1);
-    qkv_proj_kernel<MT><<<grid, kThreadsP, PLayout<MT>::kSmemTotal, stream>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.qkv_width / kNT), (unsigned)kKS, (unsigned)((p.batch + MT - 1) / MT));
+    cfg.blockDim = dim3(kThreadsP, 1, 1);
+    cfg.dynamicSmemBytes = PLayout<MT, kConvert>::kSmemTotal;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;   // the 4 K quarters of a tile
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = kKS;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = kConvert ? 1 : 2;   // dependent launch only after the split's own launch
+    return cudaLaunchKernelEx(&cfg, qkv_proj_kernel<MT, kConvert>, p);
 }
 
 }  // namespace
 
 cudaError_t prepare_qkv_proj() {
-    cudaError_t e = prepare_proj_one<16>();
-    if (e == cudaSuccess) e = prepare_proj_one<32>();
-    if (e == cudaSuccess) e = prepare_proj_one<64>();
+    cudaError_t e = prepare_proj_one<16, true>();
+    if (e == cudaSuccess) e = prepare_proj_one<32, true>();
+    if (e == cudaSuccess) e = prepare_proj_one<64, false>();
     return e;
 }
 
 cudaError_t launch_qkv_proj(const QkvProjParams& p, cudaStream_t stream) {
-    if (p.batch <= 16) return launch_proj_one<16>(p, stream);
-    if (p.batch <= 32) return launch_proj_one<32>(p, stream);
-    return launch_proj_one<64>(p, stream);
+    if (p.batch <= 16) return launch_proj_one<16, true>(p, stream);
+    if (p.batch <= 32) return launch_proj_one<32, true>(p, stream);
+    input_norm_split_kernel<<<p.batch, kPrepThreads, 0, stream>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_proj_one<64, false>(p, stream);
 }
 
 }  // namespace qda

@@ -217,7 +217,7 @@ int qwen3_decode_attn_append_and_attend_tokens(qda_handle *h,
  * stride hidden); input_norm_w bf16 [hidden]; w_qkv bf16 [N][hidden] with
  * N = (num_q_heads + 16) * 128 of the handle (row n = output feature n, the
  * layout of a torch Linear weight; q rows, then k rows, then v rows); qkv
- * bf16 [B][N] (output). hidden is a multiple of 256 in [256, 8192]
+ * bf16 [B][N] (output). hidden is a multiple of 512 in [512, 8192]
  * (Qwen3: 1024 for 0.6B, 2048, 2560, 4096, 5120 for the larger sizes).
  * Nothing is rounded before qkv, which is rounded once to bf16: the products
  * x*g are split exactly into two bf16 terms for the tensor cores and summed
@@ -225,8 +225,8 @@ int qwen3_decode_attn_append_and_attend_tokens(qda_handle *h,
  * lies within about 2^-19 (relative) of a rounding midpoint, where it may be
  * the neighbouring bf16 value.
  * Errors: INVALID_ARG (null or misaligned pointer, batch outside
- * [1, max_batch], hidden not a multiple of 256 in range), CUDA (the launch
- * failed); a wait that ran out on the device goes to the status word. */
+ * [1, max_batch], hidden not a multiple of 512 in range), CUDA (the launch
+ * failed). */
 int qwen3_decode_attn_qkv_proj(qda_handle *h,
                                const void *x,
                                const void *input_norm_w,

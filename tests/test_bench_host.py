@@ -26,6 +26,13 @@ def test_byte_counts():
     assert bench.algorithmic_bytes(L, 32, 3) == want
 
 
+def test_projection_byte_and_flop_counts():
+    # Qwen3-0.6B: weight 4096 x 1024, x and qkv rows, the gain
+    assert bench.proj_bytes(32) == 4096 * 1024 * 2 + 32 * 1024 * 2 + 1024 * 2 + 32 * 4096 * 2
+    assert bench.proj_bytes(1, hidden=5120, num_q_heads=64) == 10240 * 5120 * 2 + 5120 * 2 + 5120 * 2 + 10240 * 2
+    assert bench.proj_flops(256) == 2 * 256 * 4096 * 1024
+
+
 def test_kernel_and_workload_keys():
     assert bench.kernel_key(16, 1) == 16
     assert bench.kernel_key(16, 2) == bench.kernel_key(64, 1) == "grouped"
