@@ -128,8 +128,9 @@ qda::Params make_params(const qda_handle* h, const void* qkv, const void* q_norm
     return p;
 }
 
-cudaError_t launch_step(const qda_handle* h, const qda::Params& p, cudaStream_t stream) {
-    return p.num_q_heads == qda::kNumQHeads && p.new_tokens == 1 ? qda::launch(p, h->grid, stream)
+cudaError_t launch_step(const qda_handle* h, const qda::Params& p, cudaStream_t stream,
+                        bool after_producer = false) {
+    return p.num_q_heads == qda::kNumQHeads && p.new_tokens == 1 ? qda::launch(p, h->grid, stream, after_producer)
                                                                  : qda::launch_grouped(p, h->grid, stream);
 }
 
@@ -304,7 +305,8 @@ int qwen3_decode_attn_from_hidden(qda_handle* h, const void* x, const void* inpu
     if (qda::launch_qkv_proj(pp, st) != cudaSuccess) return QDA_ERR_CUDA;
     const qda::Params p = make_params(h, qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table,
                                       block_table_stride, k_cache, v_cache, num_pages, o, batch);
-    return launch_step(h, p, st) == cudaSuccess ? QDA_OK : QDA_ERR_CUDA;
+    // the attention starts while the projection finishes; it reads qkv only after
+    return launch_step(h, p, st, /*after_producer=*/true) == cudaSuccess ? QDA_OK : QDA_ERR_CUDA;
 }
 
 int qwen3_decode_attn_append_and_attend_host(qda_handle* h, const void* qkv_host, const void* q_norm_w,

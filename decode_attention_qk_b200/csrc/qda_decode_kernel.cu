@@ -149,6 +149,23 @@ __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, i
     uint32_t phase = 0;
     uint32_t armed = 0, armed_parity = 0;   // lane 0: slots with a phase armed, and its parity
     bool aborted = false;
+    // When this launch depends on the one producing qkv (programmatic
+    // dependent launch), the first round of stages gets its K/V copies at
+    // once and its qkv copies only after griddepcontrol.wait.
+    bool qkv_ready = p.qkv_after_wait == 0;
+    int deferred_seq[kStages];
+    uint32_t deferred = 0;   // slots of the first round whose qkv copy waits
+    int issued = 0;
+    auto release_qkv = [&]() {
+        pdl_wait();
+        asm volatile("fence.proxy.async.global;" ::: "memory");   // the bulk copies read what it wrote
+        for (int k = 0; k < kStages; ++k)
+            if (deferred & (1u << k))
+                bulk_g2s(s.stages + k * kStageBytes + kStageQkv, p.qkv + (size_t)deferred_seq[k] * kQkvWidth,
+                         (uint32_t)kQkvBytes, &s.full_bar[k]);
+        deferred = 0;
+        qkv_ready = true;
+    };
     for (int base = 0; base < count && !aborted; base += 32) {
         // 32 pages' descriptions fetched at once, one per lane.
         const int gp = start + base + lane;
@@ -174,6 +191,7 @@ __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, i
             const int seq_pos = __shfl_sync(kFull, pos, kk);
             int ok = 1;
             if (lane == 0) {
+                if (!qkv_ready && issued == kStages) release_qkv();   // before the ring's second round
                 ok = mbar_try_wait(&s.empty_bar[slot], phase ^ 1u) ||
                      mbar_wait(&s.empty_bar[slot], phase ^ 1u, p.timeout_ns, s.abort_flag);
                 if (ok) {
@@ -188,13 +206,20 @@ __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, i
                         uint8_t* dst = s.stages + slot * kStageBytes;
                         const size_t off = (size_t)page_id * kPageBytes;
                         mbar_arrive_expect_tx(&s.full_bar[slot], 2u * kv_bytes + qkv_bytes);
-                        if (qkv_bytes != 0)
-                            bulk_g2s(dst + kStageQkv, p.qkv + (size_t)seq_qkv * kQkvWidth, qkv_bytes, &s.full_bar[slot]);
                         if (kv_bytes != 0) {
                             bulk_g2s(dst + kStageK, reinterpret_cast<const uint8_t*>(p.k_cache) + off, kv_bytes,
                                      &s.full_bar[slot]);
                             bulk_g2s(dst + kStageV, reinterpret_cast<const uint8_t*>(p.v_cache) + off, kv_bytes,
                                      &s.full_bar[slot]);
+                        }
+                        if (qkv_bytes != 0) {
+                            if (qkv_ready) {
+                                bulk_g2s(dst + kStageQkv, p.qkv + (size_t)seq_qkv * kQkvWidth, qkv_bytes,
+                                         &s.full_bar[slot]);
+                            } else {
+                                deferred |= 1u << slot;
+                                deferred_seq[slot] = seq_qkv;
+                            }
                         }
                         armed |= 1u << slot;
                         armed_parity = (armed_parity & ~(1u << slot)) | (phase << slot);
@@ -211,12 +236,14 @@ __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, i
                 aborted = true;
                 break;
             }
+            ++issued;
             if (++slot == kStages) {
                 slot = 0;
                 phase ^= 1u;
             }
         }
     }
+    if (lane == 0 && !qkv_ready) release_qkv();   // a range shorter than one round of the ring
     // After an abort, copies this warp issued may still be landing in shared
     // memory: wait (bounded) for each before the CTA may exit.
     if (lane == 0 && *s.abort_flag != 0) {
@@ -846,9 +873,20 @@ cudaError_t prepare_device() {
     return cudaFuncSetAttribute(decode_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
 }
 
-cudaError_t launch(const Params& p, int grid, cudaStream_t stream) {
-    decode_attention_kernel<<<grid, kThreads, kSmemTotal, stream>>>(p);
-    return cudaGetLastError();
+cudaError_t launch(const Params& p, int grid, cudaStream_t stream, bool after_producer) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemTotal;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = after_producer ? 1 : 0;
+    Params q = p;
+    q.qkv_after_wait = after_producer ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, decode_attention_kernel, q);
 }
 
 }  // namespace qda

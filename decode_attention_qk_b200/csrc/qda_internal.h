@@ -55,6 +55,7 @@ struct Params {
     int* status;                  // sticky device error (0 = none)
     int64_t timeout_ns;           // limit of every device-side wait
     unsigned flags;
+    int qkv_after_wait;           // 16-head kernel: launched to depend on the launch writing qkv
 };
 
 // Partial rows per scratch slot of the tensor-core kernel: new tokens x query
@@ -71,8 +72,11 @@ size_t smem_bytes();
 // shared-memory limit). Returns the first CUDA error.
 cudaError_t prepare_device();
 
-// Launch one decode-attention step with `grid` CTAs on `stream` (16 query heads).
-cudaError_t launch(const Params& p, int grid, cudaStream_t stream);
+// Launch one decode-attention step with `grid` CTAs on `stream` (16 query
+// heads). after_producer: the previous launch on the stream writes qkv, and
+// this one starts early (programmatic dependent launch), its K/V streaming
+// overlapping that launch's end; qkv is read only after it completes.
+cudaError_t launch(const Params& p, int grid, cudaStream_t stream, bool after_producer = false);
 
 // The tensor-core step (32, 40 or 64 query heads with one new token; 16
 // heads with 2..4 new tokens, 32 heads with 2): the attention launch, then a

@@ -139,6 +139,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) qkv_proj_kernel(const QkvProjPar
     using Lay = PLayout<MT, kConvert>;
     constexpr int kMTiles = MT / 16;
     extern __shared__ __align__(128) uint8_t smem[];
+    pdl_launch_dependents();   // an attention launch after this one may start its K/V streaming
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
