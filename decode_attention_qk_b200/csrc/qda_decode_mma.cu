@@ -224,8 +224,9 @@ struct State {
 // or in global memory for the largest rows): q of row r = lane/4 (new
 // token r / G, head G*j + r % G) at dims 8m + 2t, 8m + 2t + 1 (t = lane%4,
 // m = 0..15), i.e. both halves of the rotation pairs 8m' + 2t + e, m' < 8.
-// Lane l forms the angles of pairs 2l, 2l+1 for every new token (reduced
-// modulo 2*pi in double, then float sin/cos); lanes fetch theirs by shuffles.
+// Lane l forms the angles of pairs 2l, 2l+1 for the first new token (reduced
+// modulo 2*pi in double, then float sin/cos) and, for the later tokens,
+// rotates them by the per-position step; lanes fetch theirs by shuffles.
 // When this CTA holds a page with new tokens, their k is formed in double.
 template <int G, int T>
 __device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s, const uint8_t* rows, int pos0,
@@ -240,13 +241,20 @@ __device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s,
     const int head = G * j + (active ? r % G : 0);
     float cf[T][2], sf[T][2];
 #pragma unroll
-    for (int u = 0; u < T; ++u)
+    for (int e = 0; e < 2; ++e) {
+        const double ang = (double)pos0 * s.inv_freq[2 * lane + e];
+        const double n = rint(ang * kInvTwoPi);
+        sincosf((float)fma(-n, kTwoPiLo, fma(-n, kTwoPiHi, ang)), &sf[0][e], &cf[0][e]);
+        if (T > 1) {   // later tokens: rotate by the step f (float error ~u * 2^-24, q stays float)
+            float ds, dc;
+            sincosf((float)s.inv_freq[2 * lane + e], &ds, &dc);
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const double ang = (double)(pos0 + u) * s.inv_freq[2 * lane + e];
-            const double n = rint(ang * kInvTwoPi);
-            sincosf((float)fma(-n, kTwoPiLo, fma(-n, kTwoPiHi, ang)), &sf[u][e], &cf[u][e]);
+            for (int u = 1; u < T; ++u) {
+                cf[u][e] = fmaf(cf[u - 1][e], dc, -sf[u - 1][e] * ds);
+                sf[u][e] = fmaf(sf[u - 1][e], dc, cf[u - 1][e] * ds);
+            }
         }
+    }
     const uint32_t* xq =
         reinterpret_cast<const uint32_t*>(rows + tt * Lay::kQkvBytes + head * (kHeadDim * 2));
     const uint32_t* gq = reinterpret_cast<const uint32_t*>(s.gains);
@@ -293,31 +301,54 @@ __device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s,
     }
 
     if (appends) {
-        // lane l: dims 2l, 2l+1 (word l of the head) and 64+2l, 65+2l (word 32+l), all in double
+        // lane l: dims 2l, 2l+1 (word l of the head) and 64+2l, 65+2l (word 32+l), all in double.
+        // The angle of token u is pos0*f + u*f: token 0's sine and cosine, then u
+        // rotations by the step f (error ~u ulp of double, far below k's bf16 rounding).
         const uint32_t* gk = reinterpret_cast<const uint32_t*>(s.gains + kHeadDim);
         const uint32_t wk_lo = gk[lane], wk_hi = gk[32 + lane];
+        double sn0, cs0, sn1, cs1, ds0, dc0, ds1, dc1;
+        sincos((double)pos0 * s.inv_freq[2 * lane], &sn0, &cs0);
+        sincos((double)pos0 * s.inv_freq[2 * lane + 1], &sn1, &cs1);
+        if (T > 1) {
+            sincos(s.inv_freq[2 * lane], &ds0, &dc0);
+            sincos(s.inv_freq[2 * lane + 1], &ds1, &dc1);
+        }
+        double ssq[T];
+        double a0[T], a1[T], b0[T], b1[T];
 #pragma unroll
         for (int u = 0; u < T; ++u) {
-            double cs0, sn0, cs1, sn1;
-            sincos((double)(pos0 + u) * s.inv_freq[2 * lane], &sn0, &cs0);
-            sincos((double)(pos0 + u) * s.inv_freq[2 * lane + 1], &sn1, &cs1);
             const uint8_t* row = rows + u * Lay::kQkvBytes;
             const uint32_t* xk = reinterpret_cast<const uint32_t*>(row + (Lay::kHq + j) * (kHeadDim * 2));
             const uint32_t* xv = reinterpret_cast<const uint32_t*>(row + (Lay::kHq + kNumKvHeads + j) * (kHeadDim * 2));
             const uint32_t xlo = xk[lane], xhi = xk[32 + lane];
-            double a0 = bf_to_d(xlo & 0xFFFFu), a1 = bf_to_d(xlo >> 16);
-            double b0 = bf_to_d(xhi & 0xFFFFu), b1 = bf_to_d(xhi >> 16);
-            const double rr = sqrt(warp_sum(a0 * a0 + a1 * a1 + b0 * b0 + b1 * b1) / 128.0 + p.rms_eps);
-            a0 = a0 / rr * bf_to_d(wk_lo & 0xFFFFu);
-            a1 = a1 / rr * bf_to_d(wk_lo >> 16);
-            b0 = b0 / rr * bf_to_d(wk_hi & 0xFFFFu);
-            b1 = b1 / rr * bf_to_d(wk_hi >> 16);
-            const double ra0 = a0 * cs0 - b0 * sn0, rb0 = b0 * cs0 + a0 * sn0;
-            const double ra1 = a1 * cs1 - b1 * sn1, rb1 = b1 * cs1 + a1 * sn1;
-            st.k_lo[u] = d_to_bf(ra0) | (d_to_bf(ra1) << 16);
-            st.k_hi[u] = d_to_bf(rb0) | (d_to_bf(rb1) << 16);
+            a0[u] = bf_to_d(xlo & 0xFFFFu);
+            a1[u] = bf_to_d(xlo >> 16);
+            b0[u] = bf_to_d(xhi & 0xFFFFu);
+            b1[u] = bf_to_d(xhi >> 16);
+            ssq[u] = a0[u] * a0[u] + a1[u] * a1[u] + b0[u] * b0[u] + b1[u] * b1[u];
             st.v_lo[u] = xv[lane];
             st.v_hi[u] = xv[32 + lane];
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+            for (int u = 0; u < T; ++u) ssq[u] += __shfl_xor_sync(kFull, ssq[u], off);
+#pragma unroll
+        for (int u = 0; u < T; ++u) {
+            const double inv_rr = 1.0 / sqrt(ssq[u] / 128.0 + p.rms_eps);
+            const double x0 = a0[u] * inv_rr * bf_to_d(wk_lo & 0xFFFFu);
+            const double x1 = a1[u] * inv_rr * bf_to_d(wk_lo >> 16);
+            const double y0 = b0[u] * inv_rr * bf_to_d(wk_hi & 0xFFFFu);
+            const double y1 = b1[u] * inv_rr * bf_to_d(wk_hi >> 16);
+            const double ra0 = x0 * cs0 - y0 * sn0, rb0 = y0 * cs0 + x0 * sn0;
+            const double ra1 = x1 * cs1 - y1 * sn1, rb1 = y1 * cs1 + x1 * sn1;
+            st.k_lo[u] = d_to_bf(ra0) | (d_to_bf(ra1) << 16);
+            st.k_hi[u] = d_to_bf(rb0) | (d_to_bf(rb1) << 16);
+            if (u + 1 < T) {   // advance both angles by one position
+                const double c0n = cs0 * dc0 - sn0 * ds0, s0n = sn0 * dc0 + cs0 * ds0;
+                const double c1n = cs1 * dc1 - sn1 * ds1, s1n = sn1 * dc1 + cs1 * ds1;
+                cs0 = c0n; sn0 = s0n; cs1 = c1n; sn1 = s1n;
+            }
         }
     }
 
