@@ -419,7 +419,7 @@ def run_gpu(args):
     # R resident copies of the step's inputs, so that a call never finds its
     # K/V in L2 from the previous call (each copy's KV is > L2 or R copies are).
     first = make_layers(args.workload, dev, rank, args.num_q_heads, T)
-    hidden = inputs.HIDDEN
+    hidden = args.hidden
     if mode == "attention":
         step_bytes = sum(kv_bytes(w.seq_lens) for w in first)
     elif mode == "from_hidden":
@@ -482,26 +482,33 @@ def run_gpu(args):
 
     n_launch = args.steps * calls_per_step
     if args.timing == "graph":
-        # The timed region replays one CUDA graph per step (graph i % rotate holds
-        # the calls of rotation set i % rotate): every call's kernel runs, back to
-        # back, with no host launch between them. Events bracket the K replays.
-        graphs = capture_graphs(calls, fn, dev, rotate)
-        for i in range(rotate):
-            graphs[i].replay()
+        # The timed region replays CUDA graphs that each hold `per_graph`
+        # consecutive steps (step i runs rotation set i % rotate; per_graph is a
+        # multiple of rotate, about 32 calls), plus one graph for the remainder:
+        # exactly K steps, every call's kernel back to back with no host launch
+        # between them. Events bracket the replays.
+        per_graph, full, rest = graph_plan(args.steps, rotate, calls_per_step)
+        g_full = capture_graphs(calls, fn, dev, rotate, per_graph) if full else None
+        g_rest = capture_graphs(calls, fn, dev, rotate, rest) if rest else None
+        for g in (g_full, g_rest):
+            if g is not None:
+                g.replay()
         torch.cuda.synchronize(dev)
         barrier(dist, dev)
         t0 = time.perf_counter()
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         start.record(stream)
-        for i in range(args.steps):
-            graphs[i % rotate].replay()
+        for _ in range(full):
+            g_full.replay()
+        if g_rest is not None:
+            g_rest.replay()
         end.record(stream)
         torch.cuda.synchronize(dev)
         t1 = time.perf_counter()
         barrier(dist, dev)
         ms_local = start.elapsed_time(end)
         kernel_ms = [ms_local / n_launch] * n_launch
-        del graphs
+        del g_full, g_rest
     else:
         t0, t1, ms_local, kernel_ms = timed_eager(args, calls, fn, dev, dist, stream, rotate, calls_per_step)
     clocks.stop()
@@ -577,9 +584,9 @@ def run_gpu(args):
             "config": {"workload": f"{args.workload}: {WORKLOADS[args.workload]}"
                                    + ("" if args.num_q_heads == 16 else f", {args.num_q_heads} query heads")
                                    + ("" if T == 1 else f", {T} new tokens per sequence (causal among them)")
-                                   + {"attention": "", "from_hidden": ", from the hidden state (input_norm + "
-                                      "qkv_proj, then the attention step)", "qkv_proj": ": input_norm + qkv_proj "
-                                      f"only (x [B, {hidden}] -> qkv)"}[mode],
+                                   + {"attention": "", "from_hidden": f", from the hidden state (input_norm + "
+                                      f"qkv_proj of x [B, {hidden}], then the attention step)",
+                                      "qkv_proj": f": input_norm + qkv_proj only (x [B, {hidden}] -> qkv)"}[mode],
                        "op": mode, "batch": first[0].batch, "layers_per_step": calls_per_step, "new_tokens": T,
                        "sum_seq_lens_per_step": int(sum(int(w.seq_lens.sum()) for w in first)),
                        "page_size": 16, "heads": f"{args.num_q_heads} q / 8 kv, D=128",
@@ -594,8 +601,9 @@ def run_gpu(args):
                          "kernel_us_median": round(statistics.median(kernel_ms) * 1e3, 3)},
             "e2e": e2e,
             **({"roofline_tensor": proj_tensor} if proj_tensor is not None else {}),
-            "timing": ("CUDA graph replay: one graph per step, K replays between two events; "
-                       "per-launch duration = region time / launches") if args.timing == "graph"
+            "timing": ("CUDA graph replay: graphs of %d consecutive steps (plus one for the remainder), "
+                       "exactly K steps between two events; per-launch duration = region time / launches"
+                       % graph_plan(args.steps, rotate, calls_per_step)[0]) if args.timing == "graph"
                       else "eager launches, an event pair around each; per-launch duration = mean of the pairs",
             ("eager" if args.timing == "graph" else "graph"): other,
             "seq_per_s": round(first[0].batch / (ms_per_step * 1e-3) * world, 1),
@@ -622,23 +630,31 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
-def capture_graphs(calls, fn, dev, rotate):
-    """One CUDA graph per rotation set, each holding that set's calls (one step)."""
+def graph_plan(steps: int, rotate: int, calls_per_step: int):
+    """(steps per graph, full graphs, steps in the remainder graph): the steps per
+    graph are a multiple of the rotation count and hold about 32 calls."""
+    per_graph = rotate * max(1, math.ceil(32 / (rotate * calls_per_step)))
+    per_graph = min(per_graph, rotate * max(1, steps // rotate))
+    full = steps // per_graph
+    return per_graph, full, steps - full * per_graph
+
+
+def capture_graphs(calls, fn, dev, rotate, steps):
+    """One CUDA graph holding `steps` consecutive steps from step 0 (step i runs
+    rotation set i % rotate)."""
     from decode_attention_qk_b200 import binding
-    graphs = []
     cap = torch.cuda.Stream(dev)
     cap.wait_stream(torch.cuda.current_stream(dev))
-    for r in range(rotate):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=cap):
-            sp = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
-            for c, _ in calls[r]:
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        sp = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+        for i in range(steps):
+            for c, _ in calls[i % rotate]:
                 rc = fn(*c[:-1], sp)
                 if rc != 0:
                     raise binding.QdaError(rc, "capture")
-        graphs.append(g)
     torch.cuda.current_stream(dev).wait_stream(cap)
-    return graphs
+    return g
 
 
 def timed_eager(args, calls, fn, dev, dist, stream, rotate, calls_per_step):
@@ -668,41 +684,34 @@ def timed_eager(args, calls, fn, dev, dist, stream, rotate, calls_per_step):
 
 
 def run_graph(args, attn, calls, fn, dev, dist, rotate, calls_per_step, kv_per_step):
-    """µs per call when the steps are replayed from a CUDA graph: one graph
-    holds a whole rotation cycle (rotate steps), replayed until at least
-    `steps` steps have run, timed by events around the replays."""
-    from decode_attention_qk_b200 import binding
-    g = torch.cuda.CUDAGraph()
-    cap = torch.cuda.Stream(dev)
-    cap.wait_stream(torch.cuda.current_stream(dev))
-    with torch.cuda.graph(g, stream=cap):
-        sp = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
-        for r in range(rotate):
-            for c, _ in calls[r]:
-                rc = fn(*c[:-1], sp)
-                if rc != 0:
-                    raise binding.QdaError(rc, "capture")
+    """µs per call when the K steps are replayed from CUDA graphs (as in the
+    default timed region), for the line timed eagerly."""
+    per_graph, full, rest = graph_plan(args.steps, rotate, calls_per_step)
+    g_full = capture_graphs(calls, fn, dev, rotate, per_graph) if full else None
+    g_rest = capture_graphs(calls, fn, dev, rotate, rest) if rest else None
     stream = torch.cuda.current_stream(dev)
-    for _ in range(2):
-        g.replay()
-    replays = max(1, math.ceil(args.steps / rotate))
+    for g in (g_full, g_rest):
+        if g is not None:
+            g.replay()
     barrier(dist, dev)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
-    for _ in range(replays):
-        g.replay()
+    for _ in range(full):
+        g_full.replay()
+    if g_rest is not None:
+        g_rest.replay()
     end.record(stream)
     torch.cuda.synchronize(dev)
     barrier(dist, dev)
     if attn.check() != 0:
         raise RuntimeError("device status after the graph replays")
     ms = reduce_max(dist, start.elapsed_time(end), dev)
-    steps = replays * rotate
-    ms_per_step = ms / steps
+    ms_per_step = ms / args.steps
     kv_total = reduce_sum(dist, kv_per_step, dev)
-    del g
+    del g_full, g_rest
     return {"us_per_call": round(ms_per_step * 1e3 / calls_per_step, 3), "ms_per_step": round(ms_per_step, 6),
-            "value": round(kv_total / (ms_per_step * 1e-3) / 1e9, 2), "unit": "GB/s", "steps": steps}
+            "value": round(kv_total / (ms_per_step * 1e-3) / 1e9, 2), "unit": "GB/s", "steps": args.steps,
+            "steps_per_graph": per_graph}
 
 
 def run_e2e_proj(args, attn, sets, dev, stream, dist, rotate, mode, fn, unit_bytes):
@@ -723,7 +732,7 @@ def run_e2e_proj(args, attn, sets, dev, stream, dist, rotate, mode, fn, unit_byt
             d = dict(x=x_dev, out=out_dev, sl=w.seq_lens.to(dev), bt=w.block_table.to(dev))
             vp = lambda t: ctypes.c_void_p(t.data_ptr())
             i32 = lambda t: ctypes.cast(ctypes.c_void_p(t.data_ptr()), ctypes.POINTER(ctypes.c_int32))
-            proj = (vp(d["x"]), vp(w.hidden_in["input_norm_w"]), vp(w.hidden_in["w_qkv"]), inputs.HIDDEN)
+            proj = (vp(d["x"]), vp(w.hidden_in["input_norm_w"]), vp(w.hidden_in["w_qkv"]), int(d["x"].shape[1]))
             if mode == "qkv_proj":
                 c = (attn.handle, *proj, vp(qkv_dev), int(w.batch), sp)
             else:
@@ -955,7 +964,8 @@ def run_reference_proj(args, cores, cpu_model):
     mode = "qkv_proj" if args.op == "qkv_proj" else "from_hidden"
     layers = make_layers(args.workload, "cpu", 0, args.num_q_heads, 1)
     for li, w in enumerate(layers):
-        w.hidden_in = inputs.hidden_inputs(w.batch, seed=7000 + li, device="cpu", num_q_heads=args.num_q_heads)
+        w.hidden_in = inputs.hidden_inputs(w.batch, seed=7000 + li, device="cpu", hidden=args.hidden,
+                                           num_q_heads=args.num_q_heads)
     budget = min(20.0, 120.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         cpu_baseline_proj(layers, mode, seconds=budget, threads=cores)
@@ -992,6 +1002,8 @@ def main(argv=None):
                     help="step: the attention step (default); qkv_proj: input_norm + qkv_proj alone")
     ap.add_argument("--from-hidden", action="store_true",
                     help="each call starts from the hidden state: input_norm + qkv_proj, then the attention step")
+    ap.add_argument("--hidden", type=int, default=inputs.HIDDEN,
+                    help="hidden size of the projection modes (1024 for Qwen3-0.6B; 2560, 4096, 5120 for 4B/8B/14B-32B)")
     ap.add_argument("--rotate", type=int, default=0, help="resident input sets cycled (0: enough to defeat L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -91,3 +91,16 @@ def test_reductions_over_two_gloo_ranks():
         assert p.exitcode == 0
     got = sorted(q.get(timeout=5) for _ in range(2))
     assert got == [(0, 5.0, 400.0), (1, 5.0, 400.0)]
+
+
+def test_graph_plan_covers_exactly_the_steps():
+    """The timed region's graphs hold exactly K steps; each graph starts on a
+    multiple of the rotation count, so step i always runs rotation set i % R."""
+    for steps, rotate, calls in [(2000, 2, 1), (1000, 1, 1), (200, 1, 28), (5, 1, 1), (7, 2, 1), (3, 8, 1),
+                                 (2000, 8, 1), (1, 1, 1)]:
+        per_graph, full, rest = bench.graph_plan(steps, rotate, calls)
+        assert per_graph * full + rest == steps
+        assert per_graph % rotate == 0 and rest < per_graph or full == 0
+        # the fewest rotation cycles that reach 32 calls (unless K steps are fewer)
+        assert per_graph == steps or per_graph * calls >= 32 or per_graph == rotate * max(1, steps // rotate)
+        assert per_graph == rotate or (per_graph - rotate) * calls < 32

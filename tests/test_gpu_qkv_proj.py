@@ -117,6 +117,29 @@ def test_attention_fed_by_the_projection(handles):
     ph.assert_o_close(o, ref["o"], "from_hidden o")
 
 
+@pytest.mark.parametrize("hq,hidden", [(32, 2560), (64, 5120)])
+def test_attention_fed_by_the_projection_at_larger_sizes(handles, hq, hidden):
+    """Qwen3-4B (hidden 2560, 32 heads) and 32B (hidden 5120, 64 heads) from the
+    hidden state: the projection, then the tensor-core attention on its qkv."""
+    attn = handles[hq]
+    lens = [1, 33, 700, 17]
+    w = inputs.custom(lens, seed=11 + hq, device="cuda", gap_fraction=0.2, num_q_heads=hq)
+    d = inputs.hidden_inputs(len(lens), seed=12 + hq, hidden=hidden, num_q_heads=hq)
+    x, g, wq = d["x"].to(DEV), d["input_norm_w"].to(DEV), d["w_qkv"].to(DEV)
+    k, v = w.k_cache.clone(), w.v_cache.clone()
+    a = ph.device_args(w, DEV)
+    o, qkv = attn.from_hidden(x, g, wq, a["q_norm_w"], a["k_norm_w"], a["seq_lens"], a["block_table"], k, v)
+    assert attn.check() == 0
+    ref_qkv = oracle.input_norm_qkv_proj(inputs.bf16_bits(d["x"]), inputs.bf16_bits(d["input_norm_w"]),
+                                         inputs.bf16_bits(d["w_qkv"]))
+    check_qkv(qkv, ref_qkv, f"Hq={hq} from_hidden qkv", d)
+    import dataclasses
+    ref = ph.oracle_full(dataclasses.replace(w, qkv=qkv), w.k_cache, w.v_cache)
+    assert np.array_equal(inputs.bf16_bits(k), ref["k_cache"])
+    assert np.array_equal(inputs.bf16_bits(v), ref["v_cache"])
+    ph.assert_o_close(o, ref["o"], f"Hq={hq} from_hidden o")
+
+
 def test_host_side_errors(handles):
     attn = handles[16]
     d = inputs.hidden_inputs(4, seed=10)
