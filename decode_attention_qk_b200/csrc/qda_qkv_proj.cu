@@ -21,8 +21,10 @@
 // of 32 columns each, a CTA needs no reduction of its own.
 //
 // Operands reach shared memory by 16-byte asynchronous copies (cp.async)
-// through a 3-stage ring of 128-wide K chunks, in rows 272 bytes apart so that
-// the 8 rows an ldmatrix phase reads fall in 8 different bank groups. (One
+// through a 3-stage ring of 128-wide K chunks (64-wide for the 64-row blocks
+// of large batches, so that two CTAs share an SM), in rows 16 bytes longer
+// than the chunk so that the 8 rows an ldmatrix phase reads fall in 8
+// different bank groups. (One
 // bulk copy per short row slice was tried first: at about one copy every
 // 45 ns per SM the copy count, not the bytes, set the time.)
 //
@@ -45,9 +47,6 @@ namespace {
 
 constexpr int kNT = kProjNTile;                // output columns per CTA
 constexpr int kKS = kProjKSplits;              // K quarters
-constexpr int kKC = 128;                       // K per chunk
-constexpr int kPitch = kKC * 2 + 16;           // 272-byte staged row pitch
-constexpr int kPieces = kKC / 8;               // 16-byte pieces per row slice
 constexpr int kStages = 3;
 constexpr int kWarps = 4;
 constexpr int kThreadsP = kWarps * 32;
@@ -57,6 +56,12 @@ constexpr int kPrepThreads = 128;
 // copies the split formed by the first launch.
 template <int MT, bool kConvert>
 struct PLayout {
+    // K per chunk: 128, or 64 for the 64-row blocks of large batches, whose
+    // CTAs then fit two to an SM
+    static constexpr int kKC = kConvert ? 128 : 64;
+    static constexpr int kPitch = kKC * 2 + 16;                      // staged row pitch (bytes)
+    static constexpr int kPieces = kKC / 8;                          // 16-byte pieces per row slice
+    static constexpr int kCtasPerSm = kConvert ? 1 : 2;
     static constexpr int kARows = kConvert ? MT : 2 * MT;            // raw x, or hi and lo
     static constexpr int kStageBytes = (kNT + kARows) * kPitch;
     static constexpr int kSmemHiLo = kStages * kStageBytes;          // convert: hi, lo of the current chunk
@@ -65,7 +70,7 @@ struct PLayout {
     static constexpr int kSmemTotal = kSmemInvR + MT * 4;
     // after the K loop the ring holds this quarter's partial tile and sums of x^2
     static_assert((MT * kNT + MT) * 4 <= kStages * kStageBytes, "partial tile fits in the ring");
-    static_assert(kSmemTotal <= 227 * 1024, "fits one CTA per SM");
+    static_assert(kCtasPerSm * (kSmemTotal + 1024) <= 228 * 1024, "CTAs per SM fit in shared memory");
     static_assert(kStageBytes % 16 == 0 && kPitch % 128 == 16, "alignment, conflict-free rows");
 };
 
@@ -135,9 +140,12 @@ __global__ void __launch_bounds__(kPrepThreads) input_norm_split_kernel(const Qk
 // The product, split along K.
 
 template <int MT, bool kConvert>
-__global__ void __launch_bounds__(kThreadsP, 1) qkv_proj_kernel(const QkvProjParams p) {
+__global__ void __launch_bounds__(kThreadsP, PLayout<MT, kConvert>::kCtasPerSm) qkv_proj_kernel(const QkvProjParams p) {
     using Lay = PLayout<MT, kConvert>;
     constexpr int kMTiles = MT / 16;
+    constexpr int kKC = Lay::kKC;
+    constexpr int kPitch = Lay::kPitch;
+    constexpr int kPieces = Lay::kPieces;
     extern __shared__ __align__(128) uint8_t smem[];
     pdl_launch_dependents();   // an attention launch after this one may start its K/V streaming
     const int tid = threadIdx.x;
