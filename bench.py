@@ -802,28 +802,61 @@ def run_e2e(args, attn, sets, dev, stream, dist, rotate):
     for i in range(args.warmup):
         for c, _, _ in host[i % rotate]:
             fn(*c)
+    h2d = sum(h["qkv"].nbytes + h["sl"].nbytes + h["bt"].nbytes for i in range(args.steps)
+              for _, h, _ in host[i % rotate])
+    d2h = sum(h["o"].nbytes for i in range(args.steps) for _, h, _ in host[i % rotate])
+
+    def eager():
+        for i in range(args.steps):
+            for c, h, w in host[i % rotate]:
+                rc = fn(*c)
+                if rc != 0:
+                    raise binding.QdaError(rc, "append_and_attend_host")
+
+    ms_eager = time_region(dist, dev, stream, eager) / args.steps
+    ms_graph, per_graph = None, None
+    if args.timing == "graph":
+        # the same calls (copies in, the step, o copied out) replayed from CUDA graphs
+        calls = [[(c, None) for c, _, _ in hl] for hl in host]
+        per_graph, full, rest = graph_plan(args.steps, rotate, len(host[0]))
+        g_full = capture_graphs(calls, fn, dev, rotate, per_graph) if full else None
+        g_rest = capture_graphs(calls, fn, dev, rotate, rest) if rest else None
+
+        def replay():
+            for _ in range(full):
+                g_full.replay()
+            if g_rest is not None:
+                g_rest.replay()
+
+        replay()
+        ms_graph = time_region(dist, dev, stream, replay) / args.steps
+        del g_full, g_rest
+    if attn.check() != 0:
+        raise RuntimeError("device status after the e2e region")
+    kv = sum(sum(kv_bytes(w.seq_lens) for w in sets[i % rotate]) for i in range(args.steps)) / args.steps
+    kv_total = reduce_sum(dist, kv, dev)
+    ms = ms_graph if ms_graph is not None else ms_eager
+    out = {"value": round(kv_total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+           "h2d_bytes_per_step": int(h2d // args.steps), "d2h_bytes_per_step": int(d2h // args.steps),
+           "ms_per_step": round(ms, 6), "api": "qwen3_decode_attn_append_and_attend_host",
+           "host_buffers": "page-locked and mapped: qkv, seq_lens and the block table read across the host "
+                           "link by one stage-in launch; o written there by the attention kernel"}
+    if ms_graph is not None:
+        out["timing"] = f"the calls replayed from CUDA graphs of {per_graph} steps, copies included"
+        out["eager"] = {"value": round(kv_total / (ms_eager * 1e-3) / 1e9, 2), "ms_per_step": round(ms_eager, 6)}
+    return out
+
+
+def time_region(dist, dev, stream, body) -> float:
+    """Milliseconds `body` takes on the device, between two events (max over ranks)."""
     barrier(dist, dev)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
-    h2d = d2h = 0
-    for i in range(args.steps):
-        for c, h, w in host[i % rotate]:
-            rc = fn(*c)
-            if rc != 0:
-                raise binding.QdaError(rc, "append_and_attend_host")
-            h2d += h["qkv"].nbytes + h["sl"].nbytes + h["bt"].nbytes
-            d2h += h["o"].nbytes
+    body()
     end.record(stream)
     torch.cuda.synchronize(dev)
     barrier(dist, dev)
-    if attn.check() != 0:
-        raise RuntimeError("device status after the e2e region")
-    ms = reduce_max(dist, start.elapsed_time(end), dev) / args.steps
-    kv = sum(sum(kv_bytes(w.seq_lens) for w in sets[i % rotate]) for i in range(args.steps)) / args.steps
-    kv_total = reduce_sum(dist, kv, dev)
-    return {"value": round(kv_total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-            "h2d_bytes_per_step": int(h2d // args.steps), "d2h_bytes_per_step": int(d2h // args.steps),
-            "ms_per_step": round(ms, 6), "api": "qwen3_decode_attn_append_and_attend_host"}
+    return reduce_max(dist, start.elapsed_time(end), dev)
 
 
 def run_e2e_tokens(args, attn, sets, dev, stream, dist, rotate):

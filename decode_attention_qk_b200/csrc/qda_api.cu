@@ -134,6 +134,20 @@ cudaError_t launch_step(const qda_handle* h, const qda::Params& p, cudaStream_t 
                                                                  : qda::launch_grouped(p, h->grid, stream);
 }
 
+// Whether the device can access `p` where it lies (page-locked host memory
+// mapped into the current device's address space); *dev receives the address
+// the device uses. Pageable or unknown memory answers no.
+bool mapped_host(const void* p, void** dev) {
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();   // not a pointer CUDA knows: clear the error
+        return false;
+    }
+    if (a.type != cudaMemoryTypeHost || a.devicePointer == nullptr) return false;
+    *dev = a.devicePointer;
+    return true;
+}
+
 // Host checks of the input_norm + qkv_proj arguments.
 int check_proj(const qda_handle* h, const void* x, const void* input_norm_w, const void* w_qkv, int hidden,
                const void* qkv, int batch) {
@@ -323,22 +337,33 @@ int qwen3_decode_attn_append_and_attend_host(qda_handle* h, const void* qkv_host
     if (!guard.ok()) return QDA_ERR_CUDA;
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     const size_t B = (size_t)batch;
-    bool ok = cudaMemcpyAsync(h->st_qkv, qkv_host, B * qkv_elems(h->cfg.num_q_heads) * sizeof(uint16_t),
-                              cudaMemcpyHostToDevice, st) == cudaSuccess &&
-              cudaMemcpyAsync(h->st_seq_lens, seq_lens_host, B * sizeof(int32_t), cudaMemcpyHostToDevice, st) ==
-                  cudaSuccess &&
-              cudaMemcpyAsync(h->st_block_table, block_table_host, B * (size_t)block_table_stride * sizeof(int32_t),
-                              cudaMemcpyHostToDevice, st) == cudaSuccess &&
-              (positions_host == nullptr ||
-               cudaMemcpyAsync(h->st_positions, positions_host, B * sizeof(int32_t), cudaMemcpyHostToDevice, st) ==
-                   cudaSuccess);
-    if (!ok) return QDA_ERR_CUDA;
+    // Inputs in page-locked host memory that the device can address are
+    // brought over by one stage-in launch; any other host memory by a copy
+    // of its own. o in such memory is written by the attention kernel where
+    // it is; otherwise it is copied out of the staging buffer.
+    qda::StageParams sp{};
+    auto bring = [&](const void* src, void* dst, size_t bytes) {
+        void* dev = nullptr;
+        if (mapped_host(src, &dev)) {
+            sp.r[sp.n++] = qda::StageRange{dev, dst, bytes};
+            return true;
+        }
+        return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, st) == cudaSuccess;
+    };
+    const bool ok = bring(qkv_host, h->st_qkv, B * qkv_elems(h->cfg.num_q_heads) * sizeof(uint16_t)) &&
+                    bring(seq_lens_host, h->st_seq_lens, B * sizeof(int32_t)) &&
+                    bring(block_table_host, h->st_block_table, B * (size_t)block_table_stride * sizeof(int32_t)) &&
+                    (positions_host == nullptr || bring(positions_host, h->st_positions, B * sizeof(int32_t)));
+    if (!ok || qda::launch_stage_in(sp, 2 * h->grid, st) != cudaSuccess) return QDA_ERR_CUDA;
+    void* o_dev = nullptr;
+    const bool o_mapped = mapped_host(o_host, &o_dev) && aligned(o_dev, 16);
     const qda::Params p = make_params(h, h->st_qkv, q_norm_w, k_norm_w, h->st_seq_lens,
                                       positions_host != nullptr ? h->st_positions : nullptr, h->st_block_table,
-                                      block_table_stride, k_cache, v_cache, num_pages, h->st_o, batch);
+                                      block_table_stride, k_cache, v_cache, num_pages, o_mapped ? o_dev : h->st_o,
+                                      batch);
     if (launch_step(h, p, st) != cudaSuccess) return QDA_ERR_CUDA;
-    if (cudaMemcpyAsync(o_host, h->st_o, B * (size_t)h->cfg.num_q_heads * qda::kHeadDim * sizeof(uint16_t),
-                        cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    if (!o_mapped && cudaMemcpyAsync(o_host, h->st_o, B * (size_t)h->cfg.num_q_heads * qda::kHeadDim * sizeof(uint16_t),
+                                     cudaMemcpyDeviceToHost, st) != cudaSuccess)
         return QDA_ERR_CUDA;
     return QDA_OK;
 }

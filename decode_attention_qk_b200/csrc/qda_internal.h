@@ -111,6 +111,22 @@ struct QkvProjParams {
 cudaError_t prepare_qkv_proj();
 cudaError_t launch_qkv_proj(const QkvProjParams& p, cudaStream_t stream);
 
+// Stage-in of the host-buffer entry point (qda_host_stage.cu): copy up to
+// kMaxStageRanges ranges from device-addressable host memory (page-locked and
+// mapped) to device memory in one launch. Every range is 4-byte aligned at
+// both ends and a multiple of 4 bytes long.
+constexpr int kMaxStageRanges = 4;
+struct StageRange {
+    const void* src;   // the device's address of the host buffer
+    void* dst;         // device memory
+    size_t bytes;
+};
+struct StageParams {
+    StageRange r[kMaxStageRanges];
+    int n;
+};
+cudaError_t launch_stage_in(const StageParams& sp, int max_ctas, cudaStream_t stream);
+
 // Whether the tensor-core kernel has an instance for this head and token count.
 bool grouped_supported(int num_q_heads, int new_tokens);
 

@@ -261,13 +261,19 @@ int qwen3_decode_attn_from_hidden(qda_handle *h,
 
 /* The same step for a caller whose per-step tensors are in HOST memory:
  * qkv_host, seq_lens_host, positions_host (or NULL) and block_table_host are
- * host pointers (pinned memory makes the copies asynchronous), and o_host is
- * the host destination of o. q_norm_w, k_norm_w, k_cache and v_cache stay
- * device pointers (weights and cache are device-resident state). The call
- * queues host-to-device copies into the handle's staging buffers, the step,
- * and the device-to-host copy of o, all on `cuda_stream`, and returns; o_host
- * is valid after the stream is synchronized. Requires block_table_stride <=
- * max_pages_per_seq. Errors as for qwen3_decode_attn_append_and_attend. */
+ * host pointers, and o_host is the host destination of o. q_norm_w, k_norm_w,
+ * k_cache and v_cache stay device pointers (weights and cache are
+ * device-resident state). qkv, seq_lens, positions and the block table are
+ * brought into the handle's device staging buffers: those in page-locked host
+ * memory that the device can address (from cudaHostAlloc / cudaMallocHost or
+ * registered with cudaHostRegister, as cudaPointerGetAttributes reports it)
+ * by one library launch that reads them across the host link, any others by
+ * a copy each. o in such memory (16-byte aligned) is written by the attention
+ * kernel where it lies; otherwise it is copied out of the staging buffer.
+ * All of it is queued on `cuda_stream` and the call returns; o_host is valid after
+ * the stream is synchronized, and the host buffers must not change before
+ * then. Requires block_table_stride <= max_pages_per_seq. Errors as for
+ * qwen3_decode_attn_append_and_attend. */
 int qwen3_decode_attn_append_and_attend_host(qda_handle *h,
                                              const void *qkv_host,
                                              const void *q_norm_w,

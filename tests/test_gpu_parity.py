@@ -159,6 +159,43 @@ def test_host_buffer_entry_point(attn):
     assert torch.equal(k0.view(torch.int16), w.k_cache.view(torch.int16))
 
 
+def pinned_at_offset(t):
+    """A page-locked copy of int32 `t` starting 4 bytes past a 16-byte boundary."""
+    flat = torch.empty(t.numel() + 1, dtype=t.dtype).pin_memory()
+    v = flat[1:].view(t.shape)
+    v.copy_(t)
+    assert v.data_ptr() % 16 == 4
+    return v
+
+
+@pytest.mark.parametrize("mapped", ["none", "inputs", "o", "all", "offset"])
+def test_host_buffer_entry_point_mixed_memory(attn, mapped):
+    """Pageable buffers go through copies, page-locked ones through the
+    stage-in launch (inputs) or in place (o), at 16-byte or only 4-byte
+    alignment; any mix gives the bytes of the device entry point."""
+    w = inputs.custom([300, 2, 16, 1025, 40], seed=25, device="cuda", gap_fraction=0.3)
+    positions = (w.seq_lens - 1 + torch.tensor([0, 5, 0, 1000, 7], dtype=torch.int32)).contiguous()
+    k0, v0 = w.k_cache.clone(), w.v_cache.clone()
+    a = ph.device_args(w, DEV)
+    o_dev = attn(a["qkv"], a["q_norm_w"], a["k_norm_w"], a["seq_lens"], a["block_table"], w.k_cache, w.v_cache,
+                 positions=positions.to(DEV))
+    torch.cuda.synchronize(DEV)
+    pin_in = mapped in ("inputs", "all")
+    host = lambda t, pin: t.cpu().pin_memory() if pin else t.cpu().clone()
+    ints = pinned_at_offset if mapped == "offset" else (lambda t: host(t, pin_in))
+    o_host = torch.full((5, 16, 128), 3.0, dtype=torch.bfloat16)
+    if mapped in ("o", "all"):
+        o_host = o_host.pin_memory()
+    binding.qwen3_decode_attn_append_and_attend_host(
+        attn.handle, host(w.qkv, pin_in or mapped == "offset"), w.q_norm_w, w.k_norm_w, ints(w.seq_lens),
+        ints(positions), ints(w.block_table), k0, v0, o_host)
+    torch.cuda.synchronize(DEV)
+    assert attn.check() == 0
+    assert torch.equal(o_host.view(torch.int16), o_dev.cpu().view(torch.int16))
+    assert torch.equal(k0.view(torch.int16), w.k_cache.view(torch.int16))
+    assert torch.equal(v0.view(torch.int16), w.v_cache.view(torch.int16))
+
+
 # ----------------------------------------------------------------------------
 # device-side errors: recorded in the status word, no out-of-range access
 
