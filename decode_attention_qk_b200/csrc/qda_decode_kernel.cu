@@ -78,7 +78,9 @@ static_assert(kSmemTotal <= 227 * 1024, "fits one CTA per SM");
 // Merging split sequences. Once every consumer warp is past its last page the
 // ring is free: warp j merges in its own 1/8 of it, copying up to kMergeBatch
 // pieces' partials (1 KiB of un-normalised output for heads 2j, 2j+1, and 16 B
-// of running max and sum) with one bulk copy per piece and lane.
+// of running max and sum per piece). The scratch holds kv head j's rows of
+// consecutive slots next to each other (part_row), so a batch of pieces is two
+// bulk copies: the output rows and the (max, sum) pairs.
 constexpr int kMergeRegion = kStages * kStageBytes / kConsumerWarps;
 constexpr int kMergeRowBytes = kGroup * kHeadDim * 4;                      // 1 KiB
 constexpr int kMergeBatch = 24;
@@ -479,6 +481,15 @@ __device__ __forceinline__ void store_bf16x8(uint16_t* dst, const float* v, floa
     *reinterpret_cast<uint4*>(dst) = w;
 }
 
+// Row of the split-piece scratch for kv head j, scratch slot `slot` and query
+// head 2j + hb: kv head major, then slot, then the head pair, so that one kv
+// head's rows of consecutive slots are contiguous. The slot stride is grid +
+// batch (slots are CTA + sequence), within the workspace's grid + max_batch.
+__device__ __forceinline__ size_t part_row(const Params& p, int j, int slot, int hb) {
+    const size_t stride = (size_t)gridDim.x + (size_t)p.batch;
+    return ((size_t)j * stride + (size_t)slot) * kGroup + (size_t)hb;
+}
+
 // End of a sequence piece: merge the 4 token groups, then write o directly
 // when this CTA holds the whole sequence, else write this piece's partial
 // (un-normalised output and its running max and sum) to scratch slot
@@ -538,11 +549,11 @@ __device__ __forceinline__ bool finish_piece(const Params& p, const Shared& s, i
         store_bf16x8(p.o + ((size_t)b * kNumQHeads + head) * kHeadDim + dim0, out, Lh > 0.f ? 1.f / Lh : 0.f);
         return false;
     }
-    const int slot = blockIdx.x + b;
-    float4* pa = reinterpret_cast<float4*>(p.part_acc + ((size_t)slot * kNumQHeads + head) * kHeadDim + dim0);
+    const size_t row = part_row(p, j, (int)blockIdx.x + b, hb);
+    float4* pa = reinterpret_cast<float4*>(p.part_acc + row * kHeadDim + dim0);
     __stcg(pa, make_float4(out[0], out[1], out[2], out[3]));
     __stcg(pa + 1, make_float4(out[4], out[5], out[6], out[7]));
-    if (c == 0 && hf == 0) __stcg(p.part_ml + (size_t)slot * kNumQHeads + head, make_float2(Mh, Lh));
+    if (c == 0 && hf == 0) __stcg(p.part_ml + row, make_float2(Mh, Lh));
     return true;
 }
 
@@ -591,10 +602,11 @@ __device__ __forceinline__ bool merge_sequence(const Params& p, const Shared& s,
         __syncwarp();
         if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)nb * (kMergeRowBytes + 16));
         __syncwarp();
-        if (lane < nb) {
-            const size_t row = (size_t)(first + b + t0 + lane) * kNumQHeads + kGroup * j;
-            bulk_g2s(region + lane * kMergeRowBytes, p.part_acc + row * kHeadDim, (uint32_t)kMergeRowBytes, bar);
-            bulk_g2s(region + kMergeMlOff + lane * 16, p.part_ml + row, 16u, bar);
+        if (lane == 0) {
+            // rows of slots first + b + t0 .. + nb - 1 for heads 2j, 2j+1: contiguous
+            const size_t row = part_row(p, j, first + b + t0, 0);
+            bulk_g2s(region, p.part_acc + row * kHeadDim, (uint32_t)nb * kMergeRowBytes, bar);
+            bulk_g2s(region + kMergeMlOff, p.part_ml + row, (uint32_t)nb * 16u, bar);
         }
         if (!warp_wait(p, s, bar, mphase, lane)) {
             // the copies may still be landing: wait once more (bounded) before leaving

@@ -47,8 +47,9 @@ struct Params {
     double rms_eps;
     // workspace
     float* part_acc;              // [num_slots][rows][128] un-normalised partial sums; rows = 16 for the
-                                  // 16-head kernel, kPartRows for the tensor-core kernel
-    float2* part_ml;              // [num_slots][rows] (running max in log2 units, sum)
+                                  // 16-head kernel (ordered kv head, slot, head pair there), kPartRows
+                                  // for the tensor-core kernel
+    float2* part_ml;              // [num_slots][rows] (running max in log2 units, sum), same row order
     int* seg;                     // [kMaxBatch + 1] page offsets of the sequences (written for the combine
                                   // launch of the 32/40/64-head kernels; unused at 16 heads)
     int* counters;                // [kMaxBatch][8] merge arrival counters, zero between calls
