@@ -808,21 +808,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_kernel(const Par
     s.done_bar = s.merge_bar + kConsumerWarps;
     s.abort_flag = reinterpret_cast<volatile int*>(smem + kSmemFlags);
 
-    // Pages per sequence (0 for a sequence whose length is out of range).
-    const int B = p.batch;
-    for (int b = threadIdx.x; b < B; b += kThreads) {
-        const int L = p.seq_lens[b];
-        const bool ok = L >= 1 && L <= p.max_seq_len && L <= kPage * p.bt_stride;
-        if (!ok && blockIdx.x == 0) record_error(p.status, QDA_ERR_BOUNDS);
-        s.lens[b] = L;
-        s.seg[b + 1] = ok ? (L + kPage - 1) / kPage : 0;
-    }
-    if (threadIdx.x < 64) {
-        // both gain vectors, one 8-byte word per thread
-        const uint16_t* src = threadIdx.x < 32 ? p.q_norm_w : p.k_norm_w;
-        reinterpret_cast<uint2*>(smem + kSmemGains)[threadIdx.x] =
-            *reinterpret_cast<const uint2*>(src + 4 * (threadIdx.x & 31));
-    } else if (threadIdx.x < 128) {
+    // Every launch is a programmatic dependent launch: the next launch on the
+    // stream may be scheduled now (its CTAs take an SM as one of these ends),
+    // and this one may have started before the previous launch finished. The
+    // prologue below touches no global memory; griddepcontrol.wait then holds
+    // until the previous launch has completed and its writes are visible
+    // (in the mode where that launch only writes qkv, the wait comes later,
+    // before the qkv copies).
+    pdl_launch_dependents();
+    if (threadIdx.x >= 64 && threadIdx.x < 128) {
         const int i = threadIdx.x - 64;
         s.inv_freq[i] = pow(p.rope_theta, -2.0 * i / 128.0);
     }
@@ -837,6 +831,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_kernel(const Par
         *s.abort_flag = 0;
         s.seg[0] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (p.qkv_after_wait == 0) pdl_wait();
+
+    // Pages per sequence (0 for a sequence whose length is out of range).
+    const int B = p.batch;
+    for (int b = threadIdx.x; b < B; b += kThreads) {
+        const int L = p.seq_lens[b];
+        const bool ok = L >= 1 && L <= p.max_seq_len && L <= kPage * p.bt_stride;
+        if (!ok && blockIdx.x == 0) record_error(p.status, QDA_ERR_BOUNDS);
+        s.lens[b] = L;
+        s.seg[b + 1] = ok ? (L + kPage - 1) / kPage : 0;
+    }
+    if (threadIdx.x < 64) {
+        // both gain vectors, one 8-byte word per thread
+        const uint16_t* src = threadIdx.x < 32 ? p.q_norm_w : p.k_norm_w;
+        reinterpret_cast<uint2*>(smem + kSmemGains)[threadIdx.x] =
+            *reinterpret_cast<const uint2*>(src + 4 * (threadIdx.x & 31));
     }
     __syncthreads();
     if (warp == 0) {  // inclusive scan of the page counts: seg[b] becomes the first page of b
@@ -895,7 +906,7 @@ cudaError_t launch(const Params& p, int grid, cudaStream_t stream, bool after_pr
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = after_producer ? 1 : 0;
+    cfg.numAttrs = 1;
     Params q = p;
     q.qkv_after_wait = after_producer ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, decode_attention_kernel, q);

@@ -38,8 +38,10 @@
 // second launch (one CTA per sequence and kv head, one warp per query row)
 // combines them with the log-sum-exp rule (Supported models, "Facts proved
 // about the specs": flashAttn_eq, softmax_shift), spreading long merges over
-// many SMs. That launch uses programmatic dependent launch so its start
-// overlaps the first kernel's tail.
+// many SMs. Both launches are programmatic dependent launches: the combine
+// launch starts while the attention launch ends, and the attention launch
+// while the previous step's last launch ends; each waits for its predecessor
+// to complete before it touches global memory.
 #include <cuda_bf16.h>
 #include <cstdint>
 
@@ -596,19 +598,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
     s.never_bar = s.qkv_empty + 1;
     s.abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kSmemFlags);
 
-    const int B = p.batch;
-    for (int b = threadIdx.x; b < B; b += kThreads) {
-        const int L = p.seq_lens[b];
-        const bool ok = L >= T && L <= p.max_seq_len && L <= kPage * p.bt_stride;
-        if (!ok && blockIdx.x == 0) record_error(p.status, QDA_ERR_BOUNDS);
-        s.lens[b] = L;
-        s.seg[b + 1] = ok ? (L + kPage - 1) / kPage : 0;
-    }
-    if (threadIdx.x < 64) {
-        const uint16_t* src = threadIdx.x < 32 ? p.q_norm_w : p.k_norm_w;
-        reinterpret_cast<uint2*>(smem + Lay::kSmemGains)[threadIdx.x] =
-            *reinterpret_cast<const uint2*>(src + 4 * (threadIdx.x & 31));
-    } else if (threadIdx.x < 128) {
+    // Launched as a programmatic dependent launch: the prologue below touches
+    // no global memory, and griddepcontrol.wait holds until the previous
+    // launch on the stream has completed and its writes are visible.
+    if (threadIdx.x >= 64 && threadIdx.x < 128) {
         const int i = threadIdx.x - 64;
         s.inv_freq[i] = pow(p.rope_theta, -2.0 * i / 128.0);
     }
@@ -623,6 +616,21 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
         *s.abort_flag = 0;
         s.seg[0] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    pdl_wait();
+
+    const int B = p.batch;
+    for (int b = threadIdx.x; b < B; b += kThreads) {
+        const int L = p.seq_lens[b];
+        const bool ok = L >= T && L <= p.max_seq_len && L <= kPage * p.bt_stride;
+        if (!ok && blockIdx.x == 0) record_error(p.status, QDA_ERR_BOUNDS);
+        s.lens[b] = L;
+        s.seg[b + 1] = ok ? (L + kPage - 1) / kPage : 0;
+    }
+    if (threadIdx.x < 64) {
+        const uint16_t* src = threadIdx.x < 32 ? p.q_norm_w : p.k_norm_w;
+        reinterpret_cast<uint2*>(smem + Lay::kSmemGains)[threadIdx.x] =
+            *reinterpret_cast<const uint2*>(src + 4 * (threadIdx.x & 31));
     }
     __syncthreads();
     if (warp == 0) {  // inclusive scan of the page counts
@@ -674,6 +682,7 @@ template <int G, int T>
 __global__ void __launch_bounds__(32 * G * T, 1) combine_kernel(const Params p, int main_grid) {
     using Lay = Layout<G, T>;
     pdl_wait();   // the first launch has finished and its writes are visible
+    pdl_launch_dependents();   // the next step's attention launch may be scheduled
     const int b = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tt = warp / G;
     const int h = G * blockIdx.y + warp % G;
@@ -734,17 +743,23 @@ cudaError_t prepare_one() {
 
 template <int G, int T>
 cudaError_t launch_one(const Params& p, int grid, cudaStream_t stream) {
-    grouped_attention_kernel<G, T><<<grid, kThreads, Layout<G, T>::kSmemTotal, stream>>>(p);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t main = {};
+    main.gridDim = dim3((unsigned)grid, 1, 1);
+    main.blockDim = dim3(kThreads, 1, 1);
+    main.dynamicSmemBytes = Layout<G, T>::kSmemTotal;
+    main.stream = stream;
+    main.attrs = attr;
+    main.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&main, grouped_attention_kernel<G, T>, p);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p.batch, (unsigned)kNumKvHeads, 1);
     cfg.blockDim = dim3(32 * G * T, 1, 1);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, combine_kernel<G, T>, p, grid);

@@ -13,6 +13,7 @@
 
 #include <cuda_runtime.h>
 
+#include "qda_device.cuh"
 #include "qda_internal.h"
 
 namespace qda {
@@ -21,6 +22,9 @@ namespace {
 constexpr int kStageThreads = 256;
 
 __global__ void __launch_bounds__(kStageThreads) stage_in_kernel(StageParams sp) {
+    // the attention launch that follows may be scheduled now; it waits for
+    // this launch to complete before it reads anything
+    pdl_launch_dependents();
     const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     const size_t nthreads = (size_t)gridDim.x * blockDim.x;
 #pragma unroll

@@ -74,9 +74,11 @@ size_t smem_bytes();
 cudaError_t prepare_device();
 
 // Launch one decode-attention step with `grid` CTAs on `stream` (16 query
-// heads). after_producer: the previous launch on the stream writes qkv, and
-// this one starts early (programmatic dependent launch), its K/V streaming
-// overlapping that launch's end; qkv is read only after it completes.
+// heads), as a programmatic dependent launch: its CTAs may be scheduled while
+// the previous launch on the stream ends, and they read and write global
+// memory only after it has completed. after_producer: that previous launch
+// writes qkv and nothing else this step reads, so K/V streaming starts at
+// once and only qkv waits for it to complete.
 cudaError_t launch(const Params& p, int grid, cudaStream_t stream, bool after_producer = false);
 
 // The tensor-core step (32, 40 or 64 query heads with one new token; 16
