@@ -582,8 +582,8 @@ __device__ __forceinline__ int pieces_of(const Shared& s, int b, int per_cta, in
 // through this warp's merge region; o = sum_t 2^(m_t - M) acc_t / sum_t
 // 2^(m_t - M) l_t with M the running maximum, rescaled between batches.
 // Returns false when a wait ran out.
-__device__ __forceinline__ bool merge_sequence(const Params& p, const Shared& s, int b, int j, int lane, int grp, int c,
-                                               int per_cta, uint32_t& mphase) {
+__device__ __forceinline__ bool merge_sequence(const Params& p, const Shared& s, int b, int j, int lane, int issuer,
+                                               int grp, int c, int per_cta, uint32_t& mphase) {
     const int hb = grp & 1;
     const int hf = grp >> 1;
     const int head = kGroup * j + hb;
@@ -600,9 +600,8 @@ __device__ __forceinline__ bool merge_sequence(const Params& p, const Shared& s,
         // earlier reads of the region come before the copies that overwrite it
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
-        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)nb * (kMergeRowBytes + 16));
-        __syncwarp();
-        if (lane == 0) {
+        if (lane == issuer) {
+            mbar_arrive_expect_tx(bar, (uint32_t)nb * (kMergeRowBytes + 16));
             // rows of slots first + b + t0 .. + nb - 1 for heads 2j, 2j+1: contiguous
             const size_t row = part_row(p, j, first + b + t0, 0);
             bulk_g2s(region, p.part_acc + row * kHeadDim, (uint32_t)nb * kMergeRowBytes, bar);
@@ -776,18 +775,20 @@ __device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, i
     int first = 0, prev = -1, need = 0;
     if (lane < npend) {
         need = pieces_of(s, mine, per_cta, first) - 1;
-        prev = atomicAdd(p.counters + mine * kNumKvHeads + j, 1);
+        // acquire: the last to arrive sees every other piece's released partial
+        prev = atomic_add_acquire(p.counters + mine * kNumKvHeads + j, 1);
     }
     const bool last0 = __shfl_sync(kFull, prev == need, 0);
     const bool last1 = __shfl_sync(kFull, prev == need, 1) && npend == 2;
     if (!last0 && !last1) return;
-    // the other pieces' partials, read through the async proxy by the merge copies
-    __threadfence();
+    // The other pieces' partials are read through the async proxy by bulk
+    // copies, each batch issued by the lane whose acquiring increment found
+    // the sequence complete (lane 0 for pending0, lane 1 for pending1).
     asm volatile("fence.proxy.async.global;" ::: "memory");
     if (!warp_wait(p, s, s.done_bar, 0u, lane)) return;
     uint32_t mphase = 0;
-    if (last0 && !merge_sequence(p, s, pending0, j, lane, grp, c, per_cta, mphase)) return;
-    if (last1) (void)merge_sequence(p, s, pending1, j, lane, grp, c, per_cta, mphase);
+    if (last0 && !merge_sequence(p, s, pending0, j, lane, 0, grp, c, per_cta, mphase)) return;
+    if (last1) (void)merge_sequence(p, s, pending1, j, lane, 1, grp, c, per_cta, mphase);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) decode_attention_kernel(const Params p) {

@@ -94,6 +94,14 @@ __device__ __forceinline__ void record_error(int* status, int code) { atomicCAS(
 
 // Programmatic dependent launch: let the next kernel in the stream start its
 // prologue, and wait for the previous kernel's results.
+// atomicAdd with acquire semantics at GPU scope: what other threads released
+// before their own increments is visible to this thread after it.
+__device__ __forceinline__ int atomic_add_acquire(int* addr, int v) {
+    int old;
+    asm volatile("atom.acquire.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+    return old;
+}
+
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
