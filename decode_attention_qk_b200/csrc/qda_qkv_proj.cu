@@ -54,39 +54,24 @@ constexpr int kPrepThreads = 128;
 
 // kConvert: the CTA forms the split itself from raw x (up to 32 rows); else it
 // copies the split formed by the first launch.
-//
-// Operand tiles are stored K-major in the tensor cores' canonical layout
-// without swizzle: core matrices of 8 rows x 16 bytes (8 bf16 along K), rows
-// 16 bytes apart; the core matrices of a row group follow one another along K
-// (128 bytes apart) and row groups follow at kKC * 16 bytes. That order is
-// simply 16-byte piece i = (row group, piece along K, row within the group),
-// so copy i lands at byte 16 i.
 template <int MT, bool kConvert>
 struct PLayout {
     // K per chunk: 128, or 64 for the 64-row blocks of large batches, whose
     // CTAs then fit two to an SM
     static constexpr int kKC = kConvert ? 128 : 64;
+    static constexpr int kPitch = kKC * 2 + 16;                      // staged row pitch (bytes)
     static constexpr int kPieces = kKC / 8;                          // 16-byte pieces per row slice
-    static constexpr uint32_t kLBO = 128;                            // next core matrix along K
-    static constexpr uint32_t kSBO = kKC * 16;                       // next group of 8 rows
     static constexpr int kCtasPerSm = kConvert ? 1 : 2;
-    static constexpr int kWBytes = kNT * kKC * 2;                    // the weight tile
-    static constexpr int kABytes = MT * kKC * 2;                     // one tile of MT rows
-    static constexpr int kStageBytes = kWBytes + (kConvert ? 1 : 2) * kABytes;   // + raw x, or hi and lo
-    static constexpr int kSmemHiLo = kStages * kStageBytes;          // convert: 2 buffers of (hi, lo)
-    static constexpr int kSmemGain = kSmemHiLo + (kConvert ? 4 * kABytes : 0);   // bf16 [hidden / 4]
-    static constexpr int kSmemSq = kSmemGain + (kConvert ? kMaxHidden / kKS * 2 : 0);   // float [MT][kPieces]
-    static constexpr int kSmemInvR = kSmemSq + (kConvert ? MT * kPieces * 4 : 0);      // float [MT]
-    static constexpr int kSmemBars = kSmemInvR + MT * 4;                               // uint64 [kStages]
-    static constexpr int kSmemTmem = kSmemBars + kStages * 8;                          // TMEM address
-    static constexpr int kSmemTotal = kSmemTmem + 16;
-    // the accumulator: 128 TMEM lanes (output columns) x MT columns (rows)
-    static constexpr uint32_t kTmemCols = MT < 32 ? 32 : MT;
+    static constexpr int kARows = kConvert ? MT : 2 * MT;            // raw x, or hi and lo
+    static constexpr int kStageBytes = (kNT + kARows) * kPitch;
+    static constexpr int kSmemHiLo = kStages * kStageBytes;          // convert: hi, lo of the current chunk
+    static constexpr int kSmemGain = kSmemHiLo + (kConvert ? 2 * MT * kPitch : 0);   // bf16 [hidden / 4]
+    static constexpr int kSmemInvR = kSmemGain + (kConvert ? kMaxHidden / kKS * 2 : 0);  // float [MT]
+    static constexpr int kSmemTotal = kSmemInvR + MT * 4;
     // after the K loop the ring holds this quarter's partial tile and sums of x^2
     static_assert((MT * kNT + MT) * 4 <= kStages * kStageBytes, "partial tile fits in the ring");
     static_assert(kCtasPerSm * (kSmemTotal + 1024) <= 228 * 1024, "CTAs per SM fit in shared memory");
-    static_assert(kStageBytes % 1024 == 0 && kSmemBars % 8 == 0, "alignment");
-    static_assert(MT % 16 == 0 && MT >= 16 && MT <= 256, "N of one tensor-core instruction");
+    static_assert(kStageBytes % 16 == 0 && kPitch % 128 == 16, "alignment, conflict-free rows");
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
@@ -95,65 +80,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-// ---------------------------------------------------------------------------
-// The 5th-generation tensor cores (tcgen05): descriptors and instructions.
-
-// Shared-memory matrix descriptor of a K-major operand in the canonical layout
-// without swizzle: start address >> 4 in bits [0,14), leading byte offset
-// (between the two core matrices of a 16-element K step) >> 4 in [16,30),
-// stride byte offset (between groups of 8 rows) >> 4 in [32,46), descriptor
-// version 1 in [46,48), base offset 0, layout 0 (no swizzle) in [61,64).
-__host__ __device__ constexpr uint64_t umma_smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
-}
-// Instruction descriptor of kind::f16: f32 accumulator (bits [4,6) = 1), bf16
-// A and B (bits [7,10) = 1, [10,13) = 1), both K-major (bits 15, 16 = 0),
-// N >> 3 in [17,23), M >> 4 in [24,29); M = 128.
-__host__ __device__ constexpr uint32_t umma_idesc_bf16_m128(int n) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
-}
-static_assert(umma_idesc_bf16_m128(64) == 0x08100490u, "instruction descriptor bits");
-static_assert(umma_smem_desc(0x400u, 128u, 1024u) == ((0x40ull) | (8ull << 16) | (64ull << 32) | (1ull << 46)),
-              "matrix descriptor bits");
-
-// D[tmem] (+)= A * B^T for one K step of 16, issued by one thread.
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-// The mbarrier gets one arrival once every tensor-core instruction this thread
-// issued before has completed (and read its shared-memory operands).
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
-                 : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-// Warp-wide: allocate `cols` TMEM columns (a power of two >= 32), address to *dst.
-__device__ __forceinline__ void tmem_alloc(void* dst, uint32_t cols) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst)), "r"(cols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
-}
-// Warp-wide: 16 consecutive columns of this warp's 32 TMEM lanes, one lane per thread.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, "
-        "[%16];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
-          "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-        : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ float warp_sum_f(float v) {
 #pragma unroll
@@ -216,9 +142,11 @@ __global__ void __launch_bounds__(kPrepThreads) input_norm_split_kernel(const Qk
 template <int MT, bool kConvert>
 __global__ void __launch_bounds__(kThreadsP, PLayout<MT, kConvert>::kCtasPerSm) qkv_proj_kernel(const QkvProjParams p) {
     using Lay = PLayout<MT, kConvert>;
+    constexpr int kMTiles = MT / 16;
     constexpr int kKC = Lay::kKC;
+    constexpr int kPitch = Lay::kPitch;
     constexpr int kPieces = Lay::kPieces;
-    extern __shared__ __align__(1024) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     pdl_launch_dependents();   // an attention launch after this one may start its K/V streaming
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -231,38 +159,28 @@ __global__ void __launch_bounds__(kThreadsP, PLayout<MT, kConvert>::kCtasPerSm) 
     const int kbase = ks * kq;
     const int chunks = kq / kKC;
     const uint32_t ring = smem_addr(smem);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kSmemBars);   // [s]: the products of a chunk in stage s
 
-    // piece i of a tile: row ((i / (8 kPieces)) * 8 + i % 8), piece (i / 8) % kPieces along K, at byte 16 i
-    auto piece_row = [](int i) { return ((i / (8 * kPieces)) << 3) | (i & 7); };
-    auto piece_k = [](int i) { return (i >> 3) % kPieces; };
-    auto weight_rows = [&](int c) {   // 128 rows x kKC: needs nothing from a first launch
+    auto weight_rows = [&](int c) {   // 128 rows x 128: needs nothing from a first launch
         const uint32_t stage = ring + (c % kStages) * Lay::kStageBytes;
-        for (int i = tid; i < kNT * kPieces; i += kThreadsP)
-            cp_async16(stage + i * 16, p.w + (size_t)(n0 + piece_row(i)) * p.hidden + (size_t)(kbase + c * kKC) +
-                                           piece_k(i) * 8);
+        for (int i = tid; i < kNT * kPieces; i += kThreadsP) {
+            const int r = i / kPieces, q = i % kPieces;
+            cp_async16(stage + r * kPitch + q * 16,
+                       p.w + (size_t)(n0 + r) * p.hidden + (size_t)(kbase + c * kKC) + q * 8);
+        }
     };
-    auto a_rows = [&](int c) {        // raw x rows, or hi and lo rows (rows past the batch are left as they are)
-        const uint32_t stage = ring + (c % kStages) * Lay::kStageBytes + Lay::kWBytes;
-        for (int i = tid; i < MT * kPieces; i += kThreadsP) {
-            const int r = piece_row(i);
-            if (r >= rows) continue;
-            const size_t src = (size_t)(m0 + r) * p.hidden + (size_t)(kbase + c * kKC) + piece_k(i) * 8;
+    auto a_rows = [&](int c) {        // raw x rows, or hi and lo rows
+        const uint32_t stage = ring + (c % kStages) * Lay::kStageBytes + kNT * kPitch;
+        for (int i = tid; i < rows * kPieces; i += kThreadsP) {
+            const int r = i / kPieces, q = i % kPieces;
+            const size_t src = (size_t)(m0 + r) * p.hidden + (size_t)(kbase + c * kKC) + q * 8;
             if (kConvert) {
-                cp_async16(stage + i * 16, p.x + src);
+                cp_async16(stage + r * kPitch + q * 16, p.x + src);
             } else {
-                cp_async16(stage + i * 16, p.xg_hi + src);
-                cp_async16(stage + Lay::kABytes + i * 16, p.xg_lo + src);
+                cp_async16(stage + r * kPitch + q * 16, p.xg_hi + src);
+                cp_async16(stage + (MT + r) * kPitch + q * 16, p.xg_lo + src);
             }
         }
     };
-
-    // the accumulator in tensor memory, and one mbarrier per stage
-    if (warp == 0) tmem_alloc(smem + Lay::kSmemTmem, Lay::kTmemCols);
-    if (tid == 0) {
-        for (int k = 0; k < kStages; ++k) mbar_init(&bars[k], 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
     // Groups, oldest first: {gain quarter and weight of chunks 0..S-2}, {A of
     // chunk 0}, ..., {A of chunk S-2}, then one group per later chunk.
     const int pre = min(kStages - 1, chunks);
@@ -275,71 +193,75 @@ __global__ void __launch_bounds__(kThreadsP, PLayout<MT, kConvert>::kCtasPerSm) 
         if (c < pre) a_rows(c);
         cp_async_commit();
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + Lay::kSmemTmem);
-    constexpr uint32_t kIdesc = umma_idesc_bf16_m128(MT);
 
-    // kConvert: thread tid splits pieces tid + 128 m of the raw x tile
+    const int g = lane >> 2, t = lane & 3;
+    // kConvert: thread tid splits pieces tid + 128 m (row (tid + 128 m) / 16,
+    // piece tid % 16); the 16 threads of a half-warp share a row
     constexpr int kConvPerThread = kConvert ? MT * kPieces / kThreadsP : 1;
     float ss[kConvPerThread];
 #pragma unroll
     for (int m = 0; m < kConvPerThread; ++m) ss[m] = 0.f;
-    bool ok = true;   // every wait so far completed
+    float acc[kMTiles][4][4];
+#pragma unroll
+    for (int i = 0; i < kMTiles; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
     for (int c = 0; c < chunks; ++c) {
-        cp_async_wait<kStages - 2>();   // this thread's copies of chunk c have landed
-        uint32_t b_hi;
-        if (kConvert) {
-            __syncthreads();            // ... and everyone's raw x
-            const uint8_t* raw = smem + (c % kStages) * Lay::kStageBytes + Lay::kWBytes;
-            // buffer c % 2: the products of chunk c - 2 that read it are complete
-            uint8_t* hilo = smem + Lay::kSmemHiLo + (c & 1) * 2 * Lay::kABytes;
-            const uint32_t* gw = reinterpret_cast<const uint32_t*>(smem + Lay::kSmemGain) + (c * kKC) / 2;
-#pragma unroll
-            for (int m = 0; m < kConvPerThread; ++m) {
-                const int i = tid + kThreadsP * m;
-                uint4 hv, lv;
-                split_piece(*reinterpret_cast<const uint4*>(raw + i * 16), gw + 4 * piece_k(i), hv, lv, ss[m]);
-                *reinterpret_cast<uint4*>(hilo + i * 16) = hv;
-                *reinterpret_cast<uint4*>(hilo + Lay::kABytes + i * 16) = lv;
-            }
-            b_hi = smem_addr(hilo);
-        } else {
-            b_hi = ring + (c % kStages) * Lay::kStageBytes + Lay::kWBytes;
-        }
-        // the staged and split operands are read by the tensor cores (async proxy)
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncthreads();
-        if (tid == 0 && ok) {
-            tc_fence_after();
-            const uint32_t a = ring + (c % kStages) * Lay::kStageBytes;
-            const uint32_t b_lo = b_hi + Lay::kABytes;
-#pragma unroll
-            for (int k = 0; k < kKC / 16; ++k) {   // 16 along K = 2 core matrices = 256 bytes
-                const uint64_t da = umma_smem_desc(a + k * 256, Lay::kLBO, Lay::kSBO);
-                umma_bf16(tmem, da, umma_smem_desc(b_hi + k * 256, Lay::kLBO, Lay::kSBO), kIdesc, (c | k) != 0);
-                umma_bf16(tmem, da, umma_smem_desc(b_lo + k * 256, Lay::kLBO, Lay::kSBO), kIdesc, 1u);
-            }
-            umma_commit(&bars[c % kStages]);
-        }
-        // refill the stage of chunk c - 1 once its products are complete
-        if (c >= 1 && ok) {
-            ok = mbar_wait(&bars[(c - 1) % kStages], (uint32_t)(((c - 1) / kStages) & 1), p.timeout_ns, nullptr);
-            if (!ok && tid == 0) record_error(p.status, QDA_ERR_TIMEOUT);
-        }
-        if (c + kStages - 1 < chunks && ok) {
+        if (c + kStages - 1 < chunks) {
             weight_rows(c + kStages - 1);
             a_rows(c + kStages - 1);
         }
         cp_async_commit();
+        cp_async_wait<kStages - 1>();   // this thread's copies of chunk c have landed ...
+        __syncthreads();                // ... and everyone's
+        const uint32_t stage = ring + (c % kStages) * Lay::kStageBytes;
+        uint32_t abase_hi, abase_lo;
+        if (kConvert) {
+            const uint8_t* raw = smem + (c % kStages) * Lay::kStageBytes + kNT * kPitch;
+            const uint32_t* gw = reinterpret_cast<const uint32_t*>(smem + Lay::kSmemGain) + (c * kKC) / 2;
+#pragma unroll
+            for (int m = 0; m < kConvPerThread; ++m) {
+                const int i = tid + kThreadsP * m;
+                const int r = i / kPieces, q = i % kPieces;
+                uint4 hv, lv;
+                split_piece(*reinterpret_cast<const uint4*>(raw + r * kPitch + q * 16), gw + 4 * q, hv, lv, ss[m]);
+                *reinterpret_cast<uint4*>(smem + Lay::kSmemHiLo + r * kPitch + q * 16) = hv;
+                *reinterpret_cast<uint4*>(smem + Lay::kSmemHiLo + (MT + r) * kPitch + q * 16) = lv;
+            }
+            __syncthreads();
+            abase_hi = ring + Lay::kSmemHiLo;
+        } else {
+            abase_hi = stage + kNT * kPitch;
+        }
+        abase_lo = abase_hi + MT * kPitch;
+        // ldmatrix row addresses: this warp's 32 weight rows as the column-major
+        // B operand, hi and lo rows as the row-major A operand
+        const uint32_t wbase =
+            stage + (32 * warp + (lane & 7) + ((lane >> 4) << 3)) * kPitch + ((lane >> 3) & 1) * 16;
+        const uint32_t aoff = ((lane & 7) + ((lane >> 3) & 1) * 8) * kPitch + ((lane >> 4) & 1) * 16;
+#pragma unroll
+        for (int kstep = 0; kstep < kKC / 16; ++kstep) {
+            const int k0 = kstep * 16;
+            uint32_t b[4][2];
+            ldsm_x4(wbase + k0 * 2, b[0][0], b[0][1], b[1][0], b[1][1]);
+            ldsm_x4(wbase + 16 * kPitch + k0 * 2, b[2][0], b[2][1], b[3][0], b[3][1]);
+#pragma unroll
+            for (int i = 0; i < kMTiles; ++i) {
+                uint32_t ahi[4], alo[4];
+                ldsm_x4(abase_hi + aoff + i * 16 * kPitch + k0 * 2, ahi[0], ahi[1], ahi[2], ahi[3]);
+                ldsm_x4(abase_lo + aoff + i * 16 * kPitch + k0 * 2, alo[0], alo[1], alo[2], alo[3]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    mma_bf16_16816(acc[i][j], ahi, b[j][0], b[j][1]);
+                    mma_bf16_16816(acc[i][j], alo, b[j][0], b[j][1]);
+                }
+            }
+        }
+        __syncthreads();                // the stage (and the hi/lo buffer) may be refilled
     }
     cp_async_wait<0>();
-    if (ok) {
-        ok = mbar_wait(&bars[(chunks - 1) % kStages], (uint32_t)(((chunks - 1) / kStages) & 1), p.timeout_ns, nullptr);
-        if (!ok && tid == 0) record_error(p.status, QDA_ERR_TIMEOUT);
-    }
-    tc_fence_after();
 
     // This quarter's partial tile (float) and, when converting, its sums of x^2,
     // in shared memory for the cluster.
@@ -347,35 +269,26 @@ __global__ void __launch_bounds__(kThreadsP, PLayout<MT, kConvert>::kCtasPerSm) 
     cg::cluster_group cluster = cg::this_cluster();
     float* tile = reinterpret_cast<float*>(smem);   // [MT][kNT], the ring is drained
     float* tss = tile + MT * kNT;                   // [MT]
-    if (kConvert) {
-        float* sq = reinterpret_cast<float*>(smem + Lay::kSmemSq);   // [MT][kPieces]
 #pragma unroll
-        for (int m = 0; m < kConvPerThread; ++m) {
-            const int i = tid + kThreadsP * m;
-            sq[piece_row(i) * kPieces + piece_k(i)] = ss[m];
+    for (int i = 0; i < kMTiles; ++i) {
+        const int r0 = 16 * i + g;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int col = 32 * warp + 8 * j + 2 * t;
+            *reinterpret_cast<float2*>(tile + r0 * kNT + col) = make_float2(acc[i][j][0], acc[i][j][1]);
+            *reinterpret_cast<float2*>(tile + (r0 + 8) * kNT + col) = make_float2(acc[i][j][2], acc[i][j][3]);
         }
     }
-    // warp w holds TMEM lanes 32w..32w+31 = output columns; TMEM column r = row r
+    if (kConvert) {
 #pragma unroll
-    for (int r0 = 0; r0 < MT; r0 += 16) {
-        uint32_t v[16];
-        tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)r0, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) tile[(r0 + j) * kNT + 32 * warp + lane] = __uint_as_float(v[j]);
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (kConvert && tid < MT) {
-        const float* sq = reinterpret_cast<const float*>(smem + Lay::kSmemSq) + tid * kPieces;
-        float v = 0.f;
-#pragma unroll
-        for (int q = 0; q < kPieces; ++q) v += sq[q];
-        tss[tid] = v;
-    }
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, Lay::kTmemCols);
+        for (int m = 0; m < kConvPerThread; ++m) {
+            float v = ss[m];
+            v += __shfl_xor_sync(kFull, v, 1);
+            v += __shfl_xor_sync(kFull, v, 2);
+            v += __shfl_xor_sync(kFull, v, 4);
+            v += __shfl_xor_sync(kFull, v, 8);
+            if ((lane & 15) == 0) tss[(tid + kThreadsP * m) / kPieces] = v;
+        }
     }
     cluster.sync();   // all four quarters' partials are in place
     const int q = (int)cluster.block_rank();   // = ks
