@@ -228,6 +228,18 @@ def hidden_inputs(B: int, seed: int = 0, device="cpu", hidden: int = HIDDEN,
     return dict(x=x, input_norm_w=g, w_qkv=w)
 
 
+def o_proj_inputs(B: int, seed: int = 0, device="cpu", hidden: int = HIDDEN,
+                  num_q_heads: int = NUM_Q_HEADS) -> dict:
+    """Inputs of attn.o_proj: x bf16 [B, Hq * 128] ~ N(0, 1) (the attention output
+    o [B, Hq, 128] read as rows); the o_proj weight bf16 [hidden, Hq * 128] ~
+    N(0, 1/(Hq * 128)), so that the outputs stay O(1)."""
+    dev = torch.device(device)
+    K = num_q_heads * HEAD_DIM
+    x = torch.randn((B, K), generator=_gen(seed * 16 + 9, dev), device=dev).to(torch.bfloat16)
+    w = (torch.randn((hidden, K), generator=_gen(seed * 16 + 10, dev), device=dev) / math.sqrt(K)).to(torch.bfloat16)
+    return dict(x=x, w_o=w)
+
+
 def bf16_bits(t: torch.Tensor):
     """numpy uint16 view of a bf16 tensor's bits (copied to the host)."""
     return t.detach().to("cpu").contiguous().view(torch.int16).numpy().view("uint16")

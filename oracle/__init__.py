@@ -68,6 +68,8 @@ def _load():
         lib.oracle_input_norm_qkv_proj.argtypes = [u16p, u16p, u16p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                     ctypes.c_double, dp, u16p]
         lib.oracle_input_norm_qkv_proj.restype = ctypes.c_int
+        lib.oracle_o_proj.argtypes = [u16p, u16p, ctypes.c_int, ctypes.c_int, ctypes.c_int, dp, u16p]
+        lib.oracle_o_proj.restype = ctypes.c_int
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_set_threads.restype = None
         lib.oracle_get_threads.argtypes = []
@@ -97,6 +99,26 @@ def input_norm_qkv_proj(x, norm_w, w, rms_eps: float = 1e-6) -> dict:
                                             _ptr(y, ctypes.c_double), _ptr(bits, ctypes.c_uint16))
     if rc != 0:
         raise ValueError(f"oracle_input_norm_qkv_proj: {_ERRORS.get(rc, rc)}")
+    return {"y": y, "bits": bits}
+
+
+def o_proj(x, w) -> dict:
+    """attn.o_proj (Model Spec, "Compute-graph nodes": linear, K = 2048, N = 1024
+    for Qwen3-0.6B): x bf16 bits [B, K] (the attention output o [B, Hq, 128] as
+    rows of Hq * 128), w [N, K] (row n = output n). Returns ``y`` float64 [B, N]
+    (exact) and ``bits`` uint16 [B, N] (y rounded once to bf16, nearest-even)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    x = x.reshape(x.shape[0], -1)
+    assert w.ndim == 2 and w.shape[1] == x.shape[1]
+    B, K = x.shape
+    N = w.shape[0]
+    y = np.empty((B, N), dtype=np.float64)
+    bits = np.empty((B, N), dtype=np.uint16)
+    rc = _load().oracle_o_proj(_ptr(x, ctypes.c_uint16), _ptr(w, ctypes.c_uint16), B, K, N,
+                               _ptr(y, ctypes.c_double), _ptr(bits, ctypes.c_uint16))
+    if rc != 0:
+        raise ValueError(f"oracle_o_proj: {_ERRORS.get(rc, rc)}")
     return {"y": y, "bits": bits}
 
 

@@ -39,7 +39,8 @@
  *
  * It also holds the two nodes that produce the step's input, input_norm and
  * attn.qkv_proj (oracle_input_norm_qkv_proj), with nothing rounded before the
- * bf16 qkv row.
+ * bf16 qkv row, and the node that consumes its output, attn.o_proj
+ * (oracle_o_proj).
  *
  * Every function names the passage it follows. The pins that tie this file to
  * the pages and to mathematics (closed forms, invariants, library routines,
@@ -397,6 +398,38 @@ int oracle_input_norm_qkv_proj(const uint16_t *x, const uint16_t *norm_w, const 
     free(g);
     free(row);
     free(xn);
+    return 0;
+}
+
+/* ---- attn.o_proj (the step's consumer) ----------------------------------- */
+
+/* The node after the attention core in the Model Spec's "Compute-graph
+ * nodes" table: attn.o_proj, a linear map y[t,n] = sum_k x[t,k] * w[n,k] with
+ * K = 2048, N = 1024 for Qwen3-0.6B and no bias. Its input x[t] is the core's
+ * output o[b] of [16][128] read as one row of 16 * 128 (the "Tensors of the
+ * main nodes" table gives attn.core's o [B, 16, 128] and attn.o_proj's
+ * x [T, 2048]).
+ *
+ *   x        bf16 [B][K]   the attention output rows
+ *   w        bf16 [N][K]   o_proj weight, row n = output feature n
+ *   y_out    double [B][N] the exact (double) product, or NULL
+ *   y_bits   bf16 [B][N]   y rounded once to bf16 (nearest-even), or NULL
+ *
+ * The sum over k runs in index order. Returns 0 or ORC_ERR_ARG. */
+int oracle_o_proj(const uint16_t *x, const uint16_t *w, int B, int K, int N, double *y_out, uint16_t *y_bits)
+{
+    if (!x || !w || B < 1 || K < 1 || N < 1 || (!y_out && !y_bits))
+        return ORC_ERR_ARG;
+    for (int b = 0; b < B; ++b) {
+        const uint16_t *xb = x + (size_t)b * K;
+        for (int n = 0; n < N; ++n) {
+            const uint16_t *wn = w + (size_t)n * K;
+            double acc = 0.0;
+            for (int k = 0; k < K; ++k) acc += oracle_bf16_to_f64(xb[k]) * oracle_bf16_to_f64(wn[k]);
+            if (y_out) y_out[(size_t)b * N + n] = acc;
+            if (y_bits) y_bits[(size_t)b * N + n] = oracle_f64_to_bf16_rne(acc);
+        }
+    }
     return 0;
 }
 
