@@ -236,7 +236,7 @@ int oracle_append_and_attend_tokens(const uint16_t *qkv, const uint16_t *q_norm_
 {
     if (!qkv || !q_norm_w || !k_norm_w || !seq_lens || !block_table || !k_cache ||
         !v_cache || !o || B < 1 || B > ORC_MAX_BATCH || bt_stride < 1 || num_pages < 1 ||
-        T < 1 || T > 16 ||
+        T < 1 || T > ORC_MAX_SEQ ||
         num_q_heads < ORC_NUM_KV_HEADS || num_q_heads % ORC_NUM_KV_HEADS != 0 || num_q_heads > 64)
         return ORC_ERR_ARG;
     const int group = num_q_heads / ORC_NUM_KV_HEADS;

@@ -498,10 +498,10 @@ def _tok_args(w, oracle_mod):
                 v_cache=inputs.bf16_bits(w.v_cache))
 
 
-@pytest.mark.parametrize("T,hq", [(2, 16), (3, 16), (4, 16), (2, 32)])
+@pytest.mark.parametrize("T,hq", [(2, 16), (3, 16), (4, 16), (2, 32), (8, 16), (5, 64), (24, 16)])
 def test_tokens_match_sdpa_with_bottom_right_causal_mask(oracle_mod, T, hq):
     from decode_attention_qk_b200 import inputs
-    w = inputs.custom([T, 17, 40], seed=50 + T, num_q_heads=hq, new_tokens=T, pool_pages=6)
+    w = inputs.custom([T, max(17, T), max(40, T + 16)], seed=50 + T, num_q_heads=hq, new_tokens=T, pool_pages=8)
     out = oracle_mod.append_and_attend_tokens(**_tok_args(w, oracle_mod), want_qk=True)
     kc, vc = out["k_cache"], out["v_cache"]
     for b, L in enumerate(w.seq_lens.tolist()):
