@@ -27,9 +27,12 @@ QDA_FLAG_INJECT_WAIT_TIMEOUT = 0x1
 
 NUM_Q_HEADS, NUM_KV_HEADS, HEAD_DIM, PAGE_SIZE, QKV_WIDTH = 16, 8, 128, 16, 4096
 SUPPORTED_Q_HEADS = (16, 32, 40, 64)   # Qwen3 0.6B/1.7B, 4B/8B, 14B, 32B
-MAX_NEW_TOKENS = 4
+MAX_NEW_TOKENS = 40960
 # (query heads, new tokens) pairs with a kernel for more than one new token
-SUPPORTED_MULTI_TOKEN = ((16, 2), (16, 3), (16, 4), (32, 2))
+# (query heads, new tokens) pairs that one launch of the multi-token step
+# takes: T >= 2 with at most 16 query rows (T * Hq / 8) per kv head; longer
+# blocks run as several launches
+SUPPORTED_MULTI_TOKEN = tuple((hq, t) for hq in (16, 32, 40, 64) for t in range(2, 9) if t * hq // 8 <= 16)
 
 
 class qda_config(ctypes.Structure):
@@ -81,6 +84,8 @@ def load_library():
         lib.qwen3_decode_attn_append_and_attend_tokens.restype = ctypes.c_int
         lib.qwen3_decode_attn_qkv_proj.argtypes = [vp, vp, vp, vp, ctypes.c_int, vp, ctypes.c_int, vp]
         lib.qwen3_decode_attn_qkv_proj.restype = ctypes.c_int
+        lib.qwen3_decode_attn_o_proj.argtypes = [vp, vp, vp, ctypes.c_int, vp, ctypes.c_int, vp]
+        lib.qwen3_decode_attn_o_proj.restype = ctypes.c_int
         lib.qwen3_decode_attn_from_hidden.argtypes = [vp, vp, vp, vp, ctypes.c_int, vp, vp, vp, i32p, i32p, i32p,
                                                       ctypes.c_int, vp, vp, ctypes.c_int, vp, ctypes.c_int, vp]
         lib.qwen3_decode_attn_from_hidden.restype = ctypes.c_int
@@ -228,6 +233,26 @@ def qwen3_decode_attn_qkv_proj(handle, num_q_heads, x, input_norm_w, w_qkv, qkv,
         raise QdaError(rc, "qwen3_decode_attn_qkv_proj")
 
 
+def qwen3_decode_attn_o_proj(handle, num_q_heads, x, w_o, y, stream=None) -> None:
+    """attn.o_proj on device tensors: x [B, Hq, 128] or [B, Hq * 128] (the attention
+    output), w_o [hidden, Hq * 128], y [B, hidden] (output)."""
+    dev = x.device
+    K = num_q_heads * HEAD_DIM
+    B = int(x.shape[0])
+    if x.dim() == 3:
+        _expect(x, "x", torch.bfloat16, (B, num_q_heads, HEAD_DIM), dev)
+    else:
+        _expect(x, "x", torch.bfloat16, (B, K), dev)
+    if w_o.dim() != 2:
+        raise ValueError("w_o must be [hidden, Hq * 128]")
+    hidden = int(w_o.shape[0])
+    _expect(w_o, "w_o", torch.bfloat16, (hidden, K), dev)
+    _expect(y, "y", torch.bfloat16, (B, hidden), dev)
+    rc = load_library().qwen3_decode_attn_o_proj(handle, _ptr(x), _ptr(w_o), hidden, _ptr(y), B, _stream(stream, dev))
+    if rc != QDA_OK:
+        raise QdaError(rc, "qwen3_decode_attn_o_proj")
+
+
 def qwen3_decode_attn_from_hidden(handle, num_q_heads, x, input_norm_w, w_qkv, qkv, q_norm_w, k_norm_w, seq_lens,
                                   positions, block_table, k_cache, v_cache, o, stream=None) -> None:
     """qkv_proj into `qkv`, then the attention step on it (one new token per sequence)."""
@@ -323,6 +348,13 @@ class DecodeAttention:
                               device=x.device)
         qwen3_decode_attn_qkv_proj(self.handle, self.config.num_q_heads, x, input_norm_w, w_qkv, qkv, stream)
         return qkv
+
+    def o_proj(self, x, w_o, y=None, stream=None) -> torch.Tensor:
+        """attn.o_proj: y [B, hidden] from the attention output x [B, Hq, 128] (or [B, Hq * 128])."""
+        if y is None:
+            y = torch.empty((x.shape[0], w_o.shape[0]), dtype=torch.bfloat16, device=x.device)
+        qwen3_decode_attn_o_proj(self.handle, self.config.num_q_heads, x, w_o, y, stream)
+        return y
 
     def from_hidden(self, x, input_norm_w, w_qkv, q_norm_w, k_norm_w, seq_lens, block_table, k_cache, v_cache,
                     qkv=None, o=None, positions=None, stream=None):

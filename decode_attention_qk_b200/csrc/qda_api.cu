@@ -18,17 +18,18 @@ struct qda_handle {
     float2* part_ml = nullptr;
     int* counters = nullptr;
     int* status = nullptr;
-    int* seg = nullptr;
     // input_norm + qkv_proj: the exact split of x*g, and 1/r per row
     uint16_t* xg_hi = nullptr;
     uint16_t* xg_lo = nullptr;
     float* inv_r = nullptr;
-    // staging of the host-buffer entry point
-    uint16_t* st_qkv = nullptr;
-    int32_t* st_seq_lens = nullptr;
-    int32_t* st_positions = nullptr;
-    int32_t* st_block_table = nullptr;
-    uint16_t* st_o = nullptr;
+    // staging of the host-buffer entry point: two sets, used by alternate
+    // calls, so that one call's stage-in overlaps the previous call's attention
+    uint16_t* st_qkv[2] = {nullptr, nullptr};
+    int32_t* st_seq_lens[2] = {nullptr, nullptr};
+    int32_t* st_positions[2] = {nullptr, nullptr};
+    int32_t* st_block_table[2] = {nullptr, nullptr};
+    uint16_t* st_o[2] = {nullptr, nullptr};
+    unsigned host_calls = 0;
 };
 
 namespace {
@@ -65,15 +66,16 @@ void free_workspace(qda_handle* h) {
     cudaFree(h->part_ml);
     cudaFree(h->counters);
     cudaFree(h->status);
-    cudaFree(h->seg);
     cudaFree(h->xg_hi);
     cudaFree(h->xg_lo);
     cudaFree(h->inv_r);
-    cudaFree(h->st_qkv);
-    cudaFree(h->st_seq_lens);
-    cudaFree(h->st_positions);
-    cudaFree(h->st_block_table);
-    cudaFree(h->st_o);
+    for (int k = 0; k < 2; ++k) {
+        cudaFree(h->st_qkv[k]);
+        cudaFree(h->st_seq_lens[k]);
+        cudaFree(h->st_positions[k]);
+        cudaFree(h->st_block_table[k]);
+        cudaFree(h->st_o[k]);
+    }
 }
 
 template <typename T>
@@ -112,6 +114,9 @@ qda::Params make_params(const qda_handle* h, const void* qkv, const void* q_norm
     p.o = static_cast<uint16_t*>(o);
     p.num_q_heads = h->cfg.num_q_heads;
     p.new_tokens = 1;
+    p.tok_stride = 1;
+    p.tok_offset = 0;
+    p.len_trim = 0;
     p.bt_stride = block_table_stride;
     p.num_pages = num_pages;
     p.batch = batch;
@@ -121,7 +126,6 @@ qda::Params make_params(const qda_handle* h, const void* qkv, const void* q_norm
     p.part_acc = h->part_acc;
     p.part_ml = h->part_ml;
     p.counters = h->counters;
-    p.seg = h->seg;
     p.status = h->status;
     p.timeout_ns = h->cfg.wait_timeout_ns > 0 ? h->cfg.wait_timeout_ns : kDefaultTimeoutNs;
     p.flags = h->cfg.flags;
@@ -240,14 +244,15 @@ int qwen3_decode_attn_create(const qda_config* cfg, int device, qda_handle** out
     bool ok = alloc(&h->part_acc, slots * rows * qda::kHeadDim * sizeof(float)) &&
               alloc(&h->part_ml, slots * rows * sizeof(float2)) &&
               alloc(&h->counters, (size_t)qda::kMaxBatch * qda::kNumKvHeads * sizeof(int)) &&
-              alloc(&h->status, sizeof(int)) && alloc(&h->seg, (size_t)(qda::kMaxBatch + 1) * sizeof(int)) &&
-              alloc(&h->st_qkv, B * qkv_elems(cfg->num_q_heads) * sizeof(uint16_t)) &&
-              alloc(&h->st_seq_lens, B * sizeof(int32_t)) && alloc(&h->st_positions, B * sizeof(int32_t)) &&
-              alloc(&h->st_block_table, B * (size_t)cfg->max_pages_per_seq * sizeof(int32_t)) &&
-              alloc(&h->st_o, B * Hq * qda::kHeadDim * sizeof(uint16_t)) &&
+              alloc(&h->status, sizeof(int)) &&
               alloc(&h->xg_hi, B * (size_t)qda::kMaxHidden * sizeof(uint16_t)) &&
               alloc(&h->xg_lo, B * (size_t)qda::kMaxHidden * sizeof(uint16_t)) &&
               alloc(&h->inv_r, B * sizeof(float));
+    for (int k = 0; k < 2 && ok; ++k)
+        ok = alloc(&h->st_qkv[k], B * qkv_elems(cfg->num_q_heads) * sizeof(uint16_t)) &&
+             alloc(&h->st_seq_lens[k], B * sizeof(int32_t)) && alloc(&h->st_positions[k], B * sizeof(int32_t)) &&
+             alloc(&h->st_block_table[k], B * (size_t)cfg->max_pages_per_seq * sizeof(int32_t)) &&
+             alloc(&h->st_o[k], B * Hq * qda::kHeadDim * sizeof(uint16_t));
     ok = ok && cudaMemset(h->counters, 0, (size_t)qda::kMaxBatch * qda::kNumKvHeads * sizeof(int)) == cudaSuccess &&
          cudaMemset(h->status, 0, sizeof(int)) == cudaSuccess && cudaDeviceSynchronize() == cudaSuccess;
     if (!ok) {
@@ -282,14 +287,34 @@ int qwen3_decode_attn_append_and_attend_tokens(qda_handle* h, const void* qkv, c
     int rc = check_call(h, qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, block_table_stride, k_cache,
                         v_cache, num_pages, o, batch);
     if (rc != QDA_OK) return rc;
-    if (new_tokens < 1 || new_tokens > QDA_MAX_NEW_TOKENS) return QDA_ERR_INVALID_ARG;
-    if (new_tokens > 1 && !qda::grouped_supported(h->cfg.num_q_heads, new_tokens)) return QDA_ERR_UNSUPPORTED;
+    if (new_tokens < 1 || new_tokens > QDA_MAX_NEW_TOKENS || new_tokens > h->cfg.max_seq_len)
+        return QDA_ERR_INVALID_ARG;
     DeviceGuard guard(h->device);
     if (!guard.ok()) return QDA_ERR_CUDA;
     qda::Params p = make_params(h, qkv, q_norm_w, k_norm_w, seq_lens, positions, block_table, block_table_stride,
                                 k_cache, v_cache, num_pages, o, batch);
-    p.new_tokens = new_tokens;
-    return launch_step(h, p, static_cast<cudaStream_t>(cuda_stream)) == cudaSuccess ? QDA_OK : QDA_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    p.tok_stride = new_tokens;
+    if (new_tokens == 1) return launch_step(h, p, st) == cudaSuccess ? QDA_OK : QDA_ERR_CUDA;
+    // A block longer than one launch takes runs as consecutive launches over
+    // consecutive chunks of its tokens. Chunk [c0, c0 + n) sees the cache plus
+    // the block's tokens up to its own (its launch trims the later ones from
+    // seq_lens), so each token still attends over exactly the slots up to its
+    // own. At 16 query heads no chunk is a single token (that is the other
+    // kernel's shape): a remainder of one borrows a token from the chunk before.
+    const int max_t = qda::grouped_max_tokens(h->cfg.num_q_heads);
+    if (max_t < 2) return QDA_ERR_UNSUPPORTED;
+    for (int c0 = 0; c0 < new_tokens;) {
+        int n = new_tokens - c0 < max_t ? new_tokens - c0 : max_t;
+        if (h->cfg.num_q_heads == qda::kNumQHeads && new_tokens - c0 - n == 1) --n;
+        p.new_tokens = n;
+        p.tok_offset = c0;
+        p.len_trim = new_tokens - c0 - n;
+        if (!qda::grouped_supported(h->cfg.num_q_heads, n)) return QDA_ERR_UNSUPPORTED;
+        if (qda::launch_grouped(p, h->grid, st) != cudaSuccess) return QDA_ERR_CUDA;
+        c0 += n;
+    }
+    return QDA_OK;
 }
 
 int qwen3_decode_attn_qkv_proj(qda_handle* h, const void* x, const void* input_norm_w, const void* w_qkv, int hidden,
@@ -300,6 +325,26 @@ int qwen3_decode_attn_qkv_proj(qda_handle* h, const void* x, const void* input_n
     if (!guard.ok()) return QDA_ERR_CUDA;
     const qda::QkvProjParams p = make_proj_params(h, x, input_norm_w, w_qkv, hidden, qkv, batch);
     return qda::launch_qkv_proj(p, static_cast<cudaStream_t>(cuda_stream)) == cudaSuccess ? QDA_OK : QDA_ERR_CUDA;
+}
+
+int qwen3_decode_attn_o_proj(qda_handle* h, const void* x, const void* w_o, int hidden, void* y, int batch,
+                             void* cuda_stream) {
+    if (h == nullptr || x == nullptr || w_o == nullptr || y == nullptr) return QDA_ERR_INVALID_ARG;
+    if (batch < 1 || batch > h->cfg.max_batch || hidden < 128 || hidden > qda::kMaxHidden || hidden % 128 != 0)
+        return QDA_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w_o, 16) || !aligned(y, 16)) return QDA_ERR_INVALID_ARG;
+    DeviceGuard guard(h->device);
+    if (!guard.ok()) return QDA_ERR_CUDA;
+    qda::OProjParams p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.w = static_cast<const uint16_t*>(w_o);
+    p.y = static_cast<uint16_t*>(y);
+    p.batch = batch;
+    p.in_features = h->cfg.num_q_heads * qda::kHeadDim;
+    p.hidden = hidden;
+    p.status = h->status;
+    p.timeout_ns = h->cfg.wait_timeout_ns > 0 ? h->cfg.wait_timeout_ns : kDefaultTimeoutNs;
+    return qda::launch_o_proj(p, static_cast<cudaStream_t>(cuda_stream)) == cudaSuccess ? QDA_OK : QDA_ERR_CUDA;
 }
 
 int qwen3_decode_attn_from_hidden(qda_handle* h, const void* x, const void* input_norm_w, const void* w_qkv,
@@ -330,13 +375,16 @@ int qwen3_decode_attn_append_and_attend_host(qda_handle* h, const void* qkv_host
                                              void* o_host, int batch, void* cuda_stream) {
     if (h == nullptr) return QDA_ERR_INVALID_ARG;
     int rc = check_call(h, qkv_host, q_norm_w, k_norm_w, seq_lens_host, positions_host, block_table_host,
-                        block_table_stride, k_cache, v_cache, num_pages, h->st_o, batch);
+                        block_table_stride, k_cache, v_cache, num_pages, h->st_o[0], batch);
     if (rc != QDA_OK) return rc;
     if (o_host == nullptr || block_table_stride > h->cfg.max_pages_per_seq) return QDA_ERR_INVALID_ARG;
     DeviceGuard guard(h->device);
     if (!guard.ok()) return QDA_ERR_CUDA;
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     const size_t B = (size_t)batch;
+    // Alternate calls use alternate staging sets, so this call's stage-in
+    // may run while the previous call's attention still reads its own set.
+    const int k = (int)(h->host_calls++ & 1u);
     // Inputs in page-locked host memory that the device can address are
     // brought over by one stage-in launch; any other host memory by a copy
     // of its own. o in such memory is written by the attention kernel where
@@ -350,19 +398,19 @@ int qwen3_decode_attn_append_and_attend_host(qda_handle* h, const void* qkv_host
         }
         return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, st) == cudaSuccess;
     };
-    const bool ok = bring(qkv_host, h->st_qkv, B * qkv_elems(h->cfg.num_q_heads) * sizeof(uint16_t)) &&
-                    bring(seq_lens_host, h->st_seq_lens, B * sizeof(int32_t)) &&
-                    bring(block_table_host, h->st_block_table, B * (size_t)block_table_stride * sizeof(int32_t)) &&
-                    (positions_host == nullptr || bring(positions_host, h->st_positions, B * sizeof(int32_t)));
+    const bool ok = bring(qkv_host, h->st_qkv[k], B * qkv_elems(h->cfg.num_q_heads) * sizeof(uint16_t)) &&
+                    bring(seq_lens_host, h->st_seq_lens[k], B * sizeof(int32_t)) &&
+                    bring(block_table_host, h->st_block_table[k], B * (size_t)block_table_stride * sizeof(int32_t)) &&
+                    (positions_host == nullptr || bring(positions_host, h->st_positions[k], B * sizeof(int32_t)));
     if (!ok || qda::launch_stage_in(sp, 2 * h->grid, st) != cudaSuccess) return QDA_ERR_CUDA;
     void* o_dev = nullptr;
     const bool o_mapped = mapped_host(o_host, &o_dev) && aligned(o_dev, 16);
-    const qda::Params p = make_params(h, h->st_qkv, q_norm_w, k_norm_w, h->st_seq_lens,
-                                      positions_host != nullptr ? h->st_positions : nullptr, h->st_block_table,
-                                      block_table_stride, k_cache, v_cache, num_pages, o_mapped ? o_dev : h->st_o,
+    const qda::Params p = make_params(h, h->st_qkv[k], q_norm_w, k_norm_w, h->st_seq_lens[k],
+                                      positions_host != nullptr ? h->st_positions[k] : nullptr, h->st_block_table[k],
+                                      block_table_stride, k_cache, v_cache, num_pages, o_mapped ? o_dev : h->st_o[k],
                                       batch);
     if (launch_step(h, p, st) != cudaSuccess) return QDA_ERR_CUDA;
-    if (!o_mapped && cudaMemcpyAsync(o_host, h->st_o, B * (size_t)h->cfg.num_q_heads * qda::kHeadDim * sizeof(uint16_t),
+    if (!o_mapped && cudaMemcpyAsync(o_host, h->st_o[k], B * (size_t)h->cfg.num_q_heads * qda::kHeadDim * sizeof(uint16_t),
                                      cudaMemcpyDeviceToHost, st) != cudaSuccess)
         return QDA_ERR_CUDA;
     return QDA_OK;

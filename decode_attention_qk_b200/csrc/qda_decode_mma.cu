@@ -34,14 +34,14 @@
 //
 // Split sequences. The work split is the 16-head kernel's (equal page ranges
 // per CTA, scratch slot g + b per piece). A piece that covers its whole
-// sequence writes o; a piece of a split sequence writes its partial, and a
-// second launch (one CTA per sequence and kv head, one warp per query row)
-// combines them with the log-sum-exp rule (Supported models, "Facts proved
-// about the specs": flashAttn_eq, softmax_shift), spreading long merges over
-// many SMs. Both launches are programmatic dependent launches: the combine
-// launch starts while the attention launch ends, and the attention launch
-// while the previous step's last launch ends; each waits for its predecessor
-// to complete before it touches global memory.
+// sequence writes o; a piece of a split sequence writes its partial and
+// counts itself on the (sequence, kv head) counter with an acquiring atomic;
+// the warp whose piece arrives last merges all the pieces' partials with the
+// log-sum-exp rule (Supported models, "Facts proved about the specs":
+// flashAttn_eq, softmax_shift), reading them in slot order from L2, writes o
+// and resets the counter. One launch per call, a programmatic dependent
+// launch: it may start while the previous launch on the stream ends, and it
+// waits for that launch to complete before it touches global memory.
 #include <cuda_bf16.h>
 #include <cstdint>
 
@@ -72,18 +72,60 @@ struct Layout {
     static constexpr bool kDirectQkv = kSlotBytes > 24576;
     static constexpr int kStages = 3;
     static constexpr int kSmemQkv = kStages * kStageBytes;
-    static constexpr int kSmemSeg = kSmemQkv + (kDirectQkv ? 0 : kSlotBytes);   // int [kMaxBatch + 4]
+    // wide instances: the new tokens' k words, [warp][token][64] (formed when a sequence starts)
+    static constexpr int kSmemNewK = kSmemQkv + (kDirectQkv ? 0 : kSlotBytes);
+    static constexpr int kNewKBytes = (kRows > 8) ? kConsumerWarps * T * 64 * 4 : 0;
+    static constexpr int kSmemSeg = kSmemNewK + kNewKBytes;                   // int [kMaxBatch + 4]
     static constexpr int kSmemLens = kSmemSeg + (kMaxBatch + 4) * 4;        // int [kMaxBatch]
     static constexpr int kSmemInvFreq = kSmemLens + kMaxBatch * 4;          // double [64]
     static constexpr int kSmemGains = kSmemInvFreq + 64 * 8;                // bf16 [2][128]
     static constexpr int kSmemMeta = kSmemGains + 2 * kHeadDim * 2;         // StageMeta [kStages] + qkv position
     static constexpr int kSmemBars = kSmemMeta + (kStages + 1) * 16;        // full, empty, qkv_full, qkv_empty, never
-    static constexpr int kSmemFlags = kSmemBars + (2 * kStages + 3) * 8;
+    static constexpr int kSmemMergeBars = kSmemBars + (2 * kStages + 3) * 8; // [8] merge copies, done
+    static constexpr int kSmemFlags = kSmemMergeBars + (kConsumerWarps + 1) * 8;
+    // Split pieces' partials, kv head major: row r of kv head j in scratch slot
+    // `slot` is row ((j * (grid + batch) + slot) * kRowPitch + r), so kv head
+    // j's rows of consecutive slots are contiguous; the pitch is even so that
+    // the (max, sum) pairs of a slot start on a 16-byte boundary.
+    static constexpr int kRowPitch = (kRows + 1) / 2 * 2;
+    // Merging: warp j uses its 1/8 of the idle ring; a batch of pieces is one
+    // bulk copy of their rows and one of their (max, sum) pairs.
+    static constexpr int kMergeRegion = kStages * kStageBytes / kConsumerWarps / 16 * 16;
+    static constexpr int kMergeBatch = kMergeRegion / (kRowPitch * (kHeadDim * 4 + 8));
+    static constexpr int kMergeMlOff = kMergeBatch * kRowPitch * kHeadDim * 4;
     static constexpr int kSmemTotal = kSmemFlags + 16;
-    static_assert(kRows <= 8, "at most 8 query rows per kv head");
+    // Up to 8 query rows per kv head, q and the probabilities enter the tensor
+    // cores as two bf16 terms (value and remainder, rows r and r + 8 of the
+    // A operand); with 9 to 16 rows ("wide"), the 16 rows are 16 query rows
+    // and q and the probabilities enter as bf16.
+    static constexpr bool kWide = kRows > 8;
+    static_assert(kRows <= 16, "at most 16 query rows per kv head");
+    static_assert(!kWide || kDirectQkv, "wide instances read their qkv rows from global memory");
     static_assert(kSmemQkv % 16 == 0 && kSmemInvFreq % 8 == 0 && kSmemBars % 8 == 0, "alignment");
+    static_assert(kMergeBatch >= 1 && kMergeBatch <= 32 && kRowPitch <= 16, "merge batches");
     static_assert(kSmemTotal <= 227 * 1024, "fits one CTA per SM");
 };
+
+// Row of a split piece's partial: query row r (new token r / G, head
+// G*j + r % G) of kv head j in scratch slot `slot` (see Layout::kRowPitch).
+template <int G, int T>
+__device__ __forceinline__ size_t part_row(const Params& p, int j, int slot, int r) {
+    const size_t stride = (size_t)gridDim.x + (size_t)p.batch;
+    return ((size_t)j * stride + (size_t)slot) * Layout<G, T>::kRowPitch + (size_t)r;
+}
+
+// Row of qkv (and of o) holding new token u of sequence b: a call may cover
+// tokens [tok_offset, tok_offset + T) of blocks of tok_stride tokens per
+// sequence (a long block of new tokens runs as several such launches).
+__device__ __forceinline__ size_t token_row(const Params& p, int b, int u) {
+    return (size_t)b * p.tok_stride + p.tok_offset + u;
+}
+
+// RoPE position of the first new token of this launch for sequence b of
+// (trimmed) length L with T new tokens in this launch.
+__device__ __forceinline__ int first_position(const Params& p, int b, int L, int T) {
+    return p.positions != nullptr ? __ldg(p.positions + b) + p.tok_offset : L - T;
+}
 
 // Prefetch `bytes` (a multiple of 16, 16-byte aligned) from global memory to L2.
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
@@ -92,6 +134,7 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes
 
 struct Shared {
     uint8_t* stages;
+    uint32_t* new_k;      // wide instances: [warp][token][64] k words of the new tokens
     uint8_t* qkv;         // the current sequence piece's T qkv rows
     int* seg;
     int* lens;
@@ -104,6 +147,8 @@ struct Shared {
     uint64_t* qkv_full;
     uint64_t* qkv_empty;
     uint64_t* never_bar;
+    uint64_t* merge_bar;  // [kConsumerWarps]: the merge copies of warp j
+    uint64_t* done_bar;   // every consumer warp is past its last page
     volatile int* abort_flag;
 };
 
@@ -132,7 +177,7 @@ __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, i
             rows = min(kPage, max(0, (s.lens[b] - T) - kPage * i));
             if (gp == start || i == 0) {
                 qkv_b = b;
-                pos = p.positions != nullptr ? __ldg(p.positions + b) : s.lens[b] - T;
+                pos = first_position(p, b, s.lens[b], T);
             }
         }
         const int n = min(32, count - base);
@@ -146,7 +191,7 @@ __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, i
             if (lane == 0) {
                 if (Lay::kDirectQkv && seq_qkv >= 0) {
                     // the consumers read these rows from global memory: have them in L2 first
-                    bulk_prefetch_l2(p.qkv + (size_t)seq_qkv * T * Lay::kQkvW, (uint32_t)Lay::kSlotBytes);
+                    bulk_prefetch_l2(p.qkv + token_row(p, seq_qkv, 0) * Lay::kQkvW, (uint32_t)Lay::kSlotBytes);
                 } else if (seq_qkv >= 0) {
                     // the qkv slot frees once every consumer has formed q from it
                     ok = mbar_try_wait(s.qkv_empty, qphase ^ 1u) ||
@@ -154,7 +199,7 @@ __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, i
                     if (ok) {
                         *s.qkv_pos = seq_pos;
                         mbar_arrive_expect_tx(s.qkv_full, (uint32_t)Lay::kSlotBytes);
-                        bulk_g2s(s.qkv, p.qkv + (size_t)seq_qkv * T * Lay::kQkvW, (uint32_t)Lay::kSlotBytes,
+                        bulk_g2s(s.qkv, p.qkv + token_row(p, seq_qkv, 0) * Lay::kQkvW, (uint32_t)Lay::kSlotBytes,
                                  s.qkv_full);
                         qarmed = true;
                         qarmed_parity = qphase;
@@ -500,31 +545,531 @@ __device__ __forceinline__ void consume_page(const Params& p, const Shared& s, i
 // else this piece's partial at scratch slot blockIdx.x + b, row t*Hq + head of
 // the slot's kPartRows.
 template <int G, int T>
-__device__ __forceinline__ void finish_piece(const Params& p, const Shared& s, int b, int j, int lane, int per_cta,
+__device__ __forceinline__ bool finish_piece(const Params& p, const Shared& s, int b, int j, int lane, int per_cta,
                                              State<T>& st) {
     using Lay = Layout<G, T>;
     const int r = lane >> 2, t = lane & 3;
     float l = st.lsum;
     l += __shfl_xor_sync(kFull, l, 1);
     l += __shfl_xor_sync(kFull, l, 2);
-    if (r >= Lay::kRows) return;
-    const int tt = r / G;
-    const int head = G * j + r % G;
     const int part_first = s.seg[b] / per_cta;
     const int part_last = (s.seg[b + 1] - 1) / per_cta;
+    if (r >= Lay::kRows) return part_first != part_last;
+    const int tt = r / G;
+    const int head = G * j + r % G;
     if (part_first == part_last) {
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        uint32_t* dst = reinterpret_cast<uint32_t*>(p.o + (((size_t)b * T + tt) * Lay::kHq + head) * kHeadDim);
+        uint32_t* dst = reinterpret_cast<uint32_t*>(p.o + (token_row(p, b, tt) * Lay::kHq + head) * kHeadDim);
 #pragma unroll
         for (int n = 0; n < 16; ++n)
             dst[4 * n + t] = pack_bf2((st.o[n][0] + st.o[n][2]) * inv, (st.o[n][1] + st.o[n][3]) * inv);
-        return;
+        return false;
     }
-    const size_t prow = (size_t)(blockIdx.x + b) * kPartRows + tt * Lay::kHq + head;
+    const size_t prow = part_row<G, T>(p, j, (int)blockIdx.x + b, r);
     float2* pa = reinterpret_cast<float2*>(p.part_acc + prow * kHeadDim);
 #pragma unroll
     for (int n = 0; n < 16; ++n) __stcg(pa + 4 * n + t, make_float2(st.o[n][0] + st.o[n][2], st.o[n][1] + st.o[n][3]));
     if (t == 0) __stcg(p.part_ml + prow, make_float2(st.m, l));
+    return true;
+}
+
+// Bounded wait of a whole warp on `bar`; on expiry records QDA_ERR_TIMEOUT and
+// sets the CTA's abort flag.
+__device__ __forceinline__ bool warp_wait(const Params& p, const Shared& s, uint64_t* bar, uint32_t phase, int lane) {
+    bool ok = mbar_try_wait(bar, phase);
+    if (__all_sync(kFull, ok)) return true;
+    ok = ok || mbar_wait(bar, phase, p.timeout_ns, s.abort_flag);
+    ok = __all_sync(kFull, ok || mbar_try_wait(bar, phase));
+    if (!ok && lane == 0) {
+        *s.abort_flag = 1;
+        record_error(p.status, QDA_ERR_TIMEOUT);
+    }
+    return ok;
+}
+
+// Merge the partials of every piece of split sequence b for the query rows of
+// kv head j (this warp's piece was the last to arrive) and write o:
+// o = sum_t 2^(m_t - M) acc_t / sum_t 2^(m_t - M) l_t, M the running maximum
+// (log-sum-exp rule; Supported models, "Facts proved about the specs":
+// flashAttn_eq, softmax_shift). Pieces come in batches through this warp's
+// 1/8 of the idle ring: one bulk copy of their rows (contiguous, kv head
+// major) and one of their (max, sum) pairs, issued by the lane whose
+// acquiring increment completed the count; the batches are merged in slot
+// order with a rescale between them. Lane l handles dims 4l..4l+3 of every
+// row. Returns false when a wait ran out.
+template <int G, int T>
+__device__ __noinline__ bool merge_sequence(const Params& p, const Shared& s, int b, int j, int lane, int issuer,
+                                            int per_cta, uint32_t& mphase) {
+    using Lay = Layout<G, T>;
+    constexpr int R = Lay::kRows;
+    constexpr int RP = Lay::kRowPitch;
+    const int first = s.seg[b] / per_cta;
+    const int n = (s.seg[b + 1] - 1) / per_cta - first + 1;
+    uint8_t* region = s.stages + j * Lay::kMergeRegion;
+    uint64_t* bar = &s.merge_bar[j];
+    float M[R], L[R];
+    float4 A[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        M[r] = -INFINITY;
+        L[r] = 0.f;
+        A[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int t0 = 0; t0 < n; t0 += Lay::kMergeBatch) {
+        const int nb = min(Lay::kMergeBatch, n - t0);
+        // earlier reads of the region come before the copies that overwrite it
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == issuer) {
+            mbar_arrive_expect_tx(bar, (uint32_t)nb * RP * (kHeadDim * 4 + 8));
+            const size_t row = part_row<G, T>(p, j, first + b + t0, 0);
+            bulk_g2s(region, p.part_acc + row * kHeadDim, (uint32_t)nb * RP * kHeadDim * 4, bar);
+            bulk_g2s(region + Lay::kMergeMlOff, p.part_ml + row, (uint32_t)nb * RP * 8, bar);
+        }
+        if (!warp_wait(p, s, bar, mphase, lane)) {
+            // the copies may still be landing: wait once more (bounded) before leaving
+            if (lane == 0) (void)mbar_wait(bar, mphase, p.timeout_ns, nullptr);
+            __syncwarp();
+            return false;
+        }
+        mphase ^= 1u;
+        const float2* ml = reinterpret_cast<const float2*>(region + Lay::kMergeMlOff);   // [piece][RP]
+        const float4* acc = reinterpret_cast<const float4*>(region);                     // [piece][RP][32]
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            float bm = -INFINITY;
+            for (int t = 0; t < nb; ++t) bm = fmaxf(bm, ml[t * RP + r].x);
+            const float nM = fmaxf(M[r], bm);
+            // what the earlier batches summed, rescaled to the new maximum (nothing on the first)
+            const float sc = M[r] == -INFINITY ? 0.f : exp2_approx(M[r] - nM);
+            L[r] *= sc;
+            A[r].x *= sc;
+            A[r].y *= sc;
+            A[r].z *= sc;
+            A[r].w *= sc;
+            for (int t = 0; t < nb; ++t) {
+                const float2 v = ml[t * RP + r];
+                // a piece whose pages were all skipped has max -inf and weight 0
+                const float w = v.x == -INFINITY ? 0.f : exp2_approx(v.x - nM);
+                L[r] = fmaf(w, v.y, L[r]);
+                const float4 x = acc[(t * RP + r) * 32 + lane];
+                A[r].x = fmaf(w, x.x, A[r].x);
+                A[r].y = fmaf(w, x.y, A[r].y);
+                A[r].z = fmaf(w, x.z, A[r].z);
+                A[r].w = fmaf(w, x.w, A[r].w);
+            }
+            M[r] = nM;
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const float inv = L[r] > 0.f ? 1.f / L[r] : 0.f;
+        const int tt = r / G, head = G * j + r % G;
+        uint2 out;
+        out.x = pack_bf2(A[r].x * inv, A[r].y * inv);
+        out.y = pack_bf2(A[r].z * inv, A[r].w * inv);
+        reinterpret_cast<uint2*>(p.o + (token_row(p, b, tt) * Lay::kHq + head) * kHeadDim)[lane] = out;
+    }
+    if (lane == 0) p.counters[b * kNumKvHeads + j] = 0;   // ready for the next call
+    return true;
+}
+
+// End of a consumer warp's run: its split pieces' partials are stored (no
+// fence yet). Count them as done (lane 0: pending0, lane 1: pending1, with
+// acquiring atomics after one fence); the warp holding the last piece of a
+// sequence merges it through the ring, which every consumer warp has left by
+// then.
+template <int G, int T>
+__device__ __forceinline__ void arrive_pending(const Params& p, const Shared& s, int j, int lane, int per_cta,
+                                               int pending0, int pending1) {
+    __threadfence();   // this warp's partial stores before its arrivals
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    const int npend = pending1 >= 0 ? 2 : 1;
+    const int mine = lane == 0 ? pending0 : pending1;
+    int prev = -1, need = 0;
+    if (lane < npend) {
+        need = (s.seg[mine + 1] - 1) / per_cta - s.seg[mine] / per_cta;
+        // acquire: the last to arrive sees every other piece's released partial
+        prev = atomic_add_acquire(p.counters + mine * kNumKvHeads + j, 1);
+    }
+    const bool last0 = __shfl_sync(kFull, prev == need, 0);
+    const bool last1 = __shfl_sync(kFull, prev == need, 1) && npend == 2;
+    if (!last0 && !last1) return;
+    // the other pieces' partials are read through the async proxy by bulk
+    // copies, issued by the lane whose acquiring increment found the count complete
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    if (!warp_wait(p, s, s.done_bar, 0u, lane)) return;
+    uint32_t mphase = 0;
+    if (last0 && !merge_sequence<G, T>(p, s, pending0, j, lane, 0, per_cta, mphase)) return;
+    if (last1) (void)merge_sequence<G, T>(p, s, pending1, j, lane, 1, per_cta, mphase);
+}
+
+// ---------------------------------------------------------------------------
+// Wide instances: 9 to 16 query rows per kv head, one row per accumulator row.
+
+struct WState {
+    uint32_t qa[8][4];    // A fragments of q per 16-dim step: rows g (regs 0, 2) and g + 8 (regs 1, 3), bf16
+    float o[16][4];       // value accumulators: 16 tiles of 8 dims, rows g (0, 1) and g + 8 (2, 3)
+    float m[2];           // running max of rows g and g + 8 (log2 units)
+    float lsum[2];        // partial softmax sums of this lane's tokens, rows g and g + 8
+};
+
+// The new tokens' k for kv head j, normed and rotated in double and rounded
+// once to bf16, into this warp's words of s.new_k. Lane l handles dims 2l,
+// 2l+1 (word l) and 64+2l, 65+2l (word 32+l); the angle of token u is token
+// 0's rotated by the step u times (error ~u ulp of double, far below k's bf16
+// rounding).
+template <int G, int T>
+__device__ __forceinline__ void form_new_k(const Params& p, const Shared& s, const uint8_t* rows, int pos0, int j,
+                                           int lane) {
+    using Lay = Layout<G, T>;
+    const uint32_t* gk = reinterpret_cast<const uint32_t*>(s.gains + kHeadDim);
+    const uint32_t wk_lo = gk[lane], wk_hi = gk[32 + lane];
+    double sn0, cs0, sn1, cs1, ds0, dc0, ds1, dc1;
+    sincos((double)pos0 * s.inv_freq[2 * lane], &sn0, &cs0);
+    sincos((double)pos0 * s.inv_freq[2 * lane + 1], &sn1, &cs1);
+    sincos(s.inv_freq[2 * lane], &ds0, &dc0);
+    sincos(s.inv_freq[2 * lane + 1], &ds1, &dc1);
+    uint32_t* dst = s.new_k + (size_t)j * T * 64;
+    // every token's words first (one round trip to L2), then the arithmetic
+    uint32_t xlo[T], xhi[T];
+#pragma unroll
+    for (int u = 0; u < T; ++u) {
+        const uint32_t* xk =
+            reinterpret_cast<const uint32_t*>(rows + u * Lay::kQkvBytes + (Lay::kHq + j) * (kHeadDim * 2));
+        xlo[u] = xk[lane];
+        xhi[u] = xk[32 + lane];
+    }
+#pragma unroll
+    for (int u = 0; u < T; ++u) {
+        double a0 = bf_to_d(xlo[u] & 0xFFFFu), a1 = bf_to_d(xlo[u] >> 16);
+        double b0 = bf_to_d(xhi[u] & 0xFFFFu), b1 = bf_to_d(xhi[u] >> 16);
+        const double inv_rr = 1.0 / sqrt(warp_sum(a0 * a0 + a1 * a1 + b0 * b0 + b1 * b1) / 128.0 + p.rms_eps);
+        a0 = a0 * inv_rr * bf_to_d(wk_lo & 0xFFFFu);
+        a1 = a1 * inv_rr * bf_to_d(wk_lo >> 16);
+        b0 = b0 * inv_rr * bf_to_d(wk_hi & 0xFFFFu);
+        b1 = b1 * inv_rr * bf_to_d(wk_hi >> 16);
+        const double ra0 = a0 * cs0 - b0 * sn0, rb0 = b0 * cs0 + a0 * sn0;
+        const double ra1 = a1 * cs1 - b1 * sn1, rb1 = b1 * cs1 + a1 * sn1;
+        dst[u * 64 + lane] = d_to_bf(ra0) | (d_to_bf(ra1) << 16);
+        dst[u * 64 + 32 + lane] = d_to_bf(rb0) | (d_to_bf(rb1) << 16);
+        const double c0n = cs0 * dc0 - sn0 * ds0, s0n = sn0 * dc0 + cs0 * ds0;   // one position on
+        const double c1n = cs1 * dc1 - sn1 * ds1, s1n = sn1 * dc1 + cs1 * ds1;
+        cs0 = c0n; sn0 = s0n; cs1 = c1n; sn1 = s1n;
+    }
+    __syncwarp();
+}
+
+// Start a sequence piece: q of rows g and g + 8 (g = lane/4; row r is new
+// token r / G, head G*j + r % G) at dims 8m + 2t, 8m + 2t + 1 (t = lane%4),
+// normed and rotated in float as in begin_sequence, then rounded to bf16.
+template <int G, int T>
+__device__ __forceinline__ void begin_sequence_wide(const Params& p, const Shared& s, const uint8_t* rows, int pos0,
+                                                    int j, int lane, bool appends, WState& st) {
+    using Lay = Layout<G, T>;
+    if (appends) form_new_k<G, T>(p, s, rows, pos0, j, lane);
+    constexpr double kTwoPiHi = 6.2831853069365025;      // 2*pi rounded to 32 significant bits
+    constexpr double kTwoPiLo = 2.430840202602477e-10;   // 2*pi - kTwoPiHi
+    constexpr double kInvTwoPi = 0.15915494309189535;
+    const int g = lane >> 2, t = lane & 3;
+    float cf[T][2], sf[T][2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const double ang = (double)pos0 * s.inv_freq[2 * lane + e];
+        const double n = rint(ang * kInvTwoPi);
+        sincosf((float)fma(-n, kTwoPiLo, fma(-n, kTwoPiHi, ang)), &sf[0][e], &cf[0][e]);
+        float ds, dc;
+        sincosf((float)s.inv_freq[2 * lane + e], &ds, &dc);
+#pragma unroll
+        for (int u = 1; u < T; ++u) {   // later tokens: rotate by the step f
+            cf[u][e] = fmaf(cf[u - 1][e], dc, -sf[u - 1][e] * ds);
+            sf[u][e] = fmaf(sf[u - 1][e], dc, cf[u - 1][e] * ds);
+        }
+    }
+    const uint32_t* gq = reinterpret_cast<const uint32_t*>(s.gains);
+    const float scale = (float)kQScale;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int r = g + 8 * h;
+        const bool active = r < Lay::kRows;
+        const int tt = active ? r / G : 0;
+        const int head = G * j + (active ? r % G : 0);
+        const uint32_t* xq = reinterpret_cast<const uint32_t*>(rows + tt * Lay::kQkvBytes + head * (kHeadDim * 2));
+        uint32_t xw[16];
+        float ss = 0.f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            xw[m] = xq[4 * m + t];
+            ss = fmaf(bf_lo(xw[m]), bf_lo(xw[m]), fmaf(bf_hi(xw[m]), bf_hi(xw[m]), ss));
+        }
+        ss += __shfl_xor_sync(kFull, ss, 1);
+        ss += __shfl_xor_sync(kFull, ss, 2);
+        const float inv_r = rsqrtf(ss * (1.f / 128.f) + (float)p.rms_eps);
+#pragma unroll
+        for (int mp = 0; mp < 8; ++mp) {
+            float qa[2], qb[2];
+            const uint32_t wlo = gq[4 * mp + t], whi = gq[32 + 4 * mp + t];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float cs = 0.f, sn = 0.f;
+#pragma unroll
+                for (int u = 0; u < T; ++u) {   // the angle of pair 8*mp + 2t + e at this row's token
+                    const float cu = __shfl_sync(kFull, cf[u][e], 4 * mp + t);
+                    const float su = __shfl_sync(kFull, sf[u][e], 4 * mp + t);
+                    cs = (u == tt) ? cu : cs;
+                    sn = (u == tt) ? su : sn;
+                }
+                const float ya = (e ? bf_hi(xw[mp]) : bf_lo(xw[mp])) * inv_r * (e ? bf_hi(wlo) : bf_lo(wlo));
+                const float yb = (e ? bf_hi(xw[mp + 8]) : bf_lo(xw[mp + 8])) * inv_r * (e ? bf_hi(whi) : bf_lo(whi));
+                qa[e] = fmaf(ya, cs, -yb * sn) * scale;   // dim 8*mp + 2t + e
+                qb[e] = fmaf(yb, cs, ya * sn) * scale;    // dim 64 + 8*mp + 2t + e
+            }
+            const int part = ((mp & 1) ? 2 : 0) + h;   // dims 16s + 2t (+1) or 16s + 8 + 2t (+1); row g or g + 8
+            st.qa[mp >> 1][part] = active ? pack_bf2(qa[0], qa[1]) : 0u;
+            st.qa[4 + (mp >> 1)][part] = active ? pack_bf2(qb[0], qb[1]) : 0u;
+        }
+    }
+#pragma unroll
+    for (int n = 0; n < 16; ++n)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) st.o[n][k] = 0.f;
+    st.m[0] = st.m[1] = -INFINITY;
+    st.lsum[0] = st.lsum[1] = 0.f;
+}
+
+// Scores, online softmax and value accumulation over one staged page for rows
+// g and g + 8, which see page tokens up to lim0 and lim1 (unless kFullPage).
+// The probabilities enter the value product as bf16, and the sums add the
+// same rounded values, so o stays a convex combination of the v rows.
+template <int G, int T, bool kFullPage>
+__device__ __forceinline__ void attend_page_wide(const uint8_t* stage, int lim0, int lim1, int j, int lane,
+                                                 WState& st) {
+    using Lay = Layout<G, T>;
+    const int g = lane >> 2, t = lane & 3;
+    const bool act0 = g < Lay::kRows, act1 = g + 8 < Lay::kRows;
+    const uint32_t kaddr = smem_addr(stage + kStageK) + j * (kHeadDim * 2) +
+                           ((lane & 7) + ((lane >> 4) << 3)) * kRowPitch + ((lane >> 3) & 1) * 16;
+    float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kaddr + s * 32, b0, b1, b2, b3);
+        mma_bf16_16816(c0, st.qa[s], b0, b1);
+        mma_bf16_16816(c1, st.qa[s], b2, b3);
+    }
+    // rows g and g + 8 at page tokens 2t, 2t+1, 8+2t, 9+2t
+    float s0[4] = {c0[0], c0[1], c1[0], c1[1]};
+    float s1[4] = {c0[2], c0[3], c1[2], c1[3]};
+    if (!kFullPage) {
+        const int tok[4] = {2 * t, 2 * t + 1, 8 + 2 * t, 9 + 2 * t};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            s0[i] = tok[i] <= lim0 ? s0[i] : -INFINITY;
+            s1[i] = tok[i] <= lim1 ? s1[i] : -INFINITY;
+        }
+    }
+    float mx0 = fmaxf(fmaxf(s0[0], s0[1]), fmaxf(s0[2], s0[3]));
+    float mx1 = fmaxf(fmaxf(s1[0], s1[1]), fmaxf(s1[2], s1[3]));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 2));
+    const bool grow0 = mx0 > st.m[0] + kRescaleThreshold;
+    const bool grow1 = mx1 > st.m[1] + kRescaleThreshold;
+    if (__any_sync(kFull, grow0 || grow1)) {
+        const float n0 = grow0 ? mx0 : st.m[0], n1 = grow1 ? mx1 : st.m[1];
+        const float a0 = grow0 ? exp2_approx(st.m[0] - n0) : 1.f;   // exp2(-inf) = 0 on the first page
+        const float a1 = grow1 ? exp2_approx(st.m[1] - n1) : 1.f;
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+            st.o[n][0] *= a0;
+            st.o[n][1] *= a0;
+            st.o[n][2] *= a1;
+            st.o[n][3] *= a1;
+        }
+        st.lsum[0] *= a0;
+        st.lsum[1] *= a1;
+        st.m[0] = n0;
+        st.m[1] = n1;
+    }
+    float p0[4], p1[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        p0[i] = (s0[i] == -INFINITY || !act0) ? 0.f : exp2_approx(s0[i] - st.m[0]);
+        p1[i] = (s1[i] == -INFINITY || !act1) ? 0.f : exp2_approx(s1[i] - st.m[1]);
+    }
+    uint32_t pa[4];
+    pa[0] = pack_bf2(p0[0], p0[1]);   // row g, tokens 2t, 2t+1
+    pa[1] = pack_bf2(p1[0], p1[1]);   // row g + 8
+    pa[2] = pack_bf2(p0[2], p0[3]);   // row g, tokens 8+2t, 9+2t
+    pa[3] = pack_bf2(p1[2], p1[3]);   // row g + 8
+    st.lsum[0] += (bf_lo(pa[0]) + bf_hi(pa[0])) + (bf_lo(pa[2]) + bf_hi(pa[2]));
+    st.lsum[1] += (bf_lo(pa[1]) + bf_hi(pa[1])) + (bf_lo(pa[3]) + bf_hi(pa[3]));
+    const uint32_t vaddr = smem_addr(stage + kStageV) + j * (kHeadDim * 2) +
+                           ((lane & 7) + (((lane >> 3) & 1) << 3)) * kRowPitch + ((lane >> 4) & 1) * 16;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_trans(vaddr + u * 32, b0, b1, b2, b3);
+        mma_bf16_16816(st.o[2 * u], pa, b0, b1);
+        mma_bf16_16816(st.o[2 * u + 1], pa, b2, b3);
+    }
+}
+
+template <int G, int T>
+__device__ __forceinline__ void consume_page_wide(const Params& p, const Shared& s, int slot, int i, int L, int j,
+                                                  int lane, const uint8_t* rows, WState& st) {
+    using Lay = Layout<G, T>;
+    uint8_t* stage = s.stages + slot * kStageBytes;
+    const int first_new = L - T;                    // slot of the first new token
+    const int ntok = min(kPage, L - kPage * i);     // rows of this page inside the sequence
+    if (s.meta[slot].bad == 0) {
+        if (kPage * i + kPage > first_new) {
+            // the new tokens on this page: k (formed when the sequence started)
+            // and v bits, to the cache and into the staged page
+            const int page = s.meta[slot].page;
+            const int u_lo = max(0, kPage * i - first_new), u_hi = min(T, kPage * i + kPage - first_new);
+            const uint32_t* nk = s.new_k + (size_t)j * T * 64;
+            // the v words of every token on the page first (one round trip to L2)
+            uint32_t vw_lo[T], vw_hi[T];
+#pragma unroll
+            for (int u = 0; u < T; ++u) {
+                if (u < u_lo || u >= u_hi) continue;
+                const uint32_t* xv = reinterpret_cast<const uint32_t*>(
+                    rows + u * Lay::kQkvBytes + (Lay::kHq + kNumKvHeads + j) * (kHeadDim * 2));
+                vw_lo[u] = xv[lane];
+                vw_hi[u] = xv[32 + lane];
+            }
+#pragma unroll
+            for (int u = 0; u < T; ++u) {
+                if (u < u_lo || u >= u_hi) continue;
+                const uint32_t k_lo = nk[u * 64 + lane], k_hi = nk[u * 64 + 32 + lane];
+                const uint32_t v_lo = vw_lo[u], v_hi = vw_hi[u];
+                const int r = first_new + u - kPage * i;
+                const size_t off =
+                    (size_t)page * (kPageBytes / 2) + (size_t)r * (kRowBytes / 2) + (size_t)j * kHeadDim;
+                uint32_t* kd = reinterpret_cast<uint32_t*>(p.k_cache + off);
+                uint32_t* vd = reinterpret_cast<uint32_t*>(p.v_cache + off);
+                kd[lane] = k_lo;
+                kd[32 + lane] = k_hi;
+                vd[lane] = v_lo;
+                vd[32 + lane] = v_hi;
+                uint32_t* kr = reinterpret_cast<uint32_t*>(stage + kStageK + r * kRowPitch + j * kHeadDim * 2);
+                uint32_t* vr = reinterpret_cast<uint32_t*>(stage + kStageV + r * kRowPitch + j * kHeadDim * 2);
+                kr[lane] = k_lo;
+                kr[32 + lane] = k_hi;
+                vr[lane] = v_lo;
+                vr[32 + lane] = v_hi;
+            }
+            // rows after the sequence hold stale bytes; a stale NaN would survive a
+            // zero probability in the tensor-core sum, so clear them
+            for (int rr = ntok; rr < kPage; ++rr) {
+                uint32_t* z = reinterpret_cast<uint32_t*>(stage + kStageV + rr * kRowPitch + j * kHeadDim * 2);
+                z[lane] = 0u;
+                z[32 + lane] = 0u;
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+        }
+        const int g = lane >> 2;
+        const int tt0 = g < Lay::kRows ? g / G : 0;
+        const int tt1 = g + 8 < Lay::kRows ? (g + 8) / G : 0;
+        const int lim0 = first_new + tt0 - kPage * i, lim1 = first_new + tt1 - kPage * i;
+        if (first_new - kPage * i >= kPage) attend_page_wide<G, T, true>(stage, lim0, lim1, j, lane, st);
+        else attend_page_wide<G, T, false>(stage, lim0, lim1, j, lane, st);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.empty_bar[slot]);
+}
+
+// End of a sequence piece (wide): o, or the piece's partial, for rows g and g + 8.
+template <int G, int T>
+__device__ __forceinline__ bool finish_piece_wide(const Params& p, const Shared& s, int b, int j, int lane,
+                                                  int per_cta, WState& st) {
+    using Lay = Layout<G, T>;
+    const int g = lane >> 2, t = lane & 3;
+    float l[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        l[h] = st.lsum[h];
+        l[h] += __shfl_xor_sync(kFull, l[h], 1);
+        l[h] += __shfl_xor_sync(kFull, l[h], 2);
+    }
+    const int part_first = s.seg[b] / per_cta;
+    const int part_last = (s.seg[b + 1] - 1) / per_cta;
+    const bool split = part_first != part_last;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int r = g + 8 * h;
+        if (r >= Lay::kRows) continue;
+        const int tt = r / G;
+        const int head = G * j + r % G;
+        if (!split) {
+            const float inv = l[h] > 0.f ? 1.f / l[h] : 0.f;
+            uint32_t* dst = reinterpret_cast<uint32_t*>(p.o + (token_row(p, b, tt) * Lay::kHq + head) * kHeadDim);
+#pragma unroll
+            for (int n = 0; n < 16; ++n) dst[4 * n + t] = pack_bf2(st.o[n][2 * h] * inv, st.o[n][2 * h + 1] * inv);
+        } else {
+            const size_t prow = part_row<G, T>(p, j, (int)blockIdx.x + b, r);
+            float2* pa = reinterpret_cast<float2*>(p.part_acc + prow * kHeadDim);
+#pragma unroll
+            for (int n = 0; n < 16; ++n) __stcg(pa + 4 * n + t, make_float2(st.o[n][2 * h], st.o[n][2 * h + 1]));
+            if (t == 0) __stcg(p.part_ml + prow, make_float2(st.m[h], l[h]));
+        }
+    }
+    return split;
+}
+
+// Consumer warp j of a wide instance: as run_consumer, with the query rows'
+// qkv and the new tokens read from global memory.
+template <int G, int T>
+__device__ __forceinline__ void run_consumer_wide(const Params& p, const Shared& s, int B, int start, int end,
+                                                  int per_cta, int warp, int lane) {
+    using Lay = Layout<G, T>;
+    const int j = warp;
+    WState st;
+    int b = find_seq(s.seg, B, start);
+    int i0 = start - s.seg[b];
+    int slot = 0;
+    uint32_t phase = 0;
+    const int count = end - start;
+    int k = 0;
+    int pending0 = -1, pending1 = -1;   // split pieces whose arrival waits for the end
+    bool aborted = false;
+    while (k < count && !aborted) {
+        const int nb = s.seg[b + 1] - s.seg[b];
+        const int L = s.lens[b];
+        const int n_here = min(nb - i0, count - k);
+        const int pos0 = first_position(p, b, L, T);
+        const uint8_t* rows = reinterpret_cast<const uint8_t*>(p.qkv + token_row(p, b, 0) * Lay::kQkvW);
+        // this CTA appends when it holds a page with one of the new tokens
+        const bool appends = s.seg[b] + (L - T) / kPage < end;
+        begin_sequence_wide<G, T>(p, s, rows, pos0, j, lane, appends, st);
+        for (int u = 0; u < n_here; ++u) {
+            if (!wait_full(p, s, &s.full_bar[slot], phase, lane)) {
+                aborted = true;
+                break;
+            }
+            consume_page_wide<G, T>(p, s, slot, i0 + u, L, j, lane, rows, st);
+            if (++slot == Lay::kStages) {
+                slot = 0;
+                phase ^= 1u;
+            }
+        }
+        if (aborted) break;
+        k += n_here;
+        if (finish_piece_wide<G, T>(p, s, b, j, lane, per_cta, st)) {
+            if (pending0 < 0) pending0 = b;
+            else pending1 = b;
+        }
+        if (k < count) {
+            do { ++b; } while (b < B && s.seg[b + 1] == s.seg[b]);
+            i0 = 0;
+        }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(s.done_bar);   // this warp no longer reads the ring
+    if (!aborted && pending0 >= 0) arrive_pending<G, T>(p, s, j, lane, per_cta, pending0, pending1);
 }
 
 template <int G, int T>
@@ -541,38 +1086,53 @@ __device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, i
     uint32_t phase = 0, qphase = 0;
     const int count = end - start;
     int k = 0;
-    while (k < count) {
+    int pending0 = -1, pending1 = -1;   // split pieces whose arrival waits for the end
+    bool aborted = false;
+    while (k < count && !aborted) {
         const int nb = s.seg[b + 1] - s.seg[b];
         const int L = s.lens[b];
         const int n_here = min(nb - i0, count - k);
         // this CTA appends when it holds a page with one of the new tokens
         const bool appends = s.seg[b] + (L - T) / kPage < end;
         if (Layout<G, T>::kDirectQkv) {
-            const int pos0 = p.positions != nullptr ? __ldg(p.positions + b) : L - T;
-            begin_sequence<G, T>(p, s, reinterpret_cast<const uint8_t*>(p.qkv + (size_t)b * T * Layout<G, T>::kQkvW),
+            const int pos0 = first_position(p, b, L, T);
+            begin_sequence<G, T>(p, s, reinterpret_cast<const uint8_t*>(p.qkv + token_row(p, b, 0) * Layout<G, T>::kQkvW),
                                  pos0, j, lane, appends, st);
         } else {
-            if (!wait_full(p, s, s.qkv_full, qphase, lane)) return;
+            if (!wait_full(p, s, s.qkv_full, qphase, lane)) {
+                aborted = true;
+                break;
+            }
             begin_sequence<G, T>(p, s, s.qkv, *s.qkv_pos, j, lane, appends, st);
             __syncwarp();
             if (lane == 0) mbar_arrive(s.qkv_empty);
             qphase ^= 1u;
         }
         for (int u = 0; u < n_here; ++u) {
-            if (!wait_full(p, s, &s.full_bar[slot], phase, lane)) return;
+            if (!wait_full(p, s, &s.full_bar[slot], phase, lane)) {
+                aborted = true;
+                break;
+            }
             consume_page<G, T>(p, s, slot, i0 + u, L, j, lane, st);
             if (++slot == kStages) {
                 slot = 0;
                 phase ^= 1u;
             }
         }
+        if (aborted) break;
         k += n_here;
-        finish_piece<G, T>(p, s, b, j, lane, per_cta, st);
+        if (finish_piece<G, T>(p, s, b, j, lane, per_cta, st)) {
+            if (pending0 < 0) pending0 = b;
+            else pending1 = b;
+        }
         if (k < count) {
             do { ++b; } while (b < B && s.seg[b + 1] == s.seg[b]);
             i0 = 0;
         }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(s.done_bar);   // this warp no longer reads the ring
+    if (!aborted && pending0 >= 0) arrive_pending<G, T>(p, s, j, lane, per_cta, pending0, pending1);
 }
 
 template <int G, int T>
@@ -585,6 +1145,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
     Shared s;
     s.stages = smem;
     s.qkv = smem + Lay::kSmemQkv;
+    s.new_k = reinterpret_cast<uint32_t*>(smem + Lay::kSmemNewK);
     s.seg = reinterpret_cast<int*>(smem + Lay::kSmemSeg);
     s.lens = reinterpret_cast<int*>(smem + Lay::kSmemLens);
     s.inv_freq = reinterpret_cast<double*>(smem + Lay::kSmemInvFreq);
@@ -596,11 +1157,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
     s.qkv_full = s.empty_bar + kStages;
     s.qkv_empty = s.qkv_full + 1;
     s.never_bar = s.qkv_empty + 1;
+    s.merge_bar = reinterpret_cast<uint64_t*>(smem + Lay::kSmemMergeBars);
+    s.done_bar = s.merge_bar + kConsumerWarps;
     s.abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kSmemFlags);
 
-    // Launched as a programmatic dependent launch: the prologue below touches
-    // no global memory, and griddepcontrol.wait holds until the previous
-    // launch on the stream has completed and its writes are visible.
+    // Launched as a programmatic dependent launch: the next launch may be
+    // scheduled now; the prologue below touches no global memory, and
+    // griddepcontrol.wait holds until the previous launch on the stream has
+    // completed and its writes are visible.
+    pdl_launch_dependents();
     if (threadIdx.x >= 64 && threadIdx.x < 128) {
         const int i = threadIdx.x - 64;
         s.inv_freq[i] = pow(p.rope_theta, -2.0 * i / 128.0);
@@ -613,6 +1178,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
         mbar_init(s.qkv_full, 1);
         mbar_init(s.qkv_empty, kConsumerWarps);
         mbar_init(s.never_bar, 1);
+        for (int k = 0; k < kConsumerWarps; ++k) mbar_init(&s.merge_bar[k], 1);
+        mbar_init(s.done_bar, kConsumerWarps);
         *s.abort_flag = 0;
         s.seg[0] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -621,9 +1188,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
 
     const int B = p.batch;
     for (int b = threadIdx.x; b < B; b += kThreads) {
-        const int L = p.seq_lens[b];
-        const bool ok = L >= T && L <= p.max_seq_len && L <= kPage * p.bt_stride;
+        // the sequence's length counts its whole block of tok_stride new tokens;
+        // this launch sees it without the block's tokens after its own
+        const int L_all = p.seq_lens[b];
+        const bool ok = L_all >= p.tok_stride && L_all <= p.max_seq_len && L_all <= kPage * p.bt_stride;
         if (!ok && blockIdx.x == 0) record_error(p.status, QDA_ERR_BOUNDS);
+        const int L = ok ? L_all - p.len_trim : 0;
         s.lens[b] = L;
         s.seg[b + 1] = ok ? (L + kPage - 1) / kPage : 0;
     }
@@ -656,8 +1226,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
         }
     }
     __syncthreads();
-    if (blockIdx.x == 0)   // page offsets for the combine launch
-        for (int b = threadIdx.x; b <= B; b += kThreads) p.seg[b] = s.seg[b];
 
     const int total = s.seg[B];
     const int per_cta = (total + (int)gridDim.x - 1) / (int)gridDim.x;
@@ -665,74 +1233,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
     const int end = min(start + per_cta, total);
     if (start < end) {
         if (warp == kConsumerWarps) run_producer<G, T>(p, s, B, start, end, lane);
+        else if constexpr (Lay::kWide) run_consumer_wide<G, T>(p, s, B, start, end, per_cta, warp, lane);
         else run_consumer<G, T>(p, s, B, start, end, per_cta, warp, lane);
     }
     if ((p.flags & QDA_FLAG_INJECT_WAIT_TIMEOUT) != 0u && blockIdx.x == 0 && warp == 0) {
         if (!mbar_wait(s.never_bar, 0u, p.timeout_ns, nullptr) && lane == 0) record_error(p.status, QDA_ERR_TIMEOUT);
     }
-    pdl_launch_dependents();
-}
-
-// Combine the partials of one split sequence (blockIdx.x) for the query rows
-// of one kv head (blockIdx.y): warp w handles new token w / G, head
-// G*y + w % G, and lane l its dims 4l..4l+3; o = sum_t 2^(m_t - M) acc_t /
-// sum_t 2^(m_t - M) l_t with M = max_t m_t. Sequences held whole by one CTA
-// were written by the first launch and are skipped.
-template <int G, int T>
-__global__ void __launch_bounds__(32 * G * T, 1) combine_kernel(const Params p, int main_grid) {
-    using Lay = Layout<G, T>;
-    pdl_wait();   // the first launch has finished and its writes are visible
-    pdl_launch_dependents();   // the next step's attention launch may be scheduled
-    const int b = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tt = warp / G;
-    const int h = G * blockIdx.y + warp % G;
-    const int lo = p.seg[b], hi = p.seg[b + 1], total = p.seg[p.batch];
-    if (hi == lo) return;   // a sequence the first launch skipped
-    const int per_cta = (total + main_grid - 1) / main_grid;
-    const int first = lo / per_cta, n = (hi - 1) / per_cta - first + 1;
-    if (n == 1) return;
-    const size_t row0 = (size_t)(first + b) * kPartRows + tt * Lay::kHq + h;   // piece t at row0 + t*kPartRows
-    const float2* ml = p.part_ml + row0;
-    float M = -INFINITY;
-    for (int t = lane; t < n; t += 32) M = fmaxf(M, __ldcg(ml + (size_t)t * kPartRows).x);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
-    const float4* src = reinterpret_cast<const float4*>(p.part_acc + row0 * kHeadDim) + lane;
-    constexpr size_t kSlotStride = (size_t)kPartRows * kHeadDim / 4;   // float4 per scratch slot
-    float Ls = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int t0 = 0; t0 < n; t0 += 32) {
-        float wt = 0.f;
-        if (t0 + lane < n) {
-            const float2 v = __ldcg(ml + (size_t)(t0 + lane) * kPartRows);
-            wt = (v.x == -INFINITY) ? 0.f : exp2_approx(v.x - M);   // a piece whose pages were all skipped
-            Ls = fmaf(wt, v.y, Ls);
-        }
-        const int m = min(32, n - t0);
-        for (int u0 = 0; u0 < m; u0 += 8) {
-            float4 x[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (u0 + u < m) x[u] = __ldcg(src + (size_t)(t0 + u0 + u) * kSlotStride);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const float w = __shfl_sync(kFull, wt, (u0 + u) & 31);
-                if (u0 + u < m) {
-                    acc.x = fmaf(w, x[u].x, acc.x);
-                    acc.y = fmaf(w, x[u].y, acc.y);
-                    acc.z = fmaf(w, x[u].z, acc.z);
-                    acc.w = fmaf(w, x[u].w, acc.w);
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) Ls += __shfl_xor_sync(kFull, Ls, off);
-    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-    uint2 out;
-    out.x = pack_bf2(acc.x * inv, acc.y * inv);
-    out.y = pack_bf2(acc.z * inv, acc.w * inv);
-    reinterpret_cast<uint2*>(p.o + (((size_t)b * T + tt) * Lay::kHq + h) * kHeadDim)[lane] = out;
 }
 
 template <int G, int T>
@@ -753,48 +1259,52 @@ cudaError_t launch_one(const Params& p, int grid, cudaStream_t stream) {
     main.stream = stream;
     main.attrs = attr;
     main.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&main, grouped_attention_kernel<G, T>, p);
-    if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)p.batch, (unsigned)kNumKvHeads, 1);
-    cfg.blockDim = dim3(32 * G * T, 1, 1);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, combine_kernel<G, T>, p, grid);
+    return cudaLaunchKernelEx(&main, grouped_attention_kernel<G, T>, p);
 }
 
 }  // namespace
 
+// The compiled (G, T) instances: every pair with T*G <= 16 query rows per kv
+// head, T = 1 at G = 2 being the 16-head decode kernel's.
+#define QDA_GROUPED_INSTANCES(X) \
+    X(4, 1) X(5, 1) X(8, 1) X(2, 2) X(2, 3) X(2, 4) X(2, 5) X(2, 6) X(2, 7) X(2, 8) \
+    X(4, 2) X(4, 3) X(4, 4) X(5, 2) X(5, 3) X(8, 2)
+
 cudaError_t prepare_grouped() {
-    cudaError_t e = prepare_one<4, 1>();
-    if (e == cudaSuccess) e = prepare_one<5, 1>();
-    if (e == cudaSuccess) e = prepare_one<8, 1>();
-    if (e == cudaSuccess) e = prepare_one<2, 2>();
-    if (e == cudaSuccess) e = prepare_one<2, 3>();
-    if (e == cudaSuccess) e = prepare_one<2, 4>();
-    if (e == cudaSuccess) e = prepare_one<4, 2>();
+    cudaError_t e = cudaSuccess;
+#define QDA_PREPARE(G, T) \
+    if (e == cudaSuccess) e = prepare_one<G, T>();
+    QDA_GROUPED_INSTANCES(QDA_PREPARE)
+#undef QDA_PREPARE
     return e;
+}
+
+int grouped_max_tokens(int num_q_heads) {
+    const int G = num_q_heads / kNumKvHeads;
+    int best = 0;
+#define QDA_MAX_T(GG, TT) \
+    if (G == GG && TT > best) best = TT;
+    QDA_GROUPED_INSTANCES(QDA_MAX_T)
+#undef QDA_MAX_T
+    return G == 2 && best < 1 ? 1 : best;
 }
 
 bool grouped_supported(int num_q_heads, int new_tokens) {
     const int G = num_q_heads / kNumKvHeads;
-    if (new_tokens == 1) return G == 4 || G == 5 || G == 8;
-    return (G == 2 && new_tokens >= 2 && new_tokens <= 4) || (G == 4 && new_tokens == 2);
+#define QDA_MATCH(GG, TT) \
+    if (G == GG && new_tokens == TT) return true;
+    QDA_GROUPED_INSTANCES(QDA_MATCH)
+#undef QDA_MATCH
+    return false;
 }
 
 cudaError_t launch_grouped(const Params& p, int grid, cudaStream_t stream) {
-    switch (p.num_q_heads * 16 + p.new_tokens) {
-        case 32 * 16 + 1: return launch_one<4, 1>(p, grid, stream);
-        case 40 * 16 + 1: return launch_one<5, 1>(p, grid, stream);
-        case 64 * 16 + 1: return launch_one<8, 1>(p, grid, stream);
-        case 16 * 16 + 2: return launch_one<2, 2>(p, grid, stream);
-        case 16 * 16 + 3: return launch_one<2, 3>(p, grid, stream);
-        case 16 * 16 + 4: return launch_one<2, 4>(p, grid, stream);
-        case 32 * 16 + 2: return launch_one<4, 2>(p, grid, stream);
-        default: return cudaErrorInvalidValue;
-    }
+    const int G = p.num_q_heads / kNumKvHeads;
+#define QDA_LAUNCH(GG, TT) \
+    if (G == GG && p.new_tokens == TT) return launch_one<GG, TT>(p, grid, stream);
+    QDA_GROUPED_INSTANCES(QDA_LAUNCH)
+#undef QDA_LAUNCH
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace qda

@@ -9,6 +9,15 @@
 // sequence length before it can start). Here all CTAs issue 16-byte loads at
 // once, so the link's latency is paid about once per launch and the transfer
 // runs at the link's bandwidth.
+//
+// Overlap with the step before. The entry point alternates between two sets
+// of staging buffers, so this launch never writes what the previous step's
+// attention reads. It is then launched as a programmatic dependent of that
+// attention: its CTAs (no shared memory, 256 threads) fit beside the
+// attention's on the same SMs and bring the next step's inputs across the
+// link while the previous step's pages stream. It waits for the previous
+// launch to complete only at its end, so that its own completion (which the
+// next attention launch waits for) still implies the previous step's.
 #include <cstdint>
 
 #include <cuda_runtime.h>
@@ -54,6 +63,9 @@ __global__ void __launch_bounds__(kStageThreads) stage_in_kernel(StageParams sp)
         uint32_t* dst = static_cast<uint32_t*>(rg.dst);
         for (size_t i = done_words + tid; i < words; i += nthreads) dst[i] = src[i];
     }
+    // complete only once the previous launch has (it may still be running when
+    // this one is a programmatic dependent of it)
+    pdl_wait();
 }
 
 }  // namespace
@@ -65,8 +77,17 @@ cudaError_t launch_stage_in(const StageParams& sp, int max_ctas, cudaStream_t st
     // one 16-byte load per thread, up to max_ctas CTAs (the rest loop)
     const size_t want = (vecs + kStageThreads - 1) / kStageThreads;
     const int grid = (int)(want < 1 ? 1 : (want > (size_t)max_ctas ? (size_t)max_ctas : want));
-    stage_in_kernel<<<grid, kStageThreads, 0, stream>>>(sp);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(kStageThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, stage_in_kernel, sp);
 }
 
 }  // namespace qda

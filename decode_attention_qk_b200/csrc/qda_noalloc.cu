@@ -9,7 +9,6 @@
 // loaded on a device and kept until the process exits; no call allocates or
 // frees anything.
 #include <cstdint>
-#include <functional>
 #include <mutex>
 
 #include <cuda_runtime.h>
@@ -32,6 +31,7 @@ constexpr size_t kOffCounters = kOffPartMl + kPartMlBytes;
 constexpr size_t kOffStatus = kOffCounters + kCounterBytes;
 // 3,469,568 bytes (about 3.3 MiB) on every device that loads the library.
 constexpr size_t kScratchBytes = kOffStatus + kStatusBytes;
+static_assert(kScratchBytes == 3469568, "the size the header states");
 static_assert(kOffPartMl % 256 == 0 && kOffCounters % 256 == 0 && kOffStatus % 256 == 0, "256-byte sections");
 
 static __device__ __align__(256) unsigned char g_qda_noalloc_scratch[kScratchBytes];
@@ -40,8 +40,8 @@ constexpr int kMaxDevices = 64;
 constexpr int64_t kTimeoutNs = 1000000000;  // 1 s per device-side wait
 
 struct DeviceSetup {
-    std::once_flag once;
-    cudaError_t err = cudaSuccess;
+    std::mutex mu;
+    bool ready = false;                // set only by a set-up that succeeded
     unsigned char* scratch = nullptr;  // device address of g_qda_noalloc_scratch
     int grid = 0;
 };
@@ -49,19 +49,27 @@ DeviceSetup g_setup[kMaxDevices];
 
 // Once per device, with that device current: look up the device address of
 // the scratch array (its name is only a host-side stand-in), raise the
-// kernel's shared-memory limit, and size the grid.
-void setup_device(int device, DeviceSetup& s) {
+// kernel's shared-memory limit, and size the grid. A set-up that fails (for
+// instance when the first call is made during a stream capture, where the
+// lookup may not run) leaves the device not ready and clears the CUDA error,
+// so a later call tries again.
+cudaError_t setup_device(int device, DeviceSetup& s) {
+    std::lock_guard<std::mutex> lock(s.mu);
+    if (s.ready) return cudaSuccess;
     void* ptr = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&ptr, g_qda_noalloc_scratch);
     if (e == cudaSuccess) e = qda::prepare_device();
     int sms = 0;
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
     if (e == cudaSuccess && sms < 1) e = cudaErrorInvalidDevice;
-    s.err = e;
-    if (e == cudaSuccess) {
-        s.scratch = static_cast<unsigned char*>(ptr);
-        s.grid = sms < kNoAllocMaxGrid ? sms : kNoAllocMaxGrid;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return e;
     }
+    s.scratch = static_cast<unsigned char*>(ptr);
+    s.grid = sms < kNoAllocMaxGrid ? sms : kNoAllocMaxGrid;
+    s.ready = true;
+    return cudaSuccess;
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -86,8 +94,7 @@ extern "C" int qwen3_decode_attn_append_and_attend_noalloc(const void* qkv, cons
     int device = 0;
     if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= kMaxDevices) return QDA_ERR_CUDA;
     DeviceSetup& s = g_setup[device];
-    std::call_once(s.once, setup_device, device, std::ref(s));
-    if (s.err != cudaSuccess) return QDA_ERR_CUDA;
+    if (setup_device(device, s) != cudaSuccess) return QDA_ERR_CUDA;
 
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     // The array keeps the previous call's contents: the merge counters must
@@ -107,6 +114,7 @@ extern "C" int qwen3_decode_attn_append_and_attend_noalloc(const void* qkv, cons
     p.o = static_cast<uint16_t*>(o);
     p.num_q_heads = qda::kNumQHeads;
     p.new_tokens = 1;
+    p.tok_stride = 1;
     p.bt_stride = block_table_stride;
     p.num_pages = num_pages;
     p.batch = batch;
@@ -116,7 +124,6 @@ extern "C" int qwen3_decode_attn_append_and_attend_noalloc(const void* qkv, cons
     p.part_acc = reinterpret_cast<float*>(s.scratch);
     p.part_ml = reinterpret_cast<float2*>(s.scratch + kOffPartMl);
     p.counters = reinterpret_cast<int*>(s.scratch + kOffCounters);
-    p.seg = nullptr;
     p.status = reinterpret_cast<int*>(s.scratch + kOffStatus);
     p.timeout_ns = kTimeoutNs;
     p.flags = 0u;

@@ -1,4 +1,6 @@
-// The two nodes that produce the attention step's input, fused: input_norm
+// The dense products around the attention step on the 5th-generation tensor
+// cores: attn.o_proj (after it) and, first, the two nodes that produce the
+// step's input, fused: input_norm
 // (RMSNorm over the hidden size H with a gain per feature) and attn.qkv_proj
 // (a linear map with no bias), Qwen3-0.6B Model Spec, "Compute-graph nodes":
 //   qkv[b, n] = sum_k ( x[b, k] / r_b * g[k] ) * W[n, k],
@@ -10,82 +12,71 @@
 // sum them in float. 1/r_b (from float sums of the exact squares x^2, finished
 // in double) scales the float sums just before the one rounding to bf16.
 //
-// Work split. The product is cut along N into 128-column tiles and along K
-// into 4 quarters: CTA (n-tile, quarter, row block) reads the 128 weight rows'
-// quarter (64 KiB at H = 1024) and its rows' quarter of the split, and writes
-// a float partial tile into its own shared memory. The four quarters of a tile
-// form a thread-block cluster: after a cluster barrier, quarter q adds the
-// four partials of columns [32q, 32q + 32) in quarter order, reading its peers'
-// shared memory directly (so the result does not depend on timing and no
-// partial goes through L2), scales by 1/r_b and writes bf16 qkv. With 4 warps
-// of 32 columns each, a CTA needs no reduction of its own.
+// Two launches. The first forms hi, lo and 1/r_b once per row into the
+// handle's workspace (the product reads each row many times). The second is
+// a dense product on the 5th-generation tensor cores (linear_tc_kernel):
 //
-// Operands reach shared memory by 16-byte asynchronous copies (cp.async)
-// through a 3-stage ring of 128-wide K chunks (64-wide for the 64-row blocks
-// of large batches, so that two CTAs share an SM), in rows 16 bytes longer
-// than the chunk so that the 8 rows an ldmatrix phase reads fall in 8
-// different bank groups. (One
-// bulk copy per short row slice was tried first: at about one copy every
-// 45 ns per SM the copy count, not the bytes, set the time.)
+//   CTA (n-tile, k-part, batch group) computes a 128 x C tile of the result
+//   transposed, D[n][b] = sum_k W[n][k] (hi[b][k] + lo[b][k]), with the 128
+//   weight rows as the A operand (M = 128) and C <= 64 batch rows as the B
+//   operand (N = C). A producer thread streams 128 x 64 weight boxes and the
+//   matching C x 64 boxes of hi and lo into a 6-stage shared ring by tiled
+//   copies with the 128-byte swizzle; one thread issues tcgen05.mma (two per
+//   16-wide K step: hi, then lo, into the same accumulator) and frees each
+//   stage with tcgen05.commit; the accumulator lives in tensor memory and the
+//   four warps read it back (tcgen05.ld) for the epilogue.
 //
-// The split of x*g. For up to 32 rows each CTA forms it for its own quarter of
-// K from raw x staged next to the weight (4x less repeated work than forming
-// it for all of K, and no second launch). For more rows a first launch forms
-// it once per row (with 1/r_b) into workspace and the product launch starts
-// with programmatic dependent launch: it issues the weight copies of its first
-// stages before it waits for the first launch.
-#include <cooperative_groups.h>
+//   The work split fills the SMs at any batch: the batch is cut in groups
+//   of at most 64 rows, and the K range in P = 1, 2, 4 or 8 parts, the
+//   fewest that keep at least 80% of the SMs busy (at 0.6B: P = 4 for
+//   qkv_proj up to 64 rows, giving 128 CTAs; P = 1 at 256 rows). The P parts
+//   of a tile form a thread-block cluster; after the products, CTA q of the
+//   cluster adds the P partial tiles of rows [q * 128/P, (q+1) * 128/P) in
+//   part order, reading its peers' shared memory (distributed shared
+//   memory), so the result does not depend on timing.
+//
+// The product launch is a programmatic dependent of the first: it allocates
+// tensor memory and issues its first weight copies before it waits for the
+// first launch's hi, lo and 1/r.
+//
+// attn.o_proj (Model Spec, "Compute-graph nodes": linear, K = 2048,
+// N = 1024 for 0.6B) is the same product with one term: the attention output
+// o [B][Hq][128], read as rows of Hq * 128, is the B operand as it is (bf16
+// products are exact in float), no row scale; it is launched as a
+// programmatic dependent of the attention, whose o it waits for after its
+// first weight copies.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
+#include <cooperative_groups.h>
 #include <cstdint>
+#include <mutex>
 
 #include "qda_device.cuh"
 #include "qda_internal.h"
+#include "qda_tc.cuh"
 #include "qwen3_decode_attn.h"
 
 namespace qda {
 namespace {
 
-constexpr int kNT = kProjNTile;                // output columns per CTA
-constexpr int kKS = kProjKSplits;              // K quarters
-constexpr int kStages = 3;
-constexpr int kWarps = 4;
-constexpr int kThreadsP = kWarps * 32;
 constexpr int kPrepThreads = 128;
 
-// kConvert: the CTA forms the split itself from raw x (up to 32 rows); else it
-// copies the split formed by the first launch.
-template <int MT, bool kConvert>
-struct PLayout {
-    // K per chunk: 128, or 64 for the 64-row blocks of large batches, whose
-    // CTAs then fit two to an SM
-    static constexpr int kKC = kConvert ? 128 : 64;
-    static constexpr int kPitch = kKC * 2 + 16;                      // staged row pitch (bytes)
-    static constexpr int kPieces = kKC / 8;                          // 16-byte pieces per row slice
-    static constexpr int kCtasPerSm = kConvert ? 1 : 2;
-    static constexpr int kARows = kConvert ? MT : 2 * MT;            // raw x, or hi and lo
-    static constexpr int kStageBytes = (kNT + kARows) * kPitch;
-    static constexpr int kSmemHiLo = kStages * kStageBytes;          // convert: hi, lo of the current chunk
-    static constexpr int kSmemGain = kSmemHiLo + (kConvert ? 2 * MT * kPitch : 0);   // bf16 [hidden / 4]
-    static constexpr int kSmemInvR = kSmemGain + (kConvert ? kMaxHidden / kKS * 2 : 0);  // float [MT]
-    static constexpr int kSmemTotal = kSmemInvR + MT * 4;
-    // after the K loop the ring holds this quarter's partial tile and sums of x^2
-    static_assert((MT * kNT + MT) * 4 <= kStages * kStageBytes, "partial tile fits in the ring");
-    static_assert(kCtasPerSm * (kSmemTotal + 1024) <= 228 * 1024, "CTAs per SM fit in shared memory");
-    static_assert(kStageBytes % 16 == 0 && kPitch % 128 == 16, "alignment, conflict-free rows");
-};
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-__device__ __forceinline__ float warp_sum_f(float v) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
-    return v;
-}
+constexpr int kLinThreads = 128;                      // 4 warps: producer, MMA issuer, and all four for the epilogue
+constexpr int kLinM = 128;                            // weight rows per CTA (the instruction's M)
+constexpr int kLinKC = 64;                            // K per stage: one 128-byte swizzle row
+constexpr int kLinStages = 6;
+constexpr int kLinMaxCols = 64;                       // batch rows per CTA (the instruction's N)
+constexpr int kLinABytes = kLinM * kLinKC * 2;        // 16 KiB of weight per stage
+constexpr int kLinBBytes = 2 * kLinMaxCols * kLinKC * 2;   // hi and lo boxes: up to 16 KiB
+constexpr int kLinStageBytes = kLinABytes + kLinBBytes;
+constexpr int kLinSmemBars = kLinStages * kLinStageBytes;   // full[S], empty[S], acc, tmem address, abort
+constexpr int kLinSmemUsed = kLinSmemBars + (2 * kLinStages + 1) * 8 + 16;
+constexpr int kLinSmemTotal = kLinSmemUsed + 1024;    // slack to align the ring to 1024 bytes
+constexpr uint32_t kLinTmemCols = 64;
+static_assert(kLinStageBytes % 1024 == 0 && kLinABytes % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
+static_assert(kLinSmemTotal <= 227 * 1024, "fits one CTA per SM");
+static_assert(kLinMaxCols * kLinM * 4 <= kLinSmemBars, "the partial tile fits in the drained ring");
 
 // The exact split of the products x*g of one 16-byte piece (8 values): hi, lo
 // words, and the squares of x added to ss.
@@ -106,8 +97,14 @@ __device__ __forceinline__ void split_piece(const uint4& xv, const uint32_t* gw,
     lv = make_uint4(lw[0], lw[1], lw[2], lw[3]);
 }
 
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+    return v;
+}
+
 // ---------------------------------------------------------------------------
-// First launch (more than 32 rows): per row b, the split of x[b, k] * g[k] and 1 / r_b.
+// First launch: per row b, the split of x[b, k] * g[k] and 1 / r_b.
 
 __global__ void __launch_bounds__(kPrepThreads) input_norm_split_kernel(const QkvProjParams p) {
     pdl_launch_dependents();   // the product may start streaming the weight now
@@ -137,237 +134,292 @@ __global__ void __launch_bounds__(kPrepThreads) input_norm_split_kernel(const Qk
 }
 
 // ---------------------------------------------------------------------------
-// The product, split along K.
+// The dense product on tcgen05.
 
-template <int MT, bool kConvert>
-__global__ void __launch_bounds__(kThreadsP, PLayout<MT, kConvert>::kCtasPerSm) qkv_proj_kernel(const QkvProjParams p) {
-    using Lay = PLayout<MT, kConvert>;
-    constexpr int kMTiles = MT / 16;
-    constexpr int kKC = Lay::kKC;
-    constexpr int kPitch = Lay::kPitch;
-    constexpr int kPieces = Lay::kPieces;
-    extern __shared__ __align__(128) uint8_t smem[];
-    pdl_launch_dependents();   // an attention launch after this one may start its K/V streaming
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5;
-    const int lane = tid & 31;
-    const int nt = (int)blockIdx.x, ks = (int)blockIdx.y, mb = (int)blockIdx.z;
-    const int n0 = nt * kNT;
-    const int m0 = mb * MT;
-    const int rows = min(MT, p.batch - m0);
-    const int kq = p.hidden / kKS;           // this CTA's K range: [ks*kq, ks*kq + kq)
-    const int kbase = ks * kq;
-    const int chunks = kq / kKC;
+// Bounded wait of one thread; on expiry records QDA_ERR_TIMEOUT and sets the
+// CTA's abort flag.
+__device__ __forceinline__ bool lin_wait(uint64_t* bar, uint32_t parity, const LinearParams& p,
+                                         volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_wait(bar, parity, p.timeout_ns, abort_flag)) return true;
+    *abort_flag = 1;
+    record_error(p.status, QDA_ERR_TIMEOUT);
+    return false;
+}
+
+__global__ void __launch_bounds__(kLinThreads, 1)
+    linear_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_hi,
+                     const __grid_constant__ CUtensorMap tm_lo, const LinearParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    // the ring must start on a 1024-byte boundary (the swizzle atom)
+    uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     const uint32_t ring = smem_addr(smem);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kLinSmemBars);
+    uint64_t* empty = full + kLinStages;
+    uint64_t* acc_bar = empty + kLinStages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_bar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-    auto weight_rows = [&](int c) {   // 128 rows x 128: needs nothing from a first launch
-        const uint32_t stage = ring + (c % kStages) * Lay::kStageBytes;
-        for (int i = tid; i < kNT * kPieces; i += kThreadsP) {
-            const int r = i / kPieces, q = i % kPieces;
-            cp_async16(stage + r * kPitch + q * 16,
-                       p.w + (size_t)(n0 + r) * p.hidden + (size_t)(kbase + c * kKC) + q * 8);
+    pdl_launch_dependents();   // a launch consuming this result may be scheduled now
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = (int)blockIdx.x * kLinM;
+    const int part = (int)blockIdx.y;               // K part = rank in the cluster when k_split > 1
+    const int b0 = (int)blockIdx.z * p.cols;
+    const int chunks = p.k / kLinKC / p.k_split;    // K stages of this CTA
+    const int c0 = part * chunks;
+    const uint32_t term_bytes = (uint32_t)p.cols * kLinKC * 2;
+    const uint32_t stage_tx = (uint32_t)kLinABytes + (p.two_terms ? 2u : 1u) * term_bytes;
+
+    if (warp == 0) tmem_alloc(tmem_slot, kLinTmemCols);
+    if (threadIdx.x == 32) {
+        for (int s = 0; s < kLinStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
         }
-    };
-    auto a_rows = [&](int c) {        // raw x rows, or hi and lo rows
-        const uint32_t stage = ring + (c % kStages) * Lay::kStageBytes + kNT * kPitch;
-        for (int i = tid; i < rows * kPieces; i += kThreadsP) {
-            const int r = i / kPieces, q = i % kPieces;
-            const size_t src = (size_t)(m0 + r) * p.hidden + (size_t)(kbase + c * kKC) + q * 8;
-            if (kConvert) {
-                cp_async16(stage + r * kPitch + q * 16, p.x + src);
-            } else {
-                cp_async16(stage + r * kPitch + q * 16, p.xg_hi + src);
-                cp_async16(stage + (MT + r) * kPitch + q * 16, p.xg_lo + src);
-            }
-        }
-    };
-    // Groups, oldest first: {gain quarter and weight of chunks 0..S-2}, {A of
-    // chunk 0}, ..., {A of chunk S-2}, then one group per later chunk.
-    const int pre = min(kStages - 1, chunks);
-    if (kConvert)
-        for (int i = tid; i < kq / 8; i += kThreadsP) cp_async16(ring + Lay::kSmemGain + i * 16, p.norm_w + kbase + i * 8);
-    for (int c = 0; c < pre; ++c) weight_rows(c);
-    cp_async_commit();
-    if (!kConvert) pdl_wait();   // hi, lo and 1/r are complete and visible from here on
-    for (int c = 0; c < kStages - 1; ++c) {
-        if (c < pre) a_rows(c);
-        cp_async_commit();
+        mbar_init(acc_bar, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
 
-    const int g = lane >> 2, t = lane & 3;
-    // kConvert: thread tid splits pieces tid + 128 m (row (tid + 128 m) / 16,
-    // piece tid % 16); the 16 threads of a half-warp share a row
-    constexpr int kConvPerThread = kConvert ? MT * kPieces / kThreadsP : 1;
-    float ss[kConvPerThread];
-#pragma unroll
-    for (int m = 0; m < kConvPerThread; ++m) ss[m] = 0.f;
-    float acc[kMTiles][4][4];
-#pragma unroll
-    for (int i = 0; i < kMTiles; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
-    for (int c = 0; c < chunks; ++c) {
-        if (c + kStages - 1 < chunks) {
-            weight_rows(c + kStages - 1);
-            a_rows(c + kStages - 1);
+    if (warp == 0 && lane == 0) {
+        // Producer. The weight boxes of the first round need nothing from the
+        // previous launch; the activation boxes wait for it.
+        tma_prefetch_desc(&tm_w);
+        tma_prefetch_desc(&tm_hi);
+        if (p.two_terms) tma_prefetch_desc(&tm_lo);
+        const int pre = min(kLinStages, chunks);
+        for (int c = 0; c < pre; ++c) {
+            mbar_arrive_expect_tx(&full[c], stage_tx);
+            tma_load_2d(ring + c * kLinStageBytes, &tm_w, (c0 + c) * kLinKC, n0, &full[c]);
         }
-        cp_async_commit();
-        cp_async_wait<kStages - 1>();   // this thread's copies of chunk c have landed ...
-        __syncthreads();                // ... and everyone's
-        const uint32_t stage = ring + (c % kStages) * Lay::kStageBytes;
-        uint32_t abase_hi, abase_lo;
-        if (kConvert) {
-            const uint8_t* raw = smem + (c % kStages) * Lay::kStageBytes + kNT * kPitch;
-            const uint32_t* gw = reinterpret_cast<const uint32_t*>(smem + Lay::kSmemGain) + (c * kKC) / 2;
+        if (p.wait_acts) {
+            pdl_wait();
+            asm volatile("fence.proxy.async.global;" ::: "memory");   // the copies read what it wrote
+        }
+        auto acts = [&](int c, int s) {
+            const uint32_t b = ring + s * kLinStageBytes + kLinABytes;
+            tma_load_2d(b, &tm_hi, (c0 + c) * kLinKC, b0, &full[s]);
+            if (p.two_terms) tma_load_2d(b + term_bytes, &tm_lo, (c0 + c) * kLinKC, b0, &full[s]);
+        };
+        for (int c = 0; c < pre; ++c) acts(c, c);
+        int issued = pre;
+        for (int c = pre; c < chunks; ++c) {
+            const int s = c % kLinStages;
+            if (!lin_wait(&empty[s], (uint32_t)((c / kLinStages - 1) & 1), p, abort_flag)) break;
+            mbar_arrive_expect_tx(&full[s], stage_tx);
+            tma_load_2d(ring + s * kLinStageBytes, &tm_w, (c0 + c) * kLinKC, n0, &full[s]);
+            acts(c, s);
+            issued = c + 1;
+        }
+        if (*abort_flag != 0) {
+            // copies still landing in this CTA's shared memory: wait (bounded) for the last round
+            for (int c = max(0, issued - kLinStages); c < issued; ++c)
+                (void)mbar_wait(&full[c % kLinStages], (uint32_t)((c / kLinStages) & 1), p.timeout_ns, nullptr);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // MMA issuer: two products per 16-wide K step (hi, then lo) into one accumulator.
+        const uint32_t idesc = umma_idesc_bf16_m128(p.cols);
+        for (int c = 0; c < chunks; ++c) {
+            const int s = c % kLinStages;
+            if (!lin_wait(&full[s], (uint32_t)((c / kLinStages) & 1), p, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t a = ring + s * kLinStageBytes;
+            const uint32_t b = a + kLinABytes;
 #pragma unroll
-            for (int m = 0; m < kConvPerThread; ++m) {
-                const int i = tid + kThreadsP * m;
-                const int r = i / kPieces, q = i % kPieces;
-                uint4 hv, lv;
-                split_piece(*reinterpret_cast<const uint4*>(raw + r * kPitch + q * 16), gw + 4 * q, hv, lv, ss[m]);
-                *reinterpret_cast<uint4*>(smem + Lay::kSmemHiLo + r * kPitch + q * 16) = hv;
-                *reinterpret_cast<uint4*>(smem + Lay::kSmemHiLo + (MT + r) * kPitch + q * 16) = lv;
+            for (int kk = 0; kk < kLinKC / 16; ++kk) {
+                const uint64_t da = umma_desc_sw128(a + 32 * kk);
+                umma_bf16(tmem, da, umma_desc_sw128(b + 32 * kk), idesc, (c | kk) != 0 ? 1u : 0u);
+                if (p.two_terms) umma_bf16(tmem, da, umma_desc_sw128(b + term_bytes + 32 * kk), idesc, 1u);
             }
-            __syncthreads();
-            abase_hi = ring + Lay::kSmemHiLo;
-        } else {
-            abase_hi = stage + kNT * kPitch;
+            umma_commit(&empty[s]);   // the stage is free once these products have read it
         }
-        abase_lo = abase_hi + MT * kPitch;
-        // ldmatrix row addresses: this warp's 32 weight rows as the column-major
-        // B operand, hi and lo rows as the row-major A operand
-        const uint32_t wbase =
-            stage + (32 * warp + (lane & 7) + ((lane >> 4) << 3)) * kPitch + ((lane >> 3) & 1) * 16;
-        const uint32_t aoff = ((lane & 7) + ((lane >> 3) & 1) * 8) * kPitch + ((lane >> 4) & 1) * 16;
+        umma_commit(acc_bar);         // every product issued above has completed
+    }
+    __syncwarp();
+
+    // Epilogue: warp w holds tensor-memory lanes 32w..32w+31 = weight rows n0 + 32w + lane.
+    const bool ok = lin_wait(acc_bar, 0u, p, abort_flag) && *abort_flag == 0;
+    tc_fence_after();
+    if (p.wait_acts) pdl_wait();     // the row scales come from the previous launch
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+    if (p.k_split == 1) {
+        const int n = n0 + 32 * warp + lane;
+        for (int j0 = 0; j0 < p.cols && ok; j0 += 16) {
+            uint32_t v[16];
+            tmem_ld16(lane_base + (uint32_t)j0, v);
+            tmem_ld_wait();
 #pragma unroll
-        for (int kstep = 0; kstep < kKC / 16; ++kstep) {
-            const int k0 = kstep * 16;
-            uint32_t b[4][2];
-            ldsm_x4(wbase + k0 * 2, b[0][0], b[0][1], b[1][0], b[1][1]);
-            ldsm_x4(wbase + 16 * kPitch + k0 * 2, b[2][0], b[2][1], b[3][0], b[3][1]);
-#pragma unroll
-            for (int i = 0; i < kMTiles; ++i) {
-                uint32_t ahi[4], alo[4];
-                ldsm_x4(abase_hi + aoff + i * 16 * kPitch + k0 * 2, ahi[0], ahi[1], ahi[2], ahi[3]);
-                ldsm_x4(abase_lo + aoff + i * 16 * kPitch + k0 * 2, alo[0], alo[1], alo[2], alo[3]);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    mma_bf16_16816(acc[i][j], ahi, b[j][0], b[j][1]);
-                    mma_bf16_16816(acc[i][j], alo, b[j][0], b[j][1]);
+            for (int i = 0; i < 16; ++i) {
+                const int b = b0 + j0 + i;
+                if (b < p.batch) {
+                    const float sc = p.row_scale != nullptr ? __ldg(p.row_scale + b) : 1.f;
+                    p.y[(size_t)b * p.n_out + n] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[i]) * sc));
                 }
             }
         }
-        __syncthreads();                // the stage (and the hi/lo buffer) may be refilled
-    }
-    cp_async_wait<0>();
-
-    // This quarter's partial tile (float) and, when converting, its sums of x^2,
-    // in shared memory for the cluster.
-    namespace cg = cooperative_groups;
-    cg::cluster_group cluster = cg::this_cluster();
-    float* tile = reinterpret_cast<float*>(smem);   // [MT][kNT], the ring is drained
-    float* tss = tile + MT * kNT;                   // [MT]
+    } else {
+        // the partial tile [cols][128] (float) in the drained ring, then the
+        // cluster's parts are added in part order, rows [q*R, q*R + R) by part q
+        float* tile = reinterpret_cast<float*>(smem);
+        for (int j0 = 0; j0 < p.cols && ok; j0 += 16) {
+            uint32_t v[16];
+            tmem_ld16(lane_base + (uint32_t)j0, v);
+            tmem_ld_wait();
 #pragma unroll
-    for (int i = 0; i < kMTiles; ++i) {
-        const int r0 = 16 * i + g;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int col = 32 * warp + 8 * j + 2 * t;
-            *reinterpret_cast<float2*>(tile + r0 * kNT + col) = make_float2(acc[i][j][0], acc[i][j][1]);
-            *reinterpret_cast<float2*>(tile + (r0 + 8) * kNT + col) = make_float2(acc[i][j][2], acc[i][j][3]);
+            for (int i = 0; i < 16; ++i) tile[(j0 + i) * kLinM + 32 * warp + lane] = __uint_as_float(v[i]);
         }
-    }
-    if (kConvert) {
-#pragma unroll
-        for (int m = 0; m < kConvPerThread; ++m) {
-            float v = ss[m];
-            v += __shfl_xor_sync(kFull, v, 1);
-            v += __shfl_xor_sync(kFull, v, 2);
-            v += __shfl_xor_sync(kFull, v, 4);
-            v += __shfl_xor_sync(kFull, v, 8);
-            if ((lane & 15) == 0) tss[(tid + kThreadsP * m) / kPieces] = v;
+        tc_fence_before();
+        cluster_sync_all();   // every part's tile is in place
+        namespace cg = cooperative_groups;
+        cg::cluster_group cluster = cg::this_cluster();
+        const int rows = kLinM / p.k_split;
+        const int r0 = part * rows;
+        const int pairs = rows / 2;
+        for (int e = threadIdx.x; e < pairs * p.cols; e += kLinThreads) {
+            const int j = e / pairs, row = r0 + 2 * (e % pairs);
+            const int b = b0 + j;
+            float2 sum = make_float2(0.f, 0.f);
+            for (int q = 0; q < p.k_split; ++q) {
+                const float* peer = cluster.map_shared_rank(tile, q);
+                const float2 v = *reinterpret_cast<const float2*>(peer + j * kLinM + row);
+                sum.x += v.x;
+                sum.y += v.y;
+            }
+            if (b < p.batch && *abort_flag == 0) {
+                const float sc = p.row_scale != nullptr ? __ldg(p.row_scale + b) : 1.f;
+                *reinterpret_cast<uint32_t*>(p.y + (size_t)b * p.n_out + n0 + row) = pack_bf2(sum.x * sc, sum.y * sc);
+            }
         }
+        cluster_sync_all();   // peers may still be reading this CTA's tile
     }
-    cluster.sync();   // all four quarters' partials are in place
-    const int q = (int)cluster.block_rank();   // = ks
-    const float* peer[kKS];
-    const float* peer_ss[kKS];
-#pragma unroll
-    for (int r = 0; r < kKS; ++r) {
-        peer[r] = cluster.map_shared_rank(tile, r);
-        peer_ss[r] = cluster.map_shared_rank(tss, r);
-    }
-    float* inv_r = reinterpret_cast<float*>(smem + Lay::kSmemInvR);
-    for (int r = tid; r < rows; r += kThreadsP) {
-        if (kConvert) {
-            double sum = 0.0;
-#pragma unroll
-            for (int k = 0; k < kKS; ++k) sum += (double)peer_ss[k][r];
-            inv_r[r] = (float)(1.0 / sqrt(sum / (double)p.hidden + p.eps));
-        } else {
-            inv_r[r] = __ldg(p.inv_r + m0 + r);
-        }
-    }
+    tc_fence_before();
     __syncthreads();
-    // columns [32q, 32q + 32) of the tile: 16 column pairs per row
-    for (int e = tid; e < rows * 16; e += kThreadsP) {
-        const int r = e / 16, col = 32 * q + 2 * (e % 16);
-        float2 sum = *reinterpret_cast<const float2*>(peer[0] + r * kNT + col);
-#pragma unroll
-        for (int k = 1; k < kKS; ++k) {
-            const float2 v = *reinterpret_cast<const float2*>(peer[k] + r * kNT + col);
-            sum.x += v.x;
-            sum.y += v.y;
-        }
-        const float f = inv_r[r];
-        *reinterpret_cast<uint32_t*>(p.y + (size_t)(m0 + r) * p.qkv_width + n0 + col) = pack_bf2(sum.x * f, sum.y * f);
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kLinTmemCols);
     }
-    cluster.sync();   // peers may still be reading this CTA's partial
 }
 
-template <int MT, bool kConvert>
-cudaError_t prepare_proj_one() {
-    return cudaFuncSetAttribute(qkv_proj_kernel<MT, kConvert>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                PLayout<MT, kConvert>::kSmemTotal);
+// ---------------------------------------------------------------------------
+// Host side: tensor maps and launches.
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+        else
+            cudaGetLastError();
+    });
+    return fn;
 }
 
-template <int MT, bool kConvert>
-cudaError_t launch_proj_one(const QkvProjParams& p, cudaStream_t stream) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(p.qkv_width / kNT), (unsigned)kKS, (unsigned)((p.batch + MT - 1) / MT));
-    cfg.blockDim = dim3(kThreadsP, 1, 1);
-    cfg.dynamicSmemBytes = PLayout<MT, kConvert>::kSmemTotal;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;   // the 4 K quarters of a tile
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = kKS;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = kConvert ? 1 : 2;   // dependent launch only after the split's own launch
-    return cudaLaunchKernelEx(&cfg, qkv_proj_kernel<MT, kConvert>, p);
+// A row-major bf16 matrix [rows][cols] (cols contiguous, row pitch cols * 2
+// bytes) read in boxes of 64 x box_rows with the 128-byte swizzle; rows past
+// the end read as zeros.
+bool encode_rows(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
+    const PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kLinKC, (cuuint32_t)box_rows};
+    const cuuint32_t elem[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, elem,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
+void linear_split(int batch, int n_out, int k, int sms, int& cols, int& k_split, int& groups) {
+    cols = batch <= kLinMaxCols ? (batch + 15) / 16 * 16 : kLinMaxCols;
+    groups = (batch + cols - 1) / cols;
+    // K parts (a cluster of at most 8): the fewest that give about one CTA
+    // per SM (at least 80% of the SMs busy), so that no CTA waits for a
+    // second wave and no more partial tiles are added up than needed
+    const int tiles = n_out / kLinM * groups;
+    k_split = 1;
+    while (k_split < 8 && tiles * k_split * 5 < sms * 4 && (k / kLinKC) % (2 * k_split) == 0) k_split *= 2;
+}
+
+cudaError_t launch_linear(const LinearOperands& ops, const LinearParams& p0, cudaStream_t stream) {
+    LinearParams p = p0;
+    int device = 0, sms = 0, groups = 1;
+    if (cudaGetDevice(&device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms < 1)
+        return cudaErrorInvalidDevice;
+    linear_split(p.batch, p.n_out, p.k, sms, p.cols, p.k_split, groups);
+    if (p.k % (kLinKC * p.k_split) != 0 || p.n_out % kLinM != 0) return cudaErrorInvalidValue;
+    CUtensorMap tw, th, tl;
+    if (!encode_rows(&tw, ops.w, p.n_out, p.k, kLinM) || !encode_rows(&th, ops.act_hi, p.batch, p.k, p.cols) ||
+        !encode_rows(&tl, ops.act_lo != nullptr ? ops.act_lo : ops.act_hi, p.batch, p.k, p.cols))
+        return cudaErrorInvalidValue;
+    p.two_terms = ops.act_lo != nullptr ? 1 : 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.n_out / kLinM), (unsigned)p.k_split, (unsigned)groups);
+    cfg.blockDim = dim3(kLinThreads, 1, 1);
+    cfg.dynamicSmemBytes = kLinSmemTotal;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (p.k_split > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;   // the K parts of a tile
+        attr[n].val.clusterDim.x = 1;
+        attr[n].val.clusterDim.y = (unsigned)p.k_split;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, linear_tc_kernel, tw, th, tl, p);
+}
+
 cudaError_t prepare_qkv_proj() {
-    cudaError_t e = prepare_proj_one<16, true>();
-    if (e == cudaSuccess) e = prepare_proj_one<32, true>();
-    if (e == cudaSuccess) e = prepare_proj_one<64, false>();
-    return e;
+    if (encode_fn() == nullptr) return cudaErrorNotSupported;
+    return cudaFuncSetAttribute(linear_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinSmemTotal);
+}
+
+cudaError_t launch_o_proj(const OProjParams& p, cudaStream_t stream) {
+    LinearOperands ops{p.w, p.x, nullptr};
+    LinearParams lp{};
+    lp.y = p.y;
+    lp.row_scale = nullptr;
+    lp.batch = p.batch;
+    lp.k = p.in_features;
+    lp.n_out = p.hidden;
+    lp.wait_acts = 1;
+    lp.status = p.status;
+    lp.timeout_ns = p.timeout_ns;
+    return launch_linear(ops, lp, stream);
 }
 
 cudaError_t launch_qkv_proj(const QkvProjParams& p, cudaStream_t stream) {
-    if (p.batch <= 16) return launch_proj_one<16, true>(p, stream);
-    if (p.batch <= 32) return launch_proj_one<32, true>(p, stream);
     input_norm_split_kernel<<<p.batch, kPrepThreads, 0, stream>>>(p);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    return launch_proj_one<64, false>(p, stream);
+    LinearOperands ops{p.w, p.xg_hi, p.xg_lo};
+    LinearParams lp{};
+    lp.y = p.y;
+    lp.row_scale = p.inv_r;
+    lp.batch = p.batch;
+    lp.k = p.hidden;
+    lp.n_out = p.qkv_width;
+    lp.wait_acts = 1;
+    lp.status = p.status;
+    lp.timeout_ns = p.timeout_ns;
+    return launch_linear(ops, lp, stream);
 }
 
 }  // namespace qda

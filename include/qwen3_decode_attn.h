@@ -91,7 +91,7 @@ extern "C" {
 #define QDA_QKV_WIDTH     4096
 #define QDA_MAX_BATCH     256
 #define QDA_MAX_SEQ_LEN   40960
-#define QDA_MAX_NEW_TOKENS 4   /* new tokens per sequence of one call */
+#define QDA_MAX_NEW_TOKENS 40960 /* new tokens per sequence of one call (also <= max_seq_len) */
 
 /* Return codes. */
 #define QDA_OK               0
@@ -143,8 +143,8 @@ void qwen3_decode_attn_default_config(qda_config *cfg);
 int qwen3_decode_attn_create(const qda_config *cfg, int device, qda_handle **out);
 
 /* The decode-attention step on device buffers (layouts above, with the
- * handle's Hq). At 16 query heads it is one kernel launch; at 32, 40 or 64 a
- * second launch combines sequences split across CTAs. Every pointer is a
+ * handle's Hq). One kernel launch: sequences whose pages are split across
+ * CTAs are combined inside it by the CTA finishing last. Every pointer is a
  * device pointer. qkv, k_cache, v_cache and o must be 16-byte aligned;
  * q_norm_w, k_norm_w, seq_lens, positions and block_table 4-byte aligned.
  * `batch` is B (1..max_batch); `num_pages` (>= 1) bounds every block-table
@@ -184,14 +184,18 @@ int qwen3_decode_attn_append_and_attend(qda_handle *h,
  * position positions[b] + t (or L - T + t when positions is NULL), and its
  * query attends over slots 0 .. L - T + t: the cache before the call plus the
  * new tokens up to and including itself.
- * new_tokens = 1 is exactly qwen3_decode_attn_append_and_attend. For T > 1 the
- * compiled instances are 16 query heads with T = 2, 3 or 4 and 32 query heads
- * with T = 2 (at most 8 query rows per kv head); every call is two launches
- * (attention, then the combine of split sequences).
+ * new_tokens = 1 is exactly qwen3_decode_attn_append_and_attend. For T > 1 one
+ * launch takes up to 16 query rows per kv head (T * Hq / 8 <= 16: T <= 8 at
+ * 16 query heads, 4 at 32, 3 at 40, 2 at 64); a longer block runs as
+ * consecutive launches over chunks of its tokens, each chunk attending over
+ * the cache plus the block's tokens up to its own, so the result is the same
+ * causal attention (a chunked prefill; each launch reads the sequence's whole
+ * cache again). Up to 8 query rows per kv head q and the probabilities enter
+ * the tensor cores as two bf16 terms (about 16 significant bits); with 9 to
+ * 16 rows they enter as bf16 (8 bits), with float sums either way.
  * Errors as for qwen3_decode_attn_append_and_attend, plus INVALID_ARG for
- * new_tokens outside [1, QDA_MAX_NEW_TOKENS] and UNSUPPORTED for a (query
- * heads, new_tokens) pair with no instance; on the device, a seq_len below T
- * is out of range like one above the limits. */
+ * new_tokens outside [1, min(QDA_MAX_NEW_TOKENS, max_seq_len)]; on the
+ * device, a seq_len below T is out of range like one above the limits. */
 int qwen3_decode_attn_append_and_attend_tokens(qda_handle *h,
                                                const void *qkv,
                                                const void *q_norm_w,
@@ -211,8 +215,10 @@ int qwen3_decode_attn_append_and_attend_tokens(qda_handle *h,
 /* The step's input, from the hidden state: input_norm then attn.qkv_proj
  * (Model Spec, "Compute-graph nodes": rmsnorm over H = hidden with a gain
  * per feature and eps = the handle's rms_eps; then y[t,n] = sum_k x[t,k]
- * w[n,k], no bias), one launch:
+ * w[n,k], no bias):
  *   qkv[b,n] = sum_k (x[b,k] / sqrt(sum_j x[b,j]^2 / hidden + eps) * g[k]) * w_qkv[n,k]
+ * Two launches on `cuda_stream`: one forms the normalised rows into the
+ * handle's workspace, the second is the product on the tensor cores.
  * Layouts (device pointers, 16-byte aligned): x bf16 [B][hidden] (row
  * stride hidden); input_norm_w bf16 [hidden]; w_qkv bf16 [N][hidden] with
  * N = (num_q_heads + 16) * 128 of the handle (row n = output feature n, the
@@ -225,8 +231,9 @@ int qwen3_decode_attn_append_and_attend_tokens(qda_handle *h,
  * lies within about 2^-19 (relative) of a rounding midpoint, where it may be
  * the neighbouring bf16 value.
  * Errors: INVALID_ARG (null or misaligned pointer, batch outside
- * [1, max_batch], hidden not a multiple of 512 in range), CUDA (the launch
- * failed). */
+ * [1, max_batch], hidden not a multiple of 512 in range), CUDA (a launch
+ * failed). Device-side errors (a bounded wait that ran out) go to the status
+ * word read by qwen3_decode_attn_check. */
 int qwen3_decode_attn_qkv_proj(qda_handle *h,
                                const void *x,
                                const void *input_norm_w,
@@ -236,9 +243,37 @@ int qwen3_decode_attn_qkv_proj(qda_handle *h,
                                int batch,
                                void *cuda_stream);
 
+/* The step's consumer, attn.o_proj (Model Spec, "Compute-graph nodes":
+ * linear, y[t,n] = sum_k x[t,k] w[n,k], K = 2048, N = 1024 for Qwen3-0.6B, no
+ * bias), on the tensor cores, one launch:
+ *   y[b,n] = sum_k o[b,k] * w_o[n,k]
+ * Layouts (device pointers, 16-byte aligned): x bf16 [B][Hq * 128], the
+ * attention output o [B][Hq][128] of this handle's head count read as rows
+ * (the "Tensors of the main nodes" table gives attn.core's o [B, 16, 128]
+ * and attn.o_proj's x [T, 2048]); w_o bf16 [hidden][Hq * 128] (row n =
+ * output feature n, a torch Linear weight); y bf16 [B][hidden] (output).
+ * hidden is a multiple of 128 in [128, 8192] (Qwen3: 1024 for 0.6B; 2048,
+ * 2560, 4096, 5120 for the larger sizes). The products of two bf16 values are
+ * exact and summed in float; y is rounded once to bf16. The launch is a
+ * programmatic dependent of the previous launch on the stream: its first
+ * weight copies overlap that launch's end, and it reads x only after that
+ * launch has completed, so it may directly follow the attention call that
+ * writes o.
+ * Errors: INVALID_ARG (null or misaligned pointer, batch outside
+ * [1, max_batch], hidden not a multiple of 128 in range), CUDA (the launch
+ * failed). Device-side errors (a bounded wait that ran out) go to the status
+ * word read by qwen3_decode_attn_check. */
+int qwen3_decode_attn_o_proj(qda_handle *h,
+                             const void *x,
+                             const void *w_o,
+                             int hidden,
+                             void *y,
+                             int batch,
+                             void *cuda_stream);
+
 /* qwen3_decode_attn_qkv_proj into `qkv` (caller-owned, bf16 [B][N], it
  * holds the step's qkv afterwards), then qwen3_decode_attn_append_and_attend
- * on it: the layer's attention from the hidden state, two or three launches
+ * on it: the layer's attention from the hidden state, three or four launches
  * on `cuda_stream`. Arguments and errors as for those two calls. */
 int qwen3_decode_attn_from_hidden(qda_handle *h,
                                   const void *x,
@@ -272,8 +307,11 @@ int qwen3_decode_attn_from_hidden(qda_handle *h,
  * kernel where it lies; otherwise it is copied out of the staging buffer.
  * All of it is queued on `cuda_stream` and the call returns; o_host is valid after
  * the stream is synchronized, and the host buffers must not change before
- * then. Requires block_table_stride <= max_pages_per_seq. Errors as for
- * qwen3_decode_attn_append_and_attend. */
+ * then. The stage-in launch may start while the previous launch on the stream
+ * still runs (alternate calls use alternate staging buffers): it reads the
+ * host inputs at once, so they must be final when the call is made, and must
+ * not be written by work queued before it. Requires block_table_stride <=
+ * max_pages_per_seq. Errors as for qwen3_decode_attn_append_and_attend. */
 int qwen3_decode_attn_append_and_attend_host(qda_handle *h,
                                              const void *qkv_host,
                                              const void *q_norm_w,
@@ -303,21 +341,27 @@ int qwen3_decode_attn_append_and_attend_host(qda_handle *h,
  * calling thread's current device; every pointer is a device pointer of that
  * device, with the layouts and alignment stated above. The caller still
  * passes every input and output. The kernel's scratch (partials of sequences
- * split across CTAs, merge counters, a status word) is one fixed device array
- * of 3,469,568 bytes that every GPU which loads the library holds until the
+ * split across CTAs, merge counters, a status word) is one fixed device
+ * array of 3,469,568 bytes that every GPU which loads the library holds until the
  * process exits. It is sized for at most 256 sequences per call (a larger
  * batch returns QDA_ERR_INVALID_ARG) and at most 160 CTAs per launch (the call
  * launches min(SM count, 160)).
  *
  * The first call on each device performs a one-time set-up there (it looks up
  * the array's device address and raises the kernel's shared-memory limit);
- * make that first call before any stream capture. Each call then zeroes the
- * merge counters and the status word on `cuda_stream` before it launches. All
+ * make that first call before any stream capture. A first call whose set-up
+ * fails returns QDA_ERR_CUDA and leaves the device to be set up again by the
+ * next call. Each call then zeroes the merge counters and the status word on
+ * `cuda_stream` before it launches (a memset, so the launch does not overlap
+ * the end of the work queued before it the way the handle entry point's
+ * launches do). All
  * calls share the one array, which keeps the last call's contents: calls that
  * overlap on the GPU (different streams or threads without ordering between
  * them) race on it and produce wrong results. Device-side errors (an
- * out-of-range seq_len or page id) are not reported by this entry point,
- * though the kernel still never reads or writes out of range.
+ * out-of-range seq_len or page id, a wait that ran out) are not reported by
+ * this entry point: the kernel still never reads or writes out of range, but
+ * o is then undefined for the sequences concerned and nothing tells the
+ * caller; callers who need that report use the handle entry points.
  * Errors: INVALID_ARG (as for qwen3_decode_attn_append_and_attend, or batch
  * > 256), CUDA (the set-up, the memset or the launch failed). */
 int qwen3_decode_attn_append_and_attend_noalloc(const void *qkv,

@@ -181,3 +181,94 @@ def assert_o_close(o_got, o_ref, label=""):
     assert max_abs <= GATE_ABS and rel <= GATE_REL, f"{label}: max abs {max_abs:.3g}, rel rms {rel:.3g}"
     assert strict_excess <= 0.0, f"{label}: strict bound exceeded by {strict_excess:.3g} (max abs {max_abs:.3g})"
     return max_abs, rel
+
+
+# ---------------------------------------------------------------------------
+# Instances with more than 8 query rows per kv head ("wide": T * Hq / 8 > 8)
+# enter q and the probabilities into the tensor cores as bf16. Their strict
+# check compares o with a float64 attention that uses the oracle's q rounded
+# the way the kernel rounds it (bf16 of q * log2(e) / sqrt(128), nearest-even),
+# over the oracle's post-append cache. Rounding each probability to bf16
+# (relative error <= 2^-9; the sums add the same rounded values) moves each
+# normalised weight by at most ~2^-8 of itself, so
+#   |o - o_emul| <= 2^-8 sum_t w_t |v_t - o_emul|,
+# checked with a factor 2 of margin (a float q may round to the neighbouring
+# bf16 value where the double one sits near a midpoint), plus o's own bf16
+# rounding and float sums: 2^-7 sum_t w_t |v_t - o| + 2^-8 |o| + 2e-4.
+
+Q_SCALE = 1.4426950408889634 / np.sqrt(128.0)
+
+
+def chunk_sizes(num_q_heads: int, T: int):
+    """How the library runs a block of T new tokens: one launch takes up to 16
+    query rows per kv head (T * Hq / 8); a longer block runs in chunks of that
+    many tokens, and at 16 query heads a last chunk of one token borrows one
+    from the chunk before."""
+    G = num_q_heads // 8
+    max_t = 16 // G
+    if T <= max_t:
+        return [T]
+    sizes, c0 = [], 0
+    while c0 < T:
+        n = min(max_t, T - c0)
+        if num_q_heads == 16 and T - c0 - n == 1:
+            n -= 1
+        sizes.append(n)
+        c0 += n
+    return sizes
+
+
+def wide_tokens(w: inputs.Workload):
+    """Per new token: whether its launch takes more than 8 query rows per kv
+    head (q and the probabilities then enter the tensor cores as bf16)."""
+    G = w.num_q_heads // 8
+    if w.new_tokens == 1:
+        return [False]
+    flags = []
+    for n in chunk_sizes(w.num_q_heads, w.new_tokens):
+        flags += [n * G > 8] * n
+    return flags
+
+
+def is_wide(w: inputs.Workload) -> bool:
+    return any(wide_tokens(w))
+
+
+def emulated_bf16_q_check(o_gpu, q64, seq_lens, block_table, k_bits, v_bits, T, label="", tokens=None):
+    """o_gpu [B, T, Hq, 128] against the float64 attention with bf16-rounded
+    scaled q (see above) for the new tokens `tokens` (default all); q64 the
+    oracle's q [B, T, Hq, 128]; caches post-append."""
+    got = o_gpu.detach().float().cpu().numpy().astype(np.float64)
+    B, _, Hq, D = q64.shape
+    G = Hq // 8
+    qs = oracle.bf16_to_f64(oracle.f64_to_bf16_rne(q64 * Q_SCALE))
+    worst = -np.inf
+    for b in range(B):
+        L = int(seq_lens[b])
+        slots = np.arange(L)
+        pages = block_table[b, slots // 16]
+        K = oracle.bf16_to_f64(k_bits[pages, slots % 16])   # [L, 8, 128]
+        V = oracle.bf16_to_f64(v_bits[pages, slots % 16])
+        for t in (range(T) if tokens is None else tokens):
+            n = L - T + t + 1
+            for h in range(Hq):
+                s = K[:n, h // G] @ qs[b, t, h]          # log2 units
+                wgt = np.exp2(s - s.max())
+                wgt /= wgt.sum()
+                o_em = wgt @ V[:n, h // G]
+                spread = wgt @ np.abs(V[:n, h // G] - o_em)
+                bound = 2.0 ** -7 * spread + 2.0 ** -8 * np.abs(o_em) + 2e-4
+                worst = max(worst, float(np.max(np.abs(got[b, t, h] - o_em) - bound)))
+    assert worst <= 0.0, f"{label}: bf16-q bound exceeded by {worst:.3g}"
+
+
+def oracle_sampled_qk(w: inputs.Workload, seqs, k_pre, v_pre):
+    """The oracle over the sequences `seqs` only, with q and the compact
+    post-append caches (for emulated_bf16_q_check)."""
+    seqs = torch.as_tensor(seqs, dtype=torch.int64)
+    lens, bt, kc, vc = _compact(w, seqs, k_pre, v_pre)
+    pos = None if w.positions is None else w.positions[seqs].numpy()
+    out = oracle.append_and_attend_tokens(
+        _qkv3(w)[seqs.numpy()], inputs.bf16_bits(w.q_norm_w), inputs.bf16_bits(w.k_norm_w), lens.numpy(),
+        bt.numpy(), kc, vc, positions=pos, inplace=True, want_qk=True)
+    return out, lens.numpy(), bt.numpy()

@@ -123,6 +123,8 @@ def test_calls_on_a_null_handle_are_rejected(lib):
         assert fn(None, p, p, p, i32, None, i32, 1, p, p, 1, p, 1, None) == binding.QDA_ERR_INVALID_ARG
     assert lib.qwen3_decode_attn_append_and_attend_tokens(None, p, p, p, i32, None, i32, 1, p, p, 1, p, 1, 2,
                                                           None) == binding.QDA_ERR_INVALID_ARG
+    assert lib.qwen3_decode_attn_qkv_proj(None, p, p, p, 1024, p, 1, None) == binding.QDA_ERR_INVALID_ARG
+    assert lib.qwen3_decode_attn_o_proj(None, p, p, 1024, p, 1, None) == binding.QDA_ERR_INVALID_ARG
     assert lib.qwen3_decode_attn_check(None, None) == binding.QDA_ERR_INVALID_ARG
     assert lib.qwen3_decode_attn_grid_ctas(None) == 0
     lib.qwen3_decode_attn_destroy(None)

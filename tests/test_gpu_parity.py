@@ -6,6 +6,8 @@ configuration) compare the whole cache bit for bit against the pre-call cache
 plus the oracle's appended rows, and o on sampled sequences the oracle
 recomputes one by one.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -157,6 +159,35 @@ def test_host_buffer_entry_point(attn):
     assert attn.check() == 0
     assert torch.equal(o_host.view(torch.int16), o_dev.cpu().view(torch.int16))
     assert torch.equal(k0.view(torch.int16), w.k_cache.view(torch.int16))
+
+
+def test_host_buffer_calls_back_to_back(attn):
+    """Consecutive host-buffer calls on one stream, no synchronization between
+    them: each call's stage-in may run while the previous call's attention
+    still reads its staging set (alternate calls use alternate sets). Five
+    calls, each on a different batch appending into the same caches (the next
+    token of the same sequences), give the bytes of five device-entry calls."""
+    lens0 = torch.tensor([77, 1, 16, 513, 2000, 33], dtype=torch.int32)
+    w = inputs.custom((lens0 + 5).tolist(), seed=26, device="cuda", gap_fraction=0.2)
+    kd, vd = w.k_cache.clone(), w.v_cache.clone()
+    kh, vh = w.k_cache.clone(), w.v_cache.clone()
+    steps = []
+    for i in range(5):
+        qkv = inputs.custom((lens0 + 5).tolist(), seed=27 + i, device="cuda").qkv
+        steps.append(dataclasses.replace(w, qkv=qkv, seq_lens=(lens0 + 1 + i).contiguous()))
+    o_dev = [ph.run(attn, wi, DEV, kd, vd) for wi in steps]
+    torch.cuda.synchronize(DEV)
+    pin = lambda t: t.cpu().pin_memory()
+    host_in = [(pin(wi.qkv), pin(wi.seq_lens), pin(wi.block_table)) for wi in steps]
+    o_host = [torch.empty((6, 16, 128), dtype=torch.bfloat16).pin_memory() for _ in steps]
+    for (qkv_h, sl_h, bt_h), oh in zip(host_in, o_host):
+        binding.qwen3_decode_attn_append_and_attend_host(attn.handle, qkv_h, w.q_norm_w, w.k_norm_w, sl_h, None, bt_h,
+                                                         kh, vh, oh)
+    assert attn.check() == 0
+    for i in range(5):
+        assert torch.equal(o_host[i].view(torch.int16), o_dev[i].cpu().view(torch.int16)), i
+    assert torch.equal(kh.view(torch.int16), kd.view(torch.int16))
+    assert torch.equal(vh.view(torch.int16), vd.view(torch.int16))
 
 
 def pinned_at_offset(t):

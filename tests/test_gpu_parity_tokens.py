@@ -1,11 +1,13 @@
-"""Parity of the step with several new tokens per sequence (T = 2..4, causal
+"""Parity of the step with several new tokens per sequence (T = 2..8, causal
 inside the new block) with the float64 oracle, through the C ABI.
 
 Token t of sequence b goes to cache slot L - T + t (L = seq_lens[b] counts the
 new tokens) and its query attends over slots 0 .. L - T + t (Qwen3-0.6B Model
 Spec, "What to watch for": every layer is full causal attention). The checks
 are those of the one-token step: the whole cache bit for bit, o within the
-gate and the strict bound.
+gate and the strict bound. Instances with more than 8 query rows per kv head
+(T * Hq / 8 > 8) take q and the probabilities as bf16; their o is held to the
+gate against the oracle and to the bound of parity_helpers.emulated_bf16_q_check.
 """
 import dataclasses
 
@@ -25,15 +27,33 @@ CASES = list(binding.SUPPORTED_MULTI_TOKEN)   # (query heads, new tokens)
 def handles():
     from decode_attention_qk_b200 import build
     build.build_library()
-    hs = {hq: binding.DecodeAttention(device=0, num_q_heads=hq) for hq in (16, 32)}
+    hs = {hq: binding.DecodeAttention(device=0, num_q_heads=hq) for hq in (16, 32, 40, 64)}
     yield hs
     for h in hs.values():
         h.close()
 
 
+def check_o(o, ref, w, label):
+    """The required gate against the oracle over all of o; then, per new
+    token, the one-token step's strict bound, or for tokens whose launch took
+    q as bf16 (more than 8 query rows per kv head) the bf16-q bound."""
+    if not ph.is_wide(w):
+        return ph.assert_o_close(o, ref["o"], label)
+    max_abs, rel, _ = ph.o_errors(o, ref["o"])
+    assert max_abs <= ph.GATE_ABS and rel <= ph.GATE_REL, f"{label}: max abs {max_abs:.3g}, rel rms {rel:.3g}"
+    flags = ph.wide_tokens(w)
+    narrow = [t for t, f in enumerate(flags) if not f]
+    if narrow:
+        ph.assert_o_close(o[:, narrow], ref["o"][:, narrow], label + " (two-term rows)")
+    ph.emulated_bf16_q_check(o, ref["q"], ref["seq_lens"], ref["block_table"], ref["k_cache"], ref["v_cache"],
+                             w.new_tokens, label, tokens=[t for t, f in enumerate(flags) if f])
+    return max_abs, rel
+
+
 def full_check(attn, w, label, positions=None):
     k, v = w.k_cache.to(DEV), w.v_cache.to(DEV)
     ref = ph.oracle_full(w, k, v, positions=positions)
+    ref["seq_lens"], ref["block_table"] = w.seq_lens.numpy(), w.block_table.numpy()
     o = ph.run(attn, w, DEV, k, v, positions=positions)
     assert attn.check() == 0
     assert o.shape == (w.batch, w.new_tokens, w.num_q_heads, 128)
@@ -42,7 +62,7 @@ def full_check(attn, w, label, positions=None):
         bad = np.argwhere(got_k != ref["k_cache"])[:8].tolist()
         raise AssertionError(f"{label}: k cache differs at {bad}")
     assert np.array_equal(got_v, ref["v_cache"]), f"{label}: v cache differs"
-    ph.assert_o_close(o, ref["o"], label)
+    check_o(o, ref, w, label)
     return o, ref
 
 
@@ -110,6 +130,39 @@ def test_split_count_does_not_change_the_result(grid):
     a.close()
 
 
+@pytest.mark.parametrize("hq,T", [(16, 9), (16, 20), (32, 9), (40, 4), (64, 5), (64, 3)])
+def test_blocks_longer_than_one_launch(handles, hq, T):
+    """A block of more new tokens than one launch takes runs as consecutive
+    launches over chunks of it (a chunked prefill): the same cache bits and the
+    same causal attention as the oracle's single pass over the block."""
+    lens = [T, T + 1, 16, 31, 33, 47, 48, 300, 1000]
+    lens = [max(L, T) for L in lens]
+    w = inputs.custom(lens, seed=72 + hq + T, device="cuda", gap_fraction=0.2, num_q_heads=hq, new_tokens=T)
+    full_check(handles[hq], w, f"Hq={hq} T={T} in chunks")
+
+
+def test_a_long_block_over_a_long_cache(handles):
+    """64 new tokens (8 launches at 16 heads) after up to 5000 cached ones, with positions."""
+    w = inputs.custom([64, 100, 5064, 777], seed=73, device="cuda", gap_fraction=0.1, new_tokens=64)
+    full_check(handles[16], w, "T=64 in chunks", positions=torch.tensor([0, 36, 9000, 713], dtype=torch.int32))
+
+
+@pytest.mark.parametrize("grid", [1, 5, 148])
+def test_split_count_does_not_change_the_result_wide(handles, grid):
+    """The same with 8 new tokens at 16 heads (16 query rows per kv head)."""
+    a = binding.DecodeAttention(device=0, grid_ctas=grid)
+    w = inputs.custom([8, 16, 17, 23, 24, 25, 300, 2000, 33], seed=70, device="cuda", gap_fraction=0.2,
+                      new_tokens=8)
+    full_check(a, w, f"T=8 grid {grid}")
+    a.close()
+
+
+@pytest.mark.parametrize("hq,T", [(16, 8), (64, 2)])
+def test_maximum_context_wide(handles, hq, T):
+    w = inputs.custom([40960, 40955, 9], seed=71, device="cuda", stride=2560, new_tokens=T, num_q_heads=hq)
+    full_check(handles[hq], w, f"Hq={hq} T={T} L=40960")
+
+
 def test_positions_argument(handles):
     full_check(handles[16], inputs.custom([5, 100, 1234], seed=65, device="cuda", new_tokens=3),
                "T=3 positions", positions=torch.tensor([0, 7000, 40000], dtype=torch.int32))
@@ -120,12 +173,13 @@ def test_maximum_context(handles):
     full_check(handles[16], w, "T=4 L=40960")
 
 
-def test_locality_with_nan_in_unread_bytes(handles):
+@pytest.mark.parametrize("T", [4, 8])
+def test_locality_with_nan_in_unread_bytes(handles, T):
     """The new tokens' rows (written, never read before), rows past a sequence,
     pages it does not own and table entries past its last page may hold
     anything (here NaN): o and the appended rows do not change."""
-    attn, T = handles[16], 4
-    w = inputs.custom([7, 12, 40, 16, 18], seed=67, device="cuda", pool_pages=16, stride=6, new_tokens=T)
+    attn = handles[16]
+    w = inputs.custom([8, 12, 40, 16, 18], seed=67, device="cuda", pool_pages=16, stride=6, new_tokens=T)
     ka, va = w.k_cache.clone(), w.v_cache.clone()
     kb, vb = w.k_cache.clone(), w.v_cache.clone()
     bt2 = w.block_table.clone()
@@ -178,16 +232,12 @@ def test_host_side_errors(handles):
     a = ph.device_args(w, DEV)
     call = lambda h, qkv, o: binding.qwen3_decode_attn_append_and_attend_tokens(
         h, qkv, a["q_norm_w"], a["k_norm_w"], a["seq_lens"], None, a["block_table"], w.k_cache, w.v_cache, o)
-    h40 = binding.DecodeAttention(device=0, num_q_heads=40)
-    w40 = inputs.custom([20, 30], seed=69, device="cuda", num_q_heads=40, new_tokens=2)
+    small = binding.DecodeAttention(device=0, max_seq_len=8, max_pages_per_seq=8)
+    qkv9 = torch.zeros((2, 9, 4096), dtype=torch.bfloat16, device=DEV)   # more new tokens than max_seq_len
     with pytest.raises(binding.QdaError) as e:
-        call(h40.handle, w40.qkv, torch.empty((2, 2, 40, 128), dtype=torch.bfloat16, device=DEV))
-    assert e.value.code == binding.QDA_ERR_UNSUPPORTED
-    h40.close()
-    qkv5 = torch.zeros((2, 5, 4096), dtype=torch.bfloat16, device=DEV)
-    with pytest.raises(binding.QdaError) as e:
-        call(handles[16].handle, qkv5, torch.empty((2, 5, 16, 128), dtype=torch.bfloat16, device=DEV))
+        call(small.handle, qkv9, torch.empty((2, 9, 16, 128), dtype=torch.bfloat16, device=DEV))
     assert e.value.code == binding.QDA_ERR_INVALID_ARG
+    small.close()
     with pytest.raises(ValueError):   # several tokens are not taken by the one-token entry point
         binding.qwen3_decode_attn_append_and_attend(
             handles[16].handle, a["qkv"], a["q_norm_w"], a["k_norm_w"], a["seq_lens"], None, a["block_table"],
@@ -203,6 +253,19 @@ def full_size_check(attn, w, sample, label):
     k_exp, v_exp = ph.expected_cache(w, k_pre, v_pre, k_rows, v_rows)
     ph.assert_cache_equal(w.k_cache, w.v_cache, k_exp, v_exp, k64, w)
     del k_exp, v_exp
+    if ph.is_wide(w):
+        ref, lens, bt = ph.oracle_sampled_qk(w, sample, k_pre, v_pre)
+        ref["seq_lens"], ref["block_table"] = lens, bt
+        sub = o[torch.as_tensor(sample)]
+        max_abs, rel, _ = ph.o_errors(sub, ref["o"])
+        assert max_abs <= ph.GATE_ABS and rel <= ph.GATE_REL, f"{label}: max abs {max_abs:.3g}, rel rms {rel:.3g}"
+        flags = ph.wide_tokens(w)
+        narrow = [t for t, f in enumerate(flags) if not f]
+        if narrow:
+            ph.assert_o_close(sub[:, narrow], ref["o"][:, narrow], label + " (two-term rows)")
+        ph.emulated_bf16_q_check(sub, ref["q"], lens, bt, ref["k_cache"], ref["v_cache"], w.new_tokens, label,
+                                 tokens=[t for t, f in enumerate(flags) if f])
+        return max_abs, rel
     ref = ph.oracle_sampled(w, sample, k_pre, v_pre)
     return ph.assert_o_close(o[torch.as_tensor(sample)], ref, label)
 

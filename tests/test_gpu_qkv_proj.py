@@ -65,7 +65,7 @@ def run_proj(attn, d):
     return qkv
 
 
-@pytest.mark.parametrize("B", [1, 5, 16, 17, 32, 33, 64, 65, 200, 256])
+@pytest.mark.parametrize("B", [1, 5, 16, 17, 32, 33, 64, 65, 128, 129, 200, 256])
 def test_parity_at_batch_sizes(handles, B):
     d = inputs.hidden_inputs(B, seed=100 + B)
     ref = oracle.input_norm_qkv_proj(inputs.bf16_bits(d["x"]), inputs.bf16_bits(d["input_norm_w"]),
