@@ -35,6 +35,7 @@ from decode_attention_qk_b200 import inputs  # noqa: E402
 
 METRIC = "decode-attn KV GB/s and µs/call (1 B200) as fraction of HBM roofline"
 PROJ_METRIC = "input_norm + qkv_proj GB/s (weight + x + gain + qkv bytes) and µs/call (1 B200)"
+O_METRIC = "attn.o_proj GB/s (weight + x + y bytes) and µs/call (1 B200)"
 KV_BYTES_PER_TOKEN = 2 * inputs.NUM_KV_HEADS * inputs.HEAD_DIM * 2      # K and V rows: 4096 B
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
@@ -103,6 +104,16 @@ def proj_bytes(batch: int, hidden: int = inputs.HIDDEN, num_q_heads: int = 16) -
     """Least HBM traffic of input_norm + qkv_proj: the weight, x, the gain and qkv."""
     N = inputs.qkv_width(num_q_heads)
     return N * hidden * 2 + batch * hidden * 2 + hidden * 2 + batch * N * 2
+
+
+def o_bytes(batch: int, hidden: int = inputs.HIDDEN, num_q_heads: int = 16) -> int:
+    """Least HBM traffic of attn.o_proj: the weight, x (the attention output) and y."""
+    K = num_q_heads * inputs.HEAD_DIM
+    return hidden * K * 2 + batch * K * 2 + batch * hidden * 2
+
+
+def o_flops(batch: int, hidden: int = inputs.HIDDEN, num_q_heads: int = 16) -> int:
+    return 2 * batch * hidden * num_q_heads * inputs.HEAD_DIM
 
 
 def proj_flops(batch: int, hidden: int = inputs.HIDDEN, num_q_heads: int = 16) -> int:
@@ -355,9 +366,23 @@ def cpu_baseline(layers, seconds: float = 12.0, threads: int = 1):
             "cpu_model": model, "seconds": elapsed}
 
 
+def time_o_proj_oracle(w, rows) -> float:
+    """Seconds the oracle's attn.o_proj takes for the given rows of layer w."""
+    import oracle
+    d = w.o_in
+    sel = torch.tensor(list(rows), dtype=torch.int64, device=d["x"].device)
+    x = inputs.bf16_bits(d["x"].index_select(0, sel))
+    wo = inputs.bf16_bits(d["w_o"])
+    t0 = time.perf_counter()
+    oracle.o_proj(x, wo)
+    return time.perf_counter() - t0
+
+
 def time_proj_oracle(w, rows) -> float:
     """Seconds the oracle's input_norm + qkv_proj takes for the given rows of layer w."""
     import oracle
+    if getattr(w, "o_in", None) is not None:
+        return time_o_proj_oracle(w, rows)
     d = w.hidden_in
     sel = torch.tensor(list(rows), dtype=torch.int64, device=d["x"].device)
     x = inputs.bf16_bits(d["x"].index_select(0, sel))
@@ -375,13 +400,13 @@ def cpu_baseline_proj(layers, mode, seconds: float = 12.0, threads: int = 1):
     oracle.build()
     oracle.set_threads(threads)
     w0 = layers[0]
-    hidden = w0.hidden_in["x"].shape[1]
+    hidden = w0.o_in["w_o"].shape[0] if mode == "o_proj" else w0.hidden_in["x"].shape[1]
     try:
         per_row = time_proj_oracle(w0, [0])
-        if mode == "qkv_proj":
+        if mode in ("qkv_proj", "o_proj"):
             rows = list(range(min(w0.batch, max(1, int(seconds / max(per_row, 1e-6))))))
             elapsed = time_proj_oracle(w0, rows)
-            units = proj_bytes(len(rows), hidden, w0.num_q_heads)
+            units = (o_bytes if mode == "o_proj" else proj_bytes)(len(rows), hidden, w0.num_q_heads)
             desc = f"{len(rows)} of {w0.batch} rows of one call"
         else:
             probe = min(range(w0.batch), key=lambda b: int(w0.seq_lens[b]))
@@ -409,12 +434,42 @@ def run_gpu(args):
     dist, rank, world, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    result = measure(args, dist, rank, world, dev, headline=True)
+    per_config = (world == 1 and args.per_config and args.op == "step" and not args.from_hidden
+                  and args.num_q_heads == 16 and args.new_tokens == 1)
+    if per_config:
+        # every other configuration of the workload set, each timed on its own
+        # (graph replay of at least ~0.1 s, end to end through the host-buffer
+        # entry point), so that one default run covers them all
+        entries = {}
+        for wl in sorted(WORKLOADS):
+            if wl == args.workload:
+                continue
+            sub = argparse.Namespace(**vars(args))
+            sub.workload, sub.warmup, sub.rotate = wl, 5, 0
+            entries[wl] = measure(sub, dist, rank, world, dev, headline=False)
+            torch.cuda.empty_cache()
+        if rank == 0:
+            result["per_config"] = entries
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def measure(args, dist, rank, world, dev, headline: bool):
+    """Time one workload on this rank's GPU. headline: the K steps the command
+    line asks for, with the eager comparison and a sustained leg; otherwise a
+    per-configuration entry whose step count is chosen so that its timed
+    region lasts at least ~0.1 s. Returns the result dict (rank 0) or None."""
+    from decode_attention_qk_b200 import binding
+
     lib = binding.load_library()
-    attn = binding.DecodeAttention(device=local, num_q_heads=args.num_q_heads)
+    attn = binding.DecodeAttention(device=dev.index, num_q_heads=args.num_q_heads)
     T = args.new_tokens
-    mode = "qkv_proj" if args.op == "qkv_proj" else ("from_hidden" if args.from_hidden else "attention")
+    mode = args.op if args.op in ("qkv_proj", "o_proj") else ("from_hidden" if args.from_hidden else "attention")
     if mode != "attention" and T != 1:
-        raise SystemExit("--op qkv_proj and --from-hidden take one new token per sequence")
+        raise SystemExit("--op qkv_proj, --op o_proj and --from-hidden take one new token per sequence")
 
     # R resident copies of the step's inputs, so that a call never finds its
     # K/V in L2 from the previous call (each copy's KV is > L2 or R copies are).
@@ -424,19 +479,32 @@ def run_gpu(args):
         step_bytes = sum(kv_bytes(w.seq_lens) for w in first)
     elif mode == "from_hidden":
         step_bytes = sum(kv_bytes(w.seq_lens) + proj_bytes(w.batch, hidden, args.num_q_heads) for w in first)
+    elif mode == "o_proj":
+        step_bytes = sum(o_bytes(w.batch, hidden, args.num_q_heads) for w in first)
     else:
         step_bytes = sum(proj_bytes(w.batch, hidden, args.num_q_heads) for w in first)
     cap = 8 if mode == "attention" else 64
     rotate = args.rotate or max(1, min(cap, math.ceil(4 * L2_BYTES / max(step_bytes, 1))))
     step_kv = step_bytes
-    # the copies hold the same bytes in different memory, so every timed launch does the same work
-    sets = [first] + [make_layers(args.workload, dev, rank, args.num_q_heads, T) for r in range(1, rotate)]
-    if mode != "attention":
+    # the copies hold the same bytes in different memory, so every timed launch does the same work;
+    # the projection modes rotate only their own inputs (the attention's cache is not read there)
+    if mode in ("qkv_proj", "o_proj"):
+        import dataclasses
+        sets = [first] + [[dataclasses.replace(w) for w in first] for r in range(1, rotate)]
+    else:
+        sets = [first] + [make_layers(args.workload, dev, rank, args.num_q_heads, T) for r in range(1, rotate)]
+    if mode in ("qkv_proj", "from_hidden"):
         for si, layers in enumerate(sets):
             for li, w in enumerate(layers):
                 # per layer and copy: its hidden state, input_norm gain and qkv_proj weight
                 w.hidden_in = inputs.hidden_inputs(w.batch, seed=7000 + 100 * rank + li, device=dev, hidden=hidden,
                                                    num_q_heads=args.num_q_heads)
+    elif mode == "o_proj":
+        for si, layers in enumerate(sets):
+            for li, w in enumerate(layers):
+                # per layer and copy: its attention output rows and o_proj weight
+                w.o_in = inputs.o_proj_inputs(w.batch, seed=8000 + 100 * rank + li, device=dev, hidden=hidden,
+                                              num_q_heads=args.num_q_heads)
     calls_per_step = len(first)
     stream = torch.cuda.current_stream(dev)
     sp = ctypes.c_void_p(stream.cuda_stream)
@@ -449,11 +517,16 @@ def run_gpu(args):
                      o=torch.empty((*w.qkv.shape[:-1], w.num_q_heads, 128), dtype=torch.bfloat16, device=dev))
             vp = lambda k: ctypes.c_void_p(t[k].data_ptr())
             i32 = lambda k: ctypes.cast(ctypes.c_void_p(t[k].data_ptr()), ctypes.POINTER(ctypes.c_int32))
-            if mode != "attention":
+            if mode in ("qkv_proj", "from_hidden"):
                 t.update(w.hidden_in)
                 t["qkv"] = torch.empty_like(w.qkv)   # written by the projection
-            proj = (vp("x"), vp("input_norm_w"), vp("w_qkv"), hidden) if mode != "attention" else ()
-            if mode == "qkv_proj":
+            if mode == "o_proj":
+                t.update(ox=w.o_in["x"], w_o=w.o_in["w_o"],
+                         y=torch.empty((w.batch, hidden), dtype=torch.bfloat16, device=dev))
+            proj = (vp("x"), vp("input_norm_w"), vp("w_qkv"), hidden) if mode in ("qkv_proj", "from_hidden") else ()
+            if mode == "o_proj":
+                c = (attn.handle, vp("ox"), vp("w_o"), hidden, vp("y"), int(w.batch), sp)
+            elif mode == "qkv_proj":
                 c = (attn.handle, *proj, vp("qkv"), int(w.batch), sp)
             else:
                 c = ((attn.handle, *proj, vp("qkv"), vp("q"), vp("k"), i32("sl"), None, i32("bt"),
@@ -463,7 +536,8 @@ def run_gpu(args):
         return out
 
     calls = [prepared(layers) for layers in sets]
-    fn = {"qkv_proj": lib.qwen3_decode_attn_qkv_proj, "from_hidden": lib.qwen3_decode_attn_from_hidden}.get(
+    fn = {"qkv_proj": lib.qwen3_decode_attn_qkv_proj, "from_hidden": lib.qwen3_decode_attn_from_hidden,
+          "o_proj": lib.qwen3_decode_attn_o_proj}.get(
         mode, lib.qwen3_decode_attn_append_and_attend_tokens if T > 1 else lib.qwen3_decode_attn_append_and_attend)
 
     def step(i):
@@ -480,7 +554,22 @@ def run_gpu(args):
     if rc != 0:
         raise binding.QdaError(rc, "device status after warm-up")
 
+    if not headline:
+        # a step count whose graph-replayed region lasts at least ~0.1 s
+        per0 = graph_plan(10 ** 6, rotate, calls_per_step)[0]
+        g = capture_graphs(calls, fn, dev, rotate, per0)
+        g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        est_ms = max(reduce_max(dist, e0.elapsed_time(e1), dev) / per0, 1e-4)
+        del g
+        args.steps = per0 * max(1, math.ceil(100.0 / (per0 * est_ms)))
+
     n_launch = args.steps * calls_per_step
+    sustained = None
     if args.timing == "graph":
         # The timed region replays CUDA graphs that each hold `per_graph`
         # consecutive steps (step i runs rotation set i % rotate; per_graph is a
@@ -509,6 +598,9 @@ def run_gpu(args):
         ms_local = start.elapsed_time(end)
         kernel_ms = [ms_local / n_launch] * n_launch
         del g_full, g_rest
+        if headline:
+            sustained = sustained_leg(calls, fn, dev, dist, stream, rotate, calls_per_step,
+                                      ms_local / args.steps, clocks)
     else:
         t0, t1, ms_local, kernel_ms = timed_eager(args, calls, fn, dev, dist, stream, rotate, calls_per_step)
     clocks.stop()
@@ -520,9 +612,13 @@ def run_gpu(args):
     ms_per_step = ms / args.steps
     # every rotation set has its own lengths (cfg2/cfg5 draw them); average the bytes per step
     def unit_bytes(w):   # what `value` counts: the K/V bytes attended, or the projection's bytes
+        if mode == "o_proj":
+            return o_bytes(w.batch, hidden, w.num_q_heads)
         return proj_bytes(w.batch, hidden, w.num_q_heads) if mode == "qkv_proj" else kv_bytes(w.seq_lens)
 
     def alg_bytes(w):
+        if mode == "o_proj":
+            return o_bytes(w.batch, hidden, w.num_q_heads)
         b = 0 if mode == "qkv_proj" else algorithmic_bytes(w.seq_lens, w.num_q_heads, T)
         return b + (proj_bytes(w.batch, hidden, w.num_q_heads) if mode != "attention" else 0)
 
@@ -541,7 +637,9 @@ def run_gpu(args):
                if mode == "attention" else None)
 
     # the other way of timing, for comparison: eager launches with an event pair around each
-    if args.timing == "graph":
+    if not headline:
+        other = None
+    elif args.timing == "graph":
         _, _, e_ms, e_kernel = timed_eager(args, calls, fn, dev, dist, stream, rotate, calls_per_step)
         other = {"timing": "eager launches, an event pair around each",
                  "us_per_call": round(reduce_max(dist, e_ms, dev) * 1e3 / n_launch, 3),
@@ -566,16 +664,18 @@ def run_gpu(args):
     proj_tensor = None
     if mode != "attention":
         tp, tp_kind = tensor_peak()
-        fl = sum(proj_flops(w.batch, hidden, w.num_q_heads) for w in first) / calls_per_step
+        flops = o_flops if mode == "o_proj" else proj_flops
+        fl = sum(flops(w.batch, hidden, w.num_q_heads) for w in first) / calls_per_step
         t_ach = fl / (mean_kernel_ms * 1e-3) / 1e12
         proj_tensor = {"bound": "tensor", "achieved": round(t_ach, 1), "peak": tp, "unit": "TFLOP/s",
                        "frac": round(t_ach / tp, 4), "peak_kind": tp_kind,
-                       "flops_per_launch": int(fl), "note": "algorithmic flops (2 per multiply-add); the exact "
-                       "hi/lo split issues twice as many on the tensor pipe"}
+                       "flops_per_launch": int(fl), "note": "algorithmic flops (2 per multiply-add)" + (
+                           "" if mode == "o_proj" else "; the exact hi/lo split issues twice as many on the tensor pipe")}
     if rank == 0:
         clk = clocks.summary(t0, t1, t_warm)
         result = {
-            "metric": METRIC if mode != "qkv_proj" else PROJ_METRIC, "value": round(value, 2), "unit": "GB/s",
+            "metric": {"qkv_proj": PROJ_METRIC, "o_proj": O_METRIC}.get(mode, METRIC), "value": round(value, 2),
+            "unit": "GB/s",
             "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
             "us_per_call": round(ms_per_step * 1e3 / calls_per_step, 3),
@@ -586,7 +686,9 @@ def run_gpu(args):
                                    + ("" if T == 1 else f", {T} new tokens per sequence (causal among them)")
                                    + {"attention": "", "from_hidden": f", from the hidden state (input_norm + "
                                       f"qkv_proj of x [B, {hidden}], then the attention step)",
-                                      "qkv_proj": f": input_norm + qkv_proj only (x [B, {hidden}] -> qkv)"}[mode],
+                                      "qkv_proj": f": input_norm + qkv_proj only (x [B, {hidden}] -> qkv)",
+                                      "o_proj": f": attn.o_proj only (o [B, {args.num_q_heads} x 128] -> "
+                                                f"y [B, {hidden}])"}[mode],
                        "op": mode, "batch": first[0].batch, "layers_per_step": calls_per_step, "new_tokens": T,
                        "sum_seq_lens_per_step": int(sum(int(w.seq_lens.sum()) for w in first)),
                        "page_size": 16, "heads": f"{args.num_q_heads} q / 8 kv, D=128",
@@ -607,16 +709,16 @@ def run_gpu(args):
                       else "eager launches, an event pair around each; per-launch duration = mean of the pairs",
             ("eager" if args.timing == "graph" else "graph"): other,
             "seq_per_s": round(first[0].batch / (ms_per_step * 1e-3) * world, 1),
-            # one kernel per call on the 16-head decode kernel; attention + combine launches otherwise;
-            # one more per call for the projection
-            "gpu_launches": n_launch * ((0 if mode == "qkv_proj" else (1 if kernel_key(args.num_q_heads, T) == 16 else 2))
-                                        + (0 if mode == "attention" else 1)),
+            # attention: one launch per call; the projection: two (the split, the product); o_proj: one
+            "gpu_launches": n_launch * {"qkv_proj": 2, "o_proj": 1, "from_hidden": 3}.get(mode, 1),
             "clocks": clk,
         }
     if dist is not None:
         dist.barrier(device_ids=[dev.index])
     attn.close()
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if result is not None and sustained is not None:
+        result["sustained"] = sustained
+    if headline and rank == 0 and world == 1 and not args.no_cpu_baseline:
         cores, _ = host_cpu()
         if mode == "attention":
             result["cpu_baseline"] = cpu_baseline(first)
@@ -624,10 +726,43 @@ def run_gpu(args):
                 result["cpu_baseline_all_cores"] = cpu_baseline(first, seconds=8.0, threads=cores)
         else:
             result["cpu_baseline"] = cpu_baseline_proj(first, mode)
-    if rank == 0:
-        print(json.dumps(result), flush=True)
-    if dist is not None:
-        dist.destroy_process_group()
+    if result is not None and not headline:
+        # the per-configuration entry: the same figures as the headline, for this workload
+        keep = ("value", "unit", "steps", "warmup", "ms_per_step", "us_per_call", "seq_per_s", "roofline", "e2e",
+                "clocks", "gpu_launches")
+        result = {"config": result["config"]["workload"], "sum_seq_lens_per_step":
+                  result["config"]["sum_seq_lens_per_step"], "l2": result["config"]["l2"],
+                  **{k: result[k] for k in keep},
+                  "timing": "CUDA graph replay of the steps, region of at least ~0.1 s between two events"}
+    return result
+
+
+def sustained_leg(calls, fn, dev, dist, stream, rotate, calls_per_step, est_ms_per_step, clocks):
+    """Back-to-back replays of one graph for at least 0.5 s of device time, so
+    that the clock sampler sees the timed region itself (the headline region
+    can be shorter than its sampling period). Returns µs per call and the
+    clocks of that window."""
+    per = graph_plan(10 ** 6, rotate, calls_per_step)[0]
+    g = capture_graphs(calls, fn, dev, rotate, per)
+    g.replay()
+    reps = max(1, math.ceil(500.0 / max(per * est_ms_per_step, 1e-4)))
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    t0 = time.perf_counter()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(reps):
+        g.replay()
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    t1 = time.perf_counter()
+    barrier(dist, dev)
+    ms = reduce_max(dist, start.elapsed_time(end), dev)
+    del g
+    return {"steps": reps * per, "seconds": round(ms / 1e3, 3),
+            "us_per_call": round(ms * 1e3 / (reps * per * calls_per_step), 3),
+            "timing": f"{reps} back-to-back replays of one CUDA graph of {per} steps between two events",
+            "clocks": clocks.summary(t0, t1, t0)}
 
 
 def graph_plan(steps: int, rotate: int, calls_per_step: int):
@@ -723,15 +858,23 @@ def run_e2e_proj(args, attn, sets, dev, stream, dist, rotate, mode, fn, unit_byt
     for layers in sets:
         hl = []
         for w in layers:
-            x_dev = w.hidden_in["x"]
-            out_dev = torch.empty_like(w.qkv) if mode == "qkv_proj" else \
-                torch.empty((w.batch, w.num_q_heads, 128), dtype=torch.bfloat16, device=dev)
-            qkv_dev = out_dev if mode == "qkv_proj" else torch.empty_like(w.qkv)
+            x_dev = w.o_in["x"] if mode == "o_proj" else w.hidden_in["x"]
+            if mode == "o_proj":
+                out_dev = torch.empty((w.batch, w.o_in["w_o"].shape[0]), dtype=torch.bfloat16, device=dev)
+            elif mode == "qkv_proj":
+                out_dev = torch.empty_like(w.qkv)
+            else:
+                out_dev = torch.empty((w.batch, w.num_q_heads, 128), dtype=torch.bfloat16, device=dev)
+            qkv_dev = out_dev if mode != "from_hidden" else torch.empty_like(w.qkv)
             h = dict(x=x_dev.cpu().pin_memory(), out=torch.empty(out_dev.shape, dtype=torch.bfloat16).pin_memory(),
                      sl=w.seq_lens.clone().pin_memory(), bt=w.block_table.clone().pin_memory())
             d = dict(x=x_dev, out=out_dev, sl=w.seq_lens.to(dev), bt=w.block_table.to(dev))
             vp = lambda t: ctypes.c_void_p(t.data_ptr())
             i32 = lambda t: ctypes.cast(ctypes.c_void_p(t.data_ptr()), ctypes.POINTER(ctypes.c_int32))
+            if mode == "o_proj":
+                c = (attn.handle, vp(d["x"]), vp(w.o_in["w_o"]), int(out_dev.shape[1]), vp(out_dev), int(w.batch), sp)
+                hl.append((c, h, d, qkv_dev))
+                continue
             proj = (vp(d["x"]), vp(w.hidden_in["input_norm_w"]), vp(w.hidden_in["w_qkv"]), int(d["x"].shape[1]))
             if mode == "qkv_proj":
                 c = (attn.handle, *proj, vp(qkv_dev), int(w.batch), sp)
@@ -744,7 +887,7 @@ def run_e2e_proj(args, attn, sets, dev, stream, dist, rotate, mode, fn, unit_byt
 
     def call(c, h, d):
         d["x"].copy_(h["x"], non_blocking=True)
-        if mode != "qkv_proj":
+        if mode == "from_hidden":
             d["sl"].copy_(h["sl"], non_blocking=True)
             d["bt"].copy_(h["bt"], non_blocking=True)
         rc = fn(*c)
@@ -762,7 +905,7 @@ def run_e2e_proj(args, attn, sets, dev, stream, dist, rotate, mode, fn, unit_byt
     for i in range(args.steps):
         for c, h, d, _ in host[i % rotate]:
             call(c, h, d)
-            h2d += h["x"].nbytes + (0 if mode == "qkv_proj" else h["sl"].nbytes + h["bt"].nbytes)
+            h2d += h["x"].nbytes + (h["sl"].nbytes + h["bt"].nbytes if mode == "from_hidden" else 0)
             d2h += h["out"].nbytes
     end.record(stream)
     torch.cuda.synchronize(dev)
@@ -931,7 +1074,7 @@ def run_reference(args):
     import oracle
     oracle.build()
     cores, cpu_model = host_cpu()
-    if args.op == "qkv_proj" or args.from_hidden:
+    if args.op in ("qkv_proj", "o_proj") or args.from_hidden:
         run_reference_proj(args, cores, cpu_model)
         return
     oracle.set_threads(cores)
@@ -994,11 +1137,15 @@ def run_reference_proj(args, cores, cpu_model):
     """The reference arm of the projection modes: the oracle's input_norm +
     qkv_proj (and, from the hidden state, the attention too), per step a
     bounded sample."""
-    mode = "qkv_proj" if args.op == "qkv_proj" else "from_hidden"
+    mode = args.op if args.op in ("qkv_proj", "o_proj") else "from_hidden"
     layers = make_layers(args.workload, "cpu", 0, args.num_q_heads, 1)
     for li, w in enumerate(layers):
-        w.hidden_in = inputs.hidden_inputs(w.batch, seed=7000 + li, device="cpu", hidden=args.hidden,
-                                           num_q_heads=args.num_q_heads)
+        if mode == "o_proj":
+            w.o_in = inputs.o_proj_inputs(w.batch, seed=8000 + li, device="cpu", hidden=args.hidden,
+                                          num_q_heads=args.num_q_heads)
+        else:
+            w.hidden_in = inputs.hidden_inputs(w.batch, seed=7000 + li, device="cpu", hidden=args.hidden,
+                                               num_q_heads=args.num_q_heads)
     budget = min(20.0, 120.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         cpu_baseline_proj(layers, mode, seconds=budget, threads=cores)
@@ -1006,7 +1153,8 @@ def run_reference_proj(args, cores, cpu_model):
     elapsed = sum(r["seconds"] for r in runs)
     value = sum(r["value"] * r["seconds"] for r in runs) / elapsed
     print(json.dumps({
-        "impl": "reference", "metric": PROJ_METRIC if mode == "qkv_proj" else METRIC, "value": round(value, 4),
+        "impl": "reference", "metric": {"qkv_proj": PROJ_METRIC, "o_proj": O_METRIC}.get(mode, METRIC),
+        "value": round(value, 4),
         "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(elapsed * 1e3 / args.steps, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; same recipe as the GPU arm, drawn on the host)",
@@ -1031,14 +1179,17 @@ def main(argv=None):
     ap.add_argument("--timing", choices=["graph", "eager"], default="graph",
                     help="timed region: CUDA graph replay of the steps (default) or eager launches with "
                          "an event pair around each; the line also carries the other figure")
-    ap.add_argument("--op", choices=["step", "qkv_proj"], default="step",
-                    help="step: the attention step (default); qkv_proj: input_norm + qkv_proj alone")
+    ap.add_argument("--op", choices=["step", "qkv_proj", "o_proj"], default="step",
+                    help="step: the attention step (default); qkv_proj: input_norm + qkv_proj alone; "
+                         "o_proj: attn.o_proj alone")
     ap.add_argument("--from-hidden", action="store_true",
                     help="each call starts from the hidden state: input_norm + qkv_proj, then the attention step")
     ap.add_argument("--hidden", type=int, default=inputs.HIDDEN,
                     help="hidden size of the projection modes (1024 for Qwen3-0.6B; 2560, 4096, 5120 for 4B/8B/14B-32B)")
     ap.add_argument("--rotate", type=int, default=0, help="resident input sets cycled (0: enough to defeat L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", dest="per_config", action="store_false",
+                    help="skip the other configurations the default 1-GPU run also times (per_config)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
