@@ -61,11 +61,12 @@ WORKLOADS = {
 # ----------------------------------------------------------------------------
 # workloads and byte counts
 
-def make_layers(name: str, device, rank: int = 0, num_q_heads: int = 16, new_tokens: int = 1):
+def make_layers(name: str, device, rank: int = 0, num_q_heads: int = 16, new_tokens: int = 1, layers: int = 0):
     """The layers of one step (one Workload per library call). num_q_heads picks the
     Qwen3 size: 16 (0.6B), 32 (4B/8B), 40 (14B) or 64 (32B); new_tokens > 1 gives
     every sequence that many new tokens (causal among themselves). cfg1 and cfg3
-    are 0.6B with one new token only."""
+    are 0.6B with one new token only. layers > 0 keeps only the first `layers`
+    layers of cfg3 (to profile one launch without holding all 28 layers)."""
     off = 100 * rank
     if name in ("cfg1", "cfg3") and (num_q_heads != 16 or new_tokens != 1):
         raise ValueError(f"{name} is defined for Qwen3-0.6B (16 query heads) and one new token")
@@ -74,7 +75,8 @@ def make_layers(name: str, device, rank: int = 0, num_q_heads: int = 16, new_tok
     if name == "cfg2":
         return [inputs.config2(device, seed=2000 + off, num_q_heads=num_q_heads, new_tokens=new_tokens)]
     if name == "cfg3":
-        return [inputs.config3_layer(i, device, seed=3000 + off) for i in range(inputs.CONFIG3_LAYERS)]
+        n = inputs.CONFIG3_LAYERS if layers <= 0 else min(layers, inputs.CONFIG3_LAYERS)
+        return [inputs.config3_layer(i, device, seed=3000 + off) for i in range(n)]
     if name == "cfg4":
         return [inputs.config4(device, seed=4000 + off, num_q_heads=num_q_heads, new_tokens=new_tokens)]
     if name == "cfg5":
@@ -135,6 +137,23 @@ def hbm_peak():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except (OSError, KeyError, ValueError):
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def n_chunks(args) -> int:
+    """Launches of the tensor-core attention kernel per call: a block of new
+    tokens longer than one launch takes (16 query rows per kv head) runs in chunks."""
+    T, G = args.new_tokens, args.num_q_heads // 8
+    max_t = 16 // G
+    if T <= max_t:
+        return 1
+    n, c0 = 0, 0
+    while c0 < T:
+        k = min(max_t, T - c0)
+        if args.num_q_heads == 16 and T - c0 - k == 1:
+            k -= 1
+        c0 += k
+        n += 1
+    return n
 
 
 def kernel_key(num_q_heads: int = 16, new_tokens: int = 1):
@@ -473,7 +492,7 @@ def measure(args, dist, rank, world, dev, headline: bool):
 
     # R resident copies of the step's inputs, so that a call never finds its
     # K/V in L2 from the previous call (each copy's KV is > L2 or R copies are).
-    first = make_layers(args.workload, dev, rank, args.num_q_heads, T)
+    first = make_layers(args.workload, dev, rank, args.num_q_heads, T, args.layers)
     hidden = args.hidden
     if mode == "attention":
         step_bytes = sum(kv_bytes(w.seq_lens) for w in first)
@@ -492,7 +511,8 @@ def measure(args, dist, rank, world, dev, headline: bool):
         import dataclasses
         sets = [first] + [[dataclasses.replace(w) for w in first] for r in range(1, rotate)]
     else:
-        sets = [first] + [make_layers(args.workload, dev, rank, args.num_q_heads, T) for r in range(1, rotate)]
+        sets = [first] + [make_layers(args.workload, dev, rank, args.num_q_heads, T, args.layers)
+                          for r in range(1, rotate)]
     if mode in ("qkv_proj", "from_hidden"):
         for si, layers in enumerate(sets):
             for li, w in enumerate(layers):
@@ -682,6 +702,8 @@ def measure(args, dist, rank, world, dev, headline: bool):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "io_dtype": "bf16", "data": "synthetic (seeded; N(0,1) bf16 qkv and cache, gains 1+U(-0.5,0.5))",
             "config": {"workload": f"{args.workload}: {WORKLOADS[args.workload]}"
+                                   + ("" if not (args.workload == "cfg3" and args.layers > 0)
+                                      else f" (first {calls_per_step} of the 28 layers only)")
                                    + ("" if args.num_q_heads == 16 else f", {args.num_q_heads} query heads")
                                    + ("" if T == 1 else f", {T} new tokens per sequence (causal among them)")
                                    + {"attention": "", "from_hidden": f", from the hidden state (input_norm + "
@@ -709,8 +731,11 @@ def measure(args, dist, rank, world, dev, headline: bool):
                       else "eager launches, an event pair around each; per-launch duration = mean of the pairs",
             ("eager" if args.timing == "graph" else "graph"): other,
             "seq_per_s": round(first[0].batch / (ms_per_step * 1e-3) * world, 1),
-            # attention: one launch per call; the projection: two (the split, the product); o_proj: one
-            "gpu_launches": n_launch * {"qkv_proj": 2, "o_proj": 1, "from_hidden": 3}.get(mode, 1),
+            # the 16-head attention: one launch per call, the tensor-core attention two (attention,
+            # combine; per chunk of a long block); the projection two (split, product), o_proj one
+            "gpu_launches": n_launch * ({"qkv_proj": 2, "o_proj": 1, "from_hidden": 2}.get(mode, 0)
+                                        + (0 if mode in ("qkv_proj", "o_proj") else
+                                           (1 if kernel_key(args.num_q_heads, T) == 16 else 2 * n_chunks(args)))),
             "clocks": clk,
         }
     if dist is not None:
@@ -1188,6 +1213,8 @@ def main(argv=None):
                     help="hidden size of the projection modes (1024 for Qwen3-0.6B; 2560, 4096, 5120 for 4B/8B/14B-32B)")
     ap.add_argument("--rotate", type=int, default=0, help="resident input sets cycled (0: enough to defeat L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="cfg3 only: time the first N of its 28 layers (0: all; for profiling one launch)")
     ap.add_argument("--no-per-config", dest="per_config", action="store_false",
                     help="skip the other configurations the default 1-GPU run also times (per_config)")
     args = ap.parse_args(argv)

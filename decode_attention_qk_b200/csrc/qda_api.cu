@@ -17,6 +17,7 @@ struct qda_handle {
     float* part_acc = nullptr;
     float2* part_ml = nullptr;
     int* counters = nullptr;
+    int* seg = nullptr;
     int* status = nullptr;
     // input_norm + qkv_proj: the exact split of x*g, and 1/r per row
     uint16_t* xg_hi = nullptr;
@@ -65,6 +66,7 @@ void free_workspace(qda_handle* h) {
     cudaFree(h->part_acc);
     cudaFree(h->part_ml);
     cudaFree(h->counters);
+    cudaFree(h->seg);
     cudaFree(h->status);
     cudaFree(h->xg_hi);
     cudaFree(h->xg_lo);
@@ -126,6 +128,7 @@ qda::Params make_params(const qda_handle* h, const void* qkv, const void* q_norm
     p.part_acc = h->part_acc;
     p.part_ml = h->part_ml;
     p.counters = h->counters;
+    p.seg = h->seg;
     p.status = h->status;
     p.timeout_ns = h->cfg.wait_timeout_ns > 0 ? h->cfg.wait_timeout_ns : kDefaultTimeoutNs;
     p.flags = h->cfg.flags;
@@ -244,7 +247,7 @@ int qwen3_decode_attn_create(const qda_config* cfg, int device, qda_handle** out
     bool ok = alloc(&h->part_acc, slots * rows * qda::kHeadDim * sizeof(float)) &&
               alloc(&h->part_ml, slots * rows * sizeof(float2)) &&
               alloc(&h->counters, (size_t)qda::kMaxBatch * qda::kNumKvHeads * sizeof(int)) &&
-              alloc(&h->status, sizeof(int)) &&
+              alloc(&h->status, sizeof(int)) && alloc(&h->seg, (size_t)(qda::kMaxBatch + 1) * sizeof(int)) &&
               alloc(&h->xg_hi, B * (size_t)qda::kMaxHidden * sizeof(uint16_t)) &&
               alloc(&h->xg_lo, B * (size_t)qda::kMaxHidden * sizeof(uint16_t)) &&
               alloc(&h->inv_r, B * sizeof(float));

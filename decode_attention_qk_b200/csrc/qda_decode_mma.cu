@@ -34,14 +34,14 @@
 //
 // Split sequences. The work split is the 16-head kernel's (equal page ranges
 // per CTA, scratch slot g + b per piece). A piece that covers its whole
-// sequence writes o; a piece of a split sequence writes its partial and
-// counts itself on the (sequence, kv head) counter with an acquiring atomic;
-// the warp whose piece arrives last merges all the pieces' partials with the
-// log-sum-exp rule (Supported models, "Facts proved about the specs":
-// flashAttn_eq, softmax_shift), reading them in slot order from L2, writes o
-// and resets the counter. One launch per call, a programmatic dependent
-// launch: it may start while the previous launch on the stream ends, and it
-// waits for that launch to complete before it touches global memory.
+// sequence writes o; a piece of a split sequence writes its partial, and a
+// second launch (one CTA per sequence and kv head, one warp per query row)
+// combines them with the log-sum-exp rule (Supported models, "Facts proved
+// about the specs": flashAttn_eq, softmax_shift), spreading long merges over
+// many SMs. Both launches are programmatic dependent launches: the combine
+// launch starts while the attention launch ends, and the attention launch
+// while the previous step's last launch ends; each waits for its predecessor
+// to complete before it touches global memory.
 #include <cuda_bf16.h>
 #include <cstdint>
 
@@ -81,18 +81,7 @@ struct Layout {
     static constexpr int kSmemGains = kSmemInvFreq + 64 * 8;                // bf16 [2][128]
     static constexpr int kSmemMeta = kSmemGains + 2 * kHeadDim * 2;         // StageMeta [kStages] + qkv position
     static constexpr int kSmemBars = kSmemMeta + (kStages + 1) * 16;        // full, empty, qkv_full, qkv_empty, never
-    static constexpr int kSmemMergeBars = kSmemBars + (2 * kStages + 3) * 8; // [8] merge copies, done
-    static constexpr int kSmemFlags = kSmemMergeBars + (kConsumerWarps + 1) * 8;
-    // Split pieces' partials, kv head major: row r of kv head j in scratch slot
-    // `slot` is row ((j * (grid + batch) + slot) * kRowPitch + r), so kv head
-    // j's rows of consecutive slots are contiguous; the pitch is even so that
-    // the (max, sum) pairs of a slot start on a 16-byte boundary.
-    static constexpr int kRowPitch = (kRows + 1) / 2 * 2;
-    // Merging: warp j uses its 1/8 of the idle ring; a batch of pieces is one
-    // bulk copy of their rows and one of their (max, sum) pairs.
-    static constexpr int kMergeRegion = kStages * kStageBytes / kConsumerWarps / 16 * 16;
-    static constexpr int kMergeBatch = kMergeRegion / (kRowPitch * (kHeadDim * 4 + 8));
-    static constexpr int kMergeMlOff = kMergeBatch * kRowPitch * kHeadDim * 4;
+    static constexpr int kSmemFlags = kSmemBars + (2 * kStages + 3) * 8;
     static constexpr int kSmemTotal = kSmemFlags + 16;
     // Up to 8 query rows per kv head, q and the probabilities enter the tensor
     // cores as two bf16 terms (value and remainder, rows r and r + 8 of the
@@ -102,16 +91,14 @@ struct Layout {
     static_assert(kRows <= 16, "at most 16 query rows per kv head");
     static_assert(!kWide || kDirectQkv, "wide instances read their qkv rows from global memory");
     static_assert(kSmemQkv % 16 == 0 && kSmemInvFreq % 8 == 0 && kSmemBars % 8 == 0, "alignment");
-    static_assert(kMergeBatch >= 1 && kMergeBatch <= 32 && kRowPitch <= 16, "merge batches");
     static_assert(kSmemTotal <= 227 * 1024, "fits one CTA per SM");
 };
 
 // Row of a split piece's partial: query row r (new token r / G, head
-// G*j + r % G) of kv head j in scratch slot `slot` (see Layout::kRowPitch).
+// G*j + r % G) of kv head j in scratch slot `slot`.
 template <int G, int T>
-__device__ __forceinline__ size_t part_row(const Params& p, int j, int slot, int r) {
-    const size_t stride = (size_t)gridDim.x + (size_t)p.batch;
-    return ((size_t)j * stride + (size_t)slot) * Layout<G, T>::kRowPitch + (size_t)r;
+__device__ __forceinline__ size_t part_row(int j, int slot, int r) {
+    return (size_t)slot * kPartRows + (size_t)(r / G) * Layout<G, T>::kHq + G * j + r % G;
 }
 
 // Row of qkv (and of o) holding new token u of sequence b: a call may cover
@@ -147,8 +134,6 @@ struct Shared {
     uint64_t* qkv_full;
     uint64_t* qkv_empty;
     uint64_t* never_bar;
-    uint64_t* merge_bar;  // [kConsumerWarps]: the merge copies of warp j
-    uint64_t* done_bar;   // every consumer warp is past its last page
     volatile int* abort_flag;
 };
 
@@ -565,143 +550,12 @@ __device__ __forceinline__ bool finish_piece(const Params& p, const Shared& s, i
             dst[4 * n + t] = pack_bf2((st.o[n][0] + st.o[n][2]) * inv, (st.o[n][1] + st.o[n][3]) * inv);
         return false;
     }
-    const size_t prow = part_row<G, T>(p, j, (int)blockIdx.x + b, r);
+    const size_t prow = part_row<G, T>(j, (int)blockIdx.x + b, r);
     float2* pa = reinterpret_cast<float2*>(p.part_acc + prow * kHeadDim);
 #pragma unroll
     for (int n = 0; n < 16; ++n) __stcg(pa + 4 * n + t, make_float2(st.o[n][0] + st.o[n][2], st.o[n][1] + st.o[n][3]));
     if (t == 0) __stcg(p.part_ml + prow, make_float2(st.m, l));
     return true;
-}
-
-// Bounded wait of a whole warp on `bar`; on expiry records QDA_ERR_TIMEOUT and
-// sets the CTA's abort flag.
-__device__ __forceinline__ bool warp_wait(const Params& p, const Shared& s, uint64_t* bar, uint32_t phase, int lane) {
-    bool ok = mbar_try_wait(bar, phase);
-    if (__all_sync(kFull, ok)) return true;
-    ok = ok || mbar_wait(bar, phase, p.timeout_ns, s.abort_flag);
-    ok = __all_sync(kFull, ok || mbar_try_wait(bar, phase));
-    if (!ok && lane == 0) {
-        *s.abort_flag = 1;
-        record_error(p.status, QDA_ERR_TIMEOUT);
-    }
-    return ok;
-}
-
-// Merge the partials of every piece of split sequence b for the query rows of
-// kv head j (this warp's piece was the last to arrive) and write o:
-// o = sum_t 2^(m_t - M) acc_t / sum_t 2^(m_t - M) l_t, M the running maximum
-// (log-sum-exp rule; Supported models, "Facts proved about the specs":
-// flashAttn_eq, softmax_shift). Pieces come in batches through this warp's
-// 1/8 of the idle ring: one bulk copy of their rows (contiguous, kv head
-// major) and one of their (max, sum) pairs, issued by the lane whose
-// acquiring increment completed the count; the batches are merged in slot
-// order with a rescale between them. Lane l handles dims 4l..4l+3 of every
-// row. Returns false when a wait ran out.
-template <int G, int T>
-__device__ __noinline__ bool merge_sequence(const Params& p, const Shared& s, int b, int j, int lane, int issuer,
-                                            int per_cta, uint32_t& mphase) {
-    using Lay = Layout<G, T>;
-    constexpr int R = Lay::kRows;
-    constexpr int RP = Lay::kRowPitch;
-    const int first = s.seg[b] / per_cta;
-    const int n = (s.seg[b + 1] - 1) / per_cta - first + 1;
-    uint8_t* region = s.stages + j * Lay::kMergeRegion;
-    uint64_t* bar = &s.merge_bar[j];
-    float M[R], L[R];
-    float4 A[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-        M[r] = -INFINITY;
-        L[r] = 0.f;
-        A[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    for (int t0 = 0; t0 < n; t0 += Lay::kMergeBatch) {
-        const int nb = min(Lay::kMergeBatch, n - t0);
-        // earlier reads of the region come before the copies that overwrite it
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == issuer) {
-            mbar_arrive_expect_tx(bar, (uint32_t)nb * RP * (kHeadDim * 4 + 8));
-            const size_t row = part_row<G, T>(p, j, first + b + t0, 0);
-            bulk_g2s(region, p.part_acc + row * kHeadDim, (uint32_t)nb * RP * kHeadDim * 4, bar);
-            bulk_g2s(region + Lay::kMergeMlOff, p.part_ml + row, (uint32_t)nb * RP * 8, bar);
-        }
-        if (!warp_wait(p, s, bar, mphase, lane)) {
-            // the copies may still be landing: wait once more (bounded) before leaving
-            if (lane == 0) (void)mbar_wait(bar, mphase, p.timeout_ns, nullptr);
-            __syncwarp();
-            return false;
-        }
-        mphase ^= 1u;
-        const float2* ml = reinterpret_cast<const float2*>(region + Lay::kMergeMlOff);   // [piece][RP]
-        const float4* acc = reinterpret_cast<const float4*>(region);                     // [piece][RP][32]
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            float bm = -INFINITY;
-            for (int t = 0; t < nb; ++t) bm = fmaxf(bm, ml[t * RP + r].x);
-            const float nM = fmaxf(M[r], bm);
-            // what the earlier batches summed, rescaled to the new maximum (nothing on the first)
-            const float sc = M[r] == -INFINITY ? 0.f : exp2_approx(M[r] - nM);
-            L[r] *= sc;
-            A[r].x *= sc;
-            A[r].y *= sc;
-            A[r].z *= sc;
-            A[r].w *= sc;
-            for (int t = 0; t < nb; ++t) {
-                const float2 v = ml[t * RP + r];
-                // a piece whose pages were all skipped has max -inf and weight 0
-                const float w = v.x == -INFINITY ? 0.f : exp2_approx(v.x - nM);
-                L[r] = fmaf(w, v.y, L[r]);
-                const float4 x = acc[(t * RP + r) * 32 + lane];
-                A[r].x = fmaf(w, x.x, A[r].x);
-                A[r].y = fmaf(w, x.y, A[r].y);
-                A[r].z = fmaf(w, x.z, A[r].z);
-                A[r].w = fmaf(w, x.w, A[r].w);
-            }
-            M[r] = nM;
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-        const float inv = L[r] > 0.f ? 1.f / L[r] : 0.f;
-        const int tt = r / G, head = G * j + r % G;
-        uint2 out;
-        out.x = pack_bf2(A[r].x * inv, A[r].y * inv);
-        out.y = pack_bf2(A[r].z * inv, A[r].w * inv);
-        reinterpret_cast<uint2*>(p.o + (token_row(p, b, tt) * Lay::kHq + head) * kHeadDim)[lane] = out;
-    }
-    if (lane == 0) p.counters[b * kNumKvHeads + j] = 0;   // ready for the next call
-    return true;
-}
-
-// End of a consumer warp's run: its split pieces' partials are stored (no
-// fence yet). Count them as done (lane 0: pending0, lane 1: pending1, with
-// acquiring atomics after one fence); the warp holding the last piece of a
-// sequence merges it through the ring, which every consumer warp has left by
-// then.
-template <int G, int T>
-__device__ __forceinline__ void arrive_pending(const Params& p, const Shared& s, int j, int lane, int per_cta,
-                                               int pending0, int pending1) {
-    __threadfence();   // this warp's partial stores before its arrivals
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-    const int npend = pending1 >= 0 ? 2 : 1;
-    const int mine = lane == 0 ? pending0 : pending1;
-    int prev = -1, need = 0;
-    if (lane < npend) {
-        need = (s.seg[mine + 1] - 1) / per_cta - s.seg[mine] / per_cta;
-        // acquire: the last to arrive sees every other piece's released partial
-        prev = atomic_add_acquire(p.counters + mine * kNumKvHeads + j, 1);
-    }
-    const bool last0 = __shfl_sync(kFull, prev == need, 0);
-    const bool last1 = __shfl_sync(kFull, prev == need, 1) && npend == 2;
-    if (!last0 && !last1) return;
-    // the other pieces' partials are read through the async proxy by bulk
-    // copies, issued by the lane whose acquiring increment found the count complete
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-    if (!warp_wait(p, s, s.done_bar, 0u, lane)) return;
-    uint32_t mphase = 0;
-    if (last0 && !merge_sequence<G, T>(p, s, pending0, j, lane, 0, per_cta, mphase)) return;
-    if (last1) (void)merge_sequence<G, T>(p, s, pending1, j, lane, 1, per_cta, mphase);
 }
 
 // ---------------------------------------------------------------------------
@@ -1010,7 +864,7 @@ __device__ __forceinline__ bool finish_piece_wide(const Params& p, const Shared&
 #pragma unroll
             for (int n = 0; n < 16; ++n) dst[4 * n + t] = pack_bf2(st.o[n][2 * h] * inv, st.o[n][2 * h + 1] * inv);
         } else {
-            const size_t prow = part_row<G, T>(p, j, (int)blockIdx.x + b, r);
+            const size_t prow = part_row<G, T>(j, (int)blockIdx.x + b, r);
             float2* pa = reinterpret_cast<float2*>(p.part_acc + prow * kHeadDim);
 #pragma unroll
             for (int n = 0; n < 16; ++n) __stcg(pa + 4 * n + t, make_float2(st.o[n][2 * h], st.o[n][2 * h + 1]));
@@ -1034,7 +888,6 @@ __device__ __forceinline__ void run_consumer_wide(const Params& p, const Shared&
     uint32_t phase = 0;
     const int count = end - start;
     int k = 0;
-    int pending0 = -1, pending1 = -1;   // split pieces whose arrival waits for the end
     bool aborted = false;
     while (k < count && !aborted) {
         const int nb = s.seg[b + 1] - s.seg[b];
@@ -1058,18 +911,12 @@ __device__ __forceinline__ void run_consumer_wide(const Params& p, const Shared&
         }
         if (aborted) break;
         k += n_here;
-        if (finish_piece_wide<G, T>(p, s, b, j, lane, per_cta, st)) {
-            if (pending0 < 0) pending0 = b;
-            else pending1 = b;
-        }
+        (void)finish_piece_wide<G, T>(p, s, b, j, lane, per_cta, st);
         if (k < count) {
             do { ++b; } while (b < B && s.seg[b + 1] == s.seg[b]);
             i0 = 0;
         }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(s.done_bar);   // this warp no longer reads the ring
-    if (!aborted && pending0 >= 0) arrive_pending<G, T>(p, s, j, lane, per_cta, pending0, pending1);
 }
 
 template <int G, int T>
@@ -1086,7 +933,6 @@ __device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, i
     uint32_t phase = 0, qphase = 0;
     const int count = end - start;
     int k = 0;
-    int pending0 = -1, pending1 = -1;   // split pieces whose arrival waits for the end
     bool aborted = false;
     while (k < count && !aborted) {
         const int nb = s.seg[b + 1] - s.seg[b];
@@ -1121,18 +967,12 @@ __device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, i
         }
         if (aborted) break;
         k += n_here;
-        if (finish_piece<G, T>(p, s, b, j, lane, per_cta, st)) {
-            if (pending0 < 0) pending0 = b;
-            else pending1 = b;
-        }
+        (void)finish_piece<G, T>(p, s, b, j, lane, per_cta, st);
         if (k < count) {
             do { ++b; } while (b < B && s.seg[b + 1] == s.seg[b]);
             i0 = 0;
         }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(s.done_bar);   // this warp no longer reads the ring
-    if (!aborted && pending0 >= 0) arrive_pending<G, T>(p, s, j, lane, per_cta, pending0, pending1);
 }
 
 template <int G, int T>
@@ -1157,15 +997,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
     s.qkv_full = s.empty_bar + kStages;
     s.qkv_empty = s.qkv_full + 1;
     s.never_bar = s.qkv_empty + 1;
-    s.merge_bar = reinterpret_cast<uint64_t*>(smem + Lay::kSmemMergeBars);
-    s.done_bar = s.merge_bar + kConsumerWarps;
     s.abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kSmemFlags);
 
-    // Launched as a programmatic dependent launch: the next launch may be
-    // scheduled now; the prologue below touches no global memory, and
-    // griddepcontrol.wait holds until the previous launch on the stream has
-    // completed and its writes are visible.
-    pdl_launch_dependents();
+    // Launched as a programmatic dependent launch: the prologue below touches
+    // no global memory, and griddepcontrol.wait holds until the previous
+    // launch on the stream has completed and its writes are visible.
     if (threadIdx.x >= 64 && threadIdx.x < 128) {
         const int i = threadIdx.x - 64;
         s.inv_freq[i] = pow(p.rope_theta, -2.0 * i / 128.0);
@@ -1178,8 +1014,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
         mbar_init(s.qkv_full, 1);
         mbar_init(s.qkv_empty, kConsumerWarps);
         mbar_init(s.never_bar, 1);
-        for (int k = 0; k < kConsumerWarps; ++k) mbar_init(&s.merge_bar[k], 1);
-        mbar_init(s.done_bar, kConsumerWarps);
         *s.abort_flag = 0;
         s.seg[0] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -1226,6 +1060,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
         }
     }
     __syncthreads();
+    if (blockIdx.x == 0)   // page offsets for the combine launch
+        for (int b = threadIdx.x; b <= B; b += kThreads) p.seg[b] = s.seg[b];
 
     const int total = s.seg[B];
     const int per_cta = (total + (int)gridDim.x - 1) / (int)gridDim.x;
@@ -1239,6 +1075,72 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
     if ((p.flags & QDA_FLAG_INJECT_WAIT_TIMEOUT) != 0u && blockIdx.x == 0 && warp == 0) {
         if (!mbar_wait(s.never_bar, 0u, p.timeout_ns, nullptr) && lane == 0) record_error(p.status, QDA_ERR_TIMEOUT);
     }
+    pdl_launch_dependents();
+}
+
+// Combine the partials of one split sequence (blockIdx.x) for the query rows
+// of one kv head (blockIdx.y): warp w handles query row w (new token w / G,
+// head G*y + w % G), and lane l its dims 4l..4l+3; o = sum_t 2^(m_t - M)
+// acc_t / sum_t 2^(m_t - M) l_t with M = max_t m_t (log-sum-exp rule;
+// Supported models, "Facts proved about the specs": flashAttn_eq,
+// softmax_shift). Sequences held whole by one CTA were written by the first
+// launch and are skipped. Spreading the merges over a CTA per (sequence, kv
+// head) keeps each SM's share of the partials' reads small.
+template <int G, int T>
+__global__ void __launch_bounds__(32 * G * T, 1) combine_kernel(const Params p, int main_grid) {
+    using Lay = Layout<G, T>;
+    pdl_wait();   // the first launch has finished and its writes are visible
+    pdl_launch_dependents();   // the next step's attention launch may be scheduled
+    const int b = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tt = warp / G;
+    const int h = G * blockIdx.y + warp % G;
+    const int lo = p.seg[b], hi = p.seg[b + 1], total = p.seg[p.batch];
+    if (hi == lo) return;   // a sequence the first launch skipped
+    const int per_cta = (total + main_grid - 1) / main_grid;
+    const int first = lo / per_cta, n = (hi - 1) / per_cta - first + 1;
+    if (n == 1) return;
+    const size_t row0 = part_row<G, T>((int)blockIdx.y, first + b, warp);   // piece t at row0 + t*kPartRows
+    const float2* ml = p.part_ml + row0;
+    float M = -INFINITY;
+    for (int t = lane; t < n; t += 32) M = fmaxf(M, __ldcg(ml + (size_t)t * kPartRows).x);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+    const float4* src = reinterpret_cast<const float4*>(p.part_acc + row0 * kHeadDim) + lane;
+    constexpr size_t kSlotStride = (size_t)kPartRows * kHeadDim / 4;   // float4 per scratch slot
+    float Ls = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int t0 = 0; t0 < n; t0 += 32) {
+        float wt = 0.f;
+        if (t0 + lane < n) {
+            const float2 v = __ldcg(ml + (size_t)(t0 + lane) * kPartRows);
+            wt = (v.x == -INFINITY) ? 0.f : exp2_approx(v.x - M);   // a piece whose pages were all skipped
+            Ls = fmaf(wt, v.y, Ls);
+        }
+        const int m = min(32, n - t0);
+        for (int u0 = 0; u0 < m; u0 += 8) {
+            float4 x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (u0 + u < m) x[u] = __ldcg(src + (size_t)(t0 + u0 + u) * kSlotStride);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float w = __shfl_sync(kFull, wt, (u0 + u) & 31);
+                if (u0 + u < m) {
+                    acc.x = fmaf(w, x[u].x, acc.x);
+                    acc.y = fmaf(w, x[u].y, acc.y);
+                    acc.z = fmaf(w, x[u].z, acc.z);
+                    acc.w = fmaf(w, x[u].w, acc.w);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) Ls += __shfl_xor_sync(kFull, Ls, off);
+    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+    uint2 out;
+    out.x = pack_bf2(acc.x * inv, acc.y * inv);
+    out.y = pack_bf2(acc.z * inv, acc.w * inv);
+    reinterpret_cast<uint2*>(p.o + (token_row(p, b, tt) * Lay::kHq + h) * kHeadDim)[lane] = out;
 }
 
 template <int G, int T>
@@ -1259,7 +1161,16 @@ cudaError_t launch_one(const Params& p, int grid, cudaStream_t stream) {
     main.stream = stream;
     main.attrs = attr;
     main.numAttrs = 1;
-    return cudaLaunchKernelEx(&main, grouped_attention_kernel<G, T>, p);
+    cudaError_t e = cudaLaunchKernelEx(&main, grouped_attention_kernel<G, T>, p);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.batch, (unsigned)kNumKvHeads, 1);
+    cfg.blockDim = dim3(32 * G * T, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, combine_kernel<G, T>, p, grid);
 }
 
 }  // namespace

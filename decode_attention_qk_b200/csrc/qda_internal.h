@@ -58,6 +58,8 @@ struct Params {
                                   // 16-head kernel (ordered kv head, slot, head pair there), kPartRows
                                   // for the tensor-core kernel
     float2* part_ml;              // [num_slots][rows] (running max in log2 units, sum), same row order
+    int* seg;                     // [kMaxBatch + 1] page offsets of the sequences (written for the combine
+                                  // launch of the tensor-core kernel; unused at 16 heads)
     int* counters;                // [kMaxBatch][8] merge arrival counters, zero between calls
     int* status;                  // sticky device error (0 = none)
     int64_t timeout_ns;           // limit of every device-side wait
@@ -88,8 +90,8 @@ cudaError_t prepare_device();
 cudaError_t launch(const Params& p, int grid, cudaStream_t stream, bool after_producer = false);
 
 // The tensor-core step (32, 40 or 64 query heads with one new token; T new
-// tokens with T * Hq / 8 <= 16 query rows per kv head): one launch, which
-// also combines the partials of sequences split across CTAs.
+// tokens with T * Hq / 8 <= 16 query rows per kv head): the attention launch,
+// then a launch that combines the partials of sequences split across CTAs.
 cudaError_t launch_grouped(const Params& p, int grid, cudaStream_t stream);
 
 // input_norm + attn.qkv_proj (qda_qkv_proj.cu): hidden size a multiple of 512,

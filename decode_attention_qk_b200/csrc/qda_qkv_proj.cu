@@ -20,7 +20,7 @@
 //   transposed, D[n][b] = sum_k W[n][k] (hi[b][k] + lo[b][k]), with the 128
 //   weight rows as the A operand (M = 128) and C <= 64 batch rows as the B
 //   operand (N = C). A producer thread streams 128 x 64 weight boxes and the
-//   matching C x 64 boxes of hi and lo into a 6-stage shared ring by tiled
+//   matching C x 64 boxes of hi and lo into a 5-stage shared ring by tiled
 //   copies with the 128-byte swizzle; one thread issues tcgen05.mma (two per
 //   16-wide K step: hi, then lo, into the same accumulator) and frees each
 //   stage with tcgen05.commit; the accumulator lives in tensor memory and the
@@ -30,10 +30,11 @@
 //   of at most 64 rows, and the K range in P = 1, 2, 4 or 8 parts, the
 //   fewest that keep at least 80% of the SMs busy (at 0.6B: P = 4 for
 //   qkv_proj up to 64 rows, giving 128 CTAs; P = 1 at 256 rows). The P parts
-//   of a tile form a thread-block cluster; after the products, CTA q of the
-//   cluster adds the P partial tiles of rows [q * 128/P, (q+1) * 128/P) in
-//   part order, reading its peers' shared memory (distributed shared
-//   memory), so the result does not depend on timing.
+//   of a tile form a thread-block cluster. CTA q of the cluster owns rows
+//   [q * 128/P, (q+1) * 128/P) of the tile: after the products every CTA
+//   writes its partial values of those rows into CTA q's shared memory
+//   (distributed shared-memory stores), and after one cluster barrier CTA q
+//   adds the P parts in part order, so the result does not depend on timing.
 //
 // The product launch is a programmatic dependent of the first: it allocates
 // tensor memory and issues its first weight copies before it waits for the
@@ -65,18 +66,23 @@ constexpr int kPrepThreads = 128;
 constexpr int kLinThreads = 128;                      // 4 warps: producer, MMA issuer, and all four for the epilogue
 constexpr int kLinM = 128;                            // weight rows per CTA (the instruction's M)
 constexpr int kLinKC = 64;                            // K per stage: one 128-byte swizzle row
-constexpr int kLinStages = 6;
+constexpr int kLinStages = 5;
 constexpr int kLinMaxCols = 64;                       // batch rows per CTA (the instruction's N)
 constexpr int kLinABytes = kLinM * kLinKC * 2;        // 16 KiB of weight per stage
 constexpr int kLinBBytes = 2 * kLinMaxCols * kLinKC * 2;   // hi and lo boxes: up to 16 KiB
 constexpr int kLinStageBytes = kLinABytes + kLinBBytes;
-constexpr int kLinSmemBars = kLinStages * kLinStageBytes;   // full[S], empty[S], acc, tmem address, abort
+// After the ring: the output tile [K part][cols][rows of the part] (float)
+// that the cluster's CTAs write into the owner of the rows, the row scales,
+// then the barriers.
+constexpr int kLinSmemTile = kLinStages * kLinStageBytes;
+constexpr int kLinTileBytes = kLinMaxCols * kLinM * 4;      // 32 KiB: every part's share of one CTA's rows
+constexpr int kLinSmemScale = kLinSmemTile + kLinTileBytes;  // float [kLinMaxCols]
+constexpr int kLinSmemBars = kLinSmemScale + kLinMaxCols * 4;   // full[S], empty[S], acc, tmem address, abort
 constexpr int kLinSmemUsed = kLinSmemBars + (2 * kLinStages + 1) * 8 + 16;
 constexpr int kLinSmemTotal = kLinSmemUsed + 1024;    // slack to align the ring to 1024 bytes
 constexpr uint32_t kLinTmemCols = 64;
 static_assert(kLinStageBytes % 1024 == 0 && kLinABytes % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
 static_assert(kLinSmemTotal <= 227 * 1024, "fits one CTA per SM");
-static_assert(kLinMaxCols * kLinM * 4 <= kLinSmemBars, "the partial tile fits in the drained ring");
 
 // The exact split of the products x*g of one 16-byte piece (8 values): hi, lo
 // words, and the squares of x added to ss.
@@ -170,8 +176,12 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     const uint32_t term_bytes = (uint32_t)p.cols * kLinKC * 2;
     const uint32_t stage_tx = (uint32_t)kLinABytes + (p.two_terms ? 2u : 1u) * term_bytes;
 
-    if (warp == 0) tmem_alloc(tmem_slot, kLinTmemCols);
-    if (threadIdx.x == 32) {
+    float* scale_s = reinterpret_cast<float*>(smem + kLinSmemScale);
+    const int pre = min(kLinStages, chunks);
+    if (threadIdx.x == 0) {
+        // the barriers, then at once the weight boxes of the first round (they
+        // need nothing from the previous launch), while warp 1 allocates the
+        // accumulator
         for (int s = 0; s < kLinStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
@@ -179,23 +189,22 @@ __global__ void __launch_bounds__(kLinThreads, 1)
         mbar_init(acc_bar, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        tma_prefetch_desc(&tm_w);
+        for (int c = 0; c < pre; ++c) {
+            mbar_arrive_expect_tx(&full[c], stage_tx);
+            tma_load_2d(ring + c * kLinStageBytes, &tm_w, (c0 + c) * kLinKC, n0, &full[c]);
+        }
     }
+    if (warp == 1) tmem_alloc(tmem_slot, kLinTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
 
     if (warp == 0 && lane == 0) {
-        // Producer. The weight boxes of the first round need nothing from the
-        // previous launch; the activation boxes wait for it.
-        tma_prefetch_desc(&tm_w);
+        // Producer: the activation boxes wait for the previous launch.
         tma_prefetch_desc(&tm_hi);
         if (p.two_terms) tma_prefetch_desc(&tm_lo);
-        const int pre = min(kLinStages, chunks);
-        for (int c = 0; c < pre; ++c) {
-            mbar_arrive_expect_tx(&full[c], stage_tx);
-            tma_load_2d(ring + c * kLinStageBytes, &tm_w, (c0 + c) * kLinKC, n0, &full[c]);
-        }
         if (p.wait_acts) {
             pdl_wait();
             asm volatile("fence.proxy.async.global;" ::: "memory");   // the copies read what it wrote
@@ -238,67 +247,75 @@ __global__ void __launch_bounds__(kLinThreads, 1)
             umma_commit(&empty[s]);   // the stage is free once these products have read it
         }
         umma_commit(acc_bar);         // every product issued above has completed
+    } else if (warp >= 2) {
+        // the row scales of this CTA's batch rows (from the previous launch)
+        if (p.wait_acts) pdl_wait();
+        for (int j = threadIdx.x - 64; j < p.cols; j += kLinThreads - 64) {
+            const int b = b0 + j;
+            scale_s[j] = (p.row_scale != nullptr && b < p.batch) ? __ldg(p.row_scale + b) : 1.f;
+        }
     }
     __syncwarp();
 
-    // Epilogue: warp w holds tensor-memory lanes 32w..32w+31 = weight rows n0 + 32w + lane.
+    // Epilogue: warp w holds tensor-memory lanes 32w..32w+31 = weight rows
+    // n0 + 32w + lane. Each CTA owns rows [part*R, part*R + R) of the tile,
+    // R = 128 / k_split; every CTA of the cluster writes its partial values of
+    // those rows into the owner's tile region, [part][cols][R] (distributed
+    // shared-memory stores, which do not wait for an answer); after one
+    // cluster barrier each owner adds the parts in part order from its own
+    // shared memory, scales, rounds and stores 8 rows (16 bytes) at a time.
     const bool ok = lin_wait(acc_bar, 0u, p, abort_flag) && *abort_flag == 0;
     tc_fence_after();
-    if (p.wait_acts) pdl_wait();     // the row scales come from the previous launch
+    const int rows = kLinM / p.k_split;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
-    if (p.k_split == 1) {
-        const int n = n0 + 32 * warp + lane;
+    {
+        const int r = 32 * warp + lane;
+        const int owner = r / rows, rr = r % rows;
+        float* dst = reinterpret_cast<float*>(smem + kLinSmemTile);
+        if (p.k_split > 1) {
+            namespace cg = cooperative_groups;
+            dst = cg::this_cluster().map_shared_rank(dst, owner);
+        }
+        dst += (size_t)part * p.cols * rows + rr;
         for (int j0 = 0; j0 < p.cols && ok; j0 += 16) {
             uint32_t v[16];
             tmem_ld16(lane_base + (uint32_t)j0, v);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int b = b0 + j0 + i;
-                if (b < p.batch) {
-                    const float sc = p.row_scale != nullptr ? __ldg(p.row_scale + b) : 1.f;
-                    p.y[(size_t)b * p.n_out + n] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[i]) * sc));
-                }
-            }
+            for (int i = 0; i < 16; ++i) dst[(j0 + i) * rows] = __uint_as_float(v[i]);
         }
-    } else {
-        // the partial tile [cols][128] (float) in the drained ring, then the
-        // cluster's parts are added in part order, rows [q*R, q*R + R) by part q
-        float* tile = reinterpret_cast<float*>(smem);
-        for (int j0 = 0; j0 < p.cols && ok; j0 += 16) {
-            uint32_t v[16];
-            tmem_ld16(lane_base + (uint32_t)j0, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) tile[(j0 + i) * kLinM + 32 * warp + lane] = __uint_as_float(v[i]);
-        }
-        tc_fence_before();
-        cluster_sync_all();   // every part's tile is in place
-        namespace cg = cooperative_groups;
-        cg::cluster_group cluster = cg::this_cluster();
-        const int rows = kLinM / p.k_split;
-        const int r0 = part * rows;
-        const int pairs = rows / 2;
-        for (int e = threadIdx.x; e < pairs * p.cols; e += kLinThreads) {
-            const int j = e / pairs, row = r0 + 2 * (e % pairs);
-            const int b = b0 + j;
-            float2 sum = make_float2(0.f, 0.f);
-            for (int q = 0; q < p.k_split; ++q) {
-                const float* peer = cluster.map_shared_rank(tile, q);
-                const float2 v = *reinterpret_cast<const float2*>(peer + j * kLinM + row);
-                sum.x += v.x;
-                sum.y += v.y;
-            }
-            if (b < p.batch && *abort_flag == 0) {
-                const float sc = p.row_scale != nullptr ? __ldg(p.row_scale + b) : 1.f;
-                *reinterpret_cast<uint32_t*>(p.y + (size_t)b * p.n_out + n0 + row) = pack_bf2(sum.x * sc, sum.y * sc);
-            }
-        }
-        cluster_sync_all();   // peers may still be reading this CTA's tile
     }
     tc_fence_before();
+    if (p.k_split > 1) cluster_sync_all();   // every part's values are in their owners' tiles (and the scales)
+    else __syncthreads();
+    {
+        const float* tile = reinterpret_cast<const float*>(smem + kLinSmemTile);
+        const int oct = rows / 8;
+        for (int e = threadIdx.x; e < oct * p.cols; e += kLinThreads) {
+            const int j = e / oct, rr = 8 * (e % oct);
+            const int b = b0 + j;
+            float acc[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+            for (int q = 0; q < p.k_split; ++q) {
+                const float4* src = reinterpret_cast<const float4*>(tile + ((size_t)q * p.cols + j) * rows + rr);
+                const float4 x0 = src[0], x1 = src[1];
+                acc[0] += x0.x; acc[1] += x0.y; acc[2] += x0.z; acc[3] += x0.w;
+                acc[4] += x1.x; acc[5] += x1.y; acc[6] += x1.z; acc[7] += x1.w;
+            }
+            if (b < p.batch && *abort_flag == 0) {
+                const float sc = scale_s[j];
+                uint4 w;
+                w.x = pack_bf2(acc[0] * sc, acc[1] * sc);
+                w.y = pack_bf2(acc[2] * sc, acc[3] * sc);
+                w.z = pack_bf2(acc[4] * sc, acc[5] * sc);
+                w.w = pack_bf2(acc[6] * sc, acc[7] * sc);
+                *reinterpret_cast<uint4*>(p.y + (size_t)b * p.n_out + n0 + part * rows + rr) = w;
+            }
+        }
+    }
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kLinTmemCols);
     }

@@ -143,8 +143,9 @@ void qwen3_decode_attn_default_config(qda_config *cfg);
 int qwen3_decode_attn_create(const qda_config *cfg, int device, qda_handle **out);
 
 /* The decode-attention step on device buffers (layouts above, with the
- * handle's Hq). One kernel launch: sequences whose pages are split across
- * CTAs are combined inside it by the CTA finishing last. Every pointer is a
+ * handle's Hq). At 16 query heads it is one kernel launch (sequences whose
+ * pages are split across CTAs are combined inside it); at 32, 40 or 64 a
+ * second launch combines them. Every pointer is a
  * device pointer. qkv, k_cache, v_cache and o must be 16-byte aligned;
  * q_norm_w, k_norm_w, seq_lens, positions and block_table 4-byte aligned.
  * `batch` is B (1..max_batch); `num_pages` (>= 1) bounds every block-table
@@ -192,7 +193,9 @@ int qwen3_decode_attn_append_and_attend(qda_handle *h,
  * causal attention (a chunked prefill; each launch reads the sequence's whole
  * cache again). Up to 8 query rows per kv head q and the probabilities enter
  * the tensor cores as two bf16 terms (about 16 significant bits); with 9 to
- * 16 rows they enter as bf16 (8 bits), with float sums either way.
+ * 16 rows they enter as bf16 (8 bits), with float sums either way. Each
+ * launch of the tensor-core kernel is followed by one that combines the
+ * sequences split across CTAs.
  * Errors as for qwen3_decode_attn_append_and_attend, plus INVALID_ARG for
  * new_tokens outside [1, min(QDA_MAX_NEW_TOKENS, max_seq_len)]; on the
  * device, a seq_len below T is out of range like one above the limits. */
