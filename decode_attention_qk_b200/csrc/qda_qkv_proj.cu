@@ -32,11 +32,13 @@
 //   qkv_proj up to 64 rows, giving 128 CTAs; P = 1 at 256 rows). The P parts
 //   of a tile form a thread-block cluster. CTA q of the cluster owns rows
 //   [q * 128/P, (q+1) * 128/P) of the tile: after the products every CTA
-//   writes its partial values of those rows into CTA q's shared memory
-//   (distributed shared-memory stores), and after one cluster barrier CTA q
-//   adds the P parts in part order, so the result does not depend on timing.
+//   sends its partial values of those rows into CTA q's shared memory with
+//   asynchronous stores that complete on CTA q's tile barrier, and CTA q,
+//   once its barrier has seen all their bytes, adds the P parts in part
+//   order, so the result does not depend on timing.
 //
-// The product launch is a programmatic dependent of the first: it allocates
+// Both launches are programmatic dependents of the launch before them. The
+// first waits for its predecessor before it reads x; the product allocates
 // tensor memory and issues its first weight copies before it waits for the
 // first launch's hi, lo and 1/r.
 //
@@ -49,7 +51,6 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
-#include <cooperative_groups.h>
 #include <cstdint>
 #include <mutex>
 
@@ -77,8 +78,8 @@ constexpr int kLinStageBytes = kLinABytes + kLinBBytes;
 constexpr int kLinSmemTile = kLinStages * kLinStageBytes;
 constexpr int kLinTileBytes = kLinMaxCols * kLinM * 4;      // 32 KiB: every part's share of one CTA's rows
 constexpr int kLinSmemScale = kLinSmemTile + kLinTileBytes;  // float [kLinMaxCols]
-constexpr int kLinSmemBars = kLinSmemScale + kLinMaxCols * 4;   // full[S], empty[S], acc, tmem address, abort
-constexpr int kLinSmemUsed = kLinSmemBars + (2 * kLinStages + 1) * 8 + 16;
+constexpr int kLinSmemBars = kLinSmemScale + kLinMaxCols * 4;   // full[S], empty[S], acc, tile, tmem address, abort
+constexpr int kLinSmemUsed = kLinSmemBars + (2 * kLinStages + 2) * 8 + 16;
 constexpr int kLinSmemTotal = kLinSmemUsed + 1024;    // slack to align the ring to 1024 bytes
 constexpr uint32_t kLinTmemCols = 64;
 static_assert(kLinStageBytes % 1024 == 0 && kLinABytes % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
@@ -114,6 +115,7 @@ __device__ __forceinline__ float warp_sum_f(float v) {
 
 __global__ void __launch_bounds__(kPrepThreads) input_norm_split_kernel(const QkvProjParams p) {
     pdl_launch_dependents();   // the product may start streaming the weight now
+    pdl_wait();                // x may come from the launch before this one
     const int b = blockIdx.x;
     const uint4* xr = reinterpret_cast<const uint4*>(p.x + (size_t)b * p.hidden);
     const uint4* gr = reinterpret_cast<const uint4*>(p.norm_w);
@@ -163,7 +165,8 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kLinSmemBars);
     uint64_t* empty = full + kLinStages;
     uint64_t* acc_bar = empty + kLinStages;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_bar + 1);
+    uint64_t* tile_bar = acc_bar + 1;   // the cluster peers' partial values have landed in the tile
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     pdl_launch_dependents();   // a launch consuming this result may be scheduled now
@@ -175,6 +178,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     const int c0 = part * chunks;
     const uint32_t term_bytes = (uint32_t)p.cols * kLinKC * 2;
     const uint32_t stage_tx = (uint32_t)kLinABytes + (p.two_terms ? 2u : 1u) * term_bytes;
+    const int rows = kLinM / p.k_split;   // the rows of the tile this CTA owns
 
     float* scale_s = reinterpret_cast<float*>(smem + kLinSmemScale);
     const int pre = min(kLinStages, chunks);
@@ -187,8 +191,11 @@ __global__ void __launch_bounds__(kLinThreads, 1)
             mbar_init(&empty[s], 1);
         }
         mbar_init(acc_bar, 1);
+        mbar_init(tile_bar, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        // the bytes the other K parts will store into this CTA's tile
+        if (p.k_split > 1) mbar_arrive_expect_tx(tile_bar, (uint32_t)((p.k_split - 1) * p.cols * rows * 4));
         tma_prefetch_desc(&tm_w);
         for (int c = 0; c < pre; ++c) {
             mbar_arrive_expect_tx(&full[c], stage_tx);
@@ -196,6 +203,8 @@ __global__ void __launch_bounds__(kLinThreads, 1)
         }
     }
     if (warp == 1) tmem_alloc(tmem_slot, kLinTmemCols);
+    // the peers may store into this CTA's tile once their wait on this arrival ends
+    if (p.k_split > 1) cluster_arrive_relaxed();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -259,35 +268,55 @@ __global__ void __launch_bounds__(kLinThreads, 1)
 
     // Epilogue: warp w holds tensor-memory lanes 32w..32w+31 = weight rows
     // n0 + 32w + lane. Each CTA owns rows [part*R, part*R + R) of the tile,
-    // R = 128 / k_split; every CTA of the cluster writes its partial values of
-    // those rows into the owner's tile region, [part][cols][R] (distributed
-    // shared-memory stores, which do not wait for an answer); after one
-    // cluster barrier each owner adds the parts in part order from its own
-    // shared memory, scales, rounds and stores 8 rows (16 bytes) at a time.
-    const bool ok = lin_wait(acc_bar, 0u, p, abort_flag) && *abort_flag == 0;
+    // R = 128 / k_split, laid out [part][cols][R]; every CTA of the cluster
+    // stores its partial values of those rows into the owner's tile with
+    // asynchronous stores that complete their bytes on the owner's tile
+    // barrier (a CTA that gave up stores zeros, so that no owner waits in
+    // vain). Each owner waits on its own barrier only, then adds the parts in
+    // part order, scales, rounds and stores 8 rows (16 bytes) at a time.
+    // (warp-uniform: tcgen05.ld is a whole-warp instruction)
+    const bool ok = __all_sync(kFull, lin_wait(acc_bar, 0u, p, abort_flag) && *abort_flag == 0);
     tc_fence_after();
-    const int rows = kLinM / p.k_split;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
     {
         const int r = 32 * warp + lane;
         const int owner = r / rows, rr = r % rows;
-        float* dst = reinterpret_cast<float*>(smem + kLinSmemTile);
-        if (p.k_split > 1) {
-            namespace cg = cooperative_groups;
-            dst = cg::this_cluster().map_shared_rank(dst, owner);
-        }
-        dst += (size_t)part * p.cols * rows + rr;
-        for (int j0 = 0; j0 < p.cols && ok; j0 += 16) {
+        float* tile = reinterpret_cast<float*>(smem + kLinSmemTile);
+        const uint32_t elem = smem_addr(tile + (size_t)part * p.cols * rows + rr);
+        if (p.k_split > 1) cluster_wait();   // every peer's tile barrier is initialised (warp converged here)
+        const bool local = owner == part;
+        const uint32_t dst = local ? elem : cluster_map(elem, (uint32_t)owner);
+        const uint32_t dst_bar = local ? 0u : cluster_map(smem_addr(tile_bar), (uint32_t)owner);
+        for (int j0 = 0; j0 < p.cols; j0 += 16) {
             uint32_t v[16];
-            tmem_ld16(lane_base + (uint32_t)j0, v);
-            tmem_ld_wait();
+            if (ok) {
+                tmem_ld16(lane_base + (uint32_t)j0, v);
+                tmem_ld_wait();
+            } else {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) dst[(j0 + i) * rows] = __uint_as_float(v[i]);
+                for (int i = 0; i < 16; ++i) v[i] = 0u;
+            }
+            if (local) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) tile[((size_t)part * p.cols + j0 + i) * rows + rr] = __uint_as_float(v[i]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    st_async_f32(dst + (uint32_t)((j0 + i) * rows * 4), __uint_as_float(v[i]), dst_bar);
+            }
         }
     }
     tc_fence_before();
-    if (p.k_split > 1) cluster_sync_all();   // every part's values are in their owners' tiles (and the scales)
-    else __syncthreads();
+    __syncthreads();   // this CTA's own part is in the tile
+    if (p.k_split > 1) {
+        // the other parts: a bounded wait that does not give up on this CTA's
+        // abort flag, since their stores land here whatever this CTA did
+        if (threadIdx.x == 0 && !mbar_wait(tile_bar, 0u, p.timeout_ns, nullptr)) {
+            *abort_flag = 1;
+            record_error(p.status, QDA_ERR_TIMEOUT);
+        }
+        __syncthreads();
+    }
     {
         const float* tile = reinterpret_cast<const float*>(smem + kLinSmemTile);
         const int oct = rows / 8;
@@ -423,8 +452,17 @@ cudaError_t launch_o_proj(const OProjParams& p, cudaStream_t stream) {
 }
 
 cudaError_t launch_qkv_proj(const QkvProjParams& p, cudaStream_t stream) {
-    input_norm_split_kernel<<<p.batch, kPrepThreads, 0, stream>>>(p);
-    const cudaError_t e = cudaGetLastError();
+    // a programmatic dependent of the launch before it: its launch overlaps that one's end
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.batch, 1, 1);
+    cfg.blockDim = dim3(kPrepThreads, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, input_norm_split_kernel, p);
     if (e != cudaSuccess) return e;
     LinearOperands ops{p.w, p.xg_hi, p.xg_lo};
     LinearParams lp{};
