@@ -844,11 +844,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attention_kernel(const Par
         s.lens[b] = L;
         s.seg[b + 1] = ok ? (L + kPage - 1) / kPage : 0;
     }
-    if (threadIdx.x < 64) {
-        // both gain vectors, one 8-byte word per thread
-        const uint16_t* src = threadIdx.x < 32 ? p.q_norm_w : p.k_norm_w;
-        reinterpret_cast<uint2*>(smem + kSmemGains)[threadIdx.x] =
-            *reinterpret_cast<const uint2*>(src + 4 * (threadIdx.x & 31));
+    if (threadIdx.x < 128) {
+        // both gain vectors, one 4-byte word per thread (the pointers are only
+        // 4-byte aligned)
+        const uint16_t* src = threadIdx.x < 64 ? p.q_norm_w : p.k_norm_w;
+        reinterpret_cast<uint32_t*>(smem + kSmemGains)[threadIdx.x] =
+            *reinterpret_cast<const uint32_t*>(src + 2 * (threadIdx.x & 63));
     }
     __syncthreads();
     if (warp == 0) {  // inclusive scan of the page counts: seg[b] becomes the first page of b

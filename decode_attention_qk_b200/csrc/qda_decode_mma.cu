@@ -1031,10 +1031,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
         s.lens[b] = L;
         s.seg[b + 1] = ok ? (L + kPage - 1) / kPage : 0;
     }
-    if (threadIdx.x < 64) {
-        const uint16_t* src = threadIdx.x < 32 ? p.q_norm_w : p.k_norm_w;
-        reinterpret_cast<uint2*>(smem + Lay::kSmemGains)[threadIdx.x] =
-            *reinterpret_cast<const uint2*>(src + 4 * (threadIdx.x & 31));
+    if (threadIdx.x < 128) {
+        // one 4-byte word per thread (the gain pointers are only 4-byte aligned)
+        const uint16_t* src = threadIdx.x < 64 ? p.q_norm_w : p.k_norm_w;
+        reinterpret_cast<uint32_t*>(smem + Lay::kSmemGains)[threadIdx.x] =
+            *reinterpret_cast<const uint32_t*>(src + 2 * (threadIdx.x & 63));
     }
     __syncthreads();
     if (warp == 0) {  // inclusive scan of the page counts

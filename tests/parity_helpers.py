@@ -11,6 +11,7 @@ The cache is compared bit for bit.
 """
 from __future__ import annotations
 
+import dataclasses
 import numpy as np
 import torch
 
@@ -27,6 +28,18 @@ def device_args(w: inputs.Workload, dev, positions=None):
     return dict(qkv=w.qkv.to(dev), q_norm_w=w.q_norm_w.to(dev), k_norm_w=w.k_norm_w.to(dev),
                 seq_lens=w.seq_lens.to(dev), block_table=w.block_table.to(dev),
                 positions=None if pos is None else pos.to(dev))
+
+
+def gains_at_a_4_byte_offset(w: inputs.Workload) -> inputs.Workload:
+    """The same workload with q_norm_w and k_norm_w on the device at addresses
+    that are 4-byte but not 8-byte aligned (the alignment the ABI asks of them)."""
+    def at4(t):
+        buf = torch.empty(t.numel() + 8, dtype=t.dtype, device=t.device)
+        view = buf[2:2 + t.numel()]
+        view.copy_(t)
+        assert view.data_ptr() % 8 == 4
+        return view
+    return dataclasses.replace(w, q_norm_w=at4(w.q_norm_w), k_norm_w=at4(w.k_norm_w))
 
 
 def run(attn, w: inputs.Workload, dev, k_cache, v_cache, positions=None, o=None):

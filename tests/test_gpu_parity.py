@@ -58,6 +58,12 @@ def test_split_count_does_not_change_the_result(grid):
     a.close()
 
 
+def test_gains_at_a_4_byte_aligned_address(attn):
+    """The norm gains need only be 4-byte aligned (the ABI's requirement)."""
+    w = inputs.custom([1, 17, 300, 33], seed=19, device="cuda")
+    full_check(attn, ph.gains_at_a_4_byte_offset(w), "gains at +4 bytes")
+
+
 def test_page_edge_lengths(attn):
     lens = [1, 2, 15, 16, 17, 18, 31, 32, 33, 47, 48, 49, 63, 64, 65, 255, 256, 257]
     full_check(attn, inputs.custom(lens, seed=12, device="cuda", gap_fraction=0.3), "page edges")

@@ -53,6 +53,12 @@ def test_page_edges(handles, hq):
 
 
 @pytest.mark.parametrize("hq", HEADS)
+def test_gains_at_a_4_byte_aligned_address(handles, hq):
+    w = inputs.custom([1, 17, 300, 33], seed=45, device="cuda", num_q_heads=hq)
+    full_check(handles[hq], ph.gains_at_a_4_byte_offset(w), f"Hq={hq} gains at +4 bytes")
+
+
+@pytest.mark.parametrize("hq", HEADS)
 def test_single_position_returns_v_bits(handles, hq):
     w = inputs.custom([1] * 9, seed=41, device="cuda", num_q_heads=hq)
     o, _ = full_check(handles[hq], w, f"Hq={hq} L=1")

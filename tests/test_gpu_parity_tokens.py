@@ -74,6 +74,13 @@ def test_page_edges(handles, hq, T):
     full_check(handles[hq], w, f"Hq={hq} T={T} page edges")
 
 
+@pytest.mark.parametrize("hq,T", [(16, 4), (32, 2), (16, 8)])
+def test_gains_at_a_4_byte_aligned_address(handles, hq, T):
+    """The norm gains need only be 4-byte aligned (the ABI's requirement)."""
+    w = inputs.custom([T, 17, 300, 33], seed=62, device="cuda", num_q_heads=hq, new_tokens=T)
+    full_check(handles[hq], ph.gains_at_a_4_byte_offset(w), f"Hq={hq} T={T} gains at +4 bytes")
+
+
 @pytest.mark.parametrize("hq,T", CASES)
 def test_an_empty_cache_gives_the_first_token_its_own_v(handles, hq, T):
     """L = T: the first new token sees only itself, so its o is its v, bit for bit."""
