@@ -59,6 +59,11 @@ constexpr int kStageK = 0;
 constexpr int kStageV = kPage * kRowPitch;
 constexpr int kStageBytes = 2 * kPage * kRowPitch;  // 66048
 
+// Row stride (float2 entries) of the rotation table: one more than the 64
+// pairs, so that lanes reading the same pair for different tokens fall in
+// different banks.
+constexpr int kRotStride = 65;
+
 template <int G, int T>
 struct Layout {
     static constexpr int kHq = G * kNumKvHeads;
@@ -78,7 +83,11 @@ struct Layout {
     static constexpr int kSmemSeg = kSmemNewK + kNewKBytes;                   // int [kMaxBatch + 4]
     static constexpr int kSmemLens = kSmemSeg + (kMaxBatch + 4) * 4;        // int [kMaxBatch]
     static constexpr int kSmemInvFreq = kSmemLens + kMaxBatch * 4;          // double [64]
-    static constexpr int kSmemGains = kSmemInvFreq + 64 * 8;                // bf16 [2][128]
+    // (cos f_i, sin f_i) in double, the step of pair i from one position to the next
+    static constexpr int kSmemStep = kSmemInvFreq + 64 * 8;                 // double2 [64]
+    // (cos, sin) of u * f_i in float for the later new tokens u = 1..T-1
+    static constexpr int kSmemRot = kSmemStep + 64 * 16;                    // float2 [T - 1][kRotStride]
+    static constexpr int kSmemGains = kSmemRot + (T - 1) * kRotStride * 8;  // bf16 [2][128]
     static constexpr int kSmemMeta = kSmemGains + 2 * kHeadDim * 2;         // StageMeta [kStages] + qkv position
     static constexpr int kSmemBars = kSmemMeta + (kStages + 1) * 16;        // full, empty, qkv_full, qkv_empty, never
     static constexpr int kSmemFlags = kSmemBars + (2 * kStages + 3) * 8;
@@ -90,7 +99,7 @@ struct Layout {
     static constexpr bool kWide = kRows > 8;
     static_assert(kRows <= 16, "at most 16 query rows per kv head");
     static_assert(!kWide || kDirectQkv, "wide instances read their qkv rows from global memory");
-    static_assert(kSmemQkv % 16 == 0 && kSmemInvFreq % 8 == 0 && kSmemBars % 8 == 0, "alignment");
+    static_assert(kSmemQkv % 16 == 0 && kSmemInvFreq % 16 == 0 && kSmemBars % 8 == 0, "alignment");
     static_assert(kSmemTotal <= 227 * 1024, "fits one CTA per SM");
 };
 
@@ -126,6 +135,8 @@ struct Shared {
     int* seg;
     int* lens;
     double* inv_freq;
+    double2* step;        // [64] (cos f_i, sin f_i)
+    float2* rot;          // [T - 1][kRotStride] (cos, sin) of u * f_i, u = 1..T-1
     const uint16_t* gains;
     volatile StageMeta* meta;
     volatile int* qkv_pos;
@@ -243,6 +254,17 @@ __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, i
 // ---------------------------------------------------------------------------
 // Consumer warps.
 
+// x - n * 2*pi for the integer n nearest x / (2*pi), in double: 2*pi is split
+// into a 32-bit head (n * head and x - n * head are exact for the |x| < 2^20
+// here) and its double remainder, so the result carries about one ulp of x.
+__device__ __forceinline__ double reduce_two_pi(double x) {
+    constexpr double kTwoPiHi = 6.2831853069365025;      // 2*pi rounded to 32 significant bits
+    constexpr double kTwoPiLo = 2.430840202602477e-10;   // 2*pi - kTwoPiHi
+    constexpr double kInvTwoPi = 0.15915494309189535;
+    const double n = rint(x * kInvTwoPi);
+    return fma(-n, kTwoPiLo, fma(-n, kTwoPiHi, x));
+}
+
 template <int T>
 struct State {
     uint32_t qa[8][4];    // A fragments of q per 16-dim step: rows r (bf16 of q) and r+8 (remainder)
@@ -256,47 +278,52 @@ struct State {
 // or in global memory for the largest rows): q of row r = lane/4 (new
 // token r / G, head G*j + r % G) at dims 8m + 2t, 8m + 2t + 1 (t = lane%4,
 // m = 0..15), i.e. both halves of the rotation pairs 8m' + 2t + e, m' < 8.
-// Lane l forms the angles of pairs 2l, 2l+1 for the first new token (reduced
-// modulo 2*pi in double, then float sin/cos) and, for the later tokens,
-// rotates them by the per-position step; lanes fetch theirs by shuffles.
-// When this CTA holds a page with new tokens, their k is formed in double.
+// Lane l forms the first new token's angles of pairs 2l, 2l+1 (reduced
+// modulo 2*pi in double, then float sin/cos); a lane fetches those of its
+// pairs by shuffles and turns them to its row's token tt by the tabled
+// rotation of tt positions. When this CTA holds a page with new tokens, their
+// k is formed in double. Every load from the rows is issued first, so that
+// rows read from global memory cost one round trip.
 template <int G, int T>
 __device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s, const uint8_t* rows, int pos0,
                                                int j, int lane, bool appends, State<T>& st) {
     using Lay = Layout<G, T>;
-    constexpr double kTwoPiHi = 6.2831853069365025;      // 2*pi rounded to 32 significant bits
-    constexpr double kTwoPiLo = 2.430840202602477e-10;   // 2*pi - kTwoPiHi
-    constexpr double kInvTwoPi = 0.15915494309189535;
     const int r = lane >> 2, t = lane & 3;
     const bool active = r < Lay::kRows;
     const int tt = active ? r / G : 0;          // this row's new token
     const int head = G * j + (active ? r % G : 0);
-    float cf[T][2], sf[T][2];
+
+    // the loads: this row's q words, and the new tokens' k and v words
+    const uint32_t* xq =
+        reinterpret_cast<const uint32_t*>(rows + tt * Lay::kQkvBytes + head * (kHeadDim * 2));
+    uint32_t xw[16];
+#pragma unroll
+    for (int m = 0; m < 16; ++m) xw[m] = xq[4 * m + t];
+    uint32_t kx_lo[T], kx_hi[T];
+    if (appends) {
+#pragma unroll
+        for (int u = 0; u < T; ++u) {
+            const uint8_t* row = rows + u * Lay::kQkvBytes;
+            const uint32_t* xk = reinterpret_cast<const uint32_t*>(row + (Lay::kHq + j) * (kHeadDim * 2));
+            const uint32_t* xv = reinterpret_cast<const uint32_t*>(row + (Lay::kHq + kNumKvHeads + j) * (kHeadDim * 2));
+            kx_lo[u] = xk[lane];
+            kx_hi[u] = xk[32 + lane];
+            st.v_lo[u] = xv[lane];
+            st.v_hi[u] = xv[32 + lane];
+        }
+    }
+
+    // the first new token's angles of pairs 2*lane + e
+    float c0[2], s0[2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
         const double ang = (double)pos0 * s.inv_freq[2 * lane + e];
-        const double n = rint(ang * kInvTwoPi);
-        sincosf((float)fma(-n, kTwoPiLo, fma(-n, kTwoPiHi, ang)), &sf[0][e], &cf[0][e]);
-        if (T > 1) {   // later tokens: rotate by the step f (float error ~u * 2^-24, q stays float)
-            float ds, dc;
-            sincosf((float)s.inv_freq[2 * lane + e], &ds, &dc);
-#pragma unroll
-            for (int u = 1; u < T; ++u) {
-                cf[u][e] = fmaf(cf[u - 1][e], dc, -sf[u - 1][e] * ds);
-                sf[u][e] = fmaf(sf[u - 1][e], dc, cf[u - 1][e] * ds);
-            }
-        }
+        sincosf((float)reduce_two_pi(ang), &s0[e], &c0[e]);
     }
-    const uint32_t* xq =
-        reinterpret_cast<const uint32_t*>(rows + tt * Lay::kQkvBytes + head * (kHeadDim * 2));
     const uint32_t* gq = reinterpret_cast<const uint32_t*>(s.gains);
-    uint32_t xw[16];
     float ss = 0.f;
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-        xw[m] = xq[4 * m + t];
-        ss = fmaf(bf_lo(xw[m]), bf_lo(xw[m]), fmaf(bf_hi(xw[m]), bf_hi(xw[m]), ss));
-    }
+    for (int m = 0; m < 16; ++m) ss = fmaf(bf_lo(xw[m]), bf_lo(xw[m]), fmaf(bf_hi(xw[m]), bf_hi(xw[m]), ss));
     ss += __shfl_xor_sync(kFull, ss, 1);
     ss += __shfl_xor_sync(kFull, ss, 2);
     const float inv_r = rsqrtf(ss * (1.f / 128.f) + (float)p.rms_eps);
@@ -307,13 +334,14 @@ __device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s,
         const uint32_t wlo = gq[4 * mp + t], whi = gq[32 + 4 * mp + t];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            float cs = 0.f, sn = 0.f;
-#pragma unroll
-            for (int u = 0; u < T; ++u) {   // the angle of pair 8*mp + 2t + e at this row's token
-                const float cu = __shfl_sync(kFull, cf[u][e], 4 * mp + t);
-                const float su = __shfl_sync(kFull, sf[u][e], 4 * mp + t);
-                cs = (u == tt) ? cu : cs;
-                sn = (u == tt) ? su : sn;
+            // the angle of pair 8*mp + 2t + e at the first new token, then at this row's
+            float cs = __shfl_sync(kFull, c0[e], 4 * mp + t);
+            float sn = __shfl_sync(kFull, s0[e], 4 * mp + t);
+            if (T > 1 && tt > 0) {
+                const float2 rt = s.rot[(tt - 1) * kRotStride + 8 * mp + 2 * t + e];
+                const float c = fmaf(cs, rt.x, -sn * rt.y);
+                sn = fmaf(sn, rt.x, cs * rt.y);
+                cs = c;
             }
             const float ya = (e ? bf_hi(xw[mp]) : bf_lo(xw[mp])) * inv_r * (e ? bf_hi(wlo) : bf_lo(wlo));
             const float yb = (e ? bf_hi(xw[mp + 8]) : bf_lo(xw[mp + 8])) * inv_r * (e ? bf_hi(whi) : bf_lo(whi));
@@ -334,32 +362,24 @@ __device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s,
 
     if (appends) {
         // lane l: dims 2l, 2l+1 (word l of the head) and 64+2l, 65+2l (word 32+l), all in double.
-        // The angle of token u is pos0*f + u*f: token 0's sine and cosine, then u
-        // rotations by the step f (error ~u ulp of double, far below k's bf16 rounding).
+        // The angle of token u is pos0*f + u*f: token 0's sine and cosine (argument
+        // reduced modulo 2*pi first), then u rotations by the tabled step f (error
+        // ~u ulp of double, far below k's bf16 rounding).
         const uint32_t* gk = reinterpret_cast<const uint32_t*>(s.gains + kHeadDim);
         const uint32_t wk_lo = gk[lane], wk_hi = gk[32 + lane];
-        double sn0, cs0, sn1, cs1, ds0, dc0, ds1, dc1;
-        sincos((double)pos0 * s.inv_freq[2 * lane], &sn0, &cs0);
-        sincos((double)pos0 * s.inv_freq[2 * lane + 1], &sn1, &cs1);
-        if (T > 1) {
-            sincos(s.inv_freq[2 * lane], &ds0, &dc0);
-            sincos(s.inv_freq[2 * lane + 1], &ds1, &dc1);
-        }
+        double sn0, cs0, sn1, cs1;
+        sincos(reduce_two_pi((double)pos0 * s.inv_freq[2 * lane]), &sn0, &cs0);
+        sincos(reduce_two_pi((double)pos0 * s.inv_freq[2 * lane + 1]), &sn1, &cs1);
+        const double2 st0 = s.step[2 * lane], st1 = s.step[2 * lane + 1];
         double ssq[T];
         double a0[T], a1[T], b0[T], b1[T];
 #pragma unroll
         for (int u = 0; u < T; ++u) {
-            const uint8_t* row = rows + u * Lay::kQkvBytes;
-            const uint32_t* xk = reinterpret_cast<const uint32_t*>(row + (Lay::kHq + j) * (kHeadDim * 2));
-            const uint32_t* xv = reinterpret_cast<const uint32_t*>(row + (Lay::kHq + kNumKvHeads + j) * (kHeadDim * 2));
-            const uint32_t xlo = xk[lane], xhi = xk[32 + lane];
-            a0[u] = bf_to_d(xlo & 0xFFFFu);
-            a1[u] = bf_to_d(xlo >> 16);
-            b0[u] = bf_to_d(xhi & 0xFFFFu);
-            b1[u] = bf_to_d(xhi >> 16);
+            a0[u] = bf_to_d(kx_lo[u] & 0xFFFFu);
+            a1[u] = bf_to_d(kx_lo[u] >> 16);
+            b0[u] = bf_to_d(kx_hi[u] & 0xFFFFu);
+            b1[u] = bf_to_d(kx_hi[u] >> 16);
             ssq[u] = a0[u] * a0[u] + a1[u] * a1[u] + b0[u] * b0[u] + b1[u] * b1[u];
-            st.v_lo[u] = xv[lane];
-            st.v_hi[u] = xv[32 + lane];
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1)
@@ -377,8 +397,8 @@ __device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s,
             st.k_lo[u] = d_to_bf(ra0) | (d_to_bf(ra1) << 16);
             st.k_hi[u] = d_to_bf(rb0) | (d_to_bf(rb1) << 16);
             if (u + 1 < T) {   // advance both angles by one position
-                const double c0n = cs0 * dc0 - sn0 * ds0, s0n = sn0 * dc0 + cs0 * ds0;
-                const double c1n = cs1 * dc1 - sn1 * ds1, s1n = sn1 * dc1 + cs1 * ds1;
+                const double c0n = cs0 * st0.x - sn0 * st0.y, s0n = sn0 * st0.x + cs0 * st0.y;
+                const double c1n = cs1 * st1.x - sn1 * st1.y, s1n = sn1 * st1.x + cs1 * st1.y;
                 cs0 = c0n; sn0 = s0n; cs1 = c1n; sn1 = s1n;
             }
         }
@@ -579,11 +599,11 @@ __device__ __forceinline__ void form_new_k(const Params& p, const Shared& s, con
     using Lay = Layout<G, T>;
     const uint32_t* gk = reinterpret_cast<const uint32_t*>(s.gains + kHeadDim);
     const uint32_t wk_lo = gk[lane], wk_hi = gk[32 + lane];
-    double sn0, cs0, sn1, cs1, ds0, dc0, ds1, dc1;
-    sincos((double)pos0 * s.inv_freq[2 * lane], &sn0, &cs0);
-    sincos((double)pos0 * s.inv_freq[2 * lane + 1], &sn1, &cs1);
-    sincos(s.inv_freq[2 * lane], &ds0, &dc0);
-    sincos(s.inv_freq[2 * lane + 1], &ds1, &dc1);
+    double sn0, cs0, sn1, cs1;
+    sincos(reduce_two_pi((double)pos0 * s.inv_freq[2 * lane]), &sn0, &cs0);
+    sincos(reduce_two_pi((double)pos0 * s.inv_freq[2 * lane + 1]), &sn1, &cs1);
+    const double dc0 = s.step[2 * lane].x, ds0 = s.step[2 * lane].y;
+    const double dc1 = s.step[2 * lane + 1].x, ds1 = s.step[2 * lane + 1].y;
     uint32_t* dst = s.new_k + (size_t)j * T * 64;
     // every token's words first (one round trip to L2), then the arithmetic
     uint32_t xlo[T], xhi[T];
@@ -622,24 +642,10 @@ __device__ __forceinline__ void begin_sequence_wide(const Params& p, const Share
                                                     int j, int lane, bool appends, WState& st) {
     using Lay = Layout<G, T>;
     if (appends) form_new_k<G, T>(p, s, rows, pos0, j, lane);
-    constexpr double kTwoPiHi = 6.2831853069365025;      // 2*pi rounded to 32 significant bits
-    constexpr double kTwoPiLo = 2.430840202602477e-10;   // 2*pi - kTwoPiHi
-    constexpr double kInvTwoPi = 0.15915494309189535;
     const int g = lane >> 2, t = lane & 3;
-    float cf[T][2], sf[T][2];
+    float c0[2], s0[2];   // the first new token's angles of pairs 2*lane + e
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-        const double ang = (double)pos0 * s.inv_freq[2 * lane + e];
-        const double n = rint(ang * kInvTwoPi);
-        sincosf((float)fma(-n, kTwoPiLo, fma(-n, kTwoPiHi, ang)), &sf[0][e], &cf[0][e]);
-        float ds, dc;
-        sincosf((float)s.inv_freq[2 * lane + e], &ds, &dc);
-#pragma unroll
-        for (int u = 1; u < T; ++u) {   // later tokens: rotate by the step f
-            cf[u][e] = fmaf(cf[u - 1][e], dc, -sf[u - 1][e] * ds);
-            sf[u][e] = fmaf(sf[u - 1][e], dc, cf[u - 1][e] * ds);
-        }
-    }
+    for (int e = 0; e < 2; ++e) sincosf((float)reduce_two_pi((double)pos0 * s.inv_freq[2 * lane + e]), &s0[e], &c0[e]);
     const uint32_t* gq = reinterpret_cast<const uint32_t*>(s.gains);
     const float scale = (float)kQScale;
 #pragma unroll
@@ -665,13 +671,14 @@ __device__ __forceinline__ void begin_sequence_wide(const Params& p, const Share
             const uint32_t wlo = gq[4 * mp + t], whi = gq[32 + 4 * mp + t];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                float cs = 0.f, sn = 0.f;
-#pragma unroll
-                for (int u = 0; u < T; ++u) {   // the angle of pair 8*mp + 2t + e at this row's token
-                    const float cu = __shfl_sync(kFull, cf[u][e], 4 * mp + t);
-                    const float su = __shfl_sync(kFull, sf[u][e], 4 * mp + t);
-                    cs = (u == tt) ? cu : cs;
-                    sn = (u == tt) ? su : sn;
+                // the angle of pair 8*mp + 2t + e at the first new token, then at this row's
+                float cs = __shfl_sync(kFull, c0[e], 4 * mp + t);
+                float sn = __shfl_sync(kFull, s0[e], 4 * mp + t);
+                if (tt > 0) {
+                    const float2 rt = s.rot[(tt - 1) * kRotStride + 8 * mp + 2 * t + e];
+                    const float c = fmaf(cs, rt.x, -sn * rt.y);
+                    sn = fmaf(sn, rt.x, cs * rt.y);
+                    cs = c;
                 }
                 const float ya = (e ? bf_hi(xw[mp]) : bf_lo(xw[mp])) * inv_r * (e ? bf_hi(wlo) : bf_lo(wlo));
                 const float yb = (e ? bf_hi(xw[mp + 8]) : bf_lo(xw[mp + 8])) * inv_r * (e ? bf_hi(whi) : bf_lo(whi));
@@ -989,6 +996,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
     s.seg = reinterpret_cast<int*>(smem + Lay::kSmemSeg);
     s.lens = reinterpret_cast<int*>(smem + Lay::kSmemLens);
     s.inv_freq = reinterpret_cast<double*>(smem + Lay::kSmemInvFreq);
+    s.step = reinterpret_cast<double2*>(smem + Lay::kSmemStep);
+    s.rot = reinterpret_cast<float2*>(smem + Lay::kSmemRot);
     s.gains = reinterpret_cast<const uint16_t*>(smem + Lay::kSmemGains);
     s.meta = reinterpret_cast<volatile StageMeta*>(smem + Lay::kSmemMeta);
     s.qkv_pos = reinterpret_cast<volatile int*>(smem + Lay::kSmemMeta + kStages * 16);
@@ -1003,8 +1012,20 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_attention_kernel(const Pa
     // no global memory, and griddepcontrol.wait holds until the previous
     // launch on the stream has completed and its writes are visible.
     if (threadIdx.x >= 64 && threadIdx.x < 128) {
+        // the frequencies, and the angles every sequence start reuses: one
+        // position's step (double, for k) and the offsets of the later new
+        // tokens (float, for q); small arguments, so one sincos each
         const int i = threadIdx.x - 64;
-        s.inv_freq[i] = pow(p.rope_theta, -2.0 * i / 128.0);
+        const double f = pow(p.rope_theta, -2.0 * i / 128.0);
+        s.inv_freq[i] = f;
+        double sn, cs;
+        sincos(f, &sn, &cs);
+        s.step[i] = make_double2(cs, sn);
+#pragma unroll
+        for (int u = 1; u < T; ++u) {
+            sincos((double)u * f, &sn, &cs);
+            s.rot[(u - 1) * kRotStride + i] = make_float2((float)cs, (float)sn);
+        }
     }
     if (threadIdx.x == 0) {
         for (int k = 0; k < kStages; ++k) {
