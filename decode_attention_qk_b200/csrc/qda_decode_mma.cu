@@ -67,18 +67,24 @@ constexpr int kRotStride = 65;
 template <int G, int T>
 struct Layout {
     static constexpr int kHq = G * kNumKvHeads;
-    static constexpr int kRows = G * T;                                  // query rows per kv head
     static constexpr int kQkvW = (kHq + 2 * kNumKvHeads) * kHeadDim;     // elements in one token's qkv row
     static constexpr int kQkvBytes = kQkvW * 2;
     static constexpr int kSlotBytes = T * kQkvBytes;                     // a sequence's T rows
-    // Rows up to 24 KiB are staged in a shared-memory slot next to three K/V
-    // stages; larger ones (16 heads x 4 tokens: 32 KiB) would leave room for two
-    // stages only, so they are prefetched to L2 and read from global memory.
-    static constexpr bool kDirectQkv = kSlotBytes > 24576;
+    static constexpr int kQRowBytes = kHq * kHeadDim * 2;                // the q part of one row
+    static constexpr int kRows = G * T;                                  // query rows per kv head
+    static constexpr bool kWide = kRows > 8;
+    // Up to 8 query rows per kv head the rows are staged in a shared-memory
+    // slot next to three K/V stages: whole when they take up to 24 KiB, else
+    // (16 heads x 4 tokens: 32 KiB) their q parts only, the new k and v words
+    // being read from global memory (prefetched to L2) by the CTA appending
+    // them. Wide instances read the rows from global memory.
+    static constexpr bool kDirectQkv = kWide;
+    static constexpr bool kStageQOnly = !kWide && kSlotBytes > 24576;
+    static constexpr int kStagedBytes = kWide ? 0 : (kStageQOnly ? T * kQRowBytes : kSlotBytes);
     static constexpr int kStages = 3;
     static constexpr int kSmemQkv = kStages * kStageBytes;
     // wide instances: the new tokens' k words, [warp][token][64] (formed when a sequence starts)
-    static constexpr int kSmemNewK = kSmemQkv + (kDirectQkv ? 0 : kSlotBytes);
+    static constexpr int kSmemNewK = kSmemQkv + kStagedBytes;
     static constexpr int kNewKBytes = (kRows > 8) ? kConsumerWarps * T * 64 * 4 : 0;
     static constexpr int kSmemSeg = kSmemNewK + kNewKBytes;                   // int [kMaxBatch + 4]
     static constexpr int kSmemLens = kSmemSeg + (kMaxBatch + 4) * 4;        // int [kMaxBatch]
@@ -96,9 +102,8 @@ struct Layout {
     // cores as two bf16 terms (value and remainder, rows r and r + 8 of the
     // A operand); with 9 to 16 rows ("wide"), the 16 rows are 16 query rows
     // and q and the probabilities enter as bf16.
-    static constexpr bool kWide = kRows > 8;
     static_assert(kRows <= 16, "at most 16 query rows per kv head");
-    static_assert(!kWide || kDirectQkv, "wide instances read their qkv rows from global memory");
+    static_assert(kStagedBytes <= 24576, "the staged rows leave room for three K/V stages");
     static_assert(kSmemQkv % 16 == 0 && kSmemInvFreq % 16 == 0 && kSmemBars % 8 == 0, "alignment");
     static_assert(kSmemTotal <= 227 * 1024, "fits one CTA per SM");
 };
@@ -194,9 +199,18 @@ __device__ __forceinline__ void run_producer(const Params& p, const Shared& s, i
                          mbar_wait(s.qkv_empty, qphase ^ 1u, p.timeout_ns, s.abort_flag);
                     if (ok) {
                         *s.qkv_pos = seq_pos;
-                        mbar_arrive_expect_tx(s.qkv_full, (uint32_t)Lay::kSlotBytes);
-                        bulk_g2s(s.qkv, p.qkv + token_row(p, seq_qkv, 0) * Lay::kQkvW, (uint32_t)Lay::kSlotBytes,
-                                 s.qkv_full);
+                        const uint16_t* src = p.qkv + token_row(p, seq_qkv, 0) * Lay::kQkvW;
+                        mbar_arrive_expect_tx(s.qkv_full, (uint32_t)Lay::kStagedBytes);
+                        if constexpr (Lay::kStageQOnly) {
+                            // each token's q part; the k and v words to L2 for the appending CTA
+#pragma unroll
+                            for (int u = 0; u < T; ++u)
+                                bulk_g2s(s.qkv + u * Lay::kQRowBytes, src + (size_t)u * Lay::kQkvW,
+                                         (uint32_t)Lay::kQRowBytes, s.qkv_full);
+                            bulk_prefetch_l2(src, (uint32_t)Lay::kSlotBytes);
+                        } else {
+                            bulk_g2s(s.qkv, src, (uint32_t)Lay::kSlotBytes, s.qkv_full);
+                        }
                         qarmed = true;
                         qarmed_parity = qphase;
                         qphase ^= 1u;
@@ -274,8 +288,8 @@ struct State {
     uint32_t k_lo[T], k_hi[T], v_lo[T], v_hi[T];   // this lane's words of the appended k/v rows
 };
 
-// Start a sequence piece from its T qkv rows `rows` (staged in shared memory,
-// or in global memory for the largest rows): q of row r = lane/4 (new
+// Start a sequence piece from its T qkv rows (staged in shared memory, or
+// their q parts staged and the rest read from global memory): q of row r = lane/4 (new
 // token r / G, head G*j + r % G) at dims 8m + 2t, 8m + 2t + 1 (t = lane%4,
 // m = 0..15), i.e. both halves of the rotation pairs 8m' + 2t + e, m' < 8.
 // Lane l forms the first new token's angles of pairs 2l, 2l+1 (reduced
@@ -285,17 +299,18 @@ struct State {
 // k is formed in double. Every load from the rows is issued first, so that
 // rows read from global memory cost one round trip.
 template <int G, int T>
-__device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s, const uint8_t* rows, int pos0,
-                                               int j, int lane, bool appends, State<T>& st) {
+__device__ __forceinline__ void begin_sequence(const Params& p, const Shared& s, const uint8_t* qrows, int q_stride,
+                                               const uint8_t* rows, int pos0, int j, int lane, bool appends,
+                                               State<T>& st) {
     using Lay = Layout<G, T>;
     const int r = lane >> 2, t = lane & 3;
     const bool active = r < Lay::kRows;
     const int tt = active ? r / G : 0;          // this row's new token
     const int head = G * j + (active ? r % G : 0);
 
-    // the loads: this row's q words, and the new tokens' k and v words
-    const uint32_t* xq =
-        reinterpret_cast<const uint32_t*>(rows + tt * Lay::kQkvBytes + head * (kHeadDim * 2));
+    // the loads: this row's q words (token u's q part at qrows + u * q_stride),
+    // and the new tokens' k and v words (from the whole rows `rows`)
+    const uint32_t* xq = reinterpret_cast<const uint32_t*>(qrows + tt * q_stride + head * (kHeadDim * 2));
     uint32_t xw[16];
 #pragma unroll
     for (int m = 0; m < 16; ++m) xw[m] = xq[4 * m + t];
@@ -947,16 +962,17 @@ __device__ __forceinline__ void run_consumer(const Params& p, const Shared& s, i
         const int n_here = min(nb - i0, count - k);
         // this CTA appends when it holds a page with one of the new tokens
         const bool appends = s.seg[b] + (L - T) / kPage < end;
-        if (Layout<G, T>::kDirectQkv) {
-            const int pos0 = first_position(p, b, L, T);
-            begin_sequence<G, T>(p, s, reinterpret_cast<const uint8_t*>(p.qkv + token_row(p, b, 0) * Layout<G, T>::kQkvW),
-                                 pos0, j, lane, appends, st);
-        } else {
+        {
+            using Lay = Layout<G, T>;
             if (!wait_full(p, s, s.qkv_full, qphase, lane)) {
                 aborted = true;
                 break;
             }
-            begin_sequence<G, T>(p, s, s.qkv, *s.qkv_pos, j, lane, appends, st);
+            const uint8_t* rows = Lay::kStageQOnly
+                                      ? reinterpret_cast<const uint8_t*>(p.qkv + token_row(p, b, 0) * Lay::kQkvW)
+                                      : s.qkv;
+            begin_sequence<G, T>(p, s, s.qkv, Lay::kStageQOnly ? Lay::kQRowBytes : Lay::kQkvBytes, rows,
+                                 *s.qkv_pos, j, lane, appends, st);
             __syncwarp();
             if (lane == 0) mbar_arrive(s.qkv_empty);
             qphase ^= 1u;
