@@ -20,7 +20,7 @@
 //   transposed, D[n][b] = sum_k W[n][k] (hi[b][k] + lo[b][k]), with the 128
 //   weight rows as the A operand (M = 128) and C <= 64 batch rows as the B
 //   operand (N = C). A producer thread streams 128 x 64 weight boxes and the
-//   matching C x 64 boxes of hi and lo into a 5-stage shared ring by tiled
+//   matching C x 64 boxes of hi and lo into a 4-stage shared ring by tiled
 //   copies with the 128-byte swizzle; one thread issues tcgen05.mma (two per
 //   16-wide K step: hi, then lo, into the same accumulator) and frees each
 //   stage with tcgen05.commit; the accumulator lives in tensor memory and the
@@ -64,10 +64,15 @@ namespace {
 
 constexpr int kPrepThreads = 128;
 
-constexpr int kLinThreads = 128;                      // 4 warps: producer, MMA issuer, and all four for the epilogue
+constexpr int kLinThreads = 256;                      // 8 warps: producer, scales, 4 MMA issuers; warps 0-3 the epilogue
+constexpr int kLinIssuers = 4;                        // MMA-issuing threads (lane 0 of warps 4-7), one accumulator each
 constexpr int kLinM = 128;                            // weight rows per CTA (the instruction's M)
 constexpr int kLinKC = 64;                            // K per stage: one 128-byte swizzle row
-constexpr int kLinStages = 5;
+constexpr int kLinStages = 4;
+// Issuer t consumes every chunk of stage t, in order: a thread waiting on a
+// stage's full barrier is then never more than one phase ahead of it (a wait
+// on a parity two phases ahead would pass at once).
+static_assert(kLinStages == kLinIssuers, "each MMA issuer owns one stage of the ring");
 constexpr int kLinMaxCols = 64;                       // batch rows per CTA (the instruction's N)
 constexpr int kLinABytes = kLinM * kLinKC * 2;        // 16 KiB of weight per stage
 constexpr int kLinBBytes = 2 * kLinMaxCols * kLinKC * 2;   // hi and lo boxes: up to 16 KiB
@@ -81,7 +86,7 @@ constexpr int kLinSmemScale = kLinSmemTile + kLinTileBytes;  // float [kLinMaxCo
 constexpr int kLinSmemBars = kLinSmemScale + kLinMaxCols * 4;   // full[S], empty[S], acc, tile, tmem address, abort
 constexpr int kLinSmemUsed = kLinSmemBars + (2 * kLinStages + 2) * 8 + 16;
 constexpr int kLinSmemTotal = kLinSmemUsed + 1024;    // slack to align the ring to 1024 bytes
-constexpr uint32_t kLinTmemCols = 64;
+constexpr uint32_t kLinTmemCols = kLinIssuers * kLinMaxCols;   // one accumulator of up to 64 columns per issuer
 static_assert(kLinStageBytes % 1024 == 0 && kLinABytes % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
 static_assert(kLinSmemTotal <= 227 * 1024, "fits one CTA per SM");
 
@@ -190,7 +195,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(acc_bar, 1);
+        mbar_init(acc_bar, kLinIssuers);
         mbar_init(tile_bar, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -238,10 +243,16 @@ __global__ void __launch_bounds__(kLinThreads, 1)
             for (int c = max(0, issued - kLinStages); c < issued; ++c)
                 (void)mbar_wait(&full[c % kLinStages], (uint32_t)((c / kLinStages) & 1), p.timeout_ns, nullptr);
         }
-    } else if (warp == 1 && lane == 0) {
-        // MMA issuer: two products per 16-wide K step (hi, then lo) into one accumulator.
+    } else if (warp >= 4 && lane == 0) {
+        // MMA issuer t (of 4) takes chunks t, t + 4, ... (all in stage t) into
+        // its own accumulator (columns 64t..): two products per 16-wide K step
+        // (hi, then lo). An issuing thread stalls on the products it issues
+        // (about 0.45 us per 64-wide chunk at the small N here, measured), so
+        // four of them keep four chains in flight.
+        const int t = warp - 4;
         const uint32_t idesc = umma_idesc_bf16_m128(p.cols);
-        for (int c = 0; c < chunks; ++c) {
+        const uint32_t acc = tmem + (uint32_t)(kLinMaxCols * t);
+        for (int c = t; c < chunks; c += kLinIssuers) {
             const int s = c % kLinStages;
             if (!lin_wait(&full[s], (uint32_t)((c / kLinStages) & 1), p, abort_flag)) break;
             tc_fence_after();
@@ -250,24 +261,25 @@ __global__ void __launch_bounds__(kLinThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < kLinKC / 16; ++kk) {
                 const uint64_t da = umma_desc_sw128(a + 32 * kk);
-                umma_bf16(tmem, da, umma_desc_sw128(b + 32 * kk), idesc, (c | kk) != 0 ? 1u : 0u);
-                if (p.two_terms) umma_bf16(tmem, da, umma_desc_sw128(b + term_bytes + 32 * kk), idesc, 1u);
+                umma_bf16(acc, da, umma_desc_sw128(b + 32 * kk), idesc, (c != t || kk != 0) ? 1u : 0u);
+                if (p.two_terms) umma_bf16(acc, da, umma_desc_sw128(b + term_bytes + 32 * kk), idesc, 1u);
             }
             umma_commit(&empty[s]);   // the stage is free once these products have read it
         }
         umma_commit(acc_bar);         // every product issued above has completed
-    } else if (warp >= 2) {
+    } else if (warp == 1) {
         // the row scales of this CTA's batch rows (from the previous launch)
         if (p.wait_acts) pdl_wait();
-        for (int j = threadIdx.x - 64; j < p.cols; j += kLinThreads - 64) {
+        for (int j = lane; j < p.cols; j += 32) {
             const int b = b0 + j;
             scale_s[j] = (p.row_scale != nullptr && b < p.batch) ? __ldg(p.row_scale + b) : 1.f;
         }
     }
     __syncwarp();
 
-    // Epilogue: warp w holds tensor-memory lanes 32w..32w+31 = weight rows
-    // n0 + 32w + lane. Each CTA owns rows [part*R, part*R + R) of the tile,
+    // Epilogue: warp w < 4 holds tensor-memory lanes 32w..32w+31 = weight rows
+    // n0 + 32w + lane, and adds the issuers' accumulators in issuer order.
+    // Each CTA owns rows [part*R, part*R + R) of the tile,
     // R = 128 / k_split, laid out [part][cols][R]; every CTA of the cluster
     // stores its partial values of those rows into the owner's tile with
     // asynchronous stores that complete their bytes on the owner's tile
@@ -277,24 +289,31 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     // (warp-uniform: tcgen05.ld is a whole-warp instruction)
     const bool ok = __all_sync(kFull, lin_wait(acc_bar, 0u, p, abort_flag) && *abort_flag == 0);
     tc_fence_after();
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
-    {
+    if (p.k_split > 1) cluster_wait();   // every peer's tile barrier is initialised (warps converged here)
+    if (warp < 4) {
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+        const int naccs = min(kLinIssuers, chunks);   // accumulators that received products
         const int r = 32 * warp + lane;
         const int owner = r / rows, rr = r % rows;
         float* tile = reinterpret_cast<float*>(smem + kLinSmemTile);
         const uint32_t elem = smem_addr(tile + (size_t)part * p.cols * rows + rr);
-        if (p.k_split > 1) cluster_wait();   // every peer's tile barrier is initialised (warp converged here)
         const bool local = owner == part;
         const uint32_t dst = local ? elem : cluster_map(elem, (uint32_t)owner);
         const uint32_t dst_bar = local ? 0u : cluster_map(smem_addr(tile_bar), (uint32_t)owner);
         for (int j0 = 0; j0 < p.cols; j0 += 16) {
             uint32_t v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = 0u;
             if (ok) {
                 tmem_ld16(lane_base + (uint32_t)j0, v);
                 tmem_ld_wait();
-            } else {
+                for (int a = 1; a < naccs; ++a) {
+                    uint32_t w[16];
+                    tmem_ld16(lane_base + (uint32_t)(kLinMaxCols * a + j0), w);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] = 0u;
+                    for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(w[i]));
+                }
             }
             if (local) {
 #pragma unroll

@@ -47,7 +47,7 @@ def check_y(got, x, w, label):
     assert off <= 0.005, f"{label}: {off:.4%} not the correctly rounded value"
 
 
-@pytest.mark.parametrize("B", [1, 7, 16, 32, 33, 64, 65, 128, 200, 256])
+@pytest.mark.parametrize("B", [1, 2, 3, 4, 7, 8, 9, 16, 32, 33, 64, 65, 128, 200, 256])
 def test_parity_at_batch_sizes(handles, B):
     d = inputs.o_proj_inputs(B, seed=200 + B, device="cuda")
     y = handles[16].o_proj(d["x"], d["w_o"])
@@ -55,10 +55,12 @@ def test_parity_at_batch_sizes(handles, B):
     check_y(y, d["x"], d["w_o"], f"B={B}")
 
 
+@pytest.mark.parametrize("B", [3, 24])
 @pytest.mark.parametrize("hq,hidden", [(16, 2048), (32, 2560), (64, 5120)])
-def test_parity_at_larger_sizes(handles, hq, hidden):
-    """Qwen3-1.7B (hidden 2048), 4B (2560, 32 heads), 32B (5120, 64 heads)."""
-    d = inputs.o_proj_inputs(24, seed=hidden + hq, device="cuda", hidden=hidden, num_q_heads=hq)
+def test_parity_at_larger_sizes(handles, hq, hidden, B):
+    """Qwen3-1.7B (hidden 2048), 4B (2560, 32 heads), 32B (5120, 64 heads);
+    B = 3 runs the small-batch product with its K range in parts."""
+    d = inputs.o_proj_inputs(B, seed=hidden + hq + B, device="cuda", hidden=hidden, num_q_heads=hq)
     y = handles[hq].o_proj(d["x"], d["w_o"])
     assert handles[hq].check() == 0
     check_y(y, d["x"], d["w_o"], f"Hq={hq} hidden={hidden}")

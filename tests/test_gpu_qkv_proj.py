@@ -65,7 +65,7 @@ def run_proj(attn, d):
     return qkv
 
 
-@pytest.mark.parametrize("B", [1, 5, 16, 17, 32, 33, 64, 65, 128, 129, 200, 256])
+@pytest.mark.parametrize("B", [1, 2, 3, 4, 5, 8, 9, 16, 17, 32, 33, 64, 65, 128, 129, 200, 256])
 def test_parity_at_batch_sizes(handles, B):
     d = inputs.hidden_inputs(B, seed=100 + B)
     ref = oracle.input_norm_qkv_proj(inputs.bf16_bits(d["x"]), inputs.bf16_bits(d["input_norm_w"]),
@@ -73,10 +73,12 @@ def test_parity_at_batch_sizes(handles, B):
     check_qkv(run_proj(handles[16], d), ref, f"B={B}", d)
 
 
+@pytest.mark.parametrize("B", [3, 24])
 @pytest.mark.parametrize("hq,hidden", [(16, 2048), (32, 2560), (64, 5120)])
-def test_parity_at_larger_sizes(handles, hq, hidden):
-    """Qwen3-1.7B (hidden 2048), 4B (2560, 32 heads), 32B (5120, 64 heads)."""
-    d = inputs.hidden_inputs(24, seed=hidden, hidden=hidden, num_q_heads=hq)
+def test_parity_at_larger_sizes(handles, hq, hidden, B):
+    """Qwen3-1.7B (hidden 2048), 4B (2560, 32 heads), 32B (5120, 64 heads);
+    B = 3 runs the small-batch product with its K range in parts."""
+    d = inputs.hidden_inputs(B, seed=hidden + B, hidden=hidden, num_q_heads=hq)
     ref = oracle.input_norm_qkv_proj(inputs.bf16_bits(d["x"]), inputs.bf16_bits(d["input_norm_w"]),
                                      inputs.bf16_bits(d["w_qkv"]))
     check_qkv(run_proj(handles[hq], d), ref, f"Hq={hq} hidden={hidden}", d)
