@@ -160,6 +160,25 @@ __device__ __forceinline__ bool lin_wait(uint64_t* bar, uint32_t parity, const L
     return false;
 }
 
+// Columns [j0, j0 + 16) of this warp's 32 tensor-memory lanes, summed over the
+// first `naccs` accumulators (64 columns apart) in accumulator order; all the
+// loads are in flight before the one wait.
+__device__ __forceinline__ void load_acc_sum(uint32_t lane_base, int j0, int naccs, uint32_t (&v)[16]) {
+    uint32_t w[kLinIssuers][16];
+#pragma unroll
+    for (int a = 0; a < kLinIssuers; ++a)
+        if (a < naccs) tmem_ld16(lane_base + (uint32_t)(kLinMaxCols * a + j0), w[a]);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        float sum = __uint_as_float(w[0][i]);
+#pragma unroll
+        for (int a = 1; a < kLinIssuers; ++a)
+            if (a < naccs) sum += __uint_as_float(w[a][i]);
+        v[i] = __float_as_uint(sum);
+    }
+}
+
 __global__ void __launch_bounds__(kLinThreads, 1)
     linear_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_hi,
                      const __grid_constant__ CUtensorMap tm_lo, const LinearParams p) {
@@ -289,79 +308,90 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     // (warp-uniform: tcgen05.ld is a whole-warp instruction)
     const bool ok = __all_sync(kFull, lin_wait(acc_bar, 0u, p, abort_flag) && *abort_flag == 0);
     tc_fence_after();
-    if (p.k_split > 1) cluster_wait();   // every peer's tile barrier is initialised (warps converged here)
-    if (warp < 4) {
-        const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
-        const int naccs = min(kLinIssuers, chunks);   // accumulators that received products
-        const int r = 32 * warp + lane;
-        const int owner = r / rows, rr = r % rows;
-        float* tile = reinterpret_cast<float*>(smem + kLinSmemTile);
-        const uint32_t elem = smem_addr(tile + (size_t)part * p.cols * rows + rr);
-        const bool local = owner == part;
-        const uint32_t dst = local ? elem : cluster_map(elem, (uint32_t)owner);
-        const uint32_t dst_bar = local ? 0u : cluster_map(smem_addr(tile_bar), (uint32_t)owner);
-        for (int j0 = 0; j0 < p.cols; j0 += 16) {
-            uint32_t v[16];
+    const int naccs = min(kLinIssuers, chunks);   // accumulators that received products
+    if (p.k_split == 1) {
+        // No K parts: each thread scales and stores its weight row's outputs from
+        // registers (a warp's 32 lanes write 32 consecutive outputs per batch row).
+        __syncthreads();   // the row scales
+        if (warp < 4 && ok) {
+            const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+            const int n = n0 + 32 * warp + lane;
+            for (int j0 = 0; j0 < p.cols; j0 += 16) {
+                uint32_t v[16];
+                load_acc_sum(lane_base, j0, naccs, v);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = 0u;
-            if (ok) {
-                tmem_ld16(lane_base + (uint32_t)j0, v);
-                tmem_ld_wait();
-                for (int a = 1; a < naccs; ++a) {
-                    uint32_t w[16];
-                    tmem_ld16(lane_base + (uint32_t)(kLinMaxCols * a + j0), w);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(w[i]));
+                for (int i = 0; i < 16; ++i) {
+                    const int b = b0 + j0 + i;
+                    if (b < p.batch)
+                        p.y[(size_t)b * p.n_out + n] =
+                            __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[i]) * scale_s[j0 + i]));
                 }
             }
-            if (local) {
+        }
+    } else {   // K parts
+        cluster_wait();   // every peer's tile barrier is initialised (warps converged here)
+        if (warp < 4) {
+            const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+            const int r = 32 * warp + lane;
+            const int owner = r / rows, rr = r % rows;
+            float* tile = reinterpret_cast<float*>(smem + kLinSmemTile);
+            const uint32_t elem = smem_addr(tile + (size_t)part * p.cols * rows + rr);
+            const bool local = owner == part;
+            const uint32_t dst = local ? elem : cluster_map(elem, (uint32_t)owner);
+            const uint32_t dst_bar = local ? 0u : cluster_map(smem_addr(tile_bar), (uint32_t)owner);
+            for (int j0 = 0; j0 < p.cols; j0 += 16) {
+                uint32_t v[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) tile[((size_t)part * p.cols + j0 + i) * rows + rr] = __uint_as_float(v[i]);
-            } else {
+                for (int i = 0; i < 16; ++i) v[i] = 0u;
+                if (ok) load_acc_sum(lane_base, j0, naccs, v);
+                if (local) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    st_async_f32(dst + (uint32_t)((j0 + i) * rows * 4), __uint_as_float(v[i]), dst_bar);
+                    for (int i = 0; i < 16; ++i) tile[((size_t)part * p.cols + j0 + i) * rows + rr] = __uint_as_float(v[i]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        st_async_f32(dst + (uint32_t)((j0 + i) * rows * 4), __uint_as_float(v[i]), dst_bar);
+                }
+            }
+        }
+        __syncthreads();   // this CTA's own part is in the tile
+        {
+            // the other parts: a bounded wait that does not give up on this CTA's
+            // abort flag, since their stores land here whatever this CTA did
+            if (threadIdx.x == 0 && !mbar_wait(tile_bar, 0u, p.timeout_ns, nullptr)) {
+                *abort_flag = 1;
+                record_error(p.status, QDA_ERR_TIMEOUT);
+            }
+            __syncthreads();
+        }
+        {
+            const float* tile = reinterpret_cast<const float*>(smem + kLinSmemTile);
+            const int oct = rows / 8;
+            for (int e = threadIdx.x; e < oct * p.cols; e += kLinThreads) {
+                const int j = e / oct, rr = 8 * (e % oct);
+                const int b = b0 + j;
+                float acc[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+                for (int q = 0; q < p.k_split; ++q) {
+                    const float4* src = reinterpret_cast<const float4*>(tile + ((size_t)q * p.cols + j) * rows + rr);
+                    const float4 x0 = src[0], x1 = src[1];
+                    acc[0] += x0.x; acc[1] += x0.y; acc[2] += x0.z; acc[3] += x0.w;
+                    acc[4] += x1.x; acc[5] += x1.y; acc[6] += x1.z; acc[7] += x1.w;
+                }
+                if (b < p.batch && *abort_flag == 0) {
+                    const float sc = scale_s[j];
+                    uint4 w;
+                    w.x = pack_bf2(acc[0] * sc, acc[1] * sc);
+                    w.y = pack_bf2(acc[2] * sc, acc[3] * sc);
+                    w.z = pack_bf2(acc[4] * sc, acc[5] * sc);
+                    w.w = pack_bf2(acc[6] * sc, acc[7] * sc);
+                    *reinterpret_cast<uint4*>(p.y + (size_t)b * p.n_out + n0 + part * rows + rr) = w;
+                }
             }
         }
     }
     tc_fence_before();
-    __syncthreads();   // this CTA's own part is in the tile
-    if (p.k_split > 1) {
-        // the other parts: a bounded wait that does not give up on this CTA's
-        // abort flag, since their stores land here whatever this CTA did
-        if (threadIdx.x == 0 && !mbar_wait(tile_bar, 0u, p.timeout_ns, nullptr)) {
-            *abort_flag = 1;
-            record_error(p.status, QDA_ERR_TIMEOUT);
-        }
-        __syncthreads();
-    }
-    {
-        const float* tile = reinterpret_cast<const float*>(smem + kLinSmemTile);
-        const int oct = rows / 8;
-        for (int e = threadIdx.x; e < oct * p.cols; e += kLinThreads) {
-            const int j = e / oct, rr = 8 * (e % oct);
-            const int b = b0 + j;
-            float acc[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) acc[k] = 0.f;
-            for (int q = 0; q < p.k_split; ++q) {
-                const float4* src = reinterpret_cast<const float4*>(tile + ((size_t)q * p.cols + j) * rows + rr);
-                const float4 x0 = src[0], x1 = src[1];
-                acc[0] += x0.x; acc[1] += x0.y; acc[2] += x0.z; acc[3] += x0.w;
-                acc[4] += x1.x; acc[5] += x1.y; acc[6] += x1.z; acc[7] += x1.w;
-            }
-            if (b < p.batch && *abort_flag == 0) {
-                const float sc = scale_s[j];
-                uint4 w;
-                w.x = pack_bf2(acc[0] * sc, acc[1] * sc);
-                w.y = pack_bf2(acc[2] * sc, acc[3] * sc);
-                w.z = pack_bf2(acc[4] * sc, acc[5] * sc);
-                w.w = pack_bf2(acc[6] * sc, acc[7] * sc);
-                *reinterpret_cast<uint4*>(p.y + (size_t)b * p.n_out + n0 + part * rows + rr) = w;
-            }
-        }
-    }
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
