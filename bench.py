@@ -173,16 +173,16 @@ def kernel_source_hash(num_q_heads: int = 16, new_tokens: int = 1, key=None) -> 
     return h.hexdigest()
 
 
-def traffic_per_launch(workload: str, num_q_heads: int = 16, new_tokens: int = 1):
-    """DRAM bytes per call from the committed ncu summary, if it was taken on
-    this kernel source and workload (else None)."""
+def traffic_per_launch(workload: str, num_q_heads: int = 16, new_tokens: int = 1, key=None):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, if it was taken on this kernel source and workload (else None)."""
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
     except (OSError, ValueError):
         return None
     entry = t.get(workload)
-    if not entry or entry.get("kernel_source_sha256") != kernel_source_hash(num_q_heads, new_tokens):
+    if not entry or entry.get("kernel_source_sha256") != kernel_source_hash(num_q_heads, new_tokens, key):
         return None
     return entry.get("dram_bytes_per_launch")
 
@@ -653,8 +653,12 @@ def measure(args, dist, rank, world, dev, headline: bool):
     alg_per_launch = alg_per_step_local / calls_per_step
     peak, peak_kind = hbm_peak()
     achieved = alg_per_launch / (mean_kernel_ms * 1e-3) / 1e9
-    traffic = (traffic_per_launch(workload_key(args.workload, args.num_q_heads, T), args.num_q_heads, T)
-               if mode == "attention" else None)
+    if mode == "attention":
+        traffic = traffic_per_launch(workload_key(args.workload, args.num_q_heads, T), args.num_q_heads, T)
+    elif mode in ("qkv_proj", "o_proj") and args.num_q_heads == 16 and args.hidden == inputs.HIDDEN:
+        traffic = traffic_per_launch(f"{args.workload}-{mode}", key="qkv_proj")   # the product launch's
+    else:
+        traffic = None
 
     # the other way of timing, for comparison: eager launches with an event pair around each
     if not headline:
