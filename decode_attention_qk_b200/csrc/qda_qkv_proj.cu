@@ -21,10 +21,12 @@
 //   weight rows as the A operand (M = 128) and C <= 64 batch rows as the B
 //   operand (N = C). A producer thread streams 128 x 64 weight boxes and the
 //   matching C x 64 boxes of hi and lo into a 4-stage shared ring by tiled
-//   copies with the 128-byte swizzle; one thread issues tcgen05.mma (two per
-//   16-wide K step: hi, then lo, into the same accumulator) and frees each
-//   stage with tcgen05.commit; the accumulator lives in tensor memory and the
-//   four warps read it back (tcgen05.ld) for the epilogue.
+//   copies with the 128-byte swizzle; four threads issue tcgen05.mma, thread
+//   t taking every chunk of stage t into its own accumulator in tensor memory
+//   (two products per 16-wide K step: hi, then lo), and free the stage with
+//   tcgen05.commit; four warps read the accumulators back (tcgen05.ld) and
+//   add them in order for the epilogue. (One issuing thread stalls on the
+//   products it issues; four keep four chains in flight.)
 //
 //   The work split fills the SMs at any batch: the batch is cut in groups
 //   of at most 64 rows, and the K range in P = 1, 2, 4 or 8 parts, the
