@@ -139,21 +139,40 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def n_chunks(args) -> int:
-    """Launches of the tensor-core attention kernel per call: a block of new
-    tokens longer than one launch takes (16 query rows per kv head) runs in chunks."""
+PREFILL_FROM = 64   # query rows per kv head from which a block runs as the prefill
+
+
+def chunk_tokens(args) -> list:
+    """New tokens per launch of the tensor-core attention in one call: up to 16
+    query rows per kv head (T * Hq / 8) in one decode-shaped launch; from
+    PREFILL_FROM rows a chunked prefill of 128 / G tokens per chunk; in between
+    chunks of 16 / G tokens of the decode-shaped kernel (at 16 query heads a last
+    chunk of one token borrows one)."""
     T, G = args.new_tokens, args.num_q_heads // 8
-    max_t = 16 // G
-    if T <= max_t:
-        return 1
-    n, c0 = 0, 0
+    if T * G <= 16:
+        return [T]
+    prefill = T * G >= PREFILL_FROM
+    max_t = 128 // G if prefill else 16 // G
+    sizes, c0 = [], 0
     while c0 < T:
         k = min(max_t, T - c0)
-        if args.num_q_heads == 16 and T - c0 - k == 1:
+        if not prefill and args.num_q_heads == 16 and T - c0 - k == 1:
             k -= 1
+        sizes.append(k)
         c0 += k
-        n += 1
-    return n
+    return sizes
+
+
+def n_chunks(args) -> int:
+    return len(chunk_tokens(args))
+
+
+def grouped_launches(args) -> int:
+    """Kernel launches of a several-token call: per decode-shaped chunk the
+    attention and its combine, per prefill chunk the append, the attention and
+    the combine."""
+    T, G = args.new_tokens, args.num_q_heads // 8
+    return (3 if T * G >= PREFILL_FROM else 2) * n_chunks(args)
 
 
 def kernel_key(num_q_heads: int = 16, new_tokens: int = 1):
@@ -736,10 +755,11 @@ def measure(args, dist, rank, world, dev, headline: bool):
             ("eager" if args.timing == "graph" else "graph"): other,
             "seq_per_s": round(first[0].batch / (ms_per_step * 1e-3) * world, 1),
             # the 16-head attention: one launch per call, the tensor-core attention two (attention,
-            # combine; per chunk of a long block); the projection two (split, product), o_proj one
+            # combine) or three per prefill chunk (grouped_launches); the projection two (split,
+            # product), o_proj one
             "gpu_launches": n_launch * ({"qkv_proj": 2, "o_proj": 1, "from_hidden": 2}.get(mode, 0)
                                         + (0 if mode in ("qkv_proj", "o_proj") else
-                                           (1 if kernel_key(args.num_q_heads, T) == 16 else 2 * n_chunks(args)))),
+                                           (1 if kernel_key(args.num_q_heads, T) == 16 else grouped_launches(args)))),
             "clocks": clk,
         }
     if dist is not None:

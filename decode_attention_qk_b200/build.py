@@ -16,8 +16,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libqwen3_decode_attn.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("qda_decode_kernel.cu", "qda_decode_mma.cu", "qda_qkv_proj.cu", "qda_api.cu",
-                                           "qda_noalloc.cu", "qda_host_stage.cu")]
+                                           "qda_noalloc.cu", "qda_host_stage.cu", "qda_prefill.cu")]
 HEADERS = [os.path.join(CSRC, "qda_internal.h"), os.path.join(CSRC, "qda_device.cuh"), os.path.join(CSRC, "qda_tc.cuh"),
+           os.path.join(CSRC, "qda_prefill.h"),
            os.path.join(INCLUDE, "qwen3_decode_attn.h")]
 
 NVCC_FLAGS = [

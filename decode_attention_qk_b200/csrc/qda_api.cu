@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include "qda_internal.h"
+#include "qda_prefill.h"
 #include "qwen3_decode_attn.h"
 
 struct qda_handle {
@@ -18,6 +19,10 @@ struct qda_handle {
     float2* part_ml = nullptr;
     int* counters = nullptr;
     int* seg = nullptr;
+    // the chunked prefill's partials (2 slots per CTA of its attention launch)
+    float* pf_acc = nullptr;
+    float2* pf_ml = nullptr;
+    int pf_grid = 0;
     int* status = nullptr;
     // input_norm + qkv_proj: the exact split of x*g, and 1/r per row
     uint16_t* xg_hi = nullptr;
@@ -67,6 +72,8 @@ void free_workspace(qda_handle* h) {
     cudaFree(h->part_ml);
     cudaFree(h->counters);
     cudaFree(h->seg);
+    cudaFree(h->pf_acc);
+    cudaFree(h->pf_ml);
     cudaFree(h->status);
     cudaFree(h->xg_hi);
     cudaFree(h->xg_lo);
@@ -229,7 +236,7 @@ int qwen3_decode_attn_create(const qda_config* cfg, int device, qda_handle** out
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms < 1)
         return QDA_ERR_CUDA;
     if (qda::prepare_device() != cudaSuccess || qda::prepare_grouped() != cudaSuccess ||
-        qda::prepare_qkv_proj() != cudaSuccess)
+        qda::prepare_qkv_proj() != cudaSuccess || qda::prepare_prefill() != cudaSuccess)
         return QDA_ERR_CUDA;
 
     qda_handle* h = new (std::nothrow) qda_handle();
@@ -237,6 +244,7 @@ int qwen3_decode_attn_create(const qda_config* cfg, int device, qda_handle** out
     h->device = device;
     h->cfg = *cfg;
     h->grid = cfg->grid_ctas > 0 ? cfg->grid_ctas : sms;
+    h->pf_grid = sms;
 
     const size_t slots = (size_t)qda::num_slots(h->grid, cfg->max_batch);
     const size_t B = (size_t)cfg->max_batch;
@@ -248,6 +256,7 @@ int qwen3_decode_attn_create(const qda_config* cfg, int device, qda_handle** out
               alloc(&h->part_ml, slots * rows * sizeof(float2)) &&
               alloc(&h->counters, (size_t)qda::kMaxBatch * qda::kNumKvHeads * sizeof(int)) &&
               alloc(&h->status, sizeof(int)) && alloc(&h->seg, (size_t)(qda::kMaxBatch + 1) * sizeof(int)) &&
+              alloc(&h->pf_acc, qda::prefill_acc_bytes(sms)) && alloc(&h->pf_ml, qda::prefill_ml_bytes(sms)) &&
               alloc(&h->xg_hi, B * (size_t)qda::kMaxHidden * sizeof(uint16_t)) &&
               alloc(&h->xg_lo, B * (size_t)qda::kMaxHidden * sizeof(uint16_t)) &&
               alloc(&h->inv_r, B * sizeof(float));
@@ -299,6 +308,26 @@ int qwen3_decode_attn_append_and_attend_tokens(qda_handle* h, const void* qkv, c
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     p.tok_stride = new_tokens;
     if (new_tokens == 1) return launch_step(h, p, st) == cudaSuccess ? QDA_OK : QDA_ERR_CUDA;
+    const int G = h->cfg.num_q_heads / qda::kNumKvHeads;
+    if (new_tokens * G >= qda::kPrefillFrom) {
+        // Long blocks: the chunked prefill, up to kPrefillRows query rows per
+        // kv head per launch (the cache read once per chunk), each chunk seeing
+        // the cache plus the block's tokens up to its own. (Below kPrefillFrom
+        // rows the 16-row launches of the decode-shaped kernel are faster: the
+        // prefill's warps share one kv head's pages, which few rows do not
+        // keep busy.)
+        const qda::PrefillScratch sc{h->pf_acc, h->pf_ml, h->pf_grid};
+        const int max_t = qda::prefill_max_tokens(h->cfg.num_q_heads);
+        for (int c0 = 0; c0 < new_tokens;) {
+            const int n = new_tokens - c0 < max_t ? new_tokens - c0 : max_t;
+            p.new_tokens = n;
+            p.tok_offset = c0;
+            p.len_trim = new_tokens - c0 - n;
+            if (qda::launch_prefill(p, sc, st) != cudaSuccess) return QDA_ERR_CUDA;
+            c0 += n;
+        }
+        return QDA_OK;
+    }
     // A block longer than one launch takes runs as consecutive launches over
     // consecutive chunks of its tokens. Chunk [c0, c0 + n) sees the cache plus
     // the block's tokens up to its own (its launch trims the later ones from

@@ -286,3 +286,28 @@ def test_config2_shape_full_size(handles, hq, T):
 def test_config4_shape_full_size(handles):
     w = inputs.config4("cuda", new_tokens=4)
     full_size_check(handles[16], w, [1, 2], "cfg4 T=4")
+
+
+@pytest.mark.parametrize("hq,T", [(16, 130), (32, 70), (40, 30), (64, 40)])
+def test_prefill_in_several_chunks(handles, hq, T):
+    """Blocks of more than 128 query rows per kv head: several prefill launches
+    (128 / G tokens each), each seeing the block's tokens up to its own."""
+    lens = [T, T + 1, T + 15, T + 16, T + 17, T + 700, T + 1500]
+    w = inputs.custom(lens, seed=90 + hq + T, device="cuda", gap_fraction=0.2, num_q_heads=hq, new_tokens=T)
+    full_check(handles[hq], w, f"Hq={hq} T={T} prefill chunks")
+
+
+def test_prefill_with_positions(handles):
+    w = inputs.custom([33, 40, 2000, 600], seed=95, device="cuda", gap_fraction=0.1, num_q_heads=32, new_tokens=33)
+    full_check(handles[32], w, "Hq=32 T=33 positions", positions=torch.tensor([0, 7, 4000, 100], dtype=torch.int32))
+
+
+@pytest.mark.parametrize("hq,T", [(16, 16), (16, 64), (64, 16)])
+def test_config2_shape_full_size_prefill(handles, hq, T):
+    w = inputs.config2("cuda", num_q_heads=hq, new_tokens=T)
+    full_size_check(handles[hq], w, list(range(2, 32, 5)), f"cfg2 Hq={hq} T={T} prefill")
+
+
+def test_config4_shape_full_size_prefill(handles):
+    w = inputs.config4("cuda", new_tokens=32)
+    full_size_check(handles[16], w, [0, 3], "cfg4 T=32 prefill")
