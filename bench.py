@@ -47,6 +47,8 @@ KERNEL_SOURCES = {   # the files each attention kernel is built from
     16: [os.path.join(_CSRC, f) for f in ("qda_decode_kernel.cu", "qda_device.cuh", "qda_internal.h")],
     "grouped": [os.path.join(_CSRC, f) for f in ("qda_decode_mma.cu", "qda_device.cuh", "qda_internal.h")],
     "qkv_proj": [os.path.join(_CSRC, f) for f in ("qda_qkv_proj.cu", "qda_device.cuh", "qda_internal.h")],
+    "prefill": [os.path.join(_CSRC, f)
+                for f in ("qda_prefill.cu", "qda_prefill.h", "qda_tc.cuh", "qda_device.cuh", "qda_internal.h")],
 }
 
 WORKLOADS = {
@@ -139,28 +141,15 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-PREFILL_FROM = 64   # query rows per kv head from which a block runs as the prefill
-
-
 def chunk_tokens(args) -> list:
     """New tokens per launch of the tensor-core attention in one call: up to 16
-    query rows per kv head (T * Hq / 8) in one decode-shaped launch; from
-    PREFILL_FROM rows a chunked prefill of 128 / G tokens per chunk; in between
-    chunks of 16 / G tokens of the decode-shaped kernel (at 16 query heads a last
-    chunk of one token borrows one)."""
+    query rows per kv head (T * Hq / 8) in one decode-shaped launch; a longer
+    block as a chunked prefill of 128 / G tokens per chunk."""
     T, G = args.new_tokens, args.num_q_heads // 8
     if T * G <= 16:
         return [T]
-    prefill = T * G >= PREFILL_FROM
-    max_t = 128 // G if prefill else 16 // G
-    sizes, c0 = [], 0
-    while c0 < T:
-        k = min(max_t, T - c0)
-        if not prefill and args.num_q_heads == 16 and T - c0 - k == 1:
-            k -= 1
-        sizes.append(k)
-        c0 += k
-    return sizes
+    max_t = 128 // G
+    return [min(max_t, T - c0) for c0 in range(0, T, max_t)]
 
 
 def n_chunks(args) -> int:
@@ -168,16 +157,19 @@ def n_chunks(args) -> int:
 
 
 def grouped_launches(args) -> int:
-    """Kernel launches of a several-token call: per decode-shaped chunk the
-    attention and its combine, per prefill chunk the append, the attention and
-    the combine."""
+    """Kernel launches of a several-token call: the decode-shaped attention and
+    its combine, or per prefill chunk the prep, the attention and the combine."""
     T, G = args.new_tokens, args.num_q_heads // 8
-    return (3 if T * G >= PREFILL_FROM else 2) * n_chunks(args)
+    return 2 if T * G <= 16 else 3 * n_chunks(args)
 
 
 def kernel_key(num_q_heads: int = 16, new_tokens: int = 1):
-    """Which attention kernel a call runs: the 16-head decode kernel or the tensor-core one."""
-    return 16 if num_q_heads == 16 and new_tokens == 1 else "grouped"
+    """Which attention kernel a call runs: the 16-head decode kernel, the
+    decode-shaped tensor-core one (up to 16 query rows per kv head) or the
+    prefill."""
+    if num_q_heads == 16 and new_tokens == 1:
+        return 16
+    return "grouped" if new_tokens * (num_q_heads // 8) <= 16 else "prefill"
 
 
 def workload_key(workload: str, num_q_heads: int = 16, new_tokens: int = 1) -> str:

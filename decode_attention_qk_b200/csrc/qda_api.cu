@@ -19,7 +19,9 @@ struct qda_handle {
     float2* part_ml = nullptr;
     int* counters = nullptr;
     int* seg = nullptr;
-    // the chunked prefill's partials (2 slots per CTA of its attention launch)
+    // the chunked prefill: query tiles [max_batch][8], partials (2 slots per
+    // CTA of its attention launch)
+    uint16_t* pf_q = nullptr;
     float* pf_acc = nullptr;
     float2* pf_ml = nullptr;
     int pf_grid = 0;
@@ -72,6 +74,7 @@ void free_workspace(qda_handle* h) {
     cudaFree(h->part_ml);
     cudaFree(h->counters);
     cudaFree(h->seg);
+    cudaFree(h->pf_q);
     cudaFree(h->pf_acc);
     cudaFree(h->pf_ml);
     cudaFree(h->status);
@@ -256,6 +259,7 @@ int qwen3_decode_attn_create(const qda_config* cfg, int device, qda_handle** out
               alloc(&h->part_ml, slots * rows * sizeof(float2)) &&
               alloc(&h->counters, (size_t)qda::kMaxBatch * qda::kNumKvHeads * sizeof(int)) &&
               alloc(&h->status, sizeof(int)) && alloc(&h->seg, (size_t)(qda::kMaxBatch + 1) * sizeof(int)) &&
+              alloc(&h->pf_q, qda::prefill_q_bytes(cfg->max_batch)) &&
               alloc(&h->pf_acc, qda::prefill_acc_bytes(sms)) && alloc(&h->pf_ml, qda::prefill_ml_bytes(sms)) &&
               alloc(&h->xg_hi, B * (size_t)qda::kMaxHidden * sizeof(uint16_t)) &&
               alloc(&h->xg_lo, B * (size_t)qda::kMaxHidden * sizeof(uint16_t)) &&
@@ -308,42 +312,26 @@ int qwen3_decode_attn_append_and_attend_tokens(qda_handle* h, const void* qkv, c
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     p.tok_stride = new_tokens;
     if (new_tokens == 1) return launch_step(h, p, st) == cudaSuccess ? QDA_OK : QDA_ERR_CUDA;
-    const int G = h->cfg.num_q_heads / qda::kNumKvHeads;
-    if (new_tokens * G >= qda::kPrefillFrom) {
-        // Long blocks: the chunked prefill, up to kPrefillRows query rows per
-        // kv head per launch (the cache read once per chunk), each chunk seeing
-        // the cache plus the block's tokens up to its own. (Below kPrefillFrom
-        // rows the 16-row launches of the decode-shaped kernel are faster: the
-        // prefill's warps share one kv head's pages, which few rows do not
-        // keep busy.)
-        const qda::PrefillScratch sc{h->pf_acc, h->pf_ml, h->pf_grid};
-        const int max_t = qda::prefill_max_tokens(h->cfg.num_q_heads);
-        for (int c0 = 0; c0 < new_tokens;) {
-            const int n = new_tokens - c0 < max_t ? new_tokens - c0 : max_t;
-            p.new_tokens = n;
-            p.tok_offset = c0;
-            p.len_trim = new_tokens - c0 - n;
-            if (qda::launch_prefill(p, sc, st) != cudaSuccess) return QDA_ERR_CUDA;
-            c0 += n;
-        }
-        return QDA_OK;
+    if (new_tokens <= qda::grouped_max_tokens(h->cfg.num_q_heads)) {
+        // up to 16 query rows per kv head: one launch of the decode-shaped
+        // tensor-core kernel (and its combine)
+        p.new_tokens = new_tokens;
+        if (!qda::grouped_supported(h->cfg.num_q_heads, new_tokens)) return QDA_ERR_UNSUPPORTED;
+        return qda::launch_grouped(p, h->grid, st) == cudaSuccess ? QDA_OK : QDA_ERR_CUDA;
     }
-    // A block longer than one launch takes runs as consecutive launches over
-    // consecutive chunks of its tokens. Chunk [c0, c0 + n) sees the cache plus
-    // the block's tokens up to its own (its launch trims the later ones from
-    // seq_lens), so each token still attends over exactly the slots up to its
-    // own. At 16 query heads no chunk is a single token (that is the other
-    // kernel's shape): a remainder of one borrows a token from the chunk before.
-    const int max_t = qda::grouped_max_tokens(h->cfg.num_q_heads);
-    if (max_t < 2) return QDA_ERR_UNSUPPORTED;
+    // Longer blocks: the chunked prefill, up to kPrefillRows query rows per kv
+    // head per chunk (the cache read once per chunk). Chunk [c0, c0 + n) sees
+    // the cache plus the block's tokens up to its own (its launches trim the
+    // later ones from seq_lens), so each token still attends over exactly the
+    // slots up to its own.
+    const qda::PrefillScratch sc{h->pf_q, h->pf_acc, h->pf_ml, h->pf_grid};
+    const int max_t = qda::prefill_max_tokens(h->cfg.num_q_heads);
     for (int c0 = 0; c0 < new_tokens;) {
-        int n = new_tokens - c0 < max_t ? new_tokens - c0 : max_t;
-        if (h->cfg.num_q_heads == qda::kNumQHeads && new_tokens - c0 - n == 1) --n;
+        const int n = new_tokens - c0 < max_t ? new_tokens - c0 : max_t;
         p.new_tokens = n;
         p.tok_offset = c0;
         p.len_trim = new_tokens - c0 - n;
-        if (!qda::grouped_supported(h->cfg.num_q_heads, n)) return QDA_ERR_UNSUPPORTED;
-        if (qda::launch_grouped(p, h->grid, st) != cudaSuccess) return QDA_ERR_CUDA;
+        if (qda::launch_prefill(p, sc, st) != cudaSuccess) return QDA_ERR_CUDA;
         c0 += n;
     }
     return QDA_OK;

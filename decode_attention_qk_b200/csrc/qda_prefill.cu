@@ -10,28 +10,23 @@
 // launch covers a chunk of n tokens with n * G <= 128 rows per kv head and
 // reads the cache once:
 //
-//   1. prefill_append_kernel: one warp per (sequence, kv head, 32 tokens)
-//      forms the chunk's new k (RMSNorm and RoPE in double, rounded once to
-//      bf16) and writes k and v to their cache slots.
+//   1. prefill_prep_kernel: one warp per (sequence, kv head, token) forms the
+//      token's new k and writes k and v to their cache slots, and forms its G
+//      query rows of the kv head into the unit's 128-row query tile (scratch,
+//      already in the tensor cores' swizzled layout).
 //   2. prefill_kernel: the units (sequence b, kv head j) in order, each the
 //      pages of sequence b for kv head j, form one list of page-heads; CTA g
-//      takes an equal range of it (whatever the length mix). A producer
-//      thread fetches each page's 16 K rows and 16 V rows of kv head j with
-//      four tiled copies (a 3-D tensor map over the cache, boxes of 16 rows x
-//      64 dims with the 128-byte swizzle, so that the 8 rows an ldmatrix phase
-//      reads fall in 8 different bank groups; per-row copies of 256 bytes were
-//      bound by the copy engine's per-copy cost). Consumer warp w
-//      holds query rows 16w..16w+15 of the unit (row r: token r / G, head
-//      G*j + r % G) as one 16-row tile: mma.sync m16n8k16 bf16 products with
-//      float accumulators, q and the probabilities in bf16 (the running sums
-//      add the same rounded probabilities, so o stays a convex combination of
-//      the v rows), an online softmax with lazy rescaling, and each row's
-//      causal limit. A unit held whole by one CTA writes o; a split unit writes
-//      partials (running max, sum, un-normalised output) to its CTA's slot
-//      2g (the CTA's first unit) or 2g + 1 (its last).
-//   3. prefill_combine_kernel: one CTA per unit merges the partials of split
-//      units with the log-sum-exp rule (Supported models, "Facts proved about
-//      the specs": flashAttn_eq, softmax_shift).
+//      takes an equal range of it (whatever the length mix). Per unit piece
+//      the query tile is one 128-row operand of the 5th-generation tensor
+//      cores: S = Q K^T and O += P V with accumulators in tensor memory, the
+//      K and V tiles copied by the tensor memory accelerator (a 3-D tensor map
+//      over the cache, boxes of 16 rows x 64 dims with the 128-byte swizzle),
+//      the softmax one thread per row. A unit held whole by one CTA writes o;
+//      a split unit writes partials (running max, sum, un-normalised output)
+//      to its CTA's slot 2g (the CTA's first unit) or 2g + 1 (its last).
+//   3. prefill_combine_kernel: one warp per row of a split unit merges its
+//      partials with the log-sum-exp rule (Supported models, "Facts proved
+//      about the specs": flashAttn_eq, softmax_shift).
 //
 // All three are programmatic dependent launches; each waits for its
 // predecessor to complete before it touches global memory.
@@ -44,33 +39,12 @@
 #include "qda_device.cuh"
 #include "qda_internal.h"
 #include "qda_prefill.h"
+#include "qda_tc.cuh"
 #include "qwen3_decode_attn.h"
 
 namespace qda {
 namespace {
 
-constexpr int kPfWarps = 8;                          // consumer warps, 16 query rows each
-constexpr int kPfThreads = (kPfWarps + 1) * 32;
-// A stage: K dims 0-63, K dims 64-127, V dims 0-63, V dims 64-127 of one
-// page and kv head, each 16 rows x 128 bytes in the 128-byte swizzled layout
-// (row r's 16-byte piece c at piece c ^ (r % 8)).
-constexpr int kPfBoxBytes = kPage * 128;             // 2 KiB
-constexpr int kPfStageK = 0;
-constexpr int kPfStageV = 2 * kPfBoxBytes;
-constexpr int kPfStageBytes = 4 * kPfBoxBytes;       // 8 KiB
-constexpr int kPfStages = 16;
-constexpr int kPfSmemSeg = kPfStages * kPfStageBytes;            // int [kMaxBatch + 4]
-constexpr int kPfSmemLens = kPfSmemSeg + (kMaxBatch + 4) * 4;    // int [kMaxBatch]
-constexpr int kPfSmemInvFreq = kPfSmemLens + kMaxBatch * 4;      // double [64]
-constexpr int kPfSmemGains = kPfSmemInvFreq + 64 * 8;            // bf16 [128], the q gains
-constexpr int kPfSmemMeta = kPfSmemGains + kHeadDim * 2;         // StageMeta [kPfStages]
-constexpr int kPfSmemBars = kPfSmemMeta + kPfStages * 16;        // full [S], empty [S], never
-constexpr int kPfSmemFlags = kPfSmemBars + (2 * kPfStages + 1) * 8;
-constexpr int kPfSmemTotal = kPfSmemFlags + 16;
-constexpr int kPfSmemAlloc = kPfSmemTotal + 1024;   // slack to align the stages to 1024 bytes
-static_assert(kPfStageBytes % 1024 == 0 && kPfSmemInvFreq % 8 == 0 && kPfSmemBars % 8 == 0, "alignment");
-static_assert(kPfSmemAlloc <= 227 * 1024, "fits one CTA per SM");
-static_assert(kPfWarps * 16 == kPrefillRows, "one 16-row tile per consumer warp");
 
 // x - n * 2*pi for the integer n nearest x / (2*pi), in double: 2*pi is split
 // into a 32-bit head (n * head and x - n * head are exact for the |x| < 2^20
@@ -109,31 +83,37 @@ __device__ __forceinline__ int pf_first_position(const Params& p, int b, int L, 
 }
 
 // ---------------------------------------------------------------------------
-// 1. The append.
+// 1. The prep: warp w of CTA (b, j, z) takes token u = 4z + w of the chunk.
+// It forms the token's new k (RMSNorm and RoPE in double, rounded once to
+// bf16) and writes k and v to their cache slots, and forms the token's G query
+// rows of kv head j (RMSNorm and RoPE in float, the angle reduced modulo 2*pi
+// in double, scaled by log2(e)/sqrt(128), rounded to bf16) into the unit's
+// query tile in the attention's layout. Lane l holds dims 2l, 2l+1 (word l of
+// a head) and 64+2l, 65+2l (word 32+l), the RoPE pairs (i, i+64).
 
 template <int G>
-__global__ void __launch_bounds__(32) prefill_append_kernel(const Params p) {
+__global__ void __launch_bounds__(128) prefill_prep_kernel(const Params p, const PrefillScratch sc) {
     constexpr int kHq = G * kNumKvHeads;
     constexpr int kQkvW = (kHq + 2 * kNumKvHeads) * kHeadDim;
     pdl_wait();
     pdl_launch_dependents();
-    const int b = blockIdx.x, j = blockIdx.y, lane = threadIdx.x;
+    const int b = blockIdx.x, j = blockIdx.y, lane = threadIdx.x & 31;
+    const int u = 4 * (int)blockIdx.z + (int)(threadIdx.x >> 5);
     const int n = p.new_tokens;
+    if (u >= n) return;
     const int L_all = p.seq_lens[b];
     if (!length_ok(p, L_all)) return;   // the attention launch records it and skips the sequence
     const int L = L_all - p.len_trim;
-    const int pos0 = pf_first_position(p, b, L, n);
-    // lane l: dims 2l, 2l+1 (word l of the head) and 64+2l, 65+2l (word 32+l), all in double
-    const uint32_t* gk = reinterpret_cast<const uint32_t*>(p.k_norm_w);
-    const uint32_t wk_lo = gk[lane], wk_hi = gk[32 + lane];
-    const double f0 = pow(p.rope_theta, -2.0 * (2 * lane) / 128.0);
-    const double f1 = pow(p.rope_theta, -2.0 * (2 * lane + 1) / 128.0);
-    const int u_end = min(n, (int)(blockIdx.z + 1) * 32);
-    for (int u = (int)blockIdx.z * 32; u < u_end; ++u) {
-        const int slot = L - n + u;
-        const int page = __ldg(p.block_table + (size_t)b * p.bt_stride + slot / kPage);
-        if (page < 0 || page >= p.num_pages) continue;   // recorded by the attention launch
-        const uint32_t* row = reinterpret_cast<const uint32_t*>(p.qkv + pf_token_row(p, b, u) * kQkvW);
+    const double pos = (double)(pf_first_position(p, b, L, n) + u);
+    const double ang0 = reduce_angle(pos * pow(p.rope_theta, -2.0 * (2 * lane) / 128.0));
+    const double ang1 = reduce_angle(pos * pow(p.rope_theta, -2.0 * (2 * lane + 1) / 128.0));
+    const uint32_t* row = reinterpret_cast<const uint32_t*>(p.qkv + pf_token_row(p, b, u) * kQkvW);
+
+    const int slot = L - n + u;
+    const int page = __ldg(p.block_table + (size_t)b * p.bt_stride + slot / kPage);
+    if (page >= 0 && page < p.num_pages) {   // else recorded by the attention launch
+        const uint32_t* gk = reinterpret_cast<const uint32_t*>(p.k_norm_w);
+        const uint32_t wk_lo = gk[lane], wk_hi = gk[32 + lane];
         const uint32_t* xk = row + (kHq + j) * (kHeadDim / 2);
         const uint32_t* xv = row + (kHq + kNumKvHeads + j) * (kHeadDim / 2);
         const uint32_t xlo = xk[lane], xhi = xk[32 + lane];
@@ -145,10 +125,9 @@ __global__ void __launch_bounds__(32) prefill_append_kernel(const Params p) {
         a1 = a1 * inv_rr * bf_to_d(wk_lo >> 16);
         b0 = b0 * inv_rr * bf_to_d(wk_hi & 0xFFFFu);
         b1 = b1 * inv_rr * bf_to_d(wk_hi >> 16);
-        const double pos = (double)(pos0 + u);
         double sn0, cs0, sn1, cs1;
-        sincos(reduce_angle(pos * f0), &sn0, &cs0);
-        sincos(reduce_angle(pos * f1), &sn1, &cs1);
+        sincos(ang0, &sn0, &cs0);
+        sincos(ang1, &sn1, &cs1);
         const double ra0 = a0 * cs0 - b0 * sn0, rb0 = b0 * cs0 + a0 * sn0;
         const double ra1 = a1 * cs1 - b1 * sn1, rb1 = b1 * cs1 + a1 * sn1;
         const size_t off =
@@ -160,252 +139,153 @@ __global__ void __launch_bounds__(32) prefill_append_kernel(const Params p) {
         vd[lane] = vlo;
         vd[32 + lane] = vhi;
     }
+
+    float sn0, cs0, sn1, cs1;
+    sincosf((float)ang0, &sn0, &cs0);
+    sincosf((float)ang1, &sn1, &cs1);
+    const uint32_t* gq = reinterpret_cast<const uint32_t*>(p.q_norm_w);
+    const uint32_t wq_lo = gq[lane], wq_hi = gq[32 + lane];
+    const float scale = (float)kQScale;
+    uint8_t* tile = reinterpret_cast<uint8_t*>(sc.q) + (size_t)(b * kNumKvHeads + j) * kPrefillQTileBytes;
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+        const int r = u * G + hh;
+        const uint32_t* xq = row + (G * j + hh) * (kHeadDim / 2);
+        const uint32_t xlo = xq[lane], xhi = xq[32 + lane];
+        float ss = bf_lo(xlo) * bf_lo(xlo) + bf_hi(xlo) * bf_hi(xlo) + bf_lo(xhi) * bf_lo(xhi) + bf_hi(xhi) * bf_hi(xhi);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(kFull, ss, o);
+        const float inv_r = rsqrtf(ss * (1.f / 128.f) + (float)p.rms_eps);
+        const float ya0 = bf_lo(xlo) * inv_r * bf_lo(wq_lo), ya1 = bf_hi(xlo) * inv_r * bf_hi(wq_lo);
+        const float yb0 = bf_lo(xhi) * inv_r * bf_lo(wq_hi), yb1 = bf_hi(xhi) * inv_r * bf_hi(wq_hi);
+        const uint32_t qa = pack_bf2(fmaf(ya0, cs0, -yb0 * sn0) * scale, fmaf(ya1, cs1, -yb1 * sn1) * scale);
+        const uint32_t qb = pack_bf2(fmaf(yb0, cs0, ya0 * sn0) * scale, fmaf(yb1, cs1, ya1 * sn1) * scale);
+        // row r of each 64-dim half: 128 bytes, 16-byte piece c at piece c ^ (r % 8)
+        const uint32_t off = (uint32_t)r * 128u + ((((uint32_t)lane >> 2) ^ ((uint32_t)r & 7u)) << 4) + (lane & 3) * 4;
+        *reinterpret_cast<uint32_t*>(tile + off) = qa;
+        *reinterpret_cast<uint32_t*>(tile + kPrefillQTileBytes / 2 + off) = qb;
+    }
 }
 
 // ---------------------------------------------------------------------------
-// 2. The attention.
+// 2. The attention, on the 5th-generation tensor cores.
+//
+// A unit piece is (sequence b, kv head j, a range of b's pages). Its query
+// tile Q, 128 rows x 128 dims in bf16 (row r < R = n * G: token r / G, head
+// G*j + r % G; the rows from R on are never read out), is copied from the
+// prep launch's scratch into one of two shared-memory buffers, so that the
+// next piece's tile lands while this one runs. The cache arrives in stages of
+// 64 rows (4 pages) of K and V, and for each stage
+//   S = Q K^T     tcgen05.mma, M = 128 rows, N = 64 keys, K = 128 dims, into
+//                 one of two S buffers in tensor memory (S of the next stage
+//                 forms while this stage's softmax runs);
+//   softmax       one thread per row: the causal and length mask, the running
+//                 max with lazy rescaling of O, P = exp2(S - m) rounded to bf16
+//                 into shared memory (the running sum adds the same rounded
+//                 values, so o stays a convex combination of v rows);
+//   O += P V      M = 128 rows, N = 128 dims, K = 64 keys, V read MN-major
+//                 from its copied tile;
+// and O, accumulated in tensor memory over the piece, is read out once at the
+// piece's end.
+//
+// Warp roles (256 threads): warp 0 issues the copies; one thread of warp 1
+// issues the tensor-core instructions (warp 1 also allocates tensor memory);
+// warps 4-7 run the softmax and write o (warp 4 + w reads tensor-memory lanes
+// 32w..32w+31, the rows it owns). Every wait is bounded: a timeout records
+// QDA_ERR_TIMEOUT, sets the CTA's abort flag and every role leaves its loop;
+// tensor memory is freed after every issued instruction has completed.
 
-struct PfShared {
+constexpr int kTcKeys = 64;                          // cache rows per stage
+constexpr int kTcPages = kTcKeys / kPage;            // 4
+constexpr int kTcStages = 4;
+constexpr int kTcThreads = 8 * 32;
+constexpr int kTcHalf = kTcKeys * 128;               // 64 dims of a stage's rows: 8 KiB
+constexpr int kTcStageK = 0;                         // K dims 0-63 | K dims 64-127
+constexpr int kTcStageV = 2 * kTcHalf;               // V dims 0-63 | V dims 64-127
+constexpr int kTcStageBytes = 4 * kTcHalf;           // 32 KiB
+constexpr int kTcBoxBytes = kPage * 128;             // one copied box: 16 rows x 64 dims
+constexpr int kTcTile = kPrefillRows * 128;          // 64 columns of a 128-row operand: 16 KiB
+constexpr int kTcSmemQ = kTcStages * kTcStageBytes;  // 2 buffers: Q dims 0-63 | Q dims 64-127
+constexpr int kTcSmemP = kTcSmemQ + 4 * kTcTile;     // P: 128 rows x 64 keys
+constexpr int kTcSmemSeg = kTcSmemP + kTcTile;                       // int [kMaxBatch + 4]
+constexpr int kTcSmemLens = kTcSmemSeg + (kMaxBatch + 4) * 4;        // int [kMaxBatch]
+constexpr int kTcSmemMask = kTcSmemLens + kMaxBatch * 4;             // int [kTcStages]: pages not copied
+constexpr int kTcSmemBars = kTcSmemMask + kTcStages * 4;
+// kv_full[S], kv_empty[S], s_full[2], p_full, pv_done, q_full[2], q_free[2], fin
+constexpr int kTcNumBars = 2 * kTcStages + 9;
+constexpr int kTcSmemTmem = kTcSmemBars + kTcNumBars * 8;            // tensor-memory address, abort flag
+constexpr int kTcSmemTotal = kTcSmemTmem + 16;
+constexpr int kTcSmemAlloc = kTcSmemTotal + 1024;   // slack to align the tiles to 1024 bytes
+constexpr uint32_t kTcTmemCols = 256;               // S buffers at columns 0 and 64, O at 128
+constexpr uint32_t kTcTmemO = 128;
+static_assert(kTcStageBytes % 1024 == 0 && kTcSmemSeg % 1024 == 0, "swizzle atoms are 1024-byte aligned");
+static_assert(kTcSmemBars % 8 == 0 && 2 * kTcTile == kPrefillQTileBytes, "layout");
+static_assert(kTcSmemAlloc <= 227 * 1024, "fits one CTA per SM");
+static_assert(kTcKeys == 64, "a P row is one 128-byte swizzled row");
+
+struct TcShared {
     uint8_t* stages;
+    uint8_t* q;
+    uint8_t* p;
     int* seg;
     int* lens;
-    double* inv_freq;
-    const uint16_t* gains;
-    volatile StageMeta* meta;
-    uint64_t* full_bar;
-    uint64_t* empty_bar;
-    uint64_t* never_bar;
+    volatile int* mask;
+    uint64_t* kv_full;
+    uint64_t* kv_empty;
+    uint64_t* s_full;
+    uint64_t* p_full;
+    uint64_t* pv_done;
+    uint64_t* q_full;   // [2]
+    uint64_t* q_free;   // [2]
+    uint64_t* fin;
     volatile int* abort_flag;
 };
 
-// The unit holding global page-head x: sequence b, kv head j, page i of b.
-__device__ __forceinline__ void pf_locate(const PfShared& s, int B, int x, int& b, int& j, int& i) {
-    b = find_seq(s.seg, B, x >> 3);
-    const int np = s.seg[b + 1] - s.seg[b];
-    const int r = x - 8 * s.seg[b];
-    j = r / np;
-    i = r % np;
-}
-
-__device__ __forceinline__ void pf_producer(const Params& p, const PfShared& s, const CUtensorMap* tm_k,
-                                            const CUtensorMap* tm_v, int B, int start, int end, int lane) {
-    const int count = end - start;
-    int slot = 0;
-    uint32_t phase = 0;
-    uint32_t armed = 0, armed_parity = 0;
-    bool aborted = false;
-    for (int base = 0; base < count && !aborted; base += 32) {
-        const int x = start + base + lane;
-        int id = 0, head = 0;
-        if (x < end) {
-            int b, i;
-            pf_locate(s, B, x, b, head, i);
-            id = __ldg(p.block_table + (size_t)b * p.bt_stride + i);
-        }
-        const int m = min(32, count - base);
-        for (int kk = 0; kk < m; ++kk) {
-            const int page_id = __shfl_sync(kFull, id, kk);
-            const int page_head = __shfl_sync(kFull, head, kk);
-            int ok = 1;
-            if (lane == 0) {
-                ok = mbar_try_wait(&s.empty_bar[slot], phase ^ 1u) ||
-                     mbar_wait(&s.empty_bar[slot], phase ^ 1u, p.timeout_ns, s.abort_flag);
-                if (ok) {
-                    const bool bad = page_id < 0 || page_id >= p.num_pages;
-                    s.meta[slot].page = page_id;
-                    s.meta[slot].bad = bad ? 1 : 0;
-                    if (bad) record_error(p.status, QDA_ERR_BOUNDS);
-                    if (!bad) {
-                        // the page's 16 rows of kv head page_head, K and V, dims 0-63 and 64-127
-                        const uint32_t dst = smem_addr(s.stages + slot * kPfStageBytes);
-                        mbar_arrive_expect_tx(&s.full_bar[slot], (uint32_t)kPfStageBytes);
-                        for (int h = 0; h < 2; ++h) {
-                            tma_load_3d(dst + kPfStageK + h * kPfBoxBytes, tm_k, 64 * h, page_head, page_id * kPage,
-                                        &s.full_bar[slot]);
-                            tma_load_3d(dst + kPfStageV + h * kPfBoxBytes, tm_v, 64 * h, page_head, page_id * kPage,
-                                        &s.full_bar[slot]);
-                        }
-                        armed |= 1u << slot;
-                        armed_parity = (armed_parity & ~(1u << slot)) | (phase << slot);
-                    } else {
-                        mbar_arrive(&s.full_bar[slot]);
-                    }
-                } else {
-                    *s.abort_flag = 1;
-                    record_error(p.status, QDA_ERR_TIMEOUT);
-                }
-            }
-            ok = __shfl_sync(kFull, ok, 0);
-            if (!ok) {
-                aborted = true;
-                break;
-            }
-            if (++slot == kPfStages) {
-                slot = 0;
-                phase ^= 1u;
-            }
-        }
+// The unit pieces of a CTA's page-head range [start, end), in order; every
+// role walks the same sequence.
+struct PieceWalk {
+    int b, j, i0, n;   // sequence b, kv head j, pages i0 .. i0 + n - 1 of b
+    int k;             // pages of the range before this piece
+    int count;
+    __device__ __forceinline__ void begin(const int* seg, int B, int start, int end) {
+        count = end - start;
+        k = 0;
+        b = find_seq(seg, B, start >> 3);
+        const int np = seg[b + 1] - seg[b];
+        const int r = start - 8 * seg[b];
+        j = r / np;
+        i0 = r % np;
+        n = min(np - i0, count);
     }
-    if (lane == 0 && *s.abort_flag != 0) {
-        // copies still landing in this CTA's shared memory: wait (bounded) for each
-        for (int k = 0; k < kPfStages; ++k)
-            if (armed & (1u << k)) (void)mbar_wait(&s.full_bar[k], (armed_parity >> k) & 1u, p.timeout_ns, nullptr);
+    __device__ __forceinline__ bool next(const int* seg, int B) {
+        k += n;
+        if (k >= count) return false;
+        if (++j == kNumKvHeads) {
+            j = 0;
+            do { ++b; } while (b < B && seg[b + 1] == seg[b]);
+        }
+        i0 = 0;
+        n = min(seg[b + 1] - seg[b], count - k);
+        return true;
     }
-}
-
-struct PfState {
-    uint32_t qa[8][4];    // A fragments of q per 16-dim step: rows g (regs 0, 2) and g + 8 (regs 1, 3), bf16
-    float o[16][4];       // value accumulators: 16 tiles of 8 dims, rows g (0, 1) and g + 8 (2, 3)
-    float m[2];           // running max of rows g and g + 8 (log2 units)
-    float lsum[2];        // partial softmax sums of this lane's tokens, rows g and g + 8
 };
 
-// q of this warp's rows 16w + g and 16w + g + 8 of unit (b, j): RMSNorm and
-// RoPE in float (each row's angles from its token's position, the argument
-// reduced modulo 2*pi in double), scaled by log2(e)/sqrt(128) and rounded to
-// bf16, at dims 8m + 2t, 8m + 2t + 1.
-template <int G>
-__device__ __forceinline__ void pf_begin(const Params& p, const PfShared& s, int b, int j, int w, int lane, int L,
-                                         PfState& st) {
-    constexpr int kHq = G * kNumKvHeads;
-    constexpr int kQkvW = (kHq + 2 * kNumKvHeads) * kHeadDim;
-    const int g = lane >> 2, t = lane & 3;
-    const int n = p.new_tokens, R = n * G;
-    const int pos0 = pf_first_position(p, b, L, n);
-    const uint32_t* gq = reinterpret_cast<const uint32_t*>(s.gains);
-    const float scale = (float)kQScale;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int r = 16 * w + g + 8 * h;
-        const bool active = r < R;
-        const int tt = active ? r / G : 0;
-        const int head = G * j + (active ? r % G : 0);
-        const uint32_t* xq =
-            reinterpret_cast<const uint32_t*>(p.qkv + pf_token_row(p, b, tt) * kQkvW + head * kHeadDim);
-        uint32_t xw[16];
-        float ss = 0.f;
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            xw[m] = xq[4 * m + t];
-            ss = fmaf(bf_lo(xw[m]), bf_lo(xw[m]), fmaf(bf_hi(xw[m]), bf_hi(xw[m]), ss));
-        }
-        ss += __shfl_xor_sync(kFull, ss, 1);
-        ss += __shfl_xor_sync(kFull, ss, 2);
-        const float inv_r = rsqrtf(ss * (1.f / 128.f) + (float)p.rms_eps);
-        const double pos = (double)(pos0 + tt);
-#pragma unroll
-        for (int mp = 0; mp < 8; ++mp) {
-            float qa[2], qb[2];
-            const uint32_t wlo = gq[4 * mp + t], whi = gq[32 + 4 * mp + t];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                float sn, cs;
-                sincosf((float)reduce_angle(pos * s.inv_freq[8 * mp + 2 * t + e]), &sn, &cs);
-                const float ya = (e ? bf_hi(xw[mp]) : bf_lo(xw[mp])) * inv_r * (e ? bf_hi(wlo) : bf_lo(wlo));
-                const float yb = (e ? bf_hi(xw[mp + 8]) : bf_lo(xw[mp + 8])) * inv_r * (e ? bf_hi(whi) : bf_lo(whi));
-                qa[e] = fmaf(ya, cs, -yb * sn) * scale;   // dim 8*mp + 2t + e
-                qb[e] = fmaf(yb, cs, ya * sn) * scale;    // dim 64 + 8*mp + 2t + e
-            }
-            const int part = ((mp & 1) ? 2 : 0) + h;   // dims 16s + 2t (+1) or 16s + 8 + 2t (+1); row g or g + 8
-            st.qa[mp >> 1][part] = active ? pack_bf2(qa[0], qa[1]) : 0u;
-            st.qa[4 + (mp >> 1)][part] = active ? pack_bf2(qb[0], qb[1]) : 0u;
-        }
-    }
-#pragma unroll
-    for (int nn = 0; nn < 16; ++nn)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) st.o[nn][k] = 0.f;
-    st.m[0] = st.m[1] = -INFINITY;
-    st.lsum[0] = st.lsum[1] = 0.f;
+// One thread's bounded wait; a failure aborts the CTA.
+__device__ __forceinline__ bool tc_wait1(const Params& p, const TcShared& s, uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_wait(bar, parity, p.timeout_ns, s.abort_flag)) return true;
+    *s.abort_flag = 1;
+    record_error(p.status, QDA_ERR_TIMEOUT);
+    return false;
 }
 
-// Scores, online softmax and value accumulation over one staged page for rows
-// g and g + 8, which see page tokens up to lim0 and lim1 (unless kFullPage).
-// In a swizzled box, row r's 16-byte piece c sits at r * 128 + ((c ^ (r % 8)) * 16).
-template <bool kFullPage>
-__device__ __forceinline__ void pf_attend(const uint8_t* stage, int lim0, int lim1, bool act0, bool act1, int lane,
-                                          PfState& st) {
-    const int t = lane & 3;
-    const int x7 = lane & 7;   // = row % 8 for every row this lane addresses
-    // K rows as the column-major B operand: matrix lane/8 = (tokens 0-7 | 8-15) x (dims +0 | +8)
-    const uint32_t krow = smem_addr(stage + kPfStageK) + (x7 + ((lane >> 4) << 3)) * 128;
-    const int kc = (lane >> 3) & 1;
-    float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(krow + (k >> 2) * kPfBoxBytes + ((((2 * (k & 3)) + kc) ^ x7) << 4), b0, b1, b2, b3);
-        mma_bf16_16816(c0, st.qa[k], b0, b1);
-        mma_bf16_16816(c1, st.qa[k], b2, b3);
-    }
-    // rows g and g + 8 at page tokens 2t, 2t+1, 8+2t, 9+2t
-    float s0[4] = {c0[0], c0[1], c1[0], c1[1]};
-    float s1[4] = {c0[2], c0[3], c1[2], c1[3]};
-    if (!kFullPage) {
-        const int tok[4] = {2 * t, 2 * t + 1, 8 + 2 * t, 9 + 2 * t};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            s0[i] = tok[i] <= lim0 ? s0[i] : -INFINITY;
-            s1[i] = tok[i] <= lim1 ? s1[i] : -INFINITY;
-        }
-    }
-    float mx0 = fmaxf(fmaxf(s0[0], s0[1]), fmaxf(s0[2], s0[3]));
-    float mx1 = fmaxf(fmaxf(s1[0], s1[1]), fmaxf(s1[2], s1[3]));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 2));
-    const bool grow0 = mx0 > st.m[0] + kRescaleThreshold;
-    const bool grow1 = mx1 > st.m[1] + kRescaleThreshold;
-    if (__any_sync(kFull, grow0 || grow1)) {
-        const float n0 = grow0 ? mx0 : st.m[0], n1 = grow1 ? mx1 : st.m[1];
-        const float a0 = grow0 ? exp2_approx(st.m[0] - n0) : 1.f;   // exp2(-inf) = 0 on the first page
-        const float a1 = grow1 ? exp2_approx(st.m[1] - n1) : 1.f;
-#pragma unroll
-        for (int nn = 0; nn < 16; ++nn) {
-            st.o[nn][0] *= a0;
-            st.o[nn][1] *= a0;
-            st.o[nn][2] *= a1;
-            st.o[nn][3] *= a1;
-        }
-        st.lsum[0] *= a0;
-        st.lsum[1] *= a1;
-        st.m[0] = n0;
-        st.m[1] = n1;
-    }
-    float p0[4], p1[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        p0[i] = (s0[i] == -INFINITY || !act0) ? 0.f : exp2_approx(s0[i] - st.m[0]);
-        p1[i] = (s1[i] == -INFINITY || !act1) ? 0.f : exp2_approx(s1[i] - st.m[1]);
-    }
-    uint32_t pa[4];
-    pa[0] = pack_bf2(p0[0], p0[1]);   // row g, tokens 2t, 2t+1
-    pa[1] = pack_bf2(p1[0], p1[1]);   // row g + 8
-    pa[2] = pack_bf2(p0[2], p0[3]);   // row g, tokens 8+2t, 9+2t
-    pa[3] = pack_bf2(p1[2], p1[3]);   // row g + 8
-    st.lsum[0] += (bf_lo(pa[0]) + bf_hi(pa[0])) + (bf_lo(pa[2]) + bf_hi(pa[2]));
-    st.lsum[1] += (bf_lo(pa[1]) + bf_hi(pa[1])) + (bf_lo(pa[3]) + bf_hi(pa[3]));
-    // V rows as the column-major B operand (transposed load): matrix lane/8 =
-    // (tokens 0-7 | 8-15) x (dims +0 | +8)
-    const uint32_t vrow = smem_addr(stage + kPfStageV) + (x7 + (((lane >> 3) & 1) << 3)) * 128;
-    const int vc = (lane >> 4) & 1;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_trans(vrow + (u >> 2) * kPfBoxBytes + ((((2 * (u & 3)) + vc) ^ x7) << 4), b0, b1, b2, b3);
-        mma_bf16_16816(st.o[2 * u], pa, b0, b1);
-        mma_bf16_16816(st.o[2 * u + 1], pa, b2, b3);
-    }
-}
-
-__device__ __forceinline__ bool pf_wait_full(const Params& p, const PfShared& s, int slot, uint32_t phase,
+// A whole warp's bounded wait, with one verdict for all its lanes.
+__device__ __forceinline__ bool tc_wait_warp(const Params& p, const TcShared& s, uint64_t* bar, uint32_t parity,
                                              int lane) {
-    uint64_t* bar = &s.full_bar[slot];
-    bool ok = mbar_try_wait(bar, phase);
+    bool ok = mbar_try_wait(bar, parity);
     if (__all_sync(kFull, ok)) return true;
-    ok = ok || mbar_wait(bar, phase, p.timeout_ns, s.abort_flag);
-    ok = __all_sync(kFull, ok || mbar_try_wait(bar, phase));
+    ok = ok || mbar_wait(bar, parity, p.timeout_ns, s.abort_flag);
+    ok = __all_sync(kFull, ok || mbar_try_wait(bar, parity));
     if (!ok && lane == 0) {
         *s.abort_flag = 1;
         record_error(p.status, QDA_ERR_TIMEOUT);
@@ -413,153 +293,383 @@ __device__ __forceinline__ bool pf_wait_full(const Params& p, const PfShared& s,
     return ok;
 }
 
-// End of a unit piece: o for the warp's active rows when the unit is held
-// whole by this CTA, else the partials in scratch slot `slot`.
-template <int G>
-__device__ __forceinline__ void pf_finish(const Params& p, const PrefillScratch& sc, int b, int j, int w, int lane,
-                                          bool whole, int slot, PfState& st) {
-    constexpr int kHq = G * kNumKvHeads;
-    const int g = lane >> 2, t = lane & 3;
-    const int R = p.new_tokens * G;
-    float l[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        l[h] = st.lsum[h];
-        l[h] += __shfl_xor_sync(kFull, l[h], 1);
-        l[h] += __shfl_xor_sync(kFull, l[h], 2);
-    }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int r = 16 * w + g + 8 * h;
-        if (r >= R) continue;
-        if (whole) {
-            const int tt = r / G, head = G * j + r % G;
-            const float inv = l[h] > 0.f ? 1.f / l[h] : 0.f;
-            uint32_t* dst = reinterpret_cast<uint32_t*>(p.o + (pf_token_row(p, b, tt) * kHq + head) * kHeadDim);
-#pragma unroll
-            for (int nn = 0; nn < 16; ++nn) dst[4 * nn + t] = pack_bf2(st.o[nn][2 * h] * inv, st.o[nn][2 * h + 1] * inv);
-        } else {
-            const size_t prow = (size_t)slot * kPrefillRows + r;
-            float2* pa = reinterpret_cast<float2*>(sc.acc + prow * kHeadDim);
-#pragma unroll
-            for (int nn = 0; nn < 16; ++nn) __stcg(pa + 4 * nn + t, make_float2(st.o[nn][2 * h], st.o[nn][2 * h + 1]));
-            if (t == 0) __stcg(sc.ml + prow, make_float2(st.m[h], l[h]));
-        }
-    }
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-template <int G>
-__device__ __forceinline__ void pf_consumer(const Params& p, const PrefillScratch& sc, const PfShared& s, int B,
-                                            int start, int end, int per_cta, int w, int lane) {
-    const int n = p.new_tokens, R = n * G;
-    const bool active_warp = 16 * w < R;
-    const int g = lane >> 2;
-    const int r0 = 16 * w + g, r1 = r0 + 8;
-    const bool act0 = r0 < R, act1 = r1 < R;
-    const int tt0 = act0 ? r0 / G : 0, tt1 = act1 ? r1 / G : 0;
-    PfState st;
-    int b, j, i0;
-    pf_locate(s, B, start, b, j, i0);
-    int slot = 0;
-    uint32_t phase = 0;
-    const int count = end - start;
-    int k = 0;
-    bool aborted = false;
-    while (k < count && !aborted) {
-        const int np = s.seg[b + 1] - s.seg[b];
-        const int L = s.lens[b];
-        const int n_here = min(np - i0, count - k);
-        if (active_warp) pf_begin<G>(p, s, b, j, w, lane, L, st);
-        for (int u = 0; u < n_here; ++u) {
-            if (!pf_wait_full(p, s, slot, phase, lane)) {
-                aborted = true;
+__device__ __forceinline__ void fence_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Warp 0: the page ids (32 page-heads looked up at a time), then per stage
+// four tiled copies per page: K and V of kv head j, dims 0-63 and 64-127,
+// into the stage's halves at 2 KiB per page. Pages whose block-table entry is
+// out of range are not copied; the stage's mask tells the softmax.
+__device__ __forceinline__ void tc_producer(const Params& p, const PrefillScratch& sc, const TcShared& s,
+                                            const CUtensorMap* tm_k, const CUtensorMap* tm_v, int B, int start,
+                                            int end, int lane) {
+    const uint32_t q_bytes = (uint32_t)(p.new_tokens * (p.num_q_heads / kNumKvHeads)) * 128u;   // R rows per half
+    int wbase = 0x40000000, id = -1;
+    uint32_t g = 0, u = 0, armed = 0, armed_parity = 0, q_armed = 0;
+    bool ok = true;
+    asm volatile("fence.proxy.async.global;" ::: "memory");   // the copies read what the prep launch wrote
+    PieceWalk w;
+    w.begin(s.seg, B, start, end);
+    do {
+        // the piece's query tile, into buffer u % 2 once the piece two back has
+        // finished reading it
+        {
+            int good = 1;
+            if (lane == 0) {
+                if (u >= 2) good = tc_wait1(p, s, &s.q_free[u & 1u], ((u >> 1) - 1) & 1u) ? 1 : 0;
+                if (good) {
+                    const uint8_t* src = reinterpret_cast<const uint8_t*>(sc.q) +
+                                         (size_t)(w.b * kNumKvHeads + w.j) * kPrefillQTileBytes;
+                    uint8_t* dst = s.q + (u & 1u) * 2 * kTcTile;
+                    mbar_arrive_expect_tx(&s.q_full[u & 1u], 2 * q_bytes);
+                    bulk_g2s(dst, src, q_bytes, &s.q_full[u & 1u]);
+                    bulk_g2s(dst + kTcTile, src + kTcTile, q_bytes, &s.q_full[u & 1u]);
+                    q_armed = (q_armed & ~(3u << (2 * (u & 1u)))) | ((2u | ((u >> 1) & 1u)) << (2 * (u & 1u)));
+                }
+            }
+            if (!__shfl_sync(kFull, good, 0)) break;
+            ++u;
+        }
+        const int np_b = s.seg[w.b + 1] - s.seg[w.b];
+        const int x_piece = 8 * s.seg[w.b] + w.j * np_b + w.i0;
+        for (int q = 0; q < w.n; q += kTcPages, ++g) {
+            const int npg = min(kTcPages, w.n - q);
+            const int x0 = x_piece + q;
+            if (x0 < wbase || x0 + npg > wbase + 32) {
+                wbase = x0;
+                const int x = x0 + lane;
+                id = -1;
+                if (x < end) {
+                    const int bb = find_seq(s.seg, B, x >> 3);
+                    const int np = s.seg[bb + 1] - s.seg[bb];
+                    const int r = x - 8 * s.seg[bb];
+                    id = __ldg(p.block_table + (size_t)bb * p.bt_stride + r % np);
+                }
+            }
+            const int st = (int)(g % kTcStages);
+            int good = 1;
+            if (lane == 0 && g >= (uint32_t)kTcStages)
+                good = tc_wait1(p, s, &s.kv_empty[st], ((g / kTcStages) - 1) & 1u) ? 1 : 0;
+            if (!__shfl_sync(kFull, good, 0)) {
+                ok = false;
                 break;
             }
-            uint8_t* stage = s.stages + slot * kPfStageBytes;
-            const int i = i0 + u;
-            if (active_warp && s.meta[slot].bad == 0) {
-                const int rows = min(kPage, L - kPage * i);
-                if (rows < kPage) {
-                    // rows after the sequence hold stale bytes; a stale NaN times a
-                    // zero probability would still give NaN in the value product
-                    for (int rr = rows; rr < kPage; ++rr) {   // row rr of both halves (the swizzle stays in the row)
-                        reinterpret_cast<uint32_t*>(stage + kPfStageV + rr * 128)[lane] = 0u;
-                        reinterpret_cast<uint32_t*>(stage + kPfStageV + kPfBoxBytes + rr * 128)[lane] = 0u;
-                    }
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    __syncwarp();
+            const int my = __shfl_sync(kFull, id, (x0 - wbase + lane) & 31);
+            const uint32_t bad = __ballot_sync(kFull, lane < npg && (my < 0 || my >= p.num_pages));
+            if (lane == 0) {
+                s.mask[st] = (int)bad;
+                if (bad != 0) record_error(p.status, QDA_ERR_BOUNDS);
+                const int copied = npg - __popc(bad);
+                if (copied > 0) {
+                    mbar_arrive_expect_tx(&s.kv_full[st], (uint32_t)(copied * 4 * kTcBoxBytes));
+                    armed |= 1u << st;
+                    armed_parity = (armed_parity & ~(1u << st)) | (((g / kTcStages) & 1u) << st);
+                } else {
+                    mbar_arrive(&s.kv_full[st]);
                 }
-                // row r (token tt) sees slots <= L - n + tt
-                const int lim0 = (L - n + tt0) - kPage * i, lim1 = (L - n + tt1) - kPage * i;
-                if (kPage * i + kPage - 1 <= L - n) pf_attend<true>(stage, lim0, lim1, act0, act1, lane, st);
-                else pf_attend<false>(stage, lim0, lim1, act0, act1, lane, st);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.empty_bar[slot]);
-            if (++slot == kPfStages) {
-                slot = 0;
-                phase ^= 1u;
+            const uint32_t dst = smem_addr(s.stages + st * kTcStageBytes);
+            for (int k = 0; k < npg; ++k) {
+                const int page = __shfl_sync(kFull, my, k);
+                if (lane == 0 && ((bad >> k) & 1u) == 0) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        tma_load_3d(dst + kTcStageK + h * kTcHalf + k * kTcBoxBytes, tm_k, 64 * h, w.j, page * kPage,
+                                    &s.kv_full[st]);
+                        tma_load_3d(dst + kTcStageV + h * kTcHalf + k * kTcBoxBytes, tm_v, 64 * h, w.j, page * kPage,
+                                    &s.kv_full[st]);
+                    }
+                }
             }
         }
-        if (aborted) break;
-        // the unit's page-head range; a unit held whole by one CTA writes o
-        const int ustart = 8 * s.seg[b] + j * np;
-        const bool whole = ustart / per_cta == (ustart + np - 1) / per_cta;
-        const int pslot = 2 * (int)blockIdx.x + (k == 0 ? 0 : 1);   // the CTA's first piece, else its last
-        if (active_warp) pf_finish<G>(p, sc, b, j, w, lane, whole, pslot, st);
-        k += n_here;
-        if (k < count) {
-            if (++j == kNumKvHeads) {
-                j = 0;
-                do { ++b; } while (b < B && s.seg[b + 1] == s.seg[b]);
-            }
-            i0 = 0;
-        }
+    } while (ok && w.next(s.seg, B));
+    if (lane == 0 && *s.abort_flag != 0) {
+        // copies still landing in this CTA's shared memory: wait (bounded) for each
+        for (int k = 0; k < kTcStages; ++k)
+            if (armed & (1u << k)) (void)mbar_wait(&s.kv_full[k], (armed_parity >> k) & 1u, p.timeout_ns, nullptr);
+        for (int k = 0; k < 2; ++k)
+            if ((q_armed >> (2 * k)) & 2u)
+                (void)mbar_wait(&s.q_full[k], (q_armed >> (2 * k)) & 1u, p.timeout_ns, nullptr);
     }
 }
 
+// One thread of warp 1: per stage g, S_g = Q K_g^T into S buffer g % 2, then
+// O += P_{g-1} V_{g-1} once the softmax has written P_{g-1}. S_g overwrites
+// the buffer the softmax of stage g - 2 read, which it had finished before
+// writing P_{g-2}.
+__device__ __forceinline__ void tc_issuer(const Params& p, const TcShared& s, int B, int start, int end,
+                                          uint32_t tmem) {
+    const uint32_t idesc_s = umma_idesc_bf16_m128(kTcKeys);
+    const uint32_t idesc_o = umma_idesc_bf16_m128_bmn(kHeadDim);
+    const uint32_t p_base = smem_addr(s.p), st_base = smem_addr(s.stages);
+    auto pv = [&](uint32_t x, bool first) -> bool {
+        if (!tc_wait1(p, s, s.p_full, x & 1u)) return false;
+        tc_fence_after();
+        const uint32_t v = st_base + (x % kTcStages) * kTcStageBytes + kTcStageV;
+#pragma unroll
+        for (int kk = 0; kk < kTcKeys / 16; ++kk)
+            umma_bf16(tmem + kTcTmemO, umma_desc_sw128(p_base + 32 * kk),
+                      umma_desc_sw128_mn(v + 2 * 1024 * kk, kTcHalf, 1024), idesc_o, (first && kk == 0) ? 0u : 1u);
+        umma_commit(s.pv_done);
+        umma_commit(&s.kv_empty[x % kTcStages]);   // K and V of the stage have been read
+        return true;
+    };
+    uint32_t g = 0, u = 0;
+    bool prev_first = false, ok = true;
+    PieceWalk w;
+    w.begin(s.seg, B, start, end);
+    do {
+        if (!tc_wait1(p, s, &s.q_full[u & 1u], (u >> 1) & 1u)) {
+            ok = false;
+            break;
+        }
+        tc_fence_after();
+        const uint32_t q_base = smem_addr(s.q) + (u & 1u) * 2 * kTcTile;
+        for (int q = 0; q < w.n; q += kTcPages, ++g) {
+            const int st = (int)(g % kTcStages);
+            if (!tc_wait1(p, s, &s.kv_full[st], (g / kTcStages) & 1u)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t kb = st_base + st * kTcStageBytes + kTcStageK;
+            const uint32_t sd = tmem + (g & 1u) * kTcKeys;
+#pragma unroll
+            for (int kk = 0; kk < kHeadDim / 16; ++kk)
+                umma_bf16(sd, umma_desc_sw128(q_base + (kk >> 2) * kTcTile + (kk & 3) * 32),
+                          umma_desc_sw128(kb + (kk >> 2) * kTcHalf + (kk & 3) * 32), idesc_s, kk != 0 ? 1u : 0u);
+            umma_commit(&s.s_full[g & 1u]);
+            if (q + kTcPages >= w.n) umma_commit(&s.q_free[u & 1u]);   // the piece's last product reading Q
+            if (g > 0 && !pv(g - 1, prev_first)) {
+                ok = false;
+                break;
+            }
+            prev_first = q == 0;
+        }
+        ++u;
+    } while (ok && w.next(s.seg, B));
+    if (ok && g > 0) (void)pv(g - 1, prev_first);
+    umma_commit(s.fin);   // every instruction issued above has completed
+}
+
+// Warps 4-7, thread = row r = 32 * (warp - 4) + lane.
 template <int G>
-__global__ void __launch_bounds__(kPfThreads, 1)
+__device__ __forceinline__ void tc_softmax(const Params& p, const PrefillScratch& sc, const TcShared& s, int B,
+                                           int start, int end, int per_cta, int r, uint32_t tmem) {
+    constexpr int kHq = G * kNumKvHeads;
+    const int lane = r & 31;
+    const int n = p.new_tokens, R = n * G;
+    const bool active = r < R;
+    const bool warp_active = (r & ~31) < R;
+    const int tt = active ? r / G : 0;
+    const uint32_t lanes = tmem + ((uint32_t)(r & ~31) << 16);
+    const uint32_t p_row = smem_addr(s.p) + r * 128;
+    uint32_t g = 0, pv_seen = 0;
+    bool ok = true;
+    auto pv_wait = [&](uint32_t x) -> bool {   // O += P_x V_x has completed
+        if (pv_seen > x) return true;
+        if (!tc_wait_warp(p, s, s.pv_done, x & 1u, lane)) return false;
+        pv_seen = x + 1;
+        return true;
+    };
+    PieceWalk w;
+    w.begin(s.seg, B, start, end);
+    do {
+        const int np_b = s.seg[w.b + 1] - s.seg[w.b];
+        const int L = s.lens[w.b];
+        const int lim = active ? L - n + tt : -1;   // the last cache slot this row sees
+        float m = -INFINITY, lsum = 0.f;
+        for (int q = 0; q < w.n; q += kTcPages, ++g) {
+            const int npg = min(kTcPages, w.n - q);
+            const int slot0 = kPage * (w.i0 + q);
+            const int st = (int)(g % kTcStages);
+            if (!tc_wait_warp(p, s, &s.kv_full[st], (g / kTcStages) & 1u, lane)) {
+                ok = false;
+                break;
+            }
+            const uint32_t bad = (uint32_t)s.mask[st];
+            {
+                // cache rows of the stage that hold nothing valid (after the
+                // sequence, past the piece, not copied) may hold any bytes: a
+                // NaN there times a zero probability would still give NaN, so
+                // their V rows are zeroed (thread r: row r % 64, half r / 64)
+                const int kr = r & 63, pg = kr >> 4;
+                if (pg >= npg || ((bad >> pg) & 1u) != 0 || slot0 + kr >= L) {
+                    const uint32_t row = smem_addr(s.stages + st * kTcStageBytes + kTcStageV + (r >> 6) * kTcHalf) +
+                                         kr * 128;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) st_shared_v4(row + 16 * c, 0u, 0u, 0u, 0u);
+                }
+            }
+            uint32_t pw[kTcKeys / 2];
+            if (warp_active) {
+                if (!tc_wait_warp(p, s, &s.s_full[g & 1u], (g >> 1) & 1u, lane)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t raw[4][16];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld16(lanes + (g & 1u) * kTcKeys + 16 * c, raw[c]);
+                tmem_ld_wait();
+                float sv[kTcKeys];
+                // keys c <= climit are inside this row's causal window and the piece's pages
+                const int climit = min(lim - slot0, kPage * npg - 1);
+                float mx = -INFINITY;
+                if (bad == 0 && climit >= kTcKeys - 1) {
+#pragma unroll
+                    for (int c = 0; c < kTcKeys; ++c) {
+                        sv[c] = __uint_as_float(raw[c >> 4][c & 15]);
+                        mx = fmaxf(mx, sv[c]);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < kTcKeys; ++c) {
+                        const bool keep = c <= climit && ((bad >> (c >> 4)) & 1u) == 0;
+                        sv[c] = keep ? __uint_as_float(raw[c >> 4][c & 15]) : -INFINITY;
+                        mx = fmaxf(mx, sv[c]);
+                    }
+                }
+                const bool grow = mx > m + kRescaleThreshold;
+                const bool rescale = grow && m != -INFINITY;   // O holds earlier stages of this piece
+                if (__any_sync(kFull, rescale)) {
+                    if (!pv_wait(g - 1)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const float a = rescale ? exp2_approx(m - mx) : 1.f;
+#pragma unroll 1
+                    for (int c = 0; c < kHeadDim / 16; ++c) {
+                        uint32_t v[16];
+                        tmem_ld16(lanes + kTcTmemO + 16 * c, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * a);
+                        tmem_st16(lanes + kTcTmemO + 16 * c, v);
+                    }
+                    tmem_st_wait();
+                    lsum *= a;
+                }
+                if (grow) m = mx;
+                const float mb = m == -INFINITY ? 0.f : m;
+#pragma unroll
+                for (int c = 0; c < kTcKeys / 2; ++c) {
+                    pw[c] = pack_bf2(exp2_approx(sv[2 * c] - mb), exp2_approx(sv[2 * c + 1] - mb));
+                    lsum += bf_lo(pw[c]) + bf_hi(pw[c]);
+                }
+            }
+            // The previous stage's product has read the P tile. Every warp
+            // waits for it before arriving: p_full counts arrivals, and a warp
+            // must not arrive for stage g + 1 before stage g's phase is over.
+            if (g > 0 && !pv_wait(g - 1)) {
+                ok = false;
+                break;
+            }
+            if (warp_active) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    st_shared_v4(p_row + ((c ^ (r & 7)) << 4), pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+            }
+            fence_async_shared();
+            tc_fence_before();
+            mbar_arrive(s.p_full);
+        }
+        if (!ok) break;
+        if (warp_active) {
+            // the piece's last product, then o (whole unit) or the partials
+            if (!pv_wait(g - 1)) break;
+            tc_fence_after();
+            const int ustart = 8 * s.seg[w.b] + w.j * np_b;
+            const bool whole = ustart / per_cta == (ustart + np_b - 1) / per_cta;
+            const int pslot = 2 * (int)blockIdx.x + (w.k == 0 ? 0 : 1);   // the CTA's first piece, else its last
+            const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+            uint4* orow = reinterpret_cast<uint4*>(p.o + (pf_token_row(p, w.b, tt) * kHq + G * w.j + r % G) * kHeadDim);
+            const size_t prow = (size_t)pslot * kPrefillRows + r;
+            float4* arow = reinterpret_cast<float4*>(sc.acc + prow * kHeadDim);
+#pragma unroll 1
+            for (int c = 0; c < kHeadDim / 16; ++c) {
+                uint32_t v[16];
+                tmem_ld16(lanes + kTcTmemO + 16 * c, v);
+                tmem_ld_wait();
+                if (!active) {
+                } else if (whole) {
+                    uint32_t o8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        o8[e] = pack_bf2(__uint_as_float(v[2 * e]) * inv, __uint_as_float(v[2 * e + 1]) * inv);
+                    orow[2 * c] = make_uint4(o8[0], o8[1], o8[2], o8[3]);
+                    orow[2 * c + 1] = make_uint4(o8[4], o8[5], o8[6], o8[7]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        __stcg(arow + 4 * c + e, make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                                             __uint_as_float(v[4 * e + 2]),
+                                                             __uint_as_float(v[4 * e + 3])));
+                }
+                __syncwarp();
+            }
+            if (active && !whole) __stcg(sc.ml + prow, make_float2(m, lsum));
+        }
+    } while (ok && w.next(s.seg, B));
+}
+
+template <int G>
+__global__ void __launch_bounds__(kTcThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const Params p,
                    const PrefillScratch sc) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    // the stages start on a 1024-byte boundary (the swizzle atom)
+    // the tiles start on a 1024-byte boundary (the swizzle atom)
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    PfShared s;
+    TcShared s;
     s.stages = smem;
-    s.seg = reinterpret_cast<int*>(smem + kPfSmemSeg);
-    s.lens = reinterpret_cast<int*>(smem + kPfSmemLens);
-    s.inv_freq = reinterpret_cast<double*>(smem + kPfSmemInvFreq);
-    s.gains = reinterpret_cast<const uint16_t*>(smem + kPfSmemGains);
-    s.meta = reinterpret_cast<volatile StageMeta*>(smem + kPfSmemMeta);
-    s.full_bar = reinterpret_cast<uint64_t*>(smem + kPfSmemBars);
-    s.empty_bar = s.full_bar + kPfStages;
-    s.never_bar = s.empty_bar + kPfStages;
-    s.abort_flag = reinterpret_cast<volatile int*>(smem + kPfSmemFlags);
+    s.q = smem + kTcSmemQ;
+    s.p = smem + kTcSmemP;
+    s.seg = reinterpret_cast<int*>(smem + kTcSmemSeg);
+    s.lens = reinterpret_cast<int*>(smem + kTcSmemLens);
+    s.mask = reinterpret_cast<volatile int*>(smem + kTcSmemMask);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTcSmemBars);
+    s.kv_full = bars;
+    s.kv_empty = bars + kTcStages;
+    s.s_full = bars + 2 * kTcStages;
+    s.p_full = s.s_full + 2;
+    s.pv_done = s.p_full + 1;
+    s.q_full = s.pv_done + 1;
+    s.q_free = s.q_full + 2;
+    s.fin = s.q_free + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTcSmemTmem);
+    s.abort_flag = reinterpret_cast<volatile int*>(smem + kTcSmemTmem + 4);
 
     // The prologue touches no global memory; griddepcontrol.wait then holds
-    // until the append launch has completed and its cache writes are visible.
-    if (threadIdx.x >= 64 && threadIdx.x < 128) {
-        const int i = threadIdx.x - 64;
-        s.inv_freq[i] = pow(p.rope_theta, -2.0 * i / 128.0);
-    }
+    // until the prep launch has completed and its writes are visible.
     if (threadIdx.x == 0) {
-        for (int k = 0; k < kPfStages; ++k) {
-            mbar_init(&s.full_bar[k], 1);
-            mbar_init(&s.empty_bar[k], kPfWarps);
+        for (int k = 0; k < kTcStages; ++k) {
+            mbar_init(&s.kv_full[k], 1);
+            mbar_init(&s.kv_empty[k], 1);
         }
-        mbar_init(s.never_bar, 1);
+        mbar_init(&s.s_full[0], 1);
+        mbar_init(&s.s_full[1], 1);
+        mbar_init(s.p_full, 4 * 32);
+        mbar_init(s.pv_done, 1);
+        for (int k = 0; k < 2; ++k) {
+            mbar_init(&s.q_full[k], 1);
+            mbar_init(&s.q_free[k], 1);
+        }
+        mbar_init(s.fin, 1);
         *s.abort_flag = 0;
         s.seg[0] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
     }
+    if (warp == 1) tmem_alloc(tmem_slot, kTcTmemCols);
     pdl_wait();
-
     const int B = p.batch;
-    for (int b = threadIdx.x; b < B; b += kPfThreads) {
+    for (int b = threadIdx.x; b < B; b += kTcThreads) {
         const int L_all = p.seq_lens[b];
         const bool ok = length_ok(p, L_all);
         if (!ok && blockIdx.x == 0) record_error(p.status, QDA_ERR_BOUNDS);
@@ -567,11 +677,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         s.lens[b] = L;
         s.seg[b + 1] = ok ? (L + kPage - 1) / kPage : 0;
     }
-    if (threadIdx.x < kHeadDim / 2) {   // the q gains, one 4-byte word per thread
-        reinterpret_cast<uint32_t*>(smem + kPfSmemGains)[threadIdx.x] =
-            reinterpret_cast<const uint32_t*>(p.q_norm_w)[threadIdx.x];
-    }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
     if (warp == 0) {  // inclusive scan of the page counts: seg[b] becomes the first page of b
         int v[8];
         int run = 0;
@@ -596,30 +705,49 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     __syncthreads();
     if (blockIdx.x == 0)   // page offsets for the combine launch
-        for (int b = threadIdx.x; b <= B; b += kPfThreads) p.seg[b] = s.seg[b];
+        for (int b = threadIdx.x; b <= B; b += kTcThreads) p.seg[b] = s.seg[b];
 
     const int total = kNumKvHeads * s.seg[B];   // page-heads
     const int per_cta = (total + (int)gridDim.x - 1) / (int)gridDim.x;
     const int start = (int)blockIdx.x * per_cta;
     const int end = min(start + per_cta, total);
     if (start < end) {
-        if (warp == kPfWarps) pf_producer(p, s, &tm_k, &tm_v, B, start, end, lane);
-        else pf_consumer<G>(p, sc, s, B, start, end, per_cta, warp, lane);
+        if (warp == 0) {
+            tc_producer(p, sc, s, &tm_k, &tm_v, B, start, end, lane);
+        } else if (warp == 1) {
+            if (lane == 0) {
+                tc_issuer(p, s, B, start, end, tmem);
+                // nothing may still write tensor memory when it is freed
+                (void)mbar_wait(s.fin, 0u, p.timeout_ns, nullptr);
+            }
+        } else if (warp >= 4) {
+            tc_softmax<G>(p, sc, s, B, start, end, per_cta, threadIdx.x - 128, tmem);
+        }
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTcTmemCols);
     }
     pdl_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------
-// 3. The combine: CTA (b, j), warp w merges rows w, w + 8, ... of the unit;
-// lane l dims 4l..4l+3. The unit's pieces sit in consecutive CTAs g0..gk of
-// the attention launch: slot 2*g0 + 1 when the unit starts inside g0's range
-// (it is g0's last piece), else 2*g0; slot 2*g in the later CTAs.
+// 3. The combine: warp w of CTA (b, j, z) merges row 8z + w of unit (b, j)
+// when the unit was split across CTAs; lane l holds dims 4l..4l+3. The unit's
+// pieces sit in consecutive CTAs g0..gk of the attention launch: slot 2*g0 + 1
+// when the unit starts inside g0's range (it is g0's last piece), else 2*g0;
+// slot 2*g in the later CTAs.
 template <int G>
 __global__ void __launch_bounds__(256) prefill_combine_kernel(const Params p, const PrefillScratch sc) {
     constexpr int kHq = G * kNumKvHeads;
     pdl_wait();
     pdl_launch_dependents();
-    const int b = blockIdx.x, j = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.x, j = blockIdx.y, lane = threadIdx.x & 31;
+    const int r = 8 * (int)blockIdx.z + (int)(threadIdx.x >> 5);
+    if (r >= p.new_tokens * G) return;
     const int np = p.seg[b + 1] - p.seg[b];
     if (np == 0) return;   // a sequence the attention launch skipped
     const int total = kNumKvHeads * p.seg[p.batch];
@@ -627,34 +755,35 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(const Params p, co
     const int ustart = kNumKvHeads * p.seg[b] + j * np;
     const int g0 = ustart / per_cta, gk = (ustart + np - 1) / per_cta;
     if (g0 == gk) return;   // held whole by one CTA, which wrote o
-    const int R = p.new_tokens * G;
-    for (int r = warp; r < R; r += 8) {
-        float M = -INFINITY;
-        for (int g = g0; g <= gk; ++g) {
-            const int slot = (g == g0 && ustart % per_cta != 0) ? 2 * g + 1 : 2 * g;
-            M = fmaxf(M, __ldcg(sc.ml + (size_t)slot * kPrefillRows + r).x);
-        }
-        float Ls = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int g = g0; g <= gk; ++g) {
-            const int slot = (g == g0 && ustart % per_cta != 0) ? 2 * g + 1 : 2 * g;
-            const size_t prow = (size_t)slot * kPrefillRows + r;
-            const float2 ml = __ldcg(sc.ml + prow);
-            const float wt = (ml.x == -INFINITY) ? 0.f : exp2_approx(ml.x - M);   // a piece that saw no slot
-            Ls = fmaf(wt, ml.y, Ls);
-            const float4 x = __ldcg(reinterpret_cast<const float4*>(sc.acc + prow * kHeadDim) + lane);
-            acc.x = fmaf(wt, x.x, acc.x);
-            acc.y = fmaf(wt, x.y, acc.y);
-            acc.z = fmaf(wt, x.z, acc.z);
-            acc.w = fmaf(wt, x.w, acc.w);
-        }
-        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-        uint2 out;
-        out.x = pack_bf2(acc.x * inv, acc.y * inv);
-        out.y = pack_bf2(acc.z * inv, acc.w * inv);
-        const int tt = r / G, head = G * j + r % G;
-        reinterpret_cast<uint2*>(p.o + (pf_token_row(p, b, tt) * kHq + head) * kHeadDim)[lane] = out;
+    const int first = ustart % per_cta != 0 ? 2 * g0 + 1 : 2 * g0;   // slot of piece 0; piece k > 0: 2 * (g0 + k)
+    const int pieces = gk - g0 + 1;
+    float M = -INFINITY;
+    for (int k = lane; k < pieces; k += 32) {
+        const int slot = k == 0 ? first : 2 * (g0 + k);
+        M = fmaxf(M, __ldcg(sc.ml + (size_t)slot * kPrefillRows + r).x);
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+    float Ls = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int k = 0; k < pieces; ++k) {
+        const size_t prow = (size_t)(k == 0 ? first : 2 * (g0 + k)) * kPrefillRows + r;
+        const float2 ml = __ldcg(sc.ml + prow);
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(sc.acc + prow * kHeadDim) + lane);
+        const float wt = (ml.x == -INFINITY) ? 0.f : exp2_approx(ml.x - M);   // a piece that saw no slot
+        Ls = fmaf(wt, ml.y, Ls);
+        acc.x = fmaf(wt, x.x, acc.x);
+        acc.y = fmaf(wt, x.y, acc.y);
+        acc.z = fmaf(wt, x.z, acc.z);
+        acc.w = fmaf(wt, x.w, acc.w);
+    }
+    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+    uint2 out;
+    out.x = pack_bf2(acc.x * inv, acc.y * inv);
+    out.y = pack_bf2(acc.z * inv, acc.w * inv);
+    const int tt = r / G, head = G * j + r % G;
+    reinterpret_cast<uint2*>(p.o + (pf_token_row(p, b, tt) * kHq + head) * kHeadDim)[lane] = out;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 pf_encode_fn() {
@@ -699,16 +828,16 @@ cudaError_t launch_prefill_g(const Params& p, const PrefillScratch& sc, cudaStre
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cfg.gridDim = dim3((unsigned)p.batch, (unsigned)kNumKvHeads, (unsigned)((p.new_tokens + 31) / 32));
-    cfg.blockDim = dim3(32, 1, 1);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_append_kernel<G>, p);
+    cfg.gridDim = dim3((unsigned)p.batch, (unsigned)kNumKvHeads, (unsigned)((p.new_tokens + 3) / 4));
+    cfg.blockDim = dim3(128, 1, 1);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_prep_kernel<G>, p, sc);
     if (e != cudaSuccess) return e;
     cfg.gridDim = dim3((unsigned)sc.grid, 1, 1);
-    cfg.blockDim = dim3(kPfThreads, 1, 1);
-    cfg.dynamicSmemBytes = kPfSmemAlloc;
+    cfg.blockDim = dim3(kTcThreads, 1, 1);
+    cfg.dynamicSmemBytes = kTcSmemAlloc;
     e = cudaLaunchKernelEx(&cfg, prefill_kernel<G>, tk, tv, p, sc);
     if (e != cudaSuccess) return e;
-    cfg.gridDim = dim3((unsigned)p.batch, (unsigned)kNumKvHeads, 1);
+    cfg.gridDim = dim3((unsigned)p.batch, (unsigned)kNumKvHeads, (unsigned)((p.new_tokens * G + 7) / 8));
     cfg.blockDim = dim3(256, 1, 1);
     cfg.dynamicSmemBytes = 0;
     return cudaLaunchKernelEx(&cfg, prefill_combine_kernel<G>, p, sc);
@@ -718,13 +847,13 @@ cudaError_t launch_prefill_g(const Params& p, const PrefillScratch& sc, cudaStre
 
 cudaError_t prepare_prefill() {
     if (pf_encode_fn() == nullptr) return cudaErrorNotSupported;
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPfSmemAlloc);
+    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemAlloc);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(prefill_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPfSmemAlloc);
+        e = cudaFuncSetAttribute(prefill_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemAlloc);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(prefill_kernel<5>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPfSmemAlloc);
+        e = cudaFuncSetAttribute(prefill_kernel<5>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemAlloc);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(prefill_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPfSmemAlloc);
+        e = cudaFuncSetAttribute(prefill_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemAlloc);
     return e;
 }
 

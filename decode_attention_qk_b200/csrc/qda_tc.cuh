@@ -32,6 +32,23 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16_m128(int n) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 static_assert(umma_idesc_bf16_m128(64) == 0x08100490u, "instruction descriptor bits");
+
+// The same with B MN-major (bit 16): B stored with its N index contiguous,
+// as rows of K.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_m128_bmn(int n) {
+    return umma_idesc_bf16_m128(n) | (1u << 16);
+}
+
+// Shared-memory matrix descriptor of an MN-major bf16 operand in the 128-byte
+// swizzled layout: each K index is a 128-byte row of 64 consecutive MN
+// elements, 8 such rows form a 1024-byte swizzle atom; the atoms of the next 8
+// K indices are `sbo` bytes on, those of the next 64 MN elements `lbo` bytes
+// on. Same fields as umma_desc_sw128; one K step of 16 rows is 2 atoms, so it
+// advances the start by 2 * sbo.
+__host__ __device__ constexpr uint64_t umma_desc_sw128_mn(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
 static_assert(umma_desc_sw128(0x400u) == (0x40ull | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61)),
               "matrix descriptor bits");
 
@@ -81,6 +98,19 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
 }
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Warp-wide: store 16 consecutive columns of this warp's 32 lanes (the
+// inverse of tmem_ld16); tmem_st_wait() orders them before later accesses.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // One tiled copy of a 2-D box from global memory (described by `map`, a
 // kernel parameter) into this CTA's shared memory at `dst`, completing its

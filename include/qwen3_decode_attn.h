@@ -185,17 +185,21 @@ int qwen3_decode_attn_append_and_attend(qda_handle *h,
  * position positions[b] + t (or L - T + t when positions is NULL), and its
  * query attends over slots 0 .. L - T + t: the cache before the call plus the
  * new tokens up to and including itself.
- * new_tokens = 1 is exactly qwen3_decode_attn_append_and_attend. For T > 1 one
- * launch takes up to 16 query rows per kv head (T * Hq / 8 <= 16: T <= 8 at
- * 16 query heads, 4 at 32, 3 at 40, 2 at 64); a longer block runs as
- * consecutive launches over chunks of its tokens, each chunk attending over
- * the cache plus the block's tokens up to its own, so the result is the same
- * causal attention (a chunked prefill; each launch reads the sequence's whole
- * cache again). Up to 8 query rows per kv head q and the probabilities enter
- * the tensor cores as two bf16 terms (about 16 significant bits); with 9 to
- * 16 rows they enter as bf16 (8 bits), with float sums either way. Each
- * launch of the tensor-core kernel is followed by one that combines the
- * sequences split across CTAs.
+ * new_tokens = 1 is exactly qwen3_decode_attn_append_and_attend. For T > 1
+ * with up to 16 query rows per kv head (T * Hq / 8 <= 16: T <= 8 at 16 query
+ * heads, 4 at 32, 3 at 40, 2 at 64) one launch of the decode-shaped
+ * tensor-core kernel takes the block, followed by one that combines the
+ * sequences split across CTAs. Up to 8 query rows per kv head q and the
+ * probabilities enter the tensor cores as two bf16 terms (about 16
+ * significant bits); with 9 to 16 rows they enter as bf16 (8 bits), with
+ * float sums either way. A longer block runs as a chunked prefill: chunks of
+ * 128 / G tokens (G = Hq / 8; 64 tokens at 16 query heads, 32 at 32, 25 at
+ * 40, 16 at 64), each chunk attending over the cache plus the block's tokens
+ * up to its own, so the result is the same causal attention. A chunk is three
+ * launches: its k and v appended and its query rows formed, the attention
+ * (each kv head's query rows of the chunk as one 128-row tile on the tensor
+ * cores, so the cache is read once per chunk; q and the probabilities in bf16,
+ * float sums), and the combine.
  * Errors as for qwen3_decode_attn_append_and_attend, plus INVALID_ARG for
  * new_tokens outside [1, min(QDA_MAX_NEW_TOKENS, max_seq_len)]; on the
  * device, a seq_len below T is out of range like one above the limits. */

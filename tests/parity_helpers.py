@@ -212,42 +212,27 @@ def assert_o_close(o_got, o_ref, label=""):
 Q_SCALE = 1.4426950408889634 / np.sqrt(128.0)
 
 
-PREFILL_FROM = 64   # query rows per kv head from which a block runs as the prefill
-
-
 def chunk_sizes(num_q_heads: int, T: int):
     """How the library runs a block of T new tokens: up to 16 query rows per kv
-    head (T * Hq / 8) in one launch of the decode-shaped tensor-core kernel;
-    from PREFILL_FROM rows as a chunked prefill, chunks of 128 / G tokens; in
-    between as chunks of 16 / G tokens of the decode-shaped kernel (at 16 query
-    heads a last chunk of one token borrows one from the chunk before)."""
+    head (T * Hq / 8) in one launch of the decode-shaped tensor-core kernel; a
+    longer block as a chunked prefill, chunks of 128 / G tokens."""
     G = num_q_heads // 8
     if T * G <= 16:
         return [T]
-    max_t = 128 // G if T * G >= PREFILL_FROM else 16 // G
-    sizes, c0 = [], 0
-    while c0 < T:
-        n = min(max_t, T - c0)
-        if T * G < PREFILL_FROM and num_q_heads == 16 and T - c0 - n == 1:
-            n -= 1
-        sizes.append(n)
-        c0 += n
-    return sizes
+    max_t = 128 // G
+    return [min(max_t, T - c0) for c0 in range(0, T, max_t)]
 
 
 def wide_tokens(w: inputs.Workload):
     """Per new token: whether its launch takes q and the probabilities into the
-    tensor cores as bf16 (more than 8 query rows per kv head in the launch, and
-    every prefill chunk)."""
+    tensor cores as bf16 (more than 8 query rows per kv head in a decode-shaped
+    launch, and every prefill chunk)."""
     G = w.num_q_heads // 8
     if w.new_tokens == 1:
         return [False]
-    if w.new_tokens * G >= PREFILL_FROM:
+    if w.new_tokens * G > 16:
         return [True] * w.new_tokens
-    flags = []
-    for n in chunk_sizes(w.num_q_heads, w.new_tokens):
-        flags += [n * G > 8] * n
-    return flags
+    return [w.new_tokens * G > 8] * w.new_tokens
 
 
 def is_wide(w: inputs.Workload) -> bool:

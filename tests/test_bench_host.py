@@ -3,6 +3,8 @@ reductions over ranks (gloo, world size 2) and rank-distinct replicas."""
 import os
 import socket
 
+import types
+
 import pytest
 import torch
 import torch.distributed as dist
@@ -35,7 +37,15 @@ def test_projection_byte_and_flop_counts():
 
 def test_kernel_and_workload_keys():
     assert bench.kernel_key(16, 1) == 16
-    assert bench.kernel_key(16, 2) == bench.kernel_key(64, 1) == "grouped"
+    assert bench.kernel_key(16, 2) == bench.kernel_key(64, 1) == bench.kernel_key(16, 8) == "grouped"
+    assert bench.kernel_key(16, 9) == bench.kernel_key(40, 4) == bench.kernel_key(64, 3) == "prefill"
+    # prefill chunks of 128 / G tokens, three launches each
+    args = types.SimpleNamespace(new_tokens=130, num_q_heads=16)
+    assert bench.chunk_tokens(args) == [64, 64, 2] and bench.grouped_launches(args) == 9
+    args = types.SimpleNamespace(new_tokens=30, num_q_heads=40)
+    assert bench.chunk_tokens(args) == [25, 5]
+    args = types.SimpleNamespace(new_tokens=8, num_q_heads=16)
+    assert bench.chunk_tokens(args) == [8] and bench.grouped_launches(args) == 2
     assert bench.workload_key("cfg2") == "cfg2"
     assert bench.workload_key("cfg2", 64) == "cfg2-h64"
     assert bench.workload_key("cfg2", 16, 4) == "cfg2-t4"

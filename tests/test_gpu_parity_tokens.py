@@ -1,5 +1,7 @@
-"""Parity of the step with several new tokens per sequence (T = 2..8, causal
-inside the new block) with the float64 oracle, through the C ABI.
+"""Parity of the step with several new tokens per sequence (causal inside the
+new block) with the float64 oracle, through the C ABI: up to 16 query rows per
+kv head in one launch of the decode-shaped kernel, longer blocks as the chunked
+prefill (128 query rows per kv head per chunk).
 
 Token t of sequence b goes to cache slot L - T + t (L = seq_lens[b] counts the
 new tokens) and its query attends over slots 0 .. L - T + t (Qwen3-0.6B Model
@@ -139,9 +141,9 @@ def test_split_count_does_not_change_the_result(grid):
 
 @pytest.mark.parametrize("hq,T", [(16, 9), (16, 20), (32, 9), (40, 4), (64, 5), (64, 3)])
 def test_blocks_longer_than_one_launch(handles, hq, T):
-    """A block of more new tokens than one launch takes runs as consecutive
-    launches over chunks of it (a chunked prefill): the same cache bits and the
-    same causal attention as the oracle's single pass over the block."""
+    """A block of more than 16 query rows per kv head runs as the prefill: the
+    same cache bits and the same causal attention as the oracle's single pass
+    over the block."""
     lens = [T, T + 1, 16, 31, 33, 47, 48, 300, 1000]
     lens = [max(L, T) for L in lens]
     w = inputs.custom(lens, seed=72 + hq + T, device="cuda", gap_fraction=0.2, num_q_heads=hq, new_tokens=T)
@@ -149,7 +151,7 @@ def test_blocks_longer_than_one_launch(handles, hq, T):
 
 
 def test_a_long_block_over_a_long_cache(handles):
-    """64 new tokens (8 launches at 16 heads) after up to 5000 cached ones, with positions."""
+    """64 new tokens (one prefill chunk of 128 rows at 16 heads) after up to 5000 cached ones, with positions."""
     w = inputs.custom([64, 100, 5064, 777], seed=73, device="cuda", gap_fraction=0.1, new_tokens=64)
     full_check(handles[16], w, "T=64 in chunks", positions=torch.tensor([0, 36, 9000, 713], dtype=torch.int32))
 
@@ -180,13 +182,15 @@ def test_maximum_context(handles):
     full_check(handles[16], w, "T=4 L=40960")
 
 
-@pytest.mark.parametrize("T", [4, 8])
-def test_locality_with_nan_in_unread_bytes(handles, T):
+@pytest.mark.parametrize("hq,T", [(16, 4), (16, 8), (16, 20), (64, 5), (32, 40)])
+def test_locality_with_nan_in_unread_bytes(handles, hq, T):
     """The new tokens' rows (written, never read before), rows past a sequence,
     pages it does not own and table entries past its last page may hold
-    anything (here NaN): o and the appended rows do not change."""
-    attn = handles[16]
-    w = inputs.custom([8, 12, 40, 16, 18], seed=67, device="cuda", pool_pages=16, stride=6, new_tokens=T)
+    anything (here NaN): o and the appended rows do not change. T * Hq / 8 > 16
+    runs the prefill, whose stages also hold rows past a piece's last page."""
+    attn = handles[hq]
+    lens = [max(L, T) for L in [8, 12, 40, 16, 18, 70]]
+    w = inputs.custom(lens, seed=67, device="cuda", pool_pages=24, stride=6, new_tokens=T, num_q_heads=hq)
     ka, va = w.k_cache.clone(), w.v_cache.clone()
     kb, vb = w.k_cache.clone(), w.v_cache.clone()
     bt2 = w.block_table.clone()
@@ -215,22 +219,39 @@ def test_locality_with_nan_in_unread_bytes(handles, T):
         assert torch.equal(va[page, row].view(torch.int16), vb[page, row].view(torch.int16))
 
 
-def test_a_sequence_shorter_than_the_new_block_is_skipped(handles):
+@pytest.mark.parametrize("T", [4, 20])
+def test_a_sequence_shorter_than_the_new_block_is_skipped(handles, T):
     """seq_lens[b] < T is out of range on the device: that sequence is skipped
     (its cache untouched), the others are computed, and the status says BOUNDS."""
     attn = handles[16]
-    w = inputs.custom([40, 3, 30], seed=68, device="cuda", new_tokens=4)
+    w = inputs.custom([40, 3, 30], seed=68, device="cuda", new_tokens=T)
     lens = w.seq_lens.clone()
     k, v = w.k_cache.clone(), w.v_cache.clone()
     k0, v0 = w.k_cache.clone(), w.v_cache.clone()
     o = ph.run(attn, w, DEV, k, v)
     assert attn.check() == binding.QDA_ERR_BOUNDS
-    ref = ph.oracle_sampled(w, [0, 2], w.k_cache, w.v_cache)
-    ph.assert_o_close(o[[0, 2]], ref, "T=4 with a short sequence")
+    sampled_check(o, w, [0, 2], w.k_cache, w.v_cache, f"T={T} with a short sequence")
     page1 = int(w.block_table[1, 0])
     assert torch.equal(k[page1].view(torch.int16), k0[page1].view(torch.int16))
     assert torch.equal(v[page1].view(torch.int16), v0[page1].view(torch.int16))
     assert int(lens[1]) == 3
+    assert attn.check() == 0
+
+
+@pytest.mark.parametrize("hq,T", [(16, 20), (64, 5)])
+def test_prefill_out_of_range_page_ids_are_not_dereferenced(handles, hq, T):
+    """A block-table entry outside [0, num_pages) among a sequence's older
+    pages: not copied, the status says BOUNDS, the other sequences are
+    computed."""
+    attn = handles[hq]
+    w = inputs.custom([40, 70, 30], seed=69, device="cuda", pool_pages=16, stride=5, new_tokens=T, num_q_heads=hq)
+    k, v = w.k_cache.clone(), w.v_cache.clone()
+    bt = w.block_table.clone()
+    bt[1, 1] = 16
+    a = ph.device_args(w, DEV)
+    o = attn(a["qkv"], a["q_norm_w"], a["k_norm_w"], a["seq_lens"], bt.to(DEV), k, v)
+    assert attn.check() == binding.QDA_ERR_BOUNDS
+    sampled_check(o, w, [0, 2], w.k_cache, w.v_cache, f"Hq={hq} T={T} bad page id")
     assert attn.check() == 0
 
 
@@ -260,6 +281,13 @@ def full_size_check(attn, w, sample, label):
     k_exp, v_exp = ph.expected_cache(w, k_pre, v_pre, k_rows, v_rows)
     ph.assert_cache_equal(w.k_cache, w.v_cache, k_exp, v_exp, k64, w)
     del k_exp, v_exp
+    return sampled_check(o, w, sample, k_pre, v_pre, label)
+
+
+def sampled_check(o, w, sample, k_pre, v_pre, label):
+    """o of the sequences `sample` against the oracle over those sequences
+    alone (caches before the call): the gate, then the strict bound or, for
+    tokens that took q as bf16, the bf16-q bound."""
     if ph.is_wide(w):
         ref, lens, bt = ph.oracle_sampled_qk(w, sample, k_pre, v_pre)
         ref["seq_lens"], ref["block_table"] = lens, bt
