@@ -83,7 +83,7 @@ __device__ __forceinline__ int pf_first_position(const Params& p, int b, int L, 
 }
 
 // ---------------------------------------------------------------------------
-// 1. The prep: warp w of CTA (b, j, z) takes token u = 4z + w of the chunk.
+// 1. The prep: warp w of CTA (b, j, z) takes token u = 8z + w of the chunk.
 // It forms the token's new k (RMSNorm and RoPE in double, rounded once to
 // bf16) and writes k and v to their cache slots, and forms the token's G query
 // rows of kv head j (RMSNorm and RoPE in float, the angle reduced modulo 2*pi
@@ -92,21 +92,24 @@ __device__ __forceinline__ int pf_first_position(const Params& p, int b, int L, 
 // a head) and 64+2l, 65+2l (word 32+l), the RoPE pairs (i, i+64).
 
 template <int G>
-__global__ void __launch_bounds__(128) prefill_prep_kernel(const Params p, const PrefillScratch sc) {
+__global__ void __launch_bounds__(256) prefill_prep_kernel(const Params p, const PrefillScratch sc) {
     constexpr int kHq = G * kNumKvHeads;
     constexpr int kQkvW = (kHq + 2 * kNumKvHeads) * kHeadDim;
+    __shared__ double inv_freq[kHeadDim / 2];   // theta^(-2i/128), shared by the CTA's tokens
+    if (threadIdx.x < kHeadDim / 2) inv_freq[threadIdx.x] = pow(p.rope_theta, -2.0 * (int)threadIdx.x / 128.0);
     pdl_wait();
     pdl_launch_dependents();
+    __syncthreads();
     const int b = blockIdx.x, j = blockIdx.y, lane = threadIdx.x & 31;
-    const int u = 4 * (int)blockIdx.z + (int)(threadIdx.x >> 5);
+    const int u = 8 * (int)blockIdx.z + (int)(threadIdx.x >> 5);
     const int n = p.new_tokens;
     if (u >= n) return;
     const int L_all = p.seq_lens[b];
     if (!length_ok(p, L_all)) return;   // the attention launch records it and skips the sequence
     const int L = L_all - p.len_trim;
     const double pos = (double)(pf_first_position(p, b, L, n) + u);
-    const double ang0 = reduce_angle(pos * pow(p.rope_theta, -2.0 * (2 * lane) / 128.0));
-    const double ang1 = reduce_angle(pos * pow(p.rope_theta, -2.0 * (2 * lane + 1) / 128.0));
+    const double ang0 = reduce_angle(pos * inv_freq[2 * lane]);
+    const double ang1 = reduce_angle(pos * inv_freq[2 * lane + 1]);
     const uint32_t* row = reinterpret_cast<const uint32_t*>(p.qkv + pf_token_row(p, b, u) * kQkvW);
 
     const int slot = L - n + u;
@@ -188,55 +191,68 @@ __global__ void __launch_bounds__(128) prefill_prep_kernel(const Params p, const
 // and O, accumulated in tensor memory over the piece, is read out once at the
 // piece's end.
 //
-// Warp roles (256 threads): warp 0 issues the copies; one thread of warp 1
-// issues the tensor-core instructions (warp 1 also allocates tensor memory);
-// warps 4-7 run the softmax and write o (warp 4 + w reads tensor-memory lanes
-// 32w..32w+31, the rows it owns). Every wait is bounded: a timeout records
-// QDA_ERR_TIMEOUT, sets the CTA's abort flag and every role leaves its loop;
-// tensor memory is freed after every issued instruction has completed.
+// Warp roles (384 threads): warps 0 and 3 issue the copies of K (and Q) and
+// of V; one thread of warp 1 issues S and one of warp 2 issues O += P V (warp 1
+// also allocates tensor memory); warps 4-11 run the softmax in two warpgroups, each over half of a
+// stage's keys with an accumulator of its own, and write o. Every wait is
+// bounded: a timeout records QDA_ERR_TIMEOUT, sets the CTA's abort flag and
+// every role leaves its loop; tensor memory is freed after every issued
+// instruction has completed.
 
 constexpr int kTcKeys = 64;                          // cache rows per stage
 constexpr int kTcPages = kTcKeys / kPage;            // 4
-constexpr int kTcStages = 4;
-constexpr int kTcThreads = 8 * 32;
+// K and V sit in rings of their own: a K slot is free once S has read it, a V
+// slot only once O += P V has. A stage stays in a V slot from its copy through
+// S, the softmax and the product, so the V ring is the deeper one: with about
+// three stages held in processing it still keeps two or more in flight.
+constexpr int kTcKSlots = 4;
+constexpr int kTcVSlots = 5;
+constexpr int kTcThreads = 12 * 32;
 constexpr int kTcHalf = kTcKeys * 128;               // 64 dims of a stage's rows: 8 KiB
-constexpr int kTcStageK = 0;                         // K dims 0-63 | K dims 64-127
-constexpr int kTcStageV = 2 * kTcHalf;               // V dims 0-63 | V dims 64-127
-constexpr int kTcStageBytes = 4 * kTcHalf;           // 32 KiB
+constexpr int kTcSlotBytes = 2 * kTcHalf;            // a K or V slot: dims 0-63 | dims 64-127
 constexpr int kTcBoxBytes = kPage * 128;             // one copied box: 16 rows x 64 dims
 constexpr int kTcTile = kPrefillRows * 128;          // 64 columns of a 128-row operand: 16 KiB
-constexpr int kTcSmemQ = kTcStages * kTcStageBytes;  // 2 buffers: Q dims 0-63 | Q dims 64-127
-constexpr int kTcSmemP = kTcSmemQ + 4 * kTcTile;     // P: 128 rows x 64 keys
-constexpr int kTcSmemSeg = kTcSmemP + kTcTile;                       // int [kMaxBatch + 4]
-constexpr int kTcSmemLens = kTcSmemSeg + (kMaxBatch + 4) * 4;        // int [kMaxBatch]
-constexpr int kTcSmemMask = kTcSmemLens + kMaxBatch * 4;             // int [kTcStages]: pages not copied
-constexpr int kTcSmemBars = kTcSmemMask + kTcStages * 4;
-// kv_full[S], kv_empty[S], s_full[2], p_full, pv_done, q_full[2], q_free[2], fin
-constexpr int kTcNumBars = 2 * kTcStages + 9;
-constexpr int kTcSmemTmem = kTcSmemBars + kTcNumBars * 8;            // tensor-memory address, abort flag
-constexpr int kTcSmemTotal = kTcSmemTmem + 16;
-constexpr int kTcSmemAlloc = kTcSmemTotal + 1024;   // slack to align the tiles to 1024 bytes
-constexpr uint32_t kTcTmemCols = 256;               // S buffers at columns 0 and 64, O at 128
+// Shared memory: the small items first, then the tiles on the next 1024-byte
+// boundary (the swizzle atom).
+// k_full[K], k_empty[K], v_full[V], v_empty[V], s_full[2], p_full[2],
+// pv_done[2], q_full[2], q_free[2], ml_ready[2], fin
+constexpr int kTcNumBars = 2 * kTcKSlots + 2 * kTcVSlots + 13;
+constexpr int kTcSmemTmem = kTcNumBars * 8;                          // tensor-memory address, abort flag
+constexpr int kTcSmemMask = kTcSmemTmem + 16;                        // int [kTcVSlots]: pages not copied
+constexpr int kTcSmemSeg = kTcSmemMask + kTcVSlots * 4;              // int [kMaxBatch + 4]
+constexpr int kTcSmall = (kTcSmemSeg + (kMaxBatch + 4) * 4 + 15) / 16 * 16;
+constexpr int kTcTileV = kTcKSlots * kTcSlotBytes;   // from the tiles' start: K ring, V ring,
+constexpr int kTcTileQ = kTcTileV + kTcVSlots * kTcSlotBytes;   // 2 buffers of Q dims 0-63 | 64-127,
+constexpr int kTcTileP = kTcTileQ + 4 * kTcTile;                // P: 128 rows x 64 keys
+constexpr int kTcTiles = kTcTileP + kTcTile;
+constexpr int kTcSmemAlloc = kTcSmall + 1024 + kTcTiles;   // with up to 1023 bytes of padding
+// tensor-memory columns: S buffers at 0 and 64, O_0 at 128, O_1 at 256, the
+// (m, l) swap at 384
+constexpr uint32_t kTcTmemCols = 512;
 constexpr uint32_t kTcTmemO = 128;
-static_assert(kTcStageBytes % 1024 == 0 && kTcSmemSeg % 1024 == 0, "swizzle atoms are 1024-byte aligned");
-static_assert(kTcSmemBars % 8 == 0 && 2 * kTcTile == kPrefillQTileBytes, "layout");
+constexpr uint32_t kTcTmemMl = 384;
+static_assert(kTcSlotBytes % 1024 == 0 && kTcTile % 1024 == 0, "swizzle atoms are 1024-byte aligned");
+static_assert(kTcSmall % 16 == 0 && 2 * kTcTile == kPrefillQTileBytes, "layout");
 static_assert(kTcSmemAlloc <= 227 * 1024, "fits one CTA per SM");
 static_assert(kTcKeys == 64, "a P row is one 128-byte swizzled row");
 
 struct TcShared {
-    uint8_t* stages;
+    uint8_t* k;          // K ring
+    uint8_t* v;          // V ring
     uint8_t* q;
     uint8_t* p;
     int* seg;
-    int* lens;
-    volatile int* mask;
-    uint64_t* kv_full;
-    uint64_t* kv_empty;
-    uint64_t* s_full;
-    uint64_t* p_full;
-    uint64_t* pv_done;
-    uint64_t* q_full;   // [2]
-    uint64_t* q_free;   // [2]
+    volatile int* mask;  // [kTcVSlots]: pages of the stage in V slot i that were not copied
+    uint64_t* k_full;
+    uint64_t* k_empty;
+    uint64_t* v_full;
+    uint64_t* v_empty;
+    uint64_t* s_full;    // [2]: S of stage g in S buffer g % 2
+    uint64_t* p_full;    // [2]: P written for stage g (g % 2)
+    uint64_t* pv_done;   // [2]: O += P V of stage g (g % 2) completed
+    uint64_t* q_full;    // [2]
+    uint64_t* q_free;    // [2]
+    uint64_t* ml_ready;  // [2]: both warpgroups have posted (m, l) of piece u (u % 2)
     uint64_t* fin;
     volatile int* abort_flag;
 };
@@ -299,13 +315,19 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 
 __device__ __forceinline__ void fence_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// Warp 0: the page ids (32 page-heads looked up at a time), then per stage
-// four tiled copies per page: K and V of kv head j, dims 0-63 and 64-127,
-// into the stage's halves at 2 KiB per page. Pages whose block-table entry is
-// out of range are not copied; the stage's mask tells the softmax.
+// The copies, one warp per ring: warp 0 fills the K ring (and copies each
+// piece's query tile), warp 3 the V ring. Each looks the page ids up 32
+// page-heads at a time, then per stage issues two tiled copies per page (kv
+// head j, dims 0-63 and 64-127) into the slot's halves at 2 KiB per page.
+// Pages whose block-table entry is out of range are not copied; the V warp's
+// mask of them tells the softmax.
+template <bool kIsV>
 __device__ __forceinline__ void tc_producer(const Params& p, const PrefillScratch& sc, const TcShared& s,
-                                            const CUtensorMap* tm_k, const CUtensorMap* tm_v, int B, int start,
-                                            int end, int lane) {
+                                            const CUtensorMap* tm, int B, int start, int end, int lane) {
+    constexpr int kSlots = kIsV ? kTcVSlots : kTcKSlots;
+    uint64_t* full = kIsV ? s.v_full : s.k_full;
+    uint64_t* empty = kIsV ? s.v_empty : s.k_empty;
+    uint8_t* ring = kIsV ? s.v : s.k;
     const uint32_t q_bytes = (uint32_t)(p.new_tokens * (p.num_q_heads / kNumKvHeads)) * 128u;   // R rows per half
     int wbase = 0x40000000, id = -1;
     uint32_t g = 0, u = 0, armed = 0, armed_parity = 0, q_armed = 0;
@@ -314,9 +336,9 @@ __device__ __forceinline__ void tc_producer(const Params& p, const PrefillScratc
     PieceWalk w;
     w.begin(s.seg, B, start, end);
     do {
-        // the piece's query tile, into buffer u % 2 once the piece two back has
-        // finished reading it
-        {
+        if (!kIsV) {
+            // the piece's query tile, into buffer u % 2 once the piece two back
+            // has finished reading it
             int good = 1;
             if (lane == 0) {
                 if (u >= 2) good = tc_wait1(p, s, &s.q_free[u & 1u], ((u >> 1) - 1) & 1u) ? 1 : 0;
@@ -349,10 +371,9 @@ __device__ __forceinline__ void tc_producer(const Params& p, const PrefillScratc
                     id = __ldg(p.block_table + (size_t)bb * p.bt_stride + r % np);
                 }
             }
-            const int st = (int)(g % kTcStages);
+            const int st = (int)(g % kSlots);
             int good = 1;
-            if (lane == 0 && g >= (uint32_t)kTcStages)
-                good = tc_wait1(p, s, &s.kv_empty[st], ((g / kTcStages) - 1) & 1u) ? 1 : 0;
+            if (lane == 0 && g >= (uint32_t)kSlots) good = tc_wait1(p, s, &empty[st], ((g / kSlots) - 1) & 1u) ? 1 : 0;
             if (!__shfl_sync(kFull, good, 0)) {
                 ok = false;
                 break;
@@ -360,181 +381,205 @@ __device__ __forceinline__ void tc_producer(const Params& p, const PrefillScratc
             const int my = __shfl_sync(kFull, id, (x0 - wbase + lane) & 31);
             const uint32_t bad = __ballot_sync(kFull, lane < npg && (my < 0 || my >= p.num_pages));
             if (lane == 0) {
-                s.mask[st] = (int)bad;
-                if (bad != 0) record_error(p.status, QDA_ERR_BOUNDS);
+                if (kIsV) {
+                    s.mask[st] = (int)bad;
+                    if (bad != 0) record_error(p.status, QDA_ERR_BOUNDS);
+                }
                 const int copied = npg - __popc(bad);
                 if (copied > 0) {
-                    mbar_arrive_expect_tx(&s.kv_full[st], (uint32_t)(copied * 4 * kTcBoxBytes));
+                    mbar_arrive_expect_tx(&full[st], (uint32_t)(copied * 2 * kTcBoxBytes));
                     armed |= 1u << st;
-                    armed_parity = (armed_parity & ~(1u << st)) | (((g / kTcStages) & 1u) << st);
+                    armed_parity = (armed_parity & ~(1u << st)) | (((g / kSlots) & 1u) << st);
                 } else {
-                    mbar_arrive(&s.kv_full[st]);
+                    mbar_arrive(&full[st]);
                 }
             }
-            const uint32_t dst = smem_addr(s.stages + st * kTcStageBytes);
+            const uint32_t dst = smem_addr(ring + st * kTcSlotBytes);
             for (int k = 0; k < npg; ++k) {
                 const int page = __shfl_sync(kFull, my, k);
                 if (lane == 0 && ((bad >> k) & 1u) == 0) {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        tma_load_3d(dst + kTcStageK + h * kTcHalf + k * kTcBoxBytes, tm_k, 64 * h, w.j, page * kPage,
-                                    &s.kv_full[st]);
-                        tma_load_3d(dst + kTcStageV + h * kTcHalf + k * kTcBoxBytes, tm_v, 64 * h, w.j, page * kPage,
-                                    &s.kv_full[st]);
-                    }
+                    tma_load_3d(dst + k * kTcBoxBytes, tm, 0, w.j, page * kPage, &full[st]);
+                    tma_load_3d(dst + kTcHalf + k * kTcBoxBytes, tm, 64, w.j, page * kPage, &full[st]);
                 }
             }
         }
     } while (ok && w.next(s.seg, B));
     if (lane == 0 && *s.abort_flag != 0) {
         // copies still landing in this CTA's shared memory: wait (bounded) for each
-        for (int k = 0; k < kTcStages; ++k)
-            if (armed & (1u << k)) (void)mbar_wait(&s.kv_full[k], (armed_parity >> k) & 1u, p.timeout_ns, nullptr);
+        for (int k = 0; k < kSlots; ++k)
+            if (armed & (1u << k)) (void)mbar_wait(&full[k], (armed_parity >> k) & 1u, p.timeout_ns, nullptr);
         for (int k = 0; k < 2; ++k)
             if ((q_armed >> (2 * k)) & 2u)
                 (void)mbar_wait(&s.q_full[k], (q_armed >> (2 * k)) & 1u, p.timeout_ns, nullptr);
     }
 }
 
-// One thread of warp 1: per stage g, S_g = Q K_g^T into S buffer g % 2, then
-// O += P_{g-1} V_{g-1} once the softmax has written P_{g-1}. S_g overwrites
-// the buffer the softmax of stage g - 2 read, which it had finished before
-// writing P_{g-2}.
-__device__ __forceinline__ void tc_issuer(const Params& p, const TcShared& s, int B, int start, int end,
-                                          uint32_t tmem) {
+// The tensor-core instructions come from two threads, so that their issue
+// (about 0.05 us per instruction and thread, whatever its size) runs in two
+// streams: one issues S, the other O += P V.
+//
+// Lane 0 of warp 1: per stage g, S_g = Q K_g^T into S buffer g % 2, once K_g
+// has landed and the softmax of stage g - 2 has finished reading that buffer
+// (it read S before writing P_{g-2}); the K slot is free once S_g completes.
+__device__ __forceinline__ void tc_issue_s(const Params& p, const TcShared& s, int B, int start, int end,
+                                           uint32_t tmem) {
     const uint32_t idesc_s = umma_idesc_bf16_m128(kTcKeys);
-    const uint32_t idesc_o = umma_idesc_bf16_m128_bmn(kHeadDim);
-    const uint32_t p_base = smem_addr(s.p), st_base = smem_addr(s.stages);
-    auto pv = [&](uint32_t x, bool first) -> bool {
-        if (!tc_wait1(p, s, s.p_full, x & 1u)) return false;
-        tc_fence_after();
-        const uint32_t v = st_base + (x % kTcStages) * kTcStageBytes + kTcStageV;
-#pragma unroll
-        for (int kk = 0; kk < kTcKeys / 16; ++kk)
-            umma_bf16(tmem + kTcTmemO, umma_desc_sw128(p_base + 32 * kk),
-                      umma_desc_sw128_mn(v + 2 * 1024 * kk, kTcHalf, 1024), idesc_o, (first && kk == 0) ? 0u : 1u);
-        umma_commit(s.pv_done);
-        umma_commit(&s.kv_empty[x % kTcStages]);   // K and V of the stage have been read
-        return true;
-    };
+    const uint32_t k_base = smem_addr(s.k);
     uint32_t g = 0, u = 0;
-    bool prev_first = false, ok = true;
+    bool ok = true;
     PieceWalk w;
     w.begin(s.seg, B, start, end);
     do {
-        if (!tc_wait1(p, s, &s.q_full[u & 1u], (u >> 1) & 1u)) {
-            ok = false;
-            break;
-        }
+        if (!tc_wait1(p, s, &s.q_full[u & 1u], (u >> 1) & 1u)) break;
         tc_fence_after();
         const uint32_t q_base = smem_addr(s.q) + (u & 1u) * 2 * kTcTile;
         for (int q = 0; q < w.n; q += kTcPages, ++g) {
-            const int st = (int)(g % kTcStages);
-            if (!tc_wait1(p, s, &s.kv_full[st], (g / kTcStages) & 1u)) {
+            const int st = (int)(g % kTcKSlots);
+            if (!tc_wait1(p, s, &s.k_full[st], (g / kTcKSlots) & 1u) ||
+                (g >= 2 && !tc_wait1(p, s, &s.p_full[g & 1u], ((g - 2) >> 1) & 1u))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t kb = st_base + st * kTcStageBytes + kTcStageK;
+            const uint32_t kb = k_base + st * kTcSlotBytes;
             const uint32_t sd = tmem + (g & 1u) * kTcKeys;
 #pragma unroll
             for (int kk = 0; kk < kHeadDim / 16; ++kk)
                 umma_bf16(sd, umma_desc_sw128(q_base + (kk >> 2) * kTcTile + (kk & 3) * 32),
                           umma_desc_sw128(kb + (kk >> 2) * kTcHalf + (kk & 3) * 32), idesc_s, kk != 0 ? 1u : 0u);
             umma_commit(&s.s_full[g & 1u]);
+            umma_commit(&s.k_empty[st]);
             if (q + kTcPages >= w.n) umma_commit(&s.q_free[u & 1u]);   // the piece's last product reading Q
-            if (g > 0 && !pv(g - 1, prev_first)) {
-                ok = false;
-                break;
-            }
-            prev_first = q == 0;
         }
         ++u;
     } while (ok && w.next(s.seg, B));
-    if (ok && g > 0) (void)pv(g - 1, prev_first);
-    umma_commit(s.fin);   // every instruction issued above has completed
+    umma_commit(s.fin);   // counts once every instruction issued above has completed
 }
 
-// Warps 4-7, thread = row r = 32 * (warp - 4) + lane.
+// Lane 0 of warp 2: per stage x, once both softmax warpgroups have written
+// P_x, O_0 += P_x[:, 0:32] V_x[0:32] and O_1 += P_x[:, 32:64] V_x[32:64], each
+// accumulator starting afresh at its piece's first stage; the V slot (and the
+// P tile) are free once these complete.
+__device__ __forceinline__ void tc_issue_pv(const Params& p, const TcShared& s, int B, int start, int end,
+                                            uint32_t tmem) {
+    const uint32_t idesc_o = umma_idesc_bf16_m128_bmn(kHeadDim);
+    const uint32_t pb = smem_addr(s.p), v_base = smem_addr(s.v);
+    uint32_t x = 0;
+    bool ok = true;
+    PieceWalk w;
+    w.begin(s.seg, B, start, end);
+    do {
+        for (int q = 0; q < w.n; q += kTcPages, ++x) {
+            if (!tc_wait1(p, s, &s.p_full[x & 1u], (x >> 1) & 1u)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t v = v_base + (x % kTcVSlots) * kTcSlotBytes;
+#pragma unroll
+            for (int kk = 0; kk < kTcKeys / 16; ++kk)   // 16 keys per instruction; keys 32h.. go to O_h
+                umma_bf16(tmem + kTcTmemO + (kk >> 1) * kHeadDim, umma_desc_sw128(pb + 32 * kk),
+                          umma_desc_sw128_mn(v + 2 * 1024 * kk, kTcHalf, 1024), idesc_o,
+                          (q == 0 && (kk & 1) == 0) ? 0u : 1u);
+            umma_commit(&s.pv_done[x & 1u]);
+            umma_commit(&s.v_empty[x % kTcVSlots]);
+        }
+    } while (ok && w.next(s.seg, B));
+    umma_commit(s.fin);
+}
+
+// Warps 4-11, two warpgroups: thread t owns row r = t % 128 and keys 32h ..
+// 32h + 31 of every stage, h = t / 128 (warp 4 + 4h + q reads tensor-memory
+// lanes 32q..32q+31), with its own running max m_h, sum l_h and accumulator
+// O_h. At a piece's end the halves are merged (the log-sum-exp rule):
+//   M = max(m_0, m_1), a_h = exp2(m_h - M),
+//   o = (a_0 O_0 + a_1 O_1) / (a_0 l_0 + a_1 l_1),
+// warpgroup h writing dims 64h .. 64h + 63, after the two have swapped (m, l)
+// through tensor memory.
 template <int G>
 __device__ __forceinline__ void tc_softmax(const Params& p, const PrefillScratch& sc, const TcShared& s, int B,
-                                           int start, int end, int per_cta, int r, uint32_t tmem) {
+                                           int start, int end, int per_cta, int t, uint32_t tmem) {
     constexpr int kHq = G * kNumKvHeads;
-    const int lane = r & 31;
+    const int r = t & 127, h = t >> 7, lane = t & 31;
     const int n = p.new_tokens, R = n * G;
     const bool active = r < R;
     const bool warp_active = (r & ~31) < R;
     const int tt = active ? r / G : 0;
     const uint32_t lanes = tmem + ((uint32_t)(r & ~31) << 16);
+    const uint32_t o_own = lanes + kTcTmemO + (uint32_t)h * kHeadDim;
     const uint32_t p_row = smem_addr(s.p) + r * 128;
-    uint32_t g = 0, pv_seen = 0;
+    uint32_t g = 0, u = 0, pv_seen[2] = {0u, 0u};
     bool ok = true;
-    auto pv_wait = [&](uint32_t x) -> bool {   // O += P_x V_x has completed
-        if (pv_seen > x) return true;
-        if (!tc_wait_warp(p, s, s.pv_done, x & 1u, lane)) return false;
-        pv_seen = x + 1;
+    // O += P_x V_x has completed: completion x / 2 of pv_done[x % 2]. The
+    // phases of each barrier are waited for in order, and none can complete
+    // two ahead of this warp (P_{x+2} is written after this wait).
+    auto pv_wait = [&](uint32_t x) -> bool {
+        const uint32_t k = x & 1u, c = x >> 1;
+        if (pv_seen[k] > c) return true;
+        if (!tc_wait_warp(p, s, &s.pv_done[k], c & 1u, lane)) return false;
+        pv_seen[k] = c + 1;
         return true;
     };
     PieceWalk w;
     w.begin(s.seg, B, start, end);
     do {
         const int np_b = s.seg[w.b + 1] - s.seg[w.b];
-        const int L = s.lens[w.b];
-        const int lim = active ? L - n + tt : -1;   // the last cache slot this row sees
+        const int L = p.seq_lens[w.b] - p.len_trim;   // the piece's sequence passed the length checks
+        const int lim = active ? L - n + tt : -1;     // the last cache slot this row sees
         float m = -INFINITY, lsum = 0.f;
         for (int q = 0; q < w.n; q += kTcPages, ++g) {
             const int npg = min(kTcPages, w.n - q);
             const int slot0 = kPage * (w.i0 + q);
-            const int st = (int)(g % kTcStages);
-            if (!tc_wait_warp(p, s, &s.kv_full[st], (g / kTcStages) & 1u, lane)) {
+            const int st = (int)(g % kTcVSlots);
+            if (!tc_wait_warp(p, s, &s.v_full[st], (g / kTcVSlots) & 1u, lane)) {
                 ok = false;
                 break;
             }
             const uint32_t bad = (uint32_t)s.mask[st];
-            {
+            if (h == 0) {
                 // cache rows of the stage that hold nothing valid (after the
                 // sequence, past the piece, not copied) may hold any bytes: a
                 // NaN there times a zero probability would still give NaN, so
                 // their V rows are zeroed (thread r: row r % 64, half r / 64)
                 const int kr = r & 63, pg = kr >> 4;
                 if (pg >= npg || ((bad >> pg) & 1u) != 0 || slot0 + kr >= L) {
-                    const uint32_t row = smem_addr(s.stages + st * kTcStageBytes + kTcStageV + (r >> 6) * kTcHalf) +
-                                         kr * 128;
+                    const uint32_t row = smem_addr(s.v + st * kTcSlotBytes + (r >> 6) * kTcHalf) + kr * 128;
 #pragma unroll
                     for (int c = 0; c < 8; ++c) st_shared_v4(row + 16 * c, 0u, 0u, 0u, 0u);
                 }
             }
-            uint32_t pw[kTcKeys / 2];
+            uint32_t pw[8];
             if (warp_active) {
                 if (!tc_wait_warp(p, s, &s.s_full[g & 1u], (g >> 1) & 1u, lane)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                uint32_t raw[4][16];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld16(lanes + (g & 1u) * kTcKeys + 16 * c, raw[c]);
+                uint32_t raw[2][16];
+                tmem_ld16(lanes + (g & 1u) * kTcKeys + 32 * h, raw[0]);
+                tmem_ld16(lanes + (g & 1u) * kTcKeys + 32 * h + 16, raw[1]);
                 tmem_ld_wait();
-                float sv[kTcKeys];
-                // keys c <= climit are inside this row's causal window and the piece's pages
-                const int climit = min(lim - slot0, kPage * npg - 1);
+                float sv[32];
+                // key 32h + c is inside this row's causal window and the piece's pages when c <= climit
+                const int climit = min(lim - slot0, kPage * npg - 1) - 32 * h;
+                const uint32_t badh = (bad >> (2 * h)) & 3u;   // pages 2h, 2h + 1 of the stage
                 float mx = -INFINITY;
-                if (bad == 0 && climit >= kTcKeys - 1) {
+                if (badh == 0 && climit >= 31) {
 #pragma unroll
-                    for (int c = 0; c < kTcKeys; ++c) {
+                    for (int c = 0; c < 32; ++c) {
                         sv[c] = __uint_as_float(raw[c >> 4][c & 15]);
                         mx = fmaxf(mx, sv[c]);
                     }
                 } else {
 #pragma unroll
-                    for (int c = 0; c < kTcKeys; ++c) {
-                        const bool keep = c <= climit && ((bad >> (c >> 4)) & 1u) == 0;
+                    for (int c = 0; c < 32; ++c) {
+                        const bool keep = c <= climit && ((badh >> (c >> 4)) & 1u) == 0;
                         sv[c] = keep ? __uint_as_float(raw[c >> 4][c & 15]) : -INFINITY;
                         mx = fmaxf(mx, sv[c]);
                     }
                 }
                 const bool grow = mx > m + kRescaleThreshold;
-                const bool rescale = grow && m != -INFINITY;   // O holds earlier stages of this piece
+                const bool rescale = grow && m != -INFINITY;   // O_h holds earlier stages of this piece
                 if (__any_sync(kFull, rescale)) {
                     if (!pv_wait(g - 1)) {
                         ok = false;
@@ -545,11 +590,11 @@ __device__ __forceinline__ void tc_softmax(const Params& p, const PrefillScratch
 #pragma unroll 1
                     for (int c = 0; c < kHeadDim / 16; ++c) {
                         uint32_t v[16];
-                        tmem_ld16(lanes + kTcTmemO + 16 * c, v);
+                        tmem_ld16(o_own + 16 * c, v);
                         tmem_ld_wait();
 #pragma unroll
                         for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * a);
-                        tmem_st16(lanes + kTcTmemO + 16 * c, v);
+                        tmem_st16(o_own + 16 * c, v);
                     }
                     tmem_st_wait();
                     lsum *= a;
@@ -557,63 +602,103 @@ __device__ __forceinline__ void tc_softmax(const Params& p, const PrefillScratch
                 if (grow) m = mx;
                 const float mb = m == -INFINITY ? 0.f : m;
 #pragma unroll
-                for (int c = 0; c < kTcKeys / 2; ++c) {
+                for (int c = 0; c < 8; ++c) {
                     pw[c] = pack_bf2(exp2_approx(sv[2 * c] - mb), exp2_approx(sv[2 * c + 1] - mb));
                     lsum += bf_lo(pw[c]) + bf_hi(pw[c]);
                 }
-            }
-            // The previous stage's product has read the P tile. Every warp
-            // waits for it before arriving: p_full counts arrivals, and a warp
-            // must not arrive for stage g + 1 before stage g's phase is over.
-            if (g > 0 && !pv_wait(g - 1)) {
+                uint32_t pw2[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    pw2[c] = pack_bf2(exp2_approx(sv[16 + 2 * c] - mb), exp2_approx(sv[17 + 2 * c] - mb));
+                    lsum += bf_lo(pw2[c]) + bf_hi(pw2[c]);
+                }
+                // the product of stage g - 1 has read the P tile
+                if (g > 0 && !pv_wait(g - 1)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t pr = p_row;
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+                    st_shared_v4(pr + (((4 * h + c) ^ (r & 7)) << 4), pw[4 * c], pw[4 * c + 1], pw[4 * c + 2],
+                                 pw[4 * c + 3]);
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+                    st_shared_v4(pr + (((4 * h + 2 + c) ^ (r & 7)) << 4), pw2[4 * c], pw2[4 * c + 1], pw2[4 * c + 2],
+                                 pw2[4 * c + 3]);
+            } else if (g > 0 && !pv_wait(g - 1)) {
+                // every warp waits before arriving: p_full[g % 2] counts
+                // arrivals, and none may arrive for stage g + 2 before stage
+                // g's phase is over
                 ok = false;
                 break;
             }
-            if (warp_active) {
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    st_shared_v4(p_row + ((c ^ (r & 7)) << 4), pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-            }
+            // one arrival per warp, once every lane's P stores (and V zeroing)
+            // are visible to the tensor cores' proxy
             fence_async_shared();
             tc_fence_before();
-            mbar_arrive(s.p_full);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.p_full[g & 1u]);
         }
         if (!ok) break;
+        // The piece's last products, then the merge of the two halves: o
+        // (unit held whole) or the partials.
+        const uint32_t ml_col = kTcTmemMl + 4 * (u & 1u);
         if (warp_active) {
-            // the piece's last product, then o (whole unit) or the partials
             if (!pv_wait(g - 1)) break;
             tc_fence_after();
+            const uint32_t mine[2] = {__float_as_uint(m), __float_as_uint(lsum)};
+            tmem_st2(lanes + ml_col + 2 * h, mine);
+            tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.ml_ready[u & 1u]);
+        if (!tc_wait_warp(p, s, &s.ml_ready[u & 1u], (u >> 1) & 1u, lane)) break;
+        if (warp_active) {
+            tc_fence_after();
+            uint32_t other[2];
+            tmem_ld2(lanes + ml_col + 2 * (1 - h), other);
+            tmem_ld_wait();
+            const float m0 = h == 0 ? m : __uint_as_float(other[0]), l0 = h == 0 ? lsum : __uint_as_float(other[1]);
+            const float m1 = h == 0 ? __uint_as_float(other[0]) : m, l1 = h == 0 ? __uint_as_float(other[1]) : lsum;
+            const float M = fmaxf(m0, m1);
+            const float a0 = m0 == -INFINITY ? 0.f : exp2_approx(m0 - M);
+            const float a1 = m1 == -INFINITY ? 0.f : exp2_approx(m1 - M);
+            const float Lt = a0 * l0 + a1 * l1;
             const int ustart = 8 * s.seg[w.b] + w.j * np_b;
             const bool whole = ustart / per_cta == (ustart + np_b - 1) / per_cta;
             const int pslot = 2 * (int)blockIdx.x + (w.k == 0 ? 0 : 1);   // the CTA's first piece, else its last
-            const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+            const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
             uint4* orow = reinterpret_cast<uint4*>(p.o + (pf_token_row(p, w.b, tt) * kHq + G * w.j + r % G) * kHeadDim);
             const size_t prow = (size_t)pslot * kPrefillRows + r;
             float4* arow = reinterpret_cast<float4*>(sc.acc + prow * kHeadDim);
 #pragma unroll 1
-            for (int c = 0; c < kHeadDim / 16; ++c) {
-                uint32_t v[16];
-                tmem_ld16(lanes + kTcTmemO + 16 * c, v);
+            for (int c = 4 * h; c < 4 * h + 4; ++c) {   // dims 16c .. 16c + 15
+                uint32_t v0[16], v1[16];
+                tmem_ld16(lanes + kTcTmemO + 16 * c, v0);
+                tmem_ld16(lanes + kTcTmemO + kHeadDim + 16 * c, v1);
                 tmem_ld_wait();
+                float x[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) x[e] = a0 * __uint_as_float(v0[e]) + a1 * __uint_as_float(v1[e]);
                 if (!active) {
                 } else if (whole) {
                     uint32_t o8[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        o8[e] = pack_bf2(__uint_as_float(v[2 * e]) * inv, __uint_as_float(v[2 * e + 1]) * inv);
+                    for (int e = 0; e < 8; ++e) o8[e] = pack_bf2(x[2 * e] * inv, x[2 * e + 1] * inv);
                     orow[2 * c] = make_uint4(o8[0], o8[1], o8[2], o8[3]);
                     orow[2 * c + 1] = make_uint4(o8[4], o8[5], o8[6], o8[7]);
                 } else {
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        __stcg(arow + 4 * c + e, make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                                             __uint_as_float(v[4 * e + 2]),
-                                                             __uint_as_float(v[4 * e + 3])));
+                        __stcg(arow + 4 * c + e, make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]));
                 }
                 __syncwarp();
             }
-            if (active && !whole) __stcg(sc.ml + prow, make_float2(m, lsum));
+            if (active && !whole && h == 0) __stcg(sc.ml + prow, make_float2(M, Lt));
         }
+        ++u;
     } while (ok && w.next(s.seg, B));
 }
 
@@ -621,45 +706,53 @@ template <int G>
 __global__ void __launch_bounds__(kTcThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const Params p,
                    const PrefillScratch sc) {
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    // the tiles start on a 1024-byte boundary (the swizzle atom)
-    uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    extern __shared__ __align__(16) uint8_t smem[];
+    // the tiles start on the first 1024-byte boundary after the small items
+    uint8_t* tiles = smem + kTcSmall + ((1024u - ((smem_addr(smem) + kTcSmall) & 1023u)) & 1023u);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     TcShared s;
-    s.stages = smem;
-    s.q = smem + kTcSmemQ;
-    s.p = smem + kTcSmemP;
+    s.k = tiles;
+    s.v = tiles + kTcTileV;
+    s.q = tiles + kTcTileQ;
+    s.p = tiles + kTcTileP;
     s.seg = reinterpret_cast<int*>(smem + kTcSmemSeg);
-    s.lens = reinterpret_cast<int*>(smem + kTcSmemLens);
     s.mask = reinterpret_cast<volatile int*>(smem + kTcSmemMask);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTcSmemBars);
-    s.kv_full = bars;
-    s.kv_empty = bars + kTcStages;
-    s.s_full = bars + 2 * kTcStages;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+    s.k_full = bars;
+    s.k_empty = s.k_full + kTcKSlots;
+    s.v_full = s.k_empty + kTcKSlots;
+    s.v_empty = s.v_full + kTcVSlots;
+    s.s_full = s.v_empty + kTcVSlots;
     s.p_full = s.s_full + 2;
-    s.pv_done = s.p_full + 1;
-    s.q_full = s.pv_done + 1;
+    s.pv_done = s.p_full + 2;
+    s.q_full = s.pv_done + 2;
     s.q_free = s.q_full + 2;
-    s.fin = s.q_free + 2;
+    s.ml_ready = s.q_free + 2;
+    s.fin = s.ml_ready + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTcSmemTmem);
     s.abort_flag = reinterpret_cast<volatile int*>(smem + kTcSmemTmem + 4);
 
     // The prologue touches no global memory; griddepcontrol.wait then holds
     // until the prep launch has completed and its writes are visible.
     if (threadIdx.x == 0) {
-        for (int k = 0; k < kTcStages; ++k) {
-            mbar_init(&s.kv_full[k], 1);
-            mbar_init(&s.kv_empty[k], 1);
+        for (int k = 0; k < kTcKSlots; ++k) {
+            mbar_init(&s.k_full[k], 1);
+            mbar_init(&s.k_empty[k], 1);
+        }
+        for (int k = 0; k < kTcVSlots; ++k) {
+            mbar_init(&s.v_full[k], 1);
+            mbar_init(&s.v_empty[k], 1);
         }
         mbar_init(&s.s_full[0], 1);
         mbar_init(&s.s_full[1], 1);
-        mbar_init(s.p_full, 4 * 32);
-        mbar_init(s.pv_done, 1);
         for (int k = 0; k < 2; ++k) {
+            mbar_init(&s.p_full[k], 8);     // one arrival per softmax warp
+            mbar_init(&s.pv_done[k], 1);
+            mbar_init(&s.ml_ready[k], 8);
             mbar_init(&s.q_full[k], 1);
             mbar_init(&s.q_free[k], 1);
         }
-        mbar_init(s.fin, 1);
+        mbar_init(s.fin, 2);
         *s.abort_flag = 0;
         s.seg[0] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -674,7 +767,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const bool ok = length_ok(p, L_all);
         if (!ok && blockIdx.x == 0) record_error(p.status, QDA_ERR_BOUNDS);
         const int L = ok ? L_all - p.len_trim : 0;
-        s.lens[b] = L;
         s.seg[b + 1] = ok ? (L + kPage - 1) / kPage : 0;
     }
     tc_fence_before();
@@ -712,11 +804,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int start = (int)blockIdx.x * per_cta;
     const int end = min(start + per_cta, total);
     if (start < end) {
-        if (warp == 0) {
-            tc_producer(p, sc, s, &tm_k, &tm_v, B, start, end, lane);
-        } else if (warp == 1) {
+        if (warp == 0 || warp == 3) {
+            if (warp == 0) tc_producer<false>(p, sc, s, &tm_k, B, start, end, lane);
+            else tc_producer<true>(p, sc, s, &tm_v, B, start, end, lane);
+        } else if (warp == 1 || warp == 2) {
             if (lane == 0) {
-                tc_issuer(p, s, B, start, end, tmem);
+                if (warp == 1) tc_issue_s(p, s, B, start, end, tmem);
+                else tc_issue_pv(p, s, B, start, end, tmem);
                 // nothing may still write tensor memory when it is freed
                 (void)mbar_wait(s.fin, 0u, p.timeout_ns, nullptr);
             }
@@ -828,8 +922,8 @@ cudaError_t launch_prefill_g(const Params& p, const PrefillScratch& sc, cudaStre
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cfg.gridDim = dim3((unsigned)p.batch, (unsigned)kNumKvHeads, (unsigned)((p.new_tokens + 3) / 4));
-    cfg.blockDim = dim3(128, 1, 1);
+    cfg.gridDim = dim3((unsigned)p.batch, (unsigned)kNumKvHeads, (unsigned)((p.new_tokens + 7) / 8));
+    cfg.blockDim = dim3(256, 1, 1);
     cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_prep_kernel<G>, p, sc);
     if (e != cudaSuccess) return e;
     cfg.gridDim = dim3((unsigned)sc.grid, 1, 1);
