@@ -22,6 +22,7 @@ struct qda_handle {
     // the chunked prefill: query tiles [max_batch][8], partials (2 slots per
     // CTA of its attention launch)
     uint16_t* pf_q = nullptr;
+    int2* pf_unit = nullptr;
     float* pf_acc = nullptr;
     float2* pf_ml = nullptr;
     int pf_grid = 0;
@@ -75,6 +76,7 @@ void free_workspace(qda_handle* h) {
     cudaFree(h->counters);
     cudaFree(h->seg);
     cudaFree(h->pf_q);
+    cudaFree(h->pf_unit);
     cudaFree(h->pf_acc);
     cudaFree(h->pf_ml);
     cudaFree(h->status);
@@ -260,6 +262,7 @@ int qwen3_decode_attn_create(const qda_config* cfg, int device, qda_handle** out
               alloc(&h->counters, (size_t)qda::kMaxBatch * qda::kNumKvHeads * sizeof(int)) &&
               alloc(&h->status, sizeof(int)) && alloc(&h->seg, (size_t)(qda::kMaxBatch + 1) * sizeof(int)) &&
               alloc(&h->pf_q, qda::prefill_q_bytes(cfg->max_batch)) &&
+              alloc(&h->pf_unit, qda::prefill_unit_bytes(cfg->max_batch)) &&
               alloc(&h->pf_acc, qda::prefill_acc_bytes(sms)) && alloc(&h->pf_ml, qda::prefill_ml_bytes(sms)) &&
               alloc(&h->xg_hi, B * (size_t)qda::kMaxHidden * sizeof(uint16_t)) &&
               alloc(&h->xg_lo, B * (size_t)qda::kMaxHidden * sizeof(uint16_t)) &&
@@ -270,6 +273,7 @@ int qwen3_decode_attn_create(const qda_config* cfg, int device, qda_handle** out
              alloc(&h->st_block_table[k], B * (size_t)cfg->max_pages_per_seq * sizeof(int32_t)) &&
              alloc(&h->st_o[k], B * Hq * qda::kHeadDim * sizeof(uint16_t));
     ok = ok && cudaMemset(h->counters, 0, (size_t)qda::kMaxBatch * qda::kNumKvHeads * sizeof(int)) == cudaSuccess &&
+         cudaMemset(h->pf_unit, 0, qda::prefill_unit_bytes(cfg->max_batch)) == cudaSuccess &&
          cudaMemset(h->status, 0, sizeof(int)) == cudaSuccess && cudaDeviceSynchronize() == cudaSuccess;
     if (!ok) {
         free_workspace(h);
@@ -324,7 +328,7 @@ int qwen3_decode_attn_append_and_attend_tokens(qda_handle* h, const void* qkv, c
     // the cache plus the block's tokens up to its own (its launches trim the
     // later ones from seq_lens), so each token still attends over exactly the
     // slots up to its own.
-    const qda::PrefillScratch sc{h->pf_q, h->pf_acc, h->pf_ml, h->pf_grid};
+    const qda::PrefillScratch sc{h->pf_q, h->pf_acc, h->pf_ml, h->pf_unit, h->pf_grid};
     const int max_t = qda::prefill_max_tokens(h->cfg.num_q_heads);
     for (int c0 = 0; c0 < new_tokens;) {
         const int n = new_tokens - c0 < max_t ? new_tokens - c0 : max_t;

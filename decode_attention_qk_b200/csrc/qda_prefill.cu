@@ -206,7 +206,7 @@ constexpr int kTcPages = kTcKeys / kPage;            // 4
 // S, the softmax and the product, so the V ring is the deeper one: with about
 // three stages held in processing it still keeps two or more in flight.
 constexpr int kTcKSlots = 4;
-constexpr int kTcVSlots = 5;
+constexpr int kTcVSlots = 6;
 constexpr int kTcThreads = 12 * 32;
 constexpr int kTcHalf = kTcKeys * 128;               // 64 dims of a stage's rows: 8 KiB
 constexpr int kTcSlotBytes = 2 * kTcHalf;            // a K or V slot: dims 0-63 | dims 64-127
@@ -222,15 +222,15 @@ constexpr int kTcSmemMask = kTcSmemTmem + 16;                        // int [kTc
 constexpr int kTcSmemSeg = kTcSmemMask + kTcVSlots * 4;              // int [kMaxBatch + 4]
 constexpr int kTcSmall = (kTcSmemSeg + (kMaxBatch + 4) * 4 + 15) / 16 * 16;
 constexpr int kTcTileV = kTcKSlots * kTcSlotBytes;   // from the tiles' start: K ring, V ring,
-constexpr int kTcTileQ = kTcTileV + kTcVSlots * kTcSlotBytes;   // 2 buffers of Q dims 0-63 | 64-127,
-constexpr int kTcTileP = kTcTileQ + 4 * kTcTile;                // P: 128 rows x 64 keys
-constexpr int kTcTiles = kTcTileP + kTcTile;
+constexpr int kTcTileQ = kTcTileV + kTcVSlots * kTcSlotBytes;   // 2 buffers of Q dims 0-63 | 64-127
+constexpr int kTcTiles = kTcTileQ + 4 * kTcTile;
 constexpr int kTcSmemAlloc = kTcSmall + 1024 + kTcTiles;   // with up to 1023 bytes of padding
 // tensor-memory columns: S buffers at 0 and 64, O_0 at 128, O_1 at 256, the
-// (m, l) swap at 384
+// (m, l) swap at 384, P buffers (64 bf16 keys in 32 columns) at 416 and 448
 constexpr uint32_t kTcTmemCols = 512;
 constexpr uint32_t kTcTmemO = 128;
 constexpr uint32_t kTcTmemMl = 384;
+constexpr uint32_t kTcTmemP = 416;
 static_assert(kTcSlotBytes % 1024 == 0 && kTcTile % 1024 == 0, "swizzle atoms are 1024-byte aligned");
 static_assert(kTcSmall % 16 == 0 && 2 * kTcTile == kPrefillQTileBytes, "layout");
 static_assert(kTcSmemAlloc <= 227 * 1024, "fits one CTA per SM");
@@ -240,7 +240,6 @@ struct TcShared {
     uint8_t* k;          // K ring
     uint8_t* v;          // V ring
     uint8_t* q;
-    uint8_t* p;
     int* seg;
     volatile int* mask;  // [kTcVSlots]: pages of the stage in V slot i that were not copied
     uint64_t* k_full;
@@ -248,7 +247,7 @@ struct TcShared {
     uint64_t* v_full;
     uint64_t* v_empty;
     uint64_t* s_full;    // [2]: S of stage g in S buffer g % 2
-    uint64_t* p_full;    // [2]: P written for stage g (g % 2)
+    uint64_t* p_full;    // [2]: P of stage g written into P buffer g % 2
     uint64_t* pv_done;   // [2]: O += P V of stage g (g % 2) completed
     uint64_t* q_full;    // [2]
     uint64_t* q_free;    // [2]
@@ -285,6 +284,34 @@ struct PieceWalk {
         return true;
     }
 };
+
+// The split of the page-head list over the CTAs. Besides its pages, every
+// unit (b, j) costs kPieceCost page equivalents of fixed work where a CTA
+// holds a piece of it (the pipeline's drain, the merge of the halves, the
+// output; measured at about six pages' worth). CTA g takes page-heads
+// [pf_split(g), pf_split(g + 1)): the points where the running cost, units in
+// order with each unit's fixed cost before its pages, crosses g * w, w the
+// total over the grid. seg is the page prefix of the sequences.
+constexpr int kPieceCost = 6;
+
+__device__ __forceinline__ int pf_cost_before(const int* seg, int b) { return 8 * (seg[b] + kPieceCost * b); }
+
+__device__ __forceinline__ int pf_split(const int* seg, int B, int grid, int g) {
+    const int W = pf_cost_before(seg, B);
+    const int w = (W + grid - 1) / grid;
+    const long long t = (long long)g * w;
+    if (t >= W) return 8 * seg[B];
+    int lo = 0, hi = B - 1;   // the sequence whose cost range holds t
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pf_cost_before(seg, mid) <= t) lo = mid; else hi = mid - 1;
+    }
+    const int np = seg[lo + 1] - seg[lo];
+    const int r = (int)t - pf_cost_before(seg, lo);          // < 8 * (np + kPieceCost)
+    const int j = min(kNumKvHeads - 1, r / (np + kPieceCost));
+    const int off = r - j * (np + kPieceCost) - kPieceCost;   // pages into unit (lo, j); < np
+    return 8 * seg[lo] + j * np + max(0, off);
+}
 
 // One thread's bounded wait; a failure aborts the CTA.
 __device__ __forceinline__ bool tc_wait1(const Params& p, const TcShared& s, uint64_t* bar, uint32_t parity) {
@@ -357,6 +384,12 @@ __device__ __forceinline__ void tc_producer(const Params& p, const PrefillScratc
         }
         const int np_b = s.seg[w.b + 1] - s.seg[w.b];
         const int x_piece = 8 * s.seg[w.b] + w.j * np_b + w.i0;
+        if (!kIsV && lane == 0) {
+            // for the combine launch: the slot of the unit's first piece, the CTA of its last
+            int2* unit = sc.unit + w.b * kNumKvHeads + w.j;
+            if (w.i0 == 0) unit->x = 2 * (int)blockIdx.x + (w.k == 0 ? 0 : 1);
+            if (w.i0 + w.n == np_b) unit->y = (int)blockIdx.x;
+        }
         for (int q = 0; q < w.n; q += kTcPages, ++g) {
             const int npg = min(kTcPages, w.n - q);
             const int x0 = x_piece + q;
@@ -457,13 +490,14 @@ __device__ __forceinline__ void tc_issue_s(const Params& p, const TcShared& s, i
 }
 
 // Lane 0 of warp 2: per stage x, once both softmax warpgroups have written
-// P_x, O_0 += P_x[:, 0:32] V_x[0:32] and O_1 += P_x[:, 32:64] V_x[32:64], each
-// accumulator starting afresh at its piece's first stage; the V slot (and the
-// P tile) are free once these complete.
+// P_x into tensor-memory P buffer x % 2, O_0 += P_x[:, 0:32] V_x[0:32] and
+// O_1 += P_x[:, 32:64] V_x[32:64], each accumulator starting afresh at its
+// piece's first stage; the V slot and the P buffer are free once these
+// complete.
 __device__ __forceinline__ void tc_issue_pv(const Params& p, const TcShared& s, int B, int start, int end,
                                             uint32_t tmem) {
     const uint32_t idesc_o = umma_idesc_bf16_m128_bmn(kHeadDim);
-    const uint32_t pb = smem_addr(s.p), v_base = smem_addr(s.v);
+    const uint32_t v_base = smem_addr(s.v);
     uint32_t x = 0;
     bool ok = true;
     PieceWalk w;
@@ -476,11 +510,12 @@ __device__ __forceinline__ void tc_issue_pv(const Params& p, const TcShared& s, 
             }
             tc_fence_after();
             const uint32_t v = v_base + (x % kTcVSlots) * kTcSlotBytes;
+            const uint32_t pa = tmem + kTcTmemP + (x & 1u) * (kTcKeys / 2);
 #pragma unroll
-            for (int kk = 0; kk < kTcKeys / 16; ++kk)   // 16 keys per instruction; keys 32h.. go to O_h
-                umma_bf16(tmem + kTcTmemO + (kk >> 1) * kHeadDim, umma_desc_sw128(pb + 32 * kk),
-                          umma_desc_sw128_mn(v + 2 * 1024 * kk, kTcHalf, 1024), idesc_o,
-                          (q == 0 && (kk & 1) == 0) ? 0u : 1u);
+            for (int kk = 0; kk < kTcKeys / 16; ++kk)   // 16 keys (8 columns) per instruction; keys 32h.. go to O_h
+                umma_bf16_ts(tmem + kTcTmemO + (kk >> 1) * kHeadDim, pa + 8 * kk,
+                             umma_desc_sw128_mn(v + 2 * 1024 * kk, kTcHalf, 1024), idesc_o,
+                             (q == 0 && (kk & 1) == 0) ? 0u : 1u);
             umma_commit(&s.pv_done[x & 1u]);
             umma_commit(&s.v_empty[x % kTcVSlots]);
         }
@@ -498,7 +533,7 @@ __device__ __forceinline__ void tc_issue_pv(const Params& p, const TcShared& s, 
 // through tensor memory.
 template <int G>
 __device__ __forceinline__ void tc_softmax(const Params& p, const PrefillScratch& sc, const TcShared& s, int B,
-                                           int start, int end, int per_cta, int t, uint32_t tmem) {
+                                           int start, int end, int t, uint32_t tmem) {
     constexpr int kHq = G * kNumKvHeads;
     const int r = t & 127, h = t >> 7, lane = t & 31;
     const int n = p.new_tokens, R = n * G;
@@ -507,7 +542,6 @@ __device__ __forceinline__ void tc_softmax(const Params& p, const PrefillScratch
     const int tt = active ? r / G : 0;
     const uint32_t lanes = tmem + ((uint32_t)(r & ~31) << 16);
     const uint32_t o_own = lanes + kTcTmemO + (uint32_t)h * kHeadDim;
-    const uint32_t p_row = smem_addr(s.p) + r * 128;
     uint32_t g = 0, u = 0, pv_seen[2] = {0u, 0u};
     bool ok = true;
     // O += P_x V_x has completed: completion x / 2 of pv_done[x % 2]. The
@@ -546,6 +580,7 @@ __device__ __forceinline__ void tc_softmax(const Params& p, const PrefillScratch
                     const uint32_t row = smem_addr(s.v + st * kTcSlotBytes + (r >> 6) * kTcHalf) + kr * 128;
 #pragma unroll
                     for (int c = 0; c < 8; ++c) st_shared_v4(row + 16 * c, 0u, 0u, 0u, 0u);
+                    fence_async_shared();   // visible to the tensor cores' proxy before the arrival below
                 }
             }
             uint32_t pw[8];
@@ -612,30 +647,27 @@ __device__ __forceinline__ void tc_softmax(const Params& p, const PrefillScratch
                     pw2[c] = pack_bf2(exp2_approx(sv[16 + 2 * c] - mb), exp2_approx(sv[17 + 2 * c] - mb));
                     lsum += bf_lo(pw2[c]) + bf_hi(pw2[c]);
                 }
-                // the product of stage g - 1 has read the P tile
-                if (g > 0 && !pv_wait(g - 1)) {
+                // the product of stage g - 2 has read P buffer g % 2
+                if (g > 1 && !pv_wait(g - 2)) {
                     ok = false;
                     break;
                 }
-                const uint32_t pr = p_row;
+                uint32_t pcol[16];
 #pragma unroll
-                for (int c = 0; c < 2; ++c)
-                    st_shared_v4(pr + (((4 * h + c) ^ (r & 7)) << 4), pw[4 * c], pw[4 * c + 1], pw[4 * c + 2],
-                                 pw[4 * c + 3]);
-#pragma unroll
-                for (int c = 0; c < 2; ++c)
-                    st_shared_v4(pr + (((4 * h + 2 + c) ^ (r & 7)) << 4), pw2[4 * c], pw2[4 * c + 1], pw2[4 * c + 2],
-                                 pw2[4 * c + 3]);
-            } else if (g > 0 && !pv_wait(g - 1)) {
+                for (int c = 0; c < 8; ++c) {
+                    pcol[c] = pw[c];
+                    pcol[8 + c] = pw2[c];
+                }
+                tmem_st16(lanes + kTcTmemP + (g & 1u) * (kTcKeys / 2) + 16 * h, pcol);
+                tmem_st_wait();
+            } else if (g > 1 && !pv_wait(g - 2)) {
                 // every warp waits before arriving: p_full[g % 2] counts
                 // arrivals, and none may arrive for stage g + 2 before stage
                 // g's phase is over
                 ok = false;
                 break;
             }
-            // one arrival per warp, once every lane's P stores (and V zeroing)
-            // are visible to the tensor cores' proxy
-            fence_async_shared();
+            // one arrival per warp, once every lane's P (and V zeroing) is in place
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.p_full[g & 1u]);
@@ -666,8 +698,7 @@ __device__ __forceinline__ void tc_softmax(const Params& p, const PrefillScratch
             const float a0 = m0 == -INFINITY ? 0.f : exp2_approx(m0 - M);
             const float a1 = m1 == -INFINITY ? 0.f : exp2_approx(m1 - M);
             const float Lt = a0 * l0 + a1 * l1;
-            const int ustart = 8 * s.seg[w.b] + w.j * np_b;
-            const bool whole = ustart / per_cta == (ustart + np_b - 1) / per_cta;
+            const bool whole = w.i0 == 0 && w.n == np_b;   // this CTA holds the whole unit
             const int pslot = 2 * (int)blockIdx.x + (w.k == 0 ? 0 : 1);   // the CTA's first piece, else its last
             const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
             uint4* orow = reinterpret_cast<uint4*>(p.o + (pf_token_row(p, w.b, tt) * kHq + G * w.j + r % G) * kHeadDim);
@@ -714,7 +745,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     s.k = tiles;
     s.v = tiles + kTcTileV;
     s.q = tiles + kTcTileQ;
-    s.p = tiles + kTcTileP;
     s.seg = reinterpret_cast<int*>(smem + kTcSmemSeg);
     s.mask = reinterpret_cast<volatile int*>(smem + kTcSmemMask);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
@@ -800,9 +830,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int b = threadIdx.x; b <= B; b += kTcThreads) p.seg[b] = s.seg[b];
 
     const int total = kNumKvHeads * s.seg[B];   // page-heads
-    const int per_cta = (total + (int)gridDim.x - 1) / (int)gridDim.x;
-    const int start = (int)blockIdx.x * per_cta;
-    const int end = min(start + per_cta, total);
+    const int start = pf_split(s.seg, B, (int)gridDim.x, (int)blockIdx.x);
+    const int end = min(pf_split(s.seg, B, (int)gridDim.x, (int)blockIdx.x + 1), total);
     if (start < end) {
         if (warp == 0 || warp == 3) {
             if (warp == 0) tc_producer<false>(p, sc, s, &tm_k, B, start, end, lane);
@@ -815,7 +844,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 (void)mbar_wait(s.fin, 0u, p.timeout_ns, nullptr);
             }
         } else if (warp >= 4) {
-            tc_softmax<G>(p, sc, s, B, start, end, per_cta, threadIdx.x - 128, tmem);
+            tc_softmax<G>(p, sc, s, B, start, end, threadIdx.x - 128, tmem);
         }
     }
     __syncwarp();
@@ -831,9 +860,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // ---------------------------------------------------------------------------
 // 3. The combine: warp w of CTA (b, j, z) merges row 8z + w of unit (b, j)
 // when the unit was split across CTAs; lane l holds dims 4l..4l+3. The unit's
-// pieces sit in consecutive CTAs g0..gk of the attention launch: slot 2*g0 + 1
-// when the unit starts inside g0's range (it is g0's last piece), else 2*g0;
-// slot 2*g in the later CTAs.
+// pieces sit in consecutive CTAs g0..gk of the attention launch, which
+// recorded the slot of the first (2*g0 + 1 when the unit starts inside g0's
+// range, as g0's last piece; else 2*g0) and gk; the later pieces are in slots
+// 2*g.
 template <int G>
 __global__ void __launch_bounds__(256) prefill_combine_kernel(const Params p, const PrefillScratch sc) {
     constexpr int kHq = G * kNumKvHeads;
@@ -842,14 +872,11 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(const Params p, co
     const int b = blockIdx.x, j = blockIdx.y, lane = threadIdx.x & 31;
     const int r = 8 * (int)blockIdx.z + (int)(threadIdx.x >> 5);
     if (r >= p.new_tokens * G) return;
-    const int np = p.seg[b + 1] - p.seg[b];
-    if (np == 0) return;   // a sequence the attention launch skipped
-    const int total = kNumKvHeads * p.seg[p.batch];
-    const int per_cta = (total + sc.grid - 1) / sc.grid;
-    const int ustart = kNumKvHeads * p.seg[b] + j * np;
-    const int g0 = ustart / per_cta, gk = (ustart + np - 1) / per_cta;
+    if (p.seg[b + 1] == p.seg[b]) return;   // a sequence the attention launch skipped
+    const int2 info = sc.unit[b * kNumKvHeads + j];
+    const int first = info.x, g0 = info.x >> 1, gk = info.y;
     if (g0 == gk) return;   // held whole by one CTA, which wrote o
-    const int first = ustart % per_cta != 0 ? 2 * g0 + 1 : 2 * g0;   // slot of piece 0; piece k > 0: 2 * (g0 + k)
+    if (g0 < 0 || gk < g0 || gk >= sc.grid) return;   // not recorded (an attention launch that gave up)
     const int pieces = gk - g0 + 1;
     float M = -INFINITY;
     for (int k = lane; k < pieces; k += 32) {

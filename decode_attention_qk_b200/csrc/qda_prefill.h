@@ -26,9 +26,11 @@ struct PrefillScratch {
     uint16_t* q;    // [max_batch][8][kPrefillQTileBytes / 2]
     float* acc;     // [2 * grid][kPrefillRows][128]
     float2* ml;     // [2 * grid][kPrefillRows]
+    int2* unit;     // [max_batch][8]: per unit, the slot of its first piece and the CTA of its last
     int grid;       // CTAs of the attention launch
 };
 inline size_t prefill_q_bytes(int max_batch) { return (size_t)max_batch * kNumKvHeads * kPrefillQTileBytes; }
+inline size_t prefill_unit_bytes(int max_batch) { return (size_t)max_batch * kNumKvHeads * sizeof(int2); }
 inline size_t prefill_acc_bytes(int grid) { return (size_t)2 * grid * kPrefillRows * kHeadDim * sizeof(float); }
 inline size_t prefill_ml_bytes(int grid) { return (size_t)2 * grid * kPrefillRows * sizeof(float2); }
 

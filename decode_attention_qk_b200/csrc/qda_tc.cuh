@@ -63,6 +63,19 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t 
         : "memory");
 }
 
+// The same with A (M x 16, K-major) in tensor memory at a_tmem: row i in lane
+// i, two consecutive bf16 elements per 32-bit column (the lower-numbered one in
+// the low half), 8 columns per instruction.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // The mbarrier receives one arrival once every tensor-core instruction this
 // thread issued before has completed (and has read its shared operands).
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
