@@ -288,11 +288,11 @@ struct PieceWalk {
 // The split of the page-head list over the CTAs. Besides its pages, every
 // unit (b, j) costs kPieceCost page equivalents of fixed work where a CTA
 // holds a piece of it (the pipeline's drain, the merge of the halves, the
-// output; measured at about six pages' worth). CTA g takes page-heads
-// [pf_split(g), pf_split(g + 1)): the points where the running cost, units in
-// order with each unit's fixed cost before its pages, crosses g * w, w the
-// total over the grid. seg is the page prefix of the sequences.
-constexpr int kPieceCost = 6;
+// output; 12 was the best of the settings measured, 3 to 24). CTA g takes
+// page-heads [pf_split(g), pf_split(g + 1)): the points where the running
+// cost, units in order with each unit's fixed cost before its pages, crosses
+// g * w, w the total over the grid. seg is the page prefix of the sequences.
+constexpr int kPieceCost = 12;
 
 __device__ __forceinline__ int pf_cost_before(const int* seg, int b) { return 8 * (seg[b] + kPieceCost * b); }
 
