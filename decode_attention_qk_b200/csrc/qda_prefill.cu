@@ -110,19 +110,29 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(const Params p, const
     const double pos = (double)(pf_first_position(p, b, L, n) + u);
     const double ang0 = reduce_angle(pos * inv_freq[2 * lane]);
     const double ang1 = reduce_angle(pos * inv_freq[2 * lane + 1]);
+    // every load first (the token's k, v and G query rows, the gains, the
+    // page), so that their latencies overlap
     const uint32_t* row = reinterpret_cast<const uint32_t*>(p.qkv + pf_token_row(p, b, u) * kQkvW);
-
+    const uint32_t* xk = row + (kHq + j) * (kHeadDim / 2);
+    const uint32_t* xv = row + (kHq + kNumKvHeads + j) * (kHeadDim / 2);
+    const uint32_t klo = xk[lane], khi = xk[32 + lane];
+    const uint32_t vlo = xv[lane], vhi = xv[32 + lane];
+    uint32_t qlo[G], qhi[G];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+        qlo[hh] = row[(G * j + hh) * (kHeadDim / 2) + lane];
+        qhi[hh] = row[(G * j + hh) * (kHeadDim / 2) + 32 + lane];
+    }
+    const uint32_t* gk = reinterpret_cast<const uint32_t*>(p.k_norm_w);
+    const uint32_t wk_lo = gk[lane], wk_hi = gk[32 + lane];
+    const uint32_t* gq = reinterpret_cast<const uint32_t*>(p.q_norm_w);
+    const uint32_t wq_lo = gq[lane], wq_hi = gq[32 + lane];
     const int slot = L - n + u;
     const int page = __ldg(p.block_table + (size_t)b * p.bt_stride + slot / kPage);
-    if (page >= 0 && page < p.num_pages) {   // else recorded by the attention launch
-        const uint32_t* gk = reinterpret_cast<const uint32_t*>(p.k_norm_w);
-        const uint32_t wk_lo = gk[lane], wk_hi = gk[32 + lane];
-        const uint32_t* xk = row + (kHq + j) * (kHeadDim / 2);
-        const uint32_t* xv = row + (kHq + kNumKvHeads + j) * (kHeadDim / 2);
-        const uint32_t xlo = xk[lane], xhi = xk[32 + lane];
-        const uint32_t vlo = xv[lane], vhi = xv[32 + lane];
-        double a0 = bf_to_d(xlo & 0xFFFFu), a1 = bf_to_d(xlo >> 16);
-        double b0 = bf_to_d(xhi & 0xFFFFu), b1 = bf_to_d(xhi >> 16);
+
+    {
+        double a0 = bf_to_d(klo & 0xFFFFu), a1 = bf_to_d(klo >> 16);
+        double b0 = bf_to_d(khi & 0xFFFFu), b1 = bf_to_d(khi >> 16);
         const double inv_rr = 1.0 / sqrt(warp_sum(a0 * a0 + a1 * a1 + b0 * b0 + b1 * b1) / 128.0 + p.rms_eps);
         a0 = a0 * inv_rr * bf_to_d(wk_lo & 0xFFFFu);
         a1 = a1 * inv_rr * bf_to_d(wk_lo >> 16);
@@ -133,28 +143,27 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(const Params p, const
         sincos(ang1, &sn1, &cs1);
         const double ra0 = a0 * cs0 - b0 * sn0, rb0 = b0 * cs0 + a0 * sn0;
         const double ra1 = a1 * cs1 - b1 * sn1, rb1 = b1 * cs1 + a1 * sn1;
-        const size_t off =
-            (size_t)page * (kPageBytes / 2) + (size_t)(slot % kPage) * (kRowBytes / 2) + (size_t)j * kHeadDim;
-        uint32_t* kd = reinterpret_cast<uint32_t*>(p.k_cache + off);
-        uint32_t* vd = reinterpret_cast<uint32_t*>(p.v_cache + off);
-        kd[lane] = d_to_bf(ra0) | (d_to_bf(ra1) << 16);
-        kd[32 + lane] = d_to_bf(rb0) | (d_to_bf(rb1) << 16);
-        vd[lane] = vlo;
-        vd[32 + lane] = vhi;
+        if (page >= 0 && page < p.num_pages) {   // else recorded by the attention launch
+            const size_t off =
+                (size_t)page * (kPageBytes / 2) + (size_t)(slot % kPage) * (kRowBytes / 2) + (size_t)j * kHeadDim;
+            uint32_t* kd = reinterpret_cast<uint32_t*>(p.k_cache + off);
+            uint32_t* vd = reinterpret_cast<uint32_t*>(p.v_cache + off);
+            kd[lane] = d_to_bf(ra0) | (d_to_bf(ra1) << 16);
+            kd[32 + lane] = d_to_bf(rb0) | (d_to_bf(rb1) << 16);
+            vd[lane] = vlo;
+            vd[32 + lane] = vhi;
+        }
     }
 
     float sn0, cs0, sn1, cs1;
     sincosf((float)ang0, &sn0, &cs0);
     sincosf((float)ang1, &sn1, &cs1);
-    const uint32_t* gq = reinterpret_cast<const uint32_t*>(p.q_norm_w);
-    const uint32_t wq_lo = gq[lane], wq_hi = gq[32 + lane];
     const float scale = (float)kQScale;
     uint8_t* tile = reinterpret_cast<uint8_t*>(sc.q) + (size_t)(b * kNumKvHeads + j) * kPrefillQTileBytes;
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) {
         const int r = u * G + hh;
-        const uint32_t* xq = row + (G * j + hh) * (kHeadDim / 2);
-        const uint32_t xlo = xq[lane], xhi = xq[32 + lane];
+        const uint32_t xlo = qlo[hh], xhi = qhi[hh];
         float ss = bf_lo(xlo) * bf_lo(xlo) + bf_hi(xlo) * bf_hi(xlo) + bf_lo(xhi) * bf_lo(xhi) + bf_hi(xhi) * bf_hi(xhi);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(kFull, ss, o);
