@@ -224,8 +224,8 @@ constexpr int kTcTile = kPrefillRows * 128;          // 64 columns of a 128-row 
 // Shared memory: the small items first, then the tiles on the next 1024-byte
 // boundary (the swizzle atom).
 // k_full[K], k_empty[K], v_full[V], v_empty[V], s_full[2], p_full[2],
-// pv_done[2], q_full[2], q_free[2], ml_ready[2], fin
-constexpr int kTcNumBars = 2 * kTcKSlots + 2 * kTcVSlots + 13;
+// pv_done[2], q_full[2], q_free[2], ml_ready[2], fin, never (the test hook's)
+constexpr int kTcNumBars = 2 * kTcKSlots + 2 * kTcVSlots + 14;
 constexpr int kTcSmemTmem = kTcNumBars * 8;                          // tensor-memory address, abort flag
 constexpr int kTcSmemMask = kTcSmemTmem + 16;                        // int [kTcVSlots]: pages not copied
 constexpr int kTcSmemSeg = kTcSmemMask + kTcVSlots * 4;              // int [kMaxBatch + 4]
@@ -262,6 +262,7 @@ struct TcShared {
     uint64_t* q_free;    // [2]
     uint64_t* ml_ready;  // [2]: both warpgroups have posted (m, l) of piece u (u % 2)
     uint64_t* fin;
+    uint64_t* never;
     volatile int* abort_flag;
 };
 
@@ -768,6 +769,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     s.q_free = s.q_full + 2;
     s.ml_ready = s.q_free + 2;
     s.fin = s.ml_ready + 2;
+    s.never = s.fin + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTcSmemTmem);
     s.abort_flag = reinterpret_cast<volatile int*>(smem + kTcSmemTmem + 4);
 
@@ -792,6 +794,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(&s.q_free[k], 1);
         }
         mbar_init(s.fin, 2);
+        mbar_init(s.never, 1);
         *s.abort_flag = 0;
         s.seg[0] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -855,6 +858,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         } else if (warp >= 4) {
             tc_softmax<G>(p, sc, s, B, start, end, threadIdx.x - 128, tmem);
         }
+    }
+    if ((p.flags & QDA_FLAG_INJECT_WAIT_TIMEOUT) != 0u && blockIdx.x == 0 && warp == 0) {
+        // test hook: a barrier nothing arrives at; the wait must end by itself
+        if (!mbar_wait(s.never, 0u, p.timeout_ns, nullptr) && lane == 0) record_error(p.status, QDA_ERR_TIMEOUT);
     }
     __syncwarp();
     tc_fence_before();

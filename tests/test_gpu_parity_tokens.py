@@ -255,6 +255,22 @@ def test_prefill_out_of_range_page_ids_are_not_dereferenced(handles, hq, T):
     assert attn.check() == 0
 
 
+def test_prefill_wait_timeout_is_reported_and_the_handle_recovers():
+    """The prefill's bounded waits: a wait on a barrier nothing completes ends
+    after the configured limit with QDA_ERR_TIMEOUT, the call's result is still
+    right, and a new handle works."""
+    a = binding.DecodeAttention(device=0, flags=binding.QDA_FLAG_INJECT_WAIT_TIMEOUT, wait_timeout_ns=2_000_000)
+    w = inputs.custom([100, 40, 300], seed=74, device="cuda", new_tokens=20)
+    k, v = w.k_cache.clone(), w.v_cache.clone()
+    o = ph.run(a, w, DEV, k, v)
+    assert a.check() == binding.QDA_ERR_TIMEOUT
+    sampled_check(o, w, [0, 1, 2], w.k_cache, w.v_cache, "prefill timeout injection")
+    a.close()
+    b = binding.DecodeAttention(device=0)
+    full_check(b, inputs.custom([100, 40, 300], seed=74, device="cuda", new_tokens=20), "prefill after timeout")
+    b.close()
+
+
 def test_host_side_errors(handles):
     w = inputs.custom([20, 30], seed=69, device="cuda", new_tokens=2)
     a = ph.device_args(w, DEV)
