@@ -16,7 +16,8 @@
 //      already in the tensor cores' swizzled layout).
 //   2. prefill_kernel: the units (sequence b, kv head j) in order, each the
 //      pages of sequence b for kv head j, form one list of page-heads; CTA g
-//      takes an equal range of it (whatever the length mix). Per unit piece
+//      takes a range of it of equal cost (pages plus a fixed cost per unit
+//      piece), whatever the length mix. Per unit piece
 //      the query tile is one 128-row operand of the 5th-generation tensor
 //      cores: S = Q K^T and O += P V with accumulators in tensor memory, the
 //      K and V tiles copied by the tensor memory accelerator (a 3-D tensor map
@@ -164,7 +165,8 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(const Params p, const
     for (int hh = 0; hh < G; ++hh) {
         const int r = u * G + hh;
         const uint32_t xlo = qlo[hh], xhi = qhi[hh];
-        float ss = bf_lo(xlo) * bf_lo(xlo) + bf_hi(xlo) * bf_hi(xlo) + bf_lo(xhi) * bf_lo(xhi) + bf_hi(xhi) * bf_hi(xhi);
+        float ss =
+            bf_lo(xlo) * bf_lo(xlo) + bf_hi(xlo) * bf_hi(xlo) + bf_lo(xhi) * bf_lo(xhi) + bf_hi(xhi) * bf_hi(xhi);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(kFull, ss, o);
         const float inv_r = rsqrtf(ss * (1.f / 128.f) + (float)p.rms_eps);
@@ -191,22 +193,23 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(const Params p, const
 //   S = Q K^T     tcgen05.mma, M = 128 rows, N = 64 keys, K = 128 dims, into
 //                 one of two S buffers in tensor memory (S of the next stage
 //                 forms while this stage's softmax runs);
-//   softmax       one thread per row: the causal and length mask, the running
-//                 max with lazy rescaling of O, P = exp2(S - m) rounded to bf16
-//                 into shared memory (the running sum adds the same rounded
+//   softmax       one thread per row and half of the stage's keys (two
+//                 warpgroups): the causal and length mask, the running max
+//                 with lazy rescaling of O, P = exp2(S - m) rounded to bf16
+//                 into tensor memory (the running sum adds the same rounded
 //                 values, so o stays a convex combination of v rows);
-//   O += P V      M = 128 rows, N = 128 dims, K = 64 keys, V read MN-major
-//                 from its copied tile;
+//   O += P V      M = 128 rows, N = 128 dims, K = 64 keys, P read from
+//                 tensor memory and V MN-major from its copied tile;
 // and O, accumulated in tensor memory over the piece, is read out once at the
 // piece's end.
 //
 // Warp roles (384 threads): warps 0 and 3 issue the copies of K (and Q) and
-// of V; one thread of warp 1 issues S and one of warp 2 issues O += P V (warp 1
-// also allocates tensor memory); warps 4-11 run the softmax in two warpgroups, each over half of a
-// stage's keys with an accumulator of its own, and write o. Every wait is
-// bounded: a timeout records QDA_ERR_TIMEOUT, sets the CTA's abort flag and
-// every role leaves its loop; tensor memory is freed after every issued
-// instruction has completed.
+// of V; one thread of warp 1 issues S and one of warp 2 issues O += P V (warp
+// 1 also allocates tensor memory); warps 4-11 run the softmax in two
+// warpgroups, each over half of a stage's keys with an accumulator of its
+// own, and write o. Every wait is bounded: a timeout records QDA_ERR_TIMEOUT,
+// sets the CTA's abort flag and every role leaves its loop; tensor memory is
+// freed after every issued instruction has completed.
 
 constexpr int kTcKeys = 64;                          // cache rows per stage
 constexpr int kTcPages = kTcKeys / kPage;            // 4
