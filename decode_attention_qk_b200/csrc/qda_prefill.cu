@@ -649,17 +649,19 @@ __device__ __forceinline__ void tc_softmax(const Params& p, const PrefillScratch
                 }
                 if (grow) m = mx;
                 const float mb = m == -INFINITY ? 0.f : m;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    pw[c] = pack_bf2(exp2_approx(sv[2 * c] - mb), exp2_approx(sv[2 * c + 1] - mb));
-                    lsum += bf_lo(pw[c]) + bf_hi(pw[c]);
-                }
+                const f32x2 nmb = pack2(-mb, -mb);
+                f32x2 ls2 = pack2(0.f, 0.f);   // even and odd keys' sums, one packed add per pair
                 uint32_t pw2[8];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    pw2[c] = pack_bf2(exp2_approx(sv[16 + 2 * c] - mb), exp2_approx(sv[17 + 2 * c] - mb));
-                    lsum += bf_lo(pw2[c]) + bf_hi(pw2[c]);
+                for (int c = 0; c < 16; ++c) {
+                    const float2 d = unpack2(add2(pack2(sv[2 * c], sv[2 * c + 1]), nmb));
+                    const uint32_t wv = pack_bf2(exp2_approx(d.x), exp2_approx(d.y));
+                    if (c < 8) pw[c] = wv;
+                    else pw2[c - 8] = wv;
+                    ls2 = add2(ls2, bf2(wv));
                 }
+                const float2 lsp = unpack2(ls2);
+                lsum += lsp.x + lsp.y;
                 // the product of stage g - 2 has read P buffer g % 2
                 if (g > 1 && !pv_wait(g - 2)) {
                     ok = false;
