@@ -109,3 +109,106 @@ def test_partition_edge_cases():
     check([40960] * 4, 148, 2560, 4)         # long sequences over many CTAs
     check([17] * 256, 148, 2, 256)           # more sequences than CTAs
     check([40960, 1, 40960], 7, 2560, 3)     # a short sequence between two long ones
+
+
+# ----------------------------------------------------------------------------
+# The chunked prefill's split (decode_attention_qk_b200/csrc/qda_prefill.cu):
+# the page-heads of all units (sequence b, kv head j), unit-major, CTA g taking
+# [split(g), split(g + 1)), where the running cost (each unit's PIECE_COST
+# first, then one per page-head) crosses g * w, w = ceil(W / grid). A piece
+# held whole by its CTA writes o; a split unit's pieces write partials to slot
+# 2g (the CTA's first piece) or 2g + 1 (its last), and the CTA holding the
+# unit's first page records that slot, the one holding its last page its own
+# index, for the combine launch, which reads slots first, 2 (g0 + 1), ...,
+# 2 gk.
+
+PIECE_COST = 12
+
+
+def prefill_split(seg, B, grid, g):
+    """The kernel's pf_split: the first page-head of CTA g."""
+    def cost_before(b):
+        return 8 * (seg[b] + PIECE_COST * b)
+    W = cost_before(B)
+    w = (W + grid - 1) // grid
+    t = g * w
+    if t >= W:
+        return 8 * seg[B]
+    lo, hi = 0, B - 1
+    while lo < hi:
+        mid = (lo + hi + 1) >> 1
+        if cost_before(mid) <= t:
+            lo = mid
+        else:
+            hi = mid - 1
+    np_ = seg[lo + 1] - seg[lo]
+    r = t - cost_before(lo)
+    assert r < 8 * (np_ + PIECE_COST)
+    j = min(7, r // (np_ + PIECE_COST))
+    off = r - j * (np_ + PIECE_COST) - PIECE_COST
+    return 8 * seg[lo] + j * np_ + max(0, off)
+
+
+def prefill_pieces(seg, B, grid):
+    """Walk every CTA's range the way the kernel's PieceWalk does; return, per
+    unit, the pieces (cta, slot, whole) in order, and what the K producer records."""
+    total = 8 * seg[B]
+    splits = [prefill_split(seg, B, grid, g) for g in range(grid + 1)]
+    units, recorded = {}, {}
+    for g in range(grid):
+        start, end = splits[g], min(splits[g + 1], total)
+        x, k = start, 0
+        while x < end:
+            b = bisect.bisect_right(seg, x // 8) - 1
+            while seg[b + 1] == seg[b]:
+                b += 1
+            np_ = seg[b + 1] - seg[b]
+            r = x - 8 * seg[b]
+            j, i0 = r // np_, r % np_
+            n = min(np_ - i0, end - x)
+            slot = 2 * g + (0 if k == 0 else 1)
+            units.setdefault((b, j), []).append((g, slot, i0 == 0 and n == np_, n))
+            rec = recorded.setdefault((b, j), [None, None])
+            if i0 == 0:
+                rec[0] = slot
+            if i0 + n == np_:
+                rec[1] = g
+            x += n
+            k += n
+    return splits, units, recorded
+
+
+def test_prefill_split_covers_every_page_head_once_and_the_combine_finds_every_piece():
+    rng = random.Random(5)
+    for trial in range(2000):
+        B = rng.randint(1, 48)
+        grid = rng.choice([1, 2, 3, 7, 148, 300])
+        pages = [rng.choice([0, 1, 2, 5, 17, 300, 2560]) for _ in range(B)]
+        seg = [0]
+        for x in pages:
+            seg.append(seg[-1] + x)
+        total = 8 * seg[B]
+        splits, units, recorded = prefill_pieces(seg, B, grid)
+        assert splits[0] == 0 and splits[grid] == total
+        assert all(splits[i] <= splits[i + 1] for i in range(grid))
+        # every page-head in exactly one piece, every unit of a non-empty sequence present
+        assert sum(n for lst in units.values() for *_, n in lst) == total
+        assert len(units) == 8 * sum(1 for b in range(B) if seg[b + 1] > seg[b])
+        for (b, j), lst in units.items():
+            assert sum(n for *_, n in lst) == seg[b + 1] - seg[b]
+            ctas = [c for c, *_ in lst]
+            assert ctas == list(range(ctas[0], ctas[-1] + 1)), "a unit's pieces sit in consecutive CTAs"
+            first, last = recorded[(b, j)]
+            g0, gk = first >> 1, last
+            assert g0 == ctas[0] and gk == ctas[-1]
+            if g0 == gk:
+                assert len(lst) == 1 and lst[0][2], "a unit in one CTA is written whole"
+                continue
+            want = [first] + [2 * (g0 + k) for k in range(1, gk - g0 + 1)]
+            assert [s for _, s, _, _ in lst] == want, "the combine reads the slots the pieces wrote"
+            assert not any(w for _, _, w, _ in lst)
+        # slots stay inside the scratch of 2 * grid
+        for lst in units.values():
+            assert all(0 <= s < 2 * grid for _, s, _, _ in lst)
+        # the cost total stays an int32 at the largest batch (256 sequences of 40960 tokens)
+        assert 8 * (256 * 2560 + PIECE_COST * 256) < 2 ** 31
