@@ -1216,7 +1216,9 @@ def main(argv=None):
     ap.add_argument("--num-q-heads", type=int, choices=[16, 32, 40, 64], default=16,
                     help="query heads: 16 = Qwen3-0.6B (the default workload); 32/40/64 = 4B-8B/14B/32B")
     ap.add_argument("--new-tokens", type=int, default=1,
-                    help="new tokens per sequence (1 = decode; 2-4 at 16 heads, 2 at 32: several tokens at once)")
+                    help="new tokens per sequence, causal among themselves (1 = decode; up to 16 query rows "
+                         "per kv head in one launch of the decode-shaped kernel, longer blocks as the chunked "
+                         "prefill)")
     ap.add_argument("--timing", choices=["graph", "eager"], default="graph",
                     help="timed region: CUDA graph replay of the steps (default) or eager launches with "
                          "an event pair around each; the line also carries the other figure")
