@@ -335,7 +335,7 @@ __device__ __forceinline__ bool tc_wait1(const Params& p, const TcShared& s, uin
     return false;
 }
 
-// A whole warp's bounded wait, with one verdict for all its lanes.
+// A whole warp's bounded wait, with one outcome for all its lanes.
 __device__ __forceinline__ bool tc_wait_warp(const Params& p, const TcShared& s, uint64_t* bar, uint32_t parity,
                                              int lane) {
     bool ok = mbar_try_wait(bar, parity);
